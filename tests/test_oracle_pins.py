@@ -1,0 +1,362 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+Each test checks the oracle against a closed form, a special case that reduces
+to a library routine (torch's scaled_dot_product_attention in float64), a
+hand-worked fixture under tests/golden/, or an independently written brute force
+(set-based enumeration with complex-number RoPE), chosen so that a dropped term,
+a wrong index or sign, or a transposed operand in the oracle fails one of them.
+"""
+
+import cmath
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import Geometry
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+def _rand_kv(rng, T, d, scale=1.0):
+    K = rng.standard_normal((T, d)) * scale
+    V = rng.standard_normal((T, d))
+    return K, V
+
+
+# ---------------------------------------------------------------------------
+# Tree shape
+# ---------------------------------------------------------------------------
+
+def test_level_counts_match_workload_depths():
+    # 3, 4 and 6 summary levels for the 4K, 524K and 2M workload shapes.
+    assert oracle.level_counts(4096, 16, 16) == [256, 16, 1]
+    assert oracle.level_counts(524288, 64, 16) == [8192, 512, 32, 2]
+    assert oracle.level_counts(2097152, 32, 8) == [65536, 8192, 1024, 128, 16, 2]
+    assert oracle.level_counts(131072, 64, 16) == [2048, 128, 8]
+    assert oracle.level_counts(1048576, 64, 32) == [16384, 512, 16]
+    # Only complete nodes: a ragged tail adds nothing.
+    assert oracle.level_counts(4096 + 15, 16, 16) == [256, 16, 1]
+    assert oracle.level_counts(15, 16, 16) == []
+    assert oracle.level_counts(16, 16, 16) == [1]
+
+
+def test_visible_counts_definition():
+    # Brute force: node j at level l visible iff (j+1) * B * b^(l-1) <= a * B.
+    B, b, W = 4, 3, 9
+    for t in range(0, 300):
+        a, v = oracle.visible_counts(t, B, b, W)
+        assert a * B <= max(0, t + 1 - W) < a * B + B
+        for lev in range(1, 8):
+            span = B * b ** (lev - 1)
+            brute = sum(1 for j in range(400) if (j + 1) * span <= a * B)
+            got = v[lev - 1] if lev <= len(v) else 0
+            assert got == brute
+
+
+# ---------------------------------------------------------------------------
+# Pooler and tree values
+# ---------------------------------------------------------------------------
+
+def test_pool_two_key_golden(golden_dir):
+    rows = {}
+    ck, cv = [], []
+    with open(os.path.join(golden_dir, "pool_two_keys.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            name, *vals = line.split()
+            vals = [float(x) for x in vals]
+            if name == "child_key":
+                ck.append(vals)
+            elif name == "child_val":
+                cv.append(vals)
+            else:
+                rows[name] = vals
+    key = oracle.pool_keys(np.array(ck), np.array(rows["r"]))
+    np.testing.assert_allclose(key, rows["expect_key"], rtol=0, atol=1e-12)
+    # Through build_tree: a 2-token leaf block gives the same node.
+    levels = oracle.build_tree(np.array(ck), np.array(cv), np.array(rows["r"]), 2, 2)
+    np.testing.assert_allclose(levels[0][0][0], rows["expect_key"], atol=1e-12)
+    np.testing.assert_allclose(levels[0][1][0], rows["expect_val"], atol=1e-12)
+
+
+def test_pool_special_cases():
+    rng = np.random.default_rng(3)
+    keys = rng.standard_normal((7, 16))
+    # One child: the summary is the child itself.
+    np.testing.assert_allclose(oracle.pool_keys(keys[:1], rng.standard_normal(16)),
+                               keys[0], atol=1e-12)
+    # r = 0: equal scores, the summary is the plain mean.
+    np.testing.assert_allclose(oracle.pool_keys(keys, np.zeros(16)), keys.mean(0),
+                               atol=1e-12)
+    # A reference vector far along one child's key picks that child.
+    r = 1e4 * keys[3] / np.linalg.norm(keys[3])
+    np.testing.assert_allclose(oracle.pool_keys(keys, r), keys[3], atol=1e-9)
+    # The weights are a softmax: the summary lies in the convex hull.
+    r = rng.standard_normal(16)
+    key = oracle.pool_keys(keys, r)
+    assert np.all(key <= keys.max(0) + 1e-12) and np.all(key >= keys.min(0) - 1e-12)
+
+
+def test_node_value_is_mean_of_leaf_values():
+    rng = np.random.default_rng(0)
+    B, b, d = 4, 3, 8
+    K, V = _rand_kv(rng, 4 * 27 + 5, d)
+    r = rng.standard_normal(d) / math.sqrt(d)
+    levels = oracle.build_tree(K, V, r, B, b)
+    assert [len(l[0]) for l in levels] == [28, 9, 3, 1]
+    for lev, (_, vals) in enumerate(levels, start=1):
+        span = B * b ** (lev - 1)
+        for j in range(vals.shape[0]):
+            np.testing.assert_allclose(vals[j], V[j * span:(j + 1) * span].mean(0),
+                                       atol=1e-12)
+    # node_summary and LazyTree agree with build_tree.
+    lazy = oracle.LazyTree(K, V, r, B, b)
+    for lev in range(1, 5):
+        for j in range(len(levels[lev - 1][0])):
+            kk, vv = oracle.node_summary(K, V, r, B, b, lev, j)
+            np.testing.assert_allclose(kk, levels[lev - 1][0][j], atol=1e-12)
+            np.testing.assert_allclose(vv, levels[lev - 1][1][j], atol=1e-12)
+            np.testing.assert_allclose(lazy.key(lev, j), kk, atol=1e-12)
+
+
+def test_parent_key_pools_child_summaries_not_tokens():
+    # Level-2 key = pool over the level-1 *summary keys* (recursive pooling),
+    # which differs from pooling all tokens of the span at once.
+    rng = np.random.default_rng(1)
+    B, b, d = 4, 2, 4
+    K, V = _rand_kv(rng, 8, d)
+    r = rng.standard_normal(d)
+    levels = oracle.build_tree(K, V, r, B, b)
+    l1 = [oracle.pool_keys(K[0:4], r), oracle.pool_keys(K[4:8], r)]
+    np.testing.assert_allclose(levels[1][0][0], oracle.pool_keys(np.stack(l1), r),
+                               atol=1e-12)
+    assert not np.allclose(levels[1][0][0], oracle.pool_keys(K, r))
+
+
+# ---------------------------------------------------------------------------
+# RoPE
+# ---------------------------------------------------------------------------
+
+def _rope_complex(x, pos, base):
+    """Independent RoPE: pair (x_j, x_{j+d/2}) as a complex number, times e^{i p w_j}."""
+    d = len(x)
+    h = d // 2
+    out = np.empty(d)
+    for j in range(h):
+        w = base ** (-2.0 * j / d)
+        z = complex(x[j], x[j + h]) * cmath.exp(1j * pos * w)
+        out[j], out[j + h] = z.real, z.imag
+    return out
+
+
+def test_rope_matches_complex_rotation_and_is_relative():
+    rng = np.random.default_rng(2)
+    d = 16
+    x, y = rng.standard_normal(d), rng.standard_normal(d)
+    for pos in [0, 1, 7, 1000, 123457]:
+        np.testing.assert_allclose(oracle.rope_rotate(x, pos, 1e6),
+                                   _rope_complex(x, pos, 1e6), atol=1e-9)
+    np.testing.assert_allclose(oracle.rope_rotate(x, 0, 1e6), x, atol=0)
+    # <R(m) x, R(n) y> depends only on m - n.
+    a = oracle.rope_rotate(x, 50, 1e4) @ oracle.rope_rotate(y, 20, 1e4)
+    bb = oracle.rope_rotate(x, 130, 1e4) @ oracle.rope_rotate(y, 100, 1e4)
+    assert abs(a - bb) < 1e-9
+    # Dimension 0 turns by exactly `pos` radians (inverse frequency 1).
+    c, s = oracle.rope_cos_sin(np.array([3.0]), d, 1e6)
+    assert abs(c[0, 0] - math.cos(3.0)) < 1e-15 and abs(s[0, 0] - math.sin(3.0)) < 1e-15
+
+
+# ---------------------------------------------------------------------------
+# Traversal against an independent set-based brute force
+# ---------------------------------------------------------------------------
+
+def brute_force(q, t, K, V, levels, geo):
+    """Set-based restatement: classify every visible node, then one softmax.
+
+    Candidates at a level = visible nodes whose parent is kept or whose parent
+    is not visible (all visible nodes at the top level); each is scored at its
+    rank (by position) among the level's candidates with the query one past the
+    last; the best k by (score desc, rank asc) are kept.
+    """
+    d = len(q)
+    B, b, k, W = geo.leaf_block, geo.branching, geo.k, geo.window
+    a = max(0, t + 1 - W) // B
+
+    def rot(x, p):
+        return _rope_complex(x, p, geo.rope_base) if geo.rope else np.asarray(x)
+
+    vis = {}
+    for lev in range(1, len(levels) + 1):
+        span = B * b ** (lev - 1)
+        vis[lev] = [j for j in range(len(levels[lev - 1][0])) if (j + 1) * span <= a * B]
+    tops = [lev for lev in vis if vis[lev]]
+    entries = []
+    kept = {}
+    cand_sizes = {}
+    if tops:
+        top = max(tops)
+        for lev in range(top, 0, -1):
+            up_vis = set(vis.get(lev + 1, []))
+            cand = sorted(j for j in vis[lev]
+                          if lev == top or (j // b) in kept[lev + 1] or (j // b) not in up_vis)
+            rank = {j: i for i, j in enumerate(cand)}
+            qr = rot(q, len(cand))
+            score = {j: float(qr @ rot(levels[lev - 1][0][j], rank[j])) / math.sqrt(d)
+                     for j in cand}
+            best = sorted(cand, key=lambda j: (-score[j], rank[j]))[:k]
+            kept[lev] = set(best)
+            cand_sizes[lev] = len(cand)
+            for j in cand:
+                if j not in kept[lev]:
+                    entries.append((score[j], levels[lev - 1][1][j]))
+    toks = set(range(a * B, t + 1))
+    for blk in kept.get(1, set()):
+        toks |= set(range(blk * B, blk * B + B))
+    toks = sorted(toks)
+    qr = rot(q, len(toks) - 1)
+    for i, pos in enumerate(toks):
+        entries.append((float(qr @ rot(K[pos], i)) / math.sqrt(d), V[pos]))
+    m = max(e[0] for e in entries)
+    w = np.array([math.exp(e[0] - m) for e in entries])
+    out = sum(wi * e[1] for wi, e in zip(w, entries)) / w.sum()
+    return out, {lev: sorted(s) for lev, s in kept.items()}, cand_sizes, len(entries)
+
+
+@pytest.mark.parametrize("B,b,k,W,T,d,rope", [
+    (2, 2, 1, 1, 64, 8, True),
+    (4, 3, 2, 9, 200, 8, True),
+    (4, 3, 2, 9, 200, 8, False),
+    (3, 4, 3, 5, 150, 6, True),
+    (8, 2, 2, 16, 300, 4, True),
+])
+def test_traversal_matches_set_based_brute_force(B, b, k, W, T, d, rope):
+    rng = np.random.default_rng(B * 100 + b * 10 + k)
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d) / math.sqrt(d)
+    levels = oracle.build_tree(K, V, r, B, b)
+    tree = oracle.FullTree(levels)
+    geo = Geometry(d, 1, 1, B, b, k, W, rope=rope, rope_base=1e2)
+    for t in list(range(0, T, 7)) + [T - 1]:
+        q = rng.standard_normal(d) * 2.0
+        res = oracle.traverse_and_attend(q, t, K, V, tree, geo)
+        ref, kept, sizes, n_entries = brute_force(q, t, K, V, levels, geo)
+        assert {l: sorted(v) for l, v in res["kept"].items()} == kept
+        assert res["cand"] == sizes
+        assert res["entries"] == n_entries
+        np.testing.assert_allclose(res["out"], ref, atol=1e-10)
+
+
+def test_needle_recall_above_chance():
+    # Sanity, not a parity pin: with an untrained (random) pooler a planted
+    # needle's leaf block is kept far more often than chance (4 of ~252 blocks).
+    rng = np.random.default_rng(5)
+    B, b, d, T = 16, 16, 64, 4096
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d) / math.sqrt(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 1, 1, B, b, 4, 64, rope=False)
+    hits = 0
+    for _ in range(32):
+        j = int(rng.integers(0, T - 64))
+        q = 4 * K[j] + rng.standard_normal(d)
+        res = oracle.traverse_and_attend(q, T - 1, K, V, tree, geo)
+        hits += (j // B) in res["kept"][1]
+    assert hits >= 4
+
+
+# ---------------------------------------------------------------------------
+# k >= every candidate count: dense attention (library routine)
+# ---------------------------------------------------------------------------
+
+def _sdpa(q, K, V):
+    qt = torch.tensor(q, dtype=torch.float64).view(1, 1, 1, -1)
+    kt = torch.tensor(K, dtype=torch.float64).view(1, 1, K.shape[0], -1)
+    vt = torch.tensor(V, dtype=torch.float64).view(1, 1, V.shape[0], -1)
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt).view(-1).numpy()
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_keep_all_equals_dense_attention(rope):
+    rng = np.random.default_rng(7)
+    B, b, d, T, W = 4, 3, 8, 260, 5
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 1, 1, B, b, oracle.recsa.KEEP_ALL, W, rope=rope, rope_base=1e3)
+    for t in [0, 3, 4, 10, 57, 130, 259]:
+        q = rng.standard_normal(d) * 3
+        res = oracle.traverse_and_attend(q, t, K, V, tree, geo)
+        if rope:
+            qr = _rope_complex(q, t, 1e3)
+            Kr = np.stack([_rope_complex(K[j], j, 1e3) for j in range(t + 1)])
+        else:
+            qr, Kr = q, K[: t + 1]
+        ref = _sdpa(qr, Kr, V[: t + 1])
+        np.testing.assert_allclose(res["out"], ref, atol=1e-12)
+        np.testing.assert_allclose(
+            oracle.dense_causal_attention(q, t, K, V, rope=rope, rope_base=1e3), ref,
+            atol=1e-12)
+        assert res["n_exact"] == t + 1 and res["entries"] == t + 1
+
+
+def test_constant_values_give_constant_output():
+    # Normalisation is shared by summaries and exact tokens: if every token has
+    # the same value, every summary has it too and the output equals it.
+    rng = np.random.default_rng(8)
+    B, b, d, T = 4, 3, 8, 200
+    K = rng.standard_normal((T, d))
+    V = np.tile(rng.standard_normal(d), (T, 1))
+    tree = oracle.FullTree(oracle.build_tree(K, V, rng.standard_normal(d), B, b))
+    geo = Geometry(d, 1, 1, B, b, 2, 9)
+    for t in [50, 199]:
+        res = oracle.traverse_and_attend(rng.standard_normal(d), t, K, V, tree, geo)
+        assert res["entries"] > res["n_exact"]        # summaries were used
+        np.testing.assert_allclose(res["out"], V[0], atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Counts
+# ---------------------------------------------------------------------------
+
+def test_counts_closed_form_golden(golden_dir):
+    with open(os.path.join(golden_dir, "closed_form_counts.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
+    for L, B, b, k, W, D, E, R, cands in rows:
+        L, B, b, k, W, D, E, R = map(int, (L, B, b, k, W, D, E, R))
+        geo = Geometry(128, 32, 8, B, b, k, W)
+        assert len(oracle.level_counts(L, B, b)) == D
+        cf = oracle.closed_form_counts(L - 1, geo)
+        assert cf["entries"] == E and cf["keys_read"] == R
+        assert [cf["cand"][l] for l in sorted(cf["cand"])] == [int(x) for x in cands.split(",")]
+        assert E <= D * (b * k + b - 1) + B * k + W + B - 1
+
+
+@pytest.mark.parametrize("B,b,k,W", [(4, 3, 2, 9), (2, 2, 1, 1), (16, 16, 4, 64)])
+def test_traversal_counts_equal_closed_form(B, b, k, W):
+    rng = np.random.default_rng(11)
+    d, T = 8, 1200
+    K, V = _rand_kv(rng, T, d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, rng.standard_normal(d), B, b))
+    geo = Geometry(d, 1, 1, B, b, k, W)
+    for t in range(0, T, 37):
+        res = oracle.traverse_and_attend(rng.standard_normal(d), t, K, V, tree, geo)
+        cf = oracle.closed_form_counts(t, geo)
+        assert res["entries"] == cf["entries"]
+        assert res["keys_read"] == cf["keys_read"]
+        assert res["cand"] == cf["cand"]
+
+
+def test_entries_grow_logarithmically():
+    geo = Geometry(128, 32, 8, 64, 16, 8, 512)
+    prev = None
+    for L in [2**p for p in range(12, 32)]:
+        E = oracle.closed_form_counts(L - 1, geo)["entries"]
+        D = len(oracle.level_counts(L, 64, 16))
+        assert E <= D * (16 * 8 + 15) + 64 * 8 + 512 + 63
+        prev = E
+    assert prev < 2000          # 2^31 tokens: still under 2000 entries
