@@ -1,0 +1,288 @@
+// Tree build and append kernels, and the RoPE table.
+//
+// Pooling (one node from its children): weights = softmax_i(r . x_i / sqrt(d)),
+// key = sum_i weight_i x_i, value = mean of the children's values
+// ("Recursive Sparse Attention: Million-Token Length Extrapolation at
+// Logarithmic Cost", abstract: one key and one mean-pooled value per node, one
+// pooler per layer shared by all levels; "Subquadratic Attention with a
+// Hierarchical Tree-Structured Indexer", Figure 3: higher levels pool the
+// summaries of lower levels).  One warp pools one node with an online
+// softmax, so K and V are streamed exactly once; each lane owns d/32
+// contiguous channels and issues one 4..16-byte load per row.
+#include "recsa_internal.cuh"
+
+namespace recsa {
+namespace {
+
+template <typename T, int N>
+struct RowIO;
+
+template <>
+struct RowIO<float, 4> {
+  __device__ static void load(const float* row, int lane, float* x) {
+    float4 v = reinterpret_cast<const float4*>(row)[lane];
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  }
+  __device__ static void store(float* row, int lane, const float* x) {
+    reinterpret_cast<float4*>(row)[lane] = make_float4(x[0], x[1], x[2], x[3]);
+  }
+};
+template <>
+struct RowIO<float, 2> {
+  __device__ static void load(const float* row, int lane, float* x) {
+    float2 v = reinterpret_cast<const float2*>(row)[lane];
+    x[0] = v.x; x[1] = v.y;
+  }
+  __device__ static void store(float* row, int lane, const float* x) {
+    reinterpret_cast<float2*>(row)[lane] = make_float2(x[0], x[1]);
+  }
+};
+template <>
+struct RowIO<__nv_bfloat16, 4> {
+  __device__ static void load(const __nv_bfloat16* row, int lane, float* x) {
+    uint2 u = reinterpret_cast<const uint2*>(row)[lane];
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
+  }
+};
+template <>
+struct RowIO<__nv_bfloat16, 2> {
+  __device__ static void load(const __nv_bfloat16* row, int lane, float* x) {
+    __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(row)[lane];
+    float2 fa = __bfloat1622float2(a);
+    x[0] = fa.x; x[1] = fa.y;
+  }
+};
+
+// One warp pools `n` rows (keys at kbase, values at vbase, row stride d) into
+// this lane's N channels of key and value.  Rows are processed in groups of 8
+// so that eight loads per operand are in flight per lane.
+template <typename T, int N>
+__device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const float* rl,
+                          float inv_sqrt_d, int lane, float* key, float* val) {
+  float m = -INFINITY, l = 0.f;
+  float ak[N], av[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) ak[c] = av[c] = 0.f;
+  constexpr int U = 8;
+  for (int i0 = 0; i0 < n; i0 += U) {
+    float kx[U][N], vx[U][N], s[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (i0 + u < n) {
+        RowIO<T, N>::load(kbase + int64_t(i0 + u) * d, lane, kx[u]);
+        RowIO<T, N>::load(vbase + int64_t(i0 + u) * d, lane, vx[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float acc = 0.f;
+      if (i0 + u < n) {
+#pragma unroll
+        for (int c = 0; c < N; ++c) acc = fmaf(rl[c], kx[u][c], acc);
+      }
+      s[u] = acc;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) s[u] = warp_sum(s[u]) * inv_sqrt_d;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (i0 + u < n) {
+        float mn = fmaxf(m, s[u]);
+        float sc = expf(m - mn);
+        float w = expf(s[u] - mn);
+        l = l * sc + w;
+#pragma unroll
+        for (int c = 0; c < N; ++c) {
+          ak[c] = fmaf(w, kx[u][c], ak[c] * sc);
+          av[c] += vx[u][c];
+        }
+        m = mn;
+      }
+    }
+  }
+  float il = 1.f / l, in = 1.f / float(n);
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    key[c] = ak[c] * il;
+    val[c] = av[c] * in;
+  }
+}
+
+template <int N>
+__device__ void load_r(const float* r, int lane, float* rl) {
+#pragma unroll
+  for (int c = 0; c < N; ++c) rl[c] = r[lane * N + c];
+}
+
+// Level 1: one warp per leaf block of one (sequence, KV head).
+template <typename T, int N>
+__global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T* V,
+                                                   const float* r, int64_t r_stride, void* tree,
+                                                   int64_t seq, int64_t n_leaf) {
+  const int lane = threadIdx.x & 31;
+  const int64_t j = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int g = blockIdx.y;
+  if (j >= n_leaf) return;
+  float rl[N];
+  load_r<N>(r + g * r_stride, lane, rl);
+  const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
+  float key[N], val[N];
+  pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
+  float* kd = level_keys(p, tree, 1, seq, g) + j * p.d;
+  float* vd = level_vals(p, tree, 1, seq, g) + j * p.d;
+  RowIO<float, N>::store(kd, lane, key);
+  RowIO<float, N>::store(vd, lane, val);
+}
+
+// Level lev >= 2: one warp per node, pooling b child summaries.
+template <int N>
+__global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, int64_t r_stride,
+                                                     void* tree, int64_t seq, int lev,
+                                                     int64_t n_nodes) {
+  const int lane = threadIdx.x & 31;
+  const int64_t j = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int g = blockIdx.y;
+  if (j >= n_nodes) return;
+  float rl[N];
+  load_r<N>(r + g * r_stride, lane, rl);
+  const float* ck = level_keys(p, tree, lev - 1, seq, g) + j * p.b * p.d;
+  const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
+  float key[N], val[N];
+  pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
+  RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + j * p.d, lane, key);
+  RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + j * p.d, lane, val);
+}
+
+// Append one token per sequence; pool the leaf and ancestors it completes.
+// One CTA per sequence; warp w handles KV heads w, w + 8, ...
+template <typename T, int N>
+__global__ void __launch_bounds__(256) append_kernel(Params p, T* K, T* V, const T* k_new,
+                                                     const T* v_new, int64_t* len_dev,
+                                                     const float* r, int64_t r_stride,
+                                                     void* tree) {
+  const int64_t seq = blockIdx.x;
+  const int64_t len = len_dev[seq];
+  if (len >= p.cap || len < 0) {
+    if (threadIdx.x == 0) atomicOr(tree_error_word(tree), RECSA_DEVERR_APPEND_FULL);
+    return;
+  }
+  for (int idx = threadIdx.x; idx < p.hkv * p.d; idx += blockDim.x) {
+    const int g = idx / p.d, c = idx % p.d;
+    const int64_t dst = ((seq * p.hkv + g) * p.cap + len) * p.d + c;
+    const int64_t src = (seq * p.hkv + g) * p.d + c;
+    K[dst] = k_new[src];
+    V[dst] = v_new[src];
+  }
+  __syncthreads();
+  const int64_t newlen = len + 1;
+  if (newlen % p.B == 0) {
+    const int lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    const int64_t j = newlen / p.B - 1;
+    for (int g = threadIdx.x >> 5; g < p.hkv; g += nw) {
+      float rl[N];
+      load_r<N>(r + g * r_stride, lane, rl);
+      const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
+      float key[N], val[N];
+      pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
+      RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + j * p.d, lane, key);
+      RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
+      int64_t idx = j;
+      for (int lev = 2; lev <= p.lay.levels && (idx + 1) % p.b == 0; ++lev) {
+        idx = (idx + 1) / p.b - 1;
+        __syncwarp();
+        const float* ck = level_keys(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
+        const float* cv = level_vals(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
+        pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
+        RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + idx * p.d, lane, key);
+        RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + idx * p.d, lane, val);
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) len_dev[seq] = newlen;
+}
+
+// RoPE table: row i holds (cos, sin) of i * base^(-2j/d), j < d/2, computed in
+// double precision and rounded to fp32.
+__global__ void rope_table_kernel(float2* table, int rows, int half, int d, double base) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= int64_t(rows) * half) return;
+  const int64_t pos = idx / half;
+  const int j = int(idx % half);
+  const double inv = pow(base, -2.0 * double(j) / double(d));
+  double s, c;
+  sincos(double(pos) * inv, &s, &c);
+  table[idx] = make_float2(float(c), float(s));
+}
+
+template <typename T, int N>
+cudaError_t build_typed(const Params& p, const void* K, const void* V, const int64_t* len_host,
+                        const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
+  const int warps = 8;
+  for (int64_t seq = 0; seq < p.batch; ++seq) {
+    int64_t n = len_host[seq] / p.B;
+    if (n == 0) continue;
+    dim3 grid(unsigned((n + warps - 1) / warps), p.hkv);
+    leaf_kernel<T, N><<<grid, warps * 32, 0, s>>>(p, reinterpret_cast<const T*>(K),
+                                                  reinterpret_cast<const T*>(V), r, r_stride,
+                                                  tree, seq, n);
+    for (int lev = 2; lev <= p.lay.levels; ++lev) {
+      n /= p.b;
+      if (n == 0) break;
+      dim3 g2(unsigned((n + warps - 1) / warps), p.hkv);
+      parent_kernel<N><<<g2, warps * 32, 0, s>>>(p, r, r_stride, tree, seq, lev, n);
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(const Params& p, void* tree, double rope_base, cudaStream_t s) {
+  const int half = p.d / 2;
+  const int64_t n = int64_t(p.lay.rope_rows) * half;
+  float2* table = reinterpret_cast<float2*>(reinterpret_cast<char*>(tree) + p.lay.rope_off);
+  rope_table_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(table, p.lay.rope_rows, half, p.d,
+                                                               rope_base);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build(const Params& p, const void* K, const void* V, const int64_t* len_host,
+                         const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
+  if (p.dtype == RECSA_DTYPE_BF16) {
+    return p.d == 128 ? build_typed<__nv_bfloat16, 4>(p, K, V, len_host, r, r_stride, tree, s)
+                      : build_typed<__nv_bfloat16, 2>(p, K, V, len_host, r, r_stride, tree, s);
+  }
+  return p.d == 128 ? build_typed<float, 4>(p, K, V, len_host, r, r_stride, tree, s)
+                    : build_typed<float, 2>(p, K, V, len_host, r, r_stride, tree, s);
+}
+
+cudaError_t launch_append(const Params& p, void* K, void* V, const void* k_new, const void* v_new,
+                          int64_t* len_dev, const float* r, int64_t r_stride, void* tree,
+                          cudaStream_t s) {
+  dim3 grid(p.batch);
+  if (p.dtype == RECSA_DTYPE_BF16) {
+    using T = __nv_bfloat16;
+    if (p.d == 128)
+      append_kernel<T, 4><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
+                                               len_dev, r, r_stride, tree);
+    else
+      append_kernel<T, 2><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
+                                               len_dev, r, r_stride, tree);
+  } else {
+    using T = float;
+    if (p.d == 128)
+      append_kernel<T, 4><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
+                                               len_dev, r, r_stride, tree);
+    else
+      append_kernel<T, 2><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
+                                               len_dev, r, r_stride, tree);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace recsa

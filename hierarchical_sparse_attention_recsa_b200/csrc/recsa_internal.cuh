@@ -1,0 +1,90 @@
+// Internal definitions shared by the RecSA CUDA translation units: the tree
+// buffer layout, the launch parameter block and small device helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/recsa.h"
+
+namespace recsa {
+
+constexpr int kMaxLevels = RECSA_MAX_LEVELS;
+constexpr int kHeaderBytes = 256;
+constexpr int kTraceHead = 4 + 2 * kMaxLevels;  // ints before the kept-id lists
+
+// Byte layout of the caller-owned tree buffer (computed on the host).
+struct TreeLayout {
+  int32_t levels;                 // summary levels at capacity (D)
+  int32_t rope_rows;              // rows of the RoPE table
+  int64_t nodes[kMaxLevels];      // nodes per (sequence, KV head) at level l+1
+  int64_t key_off[kMaxLevels];    // fp32 keys  [batch][Hkv][nodes][d]
+  int64_t val_off[kMaxLevels];    // fp32 values, same shape
+  int64_t rope_off;               // float2 (cos, sin) [rope_rows][d/2]
+  int64_t total;
+};
+
+// Everything a kernel needs about the geometry, passed by value.
+struct Params {
+  int32_t dtype, d, hq, hkv, group, B, b, k, W, rope, batch;
+  int64_t cap;
+  float inv_sqrt_d;
+  TreeLayout lay;
+};
+
+// Device error word at offset 0 of the tree header.
+__device__ __forceinline__ unsigned int* tree_error_word(void* tree) {
+  return reinterpret_cast<unsigned int*>(tree);
+}
+
+__device__ __forceinline__ float* level_keys(const Params& p, void* tree, int lev /*1-based*/,
+                                             int64_t seq, int g) {
+  char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
+  return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.d;
+}
+__device__ __forceinline__ float* level_vals(const Params& p, void* tree, int lev, int64_t seq,
+                                             int g) {
+  char* base = reinterpret_cast<char*>(tree) + p.lay.val_off[lev - 1];
+  return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.d;
+}
+__device__ __forceinline__ const float2* rope_table(const Params& p, const void* tree) {
+  return reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tree) + p.lay.rope_off);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Element load from a K/V/Q tensor of the geometry's dtype, as fp32.
+__device__ __forceinline__ float load_elem(const void* base, int64_t idx, int dtype) {
+  if (dtype == RECSA_DTYPE_BF16)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
+  return reinterpret_cast<const float*>(base)[idx];
+}
+__device__ __forceinline__ void store_elem(void* base, int64_t idx, float v, int dtype) {
+  if (dtype == RECSA_DTYPE_BF16)
+    reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(base)[idx] = v;
+}
+
+// Host-side launchers (defined in the .cu files).
+cudaError_t launch_rope_table(const Params& p, void* tree, double rope_base, cudaStream_t s);
+cudaError_t launch_build(const Params& p, const void* K, const void* V, const int64_t* len_host,
+                         const float* r, int64_t r_stride, void* tree, cudaStream_t s);
+cudaError_t launch_append(const Params& p, void* K, void* V, const void* k_new, const void* v_new,
+                          int64_t* len_dev, const float* r, int64_t r_stride, void* tree,
+                          cudaStream_t s);
+cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const void* V,
+                          const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
+                          int decode, void* O, int32_t* trace, cudaStream_t s);
+
+}  // namespace recsa

@@ -1,0 +1,179 @@
+/*
+ * recsa.h -- C ABI of the B200 (sm_100a) RecSA hot path.
+ *
+ * Recursive Sparse Attention ("Recursive Sparse Attention: Million-Token Length
+ * Extrapolation at Logarithmic Cost", abstract) keeps a tree over one layer's
+ * KV cache.  Every node summarises its span with one key, pooled by one
+ * per-layer pooler shared by all levels, and one mean-pooled value.  A query
+ * walks the tree top-down keeping at most k candidates per level; the
+ * summaries of the unselected candidates join the exact tokens of the kept
+ * leaf blocks and of a local window in one softmax, and every entry is rotated
+ * (RoPE) to its index among the candidates of its level.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are caller-owned device memory; the library allocates
+ *     nothing and keeps no global state.  Pointers to K, V, Q, O, k_new, v_new
+ *     must be 16-byte aligned, the tree 256-byte aligned.
+ *   - Layouts are row-major:
+ *       K, V          [batch][n_kv_heads][capacity][head_dim]   (dtype)
+ *       Q, O          [batch][n_q][n_q_heads][head_dim]         (dtype)
+ *       k_new, v_new  [batch][n_kv_heads][head_dim]             (dtype)
+ *       pooler_r      [n_kv_heads][head_dim] fp32 with a head stride in
+ *                     elements (0 = one vector shared by every KV head)
+ *       len           int64 [batch]: tokens currently in each sequence
+ *     Query head h reads KV head h / (n_q_heads / n_kv_heads).
+ *   - Work is enqueued on `stream` (a cudaStream_t, 0 = legacy default) and
+ *     runs asynchronously.  Argument and launch errors are returned at once;
+ *     errors found on the device (a full cache on append) set a flag in the
+ *     tree header, read with recsa_tree_error().
+ *   - Inputs are assumed finite.
+ */
+#ifndef RECSA_H_
+#define RECSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum recsa_status {
+  RECSA_OK = 0,
+  RECSA_ERR_INVALID_GEOMETRY = 1, /* a geometry field is out of range */
+  RECSA_ERR_NULL = 2,             /* a required pointer is NULL */
+  RECSA_ERR_MISALIGNED = 3,       /* a pointer breaks the alignment rule */
+  RECSA_ERR_CAPACITY = 4,         /* a length or query range exceeds capacity */
+  RECSA_ERR_UNSUPPORTED = 5,      /* valid geometry outside the kernels' limits */
+  RECSA_ERR_CUDA = 6,             /* a CUDA runtime call or launch failed */
+  RECSA_ERR_DEVICE = 7            /* the tree header carries a device error */
+} recsa_status;
+
+enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
+
+/* k value meaning "keep every candidate" (the shared softmax then covers every
+ * token up to the query: dense causal attention). */
+#define RECSA_KEEP_ALL 2147483647
+
+/* Deepest tree the kernels walk (levels of summaries above the tokens). */
+#define RECSA_MAX_LEVELS 16
+/* Largest k for which a selection trace is recorded. */
+#define RECSA_TRACE_MAX_K 64
+
+/* Device error flags in the tree header (recsa_tree_error). */
+#define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
+
+/*
+ * Tree geometry and attention shape.
+ *   leaf_block (B): tokens per level-1 node.  branching (b): children per node
+ *   above level 1.  A level-l node spans B * b^(l-1) tokens; only complete nodes
+ *   exist, so a cache of T tokens holds floor(T / (B b^(l-1))) level-l nodes
+ *   ("Subquadratic Attention with a Hierarchical Tree-Structured Indexer",
+ *   Table VIII), and a level exists while it holds at least one node.
+ *   k: candidates kept per level (RecSA abstract); RECSA_KEEP_ALL keeps all.
+ *   window (W >= 1): the exact local window.  For a query at position t it is
+ *   [a*B, t] with a = floor(max(0, t + 1 - W) / B), and only nodes whose span
+ *   ends at or before a*B are visible to that query.
+ *   rope_enabled / rope_base: rotate-half RoPE at candidate-local indices
+ *   (RecSA abstract), inverse frequencies base^(-2j/d).
+ */
+typedef struct recsa_geometry {
+  int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
+  int32_t head_dim;     /* d: 64 or 128 */
+  int32_t n_q_heads;    /* query heads */
+  int32_t n_kv_heads;   /* KV heads; n_q_heads / n_kv_heads in {1, 2, 4, 8} */
+  int32_t leaf_block;   /* B, 1..1024 */
+  int32_t branching;    /* b, 2..64 */
+  int32_t k;            /* 1..RECSA_KEEP_ALL */
+  int32_t window;       /* W >= 1 */
+  int32_t rope_enabled; /* 0 or 1 */
+  float rope_base;      /* > 1 */
+  int32_t batch;        /* sequences, >= 1 */
+  int32_t reserved;     /* must be 0 */
+  int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
+} recsa_geometry;
+
+/* Human-readable name of a status code (static string). */
+const char* recsa_status_string(recsa_status s);
+
+/* Check a geometry without touching the device. */
+recsa_status recsa_validate(const recsa_geometry* geom);
+
+/* Summary levels a cache of `length` tokens holds under `geom` (0 if length < B). */
+recsa_status recsa_num_levels(const recsa_geometry* geom, int64_t length, int32_t* levels);
+
+/*
+ * Bytes of the tree buffer for `geom` at its capacity: a 256-byte header
+ * (device error flags), the RoPE cos/sin table of the indices a traversal can
+ * reach, and per level l: keys and values [batch][n_kv_heads][n_l][head_dim]
+ * in fp32, n_l the level's node count at capacity.
+ */
+recsa_status recsa_tree_bytes(const recsa_geometry* geom, size_t* bytes);
+
+/*
+ * Build the tree (RecSA abstract: one key and one mean-pooled value per node).
+ * For each sequence s, every complete node over its first len_host[s] tokens
+ * is written: level 1 pools each leaf block of B tokens, level l > 1 pools b
+ * consecutive level-(l-1) summary keys ("Subquadratic Attention with a
+ * Hierarchical Tree-Structured Indexer", Figure 3).  Pooling: weights =
+ * softmax_i(r . k_i / sqrt(d)), key = sum_i weight_i k_i; value = mean of the
+ * children's values.  Also clears the error flags and writes the RoPE table.
+ *   len_host: HOST int64 [batch], each in [0, capacity].
+ */
+recsa_status recsa_build(const recsa_geometry* geom, const void* K, const void* V,
+                         const int64_t* len_host, const float* pooler_r,
+                         int64_t pooler_head_stride, void* tree, void* stream);
+
+/*
+ * Append one token per sequence (decode-time tree maintenance): writes k_new,
+ * v_new at position len_dev[s] of K and V, increments len_dev[s], and, when the
+ * token completes a leaf block, pools that leaf and every ancestor it
+ * completes (the cost is amortised over node completions: ZHA, Table VIII).
+ * A sequence already at capacity is left unchanged and sets
+ * RECSA_DEVERR_APPEND_FULL.
+ *   len_dev: DEVICE int64 [batch].
+ */
+recsa_status recsa_append(const recsa_geometry* geom, void* K, void* V, const void* k_new,
+                          const void* v_new, int64_t* len_dev, const float* pooler_r,
+                          int64_t pooler_head_stride, void* tree, void* stream);
+
+/*
+ * Decode attention: n_q queries per sequence, all at position len_dev[s] - 1
+ * (the newest token, already appended).  O[s][i][h] = RecSA output of
+ * Q[s][i][h].  Sequences with len_dev[s] == 0 get O = 0.
+ *   trace: NULL, or DEVICE int32 [batch][n_q][n_q_heads][recsa_trace_ints()]
+ *   (requires k <= RECSA_TRACE_MAX_K).
+ */
+recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void* K,
+                          const void* V, const void* tree, const int64_t* len_dev,
+                          int32_t n_q, void* O, int32_t* trace, void* stream);
+
+/*
+ * Prefill attention: query i of sequence s sits at position q_start + i,
+ * i < n_q, causal.  The tree must have been built over at least q_start + n_q
+ * tokens of every sequence (a node is a pure function of its span, so a tree
+ * built over more tokens serves every earlier query: each query sees only the
+ * nodes that end before its window).
+ */
+recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void* K,
+                           const void* V, const void* tree, int64_t q_start, int32_t n_q,
+                           void* O, int32_t* trace, void* stream);
+
+/*
+ * Trace record length in int32 per (sequence, query, head):
+ *   [0] visible levels  [1] softmax entries  [2] keys read  [3] exact tokens
+ *   [4 + l - 1]                      candidates at level l   (l = 1..16)
+ *   [4 + 16 + l - 1]                 kept at level l
+ *   [4 + 32 + (l - 1) * k + j]       j-th kept node id at level l, in position order
+ */
+recsa_status recsa_trace_ints(const recsa_geometry* geom, int32_t* ints);
+
+/* Read (and optionally clear) the device error flags of a tree; synchronises `stream`. */
+recsa_status recsa_tree_error(const recsa_geometry* geom, void* tree, int32_t clear,
+                              uint32_t* flags, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RECSA_H_ */

@@ -265,9 +265,9 @@ def traverse_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry,
          position order, query index n0-1 (the query is the last token).
       5. One softmax over all summary and exact entries, scale 1/sqrt(d).
 
-    ``keep_override`` (level -> kept candidate indices) recomputes the output
-    for a given selection (used where several selections are correct: near
-    ties).  Returns dict(out, kept{level: node ids}, cand{level: c},
+    ``keep_override`` (level -> kept node ids) recomputes the output for a
+    given selection (used where several selections are correct: near ties);
+    the ids must be candidates of their level.  Returns dict(out, kept{level: node ids}, cand{level: c},
     scores{level: [..]}, entries, keys_read, n_exact).
     """
     q = np.asarray(q, dtype=np.float64)
@@ -299,7 +299,10 @@ def traverse_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry,
                   for i, n in enumerate(cand)]
         keys_read += c
         if keep_override is not None:
-            kept_idx = sorted(keep_override[lev])
+            want = set(int(x) for x in keep_override[lev])
+            kept_idx = [i for i, n in enumerate(cand) if n in want]
+            if len(kept_idx) != len(want):
+                raise ValueError(f"level {lev}: kept ids {sorted(want)} are not all candidates")
         else:
             kept_idx = _top_k_sorted(scores, k)
         kept_set = set(kept_idx)
