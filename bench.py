@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""RecSA benchmark: decode queries/s (append + decode per step) and prefill
+tokens/s on the Qwen3-4B-shaped layer at L = 524288, one B200 per rank.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl recsa|reference]
+
+One step = one decode step of the whole hot path for the batch: recsa_append
+of each sequence's new token (tree maintenance) then recsa_decode (level-wise
+selection + shared-softmax gather attention).  Prefill (recsa_build over the
+whole context, then recsa_prefill of every position) and a dense attention
+comparator (torch SDPA, a library kernel) are measured once per run and
+reported beside the main number.  Multi-GPU runs are independent replicas
+(weak scaling): each rank serves its own batch; the time is the max over ranks.
+
+The CPU oracle is executed only by the cpu_baseline leg and by --impl
+reference (it is the reference arm: a float64 restatement of the method).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_sparse_attention_recsa_b200 import counts, synth  # noqa: E402
+from hierarchical_sparse_attention_recsa_b200 import recsa as R  # noqa: E402
+
+METRIC = "decode queries/s and prefill tokens/s at L=524K on 1 B200; % of HBM roofline"
+WORKLOAD = "qwen3-4b-524k"
+NOMINAL_HBM_GBS = 8000.0     # roofline denominator named by the workload definition
+ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 x max SM clock
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler
+# ---------------------------------------------------------------------------
+
+class Clocks:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device}.csv")
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def geometry(w, batch, capacity) -> R.Geometry:
+    return R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                      leaf_block=w.leaf_block, branching=w.branching, k=w.k, window=w.window,
+                      batch=batch, capacity=capacity, dtype=R.DTYPE_BF16,
+                      rope_enabled=1, rope_base=w.rope_base)
+
+
+class L2Flush:
+    def __init__(self, mib=256):
+        self.buf = torch.empty(mib << 20, dtype=torch.uint8, device="cuda")
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def elapsed(a, b):
+    return a.elapsed_time(b)
+
+
+def make_prefill_queries(w, K, L, chunk=65536):
+    Q = torch.empty((1, L, w.n_q_heads, w.head_dim), dtype=w.dtype, device="cuda")
+    for c0 in range(0, L, chunk):
+        n = min(chunk, L - c0)
+        pos = (c0 + torch.arange(n, device="cuda", dtype=torch.int64))[None]
+        q, _, _ = synth.make_queries(w, K[:1], pos, seed=100 + c0 // chunk)
+        Q[:, c0:c0 + n] = q
+    return Q
+
+
+# ---------------------------------------------------------------------------
+# RecSA arm
+# ---------------------------------------------------------------------------
+
+def run_recsa(args, rank, world, dev):
+    w = synth.WORKLOADS[WORKLOAD]
+    L, batch = w.length, w.batch
+    K_steps, W_steps = args.steps, args.warmup
+    n_stage = max(K_steps, W_steps)
+    cap = L + max(512, n_stage + 1)
+    hbm_gbs, bf16_tflops, peak_kind = peaks()
+    torch.manual_seed(0)
+    Kc, Vc, r = synth.make_kv(w, cap, seed=rank, device="cuda", batch=batch)
+    r = r.contiguous()
+    g = geometry(w, batch, cap)
+    tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
+    R.recsa_build(g, Kc, Vc, [L] * batch, r, 0, tree)
+    # per-step inputs: queries at the new positions and the tokens to append
+    pos = (L + torch.arange(n_stage, device="cuda", dtype=torch.int64))[None].expand(batch, -1)
+    Qall, kind, _ = synth.make_queries(w, Kc, pos.contiguous(), seed=1 + rank)
+    Qs = Qall.permute(1, 0, 2, 3).unsqueeze(2).contiguous()       # [step][batch][1][Hq][d]
+    kn = Kc[:, :, L:L + n_stage].permute(2, 0, 1, 3).contiguous()  # [step][batch][Hkv][d]
+    vn = Vc[:, :, L:L + n_stage].permute(2, 0, 1, 3).contiguous()
+    O = torch.empty_like(Qs[0])
+    lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
+    lens0 = lens.clone()
+    ti = R.recsa_trace_ints(g)
+    traces = torch.zeros((K_steps, batch, 1, w.n_q_heads, ti), dtype=torch.int32, device="cuda")
+    flush = L2Flush()
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        R.recsa_append(g, Kc, Vc, kn[i], vn[i], lens, r, 0, tree)
+        R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O)
+
+    for i in range(W_steps):
+        step(i)
+    lens.copy_(lens0)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
+    clocks = Clocks(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(K_steps):
+        flush()
+        ev[i][0].record(stream)
+        R.recsa_append(g, Kc, Vc, kn[i], vn[i], lens, r, 0, tree)
+        ev[i][1].record(stream)
+        R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O)
+        ev[i][2].record(stream)
+        # untimed: the same decode again with its selection trace, for accounting
+        R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O, traces[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    step_ms = sum(elapsed(e[0], e[2]) for e in ev)
+    dec_ms = sum(elapsed(e[1], e[2]) for e in ev) / K_steps
+    app_ms = sum(elapsed(e[0], e[1]) for e in ev) / K_steps
+    if world > 1:
+        t = torch.tensor([step_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(t.item())
+    value = batch * K_steps * world / (step_ms / 1e3)
+
+    # algorithmic bytes of the decode launches, from the traces
+    tr = traces.cpu().numpy()
+    acc = []
+    for i in range(K_steps):
+        lens_i = np.full(batch, L + i + 1)
+        acc.append(counts.decode_bytes_from_trace(tr[i], lens_i, w.leaf_block, w.branching,
+                                                  w.window, w.n_q_heads // w.n_kv_heads,
+                                                  w.head_dim, 2, w.k))
+    dec_bytes = float(np.mean([a["bytes"] for a in acc]))
+    achieved = dec_bytes / (dec_ms / 1e3) / 1e9
+
+    # end to end through the public API with host buffers
+    Qh = Qs.cpu().pin_memory()
+    knh, vnh = kn.cpu().pin_memory(), vn.cpu().pin_memory()
+    Oh = torch.empty((K_steps,) + tuple(O.shape), dtype=O.dtype).pin_memory()
+    Qd, knd, vnd = torch.empty_like(Qs[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+    lens.copy_(lens0)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
+    torch.cuda.synchronize()
+    for i in range(K_steps):
+        flush()
+        ev2[i][0].record(stream)
+        Qd.copy_(Qh[i], non_blocking=True)
+        knd.copy_(knh[i], non_blocking=True)
+        vnd.copy_(vnh[i], non_blocking=True)
+        R.recsa_append(g, Kc, Vc, knd, vnd, lens, r, 0, tree)
+        R.recsa_decode(g, Qd, Kc, Vc, tree, lens, 1, O)
+        Oh[i].copy_(O, non_blocking=True)
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(elapsed(a, b) for a, b in ev2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": batch * K_steps * world / (e2e_ms / 1e3), "unit": "queries/s",
+           "h2d_bytes_per_step": int(Qd.numel() * 2 + knd.numel() * 2 + vnd.numel() * 2),
+           "d2h_bytes_per_step": int(O.numel() * 2)}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": K_steps, "warmup": W_steps, "ms_per_step": step_ms / K_steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: K,V ~ N(0,1) x per-channel LogNormal(0,0.5) scale, Q ~ N(0,1), "
+                "1% planted needles, seeded",
+        "config": {"workload": WORKLOAD, "L": L, "batch": batch, "q_heads": w.n_q_heads,
+                   "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                   "leaf_block": w.leaf_block, "branching": w.branching, "k": w.k,
+                   "window": w.window, "levels": R.recsa_num_levels(g, L),
+                   "step": "recsa_append + recsa_decode for the batch",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "recsa decode (attend_kernel)",
+                     "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
+                     "frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "bytes_per_launch": dec_bytes, "launch_ms": dec_ms, "traffic": None},
+        "decode_ms": dec_ms, "append_ms": app_ms,
+        "e2e": e2e, "gpu_launches": 2 * K_steps, "clocks": clk,
+    }
+    del traces, Qh, Oh
+    torch.cuda.empty_cache()
+    if not args.no_prefill:
+        out["prefill"] = run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs)
+    if not args.no_dense:
+        out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
+    if rank == 0 and world == 1 and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return out
+
+
+def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
+    L = w.length
+    gp = geometry(w, 1, cap)
+    K0, V0 = Kc[:1], Vc[:1]
+    tree = torch.zeros(R.recsa_tree_bytes(gp), dtype=torch.uint8, device="cuda")
+    Q = make_prefill_queries(w, Kc, L)
+    O = torch.empty_like(Q)
+    chunk = 65536
+
+    def once():
+        R.recsa_build(gp, K0, V0, [L], r, 0, tree)
+        for c0 in range(0, L, chunk):
+            n = min(chunk, L - c0)
+            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n])
+
+    once()
+    torch.cuda.synchronize()
+    times, build_t = [], []
+    for _ in range(args.prefill_reps):
+        flush()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        R.recsa_build(gp, K0, V0, [L], r, 0, tree)
+        e1.record(stream)
+        for c0 in range(0, L, chunk):
+            n = min(chunk, L - c0)
+            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n])
+        e2.record(stream)
+        torch.cuda.synchronize()
+        times.append(elapsed(e0, e2))
+        build_t.append(elapsed(e0, e1))
+    ms = min(times)
+    t = np.arange(L)
+    ent, keys = counts.per_query_counts(t, w.leaf_block, w.branching, w.k, w.window,
+                                        R.recsa_num_levels(gp, L))
+    flops = float(2 * w.head_dim * (ent.sum() + keys.sum()) * w.n_q_heads)
+    attend_ms = ms - min(build_t)
+    kv_bytes = 2 * L * w.n_kv_heads * w.head_dim * 2
+    build_ms = min(build_t)
+    del Q, O, tree
+    torch.cuda.empty_cache()
+    return {"value": L / (ms / 1e3), "unit": "tokens/s", "ms": ms, "reps": args.prefill_reps,
+            "build_ms": build_ms, "attend_ms": attend_ms, "queries": L,
+            "roofline": {"bound": "alu", "kernel": "recsa prefill (attend_kernel)",
+                         "achieved": flops / (attend_ms / 1e3) / 1e12,
+                         "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": flops / (attend_ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS,
+                         "flops": flops, "traffic": None},
+            "build_roofline": {"bound": "hbm", "achieved": kv_bytes / (build_ms / 1e3) / 1e9,
+                               "peak": hbm_gbs, "unit": "GB/s",
+                               "frac": kv_bytes / (build_ms / 1e3) / 1e9 / hbm_gbs}}
+
+
+def run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, prefill):
+    """Dense attention on the same GPU with torch SDPA (library kernel)."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    L = w.length
+    res = {"impl": "torch.nn.functional.scaled_dot_product_attention (flash/cuDNN/efficient)"}
+    backends = [SDPBackend.FLASH_ATTENTION, SDPBackend.CUDNN_ATTENTION,
+                SDPBackend.EFFICIENT_ATTENTION]
+    try:
+        Kd, Vd = Kc[:, :, :L], Vc[:, :, :L]
+        q = Qs[0].permute(0, 2, 1, 3)               # [batch, Hq, 1, d]
+        with sdpa_kernel(backends):
+            for _ in range(3):
+                torch.nn.functional.scaled_dot_product_attention(q, Kd, Vd, enable_gqa=True)
+            ts = []
+            for _ in range(10):
+                flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                torch.nn.functional.scaled_dot_product_attention(q, Kd, Vd, enable_gqa=True)
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ts.append(elapsed(e0, e1))
+        ms = statistics.median(ts)
+        res["decode_ms"] = ms
+        res["decode_queries_per_s"] = w.batch / (ms / 1e3)
+    except Exception as e:  # library kernel unavailable for this shape
+        res["decode_error"] = str(e).splitlines()[0][:200]
+    if prefill is not None and not args.no_dense_prefill:
+        try:
+            Q = make_prefill_queries(w, Kc, L).permute(0, 2, 1, 3)
+            Kd, Vd = Kc[:1, :, :L], Vc[:1, :, :L]
+            with sdpa_kernel(backends):
+                torch.nn.functional.scaled_dot_product_attention(Q, Kd, Vd, is_causal=True,
+                                                                 enable_gqa=True)
+                flush()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                torch.nn.functional.scaled_dot_product_attention(Q, Kd, Vd, is_causal=True,
+                                                                 enable_gqa=True)
+                e1.record(stream)
+                torch.cuda.synchronize()
+            ms = elapsed(e0, e1)
+            res["prefill_ms"] = ms
+            res["prefill_tokens_per_s"] = L / (ms / 1e3)
+            del Q
+        except Exception as e:
+            res["prefill_error"] = str(e).splitlines()[0][:200]
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle: cpu_baseline leg and the reference arm
+# ---------------------------------------------------------------------------
+
+class OracleDecode:
+    """The float64 oracle on one KV head (G = 4 query heads) of the workload."""
+
+    def __init__(self, seed=0):
+        import oracle
+        self.oracle = oracle
+        w = synth.WORKLOADS[WORKLOAD]
+        self.w1 = synth.Workload(**{**w.__dict__, "n_q_heads": 4, "n_kv_heads": 1, "batch": 1})
+        L = w.length
+        self.L = L
+        n = 64
+        K, V, r = synth.make_kv(self.w1, L + n, seed=seed, device="cpu", batch=1)
+        self.K = K[0, 0].float().numpy()
+        self.V = V[0, 0].float().numpy()
+        pos = (L + torch.arange(n, dtype=torch.int64))[None]
+        Q, _, _ = synth.make_queries(self.w1, K, pos, seed=1)
+        self.Q = Q[0].float().numpy()
+        self.geo = oracle.Geometry(w.head_dim, 4, 1, w.leaf_block, w.branching, w.k, w.window,
+                                   rope=True, rope_base=w.rope_base)
+        self.tree = oracle.LazyTree(self.K, self.V, r.double().numpy(), w.leaf_block,
+                                    w.branching)
+        self.i = 0
+        self.heads_per_query = w.n_q_heads
+        # untimed: pool the nodes the first query visits (the oracle's tree build)
+        self.query_heads(1)
+
+    def query_heads(self, n_heads):
+        done = 0
+        while done < n_heads:
+            i = self.i % self.Q.shape[0]
+            t = self.L + i - 1
+            h = done % 4
+            self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree, self.geo)
+            done += 1
+            if h == 3:
+                self.i += 1
+        return done
+
+
+def _single_thread():
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(1)
+    except Exception:
+        return None
+
+
+def cpu_baseline(seconds=15.0):
+    lim = _single_thread()
+    o = OracleDecode()
+    t0 = time.perf_counter()
+    heads = 0
+    while time.perf_counter() - t0 < seconds:
+        heads += o.query_heads(4)
+    dt = time.perf_counter() - t0
+    del lim
+    return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
+            "kind": "oracle",
+            "sample": f"{heads} query-heads (decode at t=L, one KV head's tree, G=4) in "
+                      f"{dt:.1f} s; queries/s = query-heads/32/s; tree pooling untimed"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    lim = _single_thread()
+    o = OracleDecode()
+    for _ in range(args.warmup):
+        o.query_heads(4)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.query_heads(4)
+    dt = time.perf_counter() - t0
+    del lim
+    value = args.steps * 4 / o.heads_per_query / dt
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic, seeded",
+            "config": {"workload": WORKLOAD, "L": o.L, "step": "4 query heads of one decode "
+                       "query (one KV head's tree)", "parallelism": "rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} steps x 4 query heads; "
+                                       "queries/s = query-heads/32/s"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="recsa", choices=["recsa", "reference"])
+    ap.add_argument("--prefill-reps", type=int, default=1)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-dense-prefill", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    R.lib()
+    out = run_recsa(args, rank, world, local)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

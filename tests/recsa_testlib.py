@@ -110,6 +110,8 @@ class Stats:
 
     def check(self, dtype, what=""):
         mx, mn = TOL[dtype]
+        print(f"{what}: max-abs {self.max_abs:.3e} mean-abs {self.mean_abs:.3e} "
+              f"clear {self.clear} near-tie {self.near_tie}")
         assert self.max_abs <= mx, f"{what}: max-abs {self.max_abs:.3e} > {mx}"
         assert self.mean_abs <= mn, f"{what}: mean-abs {self.mean_abs:.3e} > {mn}"
 

@@ -244,8 +244,8 @@ def test_append_matches_build_and_oracle():
     lens_d = torch.tensor(lens0, dtype=torch.int64, device="cuda")
     # The synthetic cache already holds the tokens to append at positions >= len.
     Kw, Vw = Kd.clone(), Vd.clone()
-    Kw[:, :, 4000:] = 0
-    Vw[:, :, 4000:] = 0
+    Kw[0, :, 4000:] = 0
+    Vw[0, :, 4000:] = 0
     Kw[1, :, 4031:] = 0
     Vw[1, :, 4031:] = 0
     og = oracle_geometry(g)
@@ -260,15 +260,18 @@ def test_append_matches_build_and_oracle():
             pos = torch.tensor([[L - 1] for L in lens_now], dtype=torch.int64)
             Q, _, _ = synth.make_queries(w, K, pos, seed=9 + step)
             O = torch.empty_like(Q).cuda()
-            R.recsa_decode(g, Q.cuda(), Kw, Vw, tree, lens_d, 1, O)
+            trace = torch.zeros((2, 1, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                                device="cuda")
+            R.recsa_decode(g, Q.cuda(), Kw, Vw, tree, lens_d, 1, O, trace)
             torch.cuda.synchronize()
+            tr = trace.cpu().numpy()
             for s in range(2):
                 Kh_all = to_np(K[s, :, :lens_now[s]])
                 Vh_all = to_np(V[s, :, :lens_now[s]])
                 for h in range(0, g.n_q_heads, 5):
                     Kh, Vh = Kh_all[h // G], Vh_all[h // G]
                     src = oracle.LazyTree(Kh, Vh, r.double().numpy(), g.leaf_block, g.branching)
-                    check_query(st_out, to_np(O[s, 0, h]), None, to_np(Q[s, 0, h]),
+                    check_query(st_out, to_np(O[s, 0, h]), tr[s, 0, h], to_np(Q[s, 0, h]),
                                 lens_now[s] - 1, Kh, Vh, src, og, g.k)
     torch.cuda.synchronize()
     st_out.check(torch.bfloat16, "decode after append")
