@@ -1,0 +1,586 @@
+// Decode attention on a thread-block cluster per (sequence, query, KV head).
+//
+// Same method as the generic kernel ("Recursive Sparse Attention:
+// Million-Token Length Extrapolation at Logarithmic Cost", abstract: top-down
+// selection of at most k candidates per level, unselected summaries in one
+// softmax with the exact tokens, candidate-local RoPE), laid out for B200:
+//
+//   * The CS CTAs of a cluster split every level's (head, candidate) pairs.
+//     Each CTA scores its share and stores the scores into every CTA's shared
+//     memory (distributed shared memory); one cluster barrier per level, then
+//     each CTA runs the same warp top-k on the full score table, so every CTA
+//     knows the kept nodes without a second exchange.
+//   * Work that does not depend on the selection (the window tokens) runs in
+//     the first pass; the values of a level's unselected candidates are
+//     folded in during the next level's pass, so each level costs one
+//     dependent memory round trip.
+//   * Rows (fp32 summary rows, bf16/fp32 K/V rows) are read straight into
+//     registers with 16-byte loads: a row is spread over d/8 lanes, each lane
+//     holding four rotate-half pairs (j, j + d/2), so the RoPE rotation is
+//     local to the lane.  Each lane slot keeps an online softmax state per
+//     head; states are merged across slots, warps and finally the cluster
+//     (again through distributed shared memory) without any global scratch.
+#include <cooperative_groups.h>
+
+#include "recsa_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace recsa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ unsigned order_key(float f) {
+  const unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Four rotate-half pairs (j0..j0+3, and the same + d/2) of one row, as fp32.
+template <typename T, int HALF>
+struct PairLoad;
+template <int HALF>
+struct PairLoad<float, HALF> {
+  static __device__ __forceinline__ void load(const float* row, int j0, float* x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + j0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(row + HALF + j0));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+template <int HALF>
+struct PairLoad<__nv_bfloat16, HALF> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* row, int j0, float* x) {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + j0));
+    const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + HALF + j0));
+    float2 f;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x)); x[0] = f.x; x[1] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y)); x[2] = f.x; x[3] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x)); x[4] = f.x; x[5] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y)); x[6] = f.x; x[7] = f.y;
+  }
+};
+
+__device__ __forceinline__ void load_cs(const float2* table, int64_t idx, int half, int j0,
+                                        float* cs) {
+  const float4* p = reinterpret_cast<const float4*>(table + idx * half + j0);
+  const float4 a = __ldg(p), b = __ldg(p + 1);
+  cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+  cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+}
+
+// x (4 first-half, 4 second-half values) rotated by the (cos, sin) pairs cs.
+__device__ __forceinline__ void rotate8(float* x, const float* cs) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float c = cs[2 * u], s = cs[2 * u + 1];
+    const float x1 = x[u], x2 = x[u + 4];
+    x[u] = x1 * c - x2 * s;
+    x[u + 4] = x2 * c + x1 * s;
+  }
+}
+
+template <int LPR>
+__device__ __forceinline__ float slot_sum(float v) {
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+enum ItemKind { kKey = 0, kVal = 1, kWin = 2, kTok = 3, kNone = 4 };
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
+                      const T* __restrict__ V, const void* __restrict__ tree,
+                      const int64_t* __restrict__ len_dev, int n_q, T* __restrict__ O,
+                      int32_t* __restrict__ trace, int cmax, int kmax) {
+  constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR, NSLOT = kWarps * SPW;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = int(cluster.num_blocks());
+  const int rank = int(cluster.block_rank());
+  const int qi = blockIdx.y;
+  const int64_t seq = blockIdx.z / p.hkv;
+  const int g = int(blockIdx.z % p.hkv);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane % LPR, slot = warp * SPW + lane / LPR;
+  const int j0 = 4 * sub;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* qf = reinterpret_cast<float*>(smem);          // [G][D] raw query
+  float* qlev = qf + G * D;                            // [G][D] rotated to the level's c
+  float* qtok = qlev + G * D;                          // [G][D] rotated to n0 - 1
+  float* sc = qtok + G * D;                            // [2][G][cmax] scores
+  float* wsc = sc + 2 * G * cmax;                      // [kWarps][G][D + 2] warp merge
+  float* mrg = wsc + kWarps * G * (D + 2);             // [CS][G][D + 2] cluster merge (rank 0)
+  int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
+  unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
+
+  const int64_t t = len_dev[seq] - 1;
+  const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
+  const bool empty = t < 0 || t >= p.cap;   // uniform over the cluster
+  const float2* rope = rope_table(p, tree);
+  const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
+  const int64_t a = empty ? 0 : s0 / p.B;
+  int64_t vis[kMaxLevels + 2];
+  int top = 0;
+  {
+    int64_t per = 1;
+    for (int lev = 1; lev <= p.lay.levels; ++lev) {
+      vis[lev] = a / per;
+      if (vis[lev] == 0) break;
+      top = lev;
+      per *= p.b;
+    }
+  }
+  // Candidate and kept counts per level: the same for every head.
+  int cnt_c[kMaxLevels + 2], cnt_k[kMaxLevels + 2];
+  {
+    int kup = 0;
+    for (int lev = top; lev >= 1; --lev) {
+      const int64_t vup = lev < top ? vis[lev + 1] : 0;
+      cnt_c[lev] = p.b * kup + int(vis[lev] - p.b * vup);
+      cnt_k[lev] = cnt_c[lev] < p.k ? cnt_c[lev] : p.k;
+      kup = cnt_k[lev];
+    }
+  }
+  const int nleaf = top > 0 ? cnt_k[1] : 0;
+  const int64_t n_win = empty ? 0 : t + 1 - a * p.B;
+  const int64_t n0 = int64_t(nleaf) * p.B + n_win;
+
+  for (int x = tid; x < G * D; x += kThreads)
+    qf[x] = empty ? 0.f : load_elem(Q, qrow + x, p.dtype);
+  __syncthreads();
+  auto rotate_q = [&](float* dst, int64_t idx) {
+    for (int x = tid; x < G * HALF; x += kThreads) {
+      const int h = x / HALF, j = x % HALF;
+      const float x1 = qf[h * D + j], x2 = qf[h * D + j + HALF];
+      if (p.rope) {
+        const float2 cs = rope[idx * HALF + j];
+        dst[h * D + j] = x1 * cs.x - x2 * cs.y;
+        dst[h * D + j + HALF] = x2 * cs.x + x1 * cs.y;
+      } else {
+        dst[h * D + j] = x1;
+        dst[h * D + j + HALF] = x2;
+      }
+    }
+  };
+  if (!empty) rotate_q(qtok, n0 - 1 > 0 ? n0 - 1 : 0);
+
+  // Online softmax state of this lane slot: per head (m, l) and 8 channels.
+  float m[G], l[G], acc[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
+  }
+  auto fold = [&](int h, float s, const float* v) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      if (hh == h) {
+        if (s > m[hh]) {
+          const float r = __expf(m[hh] - s);
+          l[hh] = l[hh] * r + 1.f;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[hh][c] = fmaf(acc[hh][c], r, v[c]);
+          m[hh] = s;
+        } else {
+          const float w = __expf(s - m[hh]);
+          l[hh] += w;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) acc[hh][c] = fmaf(w, v[c], acc[hh][c]);
+        }
+      }
+    }
+  };
+
+  const int64_t kvbase = (seq * p.hkv + g) * p.cap;
+  const float inv_sqrt_d = p.inv_sqrt_d;
+  const int tstride = kTraceHead + kMaxLevels * p.k;
+
+  // Node id of candidate i of head h at level lev (kept list of lev + 1 in kept[par]).
+  auto cand_node = [&](int lev, int h, int i) -> int64_t {
+    const int kup = lev < top ? cnt_k[lev + 1] : 0;
+    const int64_t vup = lev < top ? vis[lev + 1] : 0;
+    if (i < p.b * kup) return int64_t(kept[((lev + 1) & 1) * G * kmax + h * kmax + i / p.b]) * p.b + i % p.b;
+    return p.b * vup + (i - int64_t(p.b) * kup);
+  };
+
+  // One pass over this CTA's items: window rows, key pairs of level klev,
+  // unselected value pairs of level vlev, kept-leaf tokens.
+  auto run_pass = [&](int64_t w_lo, int64_t w_hi, int klev, int vlev, bool tokens) {
+    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0;
+    int64_t t_lo = 0, t_hi = 0;
+    if (klev > 0) {
+      const int tot = G * cnt_c[klev], ch = (tot + CS - 1) / CS;
+      k_lo = min(tot, rank * ch);
+      k_hi = min(tot, k_lo + ch);
+    }
+    if (vlev > 0) {
+      const int tot = G * cnt_c[vlev], ch = (tot + CS - 1) / CS;
+      v_lo = min(tot, rank * ch);
+      v_hi = min(tot, v_lo + ch);
+    }
+    if (tokens) {
+      const int64_t tot = int64_t(G) * nleaf * p.B, ch = (tot + CS - 1) / CS;
+      t_lo = min(tot, rank * ch);
+      t_hi = min(tot, t_lo + ch);
+    }
+    const int64_t nw = w_hi - w_lo, nk = k_hi - k_lo, nv = v_hi - v_lo, nt = t_hi - t_lo;
+    const int64_t total = nw + nk + nv + nt;
+    const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
+    const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
+    const int cv = vlev > 0 ? cnt_c[vlev] : 1, ck = klev > 0 ? cnt_c[klev] : 1;
+    for (int64_t base = 0; base < total; base += int64_t(NSLOT) * kUnroll) {
+      float ra[kUnroll][8], rb[kUnroll][8], cs[kUnroll][8];
+      int kind[kUnroll], head[kUnroll], idx[kUnroll];
+      float sv[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t e = base + int64_t(u) * NSLOT + slot;
+        kind[u] = kNone;
+        head[u] = 0;
+        idx[u] = 0;
+        sv[u] = 0.f;
+        if (e < nw) {
+          const int64_t pos = a * p.B + w_lo + e;
+          kind[u] = kWin;
+          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, int64_t(nleaf) * p.B + w_lo + e, HALF, j0, cs[u]);
+        } else if (e < nw + nk) {
+          const int x = int(k_lo + (e - nw));
+          const int h = x / ck, i = x % ck;
+          kind[u] = kKey;
+          head[u] = h;
+          idx[u] = i;
+          PairLoad<float, HALF>::load(keys + cand_node(klev, h, i) * D, j0, ra[u]);
+          if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
+        } else if (e < nw + nk + nv) {
+          const int x = int(v_lo + (e - nw - nk));
+          const int h = x / cv, i = x % cv;
+          if (!kfl[(vlev & 1) * G * cmax + h * cmax + i]) {
+            kind[u] = kVal;
+            head[u] = h;
+            sv[u] = sc[(vlev & 1) * G * cmax + h * cmax + i];
+            PairLoad<float, HALF>::load(vals + cand_node(vlev, h, i) * D, j0, ra[u]);
+          }
+        } else if (e < total) {
+          const int64_t x = t_lo + (e - nw - nk - nv);
+          const int h = int(x / (int64_t(nleaf) * p.B));
+          const int64_t r = x % (int64_t(nleaf) * p.B);
+          const int mb = int(r / p.B), o = int(r % p.B);
+          const int64_t pos = int64_t(kept[(1 & 1) * G * kmax + h * kmax + mb]) * p.B + o;
+          kind[u] = kTok;
+          head[u] = h;
+          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const bool rot = p.rope && (kind[u] == kWin || kind[u] == kKey || kind[u] == kTok);
+        if (rot) rotate8(ra[u], cs[u]);
+        // Dot products: all G heads for a window row, one head otherwise.
+        float sw[G], s1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) sw[h] = 0.f;
+        if (kind[u] == kWin) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float* qv = qtok + h * D;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              sw[h] = fmaf(qv[j0 + c], ra[u][c], sw[h]);
+              sw[h] = fmaf(qv[HALF + j0 + c], ra[u][4 + c], sw[h]);
+            }
+          }
+        } else if (kind[u] == kKey || kind[u] == kTok) {
+          const float* qv = (kind[u] == kKey ? qlev : qtok) + head[u] * D;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            s1 = fmaf(qv[j0 + c], ra[u][c], s1);
+            s1 = fmaf(qv[HALF + j0 + c], ra[u][4 + c], s1);
+          }
+        }
+        // Slot reductions with warp-uniform participation.
+        if (__any_sync(0xffffffffu, kind[u] == kWin)) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) sw[h] = slot_sum<LPR>(sw[h]) * inv_sqrt_d;
+        }
+        if (__any_sync(0xffffffffu, kind[u] == kKey || kind[u] == kTok))
+          s1 = slot_sum<LPR>(s1) * inv_sqrt_d;
+        if (kind[u] == kWin) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) fold(h, sw[h], rb[u]);
+        } else if (kind[u] == kKey) {
+          const int off = (klev & 1) * G * cmax + head[u] * cmax + idx[u];
+          if (sub < CS) *cluster.map_shared_rank(sc + off, sub) = s1;
+          if (sub + LPR < CS) *cluster.map_shared_rank(sc + off, sub + LPR) = s1;
+        } else if (kind[u] == kTok) {
+          fold(head[u], s1, rb[u]);
+        } else if (kind[u] == kVal) {
+          fold(head[u], sv[u], ra[u]);
+        }
+      }
+    }
+  };
+
+  // Warp top-k of head h at level lev over the full score table (every CTA).
+  auto topk = [&](int lev) {
+    const int c = cnt_c[lev], kap = cnt_k[lev];
+    const int par = lev & 1;
+    float* scl = sc + par * G * cmax;
+    unsigned char* fl = kfl + par * G * cmax;
+    int* kp = kept + par * G * kmax;
+    if (warp < G) {
+      const int h = warp;
+      for (int i = lane; i < c; i += 32) fl[h * cmax + i] = (kap >= c) ? 1 : 0;
+      __syncwarp();
+      if (kap < c) {
+        unsigned taken = 0;
+        const int nj = (c + 31) / 32;
+        for (int it = 0; it < kap; ++it) {
+          unsigned bk = 0, bi = 0xffffffffu;
+          for (int jj = 0; jj < nj; ++jj) {
+            const int i = lane + 32 * jj;
+            if (i < c && !((taken >> jj) & 1u)) {
+              const unsigned key = order_key(scl[h * cmax + i]);
+              if (key > bk) { bk = key; bi = unsigned(i); }
+            }
+          }
+          const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
+          const unsigned wi = __reduce_min_sync(0xffffffffu, bk == wk ? bi : 0xffffffffu);
+          if (lane == int(wi & 31u)) taken |= 1u << (wi >> 5);
+          if (lane == 0) fl[h * cmax + wi] = 1;
+        }
+      }
+      __syncwarp();
+      int cnt = 0;
+      for (int j = 0; j < c; j += 32) {
+        const int i = j + lane;
+        const bool f = i < c && fl[h * cmax + i];
+        const unsigned bal = __ballot_sync(0xffffffffu, f);
+        if (f) {
+          const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+          const int node = int(cand_node(lev, h, i));
+          kp[h * kmax + pos] = node;
+          if (trace && rank == 0) {
+            const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
+            trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
+          }
+        }
+        cnt += __popc(bal);
+      }
+    }
+    __syncthreads();
+  };
+
+  // Window share of this CTA (independent of the selection).
+  int64_t w_lo = 0, w_hi = 0;
+  {
+    const int64_t ch = (n_win + CS - 1) / CS;
+    w_lo = min(n_win, int64_t(rank) * ch);
+    w_hi = min(n_win, w_lo + ch);
+  }
+  if (top > 0) {
+    rotate_q(qlev, cnt_c[top]);
+    __syncthreads();
+    run_pass(w_lo, w_hi, top, 0, false);
+    cluster.sync();
+    topk(top);
+    for (int lev = top - 1; lev >= 1; --lev) {
+      rotate_q(qlev, cnt_c[lev]);
+      __syncthreads();
+      run_pass(0, 0, lev, lev + 1, false);
+      cluster.sync();
+      topk(lev);
+    }
+    run_pass(0, 0, 0, 1, true);
+  } else {
+    run_pass(w_lo, w_hi, 0, 0, false);
+  }
+
+  // Merge: slots of a warp, then warps, then the cluster (into rank 0).
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[h], o);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[h], o);
+      const float mn = fmaxf(m[h], mo);
+      const float ra_ = (m[h] == -INFINITY) ? 0.f : __expf(m[h] - mn);
+      const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
+      l[h] = l[h] * ra_ + lo * rb_;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float ao = __shfl_xor_sync(0xffffffffu, acc[h][c], o);
+        acc[h][c] = acc[h][c] * ra_ + ao * rb_;
+      }
+      m[h] = mn;
+    }
+    if (lane < LPR) {
+      float* w = wsc + (warp * G + h) * (D + 2);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        w[j0 + c] = acc[h][c];
+        w[HALF + j0 + c] = acc[h][4 + c];
+      }
+      if (lane == 0) {
+        w[D] = m[h];
+        w[D + 1] = l[h];
+      }
+    }
+  }
+  __syncthreads();
+  // CTA state -> rank 0's merge slot [rank]
+  float* dst = cluster.map_shared_rank(mrg, 0) + rank * G * (D + 2);
+  for (int x = tid; x < G * D; x += kThreads) {
+    const int h = x / D, c = x % D;
+    float mm = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wsc[(w * G + h) * (D + 2) + D]);
+    float aa = 0.f, ll = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float* ws = wsc + (w * G + h) * (D + 2);
+      const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+      aa = fmaf(ws[c], r, aa);
+      ll = fmaf(ws[D + 1], r, ll);
+    }
+    dst[h * (D + 2) + c] = aa;
+    if (c == 0) {
+      dst[h * (D + 2) + D] = mm;
+      dst[h * (D + 2) + D + 1] = ll;
+    }
+  }
+  cluster.sync();
+  if (rank == 0) {
+    for (int x = tid; x < G * D; x += kThreads) {
+      const int h = x / D, c = x % D;
+      float mm = -INFINITY;
+      for (int r = 0; r < CS; ++r) mm = fmaxf(mm, mrg[(r * G + h) * (D + 2) + D]);
+      float aa = 0.f, ll = 0.f;
+      for (int r = 0; r < CS; ++r) {
+        const float* ms = mrg + (r * G + h) * (D + 2);
+        const float w = (ms[D] == -INFINITY) ? 0.f : __expf(ms[D] - mm);
+        aa = fmaf(ms[c], w, aa);
+        ll = fmaf(ms[D + 1], w, ll);
+      }
+      const float o = (empty || ll == 0.f) ? 0.f : aa / ll;
+      store_elem(O, qrow + x, o, p.dtype);
+    }
+    if (trace && !empty) {
+      for (int x = tid; x < G * (kTraceHead + kMaxLevels * p.k); x += kThreads) {
+        const int h = x / tstride, f = x % tstride;
+        const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
+        int v = 0;
+        if (f == 0) v = top;
+        else if (f == 1 || f == 2 || f == 3) {
+          int64_t e = 0, r = 0;
+          for (int lev = 1; lev <= top; ++lev) { e += cnt_c[lev] - cnt_k[lev]; r += cnt_c[lev]; }
+          v = int(f == 1 ? e + n0 : f == 2 ? r + n0 : n0);
+        } else if (f < 4 + kMaxLevels) {
+          const int lev = f - 4 + 1;
+          v = lev <= top ? cnt_c[lev] : 0;
+        } else if (f < kTraceHead) {
+          const int lev = f - 4 - kMaxLevels + 1;
+          v = lev <= top ? cnt_k[lev] : 0;
+        } else {
+          continue;   // kept ids are written per level below
+        }
+        trace[rec + f] = v;
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace recsa
+
+namespace recsa {
+namespace {
+
+template <typename T, int D, int G>
+cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const void* V,
+                          const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
+                          int32_t* trace, cudaStream_t s, int cs) {
+  const int64_t kk = p.k < p.cap ? p.k : p.cap;
+  int64_t maxn = 1;
+  for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
+  int64_t cm = p.b * kk + p.b - 1;
+  cm = cm < maxn ? cm : maxn;
+  const int cmax = int(cm < 1 ? 1 : cm);
+  const int kmax = int(kk < cmax ? kk : cmax);
+  if (cmax > 1024) return cudaErrorNotSupported;
+  const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * G * (D + 2) +
+                        size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
+                       size_t(2) * G * cmax + 16;
+  if (bytes > 200 * 1024) return cudaErrorNotSupported;
+  auto kern = decode_cluster_kernel<T, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(bytes));
+  if (e != cudaSuccess) return e;
+  if (cs > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  if (int64_t(p.batch) * p.hkv > 65535 || n_q > 65535) return cudaErrorNotSupported;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, n_q, unsigned(p.batch * p.hkv));
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, reinterpret_cast<const T*>(Q),
+                            reinterpret_cast<const T*>(K), reinterpret_cast<const T*>(V), tree,
+                            len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax);
+}
+
+template <typename T, int D>
+cudaError_t cluster_g(const Params& p, const void* Q, const void* K, const void* V,
+                      const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
+                      int32_t* trace, cudaStream_t s, int cs) {
+  switch (p.group) {
+    case 1: return cluster_typed<T, D, 1>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+    case 2: return cluster_typed<T, D, 2>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+    case 4: return cluster_typed<T, D, 4>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace
+
+int decode_cluster_size(const Params& p, int32_t n_q) {
+  const char* env = getenv("RECSA_DECODE_CLUSTER");
+  if (env) {
+    const int v = atoi(env);
+    if (v == 1 || v == 2 || v == 4 || v == 8 || v == 16) return v;
+  }
+  const int64_t clusters = int64_t(p.batch) * p.hkv * n_q;
+  int cs = 2;
+  while (cs < 16 && clusters * cs * 2 <= 148) cs *= 2;
+  return cs;
+}
+
+cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
+                                  const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
+                                  int32_t* trace, cudaStream_t s) {
+  const int cs = decode_cluster_size(p, n_q);
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs)
+                      : cluster_g<__nv_bfloat16, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+  return p.d == 128 ? cluster_g<float, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs)
+                    : cluster_g<float, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+}
+
+}  // namespace recsa

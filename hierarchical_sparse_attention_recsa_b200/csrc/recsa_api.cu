@@ -1,5 +1,6 @@
 // C-ABI entry points: argument checks, tree layout and launches.
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -201,7 +202,13 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
   if (n_q == 0) return RECSA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_attend(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);
+  cudaError_t e = cudaErrorNotSupported;
+  if (decode && !getenv("RECSA_DECODE_GENERIC"))
+    e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_attend(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);
+  }
   if (e == cudaErrorInvalidConfiguration || e == cudaErrorInvalidValue) {
     cudaGetLastError();
     return RECSA_ERR_UNSUPPORTED;

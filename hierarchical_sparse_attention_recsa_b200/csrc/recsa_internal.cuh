@@ -86,5 +86,9 @@ cudaError_t launch_append(const Params& p, void* K, void* V, const void* k_new, 
 cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const void* V,
                           const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
                           int decode, void* O, int32_t* trace, cudaStream_t s);
+// Cluster decode kernel; cudaErrorNotSupported when the geometry is outside its limits.
+cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
+                                  const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
+                                  int32_t* trace, cudaStream_t s);
 
 }  // namespace recsa

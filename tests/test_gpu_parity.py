@@ -4,6 +4,8 @@ Sizes span several tiles and ragged tails while the oracle still finishes in
 seconds; tolerances and the selection rule are stated in recsa_testlib.
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -22,6 +24,27 @@ pytestmark = pytest.mark.gpu
 def _lib():
     build_lib.build()
     R.lib()
+
+
+@pytest.fixture(params=["cluster-auto", "cluster-2", "cluster-4", "cluster-8", "cluster-16",
+                        "generic"])
+def decode_impl(request):
+    """Select the decode kernel: the cluster kernel (auto or forced cluster size)
+    or the generic one-CTA-per-query kernel."""
+    keys = ("RECSA_DECODE_CLUSTER", "RECSA_DECODE_GENERIC")
+    old = {k: os.environ.get(k) for k in keys}
+    for k in keys:
+        os.environ.pop(k, None)
+    if request.param == "generic":
+        os.environ["RECSA_DECODE_GENERIC"] = "1"
+    elif request.param != "cluster-auto":
+        os.environ["RECSA_DECODE_CLUSTER"] = request.param.split("-")[1]
+    yield request.param
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
 
 
 def _setup(w, lens, capacity, seed=0, k=None, rope=1):
@@ -77,7 +100,7 @@ def test_tree_tiny(tiny):
     _check_tree(g, tree, trees, torch.float32)
 
 
-def test_decode_tiny_256_queries(tiny):
+def test_decode_tiny_256_queries(tiny, decode_impl):
     g, K, V, r, Kd, Vd, rd, tree, trees = tiny
     L, nq = TINY.length, TINY.n_q
     pos = torch.full((1, nq), L - 1, dtype=torch.int64)
@@ -149,7 +172,7 @@ def test_tree_model_small(model_small):
     _check_tree(g, tree, trees, torch.bfloat16)
 
 
-def test_decode_model_small(model_small):
+def test_decode_model_small(model_small, decode_impl):
     g, lens, K, V, r, Kd, Vd, rd, tree, trees = model_small
     nq = 3
     pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
