@@ -62,19 +62,30 @@ class Clocks:
     def __init__(self, device: int):
         self.proc = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device}.csv")
+        self.sel = []
         try:
-            uuid = str(torch.cuda.get_device_properties(device).uuid)
-            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+            uuid = str(torch.cuda.get_device_properties(device).uuid).lower()
+            rows = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid",
+                                   "--format=csv,noheader"], capture_output=True, text=True,
+                                  timeout=20).stdout.strip().splitlines()
+            for row in rows:
+                idx, u = [x.strip() for x in row.split(",")]
+                if uuid.replace("gpu-", "") in u.lower():
+                    self.sel = ["-i", idx]
         except Exception:
-            self.sel = []
+            pass
 
     def start(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", *self.sel, "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
+            # wait for the first sample so that the timed region is covered
+            t0 = time.time()
+            while time.time() - t0 < 10 and os.path.getsize(self.path) == 0:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
 
@@ -142,6 +153,8 @@ def make_prefill_queries(w, K, L, chunk=65536):
 
 def run_recsa(args, rank, world, dev):
     w = synth.WORKLOADS[WORKLOAD]
+    if args.length:
+        w = synth.Workload(**{**w.__dict__, "length": args.length})
     L, batch = w.length, w.batch
     K_steps, W_steps = args.steps, args.warmup
     n_stage = max(K_steps, W_steps)
@@ -171,16 +184,16 @@ def run_recsa(args, rank, world, dev):
         R.recsa_append(g, Kc, Vc, kn[i], vn[i], lens, r, 0, tree)
         R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O)
 
+    clocks = Clocks(dev)
+    clocks.start()      # samples the warm-up, the timed steps and the e2e steps
     for i in range(W_steps):
         step(i)
     lens.copy_(lens0)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
-    clocks = Clocks(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    clocks.start()
     for i in range(K_steps):
         flush()
         ev[i][0].record(stream)
@@ -193,7 +206,6 @@ def run_recsa(args, rank, world, dev):
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clk = clocks.stop()
     step_ms = sum(elapsed(e[0], e[2]) for e in ev)
     dec_ms = sum(elapsed(e[1], e[2]) for e in ev) / K_steps
     app_ms = sum(elapsed(e[0], e[1]) for e in ev) / K_steps
@@ -215,32 +227,36 @@ def run_recsa(args, rank, world, dev):
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
 
     # end to end through the public API with host buffers
-    Qh = Qs.cpu().pin_memory()
-    knh, vnh = kn.cpu().pin_memory(), vn.cpu().pin_memory()
-    Oh = torch.empty((K_steps,) + tuple(O.shape), dtype=O.dtype).pin_memory()
-    Qd, knd, vnd = torch.empty_like(Qs[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
-    lens.copy_(lens0)
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
-    torch.cuda.synchronize()
-    for i in range(K_steps):
-        flush()
-        ev2[i][0].record(stream)
-        Qd.copy_(Qh[i], non_blocking=True)
-        knd.copy_(knh[i], non_blocking=True)
-        vnd.copy_(vnh[i], non_blocking=True)
-        R.recsa_append(g, Kc, Vc, knd, vnd, lens, r, 0, tree)
-        R.recsa_decode(g, Qd, Kc, Vc, tree, lens, 1, O)
-        Oh[i].copy_(O, non_blocking=True)
-        ev2[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = sum(elapsed(a, b) for a, b in ev2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": batch * K_steps * world / (e2e_ms / 1e3), "unit": "queries/s",
-           "h2d_bytes_per_step": int(Qd.numel() * 2 + knd.numel() * 2 + vnd.numel() * 2),
-           "d2h_bytes_per_step": int(O.numel() * 2)}
+    def run_e2e():
+        Qh = Qs.cpu().pin_memory()
+        knh, vnh = kn.cpu().pin_memory(), vn.cpu().pin_memory()
+        Oh = torch.empty((K_steps,) + tuple(O.shape), dtype=O.dtype).pin_memory()
+        Qd, knd, vnd = torch.empty_like(Qs[0]), torch.empty_like(kn[0]), torch.empty_like(vn[0])
+        lens.copy_(lens0)
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
+        torch.cuda.synchronize()
+        for i in range(K_steps):
+            flush()
+            ev2[i][0].record(stream)
+            Qd.copy_(Qh[i], non_blocking=True)
+            knd.copy_(knh[i], non_blocking=True)
+            vnd.copy_(vnh[i], non_blocking=True)
+            R.recsa_append(g, Kc, Vc, knd, vnd, lens, r, 0, tree)
+            R.recsa_decode(g, Qd, Kc, Vc, tree, lens, 1, O)
+            Oh[i].copy_(O, non_blocking=True)
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(elapsed(a, b) for a, b in ev2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        return {"value": batch * K_steps * world / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": int(Qd.numel() * 2 + knd.numel() * 2 + vnd.numel() * 2),
+                "d2h_bytes_per_step": int(O.numel() * 2)}
+
+    e2e = None if args.only_decode else run_e2e()
+    clk = clocks.stop()
 
     out = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
@@ -482,8 +498,14 @@ def main():
     ap.add_argument("--no-dense-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only-decode", action="store_true",
+                    help="decode steps only (no prefill, dense, e2e or CPU legs); for profiling")
+    ap.add_argument("--length", type=int, default=0,
+                    help="override the context length (smaller cases for ncu captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.only_decode:
+        args.no_prefill = args.no_dense = args.no_cpu = True
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
