@@ -279,7 +279,7 @@ def run_recsa(args, rank, world, dev):
         "decode_ms": dec_ms, "append_ms": app_ms,
         "e2e": e2e, "gpu_launches": 2 * K_steps, "clocks": clk,
     }
-    del traces, Qh, Oh
+    del traces
     torch.cuda.empty_cache()
     if not args.no_prefill:
         out["prefill"] = run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs)

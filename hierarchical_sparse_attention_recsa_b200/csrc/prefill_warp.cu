@@ -1,0 +1,344 @@
+// Prefill attention: one warp per (query, head); a CTA's eight warps serve two
+// consecutive queries of one KV group, so their window and upper-level rows
+// are shared through L1.
+//
+// Per query ("Recursive Sparse Attention: Million-Token Length Extrapolation at
+// Logarithmic Cost", abstract): the window tokens and the top level are scored
+// in the first pass; every later pass scores one level's candidates while
+// folding the previous level's unselected summaries into the online softmax;
+// the last pass folds level 1's unselected summaries and the kept leaves'
+// tokens.  Selection is a warp top-k (redux.sync on order-preserving keys,
+// ties to the lower index).  Rows are read into registers with vector loads,
+// d/8 lanes per row, four rotate-half pairs per lane.  No block-level
+// barriers: every warp runs independently, so many queries are in flight per
+// SM to cover the dependent gathers.
+#include "recsa_internal.cuh"
+#include "rows.cuh"
+
+namespace recsa {
+namespace {
+
+constexpr int kPThreads = 256;
+constexpr int kPWarps = kPThreads / 32;
+constexpr int kPUnroll = 2;
+
+enum PItem { pKey = 0, pVal = 1, pTok = 2, pNone = 3 };
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kPThreads, 2)
+prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
+                    const T* __restrict__ V, const void* __restrict__ tree, int64_t q_start,
+                    int n_q, T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
+                    int warp_bytes) {
+  constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR;
+  const int G = p.group;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % LPR, slot = lane / LPR, j0 = 4 * sub;
+  const int64_t item = int64_t(blockIdx.x) * kPWarps + warp;
+  const int64_t seq = blockIdx.y / p.hkv;
+  const int g = int(blockIdx.y % p.hkv);
+  if (item >= int64_t(n_q) * G) return;   // whole warp exits; no block barriers follow
+  const int qi = int(item / G);
+  const int h = g * G + int(item % G);
+  const int64_t t = q_start + qi;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* qf = reinterpret_cast<float*>(smem + size_t(warp) * warp_bytes);
+  float* qlev = qf + D;
+  float* qtok = qlev + D;
+  float* sc = qtok + D;                                          // [2][cmax]
+  int* kept = reinterpret_cast<int*>(sc + 2 * cmax);             // [2][kmax]
+  unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * kmax);  // [2][cmax]
+
+  const float2* rope = rope_table(p, tree);
+  const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
+  const int64_t a = s0 / p.B;
+  int64_t vis[kMaxLevels + 2];
+  int top = 0;
+  {
+    int64_t per = 1;
+    for (int lev = 1; lev <= p.lay.levels; ++lev) {
+      vis[lev] = a / per;
+      if (vis[lev] == 0) break;
+      top = lev;
+      per *= p.b;
+    }
+  }
+  int cnt_c[kMaxLevels + 2], cnt_k[kMaxLevels + 2];
+  {
+    int kup = 0;
+    for (int lev = top; lev >= 1; --lev) {
+      const int64_t vup = lev < top ? vis[lev + 1] : 0;
+      cnt_c[lev] = p.b * kup + int(vis[lev] - p.b * vup);
+      cnt_k[lev] = cnt_c[lev] < p.k ? cnt_c[lev] : p.k;
+      kup = cnt_k[lev];
+    }
+  }
+  const int nleaf = top > 0 ? cnt_k[1] : 0;
+  const int64_t n_win = t + 1 - a * p.B;
+  const int64_t n0 = int64_t(nleaf) * p.B + n_win;
+  const int64_t qrow = ((seq * n_q + qi) * p.hq + h) * D;
+  for (int x = lane; x < D; x += 32) qf[x] = load_elem(Q, qrow + x, p.dtype);
+  __syncwarp();
+  auto rotate_q = [&](float* dst, int64_t idx) {
+    for (int j = lane; j < HALF; j += 32) {
+      const float x1 = qf[j], x2 = qf[j + HALF];
+      if (p.rope) {
+        const float2 cs = rope[idx * HALF + j];
+        dst[j] = x1 * cs.x - x2 * cs.y;
+        dst[j + HALF] = x2 * cs.x + x1 * cs.y;
+      } else {
+        dst[j] = x1;
+        dst[j + HALF] = x2;
+      }
+    }
+    __syncwarp();
+  };
+  rotate_q(qtok, n0 - 1);
+
+  float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  auto fold = [&](float s, const float* v) {
+    if (s > m) {
+      const float r = __expf(m - s);
+      l = l * r + 1.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
+      m = s;
+    } else {
+      const float w = __expf(s - m);
+      l += w;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
+    }
+  };
+
+  const int64_t kvbase = (seq * p.hkv + g) * p.cap;
+  const float inv_sqrt_d = p.inv_sqrt_d;
+  const int tstride = kTraceHead + kMaxLevels * p.k;
+  const int64_t rec = ((seq * n_q + qi) * p.hq + h) * int64_t(tstride);
+
+  auto cand_node = [&](int lev, int i) -> int64_t {
+    const int kup = lev < top ? cnt_k[lev + 1] : 0;
+    const int64_t vup = lev < top ? vis[lev + 1] : 0;
+    if (i < p.b * kup) return int64_t(kept[((lev + 1) & 1) * kmax + i / p.b]) * p.b + i % p.b;
+    return p.b * vup + (i - int64_t(p.b) * kup);
+  };
+
+  // Window rows (first pass), key pairs of klev, unselected values of vlev,
+  // kept-leaf tokens (last pass).
+  auto run_pass = [&](bool window, int klev, int vlev, bool tokens) {
+    const int64_t nw = window ? n_win : 0;
+    const int64_t nk = klev > 0 ? cnt_c[klev] : 0;
+    const int64_t nv = vlev > 0 ? cnt_c[vlev] : 0;
+    const int64_t nt = tokens ? int64_t(nleaf) * p.B : 0;
+    const int64_t total = nw + nk + nv + nt;
+    const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
+    const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
+    for (int64_t base = 0; base < total; base += int64_t(SPW) * kPUnroll) {
+      float ra[kPUnroll][8], rb[kPUnroll][8], cs[kPUnroll][8];
+      int kind[kPUnroll], idx[kPUnroll];
+      float sv[kPUnroll];
+#pragma unroll
+      for (int u = 0; u < kPUnroll; ++u) {
+        const int64_t e = base + int64_t(u) * SPW + slot;
+        kind[u] = pNone;
+        idx[u] = 0;
+        sv[u] = 0.f;
+        if (e < nw) {
+          const int64_t pos = a * p.B + e;
+          kind[u] = pTok;
+          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, int64_t(nleaf) * p.B + e, HALF, j0, cs[u]);
+        } else if (e < nw + nk) {
+          const int i = int(e - nw);
+          kind[u] = pKey;
+          idx[u] = i;
+          PairLoad<float, HALF>::load(keys + cand_node(klev, i) * D, j0, ra[u]);
+          if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
+        } else if (e < nw + nk + nv) {
+          const int i = int(e - nw - nk);
+          if (!kfl[(vlev & 1) * cmax + i]) {
+            kind[u] = pVal;
+            sv[u] = sc[(vlev & 1) * cmax + i];
+            PairLoad<float, HALF>::load(vals + cand_node(vlev, i) * D, j0, ra[u]);
+          }
+        } else if (e < total) {
+          const int64_t r = e - nw - nk - nv;
+          const int mb = int(r / p.B), o = int(r % p.B);
+          const int64_t pos = int64_t(kept[1 * kmax + mb]) * p.B + o;   // level 1 = parity 1
+          kind[u] = pTok;
+          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPUnroll; ++u) {
+        float s = 0.f;
+        if (kind[u] == pKey || kind[u] == pTok) {
+          if (p.rope) rotate8(ra[u], cs[u]);
+          const float* qv = kind[u] == pKey ? qlev : qtok;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            s = fmaf(qv[j0 + c], ra[u][c], s);
+            s = fmaf(qv[HALF + j0 + c], ra[u][4 + c], s);
+          }
+        }
+        if (__any_sync(0xffffffffu, kind[u] == pKey || kind[u] == pTok))
+          s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (kind[u] == pKey) {
+          if (sub == 0) sc[(klev & 1) * cmax + idx[u]] = s;
+        } else if (kind[u] == pTok) {
+          fold(s, rb[u]);
+        } else if (kind[u] == pVal) {
+          fold(sv[u], ra[u]);
+        }
+      }
+    }
+    __syncwarp();
+  };
+
+  auto topk = [&](int lev) {
+    const int c = cnt_c[lev], kap = cnt_k[lev];
+    const int par = lev & 1;
+    const float* scl = sc + par * cmax;
+    unsigned char* fl = kfl + par * cmax;
+    int* kp = kept + par * kmax;
+    for (int i = lane; i < c; i += 32) fl[i] = (kap >= c) ? 1 : 0;
+    __syncwarp();
+    if (kap < c) {
+      unsigned taken = 0;
+      const int nj = (c + 31) / 32;
+      for (int it = 0; it < kap; ++it) {
+        unsigned bk = 0, bi = 0xffffffffu;
+        for (int jj = 0; jj < nj; ++jj) {
+          const int i = lane + 32 * jj;
+          if (i < c && !((taken >> jj) & 1u)) {
+            const unsigned key = order_key(scl[i]);
+            if (key > bk) { bk = key; bi = unsigned(i); }
+          }
+        }
+        const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
+        const unsigned wi = __reduce_min_sync(0xffffffffu, bk == wk ? bi : 0xffffffffu);
+        if (lane == int(wi & 31u)) taken |= 1u << (wi >> 5);
+        if (lane == 0) fl[wi] = 1;
+      }
+    }
+    __syncwarp();
+    int cnt = 0;
+    for (int j = 0; j < c; j += 32) {
+      const int i = j + lane;
+      const bool f = i < c && fl[i];
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (f) {
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        const int node = int(cand_node(lev, i));
+        kp[pos] = node;
+        if (trace) trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
+      }
+      cnt += __popc(bal);
+    }
+    __syncwarp();
+  };
+
+  if (top > 0) {
+    rotate_q(qlev, cnt_c[top]);
+    run_pass(true, top, 0, false);
+    topk(top);
+    for (int lev = top - 1; lev >= 1; --lev) {
+      rotate_q(qlev, cnt_c[lev]);
+      run_pass(false, lev, lev + 1, false);
+      topk(lev);
+    }
+    run_pass(false, 0, 1, true);
+  } else {
+    run_pass(true, 0, 0, false);
+  }
+
+  // merge the lane slots, write O
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+    const float mn = fmaxf(m, mo);
+    const float ra_ = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
+    l = l * ra_ + lo * rb_;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float ao = __shfl_xor_sync(0xffffffffu, acc[c], o);
+      acc[c] = acc[c] * ra_ + ao * rb_;
+    }
+    m = mn;
+  }
+  if (lane < LPR) {
+    const float il = 1.f / l;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      store_elem(O, qrow + j0 + c, acc[c] * il, p.dtype);
+      store_elem(O, qrow + HALF + j0 + c, acc[4 + c] * il, p.dtype);
+    }
+  }
+  if (trace && lane == 0) {
+    int64_t e = 0, r = 0;
+    for (int lev = 1; lev <= top; ++lev) {
+      e += cnt_c[lev] - cnt_k[lev];
+      r += cnt_c[lev];
+    }
+    trace[rec + 0] = top;
+    trace[rec + 1] = int32_t(e + n0);
+    trace[rec + 2] = int32_t(r + n0);
+    trace[rec + 3] = int32_t(n0);
+    for (int lev = 1; lev <= kMaxLevels; ++lev) {
+      trace[rec + 4 + lev - 1] = lev <= top ? cnt_c[lev] : 0;
+      trace[rec + 4 + kMaxLevels + lev - 1] = lev <= top ? cnt_k[lev] : 0;
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const void* V,
+                          const void* tree, int64_t q_start, int32_t n_q, void* O, int32_t* trace,
+                          cudaStream_t s) {
+  const int64_t kk = p.k < p.cap ? p.k : p.cap;
+  int64_t maxn = 1;
+  for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
+  int64_t cm = p.b * kk + p.b - 1;
+  cm = cm < maxn ? cm : maxn;
+  const int cmax = int(cm < 1 ? 1 : cm);
+  const int kmax = int(kk < cmax ? kk : cmax);
+  if (cmax > 1024) return cudaErrorNotSupported;
+  const int warp_bytes = int(((3 * D + 2 * cmax) * 4 + 2 * kmax * 4 + 2 * cmax + 15) / 16 * 16);
+  const size_t bytes = size_t(warp_bytes) * kPWarps;
+  if (bytes > 200 * 1024) return cudaErrorNotSupported;
+  auto kern = prefill_warp_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(bytes));
+  if (e != cudaSuccess) return e;
+  const int64_t items = int64_t(n_q) * p.group;
+  const int64_t blocks = (items + kPWarps - 1) / kPWarps;
+  if (blocks > 0x7fffffff || int64_t(p.batch) * p.hkv > 65535) return cudaErrorNotSupported;
+  dim3 grid(unsigned(blocks), unsigned(p.batch * p.hkv));
+  kern<<<grid, kPThreads, bytes, s>>>(p, reinterpret_cast<const T*>(Q),
+                                      reinterpret_cast<const T*>(K),
+                                      reinterpret_cast<const T*>(V), tree, q_start, n_q,
+                                      reinterpret_cast<T*>(O), trace, cmax, kmax, warp_bytes);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
+                                const void* tree, int64_t q_start, int32_t n_q, void* O,
+                                int32_t* trace, cudaStream_t s) {
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, s)
+                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, s)
+                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+}
+
+}  // namespace recsa

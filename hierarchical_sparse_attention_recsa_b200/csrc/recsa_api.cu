@@ -205,6 +205,8 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   cudaError_t e = cudaErrorNotSupported;
   if (decode && !getenv("RECSA_DECODE_GENERIC"))
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
+  if (!decode && !getenv("RECSA_PREFILL_GENERIC"))
+    e = launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, s);
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
     e = launch_attend(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);

@@ -90,5 +90,9 @@ cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const v
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);
+// Warp-per-(query, head) prefill kernel; cudaErrorNotSupported outside its limits.
+cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
+                                const void* tree, int64_t q_start, int32_t n_q, void* O,
+                                int32_t* trace, cudaStream_t s);
 
 }  // namespace recsa

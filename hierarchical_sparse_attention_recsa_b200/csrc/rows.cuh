@@ -1,0 +1,68 @@
+// Row-access helpers shared by the cluster decode and the warp prefill kernels.
+//
+// A row of d values is spread over d/8 lanes; each lane holds four rotate-half
+// pairs (j0..j0+3 and j0+d/2..j0+d/2+3), so RoPE rotation is local to the lane
+// and every load is a 16-byte (fp32) or 8-byte (bf16) vector.
+#pragma once
+
+#include "recsa_internal.cuh"
+
+namespace recsa {
+
+__device__ __forceinline__ unsigned order_key(float f) {
+  const unsigned u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Four rotate-half pairs (j0..j0+3, and the same + d/2) of one row, as fp32.
+template <typename T, int HALF>
+struct PairLoad;
+template <int HALF>
+struct PairLoad<float, HALF> {
+  static __device__ __forceinline__ void load(const float* row, int j0, float* x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(row + j0));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(row + HALF + j0));
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+template <int HALF>
+struct PairLoad<__nv_bfloat16, HALF> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* row, int j0, float* x) {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + j0));
+    const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + HALF + j0));
+    float2 f;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x)); x[0] = f.x; x[1] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y)); x[2] = f.x; x[3] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x)); x[4] = f.x; x[5] = f.y;
+    f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y)); x[6] = f.x; x[7] = f.y;
+  }
+};
+
+__device__ __forceinline__ void load_cs(const float2* table, int64_t idx, int half, int j0,
+                                        float* cs) {
+  const float4* p = reinterpret_cast<const float4*>(table + idx * half + j0);
+  const float4 a = __ldg(p), b = __ldg(p + 1);
+  cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+  cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+}
+
+// x (4 first-half, 4 second-half values) rotated by the (cos, sin) pairs cs.
+__device__ __forceinline__ void rotate8(float* x, const float* cs) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float c = cs[2 * u], s = cs[2 * u + 1];
+    const float x1 = x[u], x2 = x[u + 4];
+    x[u] = x1 * c - x2 * s;
+    x[u + 4] = x2 * c + x1 * s;
+  }
+}
+
+template <int LPR>
+__device__ __forceinline__ float slot_sum(float v) {
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace recsa

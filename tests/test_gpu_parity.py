@@ -47,6 +47,18 @@ def decode_impl(request):
             os.environ[k] = v
 
 
+@pytest.fixture(params=["warp", "generic"])
+def prefill_impl(request):
+    """Select the prefill kernel: warp-per-(query, head) or the generic kernel."""
+    old = os.environ.pop("RECSA_PREFILL_GENERIC", None)
+    if request.param == "generic":
+        os.environ["RECSA_PREFILL_GENERIC"] = "1"
+    yield request.param
+    os.environ.pop("RECSA_PREFILL_GENERIC", None)
+    if old is not None:
+        os.environ["RECSA_PREFILL_GENERIC"] = old
+
+
 def _setup(w, lens, capacity, seed=0, k=None, rope=1):
     batch = len(lens)
     g = geometry(w, capacity, batch, k=k, rope=rope)
@@ -126,7 +138,7 @@ def test_decode_tiny_256_queries(tiny, decode_impl):
     assert st.clear > 0.8 * nq * g.n_q_heads
 
 
-def test_prefill_tiny_all_positions(tiny):
+def test_prefill_tiny_all_positions(tiny, prefill_impl):
     g, K, V, r, Kd, Vd, rd, tree, trees = tiny
     L = TINY.length
     pos = torch.arange(L, dtype=torch.int64)[None]
@@ -197,7 +209,7 @@ def test_decode_model_small(model_small, decode_impl):
     st.check(torch.bfloat16, "decode model small")
 
 
-def test_prefill_model_small(model_small):
+def test_prefill_model_small(model_small, prefill_impl):
     g, lens, K, V, r, Kd, Vd, rd, tree, trees = model_small
     q0, nq = 12000, 1001                # ends at 13001 = the shorter sequence's length
     pos = (q0 + torch.arange(nq, dtype=torch.int64))[None].expand(2, nq)
@@ -227,7 +239,7 @@ def test_prefill_model_small(model_small):
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("wname,rope", [("tiny-4k", 1), ("tiny-4k", 0), ("qwen3-4b-131k", 1)])
-def test_keep_all_is_dense(wname, rope):
+def test_keep_all_is_dense(wname, rope, prefill_impl):
     w = synth.WORKLOADS[wname]
     L = 1500 if w.head_dim == 64 else 700
     g, K, V, r, Kd, Vd, rd, tree = _setup(w, [L], L, seed=6, k=R.KEEP_ALL, rope=rope)
