@@ -30,9 +30,9 @@ namespace cg = cooperative_groups;
 namespace recsa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;
 
 enum ItemKind { kKey = 0, kVal = 1, kWin = 2, kTok = 3, kNone = 4 };
 
@@ -148,89 +148,122 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int tstride = kTraceHead + kMaxLevels * p.k;
 
   // Node id of candidate i of head h at level lev (kept list of lev + 1 in kept[par]).
-  auto cand_node = [&](int lev, int h, int i) -> int64_t {
+  auto cand_node = [&](int lev, int h, int i) -> int {
     const int kup = lev < top ? cnt_k[lev + 1] : 0;
-    const int64_t vup = lev < top ? vis[lev + 1] : 0;
-    if (i < p.b * kup) return int64_t(kept[((lev + 1) & 1) * G * kmax + h * kmax + i / p.b]) * p.b + i % p.b;
-    return p.b * vup + (i - int64_t(p.b) * kup);
+    const int vup = lev < top ? int(vis[lev + 1]) : 0;
+    if (i < p.b * kup)
+      return kept[((lev + 1) & 1) * G * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
+    return p.b * vup + (i - p.b * kup);
+  };
+  // Head of flattened pair x with c pairs per head (G <= 4: compares only).
+  auto head_of = [&](int x, int c) -> int {
+    int h = 0;
+#pragma unroll
+    for (int hh = 1; hh < G; ++hh) h += x >= hh * c;
+    return h;
   };
 
   // One pass over this CTA's items: window rows, key pairs of level klev,
-  // unselected value pairs of level vlev, kept-leaf tokens.
-  auto run_pass = [&](int64_t w_lo, int64_t w_hi, int klev, int vlev, bool tokens) {
-    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0;
-    int64_t t_lo = 0, t_hi = 0;
+  // unselected value pairs of level vlev, kept-leaf tokens.  All index math is
+  // 32-bit and the per-level constants are hoisted out of the item loop.
+  auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
+    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0, t_lo = 0, t_hi = 0;
+    const int ck = klev > 0 ? cnt_c[klev] : 1, cv = vlev > 0 ? cnt_c[vlev] : 1;
+    const int nlb = nleaf * p.B;
     if (klev > 0) {
-      const int tot = G * cnt_c[klev], ch = (tot + CS - 1) / CS;
+      const int tot = G * ck, ch = (tot + CS - 1) / CS;
       k_lo = min(tot, rank * ch);
       k_hi = min(tot, k_lo + ch);
     }
     if (vlev > 0) {
-      const int tot = G * cnt_c[vlev], ch = (tot + CS - 1) / CS;
+      const int tot = G * cv, ch = (tot + CS - 1) / CS;
       v_lo = min(tot, rank * ch);
       v_hi = min(tot, v_lo + ch);
     }
     if (tokens) {
-      const int64_t tot = int64_t(G) * nleaf * p.B, ch = (tot + CS - 1) / CS;
+      const int tot = G * nlb, ch = (tot + CS - 1) / CS;
       t_lo = min(tot, rank * ch);
       t_hi = min(tot, t_lo + ch);
     }
-    const int64_t nw = w_hi - w_lo, nk = k_hi - k_lo, nv = v_hi - v_lo, nt = t_hi - t_lo;
-    const int64_t total = nw + nk + nv + nt;
+    const int nw = w_hi - w_lo, nk = k_hi - k_lo, nv = v_hi - v_lo, nt = t_hi - t_lo;
+    const int total = nw + nk + nv + nt;
     const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
     const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
-    const int cv = vlev > 0 ? cnt_c[vlev] : 1, ck = klev > 0 ? cnt_c[klev] : 1;
-    for (int64_t base = 0; base < total; base += int64_t(NSLOT) * kUnroll) {
-      float ra[kUnroll][8], rb[kUnroll][8], cs[kUnroll][8];
+    // candidate -> node maps of the two levels: i < nch -> kept parent child, else orph + i
+    const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
+    const int nchK = p.b * kupK;
+    const int orphK = (klev > 0 && klev < top) ? p.b * int(vis[klev + 1]) - nchK : 0;
+    const int* keptK = kept + ((klev + 1) & 1) * G * kmax;
+    const int kupV = (vlev > 0 && vlev < top) ? cnt_k[vlev + 1] : 0;
+    const int nchV = p.b * kupV;
+    const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
+    const int* keptV = kept + ((vlev + 1) & 1) * G * kmax;
+    const int* kept1 = kept + 1 * G * kmax;                       // level 1 = parity 1
+    const float* scV = sc + (vlev & 1) * G * cmax;
+    const unsigned char* flV = kfl + (vlev & 1) * G * cmax;
+    const int win0 = int(a) * p.B + w_lo;
+    const int widx0 = nlb + w_lo;
+    for (int base = 0; base < total; base += NSLOT * kUnroll) {
+      RawPairs ra[kUnroll], rb[kUnroll];
+      float cs[kUnroll][8];
       int kind[kUnroll], head[kUnroll], idx[kUnroll];
       float sv[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        const int64_t e = base + int64_t(u) * NSLOT + slot;
+        const int e = base + u * NSLOT + slot;
         kind[u] = kNone;
         head[u] = 0;
         idx[u] = 0;
         sv[u] = 0.f;
         if (e < nw) {
-          const int64_t pos = a * p.B + w_lo + e;
+          const int pos = win0 + e;
           kind[u] = kWin;
-          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
-          if (p.rope) load_cs(rope, int64_t(nleaf) * p.B + w_lo + e, HALF, j0, cs[u]);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
         } else if (e < nw + nk) {
-          const int x = int(k_lo + (e - nw));
-          const int h = x / ck, i = x % ck;
+          const int x = k_lo + (e - nw);
+          const int h = head_of(x, ck), i = x - h * ck;
+          const int node = i < nchK ? keptK[h * kmax + div_b(p, i)] * p.b + mod_b(p, i)
+                                    : orphK + i;
           kind[u] = kKey;
           head[u] = h;
           idx[u] = i;
-          PairLoad<float, HALF>::load(keys + cand_node(klev, h, i) * D, j0, ra[u]);
+          RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
           if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
         } else if (e < nw + nk + nv) {
-          const int x = int(v_lo + (e - nw - nk));
-          const int h = x / cv, i = x % cv;
-          if (!kfl[(vlev & 1) * G * cmax + h * cmax + i]) {
+          const int x = v_lo + (e - nw - nk);
+          const int h = head_of(x, cv), i = x - h * cv;
+          if (!flV[h * cmax + i]) {
+            const int node = i < nchV ? keptV[h * kmax + div_b(p, i)] * p.b + mod_b(p, i)
+                                      : orphV + i;
             kind[u] = kVal;
             head[u] = h;
-            sv[u] = sc[(vlev & 1) * G * cmax + h * cmax + i];
-            PairLoad<float, HALF>::load(vals + cand_node(vlev, h, i) * D, j0, ra[u]);
+            sv[u] = scV[h * cmax + i];
+            RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
           }
         } else if (e < total) {
-          const int64_t x = t_lo + (e - nw - nk - nv);
-          const int h = int(x / (int64_t(nleaf) * p.B));
-          const int64_t r = x % (int64_t(nleaf) * p.B);
-          const int mb = int(r / p.B), o = int(r % p.B);
-          const int64_t pos = int64_t(kept[(1 & 1) * G * kmax + h * kmax + mb]) * p.B + o;
+          const int x = t_lo + (e - nw - nk - nv);
+          const int h = head_of(x, nlb), r = x - h * nlb;
+          const int pos = kept1[h * kmax + div_B(p, r)] * p.B + mod_B(p, r);
           kind[u] = kTok;
           head[u] = h;
-          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
           if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
+        float xa[8], xb[8];
+        if (kind[u] == kKey || kind[u] == kVal) {
+          RawLoad<float, HALF>::cvt(ra[u], xa);
+        } else {
+          RawLoad<T, HALF>::cvt(ra[u], xa);
+          RawLoad<T, HALF>::cvt(rb[u], xb);
+        }
         const bool rot = p.rope && (kind[u] == kWin || kind[u] == kKey || kind[u] == kTok);
-        if (rot) rotate8(ra[u], cs[u]);
+        if (rot) rotate8(xa, cs[u]);
         // Dot products: all G heads for a window row, one head otherwise.
         float sw[G], s1 = 0.f;
 #pragma unroll
@@ -241,16 +274,16 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
             const float* qv = qtok + h * D;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              sw[h] = fmaf(qv[j0 + c], ra[u][c], sw[h]);
-              sw[h] = fmaf(qv[HALF + j0 + c], ra[u][4 + c], sw[h]);
+              sw[h] = fmaf(qv[j0 + c], xa[c], sw[h]);
+              sw[h] = fmaf(qv[HALF + j0 + c], xa[4 + c], sw[h]);
             }
           }
         } else if (kind[u] == kKey || kind[u] == kTok) {
           const float* qv = (kind[u] == kKey ? qlev : qtok) + head[u] * D;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            s1 = fmaf(qv[j0 + c], ra[u][c], s1);
-            s1 = fmaf(qv[HALF + j0 + c], ra[u][4 + c], s1);
+            s1 = fmaf(qv[j0 + c], xa[c], s1);
+            s1 = fmaf(qv[HALF + j0 + c], xa[4 + c], s1);
           }
         }
         // Slot reductions with warp-uniform participation.
@@ -262,15 +295,15 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
           s1 = slot_sum<LPR>(s1) * inv_sqrt_d;
         if (kind[u] == kWin) {
 #pragma unroll
-          for (int h = 0; h < G; ++h) fold(h, sw[h], rb[u]);
+          for (int h = 0; h < G; ++h) fold(h, sw[h], xb);
         } else if (kind[u] == kKey) {
           const int off = (klev & 1) * G * cmax + head[u] * cmax + idx[u];
           if (sub < CS) *cluster.map_shared_rank(sc + off, sub) = s1;
           if (sub + LPR < CS) *cluster.map_shared_rank(sc + off, sub + LPR) = s1;
         } else if (kind[u] == kTok) {
-          fold(head[u], s1, rb[u]);
+          fold(head[u], s1, xb);
         } else if (kind[u] == kVal) {
-          fold(head[u], sv[u], ra[u]);
+          fold(head[u], sv[u], xa);
         }
       }
     }
@@ -313,7 +346,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         const unsigned bal = __ballot_sync(0xffffffffu, f);
         if (f) {
           const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-          const int node = int(cand_node(lev, h, i));
+          const int node = cand_node(lev, h, i);
           kp[h * kmax + pos] = node;
           if (trace && rank == 0) {
             const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
@@ -327,11 +360,11 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   };
 
   // Window share of this CTA (independent of the selection).
-  int64_t w_lo = 0, w_hi = 0;
+  int w_lo = 0, w_hi = 0;
   {
-    const int64_t ch = (n_win + CS - 1) / CS;
-    w_lo = min(n_win, int64_t(rank) * ch);
-    w_hi = min(n_win, w_lo + ch);
+    const int nw = int(n_win), ch = (nw + CS - 1) / CS;
+    w_lo = min(nw, rank * ch);
+    w_hi = min(nw, w_lo + ch);
   }
   if (top > 0) {
     rotate_q(qlev, cnt_c[top]);

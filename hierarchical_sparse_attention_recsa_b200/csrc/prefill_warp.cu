@@ -119,72 +119,93 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   const int tstride = kTraceHead + kMaxLevels * p.k;
   const int64_t rec = ((seq * n_q + qi) * p.hq + h) * int64_t(tstride);
 
-  auto cand_node = [&](int lev, int i) -> int64_t {
+  auto cand_node = [&](int lev, int i) -> int {
     const int kup = lev < top ? cnt_k[lev + 1] : 0;
-    const int64_t vup = lev < top ? vis[lev + 1] : 0;
-    if (i < p.b * kup) return int64_t(kept[((lev + 1) & 1) * kmax + i / p.b]) * p.b + i % p.b;
-    return p.b * vup + (i - int64_t(p.b) * kup);
+    const int vup = lev < top ? int(vis[lev + 1]) : 0;
+    if (i < p.b * kup) return kept[((lev + 1) & 1) * kmax + div_b(p, i)] * p.b + mod_b(p, i);
+    return p.b * vup + (i - p.b * kup);
   };
 
   // Window rows (first pass), key pairs of klev, unselected values of vlev,
-  // kept-leaf tokens (last pass).
+  // kept-leaf tokens (last pass).  32-bit index math, constants hoisted.
   auto run_pass = [&](bool window, int klev, int vlev, bool tokens) {
-    const int64_t nw = window ? n_win : 0;
-    const int64_t nk = klev > 0 ? cnt_c[klev] : 0;
-    const int64_t nv = vlev > 0 ? cnt_c[vlev] : 0;
-    const int64_t nt = tokens ? int64_t(nleaf) * p.B : 0;
-    const int64_t total = nw + nk + nv + nt;
+    const int nw = window ? int(n_win) : 0;
+    const int nk = klev > 0 ? cnt_c[klev] : 0;
+    const int nv = vlev > 0 ? cnt_c[vlev] : 0;
+    const int nt = tokens ? nleaf * p.B : 0;
+    const int total = nw + nk + nv + nt;
     const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
     const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
-    for (int64_t base = 0; base < total; base += int64_t(SPW) * kPUnroll) {
-      float ra[kPUnroll][8], rb[kPUnroll][8], cs[kPUnroll][8];
+    const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
+    const int nchK = p.b * kupK;
+    const int orphK = (klev > 0 && klev < top) ? p.b * int(vis[klev + 1]) - nchK : 0;
+    const int* keptK = kept + ((klev + 1) & 1) * kmax;
+    const int kupV = (vlev > 0 && vlev < top) ? cnt_k[vlev + 1] : 0;
+    const int nchV = p.b * kupV;
+    const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
+    const int* keptV = kept + ((vlev + 1) & 1) * kmax;
+    const int* kept1 = kept + 1 * kmax;                           // level 1 = parity 1
+    const float* scV = sc + (vlev & 1) * cmax;
+    const unsigned char* flV = kfl + (vlev & 1) * cmax;
+    const int win0 = int(a) * p.B;
+    const int widx0 = nleaf * p.B;
+    for (int base = 0; base < total; base += SPW * kPUnroll) {
+      RawPairs ra[kPUnroll], rb[kPUnroll];
+      float cs[kPUnroll][8];
       int kind[kPUnroll], idx[kPUnroll];
       float sv[kPUnroll];
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
-        const int64_t e = base + int64_t(u) * SPW + slot;
+        const int e = base + u * SPW + slot;
         kind[u] = pNone;
         idx[u] = 0;
         sv[u] = 0.f;
         if (e < nw) {
-          const int64_t pos = a * p.B + e;
+          const int pos = win0 + e;
           kind[u] = pTok;
-          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
-          if (p.rope) load_cs(rope, int64_t(nleaf) * p.B + e, HALF, j0, cs[u]);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
         } else if (e < nw + nk) {
-          const int i = int(e - nw);
+          const int i = e - nw;
+          const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
           kind[u] = pKey;
           idx[u] = i;
-          PairLoad<float, HALF>::load(keys + cand_node(klev, i) * D, j0, ra[u]);
+          RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
           if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
         } else if (e < nw + nk + nv) {
-          const int i = int(e - nw - nk);
-          if (!kfl[(vlev & 1) * cmax + i]) {
+          const int i = e - nw - nk;
+          if (!flV[i]) {
+            const int node = i < nchV ? keptV[div_b(p, i)] * p.b + mod_b(p, i) : orphV + i;
             kind[u] = pVal;
-            sv[u] = sc[(vlev & 1) * cmax + i];
-            PairLoad<float, HALF>::load(vals + cand_node(vlev, i) * D, j0, ra[u]);
+            sv[u] = scV[i];
+            RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
           }
         } else if (e < total) {
-          const int64_t r = e - nw - nk - nv;
-          const int mb = int(r / p.B), o = int(r % p.B);
-          const int64_t pos = int64_t(kept[1 * kmax + mb]) * p.B + o;   // level 1 = parity 1
+          const int r = e - nw - nk - nv;
+          const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
           kind[u] = pTok;
-          PairLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          PairLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
           if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
-        float s = 0.f;
+        float s = 0.f, xa[8], xb[8];
+        if (kind[u] == pKey || kind[u] == pVal) {
+          RawLoad<float, HALF>::cvt(ra[u], xa);
+        } else {
+          RawLoad<T, HALF>::cvt(ra[u], xa);
+          RawLoad<T, HALF>::cvt(rb[u], xb);
+        }
         if (kind[u] == pKey || kind[u] == pTok) {
-          if (p.rope) rotate8(ra[u], cs[u]);
+          if (p.rope) rotate8(xa, cs[u]);
           const float* qv = kind[u] == pKey ? qlev : qtok;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            s = fmaf(qv[j0 + c], ra[u][c], s);
-            s = fmaf(qv[HALF + j0 + c], ra[u][4 + c], s);
+            s = fmaf(qv[j0 + c], xa[c], s);
+            s = fmaf(qv[HALF + j0 + c], xa[4 + c], s);
           }
         }
         if (__any_sync(0xffffffffu, kind[u] == pKey || kind[u] == pTok))
@@ -192,9 +213,9 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         if (kind[u] == pKey) {
           if (sub == 0) sc[(klev & 1) * cmax + idx[u]] = s;
         } else if (kind[u] == pTok) {
-          fold(s, rb[u]);
+          fold(s, xb);
         } else if (kind[u] == pVal) {
-          fold(sv[u], ra[u]);
+          fold(sv[u], xa);
         }
       }
     }
@@ -235,7 +256,7 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       const unsigned bal = __ballot_sync(0xffffffffu, f);
       if (f) {
         const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-        const int node = int(cand_node(lev, i));
+        const int node = cand_node(lev, i);
         kp[pos] = node;
         if (trace) trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
       }

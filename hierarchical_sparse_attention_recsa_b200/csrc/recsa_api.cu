@@ -90,6 +90,11 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->rope = g->rope_enabled;
   p->batch = g->batch;
   p->cap = g->capacity;
+  p->Bsh = p->bsh = -1;
+  for (int sh = 0; sh < 31; ++sh) {
+    if ((1 << sh) == p->B) p->Bsh = sh;
+    if ((1 << sh) == p->b) p->bsh = sh;
+  }
   p->inv_sqrt_d = 1.0f / sqrtf(float(g->head_dim));
   return RECSA_OK;
 }

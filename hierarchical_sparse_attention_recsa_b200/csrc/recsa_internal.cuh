@@ -28,10 +28,17 @@ struct TreeLayout {
 // Everything a kernel needs about the geometry, passed by value.
 struct Params {
   int32_t dtype, d, hq, hkv, group, B, b, k, W, rope, batch;
+  int32_t Bsh, bsh;   // log2 of B and b when powers of two, else -1
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;
 };
+
+// x / B, x % B, x / b, x % b for non-negative 32-bit x (shifts when powers of two).
+__device__ __forceinline__ int div_B(const Params& p, int x) { return p.Bsh >= 0 ? x >> p.Bsh : x / p.B; }
+__device__ __forceinline__ int mod_B(const Params& p, int x) { return p.Bsh >= 0 ? x & (p.B - 1) : x % p.B; }
+__device__ __forceinline__ int div_b(const Params& p, int x) { return p.bsh >= 0 ? x >> p.bsh : x / p.b; }
+__device__ __forceinline__ int mod_b(const Params& p, int x) { return p.bsh >= 0 ? x & (p.b - 1) : x % p.b; }
 
 // Device error word at offset 0 of the tree header.
 __device__ __forceinline__ unsigned int* tree_error_word(void* tree) {

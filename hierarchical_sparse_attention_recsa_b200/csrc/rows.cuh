@@ -66,3 +66,45 @@ __device__ __forceinline__ float slot_sum(float v) {
 }
 
 }  // namespace recsa
+
+namespace recsa {
+
+// Raw bytes of a lane's four pairs: loads of a whole batch are issued before
+// any of them is consumed, and converted to fp32 only afterwards, so the
+// loads of an unrolled batch overlap in flight.
+struct RawPairs {
+  uint4 a, b;
+};
+
+template <typename T, int HALF>
+struct RawLoad;
+template <int HALF>
+struct RawLoad<float, HALF> {
+  static __device__ __forceinline__ void load(const float* row, int j0, RawPairs& r) {
+    r.a = __ldg(reinterpret_cast<const uint4*>(row + j0));
+    r.b = __ldg(reinterpret_cast<const uint4*>(row + HALF + j0));
+  }
+  static __device__ __forceinline__ void cvt(const RawPairs& r, float* x) {
+    x[0] = __uint_as_float(r.a.x); x[1] = __uint_as_float(r.a.y);
+    x[2] = __uint_as_float(r.a.z); x[3] = __uint_as_float(r.a.w);
+    x[4] = __uint_as_float(r.b.x); x[5] = __uint_as_float(r.b.y);
+    x[6] = __uint_as_float(r.b.z); x[7] = __uint_as_float(r.b.w);
+  }
+};
+template <int HALF>
+struct RawLoad<__nv_bfloat16, HALF> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* row, int j0, RawPairs& r) {
+    const uint2 a = __ldg(reinterpret_cast<const uint2*>(row + j0));
+    const uint2 b = __ldg(reinterpret_cast<const uint2*>(row + HALF + j0));
+    r.a.x = a.x; r.a.y = a.y;
+    r.b.x = b.x; r.b.y = b.y;
+  }
+  static __device__ __forceinline__ float lo(unsigned u) { return __uint_as_float(u << 16); }
+  static __device__ __forceinline__ float hi(unsigned u) { return __uint_as_float(u & 0xffff0000u); }
+  static __device__ __forceinline__ void cvt(const RawPairs& r, float* x) {
+    x[0] = lo(r.a.x); x[1] = hi(r.a.x); x[2] = lo(r.a.y); x[3] = hi(r.a.y);
+    x[4] = lo(r.b.x); x[5] = hi(r.b.x); x[6] = lo(r.b.y); x[7] = hi(r.b.y);
+  }
+};
+
+}  // namespace recsa
