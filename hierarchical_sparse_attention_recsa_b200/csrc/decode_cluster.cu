@@ -32,9 +32,9 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 2;
+constexpr int kUnroll = 3;
 
-enum ItemKind { kKey = 0, kVal = 1, kWin = 2, kTok = 3, kNone = 4 };
+enum ItemKind { kKey = 0, kVal = 1, kTok = 2, kNone = 3 };
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -58,8 +58,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* qlev = qf + G * D;                            // [G][D] rotated to the level's c
   float* qtok = qlev + G * D;                          // [G][D] rotated to n0 - 1
   float* sc = qtok + G * D;                            // [2][G][cmax] scores
-  float* wsc = sc + 2 * G * cmax;                      // [kWarps][G][D + 2] warp merge
-  float* mrg = wsc + kWarps * G * (D + 2);             // [CS][G][D + 2] cluster merge (rank 0)
+  float* wsc = sc + 2 * G * cmax;                      // [kWarps][D + 2] warp merge
+  float* mrg = wsc + kWarps * (D + 2);                 // [CS][G][D + 2] cluster merge (rank 0)
   int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
   unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
 
@@ -114,32 +114,26 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   };
   if (!empty) rotate_q(qtok, n0 - 1 > 0 ? n0 - 1 : 0);
 
-  // Online softmax state of this lane slot: per head (m, l) and 8 channels.
-  float m[G], l[G], acc[G][8];
+  // Warps are specialised by head: warps [h * WPH, (h + 1) * WPH) serve query
+  // head h of the group, so every lane slot keeps one online-softmax state.
+  constexpr int WPH = kWarps / G, HSLOT = WPH * SPW;
+  const int hw = warp / WPH;                          // this warp's head
+  const int hs = (warp % WPH) * SPW + lane / LPR;     // slot index within the head's warps
+  float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  auto fold = [&](float s, const float* v) {
+    if (s > m) {
+      const float r = __expf(m - s);
+      l = l * r + 1.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[h][c] = 0.f;
-  }
-  auto fold = [&](int h, float s, const float* v) {
+      for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
+      m = s;
+    } else {
+      const float w = __expf(s - m);
+      l += w;
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      if (hh == h) {
-        if (s > m[hh]) {
-          const float r = __expf(m[hh] - s);
-          l[hh] = l[hh] * r + 1.f;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[hh][c] = fmaf(acc[hh][c], r, v[c]);
-          m[hh] = s;
-        } else {
-          const float w = __expf(s - m[hh]);
-          l[hh] += w;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) acc[hh][c] = fmaf(w, v[c], acc[hh][c]);
-        }
-      }
+      for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
     }
   };
 
@@ -155,99 +149,77 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       return kept[((lev + 1) & 1) * G * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
     return p.b * vup + (i - p.b * kup);
   };
-  // Head of flattened pair x with c pairs per head (G <= 4: compares only).
-  auto head_of = [&](int x, int c) -> int {
-    int h = 0;
-#pragma unroll
-    for (int hh = 1; hh < G; ++hh) h += x >= hh * c;
-    return h;
+  auto share = [&](int tot, int& lo, int& hi) {
+    const int ch = (tot + CS - 1) / CS;
+    lo = min(tot, rank * ch);
+    hi = min(tot, lo + ch);
   };
 
-  // One pass over this CTA's items: window rows, key pairs of level klev,
-  // unselected value pairs of level vlev, kept-leaf tokens.  All index math is
-  // 32-bit and the per-level constants are hoisted out of the item loop.
+  // One pass over this CTA's share of head hw's items: window rows, key
+  // candidates of level klev, unselected values of level vlev, kept-leaf
+  // tokens.  All index math is 32-bit, the per-level constants are hoisted.
   auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
     int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0, t_lo = 0, t_hi = 0;
-    const int ck = klev > 0 ? cnt_c[klev] : 1, cv = vlev > 0 ? cnt_c[vlev] : 1;
     const int nlb = nleaf * p.B;
-    if (klev > 0) {
-      const int tot = G * ck, ch = (tot + CS - 1) / CS;
-      k_lo = min(tot, rank * ch);
-      k_hi = min(tot, k_lo + ch);
-    }
-    if (vlev > 0) {
-      const int tot = G * cv, ch = (tot + CS - 1) / CS;
-      v_lo = min(tot, rank * ch);
-      v_hi = min(tot, v_lo + ch);
-    }
-    if (tokens) {
-      const int tot = G * nlb, ch = (tot + CS - 1) / CS;
-      t_lo = min(tot, rank * ch);
-      t_hi = min(tot, t_lo + ch);
-    }
+    if (klev > 0) share(cnt_c[klev], k_lo, k_hi);
+    if (vlev > 0) share(cnt_c[vlev], v_lo, v_hi);
+    if (tokens) share(nlb, t_lo, t_hi);
     const int nw = w_hi - w_lo, nk = k_hi - k_lo, nv = v_hi - v_lo, nt = t_hi - t_lo;
     const int total = nw + nk + nv + nt;
     const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
     const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
-    // candidate -> node maps of the two levels: i < nch -> kept parent child, else orph + i
     const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
     const int nchK = p.b * kupK;
     const int orphK = (klev > 0 && klev < top) ? p.b * int(vis[klev + 1]) - nchK : 0;
-    const int* keptK = kept + ((klev + 1) & 1) * G * kmax;
+    const int* keptK = kept + ((klev + 1) & 1) * G * kmax + hw * kmax;
     const int kupV = (vlev > 0 && vlev < top) ? cnt_k[vlev + 1] : 0;
     const int nchV = p.b * kupV;
     const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
-    const int* keptV = kept + ((vlev + 1) & 1) * G * kmax;
-    const int* kept1 = kept + 1 * G * kmax;                       // level 1 = parity 1
-    const float* scV = sc + (vlev & 1) * G * cmax;
-    const unsigned char* flV = kfl + (vlev & 1) * G * cmax;
+    const int* keptV = kept + ((vlev + 1) & 1) * G * kmax + hw * kmax;
+    const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
+    const float* scV = sc + (vlev & 1) * G * cmax + hw * cmax;
+    const unsigned char* flV = kfl + (vlev & 1) * G * cmax + hw * cmax;
+    float* scK = sc + (klev & 1) * G * cmax + hw * cmax;
+    const float* ql = qlev + hw * D;
+    const float* qt = qtok + hw * D;
     const int win0 = int(a) * p.B + w_lo;
     const int widx0 = nlb + w_lo;
-    for (int base = 0; base < total; base += NSLOT * kUnroll) {
+    for (int base = 0; base < total; base += HSLOT * kUnroll) {
       RawPairs ra[kUnroll], rb[kUnroll];
       float cs[kUnroll][8];
-      int kind[kUnroll], head[kUnroll], idx[kUnroll];
+      int kind[kUnroll], idx[kUnroll];
       float sv[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        const int e = base + u * NSLOT + slot;
+        const int e = base + u * HSLOT + hs;
         kind[u] = kNone;
-        head[u] = 0;
         idx[u] = 0;
         sv[u] = 0.f;
         if (e < nw) {
           const int pos = win0 + e;
-          kind[u] = kWin;
+          kind[u] = kTok;
           RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
           RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
           if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
         } else if (e < nw + nk) {
-          const int x = k_lo + (e - nw);
-          const int h = head_of(x, ck), i = x - h * ck;
-          const int node = i < nchK ? keptK[h * kmax + div_b(p, i)] * p.b + mod_b(p, i)
-                                    : orphK + i;
+          const int i = k_lo + (e - nw);
+          const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
           kind[u] = kKey;
-          head[u] = h;
           idx[u] = i;
           RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
           if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
         } else if (e < nw + nk + nv) {
-          const int x = v_lo + (e - nw - nk);
-          const int h = head_of(x, cv), i = x - h * cv;
-          if (!flV[h * cmax + i]) {
-            const int node = i < nchV ? keptV[h * kmax + div_b(p, i)] * p.b + mod_b(p, i)
-                                      : orphV + i;
+          const int i = v_lo + (e - nw - nk);
+          if (!flV[i]) {
+            const int node = i < nchV ? keptV[div_b(p, i)] * p.b + mod_b(p, i) : orphV + i;
             kind[u] = kVal;
-            head[u] = h;
-            sv[u] = scV[h * cmax + i];
+            sv[u] = scV[i];
             RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
           }
         } else if (e < total) {
-          const int x = t_lo + (e - nw - nk - nv);
-          const int h = head_of(x, nlb), r = x - h * nlb;
-          const int pos = kept1[h * kmax + div_B(p, r)] * p.B + mod_B(p, r);
+          const int r = t_lo + (e - nw - nk - nv);
+          const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
           kind[u] = kTok;
-          head[u] = h;
           RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
           RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
           if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
@@ -255,55 +227,32 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        float xa[8], xb[8];
+        float s = 0.f, xa[8], xb[8];
         if (kind[u] == kKey || kind[u] == kVal) {
           RawLoad<float, HALF>::cvt(ra[u], xa);
         } else {
           RawLoad<T, HALF>::cvt(ra[u], xa);
           RawLoad<T, HALF>::cvt(rb[u], xb);
         }
-        const bool rot = p.rope && (kind[u] == kWin || kind[u] == kKey || kind[u] == kTok);
-        if (rot) rotate8(xa, cs[u]);
-        // Dot products: all G heads for a window row, one head otherwise.
-        float sw[G], s1 = 0.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) sw[h] = 0.f;
-        if (kind[u] == kWin) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float* qv = qtok + h * D;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              sw[h] = fmaf(qv[j0 + c], xa[c], sw[h]);
-              sw[h] = fmaf(qv[HALF + j0 + c], xa[4 + c], sw[h]);
-            }
-          }
-        } else if (kind[u] == kKey || kind[u] == kTok) {
-          const float* qv = (kind[u] == kKey ? qlev : qtok) + head[u] * D;
+        if (kind[u] == kKey || kind[u] == kTok) {
+          if (p.rope) rotate8(xa, cs[u]);
+          const float* qv = kind[u] == kKey ? ql : qt;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            s1 = fmaf(qv[j0 + c], xa[c], s1);
-            s1 = fmaf(qv[HALF + j0 + c], xa[4 + c], s1);
+            s = fmaf(qv[j0 + c], xa[c], s);
+            s = fmaf(qv[HALF + j0 + c], xa[4 + c], s);
           }
         }
-        // Slot reductions with warp-uniform participation.
-        if (__any_sync(0xffffffffu, kind[u] == kWin)) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) sw[h] = slot_sum<LPR>(sw[h]) * inv_sqrt_d;
-        }
         if (__any_sync(0xffffffffu, kind[u] == kKey || kind[u] == kTok))
-          s1 = slot_sum<LPR>(s1) * inv_sqrt_d;
-        if (kind[u] == kWin) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) fold(h, sw[h], xb);
-        } else if (kind[u] == kKey) {
-          const int off = (klev & 1) * G * cmax + head[u] * cmax + idx[u];
-          if (sub < CS) *cluster.map_shared_rank(sc + off, sub) = s1;
-          if (sub + LPR < CS) *cluster.map_shared_rank(sc + off, sub + LPR) = s1;
+          s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (kind[u] == kKey) {
+          float* dstp = scK + idx[u];
+          if (sub < CS) *cluster.map_shared_rank(dstp, sub) = s;
+          if (sub + LPR < CS) *cluster.map_shared_rank(dstp, sub + LPR) = s;
         } else if (kind[u] == kTok) {
-          fold(head[u], s1, xb);
+          fold(s, xb);
         } else if (kind[u] == kVal) {
-          fold(head[u], sv[u], xa);
+          fold(sv[u], xa);
         }
       }
     }
@@ -384,47 +333,45 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     run_pass(w_lo, w_hi, 0, 0, false);
   }
 
-  // Merge: slots of a warp, then warps, then the cluster (into rank 0).
+  // Merge: slots of a warp, then the warps of each head, then the cluster
+  // (into rank 0).
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
+  for (int o = LPR; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+    const float mn = fmaxf(m, mo);
+    const float ra_ = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
+    l = l * ra_ + lo * rb_;
 #pragma unroll
-    for (int o = LPR; o < 32; o <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[h], o);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[h], o);
-      const float mn = fmaxf(m[h], mo);
-      const float ra_ = (m[h] == -INFINITY) ? 0.f : __expf(m[h] - mn);
-      const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
-      l[h] = l[h] * ra_ + lo * rb_;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float ao = __shfl_xor_sync(0xffffffffu, acc[h][c], o);
-        acc[h][c] = acc[h][c] * ra_ + ao * rb_;
-      }
-      m[h] = mn;
+    for (int c = 0; c < 8; ++c) {
+      const float ao = __shfl_xor_sync(0xffffffffu, acc[c], o);
+      acc[c] = acc[c] * ra_ + ao * rb_;
     }
-    if (lane < LPR) {
-      float* w = wsc + (warp * G + h) * (D + 2);
+    m = mn;
+  }
+  if (lane < LPR) {
+    float* w = wsc + warp * (D + 2);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        w[j0 + c] = acc[h][c];
-        w[HALF + j0 + c] = acc[h][4 + c];
-      }
-      if (lane == 0) {
-        w[D] = m[h];
-        w[D + 1] = l[h];
-      }
+    for (int c = 0; c < 4; ++c) {
+      w[j0 + c] = acc[c];
+      w[HALF + j0 + c] = acc[4 + c];
+    }
+    if (lane == 0) {
+      w[D] = m;
+      w[D + 1] = l;
     }
   }
   __syncthreads();
-  // CTA state -> rank 0's merge slot [rank]
+  // CTA state of each head -> rank 0's merge slot [rank]
   float* dst = cluster.map_shared_rank(mrg, 0) + rank * G * (D + 2);
   for (int x = tid; x < G * D; x += kThreads) {
     const int h = x / D, c = x % D;
     float mm = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wsc[(w * G + h) * (D + 2) + D]);
+    for (int w = h * WPH; w < (h + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * (D + 2) + D]);
     float aa = 0.f, ll = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float* ws = wsc + (w * G + h) * (D + 2);
+    for (int w = h * WPH; w < (h + 1) * WPH; ++w) {
+      const float* ws = wsc + w * (D + 2);
       const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
       aa = fmaf(ws[c], r, aa);
       ll = fmaf(ws[D + 1], r, ll);
@@ -494,7 +441,7 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   const int cmax = int(cm < 1 ? 1 : cm);
   const int kmax = int(kk < cmax ? kk : cmax);
   if (cmax > 1024) return cudaErrorNotSupported;
-  const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * G * (D + 2) +
+  const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * (D + 2) +
                         size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
                        size_t(2) * G * cmax + 16;
   if (bytes > 200 * 1024) return cudaErrorNotSupported;
