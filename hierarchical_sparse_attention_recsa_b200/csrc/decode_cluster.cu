@@ -33,8 +33,9 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 3;
+constexpr int kWinUnroll = 1;
 
-enum ItemKind { kKey = 0, kVal = 1, kTok = 2, kNone = 3 };
+enum ItemKind { kKey = 0, kVal = 1, kNone = 2 };
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -59,7 +60,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* qtok = qlev + G * D;                          // [G][D] rotated to n0 - 1
   float* sc = qtok + G * D;                            // [2][G][cmax] scores
   float* wsc = sc + 2 * G * cmax;                      // [kWarps][D + 2] warp merge
-  float* mrg = wsc + kWarps * (D + 2);                 // [CS][G][D + 2] cluster merge (rank 0)
+  float* wwin = wsc + kWarps * (D + 2);                // [kWarps][G][D + 2] window partials
+  float* mrg = wwin + kWarps * G * (D + 2);            // [CS][G][D + 2] cluster merge (rank 0)
   int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
   unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
 
@@ -155,17 +157,110 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     hi = min(tot, lo + ch);
   };
 
-  // One pass over this CTA's share of head hw's items: window rows, key
-  // candidates of level klev, unselected values of level vlev, kept-leaf
-  // tokens.  All index math is 32-bit, the per-level constants are hoisted.
-  auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
-    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0, t_lo = 0, t_hi = 0;
-    const int nlb = nleaf * p.B;
+  // Window rows [w_lo, w_hi): every slot of the CTA takes rows, each row is
+  // loaded, rotated and scored once for all G heads.  The per-slot state of
+  // all heads is merged across the warp and left in wwin[warp][G].
+  auto window_loop = [&](int w_lo, int w_hi) {
+    float mW[G], lW[G], accW[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      mW[h] = -INFINITY;
+      lW[h] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) accW[h][c] = 0.f;
+    }
+    const int nw = w_hi - w_lo;
+    const int win0 = int(a) * p.B + w_lo;
+    const int widx0 = nleaf * p.B + w_lo;
+    const int gslot = warp * SPW + lane / LPR;
+    for (int base = 0; base < nw; base += NSLOT * kWinUnroll) {
+      RawPairs rk[kWinUnroll], rv[kWinUnroll];
+      float cs[kWinUnroll][8];
+      bool on[kWinUnroll];
+#pragma unroll
+      for (int u = 0; u < kWinUnroll; ++u) {
+        const int e = base + u * NSLOT + gslot;
+        on[u] = e < nw;
+        if (on[u]) {
+          const int pos = win0 + e;
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
+          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kWinUnroll; ++u) {
+        float xk[8], xv[8];
+        RawLoad<T, HALF>::cvt(rk[u], xk);
+        RawLoad<T, HALF>::cvt(rv[u], xv);
+        if (p.rope) rotate8(xk, cs[u]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float* qv = qtok + h * D;
+          float s = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            s = fmaf(qv[j0 + c], xk[c], s);
+            s = fmaf(qv[HALF + j0 + c], xk[4 + c], s);
+          }
+          s = slot_sum<LPR>(s) * inv_sqrt_d;
+          if (on[u]) {
+            if (s > mW[h]) {
+              const float r = __expf(mW[h] - s);
+              lW[h] = lW[h] * r + 1.f;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) accW[h][c] = fmaf(accW[h][c], r, xv[c]);
+              mW[h] = s;
+            } else {
+              const float w = __expf(s - mW[h]);
+              lW[h] += w;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) accW[h][c] = fmaf(w, xv[c], accW[h][c]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, mW[h], o);
+        const float lo = __shfl_xor_sync(0xffffffffu, lW[h], o);
+        const float mn = fmaxf(mW[h], mo);
+        const float ra_ = (mW[h] == -INFINITY) ? 0.f : __expf(mW[h] - mn);
+        const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
+        lW[h] = lW[h] * ra_ + lo * rb_;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const float ao = __shfl_xor_sync(0xffffffffu, accW[h][c], o);
+          accW[h][c] = accW[h][c] * ra_ + ao * rb_;
+        }
+        mW[h] = mn;
+      }
+      if (lane < LPR) {
+        float* w = wwin + (warp * G + h) * (D + 2);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          w[j0 + c] = accW[h][c];
+          w[HALF + j0 + c] = accW[h][4 + c];
+        }
+        if (lane == 0) {
+          w[D] = mW[h];
+          w[D + 1] = lW[h];
+        }
+      }
+    }
+  };
+
+  // Tree rows of head hw (this CTA's share): the key candidates of level klev
+  // (scored, scores broadcast to every CTA) and the unselected candidates of
+  // level vlev (values folded into the softmax).
+  auto tree_loop = [&](int klev, int vlev) {
+    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0;
     if (klev > 0) share(cnt_c[klev], k_lo, k_hi);
     if (vlev > 0) share(cnt_c[vlev], v_lo, v_hi);
-    if (tokens) share(nlb, t_lo, t_hi);
-    const int nw = w_hi - w_lo, nk = k_hi - k_lo, nv = v_hi - v_lo, nt = t_hi - t_lo;
-    const int total = nw + nk + nv + nt;
+    const int nk = k_hi - k_lo, nv = v_hi - v_lo, total = nk + nv;
     const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
     const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
     const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
@@ -176,16 +271,12 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int nchV = p.b * kupV;
     const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
     const int* keptV = kept + ((vlev + 1) & 1) * G * kmax + hw * kmax;
-    const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
     const float* scV = sc + (vlev & 1) * G * cmax + hw * cmax;
     const unsigned char* flV = kfl + (vlev & 1) * G * cmax + hw * cmax;
     float* scK = sc + (klev & 1) * G * cmax + hw * cmax;
     const float* ql = qlev + hw * D;
-    const float* qt = qtok + hw * D;
-    const int win0 = int(a) * p.B + w_lo;
-    const int widx0 = nlb + w_lo;
     for (int base = 0; base < total; base += HSLOT * kUnroll) {
-      RawPairs ra[kUnroll], rb[kUnroll];
+      RawPairs ra[kUnroll];
       float cs[kUnroll][8];
       int kind[kUnroll], idx[kUnroll];
       float sv[kUnroll];
@@ -195,67 +286,91 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         kind[u] = kNone;
         idx[u] = 0;
         sv[u] = 0.f;
-        if (e < nw) {
-          const int pos = win0 + e;
-          kind[u] = kTok;
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
-          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
-        } else if (e < nw + nk) {
-          const int i = k_lo + (e - nw);
+        if (e < nk) {
+          const int i = k_lo + e;
           const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
           kind[u] = kKey;
           idx[u] = i;
           RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
           if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
-        } else if (e < nw + nk + nv) {
-          const int i = v_lo + (e - nw - nk);
+        } else if (e < total) {
+          const int i = v_lo + (e - nk);
           if (!flV[i]) {
             const int node = i < nchV ? keptV[div_b(p, i)] * p.b + mod_b(p, i) : orphV + i;
             kind[u] = kVal;
             sv[u] = scV[i];
             RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
           }
-        } else if (e < total) {
-          const int r = t_lo + (e - nw - nk - nv);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        float x[8], s = 0.f;
+        RawLoad<float, HALF>::cvt(ra[u], x);
+        if (kind[u] == kKey) {
+          if (p.rope) rotate8(x, cs[u]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            s = fmaf(ql[j0 + c], x[c], s);
+            s = fmaf(ql[HALF + j0 + c], x[4 + c], s);
+          }
+        }
+        if (__any_sync(0xffffffffu, kind[u] == kKey)) s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (kind[u] == kKey) {
+          float* dstp = scK + idx[u];
+          if (sub < CS) *cluster.map_shared_rank(dstp, sub) = s;
+          if (sub + LPR < CS) *cluster.map_shared_rank(dstp, sub + LPR) = s;
+        } else if (kind[u] == kVal) {
+          fold(sv[u], x);
+        }
+      }
+    }
+  };
+
+  // Kept-leaf tokens of head hw (this CTA's share), after level 1's top-k.
+  auto token_loop = [&]() {
+    int t_lo = 0, t_hi = 0;
+    share(nleaf * p.B, t_lo, t_hi);
+    const int nt = t_hi - t_lo;
+    const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
+    const float* qt = qtok + hw * D;
+    for (int base = 0; base < nt; base += HSLOT * kUnroll) {
+      RawPairs rk[kUnroll], rv[kUnroll];
+      float cs[kUnroll][8];
+      bool on[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int e = base + u * HSLOT + hs;
+        on[u] = e < nt;
+        if (on[u]) {
+          const int r = t_lo + e;
           const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
-          kind[u] = kTok;
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
           if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        float s = 0.f, xa[8], xb[8];
-        if (kind[u] == kKey || kind[u] == kVal) {
-          RawLoad<float, HALF>::cvt(ra[u], xa);
-        } else {
-          RawLoad<T, HALF>::cvt(ra[u], xa);
-          RawLoad<T, HALF>::cvt(rb[u], xb);
-        }
-        if (kind[u] == kKey || kind[u] == kTok) {
-          if (p.rope) rotate8(xa, cs[u]);
-          const float* qv = kind[u] == kKey ? ql : qt;
+        float xk[8], xv[8], s = 0.f;
+        RawLoad<T, HALF>::cvt(rk[u], xk);
+        RawLoad<T, HALF>::cvt(rv[u], xv);
+        if (p.rope) rotate8(xk, cs[u]);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            s = fmaf(qv[j0 + c], xa[c], s);
-            s = fmaf(qv[HALF + j0 + c], xa[4 + c], s);
-          }
+        for (int c = 0; c < 4; ++c) {
+          s = fmaf(qt[j0 + c], xk[c], s);
+          s = fmaf(qt[HALF + j0 + c], xk[4 + c], s);
         }
-        if (__any_sync(0xffffffffu, kind[u] == kKey || kind[u] == kTok))
-          s = slot_sum<LPR>(s) * inv_sqrt_d;
-        if (kind[u] == kKey) {
-          float* dstp = scK + idx[u];
-          if (sub < CS) *cluster.map_shared_rank(dstp, sub) = s;
-          if (sub + LPR < CS) *cluster.map_shared_rank(dstp, sub + LPR) = s;
-        } else if (kind[u] == kTok) {
-          fold(s, xb);
-        } else if (kind[u] == kVal) {
-          fold(sv[u], xa);
-        }
+        s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (on[u]) fold(s, xv);
       }
     }
+  };
+
+  auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
+    if (w_hi > w_lo) window_loop(w_lo, w_hi);
+    if (klev > 0 || vlev > 0) tree_loop(klev, vlev);
+    if (tokens) token_loop();
   };
 
   // Warp top-k of head h at level lev over the full score table (every CTA).
@@ -315,6 +430,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     w_lo = min(nw, rank * ch);
     w_hi = min(nw, w_lo + ch);
   }
+  const bool has_win = w_hi > w_lo;
   if (top > 0) {
     rotate_q(qlev, cnt_c[top]);
     __syncthreads();
@@ -369,6 +485,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int h = x / D, c = x % D;
     float mm = -INFINITY;
     for (int w = h * WPH; w < (h + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * (D + 2) + D]);
+    if (has_win)
+      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * (D + 2) + D]);
     float aa = 0.f, ll = 0.f;
     for (int w = h * WPH; w < (h + 1) * WPH; ++w) {
       const float* ws = wsc + w * (D + 2);
@@ -376,6 +494,13 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       aa = fmaf(ws[c], r, aa);
       ll = fmaf(ws[D + 1], r, ll);
     }
+    if (has_win)
+      for (int w = 0; w < kWarps; ++w) {
+        const float* ws = wwin + (w * G + h) * (D + 2);
+        const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+        aa = fmaf(ws[c], r, aa);
+        ll = fmaf(ws[D + 1], r, ll);
+      }
     dst[h * (D + 2) + c] = aa;
     if (c == 0) {
       dst[h * (D + 2) + D] = mm;
@@ -442,6 +567,7 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   const int kmax = int(kk < cmax ? kk : cmax);
   if (cmax > 1024) return cudaErrorNotSupported;
   const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * (D + 2) +
+                        size_t(kWarps) * G * (D + 2) +
                         size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
                        size_t(2) * G * cmax + 16;
   if (bytes > 200 * 1024) return cudaErrorNotSupported;
