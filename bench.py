@@ -298,12 +298,15 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
     Q = make_prefill_queries(w, Kc, L)
     O = torch.empty_like(Q)
     chunk = 65536
+    ws = None if args.no_window_ws else torch.empty(R.recsa_prefill_workspace_bytes(gp, chunk),
+                                                    dtype=torch.uint8, device="cuda")
 
     def once():
         R.recsa_build(gp, K0, V0, [L], r, 0, tree)
         for c0 in range(0, L, chunk):
             n = min(chunk, L - c0)
-            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n])
+            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n],
+                            workspace=ws)
 
     once()
     torch.cuda.synchronize()
@@ -316,7 +319,8 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
         e1.record(stream)
         for c0 in range(0, L, chunk):
             n = min(chunk, L - c0)
-            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n])
+            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n],
+                            workspace=ws)
         e2.record(stream)
         torch.cuda.synchronize()
         times.append(elapsed(e0, e2))
@@ -494,6 +498,8 @@ def main():
     ap.add_argument("--impl", default="recsa", choices=["recsa", "reference"])
     ap.add_argument("--prefill-reps", type=int, default=1)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-window-ws", action="store_true",
+                    help="prefill without a workspace (window attended by the tree kernel)")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-dense-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

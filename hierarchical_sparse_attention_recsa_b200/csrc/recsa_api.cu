@@ -99,6 +99,11 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   return RECSA_OK;
 }
 
+// Window partials (max, sum) as float2 per (sequence, query, head).
+size_t prefill_workspace_need(const Params& p, int32_t n_q) {
+  return size_t(p.batch) * size_t(n_q) * size_t(p.hq) * sizeof(float2);
+}
+
 recsa_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return RECSA_OK;
   fprintf(stderr, "recsa: CUDA error: %s\n", cudaGetErrorString(e));
@@ -194,24 +199,35 @@ recsa_status recsa_append(const recsa_geometry* geom, void* K, void* V, const vo
 static recsa_status attend_common(const recsa_geometry* geom, const void* Q, const void* K,
                                   const void* V, const void* tree, const int64_t* len_dev,
                                   int64_t q_start, int32_t n_q, int decode, void* O,
-                                  int32_t* trace, void* stream) {
+                                  int32_t* trace, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
   Params p;
   recsa_status st = make_params(geom, &p);
   if (st != RECSA_OK) return st;
   if (!Q || !K || !V || !tree || !O || (decode && !len_dev)) return RECSA_ERR_NULL;
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
-      !aligned(tree, 256) || (trace && !aligned(trace, 4)) || (decode && !aligned(len_dev, 8)))
+      !aligned(tree, 256) || (trace && !aligned(trace, 4)) || (decode && !aligned(len_dev, 8)) ||
+      (workspace && !aligned(workspace, 16)))
     return RECSA_ERR_MISALIGNED;
   if (n_q < 0) return RECSA_ERR_CAPACITY;
   if (!decode && (q_start < 0 || q_start + n_q > geom->capacity)) return RECSA_ERR_CAPACITY;
   if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
+  if (workspace && workspace_bytes < prefill_workspace_need(p, n_q)) return RECSA_ERR_CAPACITY;
   if (n_q == 0) return RECSA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (decode && !getenv("RECSA_DECODE_GENERIC"))
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
-  if (!decode && !getenv("RECSA_PREFILL_GENERIC"))
-    e = launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+  if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
+    const void* wml = nullptr;
+    if (workspace) {
+      e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, O, workspace, s);
+      if (e == cudaSuccess) wml = workspace;
+      else if (e != cudaErrorNotSupported) return cuda_status(e);
+      else cudaGetLastError();
+    }
+    e = launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s);
+  }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
     e = launch_attend(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);
@@ -226,13 +242,26 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
 recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void* K,
                           const void* V, const void* tree, const int64_t* len_dev,
                           int32_t n_q, void* O, int32_t* trace, void* stream) {
-  return attend_common(geom, Q, K, V, tree, len_dev, 0, n_q, 1, O, trace, stream);
+  return attend_common(geom, Q, K, V, tree, len_dev, 0, n_q, 1, O, trace, nullptr, 0, stream);
+}
+
+recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n_q,
+                                           size_t* bytes) {
+  if (!bytes) return RECSA_ERR_NULL;
+  Params p;
+  recsa_status st = make_params(geom, &p);
+  if (st != RECSA_OK) return st;
+  if (n_q < 0) return RECSA_ERR_CAPACITY;
+  *bytes = prefill_workspace_need(p, n_q);
+  return RECSA_OK;
 }
 
 recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void* K,
                            const void* V, const void* tree, int64_t q_start, int32_t n_q,
-                           void* O, int32_t* trace, void* stream) {
-  return attend_common(geom, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, stream);
+                           void* O, int32_t* trace, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return attend_common(geom, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, workspace,
+                       workspace_bytes, stream);
 }
 
 recsa_status recsa_tree_error(const recsa_geometry* geom, void* tree, int32_t clear,

@@ -98,8 +98,15 @@ cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);
 // Warp-per-(query, head) prefill kernel; cudaErrorNotSupported outside its limits.
+// wml: window partials (max, sum) per (sequence, query, head) from
+// launch_prefill_window, or null to let this kernel attend the window itself.
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
-                                int32_t* trace, cudaStream_t s);
+                                int32_t* trace, const void* wml, cudaStream_t s);
+// Tensor-core window partials for a prefill range (bf16): normalised window
+// output into O, (max, sum) into ml; cudaErrorNotSupported outside its limits.
+cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,
+                                  const void* tree, int64_t q_start, int32_t n_q, void* O,
+                                  void* ml, cudaStream_t s);
 
 }  // namespace recsa

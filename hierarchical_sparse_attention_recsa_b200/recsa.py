@@ -38,8 +38,8 @@ STATUS = {
 }
 
 EXPORTS = ["recsa_status_string", "recsa_validate", "recsa_num_levels", "recsa_tree_bytes",
-           "recsa_build", "recsa_append", "recsa_decode", "recsa_prefill", "recsa_trace_ints",
-           "recsa_tree_error"]
+           "recsa_build", "recsa_append", "recsa_decode", "recsa_prefill",
+           "recsa_prefill_workspace_bytes", "recsa_trace_ints", "recsa_tree_error"]
 
 
 class RecsaError(RuntimeError):
@@ -115,7 +115,9 @@ def lib() -> ctypes.CDLL:
         L.recsa_build.argtypes = [G, vp, vp, ctypes.POINTER(i64), vp, i64, vp, vp]
         L.recsa_append.argtypes = [G, vp, vp, vp, vp, vp, vp, i64, vp, vp]
         L.recsa_decode.argtypes = [G, vp, vp, vp, vp, vp, i32, vp, vp, vp]
-        L.recsa_prefill.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp]
+        L.recsa_prefill.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp, ctypes.c_size_t,
+                                    vp]
+        L.recsa_prefill_workspace_bytes.argtypes = [G, i32, ctypes.POINTER(ctypes.c_size_t)]
         L.recsa_trace_ints.argtypes = [G, ctypes.POINTER(i32)]
         L.recsa_tree_error.argtypes = [G, vp, i32, ctypes.POINTER(ctypes.c_uint32), vp]
         for name in EXPORTS:
@@ -201,10 +203,21 @@ def recsa_decode(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tens
 
 def recsa_prefill(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                   tree: torch.Tensor, q_start: int, n_q: int, O: torch.Tensor,
-                  trace: Optional[torch.Tensor] = None, stream=None) -> None:
+                  trace: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
     g = geom.c()
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().recsa_prefill(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree), q_start,
-                               n_q, _ptr(O), _ptr(trace), _stream(stream)), "recsa_prefill")
+                               n_q, _ptr(O), _ptr(trace), _ptr(workspace), wbytes,
+                               _stream(stream)), "recsa_prefill")
+
+
+def recsa_prefill_workspace_bytes(geom: Geometry, n_q: int) -> int:
+    g = geom.c()
+    out = ctypes.c_size_t()
+    _check(lib().recsa_prefill_workspace_bytes(ctypes.byref(g), n_q, ctypes.byref(out)),
+           "recsa_prefill_workspace_bytes")
+    return out.value
 
 
 def recsa_tree_error(geom: Geometry, tree: torch.Tensor, clear: bool = False,

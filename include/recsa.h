@@ -154,10 +154,23 @@ recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void*
  * tokens of every sequence (a node is a pure function of its span, so a tree
  * built over more tokens serves every earlier query: each query sees only the
  * nodes that end before its window).
+ *   workspace: NULL, or DEVICE memory of at least
+ *   recsa_prefill_workspace_bytes(geom, n_q) bytes (16-byte aligned) given as
+ *   workspace_bytes.  With a workspace and bf16 data the exact window runs on
+ *   the tensor cores and its partial softmax (max, sum per query head) is kept
+ *   there until the tree kernel merges it; without one, the window is attended
+ *   by the tree kernel itself.  Both give the same result within rounding.
+ *   The workspace is only read and written by this call; calls that share one
+ *   must not overlap on the device.
  */
 recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void* K,
                            const void* V, const void* tree, int64_t q_start, int32_t n_q,
-                           void* O, int32_t* trace, void* stream);
+                           void* O, int32_t* trace, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* Workspace bytes recsa_prefill needs for n_q queries per sequence. */
+recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n_q,
+                                           size_t* bytes);
 
 /*
  * Trace record length in int32 per (sequence, query, head):

@@ -104,6 +104,11 @@ def test_tree_bytes(lib, kw):
     assert R.recsa_tree_bytes(g) == expected_tree_bytes(g)
 
 
+def test_prefill_workspace_bytes(lib):
+    g = geo(batch=2, capacity=4096)
+    assert R.recsa_prefill_workspace_bytes(g, 100) == 2 * 100 * 32 * 8
+
+
 def test_trace_ints(lib):
     assert R.recsa_trace_ints(geo(k=8)) == 4 + 32 + 16 * 8
     with pytest.raises(R.RecsaError):
@@ -124,18 +129,20 @@ def test_argument_errors_return_before_device(lib):
     # NULL pointers
     assert lib.recsa_build(ctypes.byref(cg), None, ok, lens, r, 0, ok, None) == 2
     assert lib.recsa_decode(ctypes.byref(cg), ok, ok, ok, ok, None, 1, ok, None, None) == 2
-    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, None, 0, 1, ok, None, None) == 2
+    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, None, 0, 1, ok, None, None, 0, None) == 2
     assert lib.recsa_append(ctypes.byref(cg), ok, ok, ok, ok, None, r, 0, ok, None) == 2
     # misaligned tree (needs 256) and K (needs 16)
     assert lib.recsa_build(ctypes.byref(cg), ok, ok, lens, r, 0, mis, None) == 3
     assert lib.recsa_prefill(ctypes.byref(cg), ok, ctypes.c_void_p((1 << 20) + 4), ok, ok, 0, 1,
-                             ok, None, None) == 3
+                             ok, None, None, 0, None) == 3
     # lengths and query ranges beyond capacity
     bad = (ctypes.c_int64 * 1)(4097)
     assert lib.recsa_build(ctypes.byref(cg), ok, ok, bad, r, 0, ok, None) == 4
-    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 4000, 97, ok, None, None) == 4
+    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 4000, 97, ok, None, None, 0, None) == 4
+    # a workspace smaller than recsa_prefill_workspace_bytes
+    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 0, 8, ok, None, ok, 16, None) == 4
     # trace with k beyond the trace limit
     g2 = geo(batch=1, capacity=4096, k=100).c()
     assert lib.recsa_decode(ctypes.byref(g2), ok, ok, ok, ok, ok, 1, ok, ok, None) == 5
     # zero queries: nothing to do
-    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 0, 0, ok, None, None) == 0
+    assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 0, 0, ok, None, None, 0, None) == 0

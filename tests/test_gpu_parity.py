@@ -47,9 +47,11 @@ def decode_impl(request):
             os.environ[k] = v
 
 
-@pytest.fixture(params=["warp", "generic"])
+@pytest.fixture(params=["warp", "window", "generic"])
 def prefill_impl(request):
-    """Select the prefill kernel: warp-per-(query, head) or the generic kernel."""
+    """Select the prefill path: the warp-per-(query, head) kernel alone, the
+    tensor-core window kernel plus the warp kernel (needs a workspace; bf16
+    only, fp32 falls back to the warp kernel), or the generic kernel."""
     old = os.environ.pop("RECSA_PREFILL_GENERIC", None)
     if request.param == "generic":
         os.environ["RECSA_PREFILL_GENERIC"] = "1"
@@ -57,6 +59,14 @@ def prefill_impl(request):
     os.environ.pop("RECSA_PREFILL_GENERIC", None)
     if old is not None:
         os.environ["RECSA_PREFILL_GENERIC"] = old
+
+
+def _prefill(g, impl, Q, K, V, tree, q0, nq, O, trace=None):
+    ws = None
+    if impl == "window":
+        ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8,
+                         device="cuda")
+    R.recsa_prefill(g, Q, K, V, tree, q0, nq, O, trace, workspace=ws)
 
 
 def _setup(w, lens, capacity, seed=0, k=None, rope=1):
@@ -147,7 +157,7 @@ def test_prefill_tiny_all_positions(tiny, prefill_impl):
     O = torch.empty_like(Qd)
     ti = R.recsa_trace_ints(g)
     trace = torch.zeros((1, L, g.n_q_heads, ti), dtype=torch.int32, device="cuda")
-    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O, trace)
+    _prefill(g, prefill_impl, Qd, Kd, Vd, tree, 0, L, O, trace)
     torch.cuda.synchronize()
     og = oracle_geometry(g)
     Kh, Vh, levels = trees[(0, 0)]
@@ -218,7 +228,7 @@ def test_prefill_model_small(model_small, prefill_impl):
     O = torch.empty_like(Qd)
     ti = R.recsa_trace_ints(g)
     trace = torch.zeros((2, nq, g.n_q_heads, ti), dtype=torch.int32, device="cuda")
-    R.recsa_prefill(g, Qd, Kd, Vd, tree, q0, nq, O, trace)
+    _prefill(g, prefill_impl, Qd, Kd, Vd, tree, q0, nq, O, trace)
     torch.cuda.synchronize()
     og = oracle_geometry(g)
     O_, tr = to_np(O), trace.cpu().numpy()
@@ -247,7 +257,7 @@ def test_keep_all_is_dense(wname, rope, prefill_impl):
     Q, _, _ = synth.make_queries(w, K, pos, seed=7)
     Qd = Q.cuda()
     O = torch.empty_like(Qd)
-    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O)
+    _prefill(g, prefill_impl, Qd, Kd, Vd, tree, 0, L, O)
     Od = torch.empty_like(Qd[:, :1])
     lens = torch.tensor([L], dtype=torch.int64, device="cuda")
     R.recsa_decode(g, Qd[:, -1:].contiguous(), Kd, Vd, tree, lens, 1, Od)
