@@ -22,7 +22,7 @@ constexpr int kPThreads = 256;
 constexpr int kPWarps = kPThreads / 32;
 constexpr int kPUnroll = 2;
 
-enum PItem { pKey = 0, pVal = 1, pTok = 2, pNone = 3 };
+enum PItem { pKey = 0, pVal = 1, pNone = 2 };
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kPThreads, 2)
@@ -126,14 +126,51 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     return p.b * vup + (i - p.b * kup);
   };
 
-  // Window rows (first pass), key pairs of klev, unselected values of vlev,
-  // kept-leaf tokens (last pass).  32-bit index math, constants hoisted.
-  auto run_pass = [&](bool window, int klev, int vlev, bool tokens) {
-    const int nw = window ? int(n_win) : 0;
+  // Token rows: the window [a*B, t] (when this kernel attends it) or the
+  // kept leaves' tokens, each at its token-level index; K/V rows in dtype.
+  auto token_loop = [&](bool window) {
+    const int nt = window ? int(n_win) : nleaf * p.B;
+    const int win0 = int(a) * p.B;
+    const int widx0 = nleaf * p.B;
+    const int* kept1 = kept + 1 * kmax;                           // level 1 = parity 1
+    for (int base = 0; base < nt; base += SPW * kPUnroll) {
+      RawPairs rk[kPUnroll], rv[kPUnroll];
+      float cs[kPUnroll][8];
+      bool on[kPUnroll];
+#pragma unroll
+      for (int u = 0; u < kPUnroll; ++u) {
+        const int e = base + u * SPW + slot;
+        on[u] = e < nt;
+        if (on[u]) {
+          const int pos = window ? win0 + e : kept1[div_B(p, e)] * p.B + mod_B(p, e);
+          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
+          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
+          if (p.rope) load_cs(rope, window ? widx0 + e : e, HALF, j0, cs[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPUnroll; ++u) {
+        float xk[8], xv[8], s = 0.f;
+        RawLoad<T, HALF>::cvt(rk[u], xk);
+        RawLoad<T, HALF>::cvt(rv[u], xv);
+        if (p.rope) rotate8(xk, cs[u]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          s = fmaf(qtok[j0 + c], xk[c], s);
+          s = fmaf(qtok[HALF + j0 + c], xk[4 + c], s);
+        }
+        s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (on[u]) fold(s, xv);
+      }
+    }
+  };
+
+  // Tree rows: key candidates of level klev (scored into sc) and the
+  // unselected candidates of level vlev (values folded); fp32 rows.
+  auto tree_loop = [&](int klev, int vlev) {
     const int nk = klev > 0 ? cnt_c[klev] : 0;
     const int nv = vlev > 0 ? cnt_c[vlev] : 0;
-    const int nt = tokens ? nleaf * p.B : 0;
-    const int total = nw + nk + nv + nt;
+    const int total = nk + nv;
     const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
     const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
     const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
@@ -144,13 +181,11 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     const int nchV = p.b * kupV;
     const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
     const int* keptV = kept + ((vlev + 1) & 1) * kmax;
-    const int* kept1 = kept + 1 * kmax;                           // level 1 = parity 1
     const float* scV = sc + (vlev & 1) * cmax;
     const unsigned char* flV = kfl + (vlev & 1) * cmax;
-    const int win0 = int(a) * p.B;
-    const int widx0 = nleaf * p.B;
+    float* scK = sc + (klev & 1) * cmax;
     for (int base = 0; base < total; base += SPW * kPUnroll) {
-      RawPairs ra[kPUnroll], rb[kPUnroll];
+      RawPairs ra[kPUnroll];
       float cs[kPUnroll][8];
       int kind[kPUnroll], idx[kPUnroll];
       float sv[kPUnroll];
@@ -160,65 +195,49 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         kind[u] = pNone;
         idx[u] = 0;
         sv[u] = 0.f;
-        if (e < nw) {
-          const int pos = win0 + e;
-          kind[u] = pTok;
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
-          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
-        } else if (e < nw + nk) {
-          const int i = e - nw;
+        if (e < nk) {
+          const int i = e;
           const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
           kind[u] = pKey;
           idx[u] = i;
           RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
           if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
-        } else if (e < nw + nk + nv) {
-          const int i = e - nw - nk;
+        } else if (e < total) {
+          const int i = e - nk;
           if (!flV[i]) {
             const int node = i < nchV ? keptV[div_b(p, i)] * p.b + mod_b(p, i) : orphV + i;
             kind[u] = pVal;
             sv[u] = scV[i];
             RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
           }
-        } else if (e < total) {
-          const int r = e - nw - nk - nv;
-          const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
-          kind[u] = pTok;
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, ra[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rb[u]);
-          if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
-        float s = 0.f, xa[8], xb[8];
-        if (kind[u] == pKey || kind[u] == pVal) {
-          RawLoad<float, HALF>::cvt(ra[u], xa);
-        } else {
-          RawLoad<T, HALF>::cvt(ra[u], xa);
-          RawLoad<T, HALF>::cvt(rb[u], xb);
-        }
-        if (kind[u] == pKey || kind[u] == pTok) {
-          if (p.rope) rotate8(xa, cs[u]);
-          const float* qv = kind[u] == pKey ? qlev : qtok;
+        float x[8], s = 0.f;
+        RawLoad<float, HALF>::cvt(ra[u], x);
+        if (kind[u] == pKey) {
+          if (p.rope) rotate8(x, cs[u]);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            s = fmaf(qv[j0 + c], xa[c], s);
-            s = fmaf(qv[HALF + j0 + c], xa[4 + c], s);
+            s = fmaf(qlev[j0 + c], x[c], s);
+            s = fmaf(qlev[HALF + j0 + c], x[4 + c], s);
           }
         }
-        if (__any_sync(0xffffffffu, kind[u] == pKey || kind[u] == pTok))
-          s = slot_sum<LPR>(s) * inv_sqrt_d;
+        if (__any_sync(0xffffffffu, kind[u] == pKey)) s = slot_sum<LPR>(s) * inv_sqrt_d;
         if (kind[u] == pKey) {
-          if (sub == 0) sc[(klev & 1) * cmax + idx[u]] = s;
-        } else if (kind[u] == pTok) {
-          fold(s, xb);
+          if (sub == 0) scK[idx[u]] = s;
         } else if (kind[u] == pVal) {
-          fold(sv[u], xa);
+          fold(sv[u], x);
         }
       }
     }
+  };
+
+  auto run_pass = [&](bool window, int klev, int vlev, bool tokens) {
+    if (window) token_loop(true);
+    if (klev > 0 || vlev > 0) tree_loop(klev, vlev);
+    if (tokens) token_loop(false);
     __syncwarp();
   };
 
