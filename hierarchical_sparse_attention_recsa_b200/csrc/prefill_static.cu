@@ -1,0 +1,68 @@
+// recsa_prefill_static: the tensor-core window prefill with its scratch in a
+// fixed device array instead of a caller workspace.
+//
+// Some callers cannot hand the library any device memory beyond the tensors
+// of the call: a runtime whose device memory is entirely planned ahead and
+// owned by its own arena, or a plain C host that has no device allocator on
+// its call path.  For them this entry point keeps the window partials (max,
+// sum per query head) in a file-scope device array of kStaticEntries float2
+// (4 MiB), which every GPU that loads the library holds until the process
+// exits.  Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+#include <mutex>
+
+#include "recsa_internal.cuh"
+
+namespace recsa {
+namespace {
+
+// batch * n_q * n_q_heads must not exceed this (4 MiB of float2).
+constexpr size_t kStaticEntries = size_t(1) << 19;
+
+__device__ __align__(256) float2 g_prefill_scratch[kStaticEntries];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the host-side symbol is only a stand-in for it).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+size_t prefill_static_max_entries() { return kStaticEntries; }
+
+cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,
+                                  const void* tree, int64_t q_start, int32_t n_q, void* O,
+                                  int32_t* trace, cudaStream_t s) {
+  void* ml = nullptr;
+  cudaError_t e = scratch_address(&ml);
+  if (e != cudaSuccess) return e;
+  // The window kernel writes every (max, sum) entry of the range before the
+  // tree kernel reads it, so the array needs no clearing between calls.
+  e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, O, ml, s);
+  const void* wml = ml;
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    wml = nullptr;   // geometry outside the window kernel: the tree kernel attends it
+  } else if (e != cudaSuccess) {
+    return e;
+  }
+  return launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s);
+}
+
+}  // namespace recsa

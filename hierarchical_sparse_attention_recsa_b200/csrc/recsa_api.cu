@@ -245,6 +245,41 @@ recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void*
   return attend_common(geom, Q, K, V, tree, len_dev, 0, n_q, 1, O, trace, nullptr, 0, stream);
 }
 
+recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, const void* K,
+                                  const void* V, const void* tree, int64_t q_start, int32_t n_q,
+                                  void* O, int32_t* trace, void* stream) {
+  Params p;
+  recsa_status st = make_params(geom, &p);
+  if (st != RECSA_OK) return st;
+  if (!Q || !K || !V || !tree || !O) return RECSA_ERR_NULL;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+      !aligned(tree, 256) || (trace && !aligned(trace, 4)))
+    return RECSA_ERR_MISALIGNED;
+  if (n_q < 0 || q_start < 0 || q_start + n_q > geom->capacity) return RECSA_ERR_CAPACITY;
+  if (size_t(geom->batch) * size_t(n_q) * size_t(geom->n_q_heads) >
+      prefill_static_max_entries()) {
+    fprintf(stderr,
+            "recsa_prefill_static: batch * n_q * n_q_heads = %zu exceeds the fixed scratch of "
+            "%zu query heads; split the call into smaller query ranges\n",
+            size_t(geom->batch) * size_t(n_q) * size_t(geom->n_q_heads),
+            prefill_static_max_entries());
+    return RECSA_ERR_CAPACITY;
+  }
+  if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
+  if (n_q == 0) return RECSA_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_prefill_static(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_attend(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, s);
+  }
+  if (e == cudaErrorInvalidConfiguration || e == cudaErrorInvalidValue) {
+    cudaGetLastError();
+    return RECSA_ERR_UNSUPPORTED;
+  }
+  return cuda_status(e);
+}
+
 recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n_q,
                                            size_t* bytes) {
   if (!bytes) return RECSA_ERR_NULL;

@@ -103,6 +103,12 @@ cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K,
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
                                 int32_t* trace, const void* wml, cudaStream_t s);
+// Prefill with the window partials kept in a fixed device array (no caller
+// workspace); prefill_static_max_entries() bounds batch * n_q * n_q_heads.
+cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,
+                                  const void* tree, int64_t q_start, int32_t n_q, void* O,
+                                  int32_t* trace, cudaStream_t s);
+size_t prefill_static_max_entries();
 // Tensor-core window partials for a prefill range (bf16): normalised window
 // output into O, (max, sum) into ml; cudaErrorNotSupported outside its limits.
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,

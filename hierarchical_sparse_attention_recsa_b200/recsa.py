@@ -39,7 +39,8 @@ STATUS = {
 
 EXPORTS = ["recsa_status_string", "recsa_validate", "recsa_num_levels", "recsa_tree_bytes",
            "recsa_build", "recsa_append", "recsa_decode", "recsa_prefill",
-           "recsa_prefill_workspace_bytes", "recsa_trace_ints", "recsa_tree_error"]
+           "recsa_prefill_workspace_bytes", "recsa_prefill_static", "recsa_trace_ints",
+           "recsa_tree_error"]
 
 
 class RecsaError(RuntimeError):
@@ -118,6 +119,7 @@ def lib() -> ctypes.CDLL:
         L.recsa_prefill.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp, ctypes.c_size_t,
                                     vp]
         L.recsa_prefill_workspace_bytes.argtypes = [G, i32, ctypes.POINTER(ctypes.c_size_t)]
+        L.recsa_prefill_static.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp]
         L.recsa_trace_ints.argtypes = [G, ctypes.POINTER(i32)]
         L.recsa_tree_error.argtypes = [G, vp, i32, ctypes.POINTER(ctypes.c_uint32), vp]
         for name in EXPORTS:
@@ -210,6 +212,17 @@ def recsa_prefill(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Ten
     _check(lib().recsa_prefill(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree), q_start,
                                n_q, _ptr(O), _ptr(trace), _ptr(workspace), wbytes,
                                _stream(stream)), "recsa_prefill")
+
+
+def recsa_prefill_static(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                         tree: torch.Tensor, q_start: int, n_q: int, O: torch.Tensor,
+                         trace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """recsa_prefill with the library's fixed device scratch instead of a
+    caller workspace (for callers that cannot provide device memory)."""
+    g = geom.c()
+    _check(lib().recsa_prefill_static(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree),
+                                      q_start, n_q, _ptr(O), _ptr(trace), _stream(stream)),
+           "recsa_prefill_static")
 
 
 def recsa_prefill_workspace_bytes(geom: Geometry, n_q: int) -> int:

@@ -168,6 +168,26 @@ recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void
                            void* O, int32_t* trace, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/*
+ * recsa_prefill without a workspace argument, for callers that cannot hand
+ * the library any device memory beyond the call's tensors: a runtime whose
+ * device memory is planned ahead and owned by its own arena, or a C host with
+ * no device allocator on its call path.  (The pages have no counterpart: it
+ * is a packaging variant of recsa_prefill, same arguments and result.)
+ *   Scratch: the window partials live in a fixed device array of 2^19 query
+ *   heads (4 MiB), which every GPU that loads the library holds until the
+ *   process exits.  batch * n_q * n_q_heads above 2^19 is rejected with
+ *   RECSA_ERR_CAPACITY (and a message on stderr): split the query range.
+ *   The array needs no clearing (each call writes what it reads), but every
+ *   call shares it: calls that overlap on the device race.
+ *   Set-up: the first call on each device, with that device current, looks up
+ *   the array's device address; make that first call before any stream
+ *   capture.  Nothing is allocated by this call.
+ */
+recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, const void* K,
+                                  const void* V, const void* tree, int64_t q_start, int32_t n_q,
+                                  void* O, int32_t* trace, void* stream);
+
 /* Workspace bytes recsa_prefill needs for n_q queries per sequence. */
 recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n_q,
                                            size_t* bytes);
