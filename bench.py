@@ -121,8 +121,19 @@ class Clocks:
 def geometry(w, batch, capacity) -> R.Geometry:
     return R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                       leaf_block=w.leaf_block, branching=w.branching, k=w.k, window=w.window,
-                      batch=batch, capacity=capacity, dtype=R.DTYPE_BF16,
+                      batch=batch, capacity=capacity,
+                      dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
                       rope_enabled=1, rope_base=w.rope_base)
+
+
+def metric_for(name, L):
+    if name == WORKLOAD:
+        return METRIC
+    return f"decode queries/s and prefill tokens/s at L={L} ({name}) on 1 B200; % of HBM roofline"
+
+
+def elem_bytes(w):
+    return 2 if w.dtype == torch.bfloat16 else 4
 
 
 class L2Flush:
@@ -137,13 +148,13 @@ def elapsed(a, b):
     return a.elapsed_time(b)
 
 
-def make_prefill_queries(w, K, L, chunk=65536):
-    Q = torch.empty((1, L, w.n_q_heads, w.head_dim), dtype=w.dtype, device="cuda")
-    for c0 in range(0, L, chunk):
+def make_prefill_queries(w, K, q0, L, chunk=65536):
+    Q = torch.empty((1, L - q0, w.n_q_heads, w.head_dim), dtype=w.dtype, device="cuda")
+    for c0 in range(q0, L, chunk):
         n = min(chunk, L - c0)
         pos = (c0 + torch.arange(n, device="cuda", dtype=torch.int64))[None]
         q, _, _ = synth.make_queries(w, K[:1], pos, seed=100 + c0 // chunk)
-        Q[:, c0:c0 + n] = q
+        Q[:, c0 - q0:c0 - q0 + n] = q
     return Q
 
 
@@ -152,7 +163,7 @@ def make_prefill_queries(w, K, L, chunk=65536):
 # ---------------------------------------------------------------------------
 
 def run_recsa(args, rank, world, dev):
-    w = synth.WORKLOADS[WORKLOAD]
+    w = synth.WORKLOADS[args.workload]
     if args.length:
         w = synth.Workload(**{**w.__dict__, "length": args.length})
     L, batch = w.length, w.batch
@@ -222,7 +233,7 @@ def run_recsa(args, rank, world, dev):
         lens_i = np.full(batch, L + i + 1)
         acc.append(counts.decode_bytes_from_trace(tr[i], lens_i, w.leaf_block, w.branching,
                                                   w.window, w.n_q_heads // w.n_kv_heads,
-                                                  w.head_dim, 2, w.k))
+                                                  w.head_dim, elem_bytes(w), w.k))
     dec_bytes = float(np.mean([a["bytes"] for a in acc]))
     achieved = dec_bytes / (dec_ms / 1e3) / 1e9
 
@@ -259,19 +270,21 @@ def run_recsa(args, rank, world, dev):
     clk = clocks.stop()
 
     out = {
-        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "metric": metric_for(args.workload, L), "value": value, "unit": "queries/s",
+        "n_gpus": world,
         "steps": K_steps, "warmup": W_steps, "ms_per_step": step_ms / K_steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic: K,V ~ N(0,1) x per-channel LogNormal(0,0.5) scale, Q ~ N(0,1), "
                 "1% planted needles, seeded",
-        "config": {"workload": WORKLOAD, "L": L, "batch": batch, "q_heads": w.n_q_heads,
+        "config": {"workload": args.workload, "L": L, "batch": batch, "q_heads": w.n_q_heads,
                    "kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                    "leaf_block": w.leaf_block, "branching": w.branching, "k": w.k,
                    "window": w.window, "levels": R.recsa_num_levels(g, L),
                    "step": "recsa_append + recsa_decode for the batch",
                    "l2": "flushed before every timed step (256 MiB write, outside the events)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "kernel": "recsa decode (attend_kernel)",
+        "roofline": {"bound": "hbm", "kernel": "decode_cluster_kernel",
                      "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
@@ -281,21 +294,24 @@ def run_recsa(args, rank, world, dev):
     }
     del traces
     torch.cuda.empty_cache()
-    if not args.no_prefill:
+    if not args.no_prefill and args.workload != "decode-1m":
         out["prefill"] = run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs)
     if not args.no_dense:
         out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
     if rank == 0 and world == 1 and not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
     return out
 
 
 def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
+    """recsa_build over one sequence's L tokens, then recsa_prefill of the
+    workload's query range (all L positions, or the last prefill_queries)."""
     L = w.length
+    q0 = L - w.extra.get("prefill_queries", L)
     gp = geometry(w, 1, cap)
     K0, V0 = Kc[:1], Vc[:1]
     tree = torch.zeros(R.recsa_tree_bytes(gp), dtype=torch.uint8, device="cuda")
-    Q = make_prefill_queries(w, Kc, L)
+    Q = make_prefill_queries(w, Kc, q0, L)
     O = torch.empty_like(Q)
     chunk = 65536
     ws = None if args.no_window_ws else torch.empty(R.recsa_prefill_workspace_bytes(gp, chunk),
@@ -303,10 +319,10 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
 
     def once():
         R.recsa_build(gp, K0, V0, [L], r, 0, tree)
-        for c0 in range(0, L, chunk):
+        for c0 in range(q0, L, chunk):
             n = min(chunk, L - c0)
-            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n],
-                            workspace=ws)
+            R.recsa_prefill(gp, Q[:, c0 - q0:c0 - q0 + n], K0, V0, tree, c0, n,
+                            O[:, c0 - q0:c0 - q0 + n], workspace=ws)
 
     once()
     torch.cuda.synchronize()
@@ -317,27 +333,29 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
         e0.record(stream)
         R.recsa_build(gp, K0, V0, [L], r, 0, tree)
         e1.record(stream)
-        for c0 in range(0, L, chunk):
+        for c0 in range(q0, L, chunk):
             n = min(chunk, L - c0)
-            R.recsa_prefill(gp, Q[:, c0:c0 + n], K0, V0, tree, c0, n, O[:, c0:c0 + n],
-                            workspace=ws)
+            R.recsa_prefill(gp, Q[:, c0 - q0:c0 - q0 + n], K0, V0, tree, c0, n,
+                            O[:, c0 - q0:c0 - q0 + n], workspace=ws)
         e2.record(stream)
         torch.cuda.synchronize()
         times.append(elapsed(e0, e2))
         build_t.append(elapsed(e0, e1))
     ms = min(times)
-    t = np.arange(L)
+    t = np.arange(q0, L)
     ent, keys = counts.per_query_counts(t, w.leaf_block, w.branching, w.k, w.window,
                                         R.recsa_num_levels(gp, L))
     flops = float(2 * w.head_dim * (ent.sum() + keys.sum()) * w.n_q_heads)
     attend_ms = ms - min(build_t)
-    kv_bytes = 2 * L * w.n_kv_heads * w.head_dim * 2
+    kv_bytes = 2 * L * w.n_kv_heads * w.head_dim * elem_bytes(w)
     build_ms = min(build_t)
     del Q, O, tree
     torch.cuda.empty_cache()
-    return {"value": L / (ms / 1e3), "unit": "tokens/s", "ms": ms, "reps": args.prefill_reps,
-            "build_ms": build_ms, "attend_ms": attend_ms, "queries": L,
-            "roofline": {"bound": "alu", "kernel": "recsa prefill (attend_kernel)",
+    return {"value": (L - q0) / (ms / 1e3), "unit": "tokens/s", "ms": ms,
+            "reps": args.prefill_reps, "build_ms": build_ms, "attend_ms": attend_ms,
+            "queries": L - q0, "q_start": q0, "tokens_built": L,
+            "roofline": {"bound": "alu",
+                         "kernel": "window_mma_kernel + prefill_warp_kernel",
                          "achieved": flops / (attend_ms / 1e3) / 1e12,
                          "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
                          "frac": flops / (attend_ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS,
@@ -374,9 +392,9 @@ def run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, prefill):
         res["decode_queries_per_s"] = w.batch / (ms / 1e3)
     except Exception as e:  # library kernel unavailable for this shape
         res["decode_error"] = str(e).splitlines()[0][:200]
-    if prefill is not None and not args.no_dense_prefill:
+    if prefill is not None and not args.no_dense_prefill and prefill.get("q_start", 0) == 0:
         try:
-            Q = make_prefill_queries(w, Kc, L).permute(0, 2, 1, 3)
+            Q = make_prefill_queries(w, Kc, 0, L).permute(0, 2, 1, 3)
             Kd, Vd = Kc[:1, :, :L], Vc[:1, :, :L]
             with sdpa_kernel(backends):
                 torch.nn.functional.scaled_dot_product_attention(Q, Kd, Vd, is_causal=True,
@@ -405,11 +423,13 @@ def run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, prefill):
 class OracleDecode:
     """The float64 oracle on one KV head (G = 4 query heads) of the workload."""
 
-    def __init__(self, seed=0):
+    def __init__(self, workload=WORKLOAD, seed=0):
         import oracle
         self.oracle = oracle
-        w = synth.WORKLOADS[WORKLOAD]
-        self.w1 = synth.Workload(**{**w.__dict__, "n_q_heads": 4, "n_kv_heads": 1, "batch": 1})
+        w = synth.WORKLOADS[workload]
+        G = w.n_q_heads // w.n_kv_heads
+        self.G = G
+        self.w1 = synth.Workload(**{**w.__dict__, "n_q_heads": G, "n_kv_heads": 1, "batch": 1})
         L = w.length
         self.L = L
         n = 64
@@ -419,7 +439,7 @@ class OracleDecode:
         pos = (L + torch.arange(n, dtype=torch.int64))[None]
         Q, _, _ = synth.make_queries(self.w1, K, pos, seed=1)
         self.Q = Q[0].float().numpy()
-        self.geo = oracle.Geometry(w.head_dim, 4, 1, w.leaf_block, w.branching, w.k, w.window,
+        self.geo = oracle.Geometry(w.head_dim, G, 1, w.leaf_block, w.branching, w.k, w.window,
                                    rope=True, rope_base=w.rope_base)
         self.tree = oracle.LazyTree(self.K, self.V, r.double().numpy(), w.leaf_block,
                                     w.branching)
@@ -433,10 +453,10 @@ class OracleDecode:
         while done < n_heads:
             i = self.i % self.Q.shape[0]
             t = self.L + i - 1
-            h = done % 4
+            h = done % self.G
             self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree, self.geo)
             done += 1
-            if h == 3:
+            if h == self.G - 1:
                 self.i += 1
         return done
 
@@ -449,43 +469,46 @@ def _single_thread():
         return None
 
 
-def cpu_baseline(seconds=15.0):
+def cpu_baseline(workload=WORKLOAD, seconds=15.0):
     lim = _single_thread()
-    o = OracleDecode()
+    o = OracleDecode(workload)
     t0 = time.perf_counter()
     heads = 0
     while time.perf_counter() - t0 < seconds:
-        heads += o.query_heads(4)
+        heads += o.query_heads(o.G)
     dt = time.perf_counter() - t0
     del lim
     return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
             "kind": "oracle",
-            "sample": f"{heads} query-heads (decode at t=L, one KV head's tree, G=4) in "
-                      f"{dt:.1f} s; queries/s = query-heads/32/s; tree pooling untimed"}
+            "sample": f"{heads} query-heads (decode at t=L, one KV head's tree, G={o.G}) in "
+                      f"{dt:.1f} s; queries/s = query-heads/{o.heads_per_query}/s; tree pooling "
+                      "untimed"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return None
     lim = _single_thread()
-    o = OracleDecode()
+    o = OracleDecode(args.workload)
     for _ in range(args.warmup):
-        o.query_heads(4)
+        o.query_heads(o.G)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        o.query_heads(4)
+        o.query_heads(o.G)
     dt = time.perf_counter() - t0
     del lim
-    value = args.steps * 4 / o.heads_per_query / dt
-    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
+    value = args.steps * o.G / o.heads_per_query / dt
+    return {"impl": "reference", "metric": metric_for(args.workload, o.L), "value": value,
+            "unit": "queries/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic, seeded",
-            "config": {"workload": WORKLOAD, "L": o.L, "step": "4 query heads of one decode "
-                       "query (one KV head's tree)", "parallelism": "rank 0 only"},
+            "config": {"workload": args.workload, "L": o.L,
+                       "step": f"{o.G} query heads of one decode query (one KV head's tree)",
+                       "parallelism": "rank 0 only"},
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{args.steps} steps x 4 query heads; "
-                                       "queries/s = query-heads/32/s"},
+                             "sample": f"{args.steps} steps x {o.G} query heads; queries/s = "
+                                       f"query-heads/{o.heads_per_query}/s"},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -496,6 +519,8 @@ def main():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="recsa", choices=["recsa", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS),
+                    help="workload shape (the default is the headline 524K layer)")
     ap.add_argument("--prefill-reps", type=int, default=1)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-window-ws", action="store_true",

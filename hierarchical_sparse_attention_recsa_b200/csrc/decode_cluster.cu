@@ -34,6 +34,7 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 3;
 constexpr int kWinUnroll = 1;
+constexpr int kTokUnroll = 3;
 
 enum ItemKind { kKey = 0, kVal = 1, kNone = 2 };
 
@@ -174,7 +175,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int widx0 = nleaf * p.B + w_lo;
     const int gslot = warp * SPW + lane / LPR;
     for (int base = 0; base < nw; base += NSLOT * kWinUnroll) {
-      RawPairs rk[kWinUnroll], rv[kWinUnroll];
+      TokRow<T, HALF> rk[kWinUnroll], rv[kWinUnroll];
       float cs[kWinUnroll][8];
       bool on[kWinUnroll];
 #pragma unroll
@@ -183,16 +184,16 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         on[u] = e < nw;
         if (on[u]) {
           const int pos = win0 + e;
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
+          rk[u].load(K + (kvbase + pos) * D, j0);
+          rv[u].load(V + (kvbase + pos) * D, j0);
           if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
       for (int u = 0; u < kWinUnroll; ++u) {
         float xk[8], xv[8];
-        RawLoad<T, HALF>::cvt(rk[u], xk);
-        RawLoad<T, HALF>::cvt(rv[u], xv);
+        rk[u].cvt(xk);
+        rv[u].cvt(xv);
         if (p.rope) rotate8(xk, cs[u]);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -334,27 +335,27 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int nt = t_hi - t_lo;
     const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
     const float* qt = qtok + hw * D;
-    for (int base = 0; base < nt; base += HSLOT * kUnroll) {
-      RawPairs rk[kUnroll], rv[kUnroll];
-      float cs[kUnroll][8];
-      bool on[kUnroll];
+    for (int base = 0; base < nt; base += HSLOT * kTokUnroll) {
+      TokRow<T, HALF> rk[kTokUnroll], rv[kTokUnroll];
+      float cs[kTokUnroll][8];
+      bool on[kTokUnroll];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kTokUnroll; ++u) {
         const int e = base + u * HSLOT + hs;
         on[u] = e < nt;
         if (on[u]) {
           const int r = t_lo + e;
           const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
+          rk[u].load(K + (kvbase + pos) * D, j0);
+          rv[u].load(V + (kvbase + pos) * D, j0);
           if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kTokUnroll; ++u) {
         float xk[8], xv[8], s = 0.f;
-        RawLoad<T, HALF>::cvt(rk[u], xk);
-        RawLoad<T, HALF>::cvt(rv[u], xv);
+        rk[u].cvt(xk);
+        rv[u].cvt(xv);
         if (p.rope) rotate8(xk, cs[u]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -380,28 +381,28 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     float* scl = sc + par * G * cmax;
     unsigned char* fl = kfl + par * G * cmax;
     int* kp = kept + par * G * kmax;
+    // Rank of every candidate among its head's c scores (strictly greater
+    // scores, then equal scores at a lower index), by the head's 32 * WPH
+    // threads in parallel; kept iff rank < kap.
+    {
+      const int h = hw, tl = (warp % WPH) * 32 + lane;
+      const float* row = scl + h * cmax;
+      for (int i = tl; i < c; i += 32 * WPH) {
+        int r = 0;
+        if (kap < c) {
+          const float si = row[i];
+#pragma unroll 4
+          for (int j = 0; j < c; ++j) {
+            const float sj = row[j];
+            r += (sj > si) | ((sj == si) & (j < i));
+          }
+        }
+        fl[h * cmax + i] = r < kap;
+      }
+    }
+    __syncthreads();
     if (warp < G) {
       const int h = warp;
-      for (int i = lane; i < c; i += 32) fl[h * cmax + i] = (kap >= c) ? 1 : 0;
-      __syncwarp();
-      if (kap < c) {
-        unsigned taken = 0;
-        const int nj = (c + 31) / 32;
-        for (int it = 0; it < kap; ++it) {
-          unsigned bk = 0, bi = 0xffffffffu;
-          for (int jj = 0; jj < nj; ++jj) {
-            const int i = lane + 32 * jj;
-            if (i < c && !((taken >> jj) & 1u)) {
-              const unsigned key = order_key(scl[h * cmax + i]);
-              if (key > bk) { bk = key; bi = unsigned(i); }
-            }
-          }
-          const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
-          const unsigned wi = __reduce_min_sync(0xffffffffu, bk == wk ? bi : 0xffffffffu);
-          if (lane == int(wi & 31u)) taken |= 1u << (wi >> 5);
-          if (lane == 0) fl[h * cmax + wi] = 1;
-        }
-      }
       __syncwarp();
       int cnt = 0;
       for (int j = 0; j < c; j += 32) {

@@ -4,8 +4,8 @@
 // Some callers cannot hand the library any device memory beyond the tensors
 // of the call: a runtime whose device memory is entirely planned ahead and
 // owned by its own arena, or a plain C host that has no device allocator on
-// its call path.  For them this entry point keeps the window partials (max,
-// sum per query head) in a file-scope device array of kStaticEntries float2
+// its call path.  For them this entry point keeps the window partials (an fp32
+// row of head_dim + 2 per query head) in a file-scope device array of kStaticFloats floats
 // (4 MiB), which every GPU that loads the library holds until the process
 // exits.  Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
@@ -15,10 +15,10 @@
 namespace recsa {
 namespace {
 
-// batch * n_q * n_q_heads must not exceed this (4 MiB of float2).
-constexpr size_t kStaticEntries = size_t(1) << 19;
+// batch * n_q * n_q_heads * (head_dim + 2) must not exceed this (4 MiB of fp32).
+constexpr size_t kStaticFloats = size_t(1) << 20;
 
-__device__ __align__(256) float2 g_prefill_scratch[kStaticEntries];
+__device__ __align__(256) float g_prefill_scratch[kStaticFloats];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
@@ -44,7 +44,7 @@ cudaError_t scratch_address(void** out) {
 
 }  // namespace
 
-size_t prefill_static_max_entries() { return kStaticEntries; }
+size_t prefill_static_bytes() { return kStaticFloats * sizeof(float); }
 
 cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, int64_t q_start, int32_t n_q, void* O,
@@ -52,9 +52,9 @@ cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K,
   void* ml = nullptr;
   cudaError_t e = scratch_address(&ml);
   if (e != cudaSuccess) return e;
-  // The window kernel writes every (max, sum) entry of the range before the
-  // tree kernel reads it, so the array needs no clearing between calls.
-  e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, O, ml, s);
+  // The window kernel writes every partial row of the range before the tree
+  // kernel reads it, so the array needs no clearing between calls.
+  e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, ml, s);
   const void* wml = ml;
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();

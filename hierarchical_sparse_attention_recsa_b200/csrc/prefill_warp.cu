@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
 prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                     const T* __restrict__ V, const void* __restrict__ tree, int64_t q_start,
                     int n_q, T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
-                    int warp_bytes, const float2* __restrict__ wml) {
+                    int warp_bytes, const float* __restrict__ wpart) {
   constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR;
   const int G = p.group;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -284,9 +284,9 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     __syncwarp();
   };
 
-  // With window partials from the tensor-core window kernel (wml != null) the
-  // window rows are skipped here and merged at the end.
-  const bool own_window = wml == nullptr;
+  // With window partials from the tensor-core window kernel (wpart != null)
+  // the window rows are skipped here and merged at the end.
+  const bool own_window = wpart == nullptr;
   if (top > 0) {
     rotate_q(qlev, cnt_c[top]);
     run_pass(own_window, top, 0, false);
@@ -326,16 +326,17 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         store_elem(O, qrow + HALF + j0 + c, acc[4 + c] * il, p.dtype);
       }
     } else {
-      // merge with the window's partial softmax: O holds its normalised output
-      const float2 w = wml[(seq * n_q + qi) * p.hq + h];
+      // merge with the window's partial softmax (normalised output, max, sum)
+      const float* wrow = wpart + ((seq * n_q + qi) * p.hq + h) * (D + 2);
+      const float2 w = *reinterpret_cast<const float2*>(wrow + D);
       const float mm = fmaxf(m, w.x);
       const float ra_ = (m == -INFINITY) ? 0.f : __expf(m - mm);
       const float rb_ = (w.x == -INFINITY) ? 0.f : __expf(w.x - mm) * w.y;
       const float il = 1.f / (l * ra_ + rb_);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float o1 = load_elem(O, qrow + j0 + c, p.dtype);
-        const float o2 = load_elem(O, qrow + HALF + j0 + c, p.dtype);
+        const float o1 = wrow[j0 + c];
+        const float o2 = wrow[HALF + j0 + c];
         store_elem(O, qrow + j0 + c, (acc[c] * ra_ + o1 * rb_) * il, p.dtype);
         store_elem(O, qrow + HALF + j0 + c, (acc[4 + c] * ra_ + o2 * rb_) * il, p.dtype);
       }
@@ -361,7 +362,7 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 template <typename T, int D>
 cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const void* V,
                           const void* tree, int64_t q_start, int32_t n_q, void* O, int32_t* trace,
-                          const void* wml, cudaStream_t s) {
+                          const void* wpart, cudaStream_t s) {
   const int64_t kk = p.k < p.cap ? p.k : p.cap;
   int64_t maxn = 1;
   for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
@@ -385,7 +386,7 @@ cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const v
                                       reinterpret_cast<const T*>(K),
                                       reinterpret_cast<const T*>(V), tree, q_start, n_q,
                                       reinterpret_cast<T*>(O), trace, cmax, kmax, warp_bytes,
-                                      reinterpret_cast<const float2*>(wml));
+                                      reinterpret_cast<const float*>(wpart));
   return cudaGetLastError();
 }
 
@@ -393,12 +394,12 @@ cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const v
 
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
-                                int32_t* trace, const void* wml, cudaStream_t s) {
+                                int32_t* trace, const void* wpart, cudaStream_t s) {
   if (p.dtype == RECSA_DTYPE_BF16)
-    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s)
-                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s);
-  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s)
-                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s);
+    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s)
+                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);
+  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s)
+                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);
 }
 
 }  // namespace recsa

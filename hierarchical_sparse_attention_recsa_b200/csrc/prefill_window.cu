@@ -15,9 +15,9 @@
 // with mma.sync m16n8k16 (fp32 accumulation): S = Q K^T, masked to each row's
 // band, online softmax in registers (FlashAttention-2 register reuse of S as
 // the A operand of P V), then O = P V.  The result is this window's partial
-// softmax: the normalised output is written to O (dtype) and (max, sum) per
-// (query, head) to a caller workspace; the tree kernel folds the summaries
-// and kept leaves into it.  Work per CTA is ~20 MFLOP against ~0.3 MB of
+// softmax: per (query, head) a row of the caller workspace receives the
+// normalised output, the max and the sum in fp32; the tree kernel folds the
+// summaries and kept leaves into it and writes O once.  Work per CTA is ~20 MFLOP against ~0.3 MB of
 // K/V reads, so the kernel is far from both rooflines; the tree part of the
 // prefill dominates.
 #include <cuda_fp16.h>
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kWThreads, 3)
 window_mma_kernel(Params p, const __nv_bfloat16* __restrict__ Q,
                   const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
                   const void* __restrict__ tree, int64_t q_start, int n_q,
-                  __nv_bfloat16* __restrict__ O, float2* __restrict__ ml) {
+                  float* __restrict__ part) {
   constexpr int HALF = D / 2, QP = D + 8, VP = kChunk + 8;
   const int G = p.group, QB = kRows / G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -234,26 +234,24 @@ window_mma_kernel(Params p, const __nv_bfloat16* __restrict__ Q,
     }
   }
 
-  // normalised window output -> O, (max, sum) -> ml
+  // partial row per (query, head), fp32: normalised window output [D], max, sum
   const int hA = rowA % G, hB = rowB % G;
   const float iA = lA > 0.f ? 1.f / lA : 0.f, iB = lB > 0.f ? 1.f / lB : 0.f;
   if (qqA < nqh) {
-    const int64_t rec = (seq * n_q + q0 + qqA) * p.hq + int64_t(g) * G + hA;
+    float* row = part + ((seq * n_q + q0 + qqA) * p.hq + int64_t(g) * G + hA) * (D + 2);
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      __nv_bfloat162 v = __floats2bfloat162_rn(oacc[nt][0] * iA, oacc[nt][1] * iA);
-      *reinterpret_cast<__nv_bfloat162*>(O + rec * D + nt * 8 + tig * 2) = v;
-    }
-    if (tig == 0) ml[rec] = make_float2(mA, lA);
+    for (int nt = 0; nt < D / 8; ++nt)
+      *reinterpret_cast<float2*>(row + nt * 8 + tig * 2) =
+          make_float2(oacc[nt][0] * iA, oacc[nt][1] * iA);
+    if (tig == 0) *reinterpret_cast<float2*>(row + D) = make_float2(mA, lA);
   }
   if (qqB < nqh) {
-    const int64_t rec = (seq * n_q + q0 + qqB) * p.hq + int64_t(g) * G + hB;
+    float* row = part + ((seq * n_q + q0 + qqB) * p.hq + int64_t(g) * G + hB) * (D + 2);
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-      __nv_bfloat162 v = __floats2bfloat162_rn(oacc[nt][2] * iB, oacc[nt][3] * iB);
-      *reinterpret_cast<__nv_bfloat162*>(O + rec * D + nt * 8 + tig * 2) = v;
-    }
-    if (tig == 0) ml[rec] = make_float2(mB, lB);
+    for (int nt = 0; nt < D / 8; ++nt)
+      *reinterpret_cast<float2*>(row + nt * 8 + tig * 2) =
+          make_float2(oacc[nt][2] * iB, oacc[nt][3] * iB);
+    if (tig == 0) *reinterpret_cast<float2*>(row + D) = make_float2(mB, lB);
   }
 }
 
@@ -263,8 +261,8 @@ window_mma_kernel(Params p, const __nv_bfloat16* __restrict__ Q,
 // geometry is outside this kernel's limits (bf16 only; the RoPE table must
 // reach W + B + 64/G indices).
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,
-                                  const void* tree, int64_t q_start, int32_t n_q, void* O,
-                                  void* ml, cudaStream_t s) {
+                                  const void* tree, int64_t q_start, int32_t n_q, void* part,
+                                  cudaStream_t s) {
   if (p.dtype != RECSA_DTYPE_BF16) return cudaErrorNotSupported;
   if (p.group < 1 || kRows % p.group) return cudaErrorNotSupported;
   const int QB = kRows / p.group;
@@ -281,14 +279,14 @@ cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K,
     if (e != cudaSuccess) return e;
     kern<<<grid, kWThreads, bytes, s>>>(p, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                         (const __nv_bfloat16*)V, tree, q_start, n_q,
-                                        (__nv_bfloat16*)O, (float2*)ml);
+                                        (float*)part);
   } else {
     auto kern = window_mma_kernel<64>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
     if (e != cudaSuccess) return e;
     kern<<<grid, kWThreads, bytes, s>>>(p, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                         (const __nv_bfloat16*)V, tree, q_start, n_q,
-                                        (__nv_bfloat16*)O, (float2*)ml);
+                                        (float*)part);
   }
   return cudaGetLastError();
 }

@@ -99,10 +99,15 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   return RECSA_OK;
 }
 
-// Window partials (max, sum) as float2 per (sequence, query, head).
-size_t prefill_workspace_need(const Params& p, int32_t n_q) {
-  return size_t(p.batch) * size_t(n_q) * size_t(p.hq) * sizeof(float2);
+}  // namespace
+
+// Window partials: per (sequence, query, head) an fp32 row of d + 2 (the
+// window's normalised output, its max and its sum).
+size_t recsa::prefill_workspace_need(const Params& p, int32_t n_q) {
+  return size_t(p.batch) * size_t(n_q) * size_t(p.hq) * size_t(p.d + 2) * sizeof(float);
 }
+
+namespace {
 
 recsa_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return RECSA_OK;
@@ -219,14 +224,14 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   if (decode && !getenv("RECSA_DECODE_GENERIC"))
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
   if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
-    const void* wml = nullptr;
+    const void* wpart = nullptr;
     if (workspace) {
-      e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, O, workspace, s);
-      if (e == cudaSuccess) wml = workspace;
+      e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, workspace, s);
+      if (e == cudaSuccess) wpart = workspace;
       else if (e != cudaErrorNotSupported) return cuda_status(e);
       else cudaGetLastError();
     }
-    e = launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, wml, s);
+    e = launch_prefill_warp(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);
   }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
@@ -256,13 +261,12 @@ recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, con
       !aligned(tree, 256) || (trace && !aligned(trace, 4)))
     return RECSA_ERR_MISALIGNED;
   if (n_q < 0 || q_start < 0 || q_start + n_q > geom->capacity) return RECSA_ERR_CAPACITY;
-  if (size_t(geom->batch) * size_t(n_q) * size_t(geom->n_q_heads) >
-      prefill_static_max_entries()) {
+  if (prefill_workspace_need(p, n_q) > prefill_static_bytes()) {
     fprintf(stderr,
-            "recsa_prefill_static: batch * n_q * n_q_heads = %zu exceeds the fixed scratch of "
-            "%zu query heads; split the call into smaller query ranges\n",
-            size_t(geom->batch) * size_t(n_q) * size_t(geom->n_q_heads),
-            prefill_static_max_entries());
+            "recsa_prefill_static: %zu bytes of window partials (batch * n_q * n_q_heads * "
+            "(head_dim + 2) * 4) exceed the fixed scratch of %zu bytes; split the call into "
+            "smaller query ranges\n",
+            prefill_workspace_need(p, n_q), prefill_static_bytes());
     return RECSA_ERR_CAPACITY;
   }
   if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;

@@ -98,21 +98,24 @@ cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);
 // Warp-per-(query, head) prefill kernel; cudaErrorNotSupported outside its limits.
-// wml: window partials (max, sum) per (sequence, query, head) from
-// launch_prefill_window, or null to let this kernel attend the window itself.
+// wpart: window partials from launch_prefill_window (fp32 rows of d + 2 per
+// (sequence, query, head): normalised output, max, sum), or null to let this
+// kernel attend the window itself.
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
-                                int32_t* trace, const void* wml, cudaStream_t s);
+                                int32_t* trace, const void* wpart, cudaStream_t s);
 // Prefill with the window partials kept in a fixed device array (no caller
-// workspace); prefill_static_max_entries() bounds batch * n_q * n_q_heads.
+// workspace) of prefill_static_bytes() bytes.
 cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, int64_t q_start, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);
-size_t prefill_static_max_entries();
-// Tensor-core window partials for a prefill range (bf16): normalised window
-// output into O, (max, sum) into ml; cudaErrorNotSupported outside its limits.
+size_t prefill_static_bytes();
+// Bytes of window partials for n_q queries per sequence (fp32 rows of d + 2).
+size_t prefill_workspace_need(const Params& p, int32_t n_q);
+// Tensor-core window partials for a prefill range (bf16) into part (fp32
+// rows of d + 2); cudaErrorNotSupported outside its limits.
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,
-                                  const void* tree, int64_t q_start, int32_t n_q, void* O,
-                                  void* ml, cudaStream_t s);
+                                  const void* tree, int64_t q_start, int32_t n_q, void* part,
+                                  cudaStream_t s);
 
 }  // namespace recsa

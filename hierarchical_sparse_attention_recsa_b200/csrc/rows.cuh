@@ -108,3 +108,39 @@ struct RawLoad<__nv_bfloat16, HALF> {
 };
 
 }  // namespace recsa
+
+namespace recsa {
+
+// Raw bytes of a lane's four pairs of a bf16 row (half the registers of
+// RawPairs); loaded first, converted after the whole batch is in flight.
+struct RawBf {
+  uint2 a, b;
+};
+template <int HALF>
+__device__ __forceinline__ void raw_load_bf(const __nv_bfloat16* row, int j0, RawBf& r) {
+  r.a = __ldg(reinterpret_cast<const uint2*>(row + j0));
+  r.b = __ldg(reinterpret_cast<const uint2*>(row + HALF + j0));
+}
+__device__ __forceinline__ void raw_cvt_bf(const RawBf& r, float* x) {
+  x[0] = __uint_as_float(r.a.x << 16); x[1] = __uint_as_float(r.a.x & 0xffff0000u);
+  x[2] = __uint_as_float(r.a.y << 16); x[3] = __uint_as_float(r.a.y & 0xffff0000u);
+  x[4] = __uint_as_float(r.b.x << 16); x[5] = __uint_as_float(r.b.x & 0xffff0000u);
+  x[6] = __uint_as_float(r.b.y << 16); x[7] = __uint_as_float(r.b.y & 0xffff0000u);
+}
+// Token-row loader for either dtype: bf16 rows use RawBf, fp32 rows RawPairs.
+template <typename T, int HALF>
+struct TokRow {
+  RawPairs r;
+  __device__ __forceinline__ void load(const T* row, int j0) { RawLoad<T, HALF>::load(row, j0, r); }
+  __device__ __forceinline__ void cvt(float* x) const { RawLoad<T, HALF>::cvt(r, x); }
+};
+template <int HALF>
+struct TokRow<__nv_bfloat16, HALF> {
+  RawBf r;
+  __device__ __forceinline__ void load(const __nv_bfloat16* row, int j0) {
+    raw_load_bf<HALF>(row, j0, r);
+  }
+  __device__ __forceinline__ void cvt(float* x) const { raw_cvt_bf(r, x); }
+};
+
+}  // namespace recsa

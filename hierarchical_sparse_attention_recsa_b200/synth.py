@@ -80,18 +80,25 @@ def make_kv(w: Workload, capacity: int, seed: int = 0, device="cpu",
     """
     batch = w.batch if batch is None else batch
     g = _gen(seed, device)
-    shape = (batch, w.n_kv_heads, capacity, w.head_dim)
-    K = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
-    V = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    sk = sv = None
     if w.channel_scale:
         sk = torch.exp(0.5 * torch.randn((w.n_kv_heads, w.head_dim), generator=g,
                                          device=device))
         sv = torch.exp(0.5 * torch.randn((w.n_kv_heads, w.head_dim), generator=g,
                                          device=device))
-        K.mul_(sk[None, :, None, :])
-        V.mul_(sv[None, :, None, :])
     r = torch.randn((w.head_dim,), generator=g, device=device) / (w.head_dim ** 0.5)
-    return K.to(w.dtype), V.to(w.dtype), r.float()
+    shape = (batch, w.n_kv_heads, capacity, w.head_dim)
+    K = torch.empty(shape, dtype=w.dtype, device=device)
+    V = torch.empty(shape, dtype=w.dtype, device=device)
+    # one sequence at a time in fp32, so the peak memory is one sequence's worth
+    for s in range(batch):
+        for dst, scale in ((K, sk), (V, sv)):
+            x = torch.randn(shape[1:], generator=g, device=device, dtype=torch.float32)
+            if scale is not None:
+                x.mul_(scale[:, None, :])
+            dst[s].copy_(x)
+            del x
+    return K, V, r.float()
 
 
 def make_queries(w: Workload, K: torch.Tensor, positions: torch.Tensor, seed: int = 1,

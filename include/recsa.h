@@ -12,7 +12,8 @@
  *
  * Conventions for every entry point:
  *   - All tensors are caller-owned device memory; the library allocates
- *     nothing and keeps no global state.  Pointers to K, V, Q, O, k_new, v_new
+ *     nothing, and its only global state is the fixed scratch array of
+ *     recsa_prefill_static.  Pointers to K, V, Q, O, k_new, v_new
  *     must be 16-byte aligned, the tree 256-byte aligned.
  *   - Layouts are row-major:
  *       K, V          [batch][n_kv_heads][capacity][head_dim]   (dtype)
@@ -157,9 +158,11 @@ recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void*
  *   workspace: NULL, or DEVICE memory of at least
  *   recsa_prefill_workspace_bytes(geom, n_q) bytes (16-byte aligned) given as
  *   workspace_bytes.  With a workspace and bf16 data the exact window runs on
- *   the tensor cores and its partial softmax (max, sum per query head) is kept
- *   there until the tree kernel merges it; without one, the window is attended
- *   by the tree kernel itself.  Both give the same result within rounding.
+ *   the tensor cores and its partial softmax (per query head an fp32 row of
+ *   head_dim + 2: the window's normalised output, max and sum) is kept there
+ *   until the tree kernel merges it and writes O once; without one, the window
+ *   is attended by the tree kernel itself.  Both give the same result within
+ *   rounding.
  *   The workspace is only read and written by this call; calls that share one
  *   must not overlap on the device.
  */
@@ -174,10 +177,12 @@ recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void
  * device memory is planned ahead and owned by its own arena, or a C host with
  * no device allocator on its call path.  (The pages have no counterpart: it
  * is a packaging variant of recsa_prefill, same arguments and result.)
- *   Scratch: the window partials live in a fixed device array of 2^19 query
- *   heads (4 MiB), which every GPU that loads the library holds until the
- *   process exits.  batch * n_q * n_q_heads above 2^19 is rejected with
- *   RECSA_ERR_CAPACITY (and a message on stderr): split the query range.
+ *   Scratch: the window partials live in a fixed 4 MiB device array, which
+ *   every GPU that loads the library holds until the process exits.  A call
+ *   needs batch * n_q * n_q_heads * (head_dim + 2) * 4 bytes of it (8065 query
+ *   heads at head_dim 128, e.g. 252 queries of 32 heads); a larger call is
+ *   rejected with RECSA_ERR_CAPACITY (and a message on stderr): split the
+ *   query range.
  *   The array needs no clearing (each call writes what it reads), but every
  *   call shares it: calls that overlap on the device race.
  *   Set-up: the first call on each device, with that device current, looks up

@@ -106,7 +106,7 @@ def test_tree_bytes(lib, kw):
 
 def test_prefill_workspace_bytes(lib):
     g = geo(batch=2, capacity=4096)
-    assert R.recsa_prefill_workspace_bytes(g, 100) == 2 * 100 * 32 * 8
+    assert R.recsa_prefill_workspace_bytes(g, 100) == 2 * 100 * 32 * (128 + 2) * 4
 
 
 def test_trace_ints(lib):

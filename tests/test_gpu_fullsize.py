@@ -1,0 +1,188 @@
+"""Parity at the workloads' full sizes, on sampled outputs the oracle computes
+one by one (its tree is built lazily from each sampled head's cache).
+
+* 524K (32q/8kv, d=128, B64 b16 k8 W512, 4 levels): decode at batch 4 after an
+  append, in the launch configuration the benchmark times (cluster size
+  chosen automatically); full causal prefill of one sequence in 64K-query
+  chunks with the tensor-core window workspace, as the benchmark runs it.
+* 131K: decode (3 levels).
+* 1M (b32, 3 levels): decode with needle and mixture queries.
+* 2M (B32 b8 k16 W1024, 6 levels): decode, and the 65536-query chunked
+  prefill at the end of the context; entries read per query are checked
+  against the closed form from the selection trace.
+
+Tolerances and the selection rule are those of recsa_testlib.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
+from hierarchical_sparse_attention_recsa_b200 import recsa as R
+
+from recsa_testlib import Stats, alloc_tree, check_query, geometry, oracle_geometry, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build_lib.build()
+    R.lib()
+
+
+def _host_head(K, V, s, g, n):
+    return (K[s, g, :n].float().cpu().numpy(), V[s, g, :n].float().cpu().numpy())
+
+
+def _decode_case(wname, batch, appended=1, samples=((0, 0), (0, 13), (0, 31)), seed=0):
+    w = synth.WORKLOADS[wname]
+    L = w.length
+    cap = L + 64
+    g = geometry(w, cap, batch)
+    K, V, r = synth.make_kv(w, cap, seed=seed, device="cuda", batch=batch)
+    tree = alloc_tree(g)
+    R.recsa_build(g, K, V, [L] * batch, r, 0, tree)
+    lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
+    for i in range(appended):      # the step the benchmark times: append, then decode
+        kn = K[:, :, L + i].contiguous()
+        vn = V[:, :, L + i].contiguous()
+        R.recsa_append(g, K, V, kn, vn, lens, r, 0, tree)
+    n = L + appended
+    pos = torch.full((batch, 1), n - 1, dtype=torch.int64, device="cuda")
+    Q, kind, _ = synth.make_queries(w, K, pos, seed=seed + 1, n_needles=None)
+    O = torch.empty_like(Q)
+    trace = torch.zeros((batch, 1, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    R.recsa_decode(g, Q, K, V, tree, lens, 1, O, trace)
+    torch.cuda.synchronize()
+    assert lens.cpu().tolist() == [n] * batch
+    og = oracle_geometry(g)
+    G = g.n_q_heads // g.n_kv_heads
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    heads = {}
+    for s, h in samples:
+        kv = h // G
+        if (s, kv) not in heads:
+            Kh, Vh = _host_head(K, V, s, kv, n)
+            heads[(s, kv)] = (Kh, Vh, oracle.LazyTree(Kh, Vh, r.double().cpu().numpy(),
+                                                       g.leaf_block, g.branching))
+        Kh, Vh, src = heads[(s, kv)]
+        check_query(st, O_[s, 0, h], tr[s, 0, h], to_np(Q[s, 0, h]), n - 1, Kh, Vh, src, og, g.k)
+    st.check(w.dtype, f"decode {wname}")
+    return st
+
+
+def test_decode_524k_batch4_bench_config():
+    _decode_case("qwen3-4b-524k", 4, samples=((0, 0), (1, 9), (2, 18), (3, 31), (3, 30)))
+
+
+def test_decode_131k():
+    _decode_case("qwen3-4b-131k", 1, samples=((0, 0), (0, 7), (0, 22)), seed=3)
+
+
+def test_decode_1m_needles_and_mixtures():
+    _decode_case("decode-1m", 1, samples=((0, 0), (0, 3), (0, 17)), seed=5)
+
+
+def test_decode_2m_six_levels():
+    st = _decode_case("stress-2m", 1, samples=((0, 0), (0, 12)), seed=7)
+    assert st.clear + st.near_tie == 2
+
+
+def test_prefill_524k_bench_config():
+    """Full causal prefill of one 524K sequence in 64K-query chunks with the
+    window workspace, as the benchmark runs it; sampled outputs checked."""
+    w = synth.WORKLOADS["qwen3-4b-524k"]
+    L = w.length
+    g = geometry(w, L, 1)
+    K, V, r = synth.make_kv(w, L, seed=11, device="cuda", batch=1)
+    tree = alloc_tree(g)
+    R.recsa_build(g, K, V, [L], r, 0, tree)
+    chunk = 65536
+    ws = torch.empty(R.recsa_prefill_workspace_bytes(g, chunk), dtype=torch.uint8, device="cuda")
+    rng = np.random.default_rng(0)
+    sample_t = sorted(set([0, 511, 512, 575, 576, 4095, 65535, 65536, L - 1] +
+                          list(rng.integers(0, L, 7))))
+    picked = {}
+    for c0 in range(0, L, chunk):
+        pos = (c0 + torch.arange(chunk, device="cuda", dtype=torch.int64))[None]
+        Q, _, _ = synth.make_queries(w, K, pos, seed=40 + c0 // chunk)
+        O = torch.empty_like(Q)
+        R.recsa_prefill(g, Q, K, V, tree, c0, chunk, O, workspace=ws)
+        for t in sample_t:
+            if c0 <= t < c0 + chunk:
+                picked[t] = (Q[0, t - c0].float().cpu().numpy(), O[0, t - c0].float().cpu().numpy())
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    G = g.n_q_heads // g.n_kv_heads
+    st = Stats()
+    for kv in (0, 5):
+        Kh, Vh = _host_head(K, V, 0, kv, L)
+        src = oracle.LazyTree(Kh, Vh, r.double().cpu().numpy(), g.leaf_block, g.branching)
+        for t, (q, o) in picked.items():
+            for h in (kv * G, kv * G + G - 1):
+                res = oracle.traverse_and_attend(q[h].astype(np.float64), t, Kh, Vh, src, og)
+                # no trace here: near-tie queries would need the GPU selection,
+                # so keep the ones with clear gaps (the rest are counted)
+                from recsa_testlib import gaps_clear
+                if gaps_clear(res, g.k):
+                    st.clear += 1
+                    st.add(o[h], res["out"])
+                else:
+                    st.near_tie += 1
+    st.check(w.dtype, "prefill 524K")
+    assert st.clear >= 0.6 * (st.clear + st.near_tie)
+
+
+def test_prefill_2m_last_64k_chunk_and_counts():
+    """The 65536-query chunked prefill at the end of the 2M context; entries
+    read per query (from the trace of a traced sub-range) equal the closed form
+    and stay within the O(log L) bound."""
+    w = synth.WORKLOADS["stress-2m"]
+    L = w.length
+    nq = w.extra["prefill_queries"]
+    q0 = L - nq
+    g = geometry(w, L, 1)
+    K, V, r = synth.make_kv(w, L, seed=13, device="cuda", batch=1)
+    tree = alloc_tree(g)
+    R.recsa_build(g, K, V, [L], r, 0, tree)
+    pos = (q0 + torch.arange(nq, device="cuda", dtype=torch.int64))[None]
+    Q, _, _ = synth.make_queries(w, K, pos, seed=14)
+    O = torch.empty_like(Q)
+    ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8, device="cuda")
+    R.recsa_prefill(g, Q, K, V, tree, q0, nq, O, workspace=ws)
+    # traced sub-range at the very end (same kernels, smaller trace buffer)
+    nt = 256
+    trace = torch.zeros((1, nt, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    O2 = torch.empty_like(Q[:, -nt:])
+    R.recsa_prefill(g, Q[:, -nt:].contiguous(), K, V, tree, L - nt, nt, O2, trace,
+                    workspace=ws)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(O2.float(), O[:, -nt:].float(), rtol=0, atol=0)
+    og = oracle_geometry(g)
+    tr = trace.cpu().numpy()
+    levels = len(oracle.level_counts(L, g.leaf_block, g.branching))
+    bound = levels * (g.branching * g.k + g.branching - 1) + g.leaf_block * g.k + g.window + \
+        g.leaf_block - 1
+    for i in range(nt):
+        cf = oracle.closed_form_counts(L - nt + i, og)
+        for h in range(0, g.n_q_heads, 7):
+            rec = tr[0, i, h]
+            assert int(rec[1]) == cf["entries"] and int(rec[2]) == cf["keys_read"]
+            assert int(rec[1]) <= bound
+    # sampled outputs of the full chunk against the oracle, with the trace's selection
+    G = g.n_q_heads // g.n_kv_heads
+    Kh, Vh = _host_head(K, V, 0, 0, L)
+    src = oracle.LazyTree(Kh, Vh, r.double().cpu().numpy(), g.leaf_block, g.branching)
+    st = Stats()
+    O_ = to_np(O2)
+    for i in (0, 100, nt - 1):
+        for h in range(G):
+            check_query(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, nq - nt + i, h]), L - nt + i,
+                        Kh, Vh, src, og, g.k)
+    st.check(w.dtype, "prefill 2M")

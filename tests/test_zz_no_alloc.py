@@ -19,7 +19,7 @@ import torch
 from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
 from hierarchical_sparse_attention_recsa_b200 import recsa as R
 
-MAX_ENTRIES = 1 << 19          # query heads the fixed scratch holds
+SCRATCH_BYTES = 4 << 20        # bytes of the fixed scratch
 
 
 @pytest.fixture(scope="module")
@@ -40,7 +40,7 @@ def test_static_prefill_rejects_oversize_before_device_work(lib):
     _, g = _geom(batch=2, capacity=1 << 20)
     cg = g.c()
     ok = ctypes.c_void_p(1 << 20)            # aligned fake pointers: never dereferenced
-    n_q = MAX_ENTRIES // (2 * g.n_q_heads) + 1
+    n_q = SCRATCH_BYTES // (2 * g.n_q_heads * (g.head_dim + 2) * 4) + 1
     assert lib.recsa_prefill_static(ctypes.byref(cg), ok, ok, ok, ok, 0, n_q, ok, None,
                                     None) == 4
     # a NULL output is refused too
@@ -50,14 +50,15 @@ def test_static_prefill_rejects_oversize_before_device_work(lib):
 
 @pytest.mark.gpu
 def test_static_prefill_matches_workspace_prefill_on_two_calls(lib):
-    lens = [6000, 5000]
+    lens = [6000]
     cap = 6144
-    w, g = _geom(batch=2, capacity=cap)
-    K, V, r = synth.make_kv(w, cap, seed=21, device="cuda", batch=2)
+    w, g = _geom(batch=1, capacity=cap)
+    K, V, r = synth.make_kv(w, cap, seed=21, device="cuda", batch=1)
     tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
     R.recsa_build(g, K, V, lens, r, 0, tree)
-    for call, (q0, nq) in enumerate([(1000, 1500), (3000, 2000)]):
-        pos = (q0 + torch.arange(nq, device="cuda", dtype=torch.int64))[None].expand(2, nq)
+    # 252 queries x 32 heads x (128 + 2) fp32 is the largest range the scratch holds
+    for call, (q0, nq) in enumerate([(1000, 200), (5748, 252)]):
+        pos = (q0 + torch.arange(nq, device="cuda", dtype=torch.int64))[None].expand(1, nq)
         Q, _, _ = synth.make_queries(w, K, pos.contiguous(), seed=30 + call)
         ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8,
                          device="cuda")
