@@ -33,7 +33,6 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 3;
-constexpr int kWinUnroll = 1;
 constexpr int kTokUnroll = 3;
 
 enum ItemKind { kKey = 0, kVal = 1, kNone = 2 };
@@ -43,7 +42,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                       const T* __restrict__ V, const void* __restrict__ tree,
                       const int64_t* __restrict__ len_dev, int n_q, T* __restrict__ O,
-                      int32_t* __restrict__ trace, int cmax, int kmax) {
+                      int32_t* __restrict__ trace, int cmax, int kmax, int wrows) {
   constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR, NSLOT = kWarps * SPW;
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = int(cluster.num_blocks());
@@ -52,7 +51,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int64_t seq = blockIdx.z / p.hkv;
   const int g = int(blockIdx.z % p.hkv);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int sub = lane % LPR, slot = warp * SPW + lane / LPR;
+  const int sub = lane % LPR;
   const int j0 = 4 * sub;
 
   extern __shared__ __align__(16) unsigned char smem[];
@@ -65,6 +64,13 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* mrg = wwin + kWarps * G * (D + 2);            // [CS][G][D + 2] cluster merge (rank 0)
   int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
   unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
+  // top-k finalists: [G][ceil(cmax / 32)][32] keys
+  const int nseg_max = (cmax + 31) / 32;
+  unsigned long long* finbuf = reinterpret_cast<unsigned long long*>(
+      (reinterpret_cast<uintptr_t>(kfl + 2 * G * cmax) + 15) & ~uintptr_t(15));
+  // window rows of this CTA staged by cp.async: K then V, [wrows][D] each
+  T* winK = reinterpret_cast<T*>(finbuf + size_t(G) * nseg_max * 32);
+  T* winV = winK + size_t(wrows) * D;
 
   const int64_t t = len_dev[seq] - 1;
   const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
@@ -171,30 +177,31 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       for (int c = 0; c < 8; ++c) accW[h][c] = 0.f;
     }
     const int nw = w_hi - w_lo;
-    const int win0 = int(a) * p.B + w_lo;
     const int widx0 = nleaf * p.B + w_lo;
     const int gslot = warp * SPW + lane / LPR;
-    for (int base = 0; base < nw; base += NSLOT * kWinUnroll) {
-      TokRow<T, HALF> rk[kWinUnroll], rv[kWinUnroll];
-      float cs[kWinUnroll][8];
-      bool on[kWinUnroll];
-#pragma unroll
-      for (int u = 0; u < kWinUnroll; ++u) {
-        const int e = base + u * NSLOT + gslot;
-        on[u] = e < nw;
-        if (on[u]) {
-          const int pos = win0 + e;
-          rk[u].load(K + (kvbase + pos) * D, j0);
-          rv[u].load(V + (kvbase + pos) * D, j0);
-          if (p.rope) load_cs(rope, widx0 + e, HALF, j0, cs[u]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kWinUnroll; ++u) {
+    // Rows come from the staged copy in shared memory; the slot's RoPE index
+    // grows by NSLOT per row, so its (cos, sin) advance by a fixed rotation.
+    float csc[8], cstep[8];
+    const int rmax = p.lay.rope_rows - 1;
+    const bool recur = NSLOT <= rmax;   // the step rotation is a table row
+    if (p.rope && recur) {
+      load_cs(rope, min(widx0 + gslot, rmax), HALF, j0, csc);
+      load_cs(rope, NSLOT, HALF, j0, cstep);
+    }
+    for (int base = 0; base < nw; base += NSLOT) {
+      {
+        const int e = base + gslot;
+        const bool on = e < nw;
         float xk[8], xv[8];
-        rk[u].cvt(xk);
-        rv[u].cvt(xv);
-        if (p.rope) rotate8(xk, cs[u]);
+        const int ee = on ? e : 0;
+        SharedPairs<T, HALF>::load(winK + size_t(ee) * D, j0, xk);
+        SharedPairs<T, HALF>::load(winV + size_t(ee) * D, j0, xv);
+        if (p.rope) {
+          if (!recur) load_cs(rope, min(widx0 + e, rmax), HALF, j0, csc);
+          rotate8(xk, csc);
+          if (recur) advance_cs(csc, cstep);
+        }
+        const bool on_u = on;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float* qv = qtok + h * D;
@@ -205,7 +212,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
             s = fmaf(qv[HALF + j0 + c], xk[4 + c], s);
           }
           s = slot_sum<LPR>(s) * inv_sqrt_d;
-          if (on[u]) {
+          if (on_u) {
             if (s > mW[h]) {
               const float r = __expf(mW[h] - s);
               lW[h] = lW[h] * r + 1.f;
@@ -276,10 +283,15 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const unsigned char* flV = kfl + (vlev & 1) * G * cmax + hw * cmax;
     float* scK = sc + (klev & 1) * G * cmax + hw * cmax;
     const float* ql = qlev + hw * D;
+    // key items step their RoPE index by HSLOT per slot: seeded once per batch
+    const int rmax = p.lay.rope_rows - 1;
+    float cstep[8];
+    if (p.rope) load_cs(rope, HSLOT, HALF, j0, cstep);
     for (int base = 0; base < total; base += HSLOT * kUnroll) {
       RawPairs ra[kUnroll];
-      float cs[kUnroll][8];
+      float csc[8];
       int kind[kUnroll], idx[kUnroll];
+      if (p.rope) load_cs(rope, min(k_lo + base + hs, rmax), HALF, j0, csc);
       float sv[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -293,7 +305,6 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
           kind[u] = kKey;
           idx[u] = i;
           RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
-          if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
         } else if (e < total) {
           const int i = v_lo + (e - nk);
           if (!flV[i]) {
@@ -308,8 +319,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       for (int u = 0; u < kUnroll; ++u) {
         float x[8], s = 0.f;
         RawLoad<float, HALF>::cvt(ra[u], x);
+        if (kind[u] == kKey && p.rope) rotate8(x, csc);
+        if (p.rope) advance_cs(csc, cstep);
         if (kind[u] == kKey) {
-          if (p.rope) rotate8(x, cs[u]);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             s = fmaf(ql[j0 + c], x[c], s);
@@ -335,10 +347,14 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int nt = t_hi - t_lo;
     const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
     const float* qt = qtok + hw * D;
+    const int rmax = p.lay.rope_rows - 1;
+    float cstep[8];
+    if (p.rope) load_cs(rope, HSLOT, HALF, j0, cstep);
     for (int base = 0; base < nt; base += HSLOT * kTokUnroll) {
       TokRow<T, HALF> rk[kTokUnroll], rv[kTokUnroll];
-      float cs[kTokUnroll][8];
+      float csc[8];
       bool on[kTokUnroll];
+      if (p.rope) load_cs(rope, min(t_lo + base + hs, rmax), HALF, j0, csc);
 #pragma unroll
       for (int u = 0; u < kTokUnroll; ++u) {
         const int e = base + u * HSLOT + hs;
@@ -348,7 +364,6 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
           const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
           rk[u].load(K + (kvbase + pos) * D, j0);
           rv[u].load(V + (kvbase + pos) * D, j0);
-          if (p.rope) load_cs(rope, r, HALF, j0, cs[u]);
         }
       }
 #pragma unroll
@@ -356,7 +371,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         float xk[8], xv[8], s = 0.f;
         rk[u].cvt(xk);
         rv[u].cvt(xv);
-        if (p.rope) rotate8(xk, cs[u]);
+        if (p.rope) {
+          rotate8(xk, csc);
+          advance_cs(csc, cstep);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           s = fmaf(qt[j0 + c], xk[c], s);
@@ -369,7 +387,11 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   };
 
   auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
-    if (w_hi > w_lo) window_loop(w_lo, w_hi);
+    if (w_hi > w_lo) {
+      cp_async_wait_all();
+      __syncthreads();
+      window_loop(w_lo, w_hi);
+    }
     if (klev > 0 || vlev > 0) tree_loop(klev, vlev);
     if (tokens) token_loop();
   };
@@ -381,23 +403,58 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     float* scl = sc + par * G * cmax;
     unsigned char* fl = kfl + par * G * cmax;
     int* kp = kept + par * G * kmax;
-    // Rank of every candidate among its head's c scores (strictly greater
-    // scores, then equal scores at a lower index), by the head's 32 * WPH
-    // threads in parallel; kept iff rank < kap.
+    // Selection, by the head's WPH warps: each 32-candidate segment is sorted
+    // by a warp bitonic network on (score, -index) keys, its best kap keys
+    // become finalists, and one warp ranks the finalists (a candidate is in
+    // the top kap iff it is in its segment's top kap).  Ties go to the lower
+    // index.  kap > 32 falls back to rank counting over all candidates.
     {
-      const int h = hw, tl = (warp % WPH) * 32 + lane;
+      const int h = hw, wl = warp % WPH, tl = wl * 32 + lane;
       const float* row = scl + h * cmax;
-      for (int i = tl; i < c; i += 32 * WPH) {
-        int r = 0;
-        if (kap < c) {
+      for (int i = tl; i < c; i += 32 * WPH) fl[h * cmax + i] = kap >= c;
+      const int nseg = (c + 31) / 32;
+      unsigned long long* fin = finbuf + size_t(h) * nseg_max * 32;
+      if (kap < c && kap <= 32) {
+        for (int m = wl; m < nseg; m += WPH) {
+          const int i = m * 32 + lane;
+          unsigned long long key =
+              i < c ? (static_cast<unsigned long long>(order_key(row[i])) << 32) |
+                          (0xffffffffu - unsigned(i))
+                    : 0ull;
+#pragma unroll
+          for (int kk = 2; kk <= 32; kk <<= 1) {
+#pragma unroll
+            for (int j = kk >> 1; j > 0; j >>= 1) {
+              const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, j);
+              const bool keep_max = ((lane & j) == 0) == ((lane & kk) == 0);
+              key = keep_max ? (key > o ? key : o) : (key < o ? key : o);
+            }
+          }
+          if (lane < kap) fin[m * kap + lane] = key;   // compact: nseg * kap finalists
+        }
+      } else if (kap < c) {
+        for (int i = tl; i < c; i += 32 * WPH) {
           const float si = row[i];
-#pragma unroll 4
+          int r = 0;
           for (int j = 0; j < c; ++j) {
             const float sj = row[j];
             r += (sj > si) | ((sj == si) & (j < i));
           }
+          fl[h * cmax + i] = r < kap;
         }
-        fl[h * cmax + i] = r < kap;
+      }
+      __syncthreads();
+      if (kap < c && kap <= 32) {
+        // rank of each finalist among all finalists, one per thread of the head
+        const int nf = nseg * kap;
+        for (int f = tl; f < nf; f += 32 * WPH) {
+          const unsigned long long kf = fin[f];
+          if (kf == 0ull) continue;
+          int r = 0;
+#pragma unroll 8
+          for (int j = 0; j < nf; ++j) r += fin[j] > kf;
+          if (r < kap) fl[h * cmax + int(0xffffffffu - unsigned(kf & 0xffffffffu))] = 1;
+        }
       }
     }
     __syncthreads();
@@ -417,8 +474,34 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
             const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
             trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
           }
+          // The next pass reads this node's children (keys and values one
+          // level down) or, at level 1, its tokens: start pulling them into
+          // L2 now, one bulk prefetch per contiguous run, spread over the
+          // cluster's CTAs.
+          if ((h * kmax + pos) % CS == rank) {
+            if (lev > 1) {
+              const unsigned bytes = unsigned(p.b) * D * 4;
+              prefetch_l2(level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) +
+                              int64_t(node) * p.b * D, bytes);
+              prefetch_l2(level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) +
+                              int64_t(node) * p.b * D, bytes);
+            } else {
+              const unsigned bytes = unsigned(p.B) * D * unsigned(sizeof(T));
+              prefetch_l2(K + (kvbase + int64_t(node) * p.B) * D, bytes);
+              prefetch_l2(V + (kvbase + int64_t(node) * p.B) * D, bytes);
+            }
+          }
         }
         cnt += __popc(bal);
+      }
+      // orphans one level down (shared by every head)
+      if (lev > 1 && h == 0 && lane == 0 && rank == (CS - 1)) {
+        const int64_t o0 = int64_t(p.b) * vis[lev], o1 = vis[lev - 1];
+        if (o1 > o0) {
+          const unsigned bytes = unsigned(o1 - o0) * D * 4;
+          prefetch_l2(level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) + o0 * D, bytes);
+          prefetch_l2(level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) + o0 * D, bytes);
+        }
       }
     }
     __syncthreads();
@@ -432,6 +515,27 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     w_hi = min(nw, w_lo + ch);
   }
   const bool has_win = w_hi > w_lo;
+  // the top level's candidates (keys and values), pulled into L2 by rank 0
+  if (top > 0 && rank == 0 && tid == 0) {
+    const unsigned bytes = unsigned(vis[top]) * D * 4;
+    prefetch_l2(level_keys(p, const_cast<void*>(tree), top, seq, g), bytes);
+    prefetch_l2(level_vals(p, const_cast<void*>(tree), top, seq, g), bytes);
+  }
+  // Stage this CTA's window rows now: they do not depend on the selection,
+  // so the copies are in flight during the first level pass.
+  {
+    constexpr int CPR = D * int(sizeof(T)) / 16;       // 16-byte pieces per row
+    const int rows = w_hi - w_lo;
+    const int64_t row0 = kvbase + int64_t(a) * p.B + w_lo;
+    for (int x = tid; x < rows * CPR; x += kThreads) {
+      const int r = x / CPR, c = x % CPR;
+      cp_async16(reinterpret_cast<char*>(winK + size_t(r) * D) + c * 16,
+                 reinterpret_cast<const char*>(K + (row0 + r) * D) + c * 16);
+      cp_async16(reinterpret_cast<char*>(winV + size_t(r) * D) + c * 16,
+                 reinterpret_cast<const char*>(V + (row0 + r) * D) + c * 16);
+    }
+    cp_async_commit();
+  }
   if (top > 0) {
     rotate_q(qlev, cnt_c[top]);
     __syncthreads();
@@ -567,10 +671,13 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   const int cmax = int(cm < 1 ? 1 : cm);
   const int kmax = int(kk < cmax ? kk : cmax);
   if (cmax > 1024) return cudaErrorNotSupported;
+  // window rows staged per CTA: at most ceil((W + B - 1) / cs)
+  const int wrows = int((int64_t(p.W) + p.B - 1 + cs - 1) / cs);
   const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * (D + 2) +
                         size_t(kWarps) * G * (D + 2) +
                         size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
-                       size_t(2) * G * cmax + 16;
+                       size_t(2) * G * cmax + 16 + size_t(G) * ((cmax + 31) / 32) * 32 * 8 +
+                       size_t(2) * wrows * D * sizeof(T) + 16;
   if (bytes > 200 * 1024) return cudaErrorNotSupported;
   auto kern = decode_cluster_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -595,7 +702,8 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p, reinterpret_cast<const T*>(Q),
                             reinterpret_cast<const T*>(K), reinterpret_cast<const T*>(V), tree,
-                            len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax);
+                            len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax,
+                            wrows);
 }
 
 template <typename T, int D>

@@ -51,6 +51,7 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * kmax);  // [2][cmax]
 
   const float2* rope = rope_table(p, tree);
+  const int rmax = p.lay.rope_rows - 1;
   const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
   const int64_t a = s0 / p.B;
   int64_t vis[kMaxLevels + 2];
@@ -133,27 +134,35 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     const int win0 = int(a) * p.B;
     const int widx0 = nleaf * p.B;
     const int* kept1 = kept + 1 * kmax;                           // level 1 = parity 1
+    // A slot's items step their RoPE index by SPW: (cos, sin) are seeded from
+    // the table once per batch and advanced by the fixed rotation of SPW.
+    const int idx0 = window ? widx0 : 0;
+    float cstep[8];
+    if (p.rope) load_cs(rope, SPW, HALF, j0, cstep);
     for (int base = 0; base < nt; base += SPW * kPUnroll) {
-      RawPairs rk[kPUnroll], rv[kPUnroll];
-      float cs[kPUnroll][8];
+      TokRow<T, HALF> rk[kPUnroll], rv[kPUnroll];
+      float csc[8];
       bool on[kPUnroll];
+      if (p.rope) load_cs(rope, min(idx0 + base + slot, rmax), HALF, j0, csc);
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
         const int e = base + u * SPW + slot;
         on[u] = e < nt;
         if (on[u]) {
           const int pos = window ? win0 + e : kept1[div_B(p, e)] * p.B + mod_B(p, e);
-          RawLoad<T, HALF>::load(K + (kvbase + pos) * D, j0, rk[u]);
-          RawLoad<T, HALF>::load(V + (kvbase + pos) * D, j0, rv[u]);
-          if (p.rope) load_cs(rope, window ? widx0 + e : e, HALF, j0, cs[u]);
+          rk[u].load(K + (kvbase + pos) * D, j0);
+          rv[u].load(V + (kvbase + pos) * D, j0);
         }
       }
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
         float xk[8], xv[8], s = 0.f;
-        RawLoad<T, HALF>::cvt(rk[u], xk);
-        RawLoad<T, HALF>::cvt(rv[u], xv);
-        if (p.rope) rotate8(xk, cs[u]);
+        rk[u].cvt(xk);
+        rv[u].cvt(xv);
+        if (p.rope) {
+          rotate8(xk, csc);
+          advance_cs(csc, cstep);
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           s = fmaf(qtok[j0 + c], xk[c], s);
@@ -184,10 +193,13 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     const float* scV = sc + (vlev & 1) * cmax;
     const unsigned char* flV = kfl + (vlev & 1) * cmax;
     float* scK = sc + (klev & 1) * cmax;
+    float cstep[8];
+    if (p.rope) load_cs(rope, SPW, HALF, j0, cstep);
     for (int base = 0; base < total; base += SPW * kPUnroll) {
       RawPairs ra[kPUnroll];
-      float cs[kPUnroll][8];
+      float csc[8];
       int kind[kPUnroll], idx[kPUnroll];
+      if (p.rope) load_cs(rope, min(base + slot, rmax), HALF, j0, csc);
       float sv[kPUnroll];
 #pragma unroll
       for (int u = 0; u < kPUnroll; ++u) {
@@ -201,7 +213,6 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           kind[u] = pKey;
           idx[u] = i;
           RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
-          if (p.rope) load_cs(rope, i, HALF, j0, cs[u]);
         } else if (e < total) {
           const int i = e - nk;
           if (!flV[i]) {
@@ -216,8 +227,9 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       for (int u = 0; u < kPUnroll; ++u) {
         float x[8], s = 0.f;
         RawLoad<float, HALF>::cvt(ra[u], x);
+        if (kind[u] == pKey && p.rope) rotate8(x, csc);
+        if (p.rope) advance_cs(csc, cstep);
         if (kind[u] == pKey) {
-          if (p.rope) rotate8(x, cs[u]);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             s = fmaf(qlev[j0 + c], x[c], s);

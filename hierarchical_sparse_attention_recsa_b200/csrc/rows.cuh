@@ -144,3 +144,61 @@ struct TokRow<__nv_bfloat16, HALF> {
 };
 
 }  // namespace recsa
+
+namespace recsa {
+
+// Asynchronous 16-byte global -> shared copies (no registers held while in
+// flight); wait with cp_async_wait_all() and a barrier before reading.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gsrc));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// A lane's four pairs of a row held in shared memory (dtype T), as fp32.
+template <typename T, int HALF>
+struct SharedPairs;
+template <int HALF>
+struct SharedPairs<__nv_bfloat16, HALF> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* row, int j0, float* x) {
+    RawBf r;
+    r.a = *reinterpret_cast<const uint2*>(row + j0);
+    r.b = *reinterpret_cast<const uint2*>(row + HALF + j0);
+    raw_cvt_bf(r, x);
+  }
+};
+template <int HALF>
+struct SharedPairs<float, HALF> {
+  static __device__ __forceinline__ void load(const float* row, int j0, float* x) {
+    const float4 a = *reinterpret_cast<const float4*>(row + j0);
+    const float4 b = *reinterpret_cast<const float4*>(row + HALF + j0);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// (cos, sin) pairs advanced by a fixed rotation: cs <- cs * step (per pair,
+// as complex numbers), for rows whose RoPE index grows by a constant stride.
+__device__ __forceinline__ void advance_cs(float* cs, const float* step) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float c = cs[2 * u], s = cs[2 * u + 1];
+    cs[2 * u] = c * step[2 * u] - s * step[2 * u + 1];
+    cs[2 * u + 1] = s * step[2 * u] + c * step[2 * u + 1];
+  }
+}
+
+}  // namespace recsa
+
+namespace recsa {
+
+// Bulk prefetch of a contiguous global range into L2 by the TMA unit (one
+// instruction per range; 16-byte aligned address, size a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(bytes) : "memory");
+}
+
+}  // namespace recsa
