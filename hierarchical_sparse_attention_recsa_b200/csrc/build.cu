@@ -10,112 +10,10 @@
 // softmax, so K and V are streamed exactly once; each lane owns d/32
 // contiguous channels and issues one 4..16-byte load per row.
 #include "recsa_internal.cuh"
+#include "pool.cuh"
 
 namespace recsa {
 namespace {
-
-template <typename T, int N>
-struct RowIO;
-
-template <>
-struct RowIO<float, 4> {
-  __device__ static void load(const float* row, int lane, float* x) {
-    float4 v = reinterpret_cast<const float4*>(row)[lane];
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-  }
-  __device__ static void store(float* row, int lane, const float* x) {
-    reinterpret_cast<float4*>(row)[lane] = make_float4(x[0], x[1], x[2], x[3]);
-  }
-};
-template <>
-struct RowIO<float, 2> {
-  __device__ static void load(const float* row, int lane, float* x) {
-    float2 v = reinterpret_cast<const float2*>(row)[lane];
-    x[0] = v.x; x[1] = v.y;
-  }
-  __device__ static void store(float* row, int lane, const float* x) {
-    reinterpret_cast<float2*>(row)[lane] = make_float2(x[0], x[1]);
-  }
-};
-template <>
-struct RowIO<__nv_bfloat16, 4> {
-  __device__ static void load(const __nv_bfloat16* row, int lane, float* x) {
-    uint2 u = reinterpret_cast<const uint2*>(row)[lane];
-    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x);
-    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
-    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-    x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
-  }
-};
-template <>
-struct RowIO<__nv_bfloat16, 2> {
-  __device__ static void load(const __nv_bfloat16* row, int lane, float* x) {
-    __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(row)[lane];
-    float2 fa = __bfloat1622float2(a);
-    x[0] = fa.x; x[1] = fa.y;
-  }
-};
-
-// One warp pools `n` rows (keys at kbase, values at vbase, row stride d) into
-// this lane's N channels of key and value.  Rows are processed in groups of 8
-// so that eight loads per operand are in flight per lane.
-template <typename T, int N>
-__device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const float* rl,
-                          float inv_sqrt_d, int lane, float* key, float* val) {
-  float m = -INFINITY, l = 0.f;
-  float ak[N], av[N];
-#pragma unroll
-  for (int c = 0; c < N; ++c) ak[c] = av[c] = 0.f;
-  constexpr int U = 8;
-  for (int i0 = 0; i0 < n; i0 += U) {
-    float kx[U][N], vx[U][N], s[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (i0 + u < n) {
-        RowIO<T, N>::load(kbase + int64_t(i0 + u) * d, lane, kx[u]);
-        RowIO<T, N>::load(vbase + int64_t(i0 + u) * d, lane, vx[u]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float acc = 0.f;
-      if (i0 + u < n) {
-#pragma unroll
-        for (int c = 0; c < N; ++c) acc = fmaf(rl[c], kx[u][c], acc);
-      }
-      s[u] = acc;
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) s[u] = warp_sum(s[u]) * inv_sqrt_d;
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (i0 + u < n) {
-        float mn = fmaxf(m, s[u]);
-        float sc = expf(m - mn);
-        float w = expf(s[u] - mn);
-        l = l * sc + w;
-#pragma unroll
-        for (int c = 0; c < N; ++c) {
-          ak[c] = fmaf(w, kx[u][c], ak[c] * sc);
-          av[c] += vx[u][c];
-        }
-        m = mn;
-      }
-    }
-  }
-  float il = 1.f / l, in = 1.f / float(n);
-#pragma unroll
-  for (int c = 0; c < N; ++c) {
-    key[c] = ak[c] * il;
-    val[c] = av[c] * in;
-  }
-}
-
-template <int N>
-__device__ void load_r(const float* r, int lane, float* rl) {
-#pragma unroll
-  for (int c = 0; c < N; ++c) rl[c] = r[lane * N + c];
-}
 
 // Level 1: one warp per leaf block of one (sequence, KV head).
 template <typename T, int N>

@@ -24,6 +24,7 @@
 
 #include "recsa_internal.cuh"
 #include "rows.cuh"
+#include "pool.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -37,12 +38,25 @@ constexpr int kTokUnroll = 3;
 
 enum ItemKind { kKey = 0, kVal = 1, kNone = 2 };
 
+// Fused decode step (append + decode in one launch): the new token, the pooler
+// and the per-sequence step counters in the tree header.
+struct StepArgs {
+  const void* k_new;
+  const void* v_new;
+  const float* r;
+  int64_t r_stride;
+  int64_t* len_w;
+  int* counters;
+  int fuse;
+};
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                       const T* __restrict__ V, const void* __restrict__ tree,
                       const int64_t* __restrict__ len_dev, int n_q, T* __restrict__ O,
-                      int32_t* __restrict__ trace, int cmax, int kmax, int wrows) {
+                      int32_t* __restrict__ trace, int cmax, int kmax, int wrows,
+                      StepArgs st) {
   constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR, NSLOT = kWarps * SPW;
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = int(cluster.num_blocks());
@@ -72,7 +86,14 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   T* winK = reinterpret_cast<T*>(finbuf + size_t(G) * nseg_max * 32);
   T* winV = winK + size_t(wrows) * D;
 
-  const int64_t t = len_dev[seq] - 1;
+  // Fused step: the new token is appended at len (this kernel writes it and
+  // pools what it completes), and the query sits on it.  A full sequence is
+  // flagged and decoded without the append, as recsa_append would leave it.
+  const int64_t len0 = len_dev[seq];
+  const bool do_append = st.fuse && len0 >= 0 && len0 < p.cap;
+  const int64_t t = do_append ? len0 : len0 - 1;
+  const T* knew = reinterpret_cast<const T*>(st.k_new) + (seq * p.hkv + g) * D;
+  const T* vnew = reinterpret_cast<const T*>(st.v_new) + (seq * p.hkv + g) * D;
   const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
   const bool empty = t < 0 || t >= p.cap;   // uniform over the cluster
   const float2* rope = rope_table(p, tree);
@@ -527,12 +548,15 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     constexpr int CPR = D * int(sizeof(T)) / 16;       // 16-byte pieces per row
     const int rows = w_hi - w_lo;
     const int64_t row0 = kvbase + int64_t(a) * p.B + w_lo;
+    const int64_t tnew = do_append ? t - (int64_t(a) * p.B + w_lo) : -1;   // new token's row
     for (int x = tid; x < rows * CPR; x += kThreads) {
       const int r = x / CPR, c = x % CPR;
+      const T* ks = r == tnew ? knew : K + (row0 + r) * D;
+      const T* vs = r == tnew ? vnew : V + (row0 + r) * D;
       cp_async16(reinterpret_cast<char*>(winK + size_t(r) * D) + c * 16,
-                 reinterpret_cast<const char*>(K + (row0 + r) * D) + c * 16);
+                 reinterpret_cast<const char*>(ks) + c * 16);
       cp_async16(reinterpret_cast<char*>(winV + size_t(r) * D) + c * 16,
-                 reinterpret_cast<const char*>(V + (row0 + r) * D) + c * 16);
+                 reinterpret_cast<const char*>(vs) + c * 16);
     }
     cp_async_commit();
   }
@@ -651,6 +675,59 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       }
     }
   }
+
+  if (st.fuse) {
+    // Append: the first query's cluster of each (sequence, KV head) writes the
+    // token and pools the leaf and ancestors it completes (none of them is
+    // visible to this step's query: they end inside its window).
+    if (rank == 0 && qi == 0 && do_append) {
+      T* Kw = const_cast<T*>(K) + (kvbase + t) * D;
+      T* Vw = const_cast<T*>(V) + (kvbase + t) * D;
+      for (int x = tid; x < D; x += kThreads) {
+        Kw[x] = knew[x];
+        Vw[x] = vnew[x];
+      }
+      __syncthreads();
+      if ((t + 1) % p.B == 0 && warp == 0) {
+        constexpr int N = D / 32;
+        float rl[N], key[N], val[N];
+        load_r<N>(st.r + g * st.r_stride, lane, rl);
+        int64_t j = (t + 1) / p.B - 1;
+        const int64_t row0 = (kvbase + j * p.B) * D;
+        pool_rows<T, N>(K + row0, V + row0, p.B, D, rl, inv_sqrt_d, lane, key, val);
+        RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane,
+                               key);
+        RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane,
+                               val);
+        for (int lev = 2; lev <= p.lay.levels && (j + 1) % p.b == 0; ++lev) {
+          j = (j + 1) / p.b - 1;
+          __syncwarp();
+          const float* ck = level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
+          const float* cv = level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
+          pool_rows<float, N>(ck, cv, p.b, D, rl, inv_sqrt_d, lane, key, val);
+          RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), lev, seq, g) + j * D,
+                                 lane, key);
+          RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), lev, seq, g) + j * D,
+                                 lane, val);
+        }
+      }
+    }
+    // Length: every cluster of the sequence read len at its start; the last
+    // one to finish (per-sequence counter) publishes len + 1 and resets it.
+    if (rank == 0 && tid == 0) {
+      if (!do_append) {
+        if (len0 >= p.cap) atomicOr(tree_error_word(const_cast<void*>(tree)),
+                                    RECSA_DEVERR_APPEND_FULL);
+      } else {
+        __threadfence();
+        const int done = atomicAdd(st.counters + seq, 1);
+        if (done == p.hkv * n_q - 1) {
+          st.counters[seq] = 0;
+          st.len_w[seq] = len0 + 1;
+        }
+      }
+    }
+  }
 }
 
 }  // namespace
@@ -662,7 +739,7 @@ namespace {
 template <typename T, int D, int G>
 cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const void* V,
                           const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
-                          int32_t* trace, cudaStream_t s, int cs) {
+                          int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
   const int64_t kk = p.k < p.cap ? p.k : p.cap;
   int64_t maxn = 1;
   for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
@@ -703,19 +780,29 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   return cudaLaunchKernelEx(&cfg, kern, p, reinterpret_cast<const T*>(Q),
                             reinterpret_cast<const T*>(K), reinterpret_cast<const T*>(V), tree,
                             len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax,
-                            wrows);
+                            wrows, st);
 }
 
 template <typename T, int D>
 cudaError_t cluster_g(const Params& p, const void* Q, const void* K, const void* V,
                       const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
-                      int32_t* trace, cudaStream_t s, int cs) {
+                      int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
   switch (p.group) {
-    case 1: return cluster_typed<T, D, 1>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
-    case 2: return cluster_typed<T, D, 2>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
-    case 4: return cluster_typed<T, D, 4>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+    case 1: return cluster_typed<T, D, 1>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
+    case 2: return cluster_typed<T, D, 2>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
+    case 4: return cluster_typed<T, D, 4>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
     default: return cudaErrorNotSupported;
   }
+}
+
+cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, const void* V,
+                             const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
+                             int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st)
+                      : cluster_g<__nv_bfloat16, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
+  return p.d == 128 ? cluster_g<float, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st)
+                    : cluster_g<float, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
 }
 
 }  // namespace
@@ -735,12 +822,26 @@ int decode_cluster_size(const Params& p, int32_t n_q) {
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s) {
-  const int cs = decode_cluster_size(p, n_q);
-  if (p.dtype == RECSA_DTYPE_BF16)
-    return p.d == 128 ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs)
-                      : cluster_g<__nv_bfloat16, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
-  return p.d == 128 ? cluster_g<float, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs)
-                    : cluster_g<float, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs);
+  StepArgs st = {};
+  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s,
+                          decode_cluster_size(p, n_q), st);
+}
+
+cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
+                               const void* k_new, const void* v_new, int64_t* len_dev,
+                               const float* r, int64_t r_stride, void* tree, int32_t n_q,
+                               void* O, int32_t* trace, cudaStream_t s) {
+  if (p.batch > kStepCounters) return cudaErrorNotSupported;
+  StepArgs st;
+  st.k_new = k_new;
+  st.v_new = v_new;
+  st.r = r;
+  st.r_stride = r_stride;
+  st.len_w = len_dev;
+  st.counters = reinterpret_cast<int*>(reinterpret_cast<char*>(tree) + kStepCounterOffset);
+  st.fuse = 1;
+  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s,
+                          decode_cluster_size(p, n_q), st);
 }
 
 }  // namespace recsa

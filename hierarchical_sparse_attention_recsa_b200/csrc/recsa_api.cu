@@ -250,6 +250,42 @@ recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void*
   return attend_common(geom, Q, K, V, tree, len_dev, 0, n_q, 1, O, trace, nullptr, 0, stream);
 }
 
+recsa_status recsa_decode_step(const recsa_geometry* geom, const void* Q, void* K, void* V,
+                               const void* k_new, const void* v_new, int64_t* len_dev,
+                               const float* pooler_r, int64_t pooler_head_stride, void* tree,
+                               int32_t n_q, void* O, int32_t* trace, void* stream) {
+  Params p;
+  recsa_status st = make_params(geom, &p);
+  if (st != RECSA_OK) return st;
+  if (!Q || !K || !V || !k_new || !v_new || !len_dev || !pooler_r || !tree || !O)
+    return RECSA_ERR_NULL;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(k_new, 16) ||
+      !aligned(v_new, 16) || !aligned(O, 16) || !aligned(tree, 256) || !aligned(len_dev, 8) ||
+      !aligned(pooler_r, 4) || (trace && !aligned(trace, 4)))
+    return RECSA_ERR_MISALIGNED;
+  if (pooler_head_stride < 0) return RECSA_ERR_INVALID_GEOMETRY;
+  if (n_q < 1) return RECSA_ERR_CAPACITY;
+  if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorNotSupported;
+  if (!getenv("RECSA_DECODE_GENERIC"))
+    e = launch_decode_step(p, Q, K, V, k_new, v_new, len_dev, pooler_r, pooler_head_stride,
+                           tree, n_q, O, trace, s);
+  if (e == cudaErrorNotSupported) {
+    // outside the fused kernel's limits: the same step as two launches
+    cudaGetLastError();
+    e = launch_append(p, K, V, k_new, v_new, len_dev, pooler_r, pooler_head_stride, tree, s);
+    if (e == cudaSuccess)
+      return attend_common(geom, Q, K, V, tree, len_dev, 0, n_q, 1, O, trace, nullptr, 0,
+                           stream);
+  }
+  if (e == cudaErrorInvalidConfiguration || e == cudaErrorInvalidValue) {
+    cudaGetLastError();
+    return RECSA_ERR_UNSUPPORTED;
+  }
+  return cuda_status(e);
+}
+
 recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, const void* K,
                                   const void* V, const void* tree, int64_t q_start, int32_t n_q,
                                   void* O, int32_t* trace, void* stream) {

@@ -13,6 +13,9 @@ namespace recsa {
 constexpr int kMaxLevels = RECSA_MAX_LEVELS;
 constexpr int kHeaderBytes = 256;
 constexpr int kTraceHead = 4 + 2 * kMaxLevels;  // ints before the kept-id lists
+// Per-sequence step counters of the fused decode step live in the tree header.
+constexpr int kStepCounterOffset = 64;
+constexpr int kStepCounters = (kHeaderBytes - kStepCounterOffset) / 4;
 
 // Byte layout of the caller-owned tree buffer (computed on the host).
 struct TreeLayout {
@@ -97,6 +100,13 @@ cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const v
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);
+// Fused decode step: append (token write, pooling of completed nodes, length
+// update) and decode in one cluster launch; cudaErrorNotSupported when the
+// geometry or batch is outside its limits.
+cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
+                               const void* k_new, const void* v_new, int64_t* len_dev,
+                               const float* r, int64_t r_stride, void* tree, int32_t n_q,
+                               void* O, int32_t* trace, cudaStream_t s);
 // Warp-per-(query, head) prefill kernel; cudaErrorNotSupported outside its limits.
 // wpart: window partials from launch_prefill_window (fp32 rows of d + 2 per
 // (sequence, query, head): normalised output, max, sum), or null to let this

@@ -38,7 +38,7 @@ STATUS = {
 }
 
 EXPORTS = ["recsa_status_string", "recsa_validate", "recsa_num_levels", "recsa_tree_bytes",
-           "recsa_build", "recsa_append", "recsa_decode", "recsa_prefill",
+           "recsa_build", "recsa_append", "recsa_decode", "recsa_decode_step", "recsa_prefill",
            "recsa_prefill_workspace_bytes", "recsa_prefill_static", "recsa_trace_ints",
            "recsa_tree_error"]
 
@@ -116,6 +116,7 @@ def lib() -> ctypes.CDLL:
         L.recsa_build.argtypes = [G, vp, vp, ctypes.POINTER(i64), vp, i64, vp, vp]
         L.recsa_append.argtypes = [G, vp, vp, vp, vp, vp, vp, i64, vp, vp]
         L.recsa_decode.argtypes = [G, vp, vp, vp, vp, vp, i32, vp, vp, vp]
+        L.recsa_decode_step.argtypes = [G, vp, vp, vp, vp, vp, vp, vp, i64, vp, i32, vp, vp, vp]
         L.recsa_prefill.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp, ctypes.c_size_t,
                                     vp]
         L.recsa_prefill_workspace_bytes.argtypes = [G, i32, ctypes.POINTER(ctypes.c_size_t)]
@@ -201,6 +202,18 @@ def recsa_decode(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tens
     _check(lib().recsa_decode(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree),
                               _ptr(len_dev), n_q, _ptr(O), _ptr(trace), _stream(stream)),
            "recsa_decode")
+
+
+def recsa_decode_step(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                      k_new: torch.Tensor, v_new: torch.Tensor, len_dev: torch.Tensor,
+                      pooler_r: torch.Tensor, pooler_head_stride: int, tree: torch.Tensor,
+                      n_q: int, O: torch.Tensor, trace: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    g = geom.c()
+    _check(lib().recsa_decode_step(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(k_new),
+                                   _ptr(v_new), _ptr(len_dev), _ptr(pooler_r),
+                                   pooler_head_stride, _ptr(tree), n_q, _ptr(O), _ptr(trace),
+                                   _stream(stream)), "recsa_decode_step")
 
 
 def recsa_prefill(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,

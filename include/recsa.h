@@ -150,6 +150,24 @@ recsa_status recsa_decode(const recsa_geometry* geom, const void* Q, const void*
                           int32_t n_q, void* O, int32_t* trace, void* stream);
 
 /*
+ * One decode step in a single launch: recsa_append of k_new, v_new followed by
+ * recsa_decode of the n_q queries at the new token's position, with the same
+ * results (the new token is read from k_new/v_new by the attention, written
+ * to K/V, and the leaf and ancestors it completes are pooled; none of those
+ * nodes is visible to the step's own query, whose window holds them).  A
+ * sequence at capacity is flagged (RECSA_DEVERR_APPEND_FULL) and decoded
+ * without the append, as the two separate calls would do.
+ *   len_dev: DEVICE int64 [batch], incremented for every appended sequence.
+ *   Per-sequence step counters live in the tree header (zeroed by
+ *   recsa_build); for batch > 48 the step runs as the two separate launches.
+ *   Steps on one tree must not overlap on the device.
+ */
+recsa_status recsa_decode_step(const recsa_geometry* geom, const void* Q, void* K, void* V,
+                               const void* k_new, const void* v_new, int64_t* len_dev,
+                               const float* pooler_r, int64_t pooler_head_stride, void* tree,
+                               int32_t n_q, void* O, int32_t* trace, void* stream);
+
+/*
  * Prefill attention: query i of sequence s sits at position q_start + i,
  * i < n_q, causal.  The tree must have been built over at least q_start + n_q
  * tokens of every sequence (a node is a pure function of its span, so a tree

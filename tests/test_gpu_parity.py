@@ -339,6 +339,80 @@ def test_append_matches_build_and_oracle():
     _check_tree(g, tree, trees, torch.bfloat16)
 
 
+@pytest.mark.parametrize("nq", [1, 2])
+def test_decode_step_equals_append_then_decode(nq):
+    """The fused step (one launch) gives the same outputs, cache, tree and
+    lengths as recsa_append followed by recsa_decode, across leaf and level-2
+    completions, and matches the oracle on sampled steps."""
+    w = MODEL
+    lens0 = [4000, 4031]
+    steps = 130
+    cap = 4096 + 256
+    g, K, V, r, Kd, Vd, rd, tree_a = _setup(w, lens0, cap, seed=12)
+    tree_b = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, lens0, rd, 0, tree_b)
+    Ka, Va, Kb, Vb = Kd.clone(), Vd.clone(), Kd.clone(), Vd.clone()
+    for X in (Ka, Va, Kb, Vb):
+        X[0, :, 4000:] = 0
+        X[1, :, 4031:] = 0
+    la = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    lb = la.clone()
+    og = oracle_geometry(g)
+    G = g.n_q_heads // g.n_kv_heads
+    st = Stats()
+    ti = R.recsa_trace_ints(g)
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        lens_now = [L + step + 1 for L in lens0]
+        pos = torch.tensor([[L - 1] * nq for L in lens_now], dtype=torch.int64)
+        Q, _, _ = synth.make_queries(w, K, pos, seed=100 + step)
+        Qd = Q.cuda()
+        Oa = torch.empty_like(Qd)
+        Ob = torch.empty_like(Qd)
+        trace = torch.zeros((2, nq, g.n_q_heads, ti), dtype=torch.int32, device="cuda")
+        R.recsa_decode_step(g, Qd, Ka, Va, kn, vn, la, rd, 0, tree_a, nq, Oa, trace)
+        R.recsa_append(g, Kb, Vb, kn, vn, lb, rd, 0, tree_b)
+        R.recsa_decode(g, Qd, Kb, Vb, tree_b, lb, nq, Ob)
+        torch.cuda.synchronize()
+        assert torch.equal(Oa, Ob), step
+        assert la.cpu().tolist() == lens_now
+        if step in (31, 95, steps - 1):
+            tr = trace.cpu().numpy()
+            for s in range(2):
+                Kh_all = to_np(K[s, :, :lens_now[s]])
+                Vh_all = to_np(V[s, :, :lens_now[s]])
+                for h in range(0, g.n_q_heads, 9):
+                    Kh, Vh = Kh_all[h // G], Vh_all[h // G]
+                    src = oracle.LazyTree(Kh, Vh, r.double().numpy(), g.leaf_block, g.branching)
+                    check_query(st, to_np(Oa[s, nq - 1, h]), tr[s, nq - 1, h],
+                                to_np(Q[s, nq - 1, h]), lens_now[s] - 1, Kh, Vh, src, og, g.k)
+    st.check(torch.bfloat16, "decode step")
+    assert torch.equal(Ka, Kb) and torch.equal(Va, Vb)
+    assert torch.equal(tree_a[256:], tree_b[256:])
+
+
+def test_decode_step_at_capacity_flags_and_decodes_without_append():
+    w = MODEL
+    cap = 320
+    g, K, V, r, Kd, Vd, rd, tree = _setup(w, [cap, 200], cap, seed=13)
+    lens = torch.tensor([cap, 200], dtype=torch.int64, device="cuda")
+    kn = Kd[:, :, 0].contiguous()
+    vn = Vd[:, :, 0].contiguous()
+    Q = torch.randn((2, 1, g.n_q_heads, g.head_dim), device="cuda").to(Kd.dtype)
+    O = torch.empty_like(Q)
+    K_before = Kd.clone()
+    R.recsa_decode_step(g, Q, Kd, Vd, kn, vn, lens, rd, 0, tree, 1, O)
+    assert R.recsa_tree_error(g, tree, clear=True) == R.DEVERR_APPEND_FULL
+    assert lens.cpu().tolist() == [cap, 201]
+    assert torch.equal(Kd[0], K_before[0])                    # full sequence untouched
+    Ob = torch.empty_like(Q)
+    R.recsa_decode(g, Q, Kd, Vd, tree, lens, 1, Ob)
+    torch.cuda.synchronize()
+    assert torch.equal(O[0], Ob[0])                           # decoded at len - 1
+    assert torch.equal(O[1], Ob[1])                           # appended, then decoded
+
+
 def test_append_at_capacity_sets_flag_and_keeps_len():
     w = MODEL
     cap = 256
