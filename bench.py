@@ -137,11 +137,18 @@ def elem_bytes(w):
 
 
 class L2Flush:
-    def __init__(self, mib=256):
+    """Write 256 MiB (twice the L2) before a timed region, then keep the GPU
+    busy for ~100 us so that the host has queued the timed launch before the
+    start event is reached: the events then bracket device time only, not the
+    host's launch latency."""
+
+    def __init__(self, mib=256, spin_cycles=200_000):
         self.buf = torch.empty(mib << 20, dtype=torch.uint8, device="cuda")
+        self.spin = spin_cycles
 
     def __call__(self):
         self.buf.fill_(1)
+        torch.cuda._sleep(self.spin)
 
 
 def elapsed(a, b):
@@ -291,7 +298,9 @@ def run_recsa(args, rank, world, dev):
                    "leaf_block": w.leaf_block, "branching": w.branching, "k": w.k,
                    "window": w.window, "levels": R.recsa_num_levels(g, L),
                    "step": "recsa_decode_step (append + decode in one launch) for the batch",
-                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "l2": "flushed before every timed step (256 MiB write, outside the events; "
+                         "the GPU is kept busy past the flush so the events bracket device "
+                         "time, not host launch latency)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "kernel": "decode_cluster_kernel (fused step)",
                      "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
