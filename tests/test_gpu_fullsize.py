@@ -2,8 +2,8 @@
 one by one (its tree is built lazily from each sampled head's cache).
 
 * 524K (32q/8kv, d=128, B64 b16 k8 W512, 4 levels): decode at batch 4 after an
-  append, in the launch configuration the benchmark times (cluster size
-  chosen automatically); full causal prefill of one sequence in 64K-query
+  append, and the fused append + decode step the benchmark times, in its
+  launch configuration (cluster size chosen automatically); full causal prefill of one sequence in 64K-query
   chunks with the tensor-core window workspace, as the benchmark runs it.
 * 131K: decode (3 levels).
 * 1M (b32, 3 levels): decode with needle and mixture queries.
@@ -37,7 +37,8 @@ def _host_head(K, V, s, g, n):
     return (K[s, g, :n].float().cpu().numpy(), V[s, g, :n].float().cpu().numpy())
 
 
-def _decode_case(wname, batch, appended=1, samples=((0, 0), (0, 13), (0, 31)), seed=0):
+def _decode_case(wname, batch, appended=1, samples=((0, 0), (0, 13), (0, 31)), seed=0,
+                 fused=False):
     w = synth.WORKLOADS[wname]
     L = w.length
     cap = L + 64
@@ -46,17 +47,22 @@ def _decode_case(wname, batch, appended=1, samples=((0, 0), (0, 13), (0, 31)), s
     tree = alloc_tree(g)
     R.recsa_build(g, K, V, [L] * batch, r, 0, tree)
     lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
-    for i in range(appended):      # the step the benchmark times: append, then decode
-        kn = K[:, :, L + i].contiguous()
-        vn = V[:, :, L + i].contiguous()
-        R.recsa_append(g, K, V, kn, vn, lens, r, 0, tree)
     n = L + appended
     pos = torch.full((batch, 1), n - 1, dtype=torch.int64, device="cuda")
     Q, kind, _ = synth.make_queries(w, K, pos, seed=seed + 1, n_needles=None)
     O = torch.empty_like(Q)
     trace = torch.zeros((batch, 1, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
                         device="cuda")
-    R.recsa_decode(g, Q, K, V, tree, lens, 1, O, trace)
+    for i in range(appended):
+        kn = K[:, :, L + i].contiguous()
+        vn = V[:, :, L + i].contiguous()
+        if fused and i == appended - 1:
+            # the step the benchmark times: append and decode in one launch
+            R.recsa_decode_step(g, Q, K, V, kn, vn, lens, r, 0, tree, 1, O, trace)
+        else:
+            R.recsa_append(g, K, V, kn, vn, lens, r, 0, tree)
+    if not fused:
+        R.recsa_decode(g, Q, K, V, tree, lens, 1, O, trace)
     torch.cuda.synchronize()
     assert lens.cpu().tolist() == [n] * batch
     og = oracle_geometry(g)
@@ -78,6 +84,14 @@ def _decode_case(wname, batch, appended=1, samples=((0, 0), (0, 13), (0, 31)), s
 
 def test_decode_524k_batch4_bench_config():
     _decode_case("qwen3-4b-524k", 4, samples=((0, 0), (1, 9), (2, 18), (3, 31), (3, 30)))
+
+
+def test_decode_step_524k_batch4_bench_call():
+    """The exact call the benchmark times: recsa_decode_step for the batch,
+    here after 63 plain appends so the step itself completes a leaf block and
+    pools it in-kernel."""
+    _decode_case("qwen3-4b-524k", 4, appended=64, fused=True,
+                 samples=((0, 1), (1, 8), (2, 23), (3, 29)), seed=2)
 
 
 def test_decode_131k():
