@@ -33,6 +33,7 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kRegSlots = 8;      // top-k candidates held in registers: 32 per slot
 constexpr int kUnroll = 3;
 constexpr int kTokUnroll = 3;
 
@@ -78,12 +79,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* mrg = wwin + kWarps * G * (D + 2);            // [CS][G][D + 2] cluster merge (rank 0)
   int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
   unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
-  // top-k finalists: [G][ceil(cmax / 32)][32] keys
-  const int nseg_max = (cmax + 31) / 32;
-  unsigned long long* finbuf = reinterpret_cast<unsigned long long*>(
-      (reinterpret_cast<uintptr_t>(kfl + 2 * G * cmax) + 15) & ~uintptr_t(15));
   // window rows of this CTA staged by cp.async: K then V, [wrows][D] each
-  T* winK = reinterpret_cast<T*>(finbuf + size_t(G) * nseg_max * 32);
+  T* winK = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(kfl + 2 * G * cmax) + 15) &
+                                 ~uintptr_t(15));
   T* winV = winK + size_t(wrows) * D;
 
   // Fused step: the new token is appended at len (this kernel writes it and
@@ -417,80 +415,81 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     if (tokens) token_loop();
   };
 
-  // Warp top-k of head h at level lev over the full score table (every CTA).
+  // Top-k of head h at level lev over the full score table (every CTA runs
+  // the same selection on the same broadcast scores).  One warp per head
+  // takes kap rounds of a warp arg-max: lane l holds the order-preserving
+  // keys of candidates l, l + 32, ... in registers (0 = none or taken; every
+  // finite score maps above 0); redux.sync gives the round's maximum, a
+  // ballot the lanes holding it, and on a tie of keys across lanes the lowest
+  // index wins (within a lane the lowest slot).  Bit s of `taken` marks
+  // candidate 32 s + l as kept.  Candidates beyond 32 * kRegSlots are read
+  // from shared memory in the same rounds.  The kept list is compacted in
+  // index order with one ballot per slot row.  The selecting warp of head h
+  // is h * WPH + (h % 4), so the G selections run on different schedulers.
   auto topk = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
-    float* scl = sc + par * G * cmax;
-    unsigned char* fl = kfl + par * G * cmax;
-    int* kp = kept + par * G * kmax;
-    // Selection, by the head's WPH warps: each 32-candidate segment is sorted
-    // by a warp bitonic network on (score, -index) keys, its best kap keys
-    // become finalists, and one warp ranks the finalists (a candidate is in
-    // the top kap iff it is in its segment's top kap).  Ties go to the lower
-    // index.  kap > 32 falls back to rank counting over all candidates.
-    {
-      const int h = hw, wl = warp % WPH, tl = wl * 32 + lane;
-      const float* row = scl + h * cmax;
-      for (int i = tl; i < c; i += 32 * WPH) fl[h * cmax + i] = kap >= c;
-      const int nseg = (c + 31) / 32;
-      unsigned long long* fin = finbuf + size_t(h) * nseg_max * 32;
-      if (kap < c && kap <= 32) {
-        for (int m = wl; m < nseg; m += WPH) {
-          const int i = m * 32 + lane;
-          unsigned long long key =
-              i < c ? (static_cast<unsigned long long>(order_key(row[i])) << 32) |
-                          (0xffffffffu - unsigned(i))
-                    : 0ull;
+    if (warp == hw * WPH + (hw & 3) % WPH) {
+      const int h = hw;
+      const float* row = sc + par * G * cmax + h * cmax;
+      const int ns = (c + 31) >> 5;
+      unsigned taken = 0;
+      if (kap >= c) {
+        for (int s = 0; s < ns; ++s)
+          if (s * 32 + lane < c) taken |= 1u << s;
+      } else {
+        unsigned key[kRegSlots];
 #pragma unroll
-          for (int kk = 2; kk <= 32; kk <<= 1) {
+        for (int s = 0; s < kRegSlots; ++s) {
+          const int i = s * 32 + lane;
+          key[s] = i < c ? order_key(row[i]) : 0u;
+        }
+        for (int r = 0; r < kap; ++r) {
+          unsigned bk = key[0];
+          int bs = 0;
 #pragma unroll
-            for (int j = kk >> 1; j > 0; j >>= 1) {
-              const unsigned long long o = __shfl_xor_sync(0xffffffffu, key, j);
-              const bool keep_max = ((lane & j) == 0) == ((lane & kk) == 0);
-              key = keep_max ? (key > o ? key : o) : (key < o ? key : o);
+          for (int s = 1; s < kRegSlots; ++s)
+            if (key[s] > bk) {
+              bk = key[s];
+              bs = s;
+            }
+          for (int s = kRegSlots; s < ns; ++s) {
+            const int i = s * 32 + lane;
+            if (i < c && !((taken >> s) & 1u)) {
+              const unsigned kk = order_key(row[i]);
+              if (kk > bk) {
+                bk = kk;
+                bs = s;
+              }
             }
           }
-          if (lane < kap) fin[m * kap + lane] = key;   // compact: nseg * kap finalists
-        }
-      } else if (kap < c) {
-        for (int i = tl; i < c; i += 32 * WPH) {
-          const float si = row[i];
-          int r = 0;
-          for (int j = 0; j < c; ++j) {
-            const float sj = row[j];
-            r += (sj > si) | ((sj == si) & (j < i));
+          const unsigned M = __reduce_max_sync(0xffffffffu, bk);
+          unsigned who = __ballot_sync(0xffffffffu, bk == M);
+          if (__popc(who) > 1) {
+            const unsigned I =
+                __reduce_min_sync(0xffffffffu, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
+            who = 1u << (I & 31u);
           }
-          fl[h * cmax + i] = r < kap;
+          if ((who >> lane) & 1u) {
+            taken |= 1u << bs;
+#pragma unroll
+            for (int s = 0; s < kRegSlots; ++s)
+              if (s == bs) key[s] = 0u;
+          }
         }
       }
-      __syncthreads();
-      if (kap < c && kap <= 32) {
-        // rank of each finalist among all finalists, one per thread of the head
-        const int nf = nseg * kap;
-        for (int f = tl; f < nf; f += 32 * WPH) {
-          const unsigned long long kf = fin[f];
-          if (kf == 0ull) continue;
-          int r = 0;
-#pragma unroll 8
-          for (int j = 0; j < nf; ++j) r += fin[j] > kf;
-          if (r < kap) fl[h * cmax + int(0xffffffffu - unsigned(kf & 0xffffffffu))] = 1;
-        }
-      }
-    }
-    __syncthreads();
-    if (warp < G) {
-      const int h = warp;
-      __syncwarp();
+      unsigned char* fl = kfl + par * G * cmax + h * cmax;
+      int* kp = kept + par * G * kmax + h * kmax;
       int cnt = 0;
-      for (int j = 0; j < c; j += 32) {
-        const int i = j + lane;
-        const bool f = i < c && fl[h * cmax + i];
+      for (int s = 0; s < ns; ++s) {
+        const int i = s * 32 + lane;
+        const bool f = i < c && ((taken >> s) & 1u);
+        if (i < c) fl[i] = f;
         const unsigned bal = __ballot_sync(0xffffffffu, f);
         if (f) {
           const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
           const int node = cand_node(lev, h, i);
-          kp[h * kmax + pos] = node;
+          kp[pos] = node;
           if (trace && rank == 0) {
             const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
             trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
@@ -753,8 +752,7 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * (D + 2) +
                         size_t(kWarps) * G * (D + 2) +
                         size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
-                       size_t(2) * G * cmax + 16 + size_t(G) * ((cmax + 31) / 32) * 32 * 8 +
-                       size_t(2) * wrows * D * sizeof(T) + 16;
+                       size_t(2) * G * cmax + 16 + size_t(2) * wrows * D * sizeof(T);
   if (bytes > 200 * 1024) return cudaErrorNotSupported;
   auto kern = decode_cluster_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
