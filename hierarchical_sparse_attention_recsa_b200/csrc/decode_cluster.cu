@@ -5,22 +5,38 @@
 // selection of at most k candidates per level, unselected summaries in one
 // softmax with the exact tokens, candidate-local RoPE), laid out for B200:
 //
-//   * The CS CTAs of a cluster split every level's (head, candidate) pairs.
-//     Each CTA scores its share and stores the scores into every CTA's shared
-//     memory (distributed shared memory); one cluster barrier per level, then
-//     each CTA runs the same warp top-k on the full score table, so every CTA
-//     knows the kept nodes without a second exchange.
-//   * Work that does not depend on the selection (the window tokens) runs in
-//     the first pass; the values of a level's unselected candidates are
-//     folded in during the next level's pass, so each level costs one
-//     dependent memory round trip.
-//   * Rows (fp32 summary rows, bf16/fp32 K/V rows) are read straight into
-//     registers with 16-byte loads: a row is spread over d/8 lanes, each lane
-//     holding four rotate-half pairs (j, j + d/2), so the RoPE rotation is
-//     local to the lane.  Each lane slot keeps an online softmax state per
-//     head; states are merged across slots, warps and finally the cluster
-//     (again through distributed shared memory) without any global scratch.
+//   * Every gather of the method is a few contiguous runs: a level's
+//     candidates are the b children of each kept node (b * d contiguous fp32
+//     summary rows) plus one run of orphans, and a kept leaf is B contiguous
+//     K rows and B contiguous V rows.  Each run is copied into shared memory
+//     by one TMA bulk copy (cp.async.bulk) completing on an mbarrier, so a
+//     level's whole candidate set is in flight at once with no registers held.
+//   * A cluster of CS = (G / HPC) * S CTAs serves one (sequence, query, KV
+//     head).  CTA rank = hg * S + sh owns the HPC query heads of head group hg
+//     and share sh of their candidates and kept leaves.  With S = 1 a level's
+//     scores, top-k and kept list stay in the CTA; with S > 1 the S CTAs of a
+//     head group store their scores into each other's shared memory
+//     (distributed shared memory) and signal each other's "scores ready"
+//     mbarrier.  HPC and S are chosen per launch so that the grid fills the
+//     148 SMs.
+//   * Warps are specialised.  Twelve chain warps walk the levels (score,
+//     top-k, issue the next level's copies, fold the unselected summary
+//     values while those copies fly) and then stream the kept leaves through a
+//     ring of bulk-copy slots.  Four window warps attend the exact window,
+//     which does not depend on the selection, through their own ring of
+//     bulk-copy slots, concurrently with the chain; each CTA sends its window
+//     partial of every head to that head's owner at the end.
+//   * Rows are read from shared memory with 16-byte (fp32) or 8-byte (bf16)
+//     loads: a row is spread over d/8 lanes, each lane holding four
+//     rotate-half pairs (j, j + d/2), so the RoPE rotation is local to the
+//     lane.  Each lane slot keeps an online softmax state; states are merged
+//     across slots, warps and finally the cluster (through distributed shared
+//     memory) without any global scratch.
+//   * Every wait on an mbarrier is bounded; on expiry the kernel sets
+//     RECSA_DEVERR_WAIT_TIMEOUT in the tree header and runs to completion.
 #include <cooperative_groups.h>
+#include <cstdio>
+#include <cstdlib>
 
 #include "recsa_internal.cuh"
 #include "rows.cuh"
@@ -33,11 +49,21 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
+constexpr int kChainWarps = 12;
+constexpr int kWinWarps = kWarps - kChainWarps;
+constexpr int kChainThreads = kChainWarps * 32;
 constexpr int kRegSlots = 8;      // top-k candidates held in registers: 32 per slot
-constexpr int kUnroll = 3;
-constexpr int kTokUnroll = 3;
+constexpr int kWinRing = 4;       // window ring slots
+constexpr int kWinChunk = 16;     // window rows per ring slot
+constexpr int kMaxCluster = 16;
+constexpr int kMaxTokSlots = 4;   // kept-leaf ring slots per head
+constexpr unsigned long long kWaitNs = 50000000ull;   // a wait gives up after 50 ms
+constexpr size_t kSmemLimit = 227 * 1024;
 
-enum ItemKind { kKey = 0, kVal = 1, kNone = 2 };
+// Named barriers (0 is __syncthreads).
+constexpr int kBarChain = 1;      // the chain warps
+constexpr int kBarWindow = 2;     // the window warps
+constexpr int kBarHead0 = 3;      // + h: the chain warps of local head h
 
 // Fused decode step (append + decode in one launch): the new token, the pooler
 // and the per-sequence step counters in the tree header.
@@ -51,17 +77,245 @@ struct StepArgs {
   int fuse;
 };
 
-template <typename T, int D, int G>
+// ---------------------------------------------------------------------------
+// PTX wrappers: mbarriers, bulk copies, cluster barriers, named barriers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned smem_addr(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* mb, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(mb)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+// Arrive once on mb and add `bytes` to the transaction count of its phase.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* mb, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(mb)),
+               "r"(bytes)
+               : "memory");
+}
+// Arrive once (release at cluster scope) on the mbarrier at the same offset
+// in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* mb, int rank) {
+  unsigned remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n"
+               : "=r"(remote)
+               : "r"(smem_addr(mb)), "r"(rank));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(remote)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* mb, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(mb)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase of the given parity.  False when it did not
+// complete within kWaitNs, or when an earlier wait of this thread expired
+// (`expired` is then set, and later waits return at once so that the kernel
+// runs to completion).
+__device__ __forceinline__ bool mbar_wait(uint64_t* mb, unsigned parity, bool& expired) {
+  if (expired) return false;
+  if (mbar_try_wait(mb, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_wait(mb, parity)) return true;
+    if (global_ns() - t0 > kWaitNs) {
+      expired = true;
+      return false;
+    }
+  }
+}
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// global memory into this CTA's shared memory, completing on mb.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes,
+                                         uint64_t* mb) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(mb))
+      : "memory");
+}
+// Orders this thread's earlier shared-memory accesses (and those it has
+// synchronised with) before later bulk copies into shared memory.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+__device__ __forceinline__ void fence_cluster() {
+  asm volatile("fence.acq_rel.cluster;\n" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory");
+}
+
+// Online-softmax state (m, l, acc) of a lane slot merged with the state held by
+// the lanes `o` apart (shuffles); every lane ends with the merged state.
+__device__ __forceinline__ void merge_xor(float& m, float& l, float* acc, int o) {
+  const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+  const float lo = __shfl_xor_sync(0xffffffffu, l, o);
+  const float mn = fmaxf(m, mo);
+  const float ra = (m == -INFINITY) ? 0.f : __expf(m - mn);
+  const float rb = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
+  l = l * ra + lo * rb;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float ao = __shfl_xor_sync(0xffffffffu, acc[c], o);
+    acc[c] = acc[c] * ra + ao * rb;
+  }
+  m = mn;
+}
+
+// One online-softmax fold of score s with value pairs v.
+__device__ __forceinline__ void fold8(float& m, float& l, float* acc, float s, const float* v) {
+  if (s > m) {
+    const float r = __expf(m - s);
+    l = l * r + 1.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
+    m = s;
+  } else {
+    const float w = __expf(s - m);
+    l += w;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
+  }
+}
+
+// Two online-softmax folds (scores s0, s1 with value pairs v0, v1; a row
+// that is off is skipped) with one rescale of the state.
+__device__ __forceinline__ void fold2(float& m, float& l, float* acc, float s0, bool on0,
+                                      const float* v0, float s1, bool on1, const float* v1) {
+  s0 = on0 ? s0 : -INFINITY;
+  s1 = on1 ? s1 : -INFINITY;
+  const float mx = fmaxf(s0, s1);
+  if (mx == -INFINITY) return;
+  if (mx > m) {
+    const float r = __expf(m - mx);
+    l *= r;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] *= r;
+    m = mx;
+  }
+  const float w0 = on0 ? __expf(s0 - m) : 0.f;
+  const float w1 = on1 ? __expf(s1 - m) : 0.f;
+  l += w0 + w1;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = fmaf(w0, v0[c], fmaf(w1, v1[c], acc[c]));
+}
+
+// A lane's four rotate-half pairs of an fp32 row in shared memory.
+__device__ __forceinline__ void lds_pairs(const float* row, int j0, int half, float* x) {
+  const float4 a = *reinterpret_cast<const float4*>(row + j0);
+  const float4 b = *reinterpret_cast<const float4*>(row + half + j0);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// A lane's four (cos, sin) pairs of a RoPE table row held in shared memory.
+__device__ __forceinline__ void lds_cs8(const float* row, int j0, float* cs) {
+  const float4 a = *reinterpret_cast<const float4*>(row + 2 * j0);
+  const float4 b = *reinterpret_cast<const float4*>(row + 2 * j0 + 4);
+  cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
+  cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
+}
+// out = a * b per (cos, sin) pair, as complex numbers (rotation angles add).
+__device__ __forceinline__ void cmul8(float* out, const float* a, const float* b) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    out[2 * u] = a[2 * u] * b[2 * u] - a[2 * u + 1] * b[2 * u + 1];
+    out[2 * u + 1] = a[2 * u + 1] * b[2 * u] + a[2 * u] * b[2 * u + 1];
+  }
+}
+// Partial dot product of a lane's eight values, as two independent chains.
+__device__ __forceinline__ float dot8(const float* q, const float* x) {
+  float a = q[0] * x[0], b = q[4] * x[4];
+#pragma unroll
+  for (int c = 1; c < 4; ++c) {
+    a = fmaf(q[c], x[c], a);
+    b = fmaf(q[4 + c], x[4 + c], b);
+  }
+  return a + b;
+}
+// Two slot sums (over the LPR lanes of a row) with interleaved shuffles.
+template <int LPR>
+__device__ __forceinline__ void slot_sum2(float& a, float& b) {
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) {
+    const float ta = __shfl_xor_sync(0xffffffffu, a, o);
+    const float tb = __shfl_xor_sync(0xffffffffu, b, o);
+    a += ta;
+    b += tb;
+  }
+}
+
+// Shared-memory plan of one CTA (byte offsets), the same on host and device.
+struct Plan {
+  unsigned mb, qf, qtok, qlev, rrow, sc, wsc, wwin, mrg, kept, kfl, wbuf, kbuf, vbuf, total;
+  int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
+  unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
+};
+template <typename T, int D, int G, int HPC>
+__host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, int CS, int NRH,
+                                                   int B, int levels) {
+  constexpr unsigned RS = D + 2;
+  Plan q;
+  unsigned o = 0;
+  q.mb = o;   o += 256;                                   // mbarriers
+  q.qf = o;   o += G * D * 4;
+  q.qtok = o; o += G * D * 4;
+  q.qlev = o; o += unsigned(levels) * HPC * D * 4;        // query rotated per level
+  q.rrow = o; o += unsigned(levels + 2) * D * 4;          // RoPE table rows (cos, sin)
+  q.sc = o;   o += 2 * HPC * unsigned(cmax) * 4;
+  q.wsc = o;  o += kChainWarps * RS * 4;
+  q.wwin = o; o += kWinWarps * G * RS * 4;
+  q.mrg = o;  o += unsigned(CS) * HPC * RS * 4;
+  q.kept = o; o += 2 * HPC * unsigned(kmax) * 4;
+  q.kfl = o;  o += 2 * HPC * unsigned(cmax);
+  o = (o + 127u) & ~127u;
+  q.wbuf = o; o += kWinRing * 2 * kWinChunk * D * unsigned(sizeof(T));
+  o = (o + 127u) & ~127u;
+  q.kbuf = o;
+  q.rows = (cmax + S - 1) / S;
+  q.kbytes = HPC * unsigned(q.rows) * D * 4;
+  q.vbuf = o + q.kbytes;
+  const unsigned toks = HPC * unsigned(NRH) * 2 * unsigned(B) * D * unsigned(sizeof(T));
+  o += 2 * q.kbytes > toks ? 2 * q.kbytes : toks;
+  q.total = o;
+  return q;
+}
+
+template <typename T, int D, int G, int HPC>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                       const T* __restrict__ V, const void* __restrict__ tree,
                       const int64_t* __restrict__ len_dev, int n_q, T* __restrict__ O,
-                      int32_t* __restrict__ trace, int cmax, int kmax, int wrows,
+                      int32_t* __restrict__ trace, int cmax, int kmax, int S, int NRH,
                       StepArgs st) {
-  constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR, NSLOT = kWarps * SPW;
+  constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR;
+  constexpr int WPH = kChainWarps / HPC, HSLOT = WPH * SPW;
+  constexpr int WSL = kWinWarps * SPW;                 // window lane slots
+  constexpr int RS = D + 2;                            // merge row: acc[D], m, l
+  static_assert(kChainWarps % HPC == 0, "chain warps split evenly over the heads");
+  static_assert(kWinChunk % WSL == 0, "window slots advance evenly across chunks");
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = int(cluster.num_blocks());
   const int rank = int(cluster.block_rank());
+  const int hg = rank / S, sh = rank % S;              // head group, candidate share
   const int qi = blockIdx.y;
   const int64_t seq = blockIdx.z / p.hkv;
   const int g = int(blockIdx.z % p.hkv);
@@ -69,20 +323,29 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int sub = lane % LPR;
   const int j0 = 4 * sub;
 
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* qf = reinterpret_cast<float*>(smem);          // [G][D] raw query
-  float* qlev = qf + G * D;                            // [G][D] rotated to the level's c
-  float* qtok = qlev + G * D;                          // [G][D] rotated to n0 - 1
-  float* sc = qtok + G * D;                            // [2][G][cmax] scores
-  float* wsc = sc + 2 * G * cmax;                      // [kWarps][D + 2] warp merge
-  float* wwin = wsc + kWarps * (D + 2);                // [kWarps][G][D + 2] window partials
-  float* mrg = wwin + kWarps * G * (D + 2);            // [CS][G][D + 2] cluster merge (rank 0)
-  int* kept = reinterpret_cast<int*>(mrg + CS * G * (D + 2));   // [2][G][kmax]
-  unsigned char* kfl = reinterpret_cast<unsigned char*>(kept + 2 * G * kmax);  // [2][G][cmax]
-  // window rows of this CTA staged by cp.async: K then V, [wrows][D] each
-  T* winK = reinterpret_cast<T*>((reinterpret_cast<uintptr_t>(kfl + 2 * G * cmax) + 15) &
-                                 ~uintptr_t(15));
-  T* winV = winK + size_t(wrows) * D;
+  const Plan pl = make_plan<T, D, G, HPC>(cmax, kmax, S, CS, NRH, p.B, p.lay.levels);
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* mb_lev = reinterpret_cast<uint64_t*>(smem + pl.mb);   // level keys arrived
+  uint64_t* mb_val = mb_lev + 1;                                   // level values arrived
+  uint64_t* mb_ready = mb_lev + 2;             // [2] head group's scores by level parity (S > 1)
+  uint64_t* mb_win = mb_lev + 4;                                   // [kWinRing]
+  uint64_t* mb_tok = mb_win + kWinRing;                            // [HPC][NRH]
+  float* qf = reinterpret_cast<float*>(smem + pl.qf);       // [G][D] raw query
+  float* qtok = reinterpret_cast<float*>(smem + pl.qtok);   // [G][D] rotated to n0 - 1
+  float* qlev = reinterpret_cast<float*>(smem + pl.qlev);   // [levels][HPC][D] rotated to c_l
+  // RoPE table rows: [l - 1] = R(lo_l) (first candidate of this share at level
+  // l), [levels] = R(sh * B), [levels + 1] = R(S * B)
+  float* rrow = reinterpret_cast<float*>(smem + pl.rrow);
+  float* sc = reinterpret_cast<float*>(smem + pl.sc);       // [2][HPC][cmax] scores
+  float* wsc = reinterpret_cast<float*>(smem + pl.wsc);     // [kChainWarps][RS]
+  float* wwin = reinterpret_cast<float*>(smem + pl.wwin);   // [kWinWarps][G][RS]
+  float* mrg = reinterpret_cast<float*>(smem + pl.mrg);     // [CS][HPC][RS] received
+  int* kept = reinterpret_cast<int*>(smem + pl.kept);       // [2][HPC][kmax]
+  unsigned char* kfl = smem + pl.kfl;                       // [2][HPC][cmax]
+  T* wbuf = reinterpret_cast<T*>(smem + pl.wbuf);           // [kWinRing][2][kWinChunk][D]
+  float* kbuf = reinterpret_cast<float*>(smem + pl.kbuf);   // [HPC][rows][D] level keys
+  float* vbuf = reinterpret_cast<float*>(smem + pl.vbuf);   // [HPC][rows][D] level values
+  T* tbuf = reinterpret_cast<T*>(smem + pl.kbuf);           // [HPC][NRH][2][B][D] kept leaves
 
   // Fused step: the new token is appended at len (this kernel writes it and
   // pools what it completes), and the query sits on it.  A full sequence is
@@ -95,6 +358,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
   const bool empty = t < 0 || t >= p.cap;   // uniform over the cluster
   const float2* rope = rope_table(p, tree);
+  const int rmax = p.lay.rope_rows - 1;
   const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
   const int64_t a = empty ? 0 : s0 / p.B;
   int64_t vis[kMaxLevels + 2];
@@ -122,14 +386,144 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int nleaf = top > 0 ? cnt_k[1] : 0;
   const int64_t n_win = empty ? 0 : t + 1 - a * p.B;
   const int64_t n0 = int64_t(nleaf) * p.B + n_win;
+  const int64_t kvbase = (seq * p.hkv + g) * p.cap;
+  const float inv_sqrt_d = p.inv_sqrt_d;
+  const int tstride = kTraceHead + kMaxLevels * p.k;
+  unsigned* errw = tree_error_word(const_cast<void*>(tree));
+
+  // This CTA's share [lo, hi) of tot items split over the head group's S CTAs.
+  auto share = [&](int tot, int& lo, int& hi) {
+    const int ch = (tot + S - 1) / S;
+    lo = min(tot, sh * ch);
+    hi = min(tot, lo + ch);
+  };
+  // Window share of this CTA (rows of the whole cluster split by rank).
+  int w_lo = 0, w_hi = 0;
+  {
+    const int nw = int(n_win), ch = (nw + CS - 1) / CS;
+    w_lo = min(nw, rank * ch);
+    w_hi = min(nw, w_lo + ch);
+  }
+  const int nwr = w_hi - w_lo;
+  const int nwch = (nwr + kWinChunk - 1) / kWinChunk;
+  // kept leaves of this share (leaf ranks sh, sh + S, ...)
+  const int ntok = nleaf > sh ? (nleaf - sh + S - 1) / S : 0;
+
+  if (tid == 0) {
+    mbar_init(mb_lev, 1);
+    mbar_init(mb_val, 1);
+    mbar_init(mb_ready, unsigned(S));
+    mbar_init(mb_ready + 1, unsigned(S));
+    for (int i = 0; i < kWinRing; ++i) mbar_init(mb_win + i, 1);
+    for (int i = 0; i < HPC * NRH; ++i) mbar_init(mb_tok + i, 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (CS > 1) cluster_arrive_relaxed();   // waited on before the first remote access
+
+  // ---- producers (bulk copies) ----------------------------------------------
+  // Keys (or values) of level lev (this CTA's share [lo, hi) of the candidate
+  // list of each local head) into kbuf (vbuf), completing on mb_lev (mb_val).
+  // Run by one whole warp: lane 0 arms the barrier, the lanes copy one run
+  // each (the children of a kept node of level lev + 1, or the orphans; the
+  // top level is one run).
+  auto issue_level = [&](int lev, bool values) {
+    const int c = cnt_c[lev];
+    int lo, hi;
+    share(c, lo, hi);
+    const unsigned rb = D * 4;
+    uint64_t* mb = values ? mb_val : mb_lev;
+    float* dst = values ? vbuf : kbuf;
+    if (lane == 0) mbar_expect_tx(mb, unsigned(HPC) * unsigned(hi - lo) * rb);
+    __syncwarp();
+    if (hi <= lo) return;
+    const float* keys = values ? level_vals(p, const_cast<void*>(tree), lev, seq, g)
+                               : level_keys(p, const_cast<void*>(tree), lev, seq, g);
+    const int kup = lev < top ? cnt_k[lev + 1] : 0;
+    const int nch = p.b * kup;
+    const int orph0 = lev < top ? p.b * int(vis[lev + 1]) : 0;   // first orphan node
+    const int* keptu = kept + ((lev + 1) & 1) * HPC * kmax;
+    const int nrun = kup + 1;
+    for (int x = lane; x < HPC * nrun; x += 32) {
+      const int h = x / nrun, r = x % nrun;
+      int c0, c1, node0;
+      if (r < kup) {
+        c0 = r * p.b;
+        c1 = c0 + p.b;
+        node0 = keptu[h * kmax + r] * p.b;
+      } else {
+        c0 = nch;
+        c1 = c;
+        node0 = orph0;
+      }
+      const int a0 = max(c0, lo), a1 = min(c1, hi);
+      if (a1 > a0)
+        bulk_g2s(dst + (size_t(h) * pl.rows + (a0 - lo)) * D,
+                 keys + int64_t(node0 + (a0 - c0)) * D, unsigned(a1 - a0) * rb, mb);
+    }
+  };
+  // Window chunk ch (rows [ch * kWinChunk, ...) of this CTA's window share)
+  // into ring slot ch % kWinRing; the new token's row comes from k_new/v_new.
+  auto issue_win = [&](int ch) {
+    const int slot = ch % kWinRing;
+    const int r0 = ch * kWinChunk, r1 = min(nwr, r0 + kWinChunk);
+    const int nrow = r1 - r0;
+    const int64_t p0 = a * p.B + w_lo + r0;            // position of the first row
+    const bool newrow = do_append && p0 + nrow - 1 == t;
+    const int nk = newrow ? nrow - 1 : nrow;
+    const unsigned eb = D * unsigned(sizeof(T));
+    uint64_t* mb = mb_win + slot;
+    mbar_expect_tx(mb, 2u * unsigned(nrow) * eb);
+    T* dK = wbuf + size_t(slot) * 2 * kWinChunk * D;
+    T* dV = dK + size_t(kWinChunk) * D;
+    if (nk > 0) {
+      bulk_g2s(dK, K + (kvbase + p0) * D, unsigned(nk) * eb, mb);
+      bulk_g2s(dV, V + (kvbase + p0) * D, unsigned(nk) * eb, mb);
+    }
+    if (newrow) {
+      bulk_g2s(dK + size_t(nk) * D, knew, eb, mb);
+      bulk_g2s(dV + size_t(nk) * D, vnew, eb, mb);
+    }
+  };
+  // Kept leaf j of local head h's share (leaf rank sh + j * S) into its ring
+  // slot: B rows of K, then B rows of V.
+  auto issue_tok = [&](int h, int j) {
+    const int slot = j % NRH;
+    const int node = kept[1 * HPC * kmax + h * kmax + sh + j * S];   // level 1 = parity 1
+    const unsigned lb = unsigned(p.B) * D * unsigned(sizeof(T));
+    uint64_t* mb = mb_tok + h * NRH + slot;
+    mbar_expect_tx(mb, 2u * lb);
+    T* dK = tbuf + (size_t(h) * NRH + slot) * 2 * p.B * D;
+    bulk_g2s(dK, K + (kvbase + int64_t(node) * p.B) * D, lb, mb);
+    bulk_g2s(dK + size_t(p.B) * D, V + (kvbase + int64_t(node) * p.B) * D, lb, mb);
+  };
+
+  // Chain warps [h * WPH, (h + 1) * WPH) serve local query head h (global
+  // head hg * HPC + h); hs is the lane slot's index within the head's warps.
+  const int hw = warp / WPH;
+  const int hs = (warp % WPH) * SPW + lane / LPR;
+  // RoPE of the slot's first row and of its row step, for the recurrences
+  float cs_hs[8], cs_st[8];
+  if (p.rope && warp < kChainWarps) {
+    load_cs(rope, min(hs, rmax), HALF, j0, cs_hs);
+    load_cs(rope, min(HSLOT, rmax), HALF, j0, cs_st);
+  }
+
+  // First copies: the top level's keys and values (chain warps 0 and 1) and
+  // the first window chunks (the first window warp), before the query is
+  // loaded.
+  if (warp == 0 && top > 0) issue_level(top, false);
+  if (warp == 1 && top > 0) issue_level(top, true);
+  if (warp == kChainWarps && lane < kWinRing && lane < nwch) issue_win(lane);
 
   for (int x = tid; x < G * D; x += kThreads)
     qf[x] = empty ? 0.f : load_elem(Q, qrow + x, p.dtype);
   __syncthreads();
-  auto rotate_q = [&](float* dst, int64_t idx) {
-    for (int x = tid; x < G * HALF; x += kThreads) {
+  // qf rows [h0, h0 + nh) rotated to index idx into dst, by threads [0, nthr).
+  auto rotate_q = [&](float* dst, int h0, int nh, int64_t idx, int nthr) {
+    for (int x = tid; x < nh * HALF; x += nthr) {
       const int h = x / HALF, j = x % HALF;
-      const float x1 = qf[h * D + j], x2 = qf[h * D + j + HALF];
+      const float x1 = qf[(h0 + h) * D + j], x2 = qf[(h0 + h) * D + j + HALF];
       if (p.rope) {
         const float2 cs = rope[idx * HALF + j];
         dst[h * D + j] = x1 * cs.x - x2 * cs.y;
@@ -140,53 +534,40 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       }
     }
   };
-  if (!empty) rotate_q(qtok, n0 - 1 > 0 ? n0 - 1 : 0);
-
-  // Warps are specialised by head: warps [h * WPH, (h + 1) * WPH) serve query
-  // head h of the group, so every lane slot keeps one online-softmax state.
-  constexpr int WPH = kWarps / G, HSLOT = WPH * SPW;
-  const int hw = warp / WPH;                          // this warp's head
-  const int hs = (warp % WPH) * SPW + lane / LPR;     // slot index within the head's warps
-  float m = -INFINITY, l = 0.f, acc[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  auto fold = [&](float s, const float* v) {
-    if (s > m) {
-      const float r = __expf(m - s);
-      l = l * r + 1.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
-      m = s;
-    } else {
-      const float w = __expf(s - m);
-      l += w;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
+  if (!empty) rotate_q(qtok, 0, G, n0 - 1 > 0 ? n0 - 1 : 0, kThreads);
+  for (int lev = 1; lev <= top; ++lev)
+    rotate_q(qlev + (lev - 1) * HPC * D, hg * HPC, HPC, cnt_c[lev], kThreads);
+  if (p.rope) {
+    // table rows the chain seeds its RoPE recurrences from
+    for (int x = tid; x < (top + 2) * HALF; x += kThreads) {
+      const int r = x / HALF, j = x % HALF;
+      int idx;
+      if (r < top) {
+        int lo, hi;
+        share(cnt_c[r + 1], lo, hi);
+        idx = lo;
+      } else {
+        idx = r == top ? sh * p.B : S * p.B;
+      }
+      const float2 cs = rope[int64_t(min(idx, rmax)) * HALF + j];
+      float* dst = rrow + (r < top ? r : p.lay.levels + (r - top)) * D;
+      dst[2 * j] = cs.x;
+      dst[2 * j + 1] = cs.y;
     }
-  };
+  }
+  for (int x = tid; x < kWinWarps * G * RS; x += kThreads)
+    wwin[x] = (x % RS == D) ? -INFINITY : 0.f;
+  __syncthreads();
+  if (CS > 1) cluster_wait();
+  bool timed_out = false;   // a bounded wait of this thread expired
 
-  const int64_t kvbase = (seq * p.hkv + g) * p.cap;
-  const float inv_sqrt_d = p.inv_sqrt_d;
-  const int tstride = kTraceHead + kMaxLevels * p.k;
-
-  // Node id of candidate i of head h at level lev (kept list of lev + 1 in kept[par]).
-  auto cand_node = [&](int lev, int h, int i) -> int {
-    const int kup = lev < top ? cnt_k[lev + 1] : 0;
-    const int vup = lev < top ? int(vis[lev + 1]) : 0;
-    if (i < p.b * kup)
-      return kept[((lev + 1) & 1) * G * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
-    return p.b * vup + (i - p.b * kup);
-  };
-  auto share = [&](int tot, int& lo, int& hi) {
-    const int ch = (tot + CS - 1) / CS;
-    lo = min(tot, rank * ch);
-    hi = min(tot, lo + ch);
-  };
-
-  // Window rows [w_lo, w_hi): every slot of the CTA takes rows, each row is
-  // loaded, rotated and scored once for all G heads.  The per-slot state of
-  // all heads is merged across the warp and left in wwin[warp][G].
-  auto window_loop = [&](int w_lo, int w_hi) {
+  // ---- window warps ---------------------------------------------------------
+  // Rows of this CTA's window share, scored once for all G heads of the group
+  // (each lane slot keeps one online softmax per head), chunk by chunk through
+  // the ring; the warp's per-head partials end in wwin.
+  auto window_warps = [&]() {
+    const int wl = warp - kChainWarps;
+    const int gsl = wl * SPW + lane / LPR;
     float mW[G], lW[G], accW[G][8];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -195,32 +576,32 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
 #pragma unroll
       for (int c = 0; c < 8; ++c) accW[h][c] = 0.f;
     }
-    const int nw = w_hi - w_lo;
+    // a slot's rows are gsl, gsl + WSL, ... across all chunks: its RoPE
+    // index grows by WSL per row, so its (cos, sin) advance by a fixed step
     const int widx0 = nleaf * p.B + w_lo;
-    const int gslot = warp * SPW + lane / LPR;
-    // Rows come from the staged copy in shared memory; the slot's RoPE index
-    // grows by NSLOT per row, so its (cos, sin) advance by a fixed rotation.
     float csc[8], cstep[8];
-    const int rmax = p.lay.rope_rows - 1;
-    const bool recur = NSLOT <= rmax;   // the step rotation is a table row
-    if (p.rope && recur) {
-      load_cs(rope, min(widx0 + gslot, rmax), HALF, j0, csc);
-      load_cs(rope, NSLOT, HALF, j0, cstep);
+    const bool recur = WSL <= rmax;
+    if (p.rope && recur && nwch > 0) {
+      load_cs(rope, min(widx0 + gsl, rmax), HALF, j0, csc);
+      load_cs(rope, WSL, HALF, j0, cstep);
     }
-    for (int base = 0; base < nw; base += NSLOT) {
-      {
-        const int e = base + gslot;
-        const bool on = e < nw;
+    for (int ch = 0; ch < nwch; ++ch) {
+      const int slot = ch % kWinRing;
+      mbar_wait(mb_win + slot, unsigned(ch / kWinRing) & 1u, timed_out);
+      const T* cK = wbuf + size_t(slot) * 2 * kWinChunk * D;
+      const T* cV = cK + size_t(kWinChunk) * D;
+#pragma unroll 1
+      for (int e = gsl; e < kWinChunk; e += WSL) {
+        const int r = ch * kWinChunk + e;
+        const bool on = r < nwr;
         float xk[8], xv[8];
-        const int ee = on ? e : 0;
-        SharedPairs<T, HALF>::load(winK + size_t(ee) * D, j0, xk);
-        SharedPairs<T, HALF>::load(winV + size_t(ee) * D, j0, xv);
+        SharedPairs<T, HALF>::load(cK + size_t(e) * D, j0, xk);
+        SharedPairs<T, HALF>::load(cV + size_t(e) * D, j0, xv);
         if (p.rope) {
-          if (!recur) load_cs(rope, min(widx0 + e, rmax), HALF, j0, csc);
+          if (!recur) load_cs(rope, min(widx0 + r, rmax), HALF, j0, csc);
           rotate8(xk, csc);
           if (recur) advance_cs(csc, cstep);
         }
-        const bool on_u = on;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           const float* qv = qtok + h * D;
@@ -231,42 +612,21 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
             s = fmaf(qv[HALF + j0 + c], xk[4 + c], s);
           }
           s = slot_sum<LPR>(s) * inv_sqrt_d;
-          if (on_u) {
-            if (s > mW[h]) {
-              const float r = __expf(mW[h] - s);
-              lW[h] = lW[h] * r + 1.f;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) accW[h][c] = fmaf(accW[h][c], r, xv[c]);
-              mW[h] = s;
-            } else {
-              const float w = __expf(s - mW[h]);
-              lW[h] += w;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) accW[h][c] = fmaf(w, xv[c], accW[h][c]);
-            }
-          }
+          if (on) fold8(mW[h], lW[h], accW[h], s, xv);
         }
+      }
+      named_sync(kBarWindow, kWinWarps * 32);
+      if (warp == kChainWarps && lane == 0 && ch + kWinRing < nwch) {
+        fence_proxy_async();
+        issue_win(ch + kWinRing);
       }
     }
 #pragma unroll
     for (int h = 0; h < G; ++h) {
 #pragma unroll
-      for (int o = LPR; o < 32; o <<= 1) {
-        const float mo = __shfl_xor_sync(0xffffffffu, mW[h], o);
-        const float lo = __shfl_xor_sync(0xffffffffu, lW[h], o);
-        const float mn = fmaxf(mW[h], mo);
-        const float ra_ = (mW[h] == -INFINITY) ? 0.f : __expf(mW[h] - mn);
-        const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
-        lW[h] = lW[h] * ra_ + lo * rb_;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float ao = __shfl_xor_sync(0xffffffffu, accW[h][c], o);
-          accW[h][c] = accW[h][c] * ra_ + ao * rb_;
-        }
-        mW[h] = mn;
-      }
+      for (int o = LPR; o < 32; o <<= 1) merge_xor(mW[h], lW[h], accW[h], o);
       if (lane < LPR) {
-        float* w = wwin + (warp * G + h) * (D + 2);
+        float* w = wwin + (wl * G + h) * RS;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           w[j0 + c] = accW[h][c];
@@ -280,381 +640,399 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     }
   };
 
-  // Tree rows of head hw (this CTA's share): the key candidates of level klev
-  // (scored, scores broadcast to every CTA) and the unselected candidates of
-  // level vlev (values folded into the softmax).
-  auto tree_loop = [&](int klev, int vlev) {
-    int k_lo = 0, k_hi = 0, v_lo = 0, v_hi = 0;
-    if (klev > 0) share(cnt_c[klev], k_lo, k_hi);
-    if (vlev > 0) share(cnt_c[vlev], v_lo, v_hi);
-    const int nk = k_hi - k_lo, nv = v_hi - v_lo, total = nk + nv;
-    const float* keys = klev > 0 ? level_keys(p, const_cast<void*>(tree), klev, seq, g) : nullptr;
-    const float* vals = vlev > 0 ? level_vals(p, const_cast<void*>(tree), vlev, seq, g) : nullptr;
-    const int kupK = (klev > 0 && klev < top) ? cnt_k[klev + 1] : 0;
-    const int nchK = p.b * kupK;
-    const int orphK = (klev > 0 && klev < top) ? p.b * int(vis[klev + 1]) - nchK : 0;
-    const int* keptK = kept + ((klev + 1) & 1) * G * kmax + hw * kmax;
-    const int kupV = (vlev > 0 && vlev < top) ? cnt_k[vlev + 1] : 0;
-    const int nchV = p.b * kupV;
-    const int orphV = (vlev > 0 && vlev < top) ? p.b * int(vis[vlev + 1]) - nchV : 0;
-    const int* keptV = kept + ((vlev + 1) & 1) * G * kmax + hw * kmax;
-    const float* scV = sc + (vlev & 1) * G * cmax + hw * cmax;
-    const unsigned char* flV = kfl + (vlev & 1) * G * cmax + hw * cmax;
-    float* scK = sc + (klev & 1) * G * cmax + hw * cmax;
-    const float* ql = qlev + hw * D;
-    // key items step their RoPE index by HSLOT per slot: seeded once per batch
-    const int rmax = p.lay.rope_rows - 1;
-    float cstep[8];
-    if (p.rope) load_cs(rope, HSLOT, HALF, j0, cstep);
-    for (int base = 0; base < total; base += HSLOT * kUnroll) {
-      RawPairs ra[kUnroll];
-      float csc[8];
-      int kind[kUnroll], idx[kUnroll];
-      if (p.rope) load_cs(rope, min(k_lo + base + hs, rmax), HALF, j0, csc);
-      float sv[kUnroll];
+  // ---- chain warps ----------------------------------------------------------
+  // Every lane slot of a chain warp keeps one online-softmax state of its head.
+  float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e = base + u * HSLOT + hs;
-        kind[u] = kNone;
-        idx[u] = 0;
-        sv[u] = 0.f;
-        if (e < nk) {
-          const int i = k_lo + e;
-          const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
-          kind[u] = kKey;
-          idx[u] = i;
-          RawLoad<float, HALF>::load(keys + int64_t(node) * D, j0, ra[u]);
-        } else if (e < total) {
-          const int i = v_lo + (e - nk);
-          if (!flV[i]) {
-            const int node = i < nchV ? keptV[div_b(p, i)] * p.b + mod_b(p, i) : orphV + i;
-            kind[u] = kVal;
-            sv[u] = scV[i];
-            RawLoad<float, HALF>::load(vals + int64_t(node) * D, j0, ra[u]);
-          }
-        }
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+
+  // Node id of candidate i of local head h at level lev (kept list of lev + 1).
+  auto cand_node = [&](int lev, int h, int i) -> int {
+    const int kup = lev < top ? cnt_k[lev + 1] : 0;
+    const int vup = lev < top ? int(vis[lev + 1]) : 0;
+    if (i < p.b * kup)
+      return kept[((lev + 1) & 1) * HPC * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
+    return p.b * vup + (i - p.b * kup);
+  };
+
+  // Scores of this CTA's share of level lev's candidates (keys in kbuf) for
+  // head hw, two rows per slot at a time; with S > 1 each score is stored
+  // into every CTA of the group.  A slot's rows are lo + hs + i * HSLOT, so
+  // its (cos, sin) start at R(lo) R(hs) and advance by R(HSLOT) per row.
+  auto score_level = [&](int lev) {
+    int lo, hi;
+    share(cnt_c[lev], lo, hi);
+    const int nr = hi - lo;
+    const float* kb = kbuf + size_t(hw) * pl.rows * D;
+    float* scK = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
+    float q[8];
+    lds_pairs(qlev + ((lev - 1) * HPC + hw) * D, j0, HALF, q);
+    float csa[8], st2[8];
+    if (p.rope) {
+      if (S == 1) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) csa[c] = cs_hs[c];
+      } else {
+        float r[8];
+        lds_cs8(rrow + (lev - 1) * D, j0, r);
+        cmul8(csa, r, cs_hs);
       }
+      cmul8(st2, cs_st, cs_st);
+    }
+    for (int e = hs; e - hs < nr; e += 2 * HSLOT) {
+      const int e1 = e + HSLOT;
+      const bool on0 = e < nr, on1 = e1 < nr;
+      float x0[8], x1[8];
+      SharedPairs<float, HALF>::load(kb + size_t(on0 ? e : 0) * D, j0, x0);
+      SharedPairs<float, HALF>::load(kb + size_t(on1 ? e1 : 0) * D, j0, x1);
+      if (p.rope) {
+        float csb[8];
+        cmul8(csb, csa, cs_st);
+        rotate8(x0, csa);
+        rotate8(x1, csb);
+        float t2[8];
+        cmul8(t2, csa, st2);
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        float x[8], s = 0.f;
-        RawLoad<float, HALF>::cvt(ra[u], x);
-        if (kind[u] == kKey && p.rope) rotate8(x, csc);
-        if (p.rope) advance_cs(csc, cstep);
-        if (kind[u] == kKey) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            s = fmaf(ql[j0 + c], x[c], s);
-            s = fmaf(ql[HALF + j0 + c], x[4 + c], s);
-          }
+        for (int c = 0; c < 8; ++c) csa[c] = t2[c];
+      }
+      float s0 = dot8(q, x0), s1 = dot8(q, x1);
+      slot_sum2<LPR>(s0, s1);
+      s0 *= inv_sqrt_d;
+      s1 *= inv_sqrt_d;
+      if (S == 1) {
+        if (sub == 0) {
+          if (on0) scK[e] = s0;
+          if (on1) scK[e1] = s1;
         }
-        if (__any_sync(0xffffffffu, kind[u] == kKey)) s = slot_sum<LPR>(s) * inv_sqrt_d;
-        if (kind[u] == kKey) {
-          float* dstp = scK + idx[u];
-          if (sub < CS) *cluster.map_shared_rank(dstp, sub) = s;
-          if (sub + LPR < CS) *cluster.map_shared_rank(dstp, sub + LPR) = s;
-        } else if (kind[u] == kVal) {
-          fold(sv[u], x);
+      } else {
+        if (sub < S) {
+          if (on0) *cluster.map_shared_rank(scK + e, hg * S + sub) = s0;
+          if (on1) *cluster.map_shared_rank(scK + e1, hg * S + sub) = s1;
+        }
+        if (sub + LPR < S) {
+          if (on0) *cluster.map_shared_rank(scK + e, hg * S + sub + LPR) = s0;
+          if (on1) *cluster.map_shared_rank(scK + e1, hg * S + sub + LPR) = s1;
         }
       }
     }
   };
 
-  // Kept-leaf tokens of head hw (this CTA's share), after level 1's top-k.
-  auto token_loop = [&]() {
-    int t_lo = 0, t_hi = 0;
-    share(nleaf * p.B, t_lo, t_hi);
-    const int nt = t_hi - t_lo;
-    const int* kept1 = kept + 1 * G * kmax + hw * kmax;           // level 1 = parity 1
-    const float* qt = qtok + hw * D;
-    const int rmax = p.lay.rope_rows - 1;
-    float cstep[8];
-    if (p.rope) load_cs(rope, HSLOT, HALF, j0, cstep);
-    for (int base = 0; base < nt; base += HSLOT * kTokUnroll) {
-      TokRow<T, HALF> rk[kTokUnroll], rv[kTokUnroll];
-      float csc[8];
-      bool on[kTokUnroll];
-      if (p.rope) load_cs(rope, min(t_lo + base + hs, rmax), HALF, j0, csc);
-#pragma unroll
-      for (int u = 0; u < kTokUnroll; ++u) {
-        const int e = base + u * HSLOT + hs;
-        on[u] = e < nt;
-        if (on[u]) {
-          const int r = t_lo + e;
-          const int pos = kept1[div_B(p, r)] * p.B + mod_B(p, r);
-          rk[u].load(K + (kvbase + pos) * D, j0);
-          rv[u].load(V + (kvbase + pos) * D, j0);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kTokUnroll; ++u) {
-        float xk[8], xv[8], s = 0.f;
-        rk[u].cvt(xk);
-        rv[u].cvt(xv);
-        if (p.rope) {
-          rotate8(xk, csc);
-          advance_cs(csc, cstep);
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          s = fmaf(qt[j0 + c], xk[c], s);
-          s = fmaf(qt[HALF + j0 + c], xk[4 + c], s);
-        }
-        s = slot_sum<LPR>(s) * inv_sqrt_d;
-        if (on[u]) fold(s, xv);
-      }
+  // Values of this CTA's share of level lev's unselected candidates (head
+  // hw, rows in vbuf in candidate order), folded two rows at a time.
+  auto fold_values = [&](int lev) {
+    int lo, hi;
+    share(cnt_c[lev], lo, hi);
+    const int nr = hi - lo;
+    const float* vb = vbuf + size_t(hw) * pl.rows * D;
+    const float* scV = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
+    const unsigned char* flV = kfl + (lev & 1) * HPC * cmax + hw * cmax + lo;
+    for (int e = hs; e < nr; e += 2 * HSLOT) {
+      const int e1 = e + HSLOT;
+      const bool on0 = !flV[e], on1 = e1 < nr && !flV[e1];
+      float x0[8], x1[8];
+      SharedPairs<float, HALF>::load(vb + size_t(e) * D, j0, x0);
+      SharedPairs<float, HALF>::load(vb + size_t(on1 ? e1 : e) * D, j0, x1);
+      fold2(m, l, acc, scV[e], on0, x0, on1 ? scV[e1] : 0.f, on1, x1);
     }
   };
 
-  auto run_pass = [&](int w_lo, int w_hi, int klev, int vlev, bool tokens) {
-    if (w_hi > w_lo) {
-      cp_async_wait_all();
-      __syncthreads();
-      window_loop(w_lo, w_hi);
-    }
-    if (klev > 0 || vlev > 0) tree_loop(klev, vlev);
-    if (tokens) token_loop();
-  };
 
-  // Top-k of head h at level lev over the full score table (every CTA runs
-  // the same selection on the same broadcast scores).  One warp per head
-  // takes kap rounds of a warp arg-max: lane l holds the order-preserving
-  // keys of candidates l, l + 32, ... in registers (0 = none or taken; every
-  // finite score maps above 0); redux.sync gives the round's maximum, a
-  // ballot the lanes holding it, and on a tie of keys across lanes the lowest
-  // index wins (within a lane the lowest slot).  Bit s of `taken` marks
-  // candidate 32 s + l as kept.  Candidates beyond 32 * kRegSlots are read
-  // from shared memory in the same rounds.  The kept list is compacted in
-  // index order with one ballot per slot row.  The selecting warp of head h
-  // is h * WPH + (h % 4), so the G selections run on different schedulers.
+  // Top-k of local head h = warp (warps 0 .. HPC - 1) at level lev over the
+  // head's full score table (with S > 1 every CTA of the head group runs the
+  // same selection on the same scores).  kap rounds of a warp arg-max: lane l
+  // holds the order-preserving keys of candidates l, l + 32, ... in registers
+  // (0 = none or taken; every finite score maps above 0); redux.sync gives
+  // the round's maximum, a ballot the lanes holding it, and on a tie of keys
+  // across lanes the lowest index wins (within a lane the lowest slot).  Bit
+  // s of `taken` marks candidate 32 s + l as kept.  Candidates beyond
+  // 32 * kRegSlots are read from shared memory in the same rounds.  The kept
+  // list is compacted in index order with one ballot per slot row.
   auto topk = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
-    if (warp == hw * WPH + (hw & 3) % WPH) {
-      const int h = hw;
-      const float* row = sc + par * G * cmax + h * cmax;
-      const int ns = (c + 31) >> 5;
-      unsigned taken = 0;
-      if (kap >= c) {
-        for (int s = 0; s < ns; ++s)
-          if (s * 32 + lane < c) taken |= 1u << s;
-      } else {
-        unsigned key[kRegSlots];
+    const int h = warp;
+    const float* row = sc + par * HPC * cmax + h * cmax;
+    const int ns = (c + 31) >> 5;
+    unsigned taken = 0;
+    if (kap >= c) {
+      for (int s = 0; s < ns; ++s)
+        if (s * 32 + lane < c) taken |= 1u << s;
+    } else {
+      unsigned key[kRegSlots];
 #pragma unroll
-        for (int s = 0; s < kRegSlots; ++s) {
+      for (int s = 0; s < kRegSlots; ++s) {
+        const int i = s * 32 + lane;
+        key[s] = i < c ? order_key(row[i]) : 0u;
+      }
+      for (int r = 0; r < kap; ++r) {
+        unsigned bk = key[0];
+        int bs = 0;
+#pragma unroll
+        for (int s = 1; s < kRegSlots; ++s)
+          if (key[s] > bk) {
+            bk = key[s];
+            bs = s;
+          }
+        for (int s = kRegSlots; s < ns; ++s) {
           const int i = s * 32 + lane;
-          key[s] = i < c ? order_key(row[i]) : 0u;
-        }
-        for (int r = 0; r < kap; ++r) {
-          unsigned bk = key[0];
-          int bs = 0;
-#pragma unroll
-          for (int s = 1; s < kRegSlots; ++s)
-            if (key[s] > bk) {
-              bk = key[s];
+          if (i < c && !((taken >> s) & 1u)) {
+            const unsigned kk = order_key(row[i]);
+            if (kk > bk) {
+              bk = kk;
               bs = s;
             }
-          for (int s = kRegSlots; s < ns; ++s) {
-            const int i = s * 32 + lane;
-            if (i < c && !((taken >> s) & 1u)) {
-              const unsigned kk = order_key(row[i]);
-              if (kk > bk) {
-                bk = kk;
-                bs = s;
-              }
-            }
           }
-          const unsigned M = __reduce_max_sync(0xffffffffu, bk);
-          unsigned who = __ballot_sync(0xffffffffu, bk == M);
-          if (__popc(who) > 1) {
-            const unsigned I =
-                __reduce_min_sync(0xffffffffu, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
-            who = 1u << (I & 31u);
-          }
-          if ((who >> lane) & 1u) {
-            taken |= 1u << bs;
+        }
+        const unsigned M = __reduce_max_sync(0xffffffffu, bk);
+        unsigned who = __ballot_sync(0xffffffffu, bk == M);
+        if (__popc(who) > 1) {
+          const unsigned I =
+              __reduce_min_sync(0xffffffffu, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
+          who = 1u << (I & 31u);
+        }
+        if ((who >> lane) & 1u) {
+          taken |= 1u << bs;
 #pragma unroll
-            for (int s = 0; s < kRegSlots; ++s)
-              if (s == bs) key[s] = 0u;
-          }
-        }
-      }
-      unsigned char* fl = kfl + par * G * cmax + h * cmax;
-      int* kp = kept + par * G * kmax + h * kmax;
-      int cnt = 0;
-      for (int s = 0; s < ns; ++s) {
-        const int i = s * 32 + lane;
-        const bool f = i < c && ((taken >> s) & 1u);
-        if (i < c) fl[i] = f;
-        const unsigned bal = __ballot_sync(0xffffffffu, f);
-        if (f) {
-          const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
-          const int node = cand_node(lev, h, i);
-          kp[pos] = node;
-          if (trace && rank == 0) {
-            const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
-            trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
-          }
-          // The next pass reads this node's children (keys and values one
-          // level down) or, at level 1, its tokens: start pulling them into
-          // L2 now, one bulk prefetch per contiguous run, spread over the
-          // cluster's CTAs.
-          if ((h * kmax + pos) % CS == rank) {
-            if (lev > 1) {
-              const unsigned bytes = unsigned(p.b) * D * 4;
-              prefetch_l2(level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) +
-                              int64_t(node) * p.b * D, bytes);
-              prefetch_l2(level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) +
-                              int64_t(node) * p.b * D, bytes);
-            } else {
-              const unsigned bytes = unsigned(p.B) * D * unsigned(sizeof(T));
-              prefetch_l2(K + (kvbase + int64_t(node) * p.B) * D, bytes);
-              prefetch_l2(V + (kvbase + int64_t(node) * p.B) * D, bytes);
-            }
-          }
-        }
-        cnt += __popc(bal);
-      }
-      // orphans one level down (shared by every head)
-      if (lev > 1 && h == 0 && lane == 0 && rank == (CS - 1)) {
-        const int64_t o0 = int64_t(p.b) * vis[lev], o1 = vis[lev - 1];
-        if (o1 > o0) {
-          const unsigned bytes = unsigned(o1 - o0) * D * 4;
-          prefetch_l2(level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) + o0 * D, bytes);
-          prefetch_l2(level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) + o0 * D, bytes);
+          for (int s = 0; s < kRegSlots; ++s)
+            if (s == bs) key[s] = 0u;
         }
       }
     }
-    __syncthreads();
+    unsigned char* fl = kfl + par * HPC * cmax + h * cmax;
+    int* kp = kept + par * HPC * kmax + h * kmax;
+    int cnt = 0;
+    for (int s = 0; s < ns; ++s) {
+      const int i = s * 32 + lane;
+      const bool f = i < c && ((taken >> s) & 1u);
+      if (i < c) fl[i] = f;
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (f) {
+        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        const int node = cand_node(lev, h, i);
+        kp[pos] = node;
+        if (trace && sh == 0) {
+          const int64_t rec =
+              ((seq * n_q + qi) * p.hq + int64_t(g) * G + hg * HPC + h) * tstride;
+          trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
+        }
+      }
+      cnt += __popc(bal);
+    }
   };
 
-  // Window share of this CTA (independent of the selection).
-  int w_lo = 0, w_hi = 0;
-  {
-    const int nw = int(n_win), ch = (nw + CS - 1) / CS;
-    w_lo = min(nw, rank * ch);
-    w_hi = min(nw, w_lo + ch);
-  }
-  const bool has_win = w_hi > w_lo;
-  // the top level's candidates (keys and values), pulled into L2 by rank 0
-  if (top > 0 && rank == 0 && tid == 0) {
-    const unsigned bytes = unsigned(vis[top]) * D * 4;
-    prefetch_l2(level_keys(p, const_cast<void*>(tree), top, seq, g), bytes);
-    prefetch_l2(level_vals(p, const_cast<void*>(tree), top, seq, g), bytes);
-  }
-  // Stage this CTA's window rows now: they do not depend on the selection,
-  // so the copies are in flight during the first level pass.
-  {
-    constexpr int CPR = D * int(sizeof(T)) / 16;       // 16-byte pieces per row
-    const int rows = w_hi - w_lo;
-    const int64_t row0 = kvbase + int64_t(a) * p.B + w_lo;
-    const int64_t tnew = do_append ? t - (int64_t(a) * p.B + w_lo) : -1;   // new token's row
-    for (int x = tid; x < rows * CPR; x += kThreads) {
-      const int r = x / CPR, c = x % CPR;
-      const T* ks = r == tnew ? knew : K + (row0 + r) * D;
-      const T* vs = r == tnew ? vnew : V + (row0 + r) * D;
-      cp_async16(reinterpret_cast<char*>(winK + size_t(r) * D) + c * 16,
-                 reinterpret_cast<const char*>(ks) + c * 16);
-      cp_async16(reinterpret_cast<char*>(winV + size_t(r) * D) + c * 16,
-                 reinterpret_cast<const char*>(vs) + c * 16);
+  // Level barrier: the head group's scores of this level are complete and
+  // visible in this CTA.  With S > 1 every CTA of the group arrives on the
+  // group's "ready" barrier of the level's parity: a CTA can be at most one
+  // level ahead of another (it waits for everyone's arrival), so alternating
+  // two barriers keeps the arrivals of consecutive levels apart.
+  int use = 0;   // levels passed (mb_lev phase; mb_ready[use & 1] phase use / 2)
+  auto level_sync = [&]() {
+    if (S == 1) {
+      named_sync(kBarChain, kChainThreads);
+    } else {
+      fence_cluster();
+      named_sync(kBarChain, kChainThreads);
+      uint64_t* rb = mb_ready + (use & 1);
+      if (tid < S) mbar_arrive_remote(rb, hg * S + tid);
+      mbar_wait(rb, unsigned(use >> 1) & 1u, timed_out);
     }
-    cp_async_commit();
-  }
-  if (top > 0) {
-    rotate_q(qlev, cnt_c[top]);
-    __syncthreads();
-    run_pass(w_lo, w_hi, top, 0, false);
-    cluster.sync();
-    topk(top);
-    for (int lev = top - 1; lev >= 1; --lev) {
-      rotate_q(qlev, cnt_c[lev]);
-      __syncthreads();
-      run_pass(0, 0, lev, lev + 1, false);
-      cluster.sync();
-      topk(lev);
-    }
-    run_pass(0, 0, 0, 1, true);
-  } else {
-    run_pass(w_lo, w_hi, 0, 0, false);
-  }
+  };
 
-  // Merge: slots of a warp, then the warps of each head, then the cluster
-  // (into rank 0).
-#pragma unroll
-  for (int o = LPR; o < 32; o <<= 1) {
-    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
-    const float lo = __shfl_xor_sync(0xffffffffu, l, o);
-    const float mn = fmaxf(m, mo);
-    const float ra_ = (m == -INFINITY) ? 0.f : __expf(m - mn);
-    const float rb_ = (mo == -INFINITY) ? 0.f : __expf(mo - mn);
-    l = l * ra_ + lo * rb_;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      const float ao = __shfl_xor_sync(0xffffffffu, acc[c], o);
-      acc[c] = acc[c] * ra_ + ao * rb_;
+  // Kept-leaf tokens of head hw through its ring of NRH slots, two rows per
+  // slot at a time.  Leaf j of the share has rank sh + j * S, so its row e
+  // sits at RoPE index (sh + j * S) * B + e: the seed R((sh + j S) B) advances
+  // by R(S B) per leaf and is combined with the slot's R(hs).
+  auto token_pass = [&]() {
+    float q[8];
+    lds_pairs(qtok + (hg * HPC + hw) * D, j0, HALF, q);
+    const unsigned lbar = kBarHead0 + hw;
+    float rj[8], st2[8];
+    if (p.rope) {
+      lds_cs8(rrow + p.lay.levels * D, j0, rj);
+      cmul8(st2, cs_st, cs_st);
     }
-    m = mn;
+    const size_t slot_elems = size_t(2) * p.B * D;
+    for (int j = 0; j < ntok; ++j) {
+      const int slot = j % NRH;
+      mbar_wait(mb_tok + hw * NRH + slot, unsigned(j / NRH) & 1u, timed_out);
+      const T* cK = tbuf + (size_t(hw) * NRH + slot) * slot_elems;
+      const T* cV = cK + size_t(p.B) * D;
+      float csa[8];
+      if (p.rope) {
+        cmul8(csa, rj, cs_hs);
+        float r[8], t2[8];
+        lds_cs8(rrow + (p.lay.levels + 1) * D, j0, r);
+        cmul8(t2, rj, r);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) rj[c] = t2[c];
+      }
+      for (int e = hs; e - hs < p.B; e += 2 * HSLOT) {
+        const int e1 = e + HSLOT;
+        const bool on0 = e < p.B, on1 = e1 < p.B;
+        const int r0 = on0 ? e : 0, r1 = on1 ? e1 : 0;
+        float k0[8], k1[8], v0[8], v1[8];
+        SharedPairs<T, HALF>::load(cK + size_t(r0) * D, j0, k0);
+        SharedPairs<T, HALF>::load(cK + size_t(r1) * D, j0, k1);
+        SharedPairs<T, HALF>::load(cV + size_t(r0) * D, j0, v0);
+        SharedPairs<T, HALF>::load(cV + size_t(r1) * D, j0, v1);
+        if (p.rope) {
+          float csb[8];
+          cmul8(csb, csa, cs_st);
+          rotate8(k0, csa);
+          rotate8(k1, csb);
+          float t2[8];
+          cmul8(t2, csa, st2);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) csa[c] = t2[c];
+        }
+        float s0 = dot8(q, k0), s1 = dot8(q, k1);
+        slot_sum2<LPR>(s0, s1);
+        fold2(m, l, acc, s0 * inv_sqrt_d, on0, v0, s1 * inv_sqrt_d, on1, v1);
+      }
+      named_sync(lbar, WPH * 32);
+      if (warp == hw * WPH && lane == 0 && j + NRH < ntok) {
+        fence_proxy_async();
+        issue_tok(hw, j + NRH);
+      }
+    }
+  };
+
+  // Slot s of local head h lies inside kbuf (free once the level-1 keys are
+  // scored) rather than reaching into vbuf (free once the level-1 values are
+  // folded).
+  auto early_slot = [&](int h, int s) {
+    const size_t sb = size_t(2) * p.B * D * sizeof(T);
+    return (size_t(h) * NRH + s + 1) * sb <= pl.kbytes;
+  };
+  auto chain_warps = [&]() {
+    for (int lev = top; lev >= 1; --lev) {
+      mbar_wait(mb_lev, unsigned(use) & 1u, timed_out);
+      score_level(lev);
+      level_sync();
+      const int u = use++;
+      if (warp < HPC) topk(lev);
+      named_sync(kBarChain, kChainThreads);
+      if (lev > 1) {
+        if (warp == 0) {
+          if (lane == 0) fence_proxy_async();
+          __syncwarp();
+          issue_level(lev - 1, false);
+        }
+      } else if (warp % WPH == 0 && lane == 0) {
+        fence_proxy_async();
+        for (int j = 0; j < NRH && j < ntok; ++j)
+          if (early_slot(hw, j)) issue_tok(hw, j);
+      }
+      mbar_wait(mb_val, unsigned(u) & 1u, timed_out);
+      fold_values(lev);
+      named_sync(kBarChain, kChainThreads);
+      if (lev > 1) {
+        if (warp == 1) {
+          if (lane == 0) fence_proxy_async();
+          __syncwarp();
+          issue_level(lev - 1, true);
+        }
+      } else if (warp % WPH == 0 && lane == 0) {
+        fence_proxy_async();
+        for (int j = 0; j < NRH && j < ntok; ++j)
+          if (!early_slot(hw, j)) issue_tok(hw, j);
+      }
+    }
+    if (top > 0) token_pass();
+  };
+
+
+  if (warp >= kChainWarps)
+    window_warps();
+  else
+    chain_warps();
+
+  // ---- merge ----------------------------------------------------------------
+  // The slots of a chain warp, then per head the head's chain warps plus the
+  // window partials; each CTA sends its contribution for every head of the
+  // group to the head's owner (share 0 of its head group), which combines the
+  // CS contributions and writes O.
+  if (warp < kChainWarps) {
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1) merge_xor(m, l, acc, o);
+    if (lane < LPR) {
+      float* w = wsc + warp * RS;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        w[j0 + c] = acc[c];
+        w[HALF + j0 + c] = acc[4 + c];
+      }
+      if (lane == 0) {
+        w[D] = m;
+        w[D + 1] = l;
+      }
+    }
   }
-  if (lane < LPR) {
-    float* w = wsc + warp * (D + 2);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      w[j0 + c] = acc[c];
-      w[HALF + j0 + c] = acc[4 + c];
-    }
-    if (lane == 0) {
-      w[D] = m;
-      w[D + 1] = l;
-    }
+  if (timed_out) {
+    // the launch's output is not valid; give copies still in flight into this
+    // CTA's shared memory time to land before the CTA can exit
+    atomicOr(errw, RECSA_DEVERR_WAIT_TIMEOUT);
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < 1000000ull) __nanosleep(10000);
   }
   __syncthreads();
-  // CTA state of each head -> rank 0's merge slot [rank]
-  float* dst = cluster.map_shared_rank(mrg, 0) + rank * G * (D + 2);
   for (int x = tid; x < G * D; x += kThreads) {
     const int h = x / D, c = x % D;
+    const int lh = h % HPC;
+    const bool mine = h / HPC == hg;
     float mm = -INFINITY;
-    for (int w = h * WPH; w < (h + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * (D + 2) + D]);
-    if (has_win)
-      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * (D + 2) + D]);
+    if (mine)
+      for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * RS + D]);
+    for (int w = 0; w < kWinWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * RS + D]);
     float aa = 0.f, ll = 0.f;
-    for (int w = h * WPH; w < (h + 1) * WPH; ++w) {
-      const float* ws = wsc + w * (D + 2);
-      const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
-      aa = fmaf(ws[c], r, aa);
-      ll = fmaf(ws[D + 1], r, ll);
-    }
-    if (has_win)
-      for (int w = 0; w < kWarps; ++w) {
-        const float* ws = wwin + (w * G + h) * (D + 2);
+    if (mm != -INFINITY) {
+      if (mine)
+        for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) {
+          const float* ws = wsc + w * RS;
+          const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+          aa = fmaf(ws[c], r, aa);
+          ll = fmaf(ws[D + 1], r, ll);
+        }
+      for (int w = 0; w < kWinWarps; ++w) {
+        const float* ws = wwin + (w * G + h) * RS;
         const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
         aa = fmaf(ws[c], r, aa);
         ll = fmaf(ws[D + 1], r, ll);
       }
-    dst[h * (D + 2) + c] = aa;
+    }
+    float* dst = (CS == 1 ? mrg : cluster.map_shared_rank(mrg, (h / HPC) * S)) +
+                 (rank * HPC + lh) * RS;
+    dst[c] = aa;
     if (c == 0) {
-      dst[h * (D + 2) + D] = mm;
-      dst[h * (D + 2) + D + 1] = ll;
+      dst[D] = mm;
+      dst[D + 1] = ll;
     }
   }
-  cluster.sync();
-  if (rank == 0) {
-    for (int x = tid; x < G * D; x += kThreads) {
+  if (CS > 1)
+    cluster.sync();
+  else
+    __syncthreads();
+  if (sh == 0) {
+    for (int x = tid; x < HPC * D; x += kThreads) {
       const int h = x / D, c = x % D;
       float mm = -INFINITY;
-      for (int r = 0; r < CS; ++r) mm = fmaxf(mm, mrg[(r * G + h) * (D + 2) + D]);
+      for (int r = 0; r < CS; ++r) mm = fmaxf(mm, mrg[(r * HPC + h) * RS + D]);
       float aa = 0.f, ll = 0.f;
-      for (int r = 0; r < CS; ++r) {
-        const float* ms = mrg + (r * G + h) * (D + 2);
-        const float w = (ms[D] == -INFINITY) ? 0.f : __expf(ms[D] - mm);
-        aa = fmaf(ms[c], w, aa);
-        ll = fmaf(ms[D + 1], w, ll);
-      }
+      if (mm != -INFINITY)
+        for (int r = 0; r < CS; ++r) {
+          const float* ms = mrg + (r * HPC + h) * RS;
+          const float w = (ms[D] == -INFINITY) ? 0.f : __expf(ms[D] - mm);
+          aa = fmaf(ms[c], w, aa);
+          ll = fmaf(ms[D + 1], w, ll);
+        }
       const float o = (empty || ll == 0.f) ? 0.f : aa / ll;
-      store_elem(O, qrow + x, o, p.dtype);
+      store_elem(O, qrow + int64_t(hg * HPC + h) * D + c, o, p.dtype);
     }
     if (trace && !empty) {
-      for (int x = tid; x < G * (kTraceHead + kMaxLevels * p.k); x += kThreads) {
-        const int h = x / tstride, f = x % tstride;
-        const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
+      for (int x = tid; x < HPC * kTraceHead; x += kThreads) {
+        const int h = x / kTraceHead, f = x % kTraceHead;
+        const int64_t rec =
+            ((seq * n_q + qi) * p.hq + int64_t(g) * G + hg * HPC + h) * tstride;
         int v = 0;
         if (f == 0) v = top;
         else if (f == 1 || f == 2 || f == 3) {
@@ -664,11 +1042,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         } else if (f < 4 + kMaxLevels) {
           const int lev = f - 4 + 1;
           v = lev <= top ? cnt_c[lev] : 0;
-        } else if (f < kTraceHead) {
+        } else {
           const int lev = f - 4 - kMaxLevels + 1;
           v = lev <= top ? cnt_k[lev] : 0;
-        } else {
-          continue;   // kept ids are written per level below
         }
         trace[rec + f] = v;
       }
@@ -715,8 +1091,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     // one to finish (per-sequence counter) publishes len + 1 and resets it.
     if (rank == 0 && tid == 0) {
       if (!do_append) {
-        if (len0 >= p.cap) atomicOr(tree_error_word(const_cast<void*>(tree)),
-                                    RECSA_DEVERR_APPEND_FULL);
+        if (len0 >= p.cap) atomicOr(errw, RECSA_DEVERR_APPEND_FULL);
       } else {
         __threadfence();
         const int done = atomicAdd(st.counters + seq, 1);
@@ -735,10 +1110,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
 namespace recsa {
 namespace {
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int HPC>
 cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const void* V,
                           const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
-                          int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
+                          int32_t* trace, cudaStream_t s, int S, StepArgs st) {
   const int64_t kk = p.k < p.cap ? p.k : p.cap;
   int64_t maxn = 1;
   for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
@@ -746,17 +1121,24 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   cm = cm < maxn ? cm : maxn;
   const int cmax = int(cm < 1 ? 1 : cm);
   const int kmax = int(kk < cmax ? kk : cmax);
-  if (cmax > 1024) return cudaErrorNotSupported;
-  // window rows staged per CTA: at most ceil((W + B - 1) / cs)
-  const int wrows = int((int64_t(p.W) + p.B - 1 + cs - 1) / cs);
-  const size_t bytes = (size_t(3) * G * D + size_t(2) * G * cmax + size_t(kWarps) * (D + 2) +
-                        size_t(kWarps) * G * (D + 2) +
-                        size_t(cs) * G * (D + 2)) * 4 + size_t(2) * G * kmax * 4 +
-                       size_t(2) * G * cmax + 16 + size_t(2) * wrows * D * sizeof(T);
-  if (bytes > 200 * 1024) return cudaErrorNotSupported;
-  auto kern = decode_cluster_kernel<T, D, G>;
+  if (cmax > 32 * kRegSlots * 4) return cudaErrorNotSupported;
+  // The most kept-leaf ring slots that fit; more shares per head group when
+  // even one slot (or one share of a level's keys) does not fit.
+  int cs = (G / HPC) * S, nrh = 0;
+  Plan pl{};
+  for (;;) {
+    if (cs > kMaxCluster) return cudaErrorNotSupported;
+    for (nrh = kMaxTokSlots; nrh >= 1; --nrh) {
+      pl = make_plan<T, D, G, HPC>(cmax, kmax, S, cs, nrh, p.B, p.lay.levels);
+      if (pl.total <= kSmemLimit) break;
+    }
+    if (nrh >= 1) break;
+    S *= 2;
+    cs *= 2;
+  }
+  auto kern = decode_cluster_kernel<T, D, G, HPC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(bytes));
+                                       int(pl.total));
   if (e != cudaSuccess) return e;
   if (cs > 8) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -766,7 +1148,7 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, n_q, unsigned(p.batch * p.hkv));
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = bytes;
+  cfg.dynamicSmemBytes = pl.total;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -777,52 +1159,70 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, p, reinterpret_cast<const T*>(Q),
                             reinterpret_cast<const T*>(K), reinterpret_cast<const T*>(V), tree,
-                            len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax,
-                            wrows, st);
+                            len_dev, int(n_q), reinterpret_cast<T*>(O), trace, cmax, kmax, S,
+                            nrh, st);
 }
 
 template <typename T, int D>
 cudaError_t cluster_g(const Params& p, const void* Q, const void* K, const void* V,
                       const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
-                      int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
-  switch (p.group) {
-    case 1: return cluster_typed<T, D, 1>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
-    case 2: return cluster_typed<T, D, 2>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
-    case 4: return cluster_typed<T, D, 4>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
-    default: return cudaErrorNotSupported;
+                      int32_t* trace, cudaStream_t s, int hpc, int S, StepArgs st) {
+#define RECSA_CLUSTER_CASE(GG, HH)                                                          \
+  if (p.group == GG && hpc == HH)                                                           \
+    return cluster_typed<T, D, GG, HH>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, S, st);
+  RECSA_CLUSTER_CASE(1, 1)
+  RECSA_CLUSTER_CASE(2, 1)
+  RECSA_CLUSTER_CASE(2, 2)
+  RECSA_CLUSTER_CASE(4, 1)
+  RECSA_CLUSTER_CASE(4, 2)
+  RECSA_CLUSTER_CASE(4, 4)
+#undef RECSA_CLUSTER_CASE
+  return cudaErrorNotSupported;
+}
+
+// Heads per CTA (HPC) and candidate shares per head group (S) of a launch.
+// RECSA_DECODE_SPLIT="hpc,s" forces both (tests); otherwise the fewest heads
+// per CTA and the most shares that keep the grid within the 148 SMs.
+void decode_split(const Params& p, int32_t n_q, int& hpc, int& S) {
+  const int G = p.group;
+  const char* env = getenv("RECSA_DECODE_SPLIT");
+  if (env) {
+    int h = 0, s = 0;
+    if (sscanf(env, "%d,%d", &h, &s) == 2 && h >= 1 && h <= G && G % h == 0 &&
+        (h & (h - 1)) == 0 && s >= 1 && (s & (s - 1)) == 0 && (G / h) * s <= kMaxCluster) {
+      hpc = h;
+      S = s;
+      return;
+    }
   }
+  const int64_t pairs = int64_t(p.batch) * p.hkv * n_q;
+  hpc = 1;
+  while (hpc < G && pairs * (G / hpc) > 148) hpc *= 2;
+  const int ng = G / hpc;
+  S = 1;
+  while (ng * S * 2 <= kMaxCluster && pairs * ng * S * 2 <= 148) S *= 2;
 }
 
 cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, const void* V,
                              const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
-                             int32_t* trace, cudaStream_t s, int cs, StepArgs st) {
+                             int32_t* trace, cudaStream_t s, StepArgs st) {
+  int hpc = 1, S = 1;
+  decode_split(p, n_q, hpc, S);
   if (p.dtype == RECSA_DTYPE_BF16)
-    return p.d == 128 ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st)
-                      : cluster_g<__nv_bfloat16, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
-  return p.d == 128 ? cluster_g<float, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st)
-                    : cluster_g<float, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, cs, st);
+    return p.d == 128
+               ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, hpc, S, st)
+               : cluster_g<__nv_bfloat16, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, hpc, S, st);
+  return p.d == 128 ? cluster_g<float, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, hpc, S, st)
+                    : cluster_g<float, 64>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, hpc, S, st);
 }
 
 }  // namespace
-
-int decode_cluster_size(const Params& p, int32_t n_q) {
-  const char* env = getenv("RECSA_DECODE_CLUSTER");
-  if (env) {
-    const int v = atoi(env);
-    if (v == 1 || v == 2 || v == 4 || v == 8 || v == 16) return v;
-  }
-  const int64_t clusters = int64_t(p.batch) * p.hkv * n_q;
-  int cs = 2;
-  while (cs < 16 && clusters * cs * 2 <= 148) cs *= 2;
-  return cs;
-}
 
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s) {
   StepArgs st = {};
-  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s,
-                          decode_cluster_size(p, n_q), st);
+  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s, st);
 }
 
 cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
@@ -838,8 +1238,7 @@ cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
   st.len_w = len_dev;
   st.counters = reinterpret_cast<int*>(reinterpret_cast<char*>(tree) + kStepCounterOffset);
   st.fuse = 1;
-  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s,
-                          decode_cluster_size(p, n_q), st);
+  return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s, st);
 }
 
 }  // namespace recsa

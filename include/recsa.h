@@ -63,6 +63,9 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
 
 /* Device error flags in the tree header (recsa_tree_error). */
 #define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
+#define RECSA_DEVERR_WAIT_TIMEOUT 0x2u /* a bounded wait of the decode kernel on its own
+                                         asynchronous copies expired (the output of
+                                         that launch is not valid) */
 
 /*
  * Tree geometry and attention shape.

@@ -26,19 +26,20 @@ def _lib():
     R.lib()
 
 
-@pytest.fixture(params=["cluster-auto", "cluster-2", "cluster-4", "cluster-8", "cluster-16",
-                        "generic"])
+@pytest.fixture(params=["cluster-auto", "split-1,1", "split-1,2", "split-1,4", "split-2,1",
+                        "split-4,1", "split-4,2", "generic"])
 def decode_impl(request):
-    """Select the decode kernel: the cluster kernel (auto or forced cluster size)
-    or the generic one-CTA-per-query kernel."""
-    keys = ("RECSA_DECODE_CLUSTER", "RECSA_DECODE_GENERIC")
+    """Select the decode kernel: the cluster kernel with its automatic launch
+    shape or a forced one ("split-HPC,S": HPC query heads per CTA, S candidate
+    shares per head group), or the generic one-CTA-per-query kernel."""
+    keys = ("RECSA_DECODE_SPLIT", "RECSA_DECODE_GENERIC")
     old = {k: os.environ.get(k) for k in keys}
     for k in keys:
         os.environ.pop(k, None)
     if request.param == "generic":
         os.environ["RECSA_DECODE_GENERIC"] = "1"
     elif request.param != "cluster-auto":
-        os.environ["RECSA_DECODE_CLUSTER"] = request.param.split("-")[1]
+        os.environ["RECSA_DECODE_SPLIT"] = request.param.split("-")[1]
     yield request.param
     for k, v in old.items():
         if v is None:
