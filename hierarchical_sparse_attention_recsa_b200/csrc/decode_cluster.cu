@@ -48,13 +48,14 @@ namespace recsa {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
+
 constexpr int kChainWarps = 12;
-constexpr int kWinWarps = kWarps - kChainWarps;
+constexpr int kWinWarps = 3;
+constexpr int kProducerWarp = kChainWarps + kWinWarps;   // issues the chain's copies
 constexpr int kChainThreads = kChainWarps * 32;
 constexpr int kRegSlots = 8;      // top-k candidates held in registers: 32 per slot
 constexpr int kWinRing = 4;       // window ring slots
-constexpr int kWinChunk = 16;     // window rows per ring slot
+constexpr int kWinChunk = 24;     // window rows per ring slot
 constexpr int kMaxCluster = 16;
 constexpr int kMaxTokSlots = 4;   // kept-leaf ring slots per head
 constexpr unsigned long long kWaitNs = 50000000ull;   // a wait gives up after 50 ms
@@ -121,13 +122,23 @@ __device__ __forceinline__ unsigned long long global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
   return t;
 }
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* mb, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(mb)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase of the given parity.  False when it did not
 // complete within kWaitNs, or when an earlier wait of this thread expired
 // (`expired` is then set, and later waits return at once so that the kernel
 // runs to completion).
 __device__ __forceinline__ bool mbar_wait(uint64_t* mb, unsigned parity, bool& expired) {
   if (expired) return false;
-  if (mbar_try_wait(mb, parity)) return true;
+  if (mbar_test_wait(mb, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (;;) {
     if (mbar_try_wait(mb, parity)) return true;
@@ -145,6 +156,10 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned by
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
       ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(mb))
       : "memory");
+}
+// Arrive once on mb (release at CTA scope).
+__device__ __forceinline__ void mbar_arrive(uint64_t* mb) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(mb)) : "memory");
 }
 // Orders this thread's earlier shared-memory accesses (and those it has
 // synchronised with) before later bulk copies into shared memory.
@@ -241,6 +256,17 @@ __device__ __forceinline__ void cmul8(float* out, const float* a, const float* b
     out[2 * u + 1] = a[2 * u + 1] * b[2 * u] + a[2 * u] * b[2 * u + 1];
   }
 }
+// The lane's four rotate-half pairs of x (x[u], x[u + 4]) rotated by the
+// angles of cs taken negatively: out = R(-theta) x.
+__device__ __forceinline__ void rot_neg8(float* out, const float* x, const float* cs) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float c = cs[2 * u], sn = cs[2 * u + 1];
+    const float x1 = x[u], x2 = x[u + 4];
+    out[u] = fmaf(x1, c, x2 * sn);
+    out[u + 4] = fmaf(x2, c, -x1 * sn);
+  }
+}
 // Partial dot product of a lane's eight values, as two independent chains.
 __device__ __forceinline__ float dot8(const float* q, const float* x) {
   float a = q[0] * x[0], b = q[4] * x[4];
@@ -265,7 +291,7 @@ __device__ __forceinline__ void slot_sum2(float& a, float& b) {
 
 // Shared-memory plan of one CTA (byte offsets), the same on host and device.
 struct Plan {
-  unsigned mb, qf, qtok, qlev, rrow, sc, wsc, wwin, mrg, kept, kfl, wbuf, kbuf, vbuf, total;
+  unsigned mb, qf, qtok, qlev, rrow, sc, wsc, wwin, mrg, kept, kfl, rmask, wbuf, kbuf, vbuf, total;
   int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
   unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
 };
@@ -275,17 +301,19 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   constexpr unsigned RS = D + 2;
   Plan q;
   unsigned o = 0;
-  q.mb = o;   o += 256;                                   // mbarriers
+  q.mb = o;   o += 512;                                   // mbarriers
   q.qf = o;   o += G * D * 4;
   q.qtok = o; o += G * D * 4;
   q.qlev = o; o += unsigned(levels) * HPC * D * 4;        // query rotated per level
-  q.rrow = o; o += unsigned(levels + 2) * D * 4;          // RoPE table rows (cos, sin)
+  q.rrow = o; o += unsigned(2 * levels + 3) * D * 4;      // RoPE table rows (cos, sin)
   q.sc = o;   o += 2 * HPC * unsigned(cmax) * 4;
   q.wsc = o;  o += kChainWarps * RS * 4;
   q.wwin = o; o += kWinWarps * G * RS * 4;
   q.mrg = o;  o += unsigned(CS) * HPC * RS * 4;
   q.kept = o; o += 2 * HPC * unsigned(kmax) * 4;
   q.kfl = o;  o += 2 * HPC * unsigned(cmax);
+  o = (o + 15u) & ~15u;
+  q.rmask = o; o += HPC * 32 * 4;
   o = (o + 127u) & ~127u;
   q.wbuf = o; o += kWinRing * 2 * kWinChunk * D * unsigned(sizeof(T));
   o = (o + 127u) & ~127u;
@@ -328,13 +356,17 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   uint64_t* mb_lev = reinterpret_cast<uint64_t*>(smem + pl.mb);   // level keys arrived
   uint64_t* mb_val = mb_lev + 1;                                   // level values arrived
   uint64_t* mb_ready = mb_lev + 2;             // [2] head group's scores by level parity (S > 1)
-  uint64_t* mb_win = mb_lev + 4;                                   // [kWinRing]
-  uint64_t* mb_tok = mb_win + kWinRing;                            // [HPC][NRH]
+  uint64_t* mb_kept = mb_lev + 4;              // chain -> producer: a level's kept list is ready
+  uint64_t* mb_folded = mb_lev + 5;            // chain -> producer: a level's values are folded
+  uint64_t* mb_win = mb_lev + 6;                                   // [kWinRing]
+  uint64_t* mb_tok = mb_win + kWinRing;                            // [HPC][NRH] leaf arrived
+  uint64_t* mb_empty = mb_tok + HPC * NRH;                         // [HPC][NRH] slot consumed
   float* qf = reinterpret_cast<float*>(smem + pl.qf);       // [G][D] raw query
   float* qtok = reinterpret_cast<float*>(smem + pl.qtok);   // [G][D] rotated to n0 - 1
   float* qlev = reinterpret_cast<float*>(smem + pl.qlev);   // [levels][HPC][D] rotated to c_l
   // RoPE table rows: [l - 1] = R(lo_l) (first candidate of this share at level
-  // l), [levels] = R(sh * B), [levels + 1] = R(S * B)
+  // l), [levels] = R(sh * B), [levels + 1] = R(S * B), [levels + 1 + l] =
+  // R(c_l) (the query's index at level l), [2 levels + 2] = R(n0 - 1)
   float* rrow = reinterpret_cast<float*>(smem + pl.rrow);
   float* sc = reinterpret_cast<float*>(smem + pl.sc);       // [2][HPC][cmax] scores
   float* wsc = reinterpret_cast<float*>(smem + pl.wsc);     // [kChainWarps][RS]
@@ -342,6 +374,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* mrg = reinterpret_cast<float*>(smem + pl.mrg);     // [CS][HPC][RS] received
   int* kept = reinterpret_cast<int*>(smem + pl.kept);       // [2][HPC][kmax]
   unsigned char* kfl = smem + pl.kfl;                       // [2][HPC][cmax]
+  unsigned* rmask = reinterpret_cast<unsigned*>(smem + pl.rmask);   // [HPC][32] kept bits
   T* wbuf = reinterpret_cast<T*>(smem + pl.wbuf);           // [kWinRing][2][kWinChunk][D]
   float* kbuf = reinterpret_cast<float*>(smem + pl.kbuf);   // [HPC][rows][D] level keys
   float* vbuf = reinterpret_cast<float*>(smem + pl.vbuf);   // [HPC][rows][D] level values
@@ -412,21 +445,34 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   if (tid == 0) {
     mbar_init(mb_lev, 1);
     mbar_init(mb_val, 1);
+    mbar_init(mb_kept, 1);
+    mbar_init(mb_folded, 1);
     mbar_init(mb_ready, unsigned(S));
     mbar_init(mb_ready + 1, unsigned(S));
     for (int i = 0; i < kWinRing; ++i) mbar_init(mb_win + i, 1);
-    for (int i = 0; i < HPC * NRH; ++i) mbar_init(mb_tok + i, 1);
+    for (int i = 0; i < HPC * NRH; ++i) {
+      mbar_init(mb_tok + i, 1);
+      mbar_init(mb_empty + i, 1);
+    }
     mbar_fence_init();
   }
   __syncthreads();
   if (CS > 1) cluster_arrive_relaxed();   // waited on before the first remote access
 
   // ---- producers (bulk copies) ----------------------------------------------
+  // Node id of candidate i of local head h at level lev (kept list of lev + 1).
+  auto cand_node = [&](int lev, int h, int i) -> int {
+    const int kup = lev < top ? cnt_k[lev + 1] : 0;
+    const int vup = lev < top ? int(vis[lev + 1]) : 0;
+    if (i < p.b * kup)
+      return kept[((lev + 1) & 1) * HPC * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
+    return p.b * vup + (i - p.b * kup);
+  };
   // Keys (or values) of level lev (this CTA's share [lo, hi) of the candidate
-  // list of each local head) into kbuf (vbuf), completing on mb_lev (mb_val).
-  // Run by one whole warp: lane 0 arms the barrier, the lanes copy one run
-  // each (the children of a kept node of level lev + 1, or the orphans; the
-  // top level is one run).
+  // list of each local head) into kbuf (vbuf) in candidate order, completing
+  // on mb_lev (mb_val).  Run by the whole producer warp: lane 0 arms the
+  // barrier, the lanes copy one run each (the children of a kept node of
+  // level lev + 1, or the orphans; the top level is one run).
   auto issue_level = [&](int lev, bool values) {
     const int c = cnt_c[lev];
     int lo, hi;
@@ -437,8 +483,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     if (lane == 0) mbar_expect_tx(mb, unsigned(HPC) * unsigned(hi - lo) * rb);
     __syncwarp();
     if (hi <= lo) return;
-    const float* keys = values ? level_vals(p, const_cast<void*>(tree), lev, seq, g)
-                               : level_keys(p, const_cast<void*>(tree), lev, seq, g);
+    const float* src = values ? level_vals(p, const_cast<void*>(tree), lev, seq, g)
+                              : level_keys(p, const_cast<void*>(tree), lev, seq, g);
     const int kup = lev < top ? cnt_k[lev + 1] : 0;
     const int nch = p.b * kup;
     const int orph0 = lev < top ? p.b * int(vis[lev + 1]) : 0;   // first orphan node
@@ -459,7 +505,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       const int a0 = max(c0, lo), a1 = min(c1, hi);
       if (a1 > a0)
         bulk_g2s(dst + (size_t(h) * pl.rows + (a0 - lo)) * D,
-                 keys + int64_t(node0 + (a0 - c0)) * D, unsigned(a1 - a0) * rb, mb);
+                 src + int64_t(node0 + (a0 - c0)) * D, unsigned(a1 - a0) * rb, mb);
     }
   };
   // Window chunk ch (rows [ch * kWinChunk, ...) of this CTA's window share)
@@ -512,51 +558,63 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // First copies: the top level's keys and values (chain warps 0 and 1) and
   // the first window chunks (the first window warp), before the query is
   // loaded.
-  if (warp == 0 && top > 0) issue_level(top, false);
-  if (warp == 1 && top > 0) issue_level(top, true);
+  if (warp == kProducerWarp && top > 0) {
+    issue_level(top, false);
+    issue_level(top, true);
+  }
   if (warp == kChainWarps && lane < kWinRing && lane < nwch) issue_win(lane);
 
+  // The query and the RoPE table rows the kernel needs (loaded together: one
+  // memory round trip), then the query rotated to every level's index.
   for (int x = tid; x < G * D; x += kThreads)
     qf[x] = empty ? 0.f : load_elem(Q, qrow + x, p.dtype);
+  if (p.rope) {
+    const int lv = p.lay.levels;
+    for (int x = tid; x < (2 * lv + 3) * HALF; x += kThreads) {
+      const int r = x / HALF, j = x % HALF;
+      int64_t idx = -1;
+      if (r < lv) {
+        if (r < top) {
+          int lo, hi;
+          share(cnt_c[r + 1], lo, hi);
+          idx = lo;
+        }
+      } else if (r == lv) {
+        idx = int64_t(sh) * p.B;
+      } else if (r == lv + 1) {
+        idx = int64_t(S) * p.B;
+      } else if (r < 2 * lv + 2) {
+        if (r - lv - 1 <= top) idx = cnt_c[r - lv - 1];
+      } else {
+        idx = n0 - 1 > 0 ? n0 - 1 : 0;
+      }
+      if (idx < 0) continue;
+      const float2 cs = rope[min(idx, int64_t(rmax)) * HALF + j];
+      rrow[r * D + 2 * j] = cs.x;
+      rrow[r * D + 2 * j + 1] = cs.y;
+    }
+  }
+  for (int x = tid; x < kWinWarps * G * RS; x += kThreads)
+    wwin[x] = (x % RS == D) ? -INFINITY : 0.f;
   __syncthreads();
-  // qf rows [h0, h0 + nh) rotated to index idx into dst, by threads [0, nthr).
-  auto rotate_q = [&](float* dst, int h0, int nh, int64_t idx, int nthr) {
-    for (int x = tid; x < nh * HALF; x += nthr) {
+  // qf rows [h0, h0 + nh) rotated by table row r of rrow into dst.
+  auto rotate_q = [&](float* dst, int h0, int nh, int r) {
+    for (int x = tid; x < nh * HALF; x += kThreads) {
       const int h = x / HALF, j = x % HALF;
       const float x1 = qf[(h0 + h) * D + j], x2 = qf[(h0 + h) * D + j + HALF];
       if (p.rope) {
-        const float2 cs = rope[idx * HALF + j];
-        dst[h * D + j] = x1 * cs.x - x2 * cs.y;
-        dst[h * D + j + HALF] = x2 * cs.x + x1 * cs.y;
+        const float c = rrow[r * D + 2 * j], sn = rrow[r * D + 2 * j + 1];
+        dst[h * D + j] = x1 * c - x2 * sn;
+        dst[h * D + j + HALF] = x2 * c + x1 * sn;
       } else {
         dst[h * D + j] = x1;
         dst[h * D + j + HALF] = x2;
       }
     }
   };
-  if (!empty) rotate_q(qtok, 0, G, n0 - 1 > 0 ? n0 - 1 : 0, kThreads);
+  if (!empty) rotate_q(qtok, 0, G, 2 * p.lay.levels + 2);
   for (int lev = 1; lev <= top; ++lev)
-    rotate_q(qlev + (lev - 1) * HPC * D, hg * HPC, HPC, cnt_c[lev], kThreads);
-  if (p.rope) {
-    // table rows the chain seeds its RoPE recurrences from
-    for (int x = tid; x < (top + 2) * HALF; x += kThreads) {
-      const int r = x / HALF, j = x % HALF;
-      int idx;
-      if (r < top) {
-        int lo, hi;
-        share(cnt_c[r + 1], lo, hi);
-        idx = lo;
-      } else {
-        idx = r == top ? sh * p.B : S * p.B;
-      }
-      const float2 cs = rope[int64_t(min(idx, rmax)) * HALF + j];
-      float* dst = rrow + (r < top ? r : p.lay.levels + (r - top)) * D;
-      dst[2 * j] = cs.x;
-      dst[2 * j + 1] = cs.y;
-    }
-  }
-  for (int x = tid; x < kWinWarps * G * RS; x += kThreads)
-    wwin[x] = (x % RS == D) ? -INFINITY : 0.f;
+    rotate_q(qlev + (lev - 1) * HPC * D, hg * HPC, HPC, p.lay.levels + 1 + lev);
   __syncthreads();
   if (CS > 1) cluster_wait();
   bool timed_out = false;   // a bounded wait of this thread expired
@@ -646,56 +704,56 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.f;
 
-  // Node id of candidate i of local head h at level lev (kept list of lev + 1).
-  auto cand_node = [&](int lev, int h, int i) -> int {
-    const int kup = lev < top ? cnt_k[lev + 1] : 0;
-    const int vup = lev < top ? int(vis[lev + 1]) : 0;
-    if (i < p.b * kup)
-      return kept[((lev + 1) & 1) * HPC * kmax + h * kmax + div_b(p, i)] * p.b + mod_b(p, i);
-    return p.b * vup + (i - p.b * kup);
-  };
 
   // Scores of this CTA's share of level lev's candidates (keys in kbuf) for
   // head hw, two rows per slot at a time; with S > 1 each score is stored
-  // into every CTA of the group.  A slot's rows are lo + hs + i * HSLOT, so
-  // its (cos, sin) start at R(lo) R(hs) and advance by R(HSLOT) per row.
+  // into every CTA of the group.  The score of candidate i is
+  // <R(c) q, R(i) k> = <R(c - i) q, k>, so the query (rotated to c in qlev)
+  // is turned back by the candidate's index instead of rotating every key: a
+  // slot's rows are lo + hs + j * HSLOT, so its query starts at
+  // R(-(lo + hs)) qlev and turns by R(-HSLOT) per row.
   auto score_level = [&](int lev) {
     int lo, hi;
     share(cnt_c[lev], lo, hi);
     const int nr = hi - lo;
     const float* kb = kbuf + size_t(hw) * pl.rows * D;
     float* scK = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
-    float q[8];
-    lds_pairs(qlev + ((lev - 1) * HPC + hw) * D, j0, HALF, q);
-    float csa[8], st2[8];
+    float q0[8], st2[8];
+    lds_pairs(qlev + ((lev - 1) * HPC + hw) * D, j0, HALF, q0);
     if (p.rope) {
+      float seed[8], t[8];
       if (S == 1) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) csa[c] = cs_hs[c];
+        for (int c = 0; c < 8; ++c) seed[c] = cs_hs[c];
       } else {
         float r[8];
         lds_cs8(rrow + (lev - 1) * D, j0, r);
-        cmul8(csa, r, cs_hs);
+        cmul8(seed, r, cs_hs);
       }
+      rot_neg8(t, q0, seed);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) q0[c] = t[c];
       cmul8(st2, cs_st, cs_st);
     }
     for (int e = hs; e - hs < nr; e += 2 * HSLOT) {
       const int e1 = e + HSLOT;
       const bool on0 = e < nr, on1 = e1 < nr;
-      float x0[8], x1[8];
+      float x0[8], x1[8], q1[8];
       SharedPairs<float, HALF>::load(kb + size_t(on0 ? e : 0) * D, j0, x0);
       SharedPairs<float, HALF>::load(kb + size_t(on1 ? e1 : 0) * D, j0, x1);
       if (p.rope) {
-        float csb[8];
-        cmul8(csb, csa, cs_st);
-        rotate8(x0, csa);
-        rotate8(x1, csb);
-        float t2[8];
-        cmul8(t2, csa, st2);
+        rot_neg8(q1, q0, cs_st);
+      } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) csa[c] = t2[c];
+        for (int c = 0; c < 8; ++c) q1[c] = q0[c];
       }
-      float s0 = dot8(q, x0), s1 = dot8(q, x1);
+      float s0 = dot8(q0, x0), s1 = dot8(q1, x1);
+      if (p.rope) {
+        float t[8];
+        rot_neg8(t, q0, st2);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) q0[c] = t[c];
+      }
       slot_sum2<LPR>(s0, s1);
       s0 *= inv_sqrt_d;
       s1 *= inv_sqrt_d;
@@ -750,7 +808,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   auto topk = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
-    const int h = warp;
+    const int h = 3 - warp;
     const float* row = sc + par * HPC * cmax + h * cmax;
     const int ns = (c + 31) >> 5;
     unsigned taken = 0;
@@ -798,25 +856,37 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         }
       }
     }
-    unsigned char* fl = kfl + par * HPC * cmax + h * cmax;
-    int* kp = kept + par * HPC * kmax + h * kmax;
-    int cnt = 0;
+    // kept bits by candidate row (bit l of rmask[h][s] = candidate 32 s + l)
+    unsigned mine = 0;
     for (int s = 0; s < ns; ++s) {
-      const int i = s * 32 + lane;
-      const bool f = i < c && ((taken >> s) & 1u);
-      if (i < c) fl[i] = f;
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      const unsigned R = __ballot_sync(0xffffffffu, (taken >> s) & 1u);
+      if (lane == s) mine = R;
+    }
+    if (lane < ns) rmask[h * 32 + lane] = mine;
+  };
+
+  // Kept flags and the kept list (in index order) of level lev from the row
+  // masks, by every chain thread (one candidate each).
+  auto compact = [&](int lev) {
+    const int c = cnt_c[lev];
+    const int par = lev & 1;
+    for (int x = tid; x < HPC * c; x += kChainThreads) {
+      const int h = x / c, i = x % c;
+      const int s = i >> 5, l = i & 31;
+      const unsigned R = rmask[h * 32 + s];
+      const bool f = (R >> l) & 1u;
+      kfl[par * HPC * cmax + h * cmax + i] = f;
       if (f) {
-        const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+        int pos = __popc(R & ((1u << l) - 1u));
+        for (int t = 0; t < s; ++t) pos += __popc(rmask[h * 32 + t]);
         const int node = cand_node(lev, h, i);
-        kp[pos] = node;
+        kept[par * HPC * kmax + h * kmax + pos] = node;
         if (trace && sh == 0) {
           const int64_t rec =
               ((seq * n_q + qi) * p.hq + int64_t(g) * G + hg * HPC + h) * tstride;
           trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
         }
       }
-      cnt += __popc(bal);
     }
   };
 
@@ -840,11 +910,13 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
 
   // Kept-leaf tokens of head hw through its ring of NRH slots, two rows per
   // slot at a time.  Leaf j of the share has rank sh + j * S, so its row e
-  // sits at RoPE index (sh + j * S) * B + e: the seed R((sh + j S) B) advances
-  // by R(S B) per leaf and is combined with the slot's R(hs).
+  // sits at RoPE index (sh + j S) B + e; as for the summaries, the query
+  // (rotated to n0 - 1 in qtok) is turned back by each row's index: the seed
+  // R((sh + j S) B) advances by R(S B) per leaf and is combined with the
+  // slot's R(hs), and the query turns by R(-HSLOT) per row.
   auto token_pass = [&]() {
-    float q[8];
-    lds_pairs(qtok + (hg * HPC + hw) * D, j0, HALF, q);
+    float qt[8];
+    lds_pairs(qtok + (hg * HPC + hw) * D, j0, HALF, qt);
     const unsigned lbar = kBarHead0 + hw;
     float rj[8], st2[8];
     if (p.rope) {
@@ -857,43 +929,46 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       mbar_wait(mb_tok + hw * NRH + slot, unsigned(j / NRH) & 1u, timed_out);
       const T* cK = tbuf + (size_t(hw) * NRH + slot) * slot_elems;
       const T* cV = cK + size_t(p.B) * D;
-      float csa[8];
+      float q0[8];
       if (p.rope) {
-        cmul8(csa, rj, cs_hs);
-        float r[8], t2[8];
+        float seed[8], r[8], t2[8];
+        cmul8(seed, rj, cs_hs);
+        rot_neg8(q0, qt, seed);
         lds_cs8(rrow + (p.lay.levels + 1) * D, j0, r);
         cmul8(t2, rj, r);
 #pragma unroll
         for (int c = 0; c < 8; ++c) rj[c] = t2[c];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) q0[c] = qt[c];
       }
       for (int e = hs; e - hs < p.B; e += 2 * HSLOT) {
         const int e1 = e + HSLOT;
         const bool on0 = e < p.B, on1 = e1 < p.B;
         const int r0 = on0 ? e : 0, r1 = on1 ? e1 : 0;
-        float k0[8], k1[8], v0[8], v1[8];
+        float k0[8], k1[8], v0[8], v1[8], q1[8];
         SharedPairs<T, HALF>::load(cK + size_t(r0) * D, j0, k0);
         SharedPairs<T, HALF>::load(cK + size_t(r1) * D, j0, k1);
         SharedPairs<T, HALF>::load(cV + size_t(r0) * D, j0, v0);
         SharedPairs<T, HALF>::load(cV + size_t(r1) * D, j0, v1);
         if (p.rope) {
-          float csb[8];
-          cmul8(csb, csa, cs_st);
-          rotate8(k0, csa);
-          rotate8(k1, csb);
-          float t2[8];
-          cmul8(t2, csa, st2);
+          rot_neg8(q1, q0, cs_st);
+        } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) csa[c] = t2[c];
+          for (int c = 0; c < 8; ++c) q1[c] = q0[c];
         }
-        float s0 = dot8(q, k0), s1 = dot8(q, k1);
+        float s0 = dot8(q0, k0), s1 = dot8(q1, k1);
+        if (p.rope) {
+          float t[8];
+          rot_neg8(t, q0, st2);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) q0[c] = t[c];
+        }
         slot_sum2<LPR>(s0, s1);
         fold2(m, l, acc, s0 * inv_sqrt_d, on0, v0, s1 * inv_sqrt_d, on1, v1);
       }
       named_sync(lbar, WPH * 32);
-      if (warp == hw * WPH && lane == 0 && j + NRH < ntok) {
-        fence_proxy_async();
-        issue_tok(hw, j + NRH);
-      }
+      if (warp == hw * WPH && lane == 0 && j + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot);
     }
   };
 
@@ -910,39 +985,59 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       score_level(lev);
       level_sync();
       const int u = use++;
-      if (warp < HPC) topk(lev);
+      if (warp >= 4 - HPC && warp < 4) topk(lev);
       named_sync(kBarChain, kChainThreads);
-      if (lev > 1) {
-        if (warp == 0) {
-          if (lane == 0) fence_proxy_async();
-          __syncwarp();
-          issue_level(lev - 1, false);
-        }
-      } else if (warp % WPH == 0 && lane == 0) {
-        fence_proxy_async();
-        for (int j = 0; j < NRH && j < ntok; ++j)
-          if (early_slot(hw, j)) issue_tok(hw, j);
-      }
+      compact(lev);
+      named_sync(kBarChain, kChainThreads);
+      if (tid == 0) mbar_arrive(mb_kept);
       mbar_wait(mb_val, unsigned(u) & 1u, timed_out);
       fold_values(lev);
       named_sync(kBarChain, kChainThreads);
-      if (lev > 1) {
-        if (warp == 1) {
-          if (lane == 0) fence_proxy_async();
-          __syncwarp();
-          issue_level(lev - 1, true);
-        }
-      } else if (warp % WPH == 0 && lane == 0) {
-        fence_proxy_async();
-        for (int j = 0; j < NRH && j < ntok; ++j)
-          if (!early_slot(hw, j)) issue_tok(hw, j);
-      }
+      if (tid == 0) mbar_arrive(mb_folded);
     }
     if (top > 0) token_pass();
   };
 
+  // The producer warp issues the chain's copies as soon as their addresses
+  // are known: a level's keys once the kept list above it is compacted, its
+  // values once the level above is folded (vbuf is free), the kept leaves of
+  // level 1 (slots inside kbuf first, the rest once vbuf is free), and each
+  // ring slot again when its head's warps have consumed it.
+  auto producer_warp = [&]() {
+    for (int u = 0; u < top; ++u) {
+      const int lev = top - u;
+      mbar_wait(mb_kept, unsigned(u) & 1u, timed_out);
+      if (lane == 0) fence_proxy_async();
+      __syncwarp();
+      if (lev > 1) {
+        issue_level(lev - 1, false);
+      } else if (lane < HPC) {
+        for (int j = 0; j < NRH && j < ntok; ++j)
+          if (early_slot(lane, j)) issue_tok(lane, j);
+      }
+      mbar_wait(mb_folded, unsigned(u) & 1u, timed_out);
+      if (lane == 0) fence_proxy_async();
+      __syncwarp();
+      if (lev > 1) {
+        issue_level(lev - 1, true);
+      } else if (lane < HPC) {
+        for (int j = 0; j < NRH && j < ntok; ++j)
+          if (!early_slot(lane, j)) issue_tok(lane, j);
+      }
+    }
+    if (top > 0 && lane < HPC) {
+      const int h = lane;
+      for (int j = NRH; j < ntok; ++j) {
+        mbar_wait(mb_empty + h * NRH + j % NRH, unsigned(j / NRH - 1) & 1u, timed_out);
+        fence_proxy_async();
+        issue_tok(h, j);
+      }
+    }
+  };
 
-  if (warp >= kChainWarps)
+  if (warp == kProducerWarp)
+    producer_warp();
+  else if (warp >= kChainWarps)
     window_warps();
   else
     chain_warps();
