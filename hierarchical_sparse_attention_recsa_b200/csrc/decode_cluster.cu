@@ -196,99 +196,6 @@ __device__ __forceinline__ void merge_xor(float& m, float& l, float* acc, int o)
   m = mn;
 }
 
-// One online-softmax fold of score s with value pairs v.
-__device__ __forceinline__ void fold8(float& m, float& l, float* acc, float s, const float* v) {
-  if (s > m) {
-    const float r = __expf(m - s);
-    l = l * r + 1.f;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
-    m = s;
-  } else {
-    const float w = __expf(s - m);
-    l += w;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
-  }
-}
-
-// Two online-softmax folds (scores s0, s1 with value pairs v0, v1; a row
-// that is off is skipped) with one rescale of the state.
-__device__ __forceinline__ void fold2(float& m, float& l, float* acc, float s0, bool on0,
-                                      const float* v0, float s1, bool on1, const float* v1) {
-  s0 = on0 ? s0 : -INFINITY;
-  s1 = on1 ? s1 : -INFINITY;
-  const float mx = fmaxf(s0, s1);
-  if (mx == -INFINITY) return;
-  if (mx > m) {
-    const float r = __expf(m - mx);
-    l *= r;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] *= r;
-    m = mx;
-  }
-  const float w0 = on0 ? __expf(s0 - m) : 0.f;
-  const float w1 = on1 ? __expf(s1 - m) : 0.f;
-  l += w0 + w1;
-#pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = fmaf(w0, v0[c], fmaf(w1, v1[c], acc[c]));
-}
-
-// A lane's four rotate-half pairs of an fp32 row in shared memory.
-__device__ __forceinline__ void lds_pairs(const float* row, int j0, int half, float* x) {
-  const float4 a = *reinterpret_cast<const float4*>(row + j0);
-  const float4 b = *reinterpret_cast<const float4*>(row + half + j0);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-// A lane's four (cos, sin) pairs of a RoPE table row held in shared memory.
-__device__ __forceinline__ void lds_cs8(const float* row, int j0, float* cs) {
-  const float4 a = *reinterpret_cast<const float4*>(row + 2 * j0);
-  const float4 b = *reinterpret_cast<const float4*>(row + 2 * j0 + 4);
-  cs[0] = a.x; cs[1] = a.y; cs[2] = a.z; cs[3] = a.w;
-  cs[4] = b.x; cs[5] = b.y; cs[6] = b.z; cs[7] = b.w;
-}
-// out = a * b per (cos, sin) pair, as complex numbers (rotation angles add).
-__device__ __forceinline__ void cmul8(float* out, const float* a, const float* b) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    out[2 * u] = a[2 * u] * b[2 * u] - a[2 * u + 1] * b[2 * u + 1];
-    out[2 * u + 1] = a[2 * u + 1] * b[2 * u] + a[2 * u] * b[2 * u + 1];
-  }
-}
-// The lane's four rotate-half pairs of x (x[u], x[u + 4]) rotated by the
-// angles of cs taken negatively: out = R(-theta) x.
-__device__ __forceinline__ void rot_neg8(float* out, const float* x, const float* cs) {
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float c = cs[2 * u], sn = cs[2 * u + 1];
-    const float x1 = x[u], x2 = x[u + 4];
-    out[u] = fmaf(x1, c, x2 * sn);
-    out[u + 4] = fmaf(x2, c, -x1 * sn);
-  }
-}
-// Partial dot product of a lane's eight values, as two independent chains.
-__device__ __forceinline__ float dot8(const float* q, const float* x) {
-  float a = q[0] * x[0], b = q[4] * x[4];
-#pragma unroll
-  for (int c = 1; c < 4; ++c) {
-    a = fmaf(q[c], x[c], a);
-    b = fmaf(q[4 + c], x[4 + c], b);
-  }
-  return a + b;
-}
-// Two slot sums (over the LPR lanes of a row) with interleaved shuffles.
-template <int LPR>
-__device__ __forceinline__ void slot_sum2(float& a, float& b) {
-#pragma unroll
-  for (int o = LPR / 2; o > 0; o >>= 1) {
-    const float ta = __shfl_xor_sync(0xffffffffu, a, o);
-    const float tb = __shfl_xor_sync(0xffffffffu, b, o);
-    a += ta;
-    b += tb;
-  }
-}
-
 // Shared-memory plan of one CTA (byte offsets), the same on host and device.
 struct Plan {
   unsigned mb, qf, qtok, qlev, rrow, sc, wsc, wwin, mrg, kept, kfl, rmask, wbuf, kbuf, vbuf, total;

@@ -20,7 +20,7 @@ namespace {
 
 constexpr int kPThreads = 256;
 constexpr int kPWarps = kPThreads / 32;
-constexpr int kPUnroll = 2;
+constexpr int kPRegSlots = 8;   // top-k candidates held in registers: 32 per slot
 
 enum PItem { pKey = 0, pVal = 1, pNone = 2 };
 
@@ -100,20 +100,6 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  auto fold = [&](float s, const float* v) {
-    if (s > m) {
-      const float r = __expf(m - s);
-      l = l * r + 1.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = fmaf(acc[c], r, v[c]);
-      m = s;
-    } else {
-      const float w = __expf(s - m);
-      l += w;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
-    }
-  };
 
   const int64_t kvbase = (seq * p.hkv + g) * p.cap;
   const float inv_sqrt_d = p.inv_sqrt_d;
@@ -128,54 +114,69 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   };
 
   // Token rows: the window [a*B, t] (when this kernel attends it) or the
-  // kept leaves' tokens, each at its token-level index; K/V rows in dtype.
+  // kept leaves' tokens, each at its token-level index; K/V rows in dtype,
+  // two rows per lane slot at a time.  The score of a row at index i is
+  // <R(n0 - 1) q, R(i) k> = <R(n0 - 1 - i) q, k>: the query (rotated to
+  // n0 - 1 in qtok) is turned back by the row's index instead of rotating
+  // the key; a slot's rows advance by SPW, so its query turns by R(-SPW).
   auto token_loop = [&](bool window) {
     const int nt = window ? int(n_win) : nleaf * p.B;
     const int win0 = int(a) * p.B;
-    const int widx0 = nleaf * p.B;
+    const int idx0 = window ? nleaf * p.B : 0;
     const int* kept1 = kept + 1 * kmax;                           // level 1 = parity 1
-    // A slot's items step their RoPE index by SPW: (cos, sin) are seeded from
-    // the table once per batch and advanced by the fixed rotation of SPW.
-    const int idx0 = window ? widx0 : 0;
-    float cstep[8];
-    if (p.rope) load_cs(rope, SPW, HALF, j0, cstep);
-    for (int base = 0; base < nt; base += SPW * kPUnroll) {
-      TokRow<T, HALF> rk[kPUnroll], rv[kPUnroll];
-      float csc[8];
-      bool on[kPUnroll];
-      if (p.rope) load_cs(rope, min(idx0 + base + slot, rmax), HALF, j0, csc);
+    float q0[8], st[8], st2[8];
+    lds_pairs(qtok, j0, HALF, q0);
+    if (p.rope) {
+      float cs[8], t2[8];
+      load_cs(rope, min(idx0 + slot, rmax), HALF, j0, cs);
+      load_cs(rope, min(SPW, rmax), HALF, j0, st);
+      rot_neg8(t2, q0, cs);
 #pragma unroll
-      for (int u = 0; u < kPUnroll; ++u) {
-        const int e = base + u * SPW + slot;
-        on[u] = e < nt;
-        if (on[u]) {
-          const int pos = window ? win0 + e : kept1[div_B(p, e)] * p.B + mod_B(p, e);
-          rk[u].load(K + (kvbase + pos) * D, j0);
-          rv[u].load(V + (kvbase + pos) * D, j0);
-        }
+      for (int c = 0; c < 8; ++c) q0[c] = t2[c];
+      cmul8(st2, st, st);
+    }
+    for (int base = 0; base < nt; base += 2 * SPW) {
+      const int e0 = base + slot, e1 = e0 + SPW;
+      const bool on0 = e0 < nt, on1 = e1 < nt;
+      TokRow<T, HALF> rk0, rv0, rk1, rv1;
+      rk0.zero(); rv0.zero(); rk1.zero(); rv1.zero();
+      if (on0) {
+        const int pos = window ? win0 + e0 : kept1[div_B(p, e0)] * p.B + mod_B(p, e0);
+        rk0.load(K + (kvbase + pos) * D, j0);
+        rv0.load(V + (kvbase + pos) * D, j0);
       }
-#pragma unroll
-      for (int u = 0; u < kPUnroll; ++u) {
-        float xk[8], xv[8], s = 0.f;
-        rk[u].cvt(xk);
-        rv[u].cvt(xv);
-        if (p.rope) {
-          rotate8(xk, csc);
-          advance_cs(csc, cstep);
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          s = fmaf(qtok[j0 + c], xk[c], s);
-          s = fmaf(qtok[HALF + j0 + c], xk[4 + c], s);
-        }
-        s = slot_sum<LPR>(s) * inv_sqrt_d;
-        if (on[u]) fold(s, xv);
+      if (on1) {
+        const int pos = window ? win0 + e1 : kept1[div_B(p, e1)] * p.B + mod_B(p, e1);
+        rk1.load(K + (kvbase + pos) * D, j0);
+        rv1.load(V + (kvbase + pos) * D, j0);
       }
+      float k0[8], v0[8], k1[8], v1[8], q1[8];
+      rk0.cvt(k0);
+      rv0.cvt(v0);
+      rk1.cvt(k1);
+      rv1.cvt(v1);
+      if (p.rope) {
+        rot_neg8(q1, q0, st);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) q1[c] = q0[c];
+      }
+      float s0 = dot8(q0, k0), s1 = dot8(q1, k1);
+      if (p.rope) {
+        float t2[8];
+        rot_neg8(t2, q0, st2);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) q0[c] = t2[c];
+      }
+      slot_sum2<LPR>(s0, s1);
+      fold2(m, l, acc, s0 * inv_sqrt_d, on0, v0, s1 * inv_sqrt_d, on1, v1);
     }
   };
 
-  // Tree rows: key candidates of level klev (scored into sc) and the
-  // unselected candidates of level vlev (values folded); fp32 rows.
+  // Tree rows, two items per lane slot at a time: key candidates of level
+  // klev (scored into sc; candidate i sits at item i, and the query in qlev
+  // is turned back by i as for the tokens) and the unselected candidates of
+  // level vlev (values folded); fp32 rows.
   auto tree_loop = [&](int klev, int vlev) {
     const int nk = klev > 0 ? cnt_c[klev] : 0;
     const int nv = vlev > 0 ? cnt_c[vlev] : 0;
@@ -193,20 +194,29 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     const float* scV = sc + (vlev & 1) * cmax;
     const unsigned char* flV = kfl + (vlev & 1) * cmax;
     float* scK = sc + (klev & 1) * cmax;
-    float cstep[8];
-    if (p.rope) load_cs(rope, SPW, HALF, j0, cstep);
-    for (int base = 0; base < total; base += SPW * kPUnroll) {
-      RawPairs ra[kPUnroll];
-      float csc[8];
-      int kind[kPUnroll], idx[kPUnroll];
-      if (p.rope) load_cs(rope, min(base + slot, rmax), HALF, j0, csc);
-      float sv[kPUnroll];
+    float q0[8], st[8], st2[8];
+    lds_pairs(qlev, j0, HALF, q0);
+    if (p.rope) {
+      float cs[8], t2[8];
+      load_cs(rope, min(slot, rmax), HALF, j0, cs);
+      load_cs(rope, min(SPW, rmax), HALF, j0, st);
+      rot_neg8(t2, q0, cs);
 #pragma unroll
-      for (int u = 0; u < kPUnroll; ++u) {
+      for (int c = 0; c < 8; ++c) q0[c] = t2[c];
+      cmul8(st2, st, st);
+    }
+    for (int base = 0; base < total; base += 2 * SPW) {
+      RawPairs ra[2];
+      int kind[2], idx[2];
+      float sv[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
         const int e = base + u * SPW + slot;
         kind[u] = pNone;
         idx[u] = 0;
         sv[u] = 0.f;
+        ra[u].a = make_uint4(0u, 0u, 0u, 0u);
+        ra[u].b = make_uint4(0u, 0u, 0u, 0u);
         if (e < nk) {
           const int i = e;
           const int node = i < nchK ? keptK[div_b(p, i)] * p.b + mod_b(p, i) : orphK + i;
@@ -223,25 +233,32 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           }
         }
       }
+      float x0[8], x1[8], q1[8];
+      RawLoad<float, HALF>::cvt(ra[0], x0);
+      RawLoad<float, HALF>::cvt(ra[1], x1);
+      if (p.rope) {
+        rot_neg8(q1, q0, st);
+      } else {
 #pragma unroll
-      for (int u = 0; u < kPUnroll; ++u) {
-        float x[8], s = 0.f;
-        RawLoad<float, HALF>::cvt(ra[u], x);
-        if (kind[u] == pKey && p.rope) rotate8(x, csc);
-        if (p.rope) advance_cs(csc, cstep);
-        if (kind[u] == pKey) {
+        for (int c = 0; c < 8; ++c) q1[c] = q0[c];
+      }
+      float s0 = dot8(q0, x0), s1 = dot8(q1, x1);
+      if (p.rope) {
+        float t2[8];
+        rot_neg8(t2, q0, st2);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            s = fmaf(qlev[j0 + c], x[c], s);
-            s = fmaf(qlev[HALF + j0 + c], x[4 + c], s);
-          }
-        }
-        if (__any_sync(0xffffffffu, kind[u] == pKey)) s = slot_sum<LPR>(s) * inv_sqrt_d;
-        if (kind[u] == pKey) {
-          if (sub == 0) scK[idx[u]] = s;
-        } else if (kind[u] == pVal) {
-          fold(sv[u], x);
-        }
+        for (int c = 0; c < 8; ++c) q0[c] = t2[c];
+      }
+      if (__any_sync(0xffffffffu, kind[0] == pKey || kind[1] == pKey)) slot_sum2<LPR>(s0, s1);
+      if (kind[0] == pKey) {
+        if (sub == 0) scK[idx[0]] = s0 * inv_sqrt_d;
+      } else if (kind[0] == pVal) {
+        fold8(m, l, acc, sv[0], x0);
+      }
+      if (kind[1] == pKey) {
+        if (sub == 0) scK[idx[1]] = s1 * inv_sqrt_d;
+      } else if (kind[1] == pVal) {
+        fold8(m, l, acc, sv[1], x1);
       }
     }
   };
@@ -253,37 +270,69 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     __syncwarp();
   };
 
+  // Warp top-k: kap rounds of an arg-max over order-preserving keys held in
+  // registers (lane l holds candidates l, l + 32, ...; 0 = none or taken);
+  // redux.sync gives the round's maximum, a ballot its lanes, and on a tie of
+  // keys the lowest index wins.  Candidates beyond 32 * kPRegSlots are read
+  // from shared memory in the same rounds.  The kept list is compacted in
+  // index order with one ballot per row of 32 candidates.
   auto topk = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
     const float* scl = sc + par * cmax;
     unsigned char* fl = kfl + par * cmax;
     int* kp = kept + par * kmax;
-    for (int i = lane; i < c; i += 32) fl[i] = (kap >= c) ? 1 : 0;
-    __syncwarp();
-    if (kap < c) {
-      unsigned taken = 0;
-      const int nj = (c + 31) / 32;
-      for (int it = 0; it < kap; ++it) {
-        unsigned bk = 0, bi = 0xffffffffu;
-        for (int jj = 0; jj < nj; ++jj) {
-          const int i = lane + 32 * jj;
-          if (i < c && !((taken >> jj) & 1u)) {
-            const unsigned key = order_key(scl[i]);
-            if (key > bk) { bk = key; bi = unsigned(i); }
+    const int ns = (c + 31) >> 5;
+    unsigned taken = 0;
+    if (kap >= c) {
+      for (int s = 0; s < ns; ++s)
+        if (s * 32 + lane < c) taken |= 1u << s;
+    } else {
+      unsigned key[kPRegSlots];
+#pragma unroll
+      for (int s = 0; s < kPRegSlots; ++s) {
+        const int i = s * 32 + lane;
+        key[s] = i < c ? order_key(scl[i]) : 0u;
+      }
+      for (int r = 0; r < kap; ++r) {
+        unsigned bk = key[0];
+        int bs = 0;
+#pragma unroll
+        for (int s = 1; s < kPRegSlots; ++s)
+          if (key[s] > bk) {
+            bk = key[s];
+            bs = s;
+          }
+        for (int s = kPRegSlots; s < ns; ++s) {
+          const int i = s * 32 + lane;
+          if (i < c && !((taken >> s) & 1u)) {
+            const unsigned kk = order_key(scl[i]);
+            if (kk > bk) {
+              bk = kk;
+              bs = s;
+            }
           }
         }
-        const unsigned wk = __reduce_max_sync(0xffffffffu, bk);
-        const unsigned wi = __reduce_min_sync(0xffffffffu, bk == wk ? bi : 0xffffffffu);
-        if (lane == int(wi & 31u)) taken |= 1u << (wi >> 5);
-        if (lane == 0) fl[wi] = 1;
+        const unsigned M = __reduce_max_sync(0xffffffffu, bk);
+        unsigned who = __ballot_sync(0xffffffffu, bk == M);
+        if (__popc(who) > 1) {
+          const unsigned I =
+              __reduce_min_sync(0xffffffffu, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
+          who = 1u << (I & 31u);
+        }
+        if ((who >> lane) & 1u) {
+          taken |= 1u << bs;
+#pragma unroll
+          for (int s = 0; s < kPRegSlots; ++s)
+            if (s == bs) key[s] = 0u;
+        }
       }
     }
-    __syncwarp();
     int cnt = 0;
-    for (int j = 0; j < c; j += 32) {
-      const int i = j + lane;
-      const bool f = i < c && fl[i];
+    for (int s = 0; s < ns; ++s) {
+      const int i = s * 32 + lane;
+      const bool f = i < c && ((taken >> s) & 1u);
+      if (i < c) fl[i] = f;
       const unsigned bal = __ballot_sync(0xffffffffu, f);
       if (f) {
         const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
