@@ -25,7 +25,7 @@ constexpr int kPRegSlots = 8;   // top-k candidates held in registers: 32 per sl
 enum PItem { pKey = 0, pVal = 1, pNone = 2 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kPThreads, 2)
+__global__ void __launch_bounds__(kPThreads, 3)
 prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                     const T* __restrict__ V, const void* __restrict__ tree, int64_t q_start,
                     int n_q, T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
