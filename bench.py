@@ -19,6 +19,7 @@ reference (it is the reference arm: a float64 restatement of the method).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -149,6 +150,33 @@ class L2Flush:
     def __call__(self):
         self.buf.fill_(1)
         torch.cuda._sleep(self.spin)
+
+
+DECODE_SOURCES = ["decode_cluster.cu", "rows.cuh", "pool.cuh", "recsa_internal.cuh"]
+TRAFFIC_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                               "decode_cluster_kernel_qwen3-4b-524k_traffic.md")
+
+
+def measured_traffic(workload, L, batch):
+    """DRAM bytes per decode launch from the committed ncu capture of the same
+    workload, or None when the workload differs or the kernel sources have
+    changed since the capture (their sha256 no longer matches)."""
+    if workload != WORKLOAD or L != synth.WORKLOADS[WORKLOAD].length or \
+            batch != synth.WORKLOADS[WORKLOAD].batch or not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    fields = {}
+    for line in open(TRAFFIC_PROFILE):
+        if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch", "source_sha256"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(R.__file__)), "csrc")
+    for f in DECODE_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    if fields.get("source_sha256") != h.hexdigest() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return float(fields["traffic_bytes_per_launch"])
 
 
 def elapsed(a, b):
@@ -306,7 +334,8 @@ def run_recsa(args, rank, world, dev):
                      "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                      "frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "bytes_per_launch": dec_bytes, "launch_ms": dec_ms, "traffic": None},
+                     "bytes_per_launch": dec_bytes, "launch_ms": dec_ms,
+                     "traffic": measured_traffic(args.workload, L, batch)},
         "decode_ms": dec_ms,
         "two_launches": {"append_ms": app_ms, "decode_ms": two_dec_ms,
                          "step_ms": app_ms + two_dec_ms},
