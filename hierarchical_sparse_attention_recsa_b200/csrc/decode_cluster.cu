@@ -352,7 +352,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   if (tid == 0) {
     mbar_init(mb_lev, 1);
     mbar_init(mb_val, 1);
-    mbar_init(mb_kept, 1);
+    mbar_init(mb_kept, HPC);
     mbar_init(mb_folded, 1);
     mbar_init(mb_ready, unsigned(S));
     mbar_init(mb_ready + 1, unsigned(S));
@@ -380,7 +380,24 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // on mb_lev (mb_val).  Run by the whole producer warp: lane 0 arms the
   // barrier, the lanes copy one run each (the children of a kept node of
   // level lev + 1, or the orphans; the top level is one run).
-  auto issue_level = [&](int lev, bool values) {
+  // Index (in candidate order) of the r-th kept candidate of local head h at
+  // the level just selected, straight from the top-k's row masks (the
+  // compacted kept list may not exist yet).
+  auto kept_idx = [&](int h, int r) -> int {
+    const unsigned* msk = rmask + h * 32;
+    int acc = 0;
+    for (int s = 0; s < 32; ++s) {
+      unsigned mk = msk[s];
+      const int n = __popc(mk);
+      if (r < acc + n) {
+        for (int t = acc; t < r; ++t) mk &= mk - 1;
+        return s * 32 + __ffs(mk) - 1;
+      }
+      acc += n;
+    }
+    return 0;
+  };
+  auto issue_level = [&](int lev, bool values, bool from_mask) {
     const int c = cnt_c[lev];
     int lo, hi;
     share(c, lo, hi);
@@ -403,7 +420,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (r < kup) {
         c0 = r * p.b;
         c1 = c0 + p.b;
-        node0 = keptu[h * kmax + r] * p.b;
+        node0 = (from_mask ? cand_node(lev + 1, h, kept_idx(h, r)) : keptu[h * kmax + r]) * p.b;
       } else {
         c0 = nch;
         c1 = c;
@@ -440,9 +457,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   };
   // Kept leaf j of local head h's share (leaf rank sh + j * S) into its ring
   // slot: B rows of K, then B rows of V.
-  auto issue_tok = [&](int h, int j) {
+  auto issue_tok = [&](int h, int j, bool from_mask) {
     const int slot = j % NRH;
-    const int node = kept[1 * HPC * kmax + h * kmax + sh + j * S];   // level 1 = parity 1
+    const int node = from_mask ? cand_node(1, h, kept_idx(h, sh + j * S))
+                               : kept[1 * HPC * kmax + h * kmax + sh + j * S];   // level 1
     const unsigned lb = unsigned(p.B) * D * unsigned(sizeof(T));
     uint64_t* mb = mb_tok + h * NRH + slot;
     mbar_expect_tx(mb, 2u * lb);
@@ -462,15 +480,12 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     load_cs(rope, min(HSLOT, rmax), HALF, j0, cs_st);
   }
 
-  // First copies: the top level's keys and values (chain warps 0 and 1) and
-  // the first window chunks (the first window warp), before the query is
-  // loaded.
+  // First copies: the top level's keys and values (the producer warp), before
+  // the query is loaded.
   if (warp == kProducerWarp && top > 0) {
-    issue_level(top, false);
-    issue_level(top, true);
+    issue_level(top, false, false);
+    issue_level(top, true, false);
   }
-  if (warp == kChainWarps && lane < kWinRing && lane < nwch) issue_win(lane);
-
   // The query and the RoPE table rows the kernel needs (loaded together: one
   // memory round trip), then the query rotated to every level's index.
   for (int x = tid; x < G * D; x += kThreads)
@@ -533,6 +548,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   auto window_warps = [&]() {
     const int wl = warp - kChainWarps;
     const int gsl = wl * SPW + lane / LPR;
+    // the first chunks of the ring (issued here, off the prologue's barriers)
+    if (warp == kChainWarps && lane < kWinRing && lane < nwch) issue_win(lane);
     float mW[G], lW[G], accW[G][8];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -770,6 +787,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (lane == s) mine = R;
     }
     if (lane < ns) rmask[h * 32 + lane] = mine;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mb_kept);   // the producer reads the masks
   };
 
   // Kept flags and the kept list (in index order) of level lev from the row
@@ -896,7 +915,6 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       named_sync(kBarChain, kChainThreads);
       compact(lev);
       named_sync(kBarChain, kChainThreads);
-      if (tid == 0) mbar_arrive(mb_kept);
       mbar_wait(mb_val, unsigned(u) & 1u, timed_out);
       fold_values(lev);
       named_sync(kBarChain, kChainThreads);
@@ -917,19 +935,19 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (lane == 0) fence_proxy_async();
       __syncwarp();
       if (lev > 1) {
-        issue_level(lev - 1, false);
+        issue_level(lev - 1, false, true);
       } else if (lane < HPC) {
         for (int j = 0; j < NRH && j < ntok; ++j)
-          if (early_slot(lane, j)) issue_tok(lane, j);
+          if (early_slot(lane, j)) issue_tok(lane, j, true);
       }
       mbar_wait(mb_folded, unsigned(u) & 1u, timed_out);
       if (lane == 0) fence_proxy_async();
       __syncwarp();
       if (lev > 1) {
-        issue_level(lev - 1, true);
+        issue_level(lev - 1, true, false);
       } else if (lane < HPC) {
         for (int j = 0; j < NRH && j < ntok; ++j)
-          if (!early_slot(lane, j)) issue_tok(lane, j);
+          if (!early_slot(lane, j)) issue_tok(lane, j, false);
       }
     }
     if (top > 0 && lane < HPC) {
@@ -937,7 +955,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       for (int j = NRH; j < ntok; ++j) {
         mbar_wait(mb_empty + h * NRH + j % NRH, unsigned(j / NRH - 1) & 1u, timed_out);
         fence_proxy_async();
-        issue_tok(h, j);
+        issue_tok(h, j, false);
       }
     }
   };
