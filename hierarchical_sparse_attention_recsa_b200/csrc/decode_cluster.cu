@@ -941,6 +941,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
           if (early_slot(lane, j)) issue_tok(lane, j, true);
       }
       mbar_wait(mb_folded, unsigned(u) & 1u, timed_out);
+      // the next level's values are not needed before its top-k: let its keys
+      // land first, so that they get the memory bandwidth to themselves
+      if (lev > 1) mbar_wait(mb_lev, unsigned(u + 1) & 1u, timed_out);
       if (lane == 0) fence_proxy_async();
       __syncwarp();
       if (lev > 1) {
