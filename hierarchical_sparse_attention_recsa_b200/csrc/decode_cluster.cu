@@ -850,33 +850,43 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       cmul8(st2, cs_st, cs_st);
     }
     const size_t slot_elems = size_t(2) * p.B * D;
-    for (int j = 0; j < ntok; ++j) {
-      const int slot = j % NRH;
-      mbar_wait(mb_tok + hw * NRH + slot, unsigned(j / NRH) & 1u, timed_out);
-      const T* cK = tbuf + (size_t(hw) * NRH + slot) * slot_elems;
-      const T* cV = cK + size_t(p.B) * D;
+    // With S = 1 two consecutive leaves of the share sit at consecutive RoPE
+    // indices, so they are processed as one block of 2B rows (fewer, fuller
+    // iterations and one barrier per pair).
+    for (int j = 0; j < ntok;) {
+      const int nl = (S == 1 && NRH >= 2 && j + 1 < ntok) ? 2 : 1;
+      const int slot0 = j % NRH, slot1 = (j + 1) % NRH;
+      mbar_wait(mb_tok + hw * NRH + slot0, unsigned(j / NRH) & 1u, timed_out);
+      if (nl == 2) mbar_wait(mb_tok + hw * NRH + slot1, unsigned((j + 1) / NRH) & 1u, timed_out);
+      const T* cK0 = tbuf + (size_t(hw) * NRH + slot0) * slot_elems;
+      const T* cK1 = tbuf + (size_t(hw) * NRH + slot1) * slot_elems;
       float q0[8];
       if (p.rope) {
         float seed[8], r[8], t2[8];
         cmul8(seed, rj, cs_hs);
         rot_neg8(q0, qt, seed);
         lds_cs8(rrow + (p.lay.levels + 1) * D, j0, r);
-        cmul8(t2, rj, r);
+        for (int x = 0; x < nl; ++x) {
+          cmul8(t2, rj, r);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) rj[c] = t2[c];
+          for (int c = 0; c < 8; ++c) rj[c] = t2[c];
+        }
       } else {
 #pragma unroll
         for (int c = 0; c < 8; ++c) q0[c] = qt[c];
       }
-      for (int e = hs; e - hs < p.B; e += 2 * HSLOT) {
+      const int nrow = nl * p.B;
+      for (int e = hs; e - hs < nrow; e += 2 * HSLOT) {
         const int e1 = e + HSLOT;
-        const bool on0 = e < p.B, on1 = e1 < p.B;
+        const bool on0 = e < nrow, on1 = e1 < nrow;
         const int r0 = on0 ? e : 0, r1 = on1 ? e1 : 0;
+        const T* k0p = (r0 < p.B ? cK0 + size_t(r0) * D : cK1 + size_t(r0 - p.B) * D);
+        const T* k1p = (r1 < p.B ? cK0 + size_t(r1) * D : cK1 + size_t(r1 - p.B) * D);
         float k0[8], k1[8], v0[8], v1[8], q1[8];
-        SharedPairs<T, HALF>::load(cK + size_t(r0) * D, j0, k0);
-        SharedPairs<T, HALF>::load(cK + size_t(r1) * D, j0, k1);
-        SharedPairs<T, HALF>::load(cV + size_t(r0) * D, j0, v0);
-        SharedPairs<T, HALF>::load(cV + size_t(r1) * D, j0, v1);
+        SharedPairs<T, HALF>::load(k0p, j0, k0);
+        SharedPairs<T, HALF>::load(k1p, j0, k1);
+        SharedPairs<T, HALF>::load(k0p + size_t(p.B) * D, j0, v0);
+        SharedPairs<T, HALF>::load(k1p + size_t(p.B) * D, j0, v1);
         if (p.rope) {
           rot_neg8(q1, q0, cs_st);
         } else {
@@ -894,7 +904,11 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         fold2(m, l, acc, s0 * inv_sqrt_d, on0, v0, s1 * inv_sqrt_d, on1, v1);
       }
       named_sync(lbar, WPH * 32);
-      if (warp == hw * WPH && lane == 0 && j + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot);
+      if (warp == hw * WPH && lane == 0) {
+        if (j + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot0);
+        if (nl == 2 && j + 1 + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot1);
+      }
+      j += nl;
     }
   };
 
