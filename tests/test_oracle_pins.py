@@ -360,3 +360,93 @@ def test_entries_grow_logarithmically():
         assert E <= D * (16 * 8 + 15) + 64 * 8 + 512 + 63
         prev = E
     assert prev < 2000          # 2^31 tokens: still under 2000 entries
+
+
+# ---------------------------------------------------------------------------
+# ZHA routing variant
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_zha_full_mass_equals_dense_attention(rope):
+    """p = 1 with no cap expands every candidate: the reached leaves and the
+    window are every token up to t, at true positions -- dense causal RoPE
+    attention."""
+    rng = np.random.default_rng(11)
+    B, b, d, T, W = 4, 3, 8, 200, 6
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 1, 1, B, b, oracle.recsa.KEEP_ALL, W, rope=rope, rope_base=1e3)
+    for t in [0, 5, 6, 23, 99, 199]:
+        q = rng.standard_normal(d) * 2
+        res = oracle.zha_route_and_attend(q, t, K, V, tree, geo, top_p=1.0)
+        if rope:
+            qr = _rope_complex(q, t, 1e3)
+            Kr = np.stack([_rope_complex(K[j], j, 1e3) for j in range(t + 1)])
+        else:
+            qr, Kr = q, K[: t + 1]
+        ref = _sdpa(qr, Kr, V[: t + 1])
+        np.testing.assert_allclose(res["out"], ref, atol=1e-12)
+        assert res["n_exact"] == t + 1
+
+
+def test_zha_top_p_matches_subset_brute_force():
+    """The top-p set is the smallest set of candidates whose softmax mass
+    reaches p, and among sets of that size the heaviest (brute force over all
+    subsets); a cap limits its size."""
+    import itertools
+    rng = np.random.default_rng(3)
+    for trial in range(200):
+        n = int(rng.integers(1, 8))
+        s = rng.standard_normal(n) * float(rng.uniform(0.1, 4))
+        p = float(rng.uniform(0.05, 1.0))
+        cap = int(rng.integers(1, 9))
+        w = np.exp(s - s.max())
+        w = w / w.sum()
+        best = None
+        for m in range(1, n + 1):
+            subs = [c for c in itertools.combinations(range(n), m)]
+            heavy = max(subs, key=lambda c: (sum(w[list(c)]), [-x for x in c]))
+            if sum(w[list(heavy)]) >= p - 1e-12 or m == min(cap, n):
+                best = sorted(heavy)
+                break
+        got = oracle.top_p_prefix(list(s), p, cap)
+        assert got == best, (trial, s, p, cap, got, best)
+
+
+def test_zha_tiny_p_is_greedy_descent():
+    """With a tiny p one candidate per level is expanded: the arg-max of
+    q . key, descending from the top; checked against a greedy descent over
+    node spans written here independently of the oracle's candidate lists."""
+    rng = np.random.default_rng(5)
+    B, b, d, T, W = 4, 3, 8, 300, 4
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    levels = oracle.build_tree(K, V, r, B, b)
+    tree = oracle.FullTree(levels)
+    geo = Geometry(d, 1, 1, B, b, oracle.recsa.KEEP_ALL, W, rope=False)
+    for t in [40, 101, 299]:
+        q = rng.standard_normal(d)
+        res = oracle.zha_route_and_attend(q, t, K, V, tree, geo, top_p=1e-9)
+        a = max(0, t + 1 - W) // B
+        # greedy: at each level the arg-max among the children of the previous
+        # pick plus every visible node whose parent is not visible
+        span = [B * b ** l for l in range(len(levels))]
+        vis = [a * B // span[l] for l in range(len(levels))]
+        top = max(l + 1 for l in range(len(levels)) if vis[l] > 0)
+        pick = None
+        for lev in range(top, 0, -1):
+            nodes = set()
+            if pick is not None:
+                nodes |= {pick * b + c for c in range(b)}
+            up = vis[lev] if lev < top else 0
+            nodes |= set(range(b * up, vis[lev - 1]))
+            nodes = sorted(nodes)
+            sc = [q @ levels[lev - 1][0][n] for n in nodes]
+            pick = nodes[int(np.argmax(sc))]
+            assert res["kept"][lev] == [pick]
+        exact = list(range(pick * B, pick * B + B)) + list(range(a * B, t + 1))
+        lg = K[exact] @ q / math.sqrt(d)
+        pw = np.exp(lg - lg.max())
+        np.testing.assert_allclose(res["out"], (pw[:, None] * V[exact]).sum(0) / pw.sum(),
+                                   atol=1e-12)
