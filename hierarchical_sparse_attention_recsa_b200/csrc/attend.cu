@@ -61,6 +61,10 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   float* mrun = reinterpret_cast<float*>(tpos + G * kTokChunk);  // [G]
   float* lrun = mrun + 8;
   float* scl = lrun + 8;
+  // ZHA: per-head routed counts (the expanded node count differs per head)
+  int* zkup = reinterpret_cast<int*>(scl + 8);                 // [8] expanded one level up
+  int* zc = zkup + 8;                                          // [8][kMaxLevels + 1] candidates
+  int* zk = zc + 8 * (kMaxLevels + 1);                         // [8][kMaxLevels + 1] expanded
 
   const int64_t t = decode ? len_dev[seq] - 1 : q_start + qi;
   const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * d;
@@ -84,17 +88,20 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
   }
   for (int x = tid; x < G * d; x += kThreads) qf[x] = ld<T>(Q, qrow + x);
-  if (tid < 8) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; }
+  if (tid < 8) { mrun[tid] = -INFINITY; lrun[tid] = 0.f; zkup[tid] = 0; }
   float acc[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) acc[u] = 0.f;
   __syncthreads();
 
+  const bool zha = p.mode == RECSA_MODE_ZHA;
+  constexpr int LS = kMaxLevels + 1;
+  // Query rotated to index idx (idx < 0: copied un-rotated).
   auto rotate_q = [&](int64_t idx) {
     for (int x = tid; x < G * half; x += kThreads) {
       const int h = x / half, j = x % half;
       const float x1 = qf[h * d + j], x2 = qf[h * d + j + half];
-      if (p.rope) {
+      if (p.rope && idx >= 0) {
         const float2 cs = rope[idx * half + j];
         qr[h * d + j] = x1 * cs.x - x2 * cs.y;
         qr[h * d + j + half] = x2 * cs.x + x1 * cs.y;
@@ -104,7 +111,8 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       }
     }
   };
-  // Dot of head h's rotated query with a row rotated to index idx; warp-wide.
+  // Dot of head h's rotated query with a row rotated to index idx (idx < 0:
+  // not rotated); warp-wide.
   auto dot_row = [&](int h, const auto* row, int64_t idx) -> float {
     float s = 0.f;
 #pragma unroll
@@ -112,7 +120,7 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       const int j = lane + 32 * u;
       const float k1 = ld(row, j), k2 = ld(row, j + half);
       float r1 = k1, r2 = k2;
-      if (p.rope) {
+      if (p.rope && idx >= 0) {
         const float2 cs = rope[idx * half + j];
         r1 = k1 * cs.x - k2 * cs.y;
         r2 = k2 * cs.x + k1 * cs.y;
@@ -167,31 +175,38 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     __syncthreads();
   };
 
-  int kup = 0;
-  int64_t ent = 0, keys_read = 0;
-  int cnt_c[kMaxLevels + 1], cnt_k[kMaxLevels + 1];
+  // Per head: expanded count one level up (zkup), candidates and kept per
+  // level (zc, zk).  Under RecSA every head has the same counts; under ZHA
+  // the top-p set size, hence the next level's candidates, differ per head.
   for (int lev = top; lev >= 1; --lev) {
     const int64_t vup = lev < top ? vis[lev + 1] : 0;
-    const int nchild = p.b * kup;
-    const int c = nchild + int(vis[lev] - p.b * vup);
-    for (int x = tid; x < G * c; x += kThreads) {
-      const int h = x / c, ii = x % c;
-      cand[h * cmax + ii] = ii < nchild ? kept[h * kmax + ii / p.b] * p.b + ii % p.b
-                                        : int(p.b * vup + (ii - nchild));
+    const int norph = int(vis[lev] - p.b * vup);
+    int cmx = 0;
+    for (int h = 0; h < G; ++h) cmx = max(cmx, p.b * zkup[h] + norph);
+    for (int x = tid; x < G * cmx; x += kThreads) {
+      const int h = x / cmx, ii = x % cmx;
+      const int nchild = p.b * zkup[h];
+      if (ii < nchild + norph)
+        cand[h * cmax + ii] = ii < nchild ? kept[h * kmax + ii / p.b] * p.b + ii % p.b
+                                          : int(p.b * vup + (ii - nchild));
     }
-    rotate_q(c);
+    // RecSA: candidate-local positions, query at index c (all heads share c).
+    // ZHA: plain dot products of the un-rotated query and summary keys.
+    rotate_q(zha ? -1 : cmx);
     __syncthreads();
     const float* keys = level_keys(p, const_cast<void*>(tree), lev, seq, g);
     const float* vals = level_vals(p, const_cast<void*>(tree), lev, seq, g);
-    for (int pr = warp; pr < G * c; pr += kWarps) {
-      const int h = pr / c, ii = pr % c;
-      const float s = dot_row(h, keys + int64_t(cand[h * cmax + ii]) * d, ii);
+    for (int pr = warp; pr < G * cmx; pr += kWarps) {
+      const int h = pr / cmx, ii = pr % cmx;
+      if (ii >= p.b * zkup[h] + norph) continue;  // warp-uniform
+      const float s = dot_row(h, keys + int64_t(cand[h * cmax + ii]) * d, zha ? -1 : ii);
       if (lane == 0) score[h * cmax + ii] = s;
     }
     __syncthreads();
-    const int kap = c < p.k ? c : p.k;
-    for (int x = tid; x < G * c; x += kThreads) {
-      const int h = x / c, ii = x % c;
+    for (int x = tid; x < G * cmx; x += kThreads) {
+      const int h = x / cmx, ii = x % cmx;
+      const int c = p.b * zkup[h] + norph;
+      if (ii >= c) continue;
       const float s = score[h * cmax + ii];
       const float* row = score + h * cmax;
       int r = 0;
@@ -200,49 +215,102 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         r += (sj > s) || (sj == s && jj < ii);
       }
       rank[h * cmax + ii] = r;
+      if (zha && r == 0) scl[h] = s;  // the level's maximum score
     }
     __syncthreads();
-    for (int x = tid; x < G * c; x += kThreads) {
-      const int h = x / c, ii = x % c;
-      if (rank[h * cmax + ii] < kap) {
+    if (zha) {
+      // Top-p: weights exp(s - max) laid out in rank order, then the shortest
+      // rank prefix whose mass reaches p of the total, capped at min(k, c).
+      for (int x = tid; x < G * cmx; x += kThreads) {
+        const int h = x / cmx, ii = x % cmx;
+        if (ii < p.b * zkup[h] + norph)
+          wts[h * cmax + rank[h * cmax + ii]] = expf(score[h * cmax + ii] - scl[h]);
+      }
+      __syncthreads();
+      if (warp < G) {
+        const int h = warp;
+        const int c = p.b * zkup[h] + norph;
+        const int cap = c < p.k ? c : p.k;
+        int cnt = cap;
+        if (p.top_p < 1.f) {
+          float tot = 0.f;
+          for (int e = lane; e < c; e += 32) tot += wts[h * cmax + e];
+          const float thr = p.top_p * warp_sum(tot);
+          float run = 0.f;
+          for (int b0 = 0; b0 < c; b0 += 32) {
+            const int e = b0 + lane;
+            float x = e < c ? wts[h * cmax + e] : 0.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const float y = __shfl_up_sync(0xffffffffu, x, o);
+              if (lane >= o) x += y;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, e < c && run + x >= thr);
+            if (hit) {
+              cnt = min(cnt, b0 + __ffs(hit));
+              break;
+            }
+            run += __shfl_sync(0xffffffffu, x, 31);
+          }
+        }
+        if (lane == 0) {
+          zc[h * LS + lev] = c;
+          zk[h * LS + lev] = cnt;
+        }
+      }
+    } else if (tid < G) {
+      const int c = p.b * zkup[tid] + norph;
+      zc[tid * LS + lev] = c;
+      zk[tid * LS + lev] = c < p.k ? c : p.k;
+    }
+    __syncthreads();
+    for (int x = tid; x < G * cmx; x += kThreads) {
+      const int h = x / cmx, ii = x % cmx;
+      const int kap = zk[h * LS + lev];
+      if (ii < zc[h * LS + lev] && rank[h * cmax + ii] < kap) {
         int pos = 0;
         for (int jj = 0; jj < ii; ++jj) pos += rank[h * cmax + jj] < kap;
         kept[h * kmax + pos] = cand[h * cmax + ii];
       }
     }
     __syncthreads();
-    softmax_update(
-        score, wts, cmax, c, [&](int h, int e) { return rank[h * cmax + e] < kap; },
-        [&](int h, int e) { return vals + int64_t(cand[h * cmax + e]) * d; });
+    if (!zha)  // RecSA: unselected summaries join the softmax
+      softmax_update(
+          score, wts, cmax, cmx,
+          [&](int h, int e) { return rank[h * cmax + e] < zk[h * LS + lev]; },
+          [&](int h, int e) { return vals + int64_t(cand[h * cmax + e]) * d; });
     if (trace) {
-      for (int x = tid; x < G * kap; x += kThreads) {
-        const int h = x / kap, j = x % kap;
+      for (int x = tid; x < G * kmax; x += kThreads) {
+        const int h = x / kmax, j = x % kmax;
+        if (j >= zk[h * LS + lev]) continue;
         const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + h) * tstride;
         trace[rec + kTraceHead + (lev - 1) * p.k + j] = kept[h * kmax + j];
       }
     }
-    cnt_c[lev] = c;
-    cnt_k[lev] = kap;
-    ent += c - kap;
-    keys_read += c;
-    kup = kap;
+    if (tid < G) zkup[tid] = zk[tid * LS + lev];
+    __syncthreads();
   }
 
-  // Token level: kept leaf blocks, then the window.
-  const int nleaf = top > 0 ? kup : 0;
-  const int64_t n0 = int64_t(nleaf) * p.B + (t + 1 - a * p.B);
-  rotate_q(n0 - 1);
+  // Token level: kept leaf blocks, then the window.  RecSA indexes them
+  // 0..n0-1 with the query at n0-1; ZHA keeps their true positions.
+  auto n0_of = [&](int h) -> int64_t {
+    return int64_t(top > 0 ? zkup[h] : 0) * p.B + (t + 1 - a * p.B);
+  };
+  int64_t n0max = 0;
+  for (int h = 0; h < G; ++h) n0max = n0_of(h) > n0max ? n0_of(h) : n0max;
+  rotate_q(zha ? t : n0max - 1);
   __syncthreads();
   const int64_t kvbase = (seq * p.hkv + g) * p.cap;
-  for (int64_t base = 0; base < n0; base += kTokChunk) {
-    const int nt = int(n0 - base < kTokChunk ? n0 - base : kTokChunk);
+  for (int64_t base = 0; base < n0max; base += kTokChunk) {
+    const int nt = int(n0max - base < kTokChunk ? n0max - base : kTokChunk);
     for (int pr = warp; pr < G * nt; pr += kWarps) {
       const int h = pr / nt, tt = pr % nt;
       const int64_t ii = base + tt;
-      const int64_t pos = ii < int64_t(nleaf) * p.B
-                              ? int64_t(kept[h * kmax + ii / p.B]) * p.B + ii % p.B
-                              : a * p.B + (ii - int64_t(nleaf) * p.B);
-      const float s = dot_row(h, K + (kvbase + pos) * d, ii);
+      if (ii >= n0_of(h)) continue;  // warp-uniform
+      const int64_t nleaf = top > 0 ? zkup[h] : 0;
+      const int64_t pos = ii < nleaf * p.B ? int64_t(kept[h * kmax + ii / p.B]) * p.B + ii % p.B
+                                           : a * p.B + (ii - nleaf * p.B);
+      const float s = dot_row(h, K + (kvbase + pos) * d, zha ? pos : ii);
       if (lane == 0) {
         tsc[h * kTokChunk + tt] = s;
         tpos[h * kTokChunk + tt] = pos;
@@ -250,11 +318,9 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
     __syncthreads();
     softmax_update(
-        tsc, tw, kTokChunk, nt, [&](int, int) { return false; },
+        tsc, tw, kTokChunk, nt, [&](int h, int e) { return base + e >= n0_of(h); },
         [&](int h, int e) { return V + (kvbase + tpos[h * kTokChunk + e]) * d; });
   }
-  ent += n0;
-  keys_read += n0;
 
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -270,14 +336,20 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   }
   if (trace && tid < G) {
     const int64_t rec = ((seq * n_q + qi) * p.hq + int64_t(g) * G + tid) * tstride;
+    const int64_t n0 = n0_of(tid);
+    int64_t ent = n0, keys_read = n0;
+    for (int lev = 1; lev <= top; ++lev) {
+      keys_read += zc[tid * LS + lev];
+      if (!zha) ent += zc[tid * LS + lev] - zk[tid * LS + lev];
+    }
     trace[rec + 0] = top;
     trace[rec + 1] = int32_t(ent);
     trace[rec + 2] = int32_t(keys_read);
     trace[rec + 3] = int32_t(n0);
     for (int lev = 1; lev <= kMaxLevels; ++lev) {
       const bool on = lev <= top;
-      trace[rec + 4 + lev - 1] = on ? cnt_c[lev] : 0;
-      trace[rec + 4 + kMaxLevels + lev - 1] = on ? cnt_k[lev] : 0;
+      trace[rec + 4 + lev - 1] = on ? zc[tid * LS + lev] : 0;
+      trace[rec + 4 + kMaxLevels + lev - 1] = on ? zk[tid * LS + lev] : 0;
     }
   }
 }
@@ -296,7 +368,8 @@ cudaError_t attend_typed(const Params& p, const void* Q, const void* K, const vo
   const int kmax = int(kk < cmax ? kk : cmax);
   const int G = p.group;
   size_t bytes = size_t(G) * d * 4 * 2 + size_t(G) * cmax * 16 + size_t(G) * kmax * 4 +
-                 size_t(G) * kTokChunk * 8 + 8 + size_t(G) * kTokChunk * 8 + 3 * 8 * 4 + 64;
+                 size_t(G) * kTokChunk * 8 + 8 + size_t(G) * kTokChunk * 8 + 3 * 8 * 4 + 64 +
+                 size_t(8 + 16 * (kMaxLevels + 1)) * 4;
   if (bytes > 200 * 1024) return cudaErrorInvalidConfiguration;
   auto kern = attend_kernel<T, P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -28,6 +28,9 @@ recsa_status check_geometry(const recsa_geometry* g) {
   if (g->rope_enabled != 0 && g->rope_enabled != 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->rope_enabled && !(g->rope_base > 1.0f)) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->batch < 1 || g->capacity < 1 || g->reserved != 0) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->mode == RECSA_MODE_ZHA && !(g->top_p > 0.f && g->top_p <= 1.f))
+    return RECSA_ERR_INVALID_GEOMETRY;
   if (g->capacity > int64_t(INT32_MAX)) return RECSA_ERR_INVALID_GEOMETRY;
   return RECSA_OK;
 }
@@ -56,6 +59,8 @@ recsa_status make_layout(const recsa_geometry* g, TreeLayout* lay) {
   int64_t rows = std::max<int64_t>(g->branching * kk + g->branching,
                                    g->leaf_block * kk + int64_t(g->window) + g->leaf_block);
   rows = std::min<int64_t>(rows, cap + g->branching + 1);
+  // ZHA attends at true positions: every distance up to the capacity
+  if (g->mode == RECSA_MODE_ZHA) rows = std::max<int64_t>(rows, cap + 1);
   if (rows > (int64_t(1) << 24)) return RECSA_ERR_UNSUPPORTED;
   lay->rope_rows = int32_t(rows);
   int64_t off = kHeaderBytes;
@@ -88,6 +93,8 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->k = g->k;
   p->W = g->window;
   p->rope = g->rope_enabled;
+  p->mode = g->mode;
+  p->top_p = g->top_p;
   p->batch = g->batch;
   p->cap = g->capacity;
   p->Bsh = p->bsh = -1;
@@ -297,7 +304,8 @@ recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, con
       !aligned(tree, 256) || (trace && !aligned(trace, 4)))
     return RECSA_ERR_MISALIGNED;
   if (n_q < 0 || q_start < 0 || q_start + n_q > geom->capacity) return RECSA_ERR_CAPACITY;
-  if (prefill_workspace_need(p, n_q) > prefill_static_bytes()) {
+  // the fixed scratch holds the window partials of the RecSA path (ZHA uses none)
+  if (p.mode == RECSA_MODE_RECSA && prefill_workspace_need(p, n_q) > prefill_static_bytes()) {
     fprintf(stderr,
             "recsa_prefill_static: %zu bytes of window partials (batch * n_q * n_q_heads * "
             "(head_dim + 2) * 4) exceed the fixed scratch of %zu bytes; split the call into "

@@ -32,6 +32,8 @@ struct TreeLayout {
 struct Params {
   int32_t dtype, d, hq, hkv, group, B, b, k, W, rope, batch;
   int32_t Bsh, bsh;   // log2 of B and b when powers of two, else -1
+  int32_t mode;       // RECSA_MODE_RECSA or RECSA_MODE_ZHA
+  float top_p;        // ZHA routing mass
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;

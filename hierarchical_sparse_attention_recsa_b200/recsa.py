@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(_HERE, "librecsa.so")
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
+MODE_RECSA = 0
+MODE_ZHA = 1
 KEEP_ALL = 2**31 - 1
 MAX_LEVELS = 16
 TRACE_MAX_K = 64
@@ -62,8 +64,10 @@ class CGeometry(ctypes.Structure):
         ("rope_enabled", ctypes.c_int32),
         ("rope_base", ctypes.c_float),
         ("batch", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("mode", ctypes.c_int32),
         ("capacity", ctypes.c_int64),
+        ("top_p", ctypes.c_float),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -83,11 +87,14 @@ class Geometry:
     dtype: int = DTYPE_BF16
     rope_enabled: int = 1
     rope_base: float = 1e6
+    mode: int = 0          # MODE_RECSA or MODE_ZHA
+    top_p: float = 0.0     # ZHA routing mass
 
     def c(self) -> CGeometry:
         return CGeometry(self.dtype, self.head_dim, self.n_q_heads, self.n_kv_heads,
                          self.leaf_block, self.branching, self.k, self.window,
-                         self.rope_enabled, self.rope_base, self.batch, 0, self.capacity)
+                         self.rope_enabled, self.rope_base, self.batch, self.mode,
+                         self.capacity, self.top_p, 0)
 
     @property
     def torch_dtype(self) -> torch.dtype:

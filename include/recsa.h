@@ -61,6 +61,10 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
 /* Largest k for which a selection trace is recorded. */
 #define RECSA_TRACE_MAX_K 64
 
+/* recsa_geometry.mode */
+#define RECSA_MODE_RECSA 0
+#define RECSA_MODE_ZHA 1
+
 /* Device error flags in the tree header (recsa_tree_error). */
 #define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
 #define RECSA_DEVERR_WAIT_TIMEOUT 0x2u /* a bounded wait of the decode kernel on its own
@@ -80,6 +84,14 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   ends at or before a*B are visible to that query.
  *   rope_enabled / rope_base: rotate-half RoPE at candidate-local indices
  *   (RecSA abstract), inverse frequencies base^(-2j/d).
+ *   mode: RECSA_MODE_RECSA (the method above) or RECSA_MODE_ZHA, the routing
+ *   variant of "Subquadratic Attention with a Hierarchical Tree-Structured
+ *   Indexer" (Figure 3): the same tree and candidates, but each level expands
+ *   the smallest set of highest-scoring candidates whose softmax mass reaches
+ *   top_p (at most k of them), scores are q . key / sqrt(d) without rotation,
+ *   and the attention covers only the tokens of the reached leaves and the
+ *   window, at their true positions with standard RoPE (no summaries).  ZHA
+ *   runs on the generic kernel.
  */
 typedef struct recsa_geometry {
   int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
@@ -93,8 +105,10 @@ typedef struct recsa_geometry {
   int32_t rope_enabled; /* 0 or 1 */
   float rope_base;      /* > 1 */
   int32_t batch;        /* sequences, >= 1 */
-  int32_t reserved;     /* must be 0 */
+  int32_t mode;         /* RECSA_MODE_RECSA (0) or RECSA_MODE_ZHA (1) */
   int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
+  float top_p;          /* ZHA: routing mass in (0, 1]; ignored in RECSA mode */
+  int32_t reserved;     /* must be 0 */
 } recsa_geometry;
 
 /* Human-readable name of a status code (static string). */
@@ -203,7 +217,7 @@ recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void
  *   needs batch * n_q * n_q_heads * (head_dim + 2) * 4 bytes of it (8065 query
  *   heads at head_dim 128, e.g. 252 queries of 32 heads); a larger call is
  *   rejected with RECSA_ERR_CAPACITY (and a message on stderr): split the
- *   query range.
+ *   query range.  RECSA_MODE_ZHA uses no window partials and no scratch.
  *   The array needs no clearing (each call writes what it reads), but every
  *   call shares it: calls that overlap on the device race.
  *   Set-up: the first call on each device, with that device current, looks up

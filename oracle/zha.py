@@ -66,8 +66,9 @@ def zha_route_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry, top_p
     ``keep_override`` (level -> expanded node ids) recomputes the output for a
     given routing (used where several routings are correct: a mass within
     rounding of p, or near-equal scores).  Returns dict(out, kept{level: ids},
-    cand{level: c}, scores{level: [..]}, mass{level: [cumulative masses in
-    routing order]}, n_exact, top, a).
+    cand{level: c}, cand_ids{level: ids in candidate order}, scores{level: [..]
+    in candidate order}, mass{level: [cumulative masses in decreasing-score
+    order]}, n_exact, top, a).
     """
     q = np.asarray(q, dtype=np.float64)
     d = q.shape[0]
@@ -77,6 +78,7 @@ def zha_route_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry, top_p
     top = len(v)
     kept_nodes: Dict[int, List[int]] = {}
     cand_count: Dict[int, int] = {}
+    cand_list: Dict[int, List[int]] = {}
     level_scores: Dict[int, List[float]] = {}
     level_mass: Dict[int, List[float]] = {}
     expanded: List[int] = []
@@ -102,6 +104,7 @@ def zha_route_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry, top_p
         expanded = [cand[i] for i in idx]
         kept_nodes[lev] = expanded
         cand_count[lev] = len(cand)
+        cand_list[lev] = cand
         level_scores[lev] = scores
     exact = [blk * B + o for blk in (expanded if top > 0 else []) for o in range(B)]
     exact += list(range(a * B, t + 1))
@@ -114,5 +117,6 @@ def zha_route_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry, top_p
     logits = ks @ qr * inv_sqrt_d
     pw = np.exp(logits - logits.max())
     out = (pw[:, None] * np.asarray(V[exact], np.float64)).sum(axis=0) / pw.sum()
-    return dict(out=out, kept=kept_nodes, cand=cand_count, scores=level_scores,
+    return dict(out=out, kept=kept_nodes, cand=cand_count, cand_ids=cand_list,
+                scores=level_scores,
                 mass=level_mass, n_exact=len(exact), top=top, a=a)

@@ -28,13 +28,16 @@ GAP = 1e-3
 TOL = {torch.bfloat16: (2e-2, 2e-3), torch.float32: (2e-4, 2e-5)}
 
 
-def geometry(w, capacity: int, batch: int, k=None, rope=1) -> R.Geometry:
+def geometry(w, capacity: int, batch: int, k=None, rope=1, top_p=None) -> R.Geometry:
+    """Library geometry of a workload; top_p given: the ZHA routing variant."""
     return R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                       leaf_block=w.leaf_block, branching=w.branching,
                       k=w.k if k is None else k, window=w.window, batch=batch,
                       capacity=capacity,
                       dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
-                      rope_enabled=rope, rope_base=w.rope_base)
+                      rope_enabled=rope, rope_base=w.rope_base,
+                      mode=R.MODE_RECSA if top_p is None else R.MODE_ZHA,
+                      top_p=0.0 if top_p is None else top_p)
 
 
 def oracle_geometry(g: R.Geometry) -> oracle.Geometry:
@@ -53,6 +56,8 @@ def read_tree_level(g: R.Geometry, tree: torch.Tensor, lev: int):
     kk = min(g.k, g.capacity)
     rows = min(max(g.branching * kk + g.branching, g.leaf_block * kk + g.window + g.leaf_block),
                g.capacity + g.branching + 1)
+    if g.mode == R.MODE_ZHA:
+        rows = max(rows, g.capacity + 1)
     off = up(256 + rows * (g.head_dim // 2) * 8)
     span = g.leaf_block
     for l in range(1, lev + 1):
@@ -142,3 +147,80 @@ def check_query(stats: Stats, gpu_out, trace_rec, q, t, K, V, tree_src, og, k_tr
 
 def to_np(x: torch.Tensor) -> np.ndarray:
     return x.detach().float().cpu().numpy().astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# ZHA routing variant
+# ---------------------------------------------------------------------------
+
+MASS_EPS = 1e-3   # fp32 softmax masses vs float64: a few 1e-6; two orders of margin
+
+
+def zha_level_clear(scores, mass, n: int, p: float, cap: int, gap: float = GAP) -> bool:
+    """The top-p decision at one level cannot flip under fp32 rounding: the
+    score gap at the cut exceeds ``gap`` and the masses before and at the cut
+    are more than MASS_EPS from p (or the cap decides)."""
+    s = sorted(scores, reverse=True)
+    if n < len(s) and s[n - 1] - s[n] <= gap:
+        return False
+    if p >= 1.0:
+        return True
+    if n > 1 and mass[n - 2] >= p - MASS_EPS:
+        return False
+    if n < cap and mass[n - 1] < p + MASS_EPS:
+        return False
+    return True
+
+
+def zha_routing_valid(res: dict, p: float, k: int, gap: float = GAP) -> None:
+    """Assert that the routing in ``res`` (an oracle result, possibly for a
+    given routing) is a correct top-p choice within rounding at every level:
+    the expanded set is a score prefix (up to ties within ``gap``) and its size
+    is where the mass crosses p (within MASS_EPS) or the cap."""
+    for lev, kept in res["kept"].items():
+        ids = res["cand_ids"][lev]
+        sc = res["scores"][lev]
+        mass = res["mass"][lev]
+        n, c = len(kept), len(ids)
+        cap = min(k, c)
+        assert 1 <= n <= cap, (lev, n, cap)
+        inside = [sc[i] for i, x in enumerate(ids) if x in set(kept)]
+        outside = [sc[i] for i, x in enumerate(ids) if x not in set(kept)]
+        if outside:
+            assert min(inside) >= max(outside) - gap, (lev, min(inside), max(outside))
+        if p >= 1.0:
+            assert n == cap, (lev, n, cap)
+            continue
+        if n > 1:
+            assert mass[n - 2] < p + MASS_EPS, (lev, n, mass[n - 2], p)
+        if n < cap:
+            assert mass[n - 1] >= p - MASS_EPS, (lev, n, mass[n - 1], p)
+
+
+def check_query_zha(stats: Stats, gpu_out, trace_rec, q, t, K, V, tree_src, og, p: float,
+                    k_trace):
+    """Compare one (query, head) of the GPU's ZHA path with the oracle."""
+    res = oracle.zha_route_and_attend(q, t, K, V, tree_src, og, p)
+    if trace_rec is not None:
+        tr = parse_trace(trace_rec, k_trace)
+        assert tr["top"] == res["top"]
+        gpu_kept = {l: list(v) for l, v in tr["kept"].items()}
+        clear = all(zha_level_clear(res["scores"][l], res["mass"][l], len(res["kept"][l]), p,
+                                    min(og.k, res["cand"][l]))
+                    for l in res["kept"])
+        if clear:
+            stats.clear += 1
+            assert gpu_kept == {l: list(v) for l, v in res["kept"].items()}, (t, gpu_kept,
+                                                                              res["kept"])
+        else:
+            stats.near_tie += 1
+            if gpu_kept != {l: list(v) for l, v in res["kept"].items()}:
+                res = oracle.zha_route_and_attend(q, t, K, V, tree_src, og, p,
+                                                  keep_override=gpu_kept)
+                zha_routing_valid(res, p, og.k)
+        assert tr["cand"] == res["cand"]
+        assert tr["n_exact"] == res["n_exact"]
+        assert tr["entries"] == res["n_exact"]
+        assert tr["keys_read"] == res["n_exact"] + sum(res["cand"].values())
+    stats.add(gpu_out, res["out"])
+    return res

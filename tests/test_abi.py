@@ -41,9 +41,11 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layout_matches_header(lib):
-    # 12 int32/float fields then one int64: 56 bytes, capacity at offset 48.
-    assert ctypes.sizeof(R.CGeometry) == 56
+    # 12 int32/float fields, one int64, then top_p and reserved: 64 bytes.
+    assert ctypes.sizeof(R.CGeometry) == 64
     assert R.CGeometry.capacity.offset == 48
+    assert R.CGeometry.top_p.offset == 56
+    assert R.CGeometry.reserved.offset == 60
 
 
 def test_status_strings(lib):
@@ -58,6 +60,8 @@ def test_status_strings(lib):
     dict(branching=32, batch=8, capacity=1048576 + 256),
     dict(leaf_block=32, branching=8, k=16, window=1024, batch=1, capacity=2097152 + 128),
     dict(k=R.KEEP_ALL, capacity=8192, rope_enabled=0),
+    dict(mode=R.MODE_ZHA, top_p=0.9),
+    dict(mode=R.MODE_ZHA, top_p=1.0, k=R.KEEP_ALL, capacity=8192),
 ])
 def test_valid_geometries(lib, kw):
     R.recsa_validate(geo(**kw))
@@ -67,6 +71,8 @@ def test_valid_geometries(lib, kw):
     dict(head_dim=96), dict(n_q_heads=24), dict(n_q_heads=12, n_kv_heads=4),
     dict(branching=1), dict(window=0), dict(k=0), dict(leaf_block=0), dict(batch=0),
     dict(capacity=0), dict(dtype=7), dict(rope_base=1.0), dict(n_kv_heads=0),
+    dict(mode=2), dict(mode=R.MODE_ZHA, top_p=0.0), dict(mode=R.MODE_ZHA, top_p=1.5),
+    dict(mode=R.MODE_ZHA, top_p=float("nan")),
 ])
 def test_invalid_geometries(lib, kw):
     with pytest.raises(R.RecsaError) as e:
@@ -89,6 +95,8 @@ def expected_tree_bytes(g: R.Geometry) -> int:
     kk = min(g.k, g.capacity)
     rows = min(max(g.branching * kk + g.branching, g.leaf_block * kk + g.window + g.leaf_block),
                g.capacity + g.branching + 1)
+    if g.mode == R.MODE_ZHA:  # true positions: one row per position
+        rows = max(rows, g.capacity + 1)
     total = up(256 + rows * (g.head_dim // 2) * 8)
     span = g.leaf_block
     while g.capacity // span >= 1:
@@ -98,7 +106,8 @@ def expected_tree_bytes(g: R.Geometry) -> int:
     return total
 
 
-@pytest.mark.parametrize("kw", [dict(), dict(batch=1, capacity=4096 + 17), dict(k=R.KEEP_ALL)])
+@pytest.mark.parametrize("kw", [dict(), dict(batch=1, capacity=4096 + 17), dict(k=R.KEEP_ALL),
+                                dict(mode=R.MODE_ZHA, top_p=0.5)])
 def test_tree_bytes(lib, kw):
     g = geo(**kw)
     assert R.recsa_tree_bytes(g) == expected_tree_bytes(g)

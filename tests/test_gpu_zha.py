@@ -1,0 +1,255 @@
+"""Parity of the ZHA routing variant (geometry mode RECSA_MODE_ZHA) with the
+float64 oracle, through the C ABI.
+
+"Subquadratic Attention with a Hierarchical Tree-Structured Indexer" (ZHA),
+Figure 3 caption: top-p expansion down the tree over dot-product scores, main
+attention over the tokens of the reached leaves (plus the exact window, at
+true positions).  The routing check is bit-exact where no level's decision is
+within rounding of its threshold or of a score tie, and a validity check plus
+an output comparison under the GPU's routing elsewhere (recsa_testlib).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
+from hierarchical_sparse_attention_recsa_b200 import recsa as R
+
+from recsa_testlib import (Stats, alloc_tree, check_query_zha, geometry, oracle_geometry,
+                           parse_trace, to_np)
+
+pytestmark = pytest.mark.gpu
+
+TINY = synth.WORKLOADS["tiny-4k"]
+MODEL = synth.WORKLOADS["qwen3-4b-131k"]
+ZK = 16   # tiny tree: a cap above the typical top-p set, so the mass decides
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build_lib.build()
+    R.lib()
+
+
+def _setup(w, lens, capacity, top_p, seed=0, k=None, rope=1):
+    batch = len(lens)
+    g = geometry(w, capacity, batch, k=k, rope=rope, top_p=top_p)
+    K, V, r = synth.make_kv(w, capacity, seed=seed, device="cpu", batch=batch)
+    Kd, Vd, rd = K.cuda(), V.cuda(), r.cuda()
+    tree = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, lens, rd, 0, tree)
+    torch.cuda.synchronize()
+    return g, K, V, r, Kd, Vd, rd, tree
+
+
+def _trees(g, K, V, r, lens):
+    out = {}
+    for s, L in enumerate(lens):
+        for h in range(g.n_kv_heads):
+            Kh, Vh = to_np(K[s, h, :L]), to_np(V[s, h, :L])
+            out[(s, h)] = (Kh, Vh, oracle.FullTree(
+                oracle.build_tree(Kh, Vh, r.double().numpy(), g.leaf_block, g.branching)))
+    return out
+
+
+@pytest.mark.parametrize("top_p", [0.3, 0.9])
+def test_zha_decode_tiny(top_p):
+    L, nq = TINY.length, TINY.n_q
+    g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, top_p, seed=20, k=ZK)
+    trees = _trees(g, K, V, r, [L])
+    pos = torch.full((1, nq), L - 1, dtype=torch.int64)
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=21, n_needles=16)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    sizes = []
+    for i in range(nq):
+        for h in range(g.n_q_heads):
+            res = check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh,
+                                  Vh, src, og, top_p, g.k)
+            sizes += [len(v) for v in res["kept"].values()]
+    st.check(torch.float32, f"zha decode tiny p={top_p}")
+    assert st.clear > 0.7 * nq * g.n_q_heads
+    # the mass target, not the cap, ends some levels
+    assert min(sizes) < g.k
+
+
+@pytest.mark.parametrize("entry", ["prefill", "prefill-workspace", "prefill-static"])
+def test_zha_prefill_tiny(entry):
+    L, top_p = TINY.length, 0.8
+    g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, top_p, seed=22, k=ZK)
+    trees = _trees(g, K, V, r, [L])
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=23)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, L, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    if entry == "prefill-static":
+        R.recsa_prefill_static(g, Qd, Kd, Vd, tree, 0, L, O, trace)
+    else:
+        ws = None
+        if entry == "prefill-workspace":
+            ws = torch.empty(R.recsa_prefill_workspace_bytes(g, L), dtype=torch.uint8,
+                             device="cuda")
+        R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O, trace, workspace=ws)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    rng = np.random.default_rng(3)
+    B, W = g.leaf_block, g.window
+    sample = sorted(set([0, 1, B - 1, B, W - 1, W, W + 1, W + B - 1, W + B, 2 * W + 7, L - 2,
+                         L - 1] + list(rng.integers(0, L, 40))))
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for t in sample:
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, t, h], tr[0, t, h], to_np(Q[0, t, h]), t, Kh, Vh, src, og,
+                            top_p, g.k)
+    st.check(torch.float32, f"zha {entry} tiny")
+
+
+@pytest.mark.parametrize("top_p", [0.5, 0.95])
+def test_zha_decode_model_small(top_p):
+    lens = [20000, 13001]
+    g, K, V, r, Kd, Vd, rd, tree = _setup(MODEL, lens, 20480, top_p, seed=24)
+    trees = _trees(g, K, V, r, lens)
+    nq = 3
+    pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(MODEL, K, pos, seed=25, n_needles=2)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for i in range(nq):
+            for h in range(g.n_q_heads):
+                Kh, Vh, src = trees[(s, h // G)]
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha decode model small p={top_p}")
+
+
+@pytest.mark.parametrize("wname,rope", [("tiny-4k", 1), ("tiny-4k", 0), ("qwen3-4b-131k", 1)])
+def test_zha_full_mass_keep_all_is_dense(wname, rope):
+    """p = 1 with no cap reaches every leaf: dense causal attention."""
+    w = synth.WORKLOADS[wname]
+    L = 1500 if w.head_dim == 64 else 700
+    g, K, V, r, Kd, Vd, rd, tree = _setup(w, [L], L, 1.0, seed=26, k=R.KEEP_ALL, rope=rope)
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(w, K, pos, seed=27)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O)
+    Od = torch.empty_like(Qd[:, :1])
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd[:, -1:].contiguous(), Kd, Vd, tree, lens, 1, Od)
+    torch.cuda.synchronize()
+    G = g.n_q_heads // g.n_kv_heads
+    O_, Od_ = to_np(O), to_np(Od)
+    st = Stats()
+    for t in [0, 5, 63, 64, 65, 300, L - 1]:
+        for h in range(0, g.n_q_heads, max(1, g.n_q_heads // 4)):
+            ref = oracle.dense_causal_attention(to_np(Q[0, t, h]), t, to_np(K[0, h // G]),
+                                                to_np(V[0, h // G]), rope=bool(rope),
+                                                rope_base=w.rope_base)
+            st.add(O_[0, t, h], ref)
+            if t == L - 1:
+                st.add(Od_[0, 0, h], ref)
+    st.check(w.dtype, "zha full mass")
+
+
+def test_zha_tiny_p_expands_one_node_per_level():
+    """A mass target below every candidate's share expands only the arg-max."""
+    L = TINY.length
+    g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, 1e-6, seed=28)
+    trees = _trees(g, K, V, r, [L])
+    nq = 32
+    pos = torch.full((1, nq), L - 1, dtype=torch.int64)
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=29)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for i in range(nq):
+        for h in range(g.n_q_heads):
+            t_ = parse_trace(tr[0, i, h], g.k)
+            assert all(len(v) == 1 for v in t_["kept"].values())
+            check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh, Vh, src,
+                            og, 1e-6, g.k)
+    st.check(torch.float32, "zha tiny p")
+
+
+def test_zha_decode_step_equals_append_then_decode():
+    """In ZHA mode the one-call step (append, then the routed decode) equals
+    the two calls, across leaf completions, and matches the oracle."""
+    w, top_p = MODEL, 0.9
+    lens0 = [4000, 4031]
+    steps = 70
+    cap = 4096 + 256
+    g, K, V, r, Kd, Vd, rd, tree_a = _setup(w, lens0, cap, top_p, seed=30)
+    tree_b = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, lens0, rd, 0, tree_b)
+    Ka, Va, Kb, Vb = Kd.clone(), Vd.clone(), Kd.clone(), Vd.clone()
+    for X in (Ka, Va, Kb, Vb):
+        X[0, :, 4000:] = 0
+        X[1, :, 4031:] = 0
+    la = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    lb = la.clone()
+    og = oracle_geometry(g)
+    G = g.n_q_heads // g.n_kv_heads
+    st = Stats()
+    ti = R.recsa_trace_ints(g)
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        lens_now = [L + step + 1 for L in lens0]
+        pos = torch.tensor([[L - 1] for L in lens_now], dtype=torch.int64)
+        Q, _, _ = synth.make_queries(w, K, pos, seed=200 + step)
+        Qd = Q.cuda()
+        Oa = torch.empty_like(Qd)
+        Ob = torch.empty_like(Qd)
+        trace = torch.zeros((2, 1, g.n_q_heads, ti), dtype=torch.int32, device="cuda")
+        R.recsa_decode_step(g, Qd, Ka, Va, kn, vn, la, rd, 0, tree_a, 1, Oa, trace)
+        R.recsa_append(g, Kb, Vb, kn, vn, lb, rd, 0, tree_b)
+        R.recsa_decode(g, Qd, Kb, Vb, tree_b, lb, 1, Ob)
+        torch.cuda.synchronize()
+        assert torch.equal(Oa, Ob), step
+        assert la.cpu().tolist() == lens_now
+        if step in (31, steps - 1):
+            tr = trace.cpu().numpy()
+            for s in range(2):
+                Kh_all = to_np(K[s, :, :lens_now[s]])
+                Vh_all = to_np(V[s, :, :lens_now[s]])
+                for h in range(0, g.n_q_heads, 7):
+                    Kh, Vh = Kh_all[h // G], Vh_all[h // G]
+                    src = oracle.LazyTree(Kh, Vh, r.double().numpy(), g.leaf_block, g.branching)
+                    check_query_zha(st, to_np(Oa[s, 0, h]), tr[s, 0, h], to_np(Q[s, 0, h]),
+                                    lens_now[s] - 1, Kh, Vh, src, og, top_p, g.k)
+    st.check(torch.bfloat16, "zha decode step")
+    assert torch.equal(Ka, Kb) and torch.equal(Va, Vb)
+    assert torch.equal(tree_a[256:], tree_b[256:])
