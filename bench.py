@@ -349,7 +349,66 @@ def run_recsa(args, rank, world, dev):
         out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
+    if not args.no_zha:
+        out["zha"] = run_zha(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind,
+                             cpu=(rank == 0 and world == 1 and not args.no_cpu))
     return out
+
+
+ZHA_TOP_P = 0.9
+
+
+def run_zha(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, cpu):
+    """The ZHA routing variant (top-p expansion, exact tokens of the reached
+    leaves and the window at true positions) on the same cache: its own tree
+    (same pooling; the RoPE table covers every position), then the batch's
+    decode queries at t = L - 1, timed per launch like the main decode."""
+    batch = Kc.shape[0]
+    g = R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   leaf_block=w.leaf_block, branching=w.branching, k=w.k, window=w.window,
+                   batch=batch, capacity=cap,
+                   dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
+                   rope_enabled=1, rope_base=w.rope_base, mode=R.MODE_ZHA, top_p=ZHA_TOP_P)
+    tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
+    R.recsa_build(g, Kc, Vc, [L] * batch, r, 0, tree)
+    lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
+    O = torch.empty_like(Qs[0])
+    n = min(args.steps, Qs.shape[0])
+    traces = torch.zeros((n, batch, 1, w.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                         device="cuda")
+    for i in range(args.warmup):
+        R.recsa_decode(g, Qs[i % Qs.shape[0]], Kc, Vc, tree, lens, 1, O)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        flush()
+        ev[i][0].record(stream)
+        R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O)
+        ev[i][1].record(stream)
+        R.recsa_decode(g, Qs[i], Kc, Vc, tree, lens, 1, O, traces[i])   # untimed, for counts
+    torch.cuda.synchronize()
+    dec_ms = sum(elapsed(a, b) for a, b in ev) / n
+    tr = traces.cpu().numpy()
+    G = w.n_q_heads // w.n_kv_heads
+    nb = [counts.decode_bytes_from_trace(tr[i], np.full(batch, L), w.leaf_block, w.branching,
+                                         w.window, G, w.head_dim, elem_bytes(w), w.k,
+                                         summary_values=False)["bytes"] for i in range(n)]
+    kept = tr[..., 4 + 16:4 + 16 + R.recsa_num_levels(g, L)].astype(np.float64)
+    nbytes = float(np.mean(nb))
+    achieved = nbytes / (dec_ms / 1e3) / 1e9
+    res = {"top_p": ZHA_TOP_P, "value": batch / (dec_ms / 1e3), "unit": "queries/s",
+           "decode_ms": dec_ms, "kernel": "zha_attend_kernel (one CTA per query head)",
+           "kept_per_level_mean": [float(x) for x in kept.mean(axis=(0, 1, 2, 3))],
+           "exact_tokens_mean": float(tr[..., 3].mean()),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                        "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
+                        "bytes_per_launch": nbytes, "traffic": None}}
+    del tree, traces
+    torch.cuda.empty_cache()
+    if cpu:
+        res["cpu_baseline"] = cpu_baseline(args.workload, seconds=min(args.cpu_seconds, 10.0),
+                                           top_p=ZHA_TOP_P)
+    return res
 
 
 def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
@@ -497,13 +556,19 @@ class OracleDecode:
         # untimed: pool the nodes the first query visits (the oracle's tree build)
         self.query_heads(1)
 
-    def query_heads(self, n_heads):
+    def query_heads(self, n_heads, top_p=None):
+        """Run n_heads (query, head) pairs; top_p given: the ZHA routing variant."""
         done = 0
         while done < n_heads:
             i = self.i % self.Q.shape[0]
             t = self.L + i - 1
             h = done % self.G
-            self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree, self.geo)
+            if top_p is None:
+                self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
+                                                self.geo)
+            else:
+                self.oracle.zha_route_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
+                                                 self.geo, top_p)
             done += 1
             if h == self.G - 1:
                 self.i += 1
@@ -518,18 +583,21 @@ def _single_thread():
         return None
 
 
-def cpu_baseline(workload=WORKLOAD, seconds=15.0):
+def cpu_baseline(workload=WORKLOAD, seconds=15.0, top_p=None):
     lim = _single_thread()
     o = OracleDecode(workload)
+    if top_p is not None:
+        o.query_heads(o.G, top_p)      # untimed: pool the nodes this routing visits first
     t0 = time.perf_counter()
     heads = 0
     while time.perf_counter() - t0 < seconds:
-        heads += o.query_heads(o.G)
+        heads += o.query_heads(o.G, top_p)
     dt = time.perf_counter() - t0
     del lim
+    what = "decode" if top_p is None else f"ZHA decode (top-p {top_p})"
     return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
             "kind": "oracle",
-            "sample": f"{heads} query-heads (decode at t=L, one KV head's tree, G={o.G}) in "
+            "sample": f"{heads} query-heads ({what} at t=L, one KV head's tree, G={o.G}) in "
                       f"{dt:.1f} s; queries/s = query-heads/{o.heads_per_query}/s; tree pooling "
                       "untimed"}
 
@@ -577,6 +645,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-dense-prefill", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-zha", action="store_true",
+                    help="skip the ZHA routing-variant decode leg")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--only-decode", action="store_true",
                     help="decode steps only (no prefill, dense, e2e or CPU legs); for profiling")
@@ -585,7 +655,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.only_decode:
-        args.no_prefill = args.no_dense = args.no_cpu = True
+        args.no_prefill = args.no_dense = args.no_cpu = args.no_zha = True
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))

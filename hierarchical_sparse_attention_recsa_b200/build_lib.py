@@ -16,7 +16,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librecsa.so")
 SOURCES = ["recsa_api.cu", "build.cu", "attend.cu", "decode_cluster.cu",
            "prefill_warp.cu", "prefill_window.cu",
-           "prefill_static.cu"]
+           "prefill_static.cu", "zha_attend.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

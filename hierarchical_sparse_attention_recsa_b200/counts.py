@@ -40,14 +40,16 @@ def per_query_counts(t: np.ndarray, B: int, b: int, k: int, W: int, levels: int)
 
 
 def decode_bytes_from_trace(trace: np.ndarray, lens: np.ndarray, B: int, b: int, W: int,
-                            G: int, d: int, elem: int, k: int) -> dict:
+                            G: int, d: int, elem: int, k: int,
+                            summary_values: bool = True) -> dict:
     """Distinct bytes one decode launch must touch, from its selection trace.
 
     trace [batch, n_q, H_q, ints] (n_q = 1); lens [batch] after the append.
     Per (sequence, KV head): summary keys of the union over its G heads of the
     candidates scored (fp32 rows), summary values of the union of unselected
-    candidates (fp32 rows), K and V rows of the union of exact tokens (dtype);
-    plus Q read and O written.
+    candidates (fp32 rows; none when ``summary_values`` is False, as in the
+    ZHA routing variant, whose softmax holds exact tokens only), K and V rows
+    of the union of exact tokens (dtype); plus Q read and O written.
     """
     batch, n_q, hq, _ = trace.shape
     hkv = hq // G
@@ -88,7 +90,7 @@ def decode_bytes_from_trace(trace: np.ndarray, lens: np.ndarray, B: int, b: int,
                     for h in range(G):
                         leaves |= kept[1][h]
                 key_rows += cand_u_total
-                val_rows += unsel_total
+                val_rows += unsel_total if summary_values else 0
                 tok_rows += len(leaves) * B + (t + 1 - a * B)
     qo = 2 * batch * n_q * hq * d * elem
     tree_bytes = (key_rows + val_rows) * d * 4

@@ -228,9 +228,12 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   if (n_q == 0) return RECSA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
-  if (decode && !getenv("RECSA_DECODE_GENERIC"))
+  if (p.mode == RECSA_MODE_ZHA) {
+    if (!getenv("RECSA_ZHA_GENERIC"))
+      e = launch_zha(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);
+  } else if (decode && !getenv("RECSA_DECODE_GENERIC")) {
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
-  if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
+  } else if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
     const void* wpart = nullptr;
     if (workspace) {
       e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, workspace, s);
@@ -316,7 +319,13 @@ recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, con
   if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
   if (n_q == 0) return RECSA_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_prefill_static(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+  cudaError_t e = cudaErrorNotSupported;
+  if (p.mode == RECSA_MODE_ZHA) {
+    if (!getenv("RECSA_ZHA_GENERIC"))
+      e = launch_zha(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, s);
+  } else {
+    e = launch_prefill_static(p, Q, K, V, tree, q_start, n_q, O, trace, s);
+  }
   if (e == cudaErrorNotSupported) {
     cudaGetLastError();
     e = launch_attend(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, s);

@@ -99,6 +99,11 @@ cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const v
                           const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
                           int decode, void* O, int32_t* trace, cudaStream_t s);
 // Cluster decode kernel; cudaErrorNotSupported when the geometry is outside its limits.
+// ZHA routing variant (mode RECSA_MODE_ZHA): one CTA per (query, sequence,
+// query head).  cudaErrorNotSupported outside its limits (c <= 256).
+cudaError_t launch_zha(const Params& p, const void* Q, const void* K, const void* V,
+                       const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
+                       int decode, void* O, int32_t* trace, cudaStream_t s);
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);

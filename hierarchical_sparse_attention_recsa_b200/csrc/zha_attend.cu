@@ -1,0 +1,464 @@
+// ZHA routing variant ("Subquadratic Attention with a Hierarchical
+// Tree-Structured Indexer", Figure 3 caption): one CTA per (query, sequence,
+// query head).
+//
+// Per query at position t:
+//   * routing, top-down over the visible levels: candidates = children of the
+//     nodes expanded one level up, then the orphans; score = q . key / sqrt(d)
+//     on the un-rotated query and summary key; the expanded set is the
+//     shortest prefix in decreasing-score order (ties -> lower index) whose
+//     softmax mass over the level's candidates reaches top_p, capped at
+//     min(k, c); no summary enters the attention;
+//   * attention: one softmax over the tokens of the reached leaves and the
+//     exact window [a*B, t], at their true positions with standard RoPE.
+//
+// Layout for B200:
+//   * Warps 0-7 (the chain) walk the levels: a level's candidate key rows are
+//     copied into shared memory with 16-byte cp.async (the whole level in
+//     flight at once), scored four rows per warp at a time, and warp 0 runs
+//     the top-p rounds on order-preserving 32-bit keys held in registers
+//     (redux.sync max, ties resolved by the lowest index).
+//   * Warps 8-15 attend the window, which does not depend on the routing,
+//     while the chain runs; then all 16 warps attend the reached leaves.
+//   * Exact tokens are taken in units of up to 16 consecutive positions: the
+//     query is rotated once per unit by R(t - first position) from the RoPE
+//     table and turned by R(-1) per following token, so a key is never
+//     rotated; eight tokens' K and V rows are in flight per warp.
+//   * Each warp keeps an online softmax (max, sum, its lanes' channels of the
+//     accumulator); the 16 states are merged through shared memory.
+#include "recsa_internal.cuh"
+
+namespace recsa {
+namespace {
+
+constexpr int kZThreads = 512;
+constexpr int kZWarps = kZThreads / 32;
+constexpr int kZChain = 8;          // chain warps; the others attend the window first
+constexpr int kZSlots = 8;          // candidates per lane in the top-p rounds (c <= 256)
+constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
+constexpr int kZBatch = 8;          // tokens per warp in flight
+constexpr int kZBarChain = 1;       // named barrier of the chain warps
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+__device__ __forceinline__ void chain_sync() {
+  asm volatile("bar.sync %0, %1;\n" ::"n"(kZBarChain), "n"(kZChain * 32) : "memory");
+}
+
+// Order-preserving map of a finite float onto unsigned keys above 0 (0 marks
+// "no candidate" or "taken"), and its inverse.
+__device__ __forceinline__ unsigned ord_key(float x) {
+  const unsigned u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(unsigned k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Lane l holds channel pairs (NP * l + u, NP * l + u + D/2), u < NP, of a row.
+template <int NP>
+__device__ __forceinline__ void load_pairs(const float* row, int lane, float (&x1)[NP],
+                                           float (&x2)[NP]) {
+  constexpr int HALF = 32 * NP;
+  if constexpr (NP == 2) {
+    const float2 a = *reinterpret_cast<const float2*>(row + 2 * lane);
+    const float2 b = *reinterpret_cast<const float2*>(row + HALF + 2 * lane);
+    x1[0] = a.x; x1[1] = a.y; x2[0] = b.x; x2[1] = b.y;
+  } else {
+    x1[0] = row[lane];
+    x2[0] = row[HALF + lane];
+  }
+}
+template <int NP>
+__device__ __forceinline__ void load_pairs(const __nv_bfloat16* row, int lane, float (&x1)[NP],
+                                           float (&x2)[NP]) {
+  constexpr int HALF = 32 * NP;
+  if constexpr (NP == 2) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(row + 2 * lane));
+    const float2 b =
+        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(row + HALF + 2 * lane));
+    x1[0] = a.x; x1[1] = a.y; x2[0] = b.x; x2[1] = b.y;
+  } else {
+    x1[0] = __bfloat162float(row[lane]);
+    x2[0] = __bfloat162float(row[HALF + lane]);
+  }
+}
+
+template <typename T, int NP>
+__global__ void __launch_bounds__(kZThreads, 1)
+zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
+                  const T* __restrict__ V, const void* __restrict__ tree,
+                  const int64_t* __restrict__ len_dev, int64_t q_start, int n_q, int decode,
+                  T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax) {
+  constexpr int D = 64 * NP, HALF = 32 * NP;
+  constexpr int RS = D + 2;                      // warp state row: acc[D], m, l
+  const int qi = blockIdx.x;
+  const int64_t seq = blockIdx.y;
+  const int h = blockIdx.z;                      // query head
+  const int g = h / p.group;                     // its KV head
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* kbuf = reinterpret_cast<float*>(smem);               // [cmax][D] level keys
+  float* score = kbuf + size_t(cmax) * D;                     // [cmax]
+  float* wst = score + cmax;                                  // [kZWarps][RS] warp states
+  int* kept = reinterpret_cast<int*>(wst + kZWarps * RS);     // [2][kmax] by level parity
+  int* zc = kept + 2 * kmax;                                  // [kMaxLevels + 1] candidates
+  int* zk = zc + kMaxLevels + 1;                              // [kMaxLevels + 1] expanded
+
+  const int64_t t = decode ? len_dev[seq] - 1 : q_start + qi;
+  const int64_t orow = ((seq * n_q + qi) * p.hq + h) * D;
+  if (t < 0 || t >= p.cap) {   // empty sequence, or a length beyond capacity: zeros
+    for (int x = tid; x < D; x += kZThreads) O[orow + x] = T(0.f);
+    return;
+  }
+  const float2* rope = rope_table(p, tree);
+  const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
+  const int64_t a = s0 / p.B;
+  int64_t vis[kMaxLevels + 2];
+  int top = 0;
+  {
+    int64_t per = 1;
+    for (int lev = 1; lev <= p.lay.levels; ++lev) {
+      vis[lev] = a / per;
+      if (vis[lev] == 0) break;
+      top = lev;
+      per *= p.b;
+    }
+  }
+  const int64_t kvbase = (seq * p.hkv + g) * p.cap;
+  const int64_t n_win = t + 1 - a * p.B;
+  const int tstride = kTraceHead + kMaxLevels * p.k;
+  int32_t* rec = trace ? trace + ((seq * n_q + qi) * p.hq + h) * tstride : nullptr;
+
+  // The lane's channels of the raw query, and R(-1) for the per-token turn.
+  float q1[NP], q2[NP], c1[NP], s1[NP];
+  load_pairs<NP>(Q + orow, lane, q1, q2);
+#pragma unroll
+  for (int u = 0; u < NP; ++u) {
+    c1[u] = 1.f;
+    s1[u] = 0.f;
+    if (p.rope) {
+      const float2 cs = rope[HALF + NP * lane + u];    // table row 1
+      c1[u] = cs.x;
+      s1[u] = cs.y;
+    }
+  }
+
+  // Online softmax of this warp: m, l (warp-uniform) and the lane's channels.
+  float m_run = -INFINITY, l_run = 0.f, acc1[NP], acc2[NP];
+#pragma unroll
+  for (int u = 0; u < NP; ++u) acc1[u] = acc2[u] = 0.f;
+
+  // Exact tokens [pos0, pos0 + n), n <= kZUnit, at their true positions.
+  auto attend_unit = [&](int64_t pos0, int n) {
+    float r1[NP], r2[NP];   // query rotated by R(t - pos) for the current token
+#pragma unroll
+    for (int u = 0; u < NP; ++u) {
+      r1[u] = q1[u];
+      r2[u] = q2[u];
+      if (p.rope) {
+        const float2 cs = rope[(t - pos0) * HALF + NP * lane + u];
+        r1[u] = q1[u] * cs.x - q2[u] * cs.y;
+        r2[u] = q2[u] * cs.x + q1[u] * cs.y;
+      }
+    }
+    for (int b0 = 0; b0 < n; b0 += kZBatch) {
+      const int nb = n - b0 < kZBatch ? n - b0 : kZBatch;
+      float k1[kZBatch][NP], k2[kZBatch][NP], v1[kZBatch][NP], v2[kZBatch][NP];
+#pragma unroll
+      for (int i = 0; i < kZBatch; ++i) {
+        if (i < nb) {
+          const int64_t row = (kvbase + pos0 + b0 + i) * D;
+          load_pairs<NP>(K + row, lane, k1[i], k2[i]);
+          load_pairs<NP>(V + row, lane, v1[i], v2[i]);
+        }
+      }
+      float s[kZBatch];
+#pragma unroll
+      for (int i = 0; i < kZBatch; ++i) {
+        float d_ = 0.f;
+#pragma unroll
+        for (int u = 0; u < NP; ++u) {
+          d_ = fmaf(r1[u], i < nb ? k1[i][u] : 0.f, d_);
+          d_ = fmaf(r2[u], i < nb ? k2[i][u] : 0.f, d_);
+          // turn the query by R(-1): the next token is one position later
+          const float x1 = r1[u], x2 = r2[u];
+          r1[u] = x1 * c1[u] + x2 * s1[u];
+          r2[u] = x2 * c1[u] - x1 * s1[u];
+        }
+        s[i] = d_;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int i = 0; i < kZBatch; ++i) s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
+      float mx = m_run;
+#pragma unroll
+      for (int i = 0; i < kZBatch; ++i) {
+        s[i] = i < nb ? s[i] * p.inv_sqrt_d : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      const float scale = expf(m_run - mx);
+      l_run *= scale;
+#pragma unroll
+      for (int u = 0; u < NP; ++u) {
+        acc1[u] *= scale;
+        acc2[u] *= scale;
+      }
+#pragma unroll
+      for (int i = 0; i < kZBatch; ++i) {
+        if (i < nb) {
+          const float w = expf(s[i] - mx);
+          l_run += w;
+#pragma unroll
+          for (int u = 0; u < NP; ++u) {
+            acc1[u] = fmaf(w, v1[i][u], acc1[u]);
+            acc2[u] = fmaf(w, v2[i][u], acc2[u]);
+          }
+        }
+      }
+      m_run = mx;
+    }
+  };
+
+  if (warp < kZChain) {
+    // ---- routing chain ----------------------------------------------------
+    const int ct = tid;                          // 0 .. 255
+    int kup = 0;
+    for (int lev = top; lev >= 1; --lev) {
+      const int64_t vup = lev < top ? vis[lev + 1] : 0;
+      const int nch = p.b * kup;
+      const int c = nch + int(vis[lev] - p.b * vup);
+      const int* kprev = kept + ((lev + 1) & 1) * kmax;
+      auto node = [&](int i) -> int {
+        return i < nch ? kprev[div_b(p, i)] * p.b + mod_b(p, i) : int(p.b * vup) + (i - nch);
+      };
+      const float* keys = level_keys(p, const_cast<void*>(tree), lev, seq, g);
+      constexpr int C16 = D / 4;                 // 16-byte pieces per fp32 row
+      for (int x = ct; x < c * C16; x += kZChain * 32) {
+        const int i = x / C16, pc = x % C16;
+        cp_async16(kbuf + size_t(i) * D + pc * 4, keys + int64_t(node(i)) * D + pc * 4);
+      }
+      cp_async_wait_all();
+      chain_sync();
+      // scores: rows warp, warp + 8, ...; four rows per warp at a time
+      for (int i0 = warp; i0 < c; i0 += 4 * kZChain) {
+        float sc4[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int i = i0 + r * kZChain;
+          float x1[NP], x2[NP];
+          sc4[r] = 0.f;
+          if (i < c) {
+            load_pairs<NP>(kbuf + size_t(i) * D, lane, x1, x2);
+#pragma unroll
+            for (int u = 0; u < NP; ++u) {
+              sc4[r] = fmaf(q1[u], x1[u], sc4[r]);
+              sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) sc4[r] += __shfl_xor_sync(0xffffffffu, sc4[r], o);
+        if (lane < 4) {
+          float v = sc4[0];
+#pragma unroll
+          for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
+          const int i = i0 + lane * kZChain;
+          if (i < c) score[i] = v * p.inv_sqrt_d;
+        }
+      }
+      chain_sync();
+      if (warp == 0) {
+        // top-p rounds over the level's c <= 32 * kZSlots candidates
+        unsigned key[kZSlots];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kZSlots; ++s) {
+          const int i = lane + 32 * s;
+          const float v = i < c ? score[i] + 0.f : -INFINITY;   // + 0: -0 -> +0, one key
+          key[s] = i < c ? ord_key(v) : 0u;
+          mx = fmaxf(mx, v);
+        }
+        mx = warp_max(mx);
+        float tot = 0.f;
+#pragma unroll
+        for (int s = 0; s < kZSlots; ++s)
+          if (lane + 32 * s < c) tot += expf(ord_val(key[s]) - mx);
+        const float thr = p.top_p * warp_sum(tot);
+        const int cap = c < p.k ? c : p.k;
+        unsigned taken = 0;
+        float cum = 0.f;
+        int cnt = 0;
+        while (cnt < cap) {
+          unsigned best = 0u;
+          int bs = 0;
+#pragma unroll
+          for (int s = 0; s < kZSlots; ++s)
+            if (key[s] > best) {
+              best = key[s];
+              bs = s;
+            }
+          const unsigned wmax = __reduce_max_sync(0xffffffffu, best);
+          const unsigned hold = __ballot_sync(0xffffffffu, best == wmax);
+          const unsigned mine = best == wmax ? unsigned(bs * 32 + lane) : 0xffffffffu;
+          const unsigned idx = __popc(hold) == 1 ? __shfl_sync(0xffffffffu, mine, __ffs(hold) - 1)
+                                                 : __reduce_min_sync(0xffffffffu, mine);
+          if (lane == int(idx & 31u)) {
+#pragma unroll
+            for (int s = 0; s < kZSlots; ++s)
+              if (s == int(idx >> 5)) {
+                key[s] = 0u;
+                taken |= 1u << s;
+              }
+          }
+          ++cnt;
+          cum += expf(ord_val(wmax) - mx);
+          if (p.top_p < 1.f && cum >= thr) break;
+        }
+        // expanded nodes in candidate order
+        int* knew = kept + (lev & 1) * kmax;
+        int base = 0;
+#pragma unroll
+        for (int s = 0; s < kZSlots; ++s) {
+          const bool on = (taken >> s) & 1u;
+          const unsigned bal = __ballot_sync(0xffffffffu, on);
+          if (on) {
+            const int pos = base + __popc(bal & ((1u << lane) - 1u));
+            const int id = node(lane + 32 * s);
+            knew[pos] = id;
+            if (rec) rec[kTraceHead + (lev - 1) * p.k + pos] = id;
+          }
+          base += __popc(bal);
+        }
+        if (lane == 0) {
+          zc[lev] = c;
+          zk[lev] = cnt;
+        }
+      }
+      chain_sync();
+      kup = zk[lev];
+    }
+  } else {
+    // ---- window warps: [a*B, t], units of kZUnit positions ------------------
+    const int nu = int((n_win + kZUnit - 1) / kZUnit);
+    for (int u = warp - kZChain; u < nu; u += kZWarps - kZChain) {
+      const int64_t p0 = a * p.B + int64_t(u) * kZUnit;
+      const int n = int(n_win - int64_t(u) * kZUnit < kZUnit ? n_win - int64_t(u) * kZUnit
+                                                               : kZUnit);
+      attend_unit(p0, n);
+    }
+  }
+  __syncthreads();
+
+  // ---- reached leaves: all warps ---------------------------------------------
+  const int nleaf = top > 0 ? zk[1] : 0;
+  const int upl = (p.B + kZUnit - 1) / kZUnit;   // units per leaf
+  const int* leaves = kept + 1 * kmax;           // level 1 (odd parity)
+  // the window warps take the first units: the chain warps start later
+  for (int u = (warp + kZWarps - kZChain) % kZWarps; u < nleaf * upl; u += kZWarps) {
+    const int r = u / upl, m = u % upl;
+    const int n = p.B - m * kZUnit < kZUnit ? p.B - m * kZUnit : kZUnit;
+    attend_unit(int64_t(leaves[r]) * p.B + m * kZUnit, n);
+  }
+
+  // ---- merge the warps' states ----------------------------------------------
+  float* my = wst + warp * RS;
+#pragma unroll
+  for (int u = 0; u < NP; ++u) {
+    my[NP * lane + u] = acc1[u];
+    my[HALF + NP * lane + u] = acc2[u];
+  }
+  if (lane == 0) {
+    my[D] = m_run;
+    my[D + 1] = l_run;
+  }
+  __syncthreads();
+  if (tid < D) {
+    float M = -INFINITY;
+    for (int w = 0; w < kZWarps; ++w) M = fmaxf(M, wst[w * RS + D]);
+    float L = 0.f, A = 0.f;
+    for (int w = 0; w < kZWarps; ++w) {
+      const float mw = wst[w * RS + D];
+      if (mw == -INFINITY) continue;
+      const float e = expf(mw - M);
+      L = fmaf(wst[w * RS + D + 1], e, L);
+      A = fmaf(wst[w * RS + tid], e, A);
+    }
+    const float o = A / L;
+    if constexpr (sizeof(T) == 2)
+      O[orow + tid] = __float2bfloat16_rn(o);
+    else
+      O[orow + tid] = o;
+  }
+  if (rec && tid == 0) {
+    const int64_t n0 = int64_t(nleaf) * p.B + n_win;
+    int64_t keys_read = n0;
+    for (int lev = 1; lev <= top; ++lev) keys_read += zc[lev];
+    rec[0] = top;
+    rec[1] = int32_t(n0);
+    rec[2] = int32_t(keys_read);
+    rec[3] = int32_t(n0);
+    for (int lev = 1; lev <= kMaxLevels; ++lev) {
+      const bool on = lev <= top;
+      rec[4 + lev - 1] = on ? zc[lev] : 0;
+      rec[4 + kMaxLevels + lev - 1] = on ? zk[lev] : 0;
+    }
+  }
+}
+
+template <typename T, int NP>
+cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void* V,
+                      const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
+                      int decode, void* O, int32_t* trace, cudaStream_t s) {
+  constexpr int D = 64 * NP;
+  const int64_t kk = p.k < p.cap ? p.k : p.cap;
+  int64_t maxn = 1;
+  for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
+  int64_t cm = p.b * kk + p.b - 1;
+  cm = cm < maxn ? cm : maxn;
+  const int cmax = int(cm < 1 ? 1 : cm);
+  if (cmax > 32 * kZSlots) return cudaErrorNotSupported;   // the generic kernel serves it
+  const int kmax = int(kk < cmax ? kk : cmax);
+  const size_t bytes = (size_t(cmax) * D + cmax + kZWarps * (D + 2)) * 4 +
+                       (2 * size_t(kmax) + 2 * (kMaxLevels + 1)) * 4;
+  if (bytes > 227 * 1024) return cudaErrorNotSupported;
+  if (p.batch > 65535) return cudaErrorNotSupported;
+  auto kern = zha_attend_kernel<T, NP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(bytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_q, p.batch, p.hq);
+  kern<<<grid, kZThreads, bytes, s>>>(p, reinterpret_cast<const T*>(Q),
+                                      reinterpret_cast<const T*>(K),
+                                      reinterpret_cast<const T*>(V), tree, len_dev, q_start, n_q,
+                                      decode, reinterpret_cast<T*>(O), trace, cmax, kmax);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_zha(const Params& p, const void* Q, const void* K, const void* V,
+                       const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
+                       int decode, void* O, int32_t* trace, cudaStream_t s) {
+  if (p.mode != RECSA_MODE_ZHA) return cudaErrorNotSupported;
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? zha_typed<__nv_bfloat16, 2>(p, Q, K, V, tree, len_dev, q_start, n_q,
+                                                    decode, O, trace, s)
+                      : zha_typed<__nv_bfloat16, 1>(p, Q, K, V, tree, len_dev, q_start, n_q,
+                                                    decode, O, trace, s);
+  return p.d == 128 ? zha_typed<float, 2>(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O,
+                                          trace, s)
+                    : zha_typed<float, 1>(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O,
+                                          trace, s);
+}
+
+}  // namespace recsa

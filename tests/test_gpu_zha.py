@@ -9,6 +9,8 @@ within rounding of its threshold or of a score tie, and a validity check plus
 an output comparison under the GPU's routing elsewhere (recsa_testlib).
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -33,6 +35,19 @@ def _lib():
     R.lib()
 
 
+@pytest.fixture(params=["kernel", "generic"])
+def zha_impl(request):
+    """The dedicated ZHA kernel (one CTA per query head) or the generic
+    one-CTA-per-KV-head kernel."""
+    old = os.environ.pop("RECSA_ZHA_GENERIC", None)
+    if request.param == "generic":
+        os.environ["RECSA_ZHA_GENERIC"] = "1"
+    yield request.param
+    os.environ.pop("RECSA_ZHA_GENERIC", None)
+    if old is not None:
+        os.environ["RECSA_ZHA_GENERIC"] = old
+
+
 def _setup(w, lens, capacity, top_p, seed=0, k=None, rope=1):
     batch = len(lens)
     g = geometry(w, capacity, batch, k=k, rope=rope, top_p=top_p)
@@ -55,7 +70,7 @@ def _trees(g, K, V, r, lens):
 
 
 @pytest.mark.parametrize("top_p", [0.3, 0.9])
-def test_zha_decode_tiny(top_p):
+def test_zha_decode_tiny(top_p, zha_impl):
     L, nq = TINY.length, TINY.n_q
     g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, top_p, seed=20, k=ZK)
     trees = _trees(g, K, V, r, [L])
@@ -78,14 +93,14 @@ def test_zha_decode_tiny(top_p):
             res = check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh,
                                   Vh, src, og, top_p, g.k)
             sizes += [len(v) for v in res["kept"].values()]
-    st.check(torch.float32, f"zha decode tiny p={top_p}")
+    st.check(torch.float32, f"zha {zha_impl} decode tiny p={top_p}")
     assert st.clear > 0.7 * nq * g.n_q_heads
     # the mass target, not the cap, ends some levels
     assert min(sizes) < g.k
 
 
 @pytest.mark.parametrize("entry", ["prefill", "prefill-workspace", "prefill-static"])
-def test_zha_prefill_tiny(entry):
+def test_zha_prefill_tiny(entry, zha_impl):
     L, top_p = TINY.length, 0.8
     g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, top_p, seed=22, k=ZK)
     trees = _trees(g, K, V, r, [L])
@@ -116,11 +131,11 @@ def test_zha_prefill_tiny(entry):
         for h in range(g.n_q_heads):
             check_query_zha(st, O_[0, t, h], tr[0, t, h], to_np(Q[0, t, h]), t, Kh, Vh, src, og,
                             top_p, g.k)
-    st.check(torch.float32, f"zha {entry} tiny")
+    st.check(torch.float32, f"zha {zha_impl} {entry} tiny")
 
 
 @pytest.mark.parametrize("top_p", [0.5, 0.95])
-def test_zha_decode_model_small(top_p):
+def test_zha_decode_model_small(top_p, zha_impl):
     lens = [20000, 13001]
     g, K, V, r, Kd, Vd, rd, tree = _setup(MODEL, lens, 20480, top_p, seed=24)
     trees = _trees(g, K, V, r, lens)
@@ -144,11 +159,11 @@ def test_zha_decode_model_small(top_p):
                 Kh, Vh, src = trees[(s, h // G)]
                 check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
                                 src, og, top_p, g.k)
-    st.check(torch.bfloat16, f"zha decode model small p={top_p}")
+    st.check(torch.bfloat16, f"zha {zha_impl} decode model small p={top_p}")
 
 
 @pytest.mark.parametrize("wname,rope", [("tiny-4k", 1), ("tiny-4k", 0), ("qwen3-4b-131k", 1)])
-def test_zha_full_mass_keep_all_is_dense(wname, rope):
+def test_zha_full_mass_keep_all_is_dense(wname, rope, zha_impl):
     """p = 1 with no cap reaches every leaf: dense causal attention."""
     w = synth.WORKLOADS[wname]
     L = 1500 if w.head_dim == 64 else 700
@@ -173,10 +188,10 @@ def test_zha_full_mass_keep_all_is_dense(wname, rope):
             st.add(O_[0, t, h], ref)
             if t == L - 1:
                 st.add(Od_[0, 0, h], ref)
-    st.check(w.dtype, "zha full mass")
+    st.check(w.dtype, f"zha {zha_impl} full mass")
 
 
-def test_zha_tiny_p_expands_one_node_per_level():
+def test_zha_tiny_p_expands_one_node_per_level(zha_impl):
     """A mass target below every candidate's share expands only the arg-max."""
     L = TINY.length
     g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, 1e-6, seed=28)
@@ -201,10 +216,10 @@ def test_zha_tiny_p_expands_one_node_per_level():
             assert all(len(v) == 1 for v in t_["kept"].values())
             check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh, Vh, src,
                             og, 1e-6, g.k)
-    st.check(torch.float32, "zha tiny p")
+    st.check(torch.float32, f"zha {zha_impl} tiny p")
 
 
-def test_zha_decode_step_equals_append_then_decode():
+def test_zha_decode_step_equals_append_then_decode(zha_impl):
     """In ZHA mode the one-call step (append, then the routed decode) equals
     the two calls, across leaf completions, and matches the oracle."""
     w, top_p = MODEL, 0.9
@@ -250,6 +265,6 @@ def test_zha_decode_step_equals_append_then_decode():
                     src = oracle.LazyTree(Kh, Vh, r.double().numpy(), g.leaf_block, g.branching)
                     check_query_zha(st, to_np(Oa[s, 0, h]), tr[s, 0, h], to_np(Q[s, 0, h]),
                                     lens_now[s] - 1, Kh, Vh, src, og, top_p, g.k)
-    st.check(torch.bfloat16, "zha decode step")
+    st.check(torch.bfloat16, f"zha {zha_impl} decode step")
     assert torch.equal(Ka, Kb) and torch.equal(Va, Vb)
     assert torch.equal(tree_a[256:], tree_b[256:])
