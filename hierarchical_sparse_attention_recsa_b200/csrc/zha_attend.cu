@@ -15,15 +15,16 @@
 // Layout for B200:
 //   * Warps 0-7 (the chain) walk the levels: a level's candidate key rows are
 //     copied into shared memory with 16-byte cp.async (the whole level in
-//     flight at once), scored four rows per warp at a time, and warp 0 runs
-//     the top-p rounds on order-preserving 32-bit keys held in registers
-//     (redux.sync max, ties resolved by the lowest index).
+//     flight at once) and scored four rows per warp at a time; the top-p cut
+//     comes from every candidate's rank (one chain thread per candidate) and
+//     a warp scan of the weights laid out by rank.
 //   * Warps 8-15 attend the window, which does not depend on the routing,
 //     while the chain runs; then all 16 warps attend the reached leaves.
 //   * Exact tokens are taken in units of up to 16 consecutive positions: the
 //     query is rotated once per unit by R(t - first position) from the RoPE
 //     table and turned by R(-1) per following token, so a key is never
-//     rotated; eight tokens' K and V rows are in flight per warp.
+//     rotated.  A warp loads a whole unit's K and V rows (bf16; half a unit
+//     for fp32) into registers, still packed, before it uses any of them.
 //   * Each warp keeps an online softmax (max, sum, its lanes' channels of the
 //     accumulator); the 16 states are merged through shared memory.
 #include "recsa_internal.cuh"
@@ -34,9 +35,8 @@ namespace {
 constexpr int kZThreads = 512;
 constexpr int kZWarps = kZThreads / 32;
 constexpr int kZChain = 8;          // chain warps; the others attend the window first
-constexpr int kZSlots = 8;          // candidates per lane in the top-p rounds (c <= 256)
+constexpr int kZMaxCand = kZChain * 32;   // one chain thread per candidate
 constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
-constexpr int kZBatch = 8;          // tokens per warp in flight
 constexpr int kZBarChain = 1;       // named barrier of the chain warps
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -48,16 +48,6 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 __device__ __forceinline__ void chain_sync() {
   asm volatile("bar.sync %0, %1;\n" ::"n"(kZBarChain), "n"(kZChain * 32) : "memory");
-}
-
-// Order-preserving map of a finite float onto unsigned keys above 0 (0 marks
-// "no candidate" or "taken"), and its inverse.
-__device__ __forceinline__ unsigned ord_key(float x) {
-  const unsigned u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float ord_val(unsigned k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
 // Lane l holds channel pairs (NP * l + u, NP * l + u + D/2), u < NP, of a row.
@@ -89,6 +79,48 @@ __device__ __forceinline__ void load_pairs(const __nv_bfloat16* row, int lane, f
   }
 }
 
+// The lane's slice of a row as loaded (not yet converted): pairs
+// (NP * l + u) and (NP * l + u + D/2).
+template <typename T, int NP> struct Raw;
+template <> struct Raw<__nv_bfloat16, 2> { __nv_bfloat162 a, b; };
+template <> struct Raw<__nv_bfloat16, 1> { __nv_bfloat16 a, b; };
+template <> struct Raw<float, 2> { float2 a, b; };
+template <> struct Raw<float, 1> { float a, b; };
+
+template <typename T, int NP>
+__device__ __forceinline__ Raw<T, NP> load_raw(const T* row, int lane) {
+  constexpr int HALF = 32 * NP;
+  Raw<T, NP> r;
+  if constexpr (NP == 2) {
+    using P2 = decltype(r.a);
+    r.a = *reinterpret_cast<const P2*>(row + 2 * lane);
+    r.b = *reinterpret_cast<const P2*>(row + HALF + 2 * lane);
+  } else {
+    r.a = row[lane];
+    r.b = row[HALF + lane];
+  }
+  return r;
+}
+template <typename T, int NP>
+__device__ __forceinline__ void unpack(const Raw<T, NP>& r, float (&x1)[NP], float (&x2)[NP]) {
+  if constexpr (NP == 2) {
+    if constexpr (sizeof(T) == 2) {
+      const float2 a = __bfloat1622float2(r.a), b = __bfloat1622float2(r.b);
+      x1[0] = a.x; x1[1] = a.y; x2[0] = b.x; x2[1] = b.y;
+    } else {
+      x1[0] = r.a.x; x1[1] = r.a.y; x2[0] = r.b.x; x2[1] = r.b.y;
+    }
+  } else {
+    if constexpr (sizeof(T) == 2) {
+      x1[0] = __bfloat162float(r.a);
+      x2[0] = __bfloat162float(r.b);
+    } else {
+      x1[0] = r.a;
+      x2[0] = r.b;
+    }
+  }
+}
+
 template <typename T, int NP>
 __global__ void __launch_bounds__(kZThreads, 1)
 zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
@@ -106,10 +138,13 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   extern __shared__ __align__(16) unsigned char smem[];
   float* kbuf = reinterpret_cast<float*>(smem);               // [cmax][D] level keys
   float* score = kbuf + size_t(cmax) * D;                     // [cmax]
-  float* wst = score + cmax;                                  // [kZWarps][RS] warp states
+  float* wsort = score + cmax;                                // [cmax] weights by rank
+  float* zsum = wsort + cmax;                                 // [kZChain] sums, [kZChain] max
+  float* wst = zsum + kZChain + 1;                            // [kZWarps][RS] warp states
   int* kept = reinterpret_cast<int*>(wst + kZWarps * RS);     // [2][kmax] by level parity
   int* zc = kept + 2 * kmax;                                  // [kMaxLevels + 1] candidates
   int* zk = zc + kMaxLevels + 1;                              // [kMaxLevels + 1] expanded
+  int* zcnt = zk + kMaxLevels + 1;                            // [kZChain] expanded per warp
 
   const int64_t t = decode ? len_dev[seq] - 1 : q_start + qi;
   const int64_t orow = ((seq * n_q + qi) * p.hq + h) * D;
@@ -168,25 +203,26 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         r2[u] = q2[u] * cs.x + q1[u] * cs.y;
       }
     }
-    for (int b0 = 0; b0 < n; b0 += kZBatch) {
-      const int nb = n - b0 < kZBatch ? n - b0 : kZBatch;
-      float k1[kZBatch][NP], k2[kZBatch][NP], v1[kZBatch][NP], v2[kZBatch][NP];
+    constexpr int TB = sizeof(T) == 2 ? kZUnit : kZUnit / 2;   // tokens per batch
+    for (int b0 = 0; b0 < n; b0 += TB) {
+      const int nb = n - b0 < TB ? n - b0 : TB;
+      Raw<T, NP> kr[TB], vr[TB];
 #pragma unroll
-      for (int i = 0; i < kZBatch; ++i) {
-        if (i < nb) {
-          const int64_t row = (kvbase + pos0 + b0 + i) * D;
-          load_pairs<NP>(K + row, lane, k1[i], k2[i]);
-          load_pairs<NP>(V + row, lane, v1[i], v2[i]);
-        }
+      for (int i = 0; i < TB; ++i) {   // every load first (rows past nb repeat the last)
+        const int64_t row = (kvbase + pos0 + b0 + (i < nb ? i : nb - 1)) * D;
+        kr[i] = load_raw<T, NP>(K + row, lane);
+        vr[i] = load_raw<T, NP>(V + row, lane);
       }
-      float s[kZBatch];
+      float s[TB];
 #pragma unroll
-      for (int i = 0; i < kZBatch; ++i) {
+      for (int i = 0; i < TB; ++i) {
+        float k1[NP], k2[NP];
+        unpack<T, NP>(kr[i], k1, k2);
         float d_ = 0.f;
 #pragma unroll
         for (int u = 0; u < NP; ++u) {
-          d_ = fmaf(r1[u], i < nb ? k1[i][u] : 0.f, d_);
-          d_ = fmaf(r2[u], i < nb ? k2[i][u] : 0.f, d_);
+          d_ = fmaf(r1[u], k1[u], d_);
+          d_ = fmaf(r2[u], k2[u], d_);
           // turn the query by R(-1): the next token is one position later
           const float x1 = r1[u], x2 = r2[u];
           r1[u] = x1 * c1[u] + x2 * s1[u];
@@ -197,10 +233,10 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-        for (int i = 0; i < kZBatch; ++i) s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
+        for (int i = 0; i < TB; ++i) s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
       float mx = m_run;
 #pragma unroll
-      for (int i = 0; i < kZBatch; ++i) {
+      for (int i = 0; i < TB; ++i) {
         s[i] = i < nb ? s[i] * p.inv_sqrt_d : -INFINITY;
         mx = fmaxf(mx, s[i]);
       }
@@ -212,15 +248,15 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         acc2[u] *= scale;
       }
 #pragma unroll
-      for (int i = 0; i < kZBatch; ++i) {
-        if (i < nb) {
-          const float w = expf(s[i] - mx);
-          l_run += w;
+      for (int i = 0; i < TB; ++i) {
+        const float w = expf(s[i] - mx);   // 0 past nb
+        float v1[NP], v2[NP];
+        unpack<T, NP>(vr[i], v1, v2);
+        l_run += w;
 #pragma unroll
-          for (int u = 0; u < NP; ++u) {
-            acc1[u] = fmaf(w, v1[i][u], acc1[u]);
-            acc2[u] = fmaf(w, v2[i][u], acc2[u]);
-          }
+        for (int u = 0; u < NP; ++u) {
+          acc1[u] = fmaf(w, v1[u], acc1[u]);
+          acc2[u] = fmaf(w, v2[u], acc2[u]);
         }
       }
       m_run = mx;
@@ -252,16 +288,14 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         float sc4[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const int i = i0 + r * kZChain;
+          const int i = min(i0 + r * kZChain, c - 1);   // rows past c repeat the last
           float x1[NP], x2[NP];
+          load_pairs<NP>(kbuf + size_t(i) * D, lane, x1, x2);
           sc4[r] = 0.f;
-          if (i < c) {
-            load_pairs<NP>(kbuf + size_t(i) * D, lane, x1, x2);
 #pragma unroll
-            for (int u = 0; u < NP; ++u) {
-              sc4[r] = fmaf(q1[u], x1[u], sc4[r]);
-              sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
-            }
+          for (int u = 0; u < NP; ++u) {
+            sc4[r] = fmaf(q1[u], x1[u], sc4[r]);
+            sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
           }
         }
 #pragma unroll
@@ -277,72 +311,67 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         }
       }
       chain_sync();
+      // Top-p by ranks: chain thread ct holds candidate ct (c <= 256).  Its rank
+      // counts the better candidates (higher score, or equal at a lower
+      // index); the weights exp(s - max) are laid out by rank, and warp 0
+      // scans them for the shortest prefix whose mass reaches top_p of the
+      // total, capped at min(k, c).
+      const bool mine = ct < c;
+      const float si = mine ? score[ct] : 0.f;
+      int ri = 0;
+      if (mine) {
+        for (int j = 0; j < c; ++j) {
+          const float sj = score[j];
+          ri += (sj > si) || (sj == si && j < ct);
+        }
+        if (ri == 0) zsum[kZChain] = si;   // the level's maximum
+      }
+      chain_sync();
+      const float ei = mine ? expf(si - zsum[kZChain]) : 0.f;
+      if (mine) wsort[ri] = ei;
+      const float ws = warp_sum(ei);
+      if (lane == 0) zsum[warp] = ws;
+      chain_sync();
       if (warp == 0) {
-        // top-p rounds over the level's c <= 32 * kZSlots candidates
-        unsigned key[kZSlots];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int s = 0; s < kZSlots; ++s) {
-          const int i = lane + 32 * s;
-          const float v = i < c ? score[i] + 0.f : -INFINITY;   // + 0: -0 -> +0, one key
-          key[s] = i < c ? ord_key(v) : 0u;
-          mx = fmaxf(mx, v);
-        }
-        mx = warp_max(mx);
-        float tot = 0.f;
-#pragma unroll
-        for (int s = 0; s < kZSlots; ++s)
-          if (lane + 32 * s < c) tot += expf(ord_val(key[s]) - mx);
-        const float thr = p.top_p * warp_sum(tot);
+        const float tot = warp_sum(lane < kZChain ? zsum[lane] : 0.f);
+        const float thr = p.top_p * tot;
         const int cap = c < p.k ? c : p.k;
-        unsigned taken = 0;
-        float cum = 0.f;
-        int cnt = 0;
-        while (cnt < cap) {
-          unsigned best = 0u;
-          int bs = 0;
+        int cnt = cap;
+        if (p.top_p < 1.f) {
+          float run = 0.f;
+          for (int b0 = 0; b0 < cap; b0 += 32) {
+            const int e = b0 + lane;
+            float x = e < cap ? wsort[e] : 0.f;
 #pragma unroll
-          for (int s = 0; s < kZSlots; ++s)
-            if (key[s] > best) {
-              best = key[s];
-              bs = s;
+            for (int o = 1; o < 32; o <<= 1) {
+              const float y = __shfl_up_sync(0xffffffffu, x, o);
+              if (lane >= o) x += y;
             }
-          const unsigned wmax = __reduce_max_sync(0xffffffffu, best);
-          const unsigned hold = __ballot_sync(0xffffffffu, best == wmax);
-          const unsigned mine = best == wmax ? unsigned(bs * 32 + lane) : 0xffffffffu;
-          const unsigned idx = __popc(hold) == 1 ? __shfl_sync(0xffffffffu, mine, __ffs(hold) - 1)
-                                                 : __reduce_min_sync(0xffffffffu, mine);
-          if (lane == int(idx & 31u)) {
-#pragma unroll
-            for (int s = 0; s < kZSlots; ++s)
-              if (s == int(idx >> 5)) {
-                key[s] = 0u;
-                taken |= 1u << s;
-              }
+            const unsigned hit = __ballot_sync(0xffffffffu, e < cap && run + x >= thr);
+            if (hit) {
+              cnt = b0 + __ffs(hit);
+              break;
+            }
+            run += __shfl_sync(0xffffffffu, x, 31);
           }
-          ++cnt;
-          cum += expf(ord_val(wmax) - mx);
-          if (p.top_p < 1.f && cum >= thr) break;
-        }
-        // expanded nodes in candidate order
-        int* knew = kept + (lev & 1) * kmax;
-        int base = 0;
-#pragma unroll
-        for (int s = 0; s < kZSlots; ++s) {
-          const bool on = (taken >> s) & 1u;
-          const unsigned bal = __ballot_sync(0xffffffffu, on);
-          if (on) {
-            const int pos = base + __popc(bal & ((1u << lane) - 1u));
-            const int id = node(lane + 32 * s);
-            knew[pos] = id;
-            if (rec) rec[kTraceHead + (lev - 1) * p.k + pos] = id;
-          }
-          base += __popc(bal);
         }
         if (lane == 0) {
           zc[lev] = c;
           zk[lev] = cnt;
         }
+      }
+      chain_sync();
+      // expanded nodes in candidate order
+      const bool on = mine && ri < zk[lev];
+      const unsigned bal = __ballot_sync(0xffffffffu, on);
+      if (lane == 0) zcnt[warp] = __popc(bal);
+      chain_sync();
+      if (on) {
+        int pos = __popc(bal & ((1u << lane) - 1u));
+        for (int w = 0; w < warp; ++w) pos += zcnt[w];
+        const int id = node(ct);
+        kept[(lev & 1) * kmax + pos] = id;
+        if (rec) rec[kTraceHead + (lev - 1) * p.k + pos] = id;
       }
       chain_sync();
       kup = zk[lev];
@@ -426,10 +455,10 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   int64_t cm = p.b * kk + p.b - 1;
   cm = cm < maxn ? cm : maxn;
   const int cmax = int(cm < 1 ? 1 : cm);
-  if (cmax > 32 * kZSlots) return cudaErrorNotSupported;   // the generic kernel serves it
+  if (cmax > kZMaxCand) return cudaErrorNotSupported;   // the generic kernel serves it
   const int kmax = int(kk < cmax ? kk : cmax);
-  const size_t bytes = (size_t(cmax) * D + cmax + kZWarps * (D + 2)) * 4 +
-                       (2 * size_t(kmax) + 2 * (kMaxLevels + 1)) * 4;
+  const size_t bytes = (size_t(cmax) * D + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
+                       (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + kZChain) * 4;
   if (bytes > 227 * 1024) return cudaErrorNotSupported;
   if (p.batch > 65535) return cudaErrorNotSupported;
   auto kern = zha_attend_kernel<T, NP>;
