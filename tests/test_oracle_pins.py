@@ -450,3 +450,117 @@ def test_zha_tiny_p_is_greedy_descent():
         pw = np.exp(lg - lg.max())
         np.testing.assert_allclose(res["out"], (pw[:, None] * V[exact]).sum(0) / pw.sum(),
                                    atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Per-KV-group shared selection
+# ---------------------------------------------------------------------------
+
+class _KeyTable:
+    """A one-level tree given by its node keys and values (hand-built cases)."""
+
+    def __init__(self, keys, vals):
+        self.keys, self.vals = np.asarray(keys, float), np.asarray(vals, float)
+
+    def key(self, lev, n):
+        assert lev == 1
+        return self.keys[n]
+
+    def val(self, lev, n):
+        assert lev == 1
+        return self.vals[n]
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_group_of_one_or_identical_heads_is_per_head_recsa(rope):
+    """One head, or G copies of one head, select exactly as that head alone:
+    its summed probability is a monotone function of its own logit."""
+    rng = np.random.default_rng(21)
+    B, b, d, T, W, k = 4, 3, 8, 300, 6, 2
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 1, 1, B, b, k, W, rope=rope, rope_base=1e3)
+    for t in [30, 131, 299]:
+        q = rng.standard_normal(d) * 2
+        ref = oracle.traverse_and_attend(q, t, K, V, tree, geo)
+        for G in (1, 3):
+            res = oracle.group_traverse_and_attend(np.stack([q] * G), t, K, V, tree, geo)
+            assert res["kept"] == ref["kept"]
+            for h in range(G):
+                np.testing.assert_allclose(res["out"][h], ref["out"], atol=1e-13)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_group_keep_all_is_dense_for_every_head(rope):
+    rng = np.random.default_rng(22)
+    B, b, d, T, W = 4, 3, 8, 150, 5
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 4, 1, B, b, oracle.recsa.KEEP_ALL, W, rope=rope, rope_base=1e3)
+    for t in [0, 17, 149]:
+        Qg = rng.standard_normal((4, d)) * 2
+        res = oracle.group_traverse_and_attend(Qg, t, K, V, tree, geo)
+        for h in range(4):
+            if rope:
+                qr = _rope_complex(Qg[h], t, 1e3)
+                Kr = np.stack([_rope_complex(K[j], j, 1e3) for j in range(t + 1)])
+            else:
+                qr, Kr = Qg[h], K[: t + 1]
+            np.testing.assert_allclose(res["out"][h], _sdpa(qr, Kr, V[: t + 1]), atol=1e-12)
+
+
+def test_group_score_sums_head_probabilities():
+    """Hand-built level of three nodes (B = 1, b = 4, W = 1, t = 3: the three
+    visible leaves are orphans of the top level), k = 1, no RoPE, d = 2.
+    Head 0's logits are (5, 0, 0) and head 1's (-10, 2, 2.1): the summed
+    probabilities are about (0.987, 0.482, 0.532), so node 0 is kept; a sum
+    of logits, (-5, 2, 2.1), would keep node 2."""
+    s2 = math.sqrt(2.0)
+    keys = [[1.0, 0.0], [0.0, 1.0], [0.0, 1.05]]
+    vals = [[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]]
+    tree = _KeyTable(keys, vals)
+    Qg = np.array([[5 * s2, 0.0], [-10 * s2, 2 * s2]])
+    K = np.array([[1.0, 0.0], [0.0, 1.0], [0.0, 1.05], [0.5, 0.5]])
+    V = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [2.0, -1.0]])
+    geo = Geometry(2, 2, 1, 1, 4, 1, 1, rope=False)
+    sel = oracle.group_select(Qg, 3, tree, geo)
+    assert sel["top"] == 1 and sel["cand"] == {1: 3}
+    assert sel["kept"] == {1: [0]}
+    e5 = math.exp(5.0)
+    p1 = np.exp([-10.0, 2.0, 2.1])
+    want = np.array([e5, 1.0, 1.0]) / (e5 + 2.0) + p1 / p1.sum()
+    np.testing.assert_allclose(sel["group"][1], want, rtol=1e-12)
+    # the heads then attend over node 1, node 2 (summaries) and tokens 0, 3
+    res = oracle.group_traverse_and_attend(Qg, 3, K, V, tree, geo)
+    for h in range(2):
+        lg = np.array([Qg[h] @ keys[1], Qg[h] @ keys[2], Qg[h] @ K[0], Qg[h] @ K[3]]) / s2
+        w = np.exp(lg - lg.max())
+        ref = (w[:, None] * np.array([vals[1], vals[2], V[0], V[3]])).sum(0) / w.sum()
+        np.testing.assert_allclose(res["out"][h], ref, atol=1e-14)
+
+
+def test_group_selection_is_head_order_free_and_the_best_subset():
+    """Permuting the heads permutes the outputs only; at every level the kept
+    set has the largest total group score among all subsets of its size."""
+    import itertools
+    rng = np.random.default_rng(23)
+    B, b, d, T, W, k = 2, 3, 8, 120, 3, 2
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 4, 1, B, b, k, W, rope=True, rope_base=1e3)
+    for t in [50, 119]:
+        Qg = rng.standard_normal((4, d)) * 2
+        res = oracle.group_traverse_and_attend(Qg, t, K, V, tree, geo)
+        perm = [2, 0, 3, 1]
+        res_p = oracle.group_traverse_and_attend(Qg[perm], t, K, V, tree, geo)
+        assert res_p["kept"] == res["kept"]
+        np.testing.assert_allclose(res_p["out"], res["out"][perm], atol=1e-13)
+        for lev, kept in res["kept"].items():
+            sc, ids = res["group"][lev], res["cand_ids"][lev]
+            n = min(k, len(sc))
+            assert len(kept) == n and res["heads"][0]["kept"][lev] == kept
+            best = max(sum(sc[i] for i in s) for s in itertools.combinations(range(len(sc)), n))
+            assert abs(sum(sc[ids.index(x)] for x in kept) - best) < 1e-12
