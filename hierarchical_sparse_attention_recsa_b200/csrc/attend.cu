@@ -65,6 +65,9 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   int* zkup = reinterpret_cast<int*>(scl + 8);                 // [8] expanded one level up
   int* zc = zkup + 8;                                          // [8][kMaxLevels + 1] candidates
   int* zk = zc + 8 * (kMaxLevels + 1);                         // [8][kMaxLevels + 1] expanded
+  // GROUP: per head max and sum of exp over the level's candidates
+  float* gmx = reinterpret_cast<float*>(zk + 8 * (kMaxLevels + 1));   // [8]
+  float* gsm = gmx + 8;                                               // [8]
 
   const int64_t t = decode ? len_dev[seq] - 1 : q_start + qi;
   const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * d;
@@ -95,6 +98,7 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   __syncthreads();
 
   const bool zha = p.mode == RECSA_MODE_ZHA;
+  const bool group = p.mode == RECSA_MODE_GROUP;
   constexpr int LS = kMaxLevels + 1;
   // Query rotated to index idx (idx < 0: copied un-rotated).
   auto rotate_q = [&](int64_t idx) {
@@ -203,7 +207,41 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       if (lane == 0) score[h * cmax + ii] = s;
     }
     __syncthreads();
-    for (int x = tid; x < G * cmx; x += kThreads) {
+    if (group) {
+      // One selection for the G heads (all have c = cmx candidates): group
+      // score = sum over heads of the candidate's softmax probability, ranked
+      // with ties to the lower index; every head gets the shared ranks.
+      if (warp < G) {
+        const float* row = score + warp * cmax;
+        float mx = -INFINITY;
+        for (int e = lane; e < cmx; e += 32) mx = fmaxf(mx, row[e]);
+        mx = warp_max(mx);
+        float sm = 0.f;
+        for (int e = lane; e < cmx; e += 32) sm += expf(row[e] - mx);
+        sm = warp_sum(sm);
+        if (lane == 0) {
+          gmx[warp] = mx;
+          gsm[warp] = sm;
+        }
+      }
+      __syncthreads();
+      for (int ii = tid; ii < cmx; ii += kThreads) {
+        float agg = 0.f;
+        for (int h = 0; h < G; ++h) agg += expf(score[h * cmax + ii] - gmx[h]) / gsm[h];
+        wts[ii] = agg;
+      }
+      __syncthreads();
+      for (int ii = tid; ii < cmx; ii += kThreads) {
+        const float s = wts[ii];
+        int r = 0;
+        for (int jj = 0; jj < cmx; ++jj) {
+          const float sj = wts[jj];
+          r += (sj > s) || (sj == s && jj < ii);
+        }
+        for (int h = 0; h < G; ++h) rank[h * cmax + ii] = r;
+      }
+    }
+    for (int x = tid; x < G * cmx && !group; x += kThreads) {
       const int h = x / cmx, ii = x % cmx;
       const int c = p.b * zkup[h] + norph;
       if (ii >= c) continue;
@@ -369,7 +407,7 @@ cudaError_t attend_typed(const Params& p, const void* Q, const void* K, const vo
   const int G = p.group;
   size_t bytes = size_t(G) * d * 4 * 2 + size_t(G) * cmax * 16 + size_t(G) * kmax * 4 +
                  size_t(G) * kTokChunk * 8 + 8 + size_t(G) * kTokChunk * 8 + 3 * 8 * 4 + 64 +
-                 size_t(8 + 16 * (kMaxLevels + 1)) * 4;
+                 size_t(8 + 16 * (kMaxLevels + 1) + 16) * 4;
   if (bytes > 200 * 1024) return cudaErrorInvalidConfiguration;
   auto kern = attend_kernel<T, P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -1258,7 +1258,7 @@ cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, cons
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // ZHA: generic kernel
+  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
   StepArgs st = {};
   return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s, st);
 }
@@ -1267,7 +1267,7 @@ cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
                                const void* k_new, const void* v_new, int64_t* len_dev,
                                const float* r, int64_t r_stride, void* tree, int32_t n_q,
                                void* O, int32_t* trace, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // ZHA: generic kernel
+  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
   if (p.batch > kStepCounters) return cudaErrorNotSupported;
   StepArgs st;
   st.k_new = k_new;

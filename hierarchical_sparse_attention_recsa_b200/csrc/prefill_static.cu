@@ -49,7 +49,7 @@ size_t prefill_static_bytes() { return kStaticFloats * sizeof(float); }
 cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, int64_t q_start, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // ZHA: generic kernel
+  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
   void* ml = nullptr;
   cudaError_t e = scratch_address(&ml);
   if (e != cudaSuccess) return e;

@@ -456,7 +456,7 @@ cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const v
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
                                 int32_t* trace, const void* wpart, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // ZHA: generic kernel
+  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
   if (p.dtype == RECSA_DTYPE_BF16)
     return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s)
                       : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);

@@ -28,7 +28,8 @@ recsa_status check_geometry(const recsa_geometry* g) {
   if (g->rope_enabled != 0 && g->rope_enabled != 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->rope_enabled && !(g->rope_base > 1.0f)) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->batch < 1 || g->capacity < 1 || g->reserved != 0) return RECSA_ERR_INVALID_GEOMETRY;
-  if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA && g->mode != RECSA_MODE_GROUP)
+    return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode == RECSA_MODE_ZHA && !(g->top_p > 0.f && g->top_p <= 1.f))
     return RECSA_ERR_INVALID_GEOMETRY;
   if (g->capacity > int64_t(INT32_MAX)) return RECSA_ERR_INVALID_GEOMETRY;

@@ -23,6 +23,7 @@ DTYPE_F32 = 0
 DTYPE_BF16 = 1
 MODE_RECSA = 0
 MODE_ZHA = 1
+MODE_GROUP = 2
 KEEP_ALL = 2**31 - 1
 MAX_LEVELS = 16
 TRACE_MAX_K = 64
@@ -87,7 +88,7 @@ class Geometry:
     dtype: int = DTYPE_BF16
     rope_enabled: int = 1
     rope_base: float = 1e6
-    mode: int = 0          # MODE_RECSA or MODE_ZHA
+    mode: int = 0          # MODE_RECSA, MODE_ZHA or MODE_GROUP
     top_p: float = 0.0     # ZHA routing mass
 
     def c(self) -> CGeometry:

@@ -64,6 +64,7 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
 /* recsa_geometry.mode */
 #define RECSA_MODE_RECSA 0
 #define RECSA_MODE_ZHA 1
+#define RECSA_MODE_GROUP 2
 
 /* Device error flags in the tree header (recsa_tree_error). */
 #define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
@@ -90,8 +91,14 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   the smallest set of highest-scoring candidates whose softmax mass reaches
  *   top_p (at most k of them), scores are q . key / sqrt(d) without rotation,
  *   and the attention covers only the tokens of the reached leaves and the
- *   window, at their true positions with standard RoPE (no summaries).  ZHA
- *   runs on the generic kernel.
+ *   window, at their true positions with standard RoPE (no summaries); or
+ *   RECSA_MODE_GROUP, RecSA with one selection per KV group (the "per KV
+ *   group" convention of the same page's Table IX): the G query heads of a
+ *   KV head score the shared candidates with their own RecSA logits, a
+ *   candidate's group score is the sum over the G heads of its softmax
+ *   probability among the level's candidates, the top min(k, c) group scores
+ *   are kept (ties -> lower index) for all G heads, and each head then
+ *   attends as in RecSA.
  */
 typedef struct recsa_geometry {
   int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
@@ -105,7 +112,7 @@ typedef struct recsa_geometry {
   int32_t rope_enabled; /* 0 or 1 */
   float rope_base;      /* > 1 */
   int32_t batch;        /* sequences, >= 1 */
-  int32_t mode;         /* RECSA_MODE_RECSA (0) or RECSA_MODE_ZHA (1) */
+  int32_t mode;         /* RECSA_MODE_RECSA (0), RECSA_MODE_ZHA (1), RECSA_MODE_GROUP (2) */
   int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
   float top_p;          /* ZHA: routing mass in (0, 1]; ignored in RECSA mode */
   int32_t reserved;     /* must be 0 */

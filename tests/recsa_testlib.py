@@ -224,3 +224,51 @@ def check_query_zha(stats: Stats, gpu_out, trace_rec, q, t, K, V, tree_src, og, 
         assert tr["keys_read"] == res["n_exact"] + sum(res["cand"].values())
     stats.add(gpu_out, res["out"])
     return res
+
+
+# ---------------------------------------------------------------------------
+# Per-KV-group shared selection
+# ---------------------------------------------------------------------------
+
+GROUP_GAP = 2e-4   # group scores are sums of G probabilities; fp32 error ~1e-5 at most
+
+
+def check_group(stats: Stats, gpu_out, trace_recs, Qg, t, K, V, tree_src, og, k_trace):
+    """Compare the G heads of one KV group (GPU outputs [G, d], trace records
+    [G, ints]) with the group-selection oracle."""
+    res = oracle.group_traverse_and_attend(Qg, t, K, V, tree_src, og)
+    if trace_recs is not None:
+        trs = [parse_trace(rec, k_trace) for rec in trace_recs]
+        kept = {l: list(v) for l, v in trs[0]["kept"].items()}
+        cf = oracle.closed_form_counts(t, og)
+        for tr in trs:
+            assert {l: list(v) for l, v in tr["kept"].items()} == kept   # one selection
+            assert tr["top"] == res["top"]
+            assert tr["cand"] == res["cand"] == cf["cand"]
+            assert tr["entries"] == cf["entries"] and tr["keys_read"] == cf["keys_read"]
+        want = {l: list(v) for l, v in res["kept"].items()}
+        clear = True
+        for lev, sc in res["group"].items():
+            n = min(og.k, len(sc))
+            s = sorted(sc, reverse=True)
+            if n < len(s) and s[n - 1] - s[n] <= GROUP_GAP:
+                clear = False
+        if clear:
+            stats.clear += 1
+            assert kept == want, (t, kept, want)
+        else:
+            stats.near_tie += 1
+            if kept != want:
+                # the first level that differs has the same candidates: the
+                # GPU's set must be a top-k there within the gap
+                lev = max(l for l in want if kept[l] != want[l])
+                sc, ids = res["group"][lev], res["cand_ids"][lev]
+                inside = [sc[ids.index(x)] for x in kept[lev]]
+                outside = [sc[i] for i, x in enumerate(ids) if x not in set(kept[lev])]
+                if outside:
+                    assert min(inside) >= max(outside) - GROUP_GAP, (t, lev)
+                res = oracle.group_traverse_and_attend(Qg, t, K, V, tree_src, og,
+                                                       keep_override=kept)
+    for h in range(len(gpu_out)):
+        stats.add(gpu_out[h], res["out"][h])
+    return res

@@ -62,6 +62,7 @@ def test_status_strings(lib):
     dict(k=R.KEEP_ALL, capacity=8192, rope_enabled=0),
     dict(mode=R.MODE_ZHA, top_p=0.9),
     dict(mode=R.MODE_ZHA, top_p=1.0, k=R.KEEP_ALL, capacity=8192),
+    dict(mode=R.MODE_GROUP),
 ])
 def test_valid_geometries(lib, kw):
     R.recsa_validate(geo(**kw))
@@ -71,7 +72,7 @@ def test_valid_geometries(lib, kw):
     dict(head_dim=96), dict(n_q_heads=24), dict(n_q_heads=12, n_kv_heads=4),
     dict(branching=1), dict(window=0), dict(k=0), dict(leaf_block=0), dict(batch=0),
     dict(capacity=0), dict(dtype=7), dict(rope_base=1.0), dict(n_kv_heads=0),
-    dict(mode=2), dict(mode=R.MODE_ZHA, top_p=0.0), dict(mode=R.MODE_ZHA, top_p=1.5),
+    dict(mode=3), dict(mode=-1), dict(mode=R.MODE_ZHA, top_p=0.0), dict(mode=R.MODE_ZHA, top_p=1.5),
     dict(mode=R.MODE_ZHA, top_p=float("nan")),
 ])
 def test_invalid_geometries(lib, kw):
