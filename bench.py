@@ -349,26 +349,33 @@ def run_recsa(args, rank, world, dev):
         out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
+    cpu_leg = rank == 0 and world == 1 and not args.no_cpu
     if not args.no_zha:
-        out["zha"] = run_zha(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind,
-                             cpu=(rank == 0 and world == 1 and not args.no_cpu))
+        out["zha"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
+                                 peak_kind, R.MODE_ZHA, cpu_leg)
+    if not args.no_group:
+        out["group"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
+                                   peak_kind, R.MODE_GROUP, cpu_leg)
     return out
 
 
 ZHA_TOP_P = 0.9
 
 
-def run_zha(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, cpu):
-    """The ZHA routing variant (top-p expansion, exact tokens of the reached
-    leaves and the window at true positions) on the same cache: its own tree
-    (same pooling; the RoPE table covers every position), then the batch's
-    decode queries at t = L - 1, timed per launch like the main decode."""
+def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, mode, cpu):
+    """A selection variant on the same cache: its own tree (same pooling),
+    then the batch's decode queries at t = L - 1, timed per launch like the
+    main decode.  MODE_ZHA: top-p expansion, exact tokens of the reached
+    leaves and the window at true positions (the RoPE table covers every
+    position).  MODE_GROUP: RecSA with one selection per KV group."""
     batch = Kc.shape[0]
+    zha = mode == R.MODE_ZHA
     g = R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    leaf_block=w.leaf_block, branching=w.branching, k=w.k, window=w.window,
                    batch=batch, capacity=cap,
                    dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
-                   rope_enabled=1, rope_base=w.rope_base, mode=R.MODE_ZHA, top_p=ZHA_TOP_P)
+                   rope_enabled=1, rope_base=w.rope_base, mode=mode,
+                   top_p=ZHA_TOP_P if zha else 0.0)
     tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
     R.recsa_build(g, Kc, Vc, [L] * batch, r, 0, tree)
     lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
@@ -392,22 +399,25 @@ def run_zha(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, c
     G = w.n_q_heads // w.n_kv_heads
     nb = [counts.decode_bytes_from_trace(tr[i], np.full(batch, L), w.leaf_block, w.branching,
                                          w.window, G, w.head_dim, elem_bytes(w), w.k,
-                                         summary_values=False)["bytes"] for i in range(n)]
+                                         summary_values=not zha)["bytes"] for i in range(n)]
     kept = tr[..., 4 + 16:4 + 16 + R.recsa_num_levels(g, L)].astype(np.float64)
     nbytes = float(np.mean(nb))
     achieved = nbytes / (dec_ms / 1e3) / 1e9
-    res = {"top_p": ZHA_TOP_P, "value": batch / (dec_ms / 1e3), "unit": "queries/s",
-           "decode_ms": dec_ms, "kernel": "zha_attend_kernel (one CTA per query head)",
+    res = {"value": batch / (dec_ms / 1e3), "unit": "queries/s", "decode_ms": dec_ms,
+           "kernel": "zha_attend_kernel (one CTA per query head)" if zha else
+                     "decode_cluster_kernel (all G heads per CTA, one selection per KV group)",
            "kept_per_level_mean": [float(x) for x in kept.mean(axis=(0, 1, 2, 3))],
            "exact_tokens_mean": float(tr[..., 3].mean()),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                         "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                         "bytes_per_launch": nbytes, "traffic": None}}
+    if zha:
+        res["top_p"] = ZHA_TOP_P
     del tree, traces
     torch.cuda.empty_cache()
     if cpu:
         res["cpu_baseline"] = cpu_baseline(args.workload, seconds=min(args.cpu_seconds, 10.0),
-                                           top_p=ZHA_TOP_P)
+                                           variant="zha" if zha else "group")
     return res
 
 
@@ -556,19 +566,26 @@ class OracleDecode:
         # untimed: pool the nodes the first query visits (the oracle's tree build)
         self.query_heads(1)
 
-    def query_heads(self, n_heads, top_p=None):
-        """Run n_heads (query, head) pairs; top_p given: the ZHA routing variant."""
+    def query_heads(self, n_heads, variant=None):
+        """Run n_heads (query, head) pairs (whole groups of G for "group"):
+        RecSA, or the "zha" routing variant, or "group" shared selection."""
         done = 0
         while done < n_heads:
             i = self.i % self.Q.shape[0]
             t = self.L + i - 1
             h = done % self.G
-            if top_p is None:
+            if variant == "group":
+                self.oracle.group_traverse_and_attend(self.Q[i], t, self.K, self.V, self.tree,
+                                                      self.geo)
+                done += self.G
+                self.i += 1
+                continue
+            if variant is None:
                 self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
                                                 self.geo)
             else:
                 self.oracle.zha_route_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
-                                                 self.geo, top_p)
+                                                 self.geo, ZHA_TOP_P)
             done += 1
             if h == self.G - 1:
                 self.i += 1
@@ -583,18 +600,19 @@ def _single_thread():
         return None
 
 
-def cpu_baseline(workload=WORKLOAD, seconds=15.0, top_p=None):
+def cpu_baseline(workload=WORKLOAD, seconds=15.0, variant=None):
     lim = _single_thread()
     o = OracleDecode(workload)
-    if top_p is not None:
-        o.query_heads(o.G, top_p)      # untimed: pool the nodes this routing visits first
+    if variant is not None:
+        o.query_heads(o.G, variant)    # untimed: pool the nodes this selection visits first
     t0 = time.perf_counter()
     heads = 0
     while time.perf_counter() - t0 < seconds:
-        heads += o.query_heads(o.G, top_p)
+        heads += o.query_heads(o.G, variant)
     dt = time.perf_counter() - t0
     del lim
-    what = "decode" if top_p is None else f"ZHA decode (top-p {top_p})"
+    what = {None: "decode", "zha": f"ZHA decode (top-p {ZHA_TOP_P})",
+            "group": "group-selection decode"}[variant]
     return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
             "kind": "oracle",
             "sample": f"{heads} query-heads ({what} at t=L, one KV head's tree, G={o.G}) in "
@@ -647,6 +665,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-zha", action="store_true",
                     help="skip the ZHA routing-variant decode leg")
+    ap.add_argument("--no-group", action="store_true",
+                    help="skip the per-KV-group shared-selection decode leg")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--only-decode", action="store_true",
                     help="decode steps only (no prefill, dense, e2e or CPU legs); for profiling")
@@ -655,7 +675,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.only_decode:
-        args.no_prefill = args.no_dense = args.no_cpu = args.no_zha = True
+        args.no_prefill = args.no_dense = args.no_cpu = args.no_zha = args.no_group = True
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))

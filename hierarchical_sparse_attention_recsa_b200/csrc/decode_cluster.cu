@@ -198,13 +198,14 @@ __device__ __forceinline__ void merge_xor(float& m, float& l, float* acc, int o)
 
 // Shared-memory plan of one CTA (byte offsets), the same on host and device.
 struct Plan {
-  unsigned mb, qf, qtok, qlev, rrow, sc, wsc, wwin, mrg, kept, kfl, rmask, wbuf, kbuf, vbuf, total;
+  unsigned mb, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, mrg, kept, kfl, rmask, wbuf, kbuf, vbuf,
+      total;
   int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
   unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
 };
 template <typename T, int D, int G, int HPC>
 __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, int CS, int NRH,
-                                                   int B, int levels) {
+                                                   int B, int levels, int HB) {
   constexpr unsigned RS = D + 2;
   Plan q;
   unsigned o = 0;
@@ -214,6 +215,7 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   q.qlev = o; o += unsigned(levels) * HPC * D * 4;        // query rotated per level
   q.rrow = o; o += unsigned(2 * levels + 3) * D * 4;      // RoPE table rows (cos, sin)
   q.sc = o;   o += 2 * HPC * unsigned(cmax) * 4;
+  q.agg = o;  o += unsigned(cmax) * 4;                    // group scores (RECSA_MODE_GROUP)
   q.wsc = o;  o += kChainWarps * RS * 4;
   q.wwin = o; o += kWinWarps * G * RS * 4;
   q.mrg = o;  o += unsigned(CS) * HPC * RS * 4;
@@ -226,9 +228,9 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   o = (o + 127u) & ~127u;
   q.kbuf = o;
   q.rows = (cmax + S - 1) / S;
-  q.kbytes = HPC * unsigned(q.rows) * D * 4;
+  q.kbytes = unsigned(HB) * unsigned(q.rows) * D * 4;   // HB heads' level rows
   q.vbuf = o + q.kbytes;
-  const unsigned toks = HPC * unsigned(NRH) * 2 * unsigned(B) * D * unsigned(sizeof(T));
+  const unsigned toks = unsigned(HB) * unsigned(NRH) * 2 * unsigned(B) * D * unsigned(sizeof(T));
   o += 2 * q.kbytes > toks ? 2 * q.kbytes : toks;
   q.total = o;
   return q;
@@ -258,7 +260,12 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int sub = lane % LPR;
   const int j0 = 4 * sub;
 
-  const Plan pl = make_plan<T, D, G, HPC>(cmax, kmax, S, CS, NRH, p.B, p.lay.levels);
+  // RECSA_MODE_GROUP: the G heads share one selection, hence one copy of a
+  // level's candidate rows and one ring of kept leaves (HB = 1 buffer head).
+  // (only launched with every head of the group in the CTA: HPC == G)
+  const bool grp = HPC == G && p.mode == RECSA_MODE_GROUP;
+  const int HB = grp ? 1 : HPC;
+  const Plan pl = make_plan<T, D, G, HPC>(cmax, kmax, S, CS, NRH, p.B, p.lay.levels, HB);
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t* mb_lev = reinterpret_cast<uint64_t*>(smem + pl.mb);   // level keys arrived
   uint64_t* mb_val = mb_lev + 1;                                   // level values arrived
@@ -276,6 +283,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // R(c_l) (the query's index at level l), [2 levels + 2] = R(n0 - 1)
   float* rrow = reinterpret_cast<float*>(smem + pl.rrow);
   float* sc = reinterpret_cast<float*>(smem + pl.sc);       // [2][HPC][cmax] scores
+  float* agg = reinterpret_cast<float*>(smem + pl.agg);     // [cmax] group scores
   float* wsc = reinterpret_cast<float*>(smem + pl.wsc);     // [kChainWarps][RS]
   float* wwin = reinterpret_cast<float*>(smem + pl.wwin);   // [kWinWarps][G][RS]
   float* mrg = reinterpret_cast<float*>(smem + pl.mrg);     // [CS][HPC][RS] received
@@ -283,9 +291,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   unsigned char* kfl = smem + pl.kfl;                       // [2][HPC][cmax]
   unsigned* rmask = reinterpret_cast<unsigned*>(smem + pl.rmask);   // [HPC][32] kept bits
   T* wbuf = reinterpret_cast<T*>(smem + pl.wbuf);           // [kWinRing][2][kWinChunk][D]
-  float* kbuf = reinterpret_cast<float*>(smem + pl.kbuf);   // [HPC][rows][D] level keys
-  float* vbuf = reinterpret_cast<float*>(smem + pl.vbuf);   // [HPC][rows][D] level values
-  T* tbuf = reinterpret_cast<T*>(smem + pl.kbuf);           // [HPC][NRH][2][B][D] kept leaves
+  float* kbuf = reinterpret_cast<float*>(smem + pl.kbuf);   // [HB][rows][D] level keys
+  float* vbuf = reinterpret_cast<float*>(smem + pl.vbuf);   // [HB][rows][D] level values
+  T* tbuf = reinterpret_cast<T*>(smem + pl.kbuf);           // [HB][NRH][2][B][D] kept leaves
 
   // Fused step: the new token is appended at len (this kernel writes it and
   // pools what it completes), and the query sits on it.  A full sequence is
@@ -359,7 +367,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     for (int i = 0; i < kWinRing; ++i) mbar_init(mb_win + i, 1);
     for (int i = 0; i < HPC * NRH; ++i) {
       mbar_init(mb_tok + i, 1);
-      mbar_init(mb_empty + i, 1);
+      mbar_init(mb_empty + i, grp ? unsigned(HPC) : 1u);   // a shared slot: every head frees it
     }
     mbar_fence_init();
   }
@@ -404,7 +412,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const unsigned rb = D * 4;
     uint64_t* mb = values ? mb_val : mb_lev;
     float* dst = values ? vbuf : kbuf;
-    if (lane == 0) mbar_expect_tx(mb, unsigned(HPC) * unsigned(hi - lo) * rb);
+    if (lane == 0) mbar_expect_tx(mb, unsigned(HB) * unsigned(hi - lo) * rb);
     __syncwarp();
     if (hi <= lo) return;
     const float* src = values ? level_vals(p, const_cast<void*>(tree), lev, seq, g)
@@ -414,7 +422,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int orph0 = lev < top ? p.b * int(vis[lev + 1]) : 0;   // first orphan node
     const int* keptu = kept + ((lev + 1) & 1) * HPC * kmax;
     const int nrun = kup + 1;
-    for (int x = lane; x < HPC * nrun; x += 32) {
+    for (int x = lane; x < HB * nrun; x += 32) {
       const int h = x / nrun, r = x % nrun;
       int c0, c1, node0;
       if (r < kup) {
@@ -472,6 +480,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // Chain warps [h * WPH, (h + 1) * WPH) serve local query head h (global
   // head hg * HPC + h); hs is the lane slot's index within the head's warps.
   const int hw = warp / WPH;
+  const int hb = grp ? 0 : hw;   // its buffer head
   const int hs = (warp % WPH) * SPW + lane / LPR;
   // RoPE of the slot's first row and of its row step, for the recurrences
   float cs_hs[8], cs_st[8];
@@ -640,7 +649,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     int lo, hi;
     share(cnt_c[lev], lo, hi);
     const int nr = hi - lo;
-    const float* kb = kbuf + size_t(hw) * pl.rows * D;
+    const float* kb = kbuf + size_t(hb) * pl.rows * D;
     float* scK = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
     float q0[8], st2[8];
     lds_pairs(qlev + ((lev - 1) * HPC + hw) * D, j0, HALF, q0);
@@ -705,7 +714,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     int lo, hi;
     share(cnt_c[lev], lo, hi);
     const int nr = hi - lo;
-    const float* vb = vbuf + size_t(hw) * pl.rows * D;
+    const float* vb = vbuf + size_t(hb) * pl.rows * D;
     const float* scV = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
     const unsigned char* flV = kfl + (lev & 1) * HPC * cmax + hw * cmax + lo;
     for (int e = hs; e < nr; e += 2 * HSLOT) {
@@ -729,11 +738,39 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // s of `taken` marks candidate 32 s + l as kept.  Candidates beyond
   // 32 * kRegSlots are read from shared memory in the same rounds.  The kept
   // list is compacted in index order with one ballot per slot row.
+  // RECSA_MODE_GROUP (all G heads in the CTA): head 0's warp selects once for
+  // the group on the group scores -- the sum over the heads of each
+  // candidate's softmax probability among the level's candidates -- and
+  // hands the same masks to every head.
   auto topk = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
     const int h = 3 - warp;
+    if (grp && h != 0) return;
     const float* row = sc + par * HPC * cmax + h * cmax;
+    if (grp) {
+      float mxh[HPC], smh[HPC];
+#pragma unroll
+      for (int hh = 0; hh < HPC; ++hh) {
+        const float* rw = sc + par * HPC * cmax + hh * cmax;
+        float mx = -INFINITY;
+        for (int i = lane; i < c; i += 32) mx = fmaxf(mx, rw[i]);
+        mx = warp_max(mx);
+        float sm = 0.f;
+        for (int i = lane; i < c; i += 32) sm += expf(rw[i] - mx);
+        mxh[hh] = mx;
+        smh[hh] = warp_sum(sm);
+      }
+      for (int i = lane; i < c; i += 32) {
+        float a_ = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < HPC; ++hh)
+          a_ += expf(sc[par * HPC * cmax + hh * cmax + i] - mxh[hh]) / smh[hh];
+        agg[i] = a_;
+      }
+      __syncwarp();
+      row = agg;
+    }
     const int ns = (c + 31) >> 5;
     unsigned taken = 0;
     if (kap >= c) {
@@ -786,9 +823,17 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       const unsigned R = __ballot_sync(0xffffffffu, (taken >> s) & 1u);
       if (lane == s) mine = R;
     }
-    if (lane < ns) rmask[h * 32 + lane] = mine;
+    if (lane < ns) {
+      if (grp) {
+#pragma unroll
+        for (int hh = 0; hh < HPC; ++hh) rmask[hh * 32 + lane] = mine;
+      } else {
+        rmask[h * 32 + lane] = mine;
+      }
+    }
     __syncwarp();
-    if (lane == 0) mbar_arrive(mb_kept);   // the producer reads the masks
+    if (lane == 0)   // the producer reads the masks (one arrival per head)
+      for (int n = 0; n < (grp ? HPC : 1); ++n) mbar_arrive(mb_kept);
   };
 
   // Kept flags and the kept list (in index order) of level lev from the row
@@ -856,10 +901,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     for (int j = 0; j < ntok;) {
       const int nl = (S == 1 && NRH >= 2 && j + 1 < ntok) ? 2 : 1;
       const int slot0 = j % NRH, slot1 = (j + 1) % NRH;
-      mbar_wait(mb_tok + hw * NRH + slot0, unsigned(j / NRH) & 1u, timed_out);
-      if (nl == 2) mbar_wait(mb_tok + hw * NRH + slot1, unsigned((j + 1) / NRH) & 1u, timed_out);
-      const T* cK0 = tbuf + (size_t(hw) * NRH + slot0) * slot_elems;
-      const T* cK1 = tbuf + (size_t(hw) * NRH + slot1) * slot_elems;
+      mbar_wait(mb_tok + hb * NRH + slot0, unsigned(j / NRH) & 1u, timed_out);
+      if (nl == 2) mbar_wait(mb_tok + hb * NRH + slot1, unsigned((j + 1) / NRH) & 1u, timed_out);
+      const T* cK0 = tbuf + (size_t(hb) * NRH + slot0) * slot_elems;
+      const T* cK1 = tbuf + (size_t(hb) * NRH + slot1) * slot_elems;
       float q0[8];
       if (p.rope) {
         float seed[8], r[8], t2[8];
@@ -905,8 +950,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       }
       named_sync(lbar, WPH * 32);
       if (warp == hw * WPH && lane == 0) {
-        if (j + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot0);
-        if (nl == 2 && j + 1 + NRH < ntok) mbar_arrive(mb_empty + hw * NRH + slot1);
+        if (j + NRH < ntok) mbar_arrive(mb_empty + hb * NRH + slot0);
+        if (nl == 2 && j + 1 + NRH < ntok) mbar_arrive(mb_empty + hb * NRH + slot1);
       }
       j += nl;
     }
@@ -950,7 +995,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       __syncwarp();
       if (lev > 1) {
         issue_level(lev - 1, false, true);
-      } else if (lane < HPC) {
+      } else if (lane < HB) {
         for (int j = 0; j < NRH && j < ntok; ++j)
           if (early_slot(lane, j)) issue_tok(lane, j, true);
       }
@@ -962,12 +1007,12 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       __syncwarp();
       if (lev > 1) {
         issue_level(lev - 1, true, false);
-      } else if (lane < HPC) {
+      } else if (lane < HB) {
         for (int j = 0; j < NRH && j < ntok; ++j)
           if (!early_slot(lane, j)) issue_tok(lane, j, false);
       }
     }
-    if (top > 0 && lane < HPC) {
+    if (top > 0 && lane < HB) {
       const int h = lane;
       for (int j = NRH; j < ntok; ++j) {
         mbar_wait(mb_empty + h * NRH + j % NRH, unsigned(j / NRH - 1) & 1u, timed_out);
@@ -1166,7 +1211,8 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
   for (;;) {
     if (cs > kMaxCluster) return cudaErrorNotSupported;
     for (nrh = kMaxTokSlots; nrh >= 1; --nrh) {
-      pl = make_plan<T, D, G, HPC>(cmax, kmax, S, cs, nrh, p.B, p.lay.levels);
+      pl = make_plan<T, D, G, HPC>(cmax, kmax, S, cs, nrh, p.B, p.lay.levels,
+                                   p.mode == RECSA_MODE_GROUP ? 1 : HPC);
       if (pl.total <= kSmemLimit) break;
     }
     if (nrh >= 1) break;
@@ -1234,7 +1280,7 @@ void decode_split(const Params& p, int32_t n_q, int& hpc, int& S) {
   }
   const int64_t pairs = int64_t(p.batch) * p.hkv * n_q;
   hpc = 1;
-  while (hpc < G && pairs * (G / hpc) > 148) hpc *= 2;
+  while (hpc < G && (pairs * (G / hpc) > 148 || p.mode == RECSA_MODE_GROUP)) hpc *= 2;
   const int ng = G / hpc;
   S = 1;
   while (ng * S * 2 <= kMaxCluster && pairs * ng * S * 2 <= 148) S *= 2;
@@ -1245,6 +1291,8 @@ cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, cons
                              int32_t* trace, cudaStream_t s, StepArgs st) {
   int hpc = 1, S = 1;
   decode_split(p, n_q, hpc, S);
+  // group selection needs every head's scores in each CTA
+  if (p.mode == RECSA_MODE_GROUP && hpc != p.group) return cudaErrorNotSupported;
   if (p.dtype == RECSA_DTYPE_BF16)
     return p.d == 128
                ? cluster_g<__nv_bfloat16, 128>(p, Q, K, V, tree, len_dev, n_q, O, trace, s, hpc, S, st)
@@ -1258,7 +1306,7 @@ cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, cons
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
+  if (p.mode != RECSA_MODE_RECSA && p.mode != RECSA_MODE_GROUP) return cudaErrorNotSupported;
   StepArgs st = {};
   return cluster_dispatch(p, Q, K, V, tree, len_dev, n_q, O, trace, s, st);
 }
@@ -1267,7 +1315,7 @@ cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
                                const void* k_new, const void* v_new, int64_t* len_dev,
                                const float* r, int64_t r_stride, void* tree, int32_t n_q,
                                void* O, int32_t* trace, cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
+  if (p.mode != RECSA_MODE_RECSA && p.mode != RECSA_MODE_GROUP) return cudaErrorNotSupported;
   if (p.batch > kStepCounters) return cudaErrorNotSupported;
   StepArgs st;
   st.k_new = k_new;

@@ -9,6 +9,8 @@ validity check plus an output comparison under the GPU's selection elsewhere
 (recsa_testlib.check_group).
 """
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -29,6 +31,26 @@ MODEL = synth.WORKLOADS["qwen3-4b-131k"]
 def _lib():
     build_lib.build()
     R.lib()
+
+
+@pytest.fixture(params=["cluster-auto", "cluster-4,1", "generic"])
+def decode_impl(request):
+    """Decode on the cluster kernel (all G heads in each CTA; automatic
+    candidate shares, or one share) or on the generic kernel."""
+    keys = ("RECSA_DECODE_SPLIT", "RECSA_DECODE_GENERIC")
+    old = {k: os.environ.get(k) for k in keys}
+    for k in keys:
+        os.environ.pop(k, None)
+    if request.param == "generic":
+        os.environ["RECSA_DECODE_GENERIC"] = "1"
+    elif request.param == "cluster-4,1":
+        os.environ["RECSA_DECODE_SPLIT"] = "4,1"
+    yield request.param
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
 
 
 def _setup(w, lens, capacity, seed=0, k=None, rope=1):
@@ -53,7 +75,7 @@ def _trees(g, K, V, r, lens):
     return out
 
 
-def test_group_decode_tiny():
+def test_group_decode_tiny(decode_impl):
     L, nq = TINY.length, TINY.n_q
     g, K, V, r, Kd, Vd, rd, tree = _setup(TINY, [L], L, seed=40)
     trees = _trees(g, K, V, r, [L])
@@ -72,7 +94,7 @@ def test_group_decode_tiny():
     st = Stats()
     for i in range(nq):
         check_group(st, O_[0, i], tr[0, i], to_np(Q[0, i]), L - 1, Kh, Vh, src, og, g.k)
-    st.check(torch.float32, "group decode tiny")
+    st.check(torch.float32, f"group {decode_impl} decode tiny")
     assert st.clear > 0.6 * nq
 
 
@@ -102,7 +124,7 @@ def test_group_prefill_tiny():
     st.check(torch.float32, "group prefill tiny")
 
 
-def test_group_decode_model_small():
+def test_group_decode_model_small(decode_impl):
     lens = [20000, 13001]
     g, K, V, r, Kd, Vd, rd, tree = _setup(MODEL, lens, 20480, seed=44)
     trees = _trees(g, K, V, r, lens)
@@ -127,7 +149,7 @@ def test_group_decode_model_small():
                 hs = slice(kv * G, (kv + 1) * G)
                 check_group(st, O_[s, i, hs], tr[s, i, hs], to_np(Q[s, i, hs]), L - 1, Kh, Vh,
                             src, og, g.k)
-    st.check(torch.bfloat16, "group decode model small")
+    st.check(torch.bfloat16, f"group {decode_impl} decode model small")
 
 
 @pytest.mark.parametrize("wname,rope", [("tiny-4k", 1), ("tiny-4k", 0), ("qwen3-4b-131k", 1)])
@@ -158,7 +180,7 @@ def test_group_keep_all_is_dense(wname, rope):
     st.check(w.dtype, "group keep-all")
 
 
-def test_group_decode_step_equals_append_then_decode():
+def test_group_decode_step_equals_append_then_decode(decode_impl):
     w = MODEL
     lens0 = [4000, 4031]
     steps = 70
@@ -203,6 +225,6 @@ def test_group_decode_step_equals_append_then_decode():
                     hs = slice(kv * G, (kv + 1) * G)
                     check_group(st, to_np(Oa[s, 0, hs]), tr[s, 0, hs], to_np(Q[s, 0, hs]),
                                 lens_now[s] - 1, Kh_all[kv], Vh_all[kv], src, og, g.k)
-    st.check(torch.bfloat16, "group decode step")
+    st.check(torch.bfloat16, f"group {decode_impl} decode step")
     assert torch.equal(Ka, Kb) and torch.equal(Va, Vb)
     assert torch.equal(tree_a[256:], tree_b[256:])
