@@ -18,7 +18,8 @@ Sources (web pages, cited by title and section):
     descent) and Table VIII (only full nodes exist: n_l = floor(T / C^l)).
     Its routing variant (top-p expansion, attention over the reached leaves)
     is in ``zha.py``; its Table IX convention of a selection per KV group is
-    applied to RecSA in ``group.py``.
+    applied to RecSA in ``group.py``; several reference queries per pooler
+    (Figure 3 caption) are in ``multiref.py``.
   * "Efficient Sequence Modeling, Issue 13", highlights and editor's note on
     RecSA (normalisation shared with exact tokens; one pooler for selection and
     summary keys).
@@ -44,3 +45,4 @@ from .recsa import (  # noqa: F401
 from .dense import dense_causal_attention  # noqa: F401
 from .zha import top_p_prefix, zha_route_and_attend  # noqa: F401
 from .group import group_select, group_traverse_and_attend  # noqa: F401
+from .multiref import MultiTree, build_tree_multi  # noqa: F401

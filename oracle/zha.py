@@ -16,6 +16,8 @@ Readings (pages silent; stated here and in the design notes):
     RecSA, so that every visible token stays reachable;
   * routing scores are q . key / sqrt(d) on the un-rotated query and summary
     keys: the tree pools pre-RoPE keys, and RoPE belongs to the main attention;
+    with several reference queries (a tree source whose keys are [R, d], see
+    multiref.py) a node scores the largest of its R dot products;
   * top-p: the smallest set of highest-scoring candidates whose softmax mass
     (over the level's candidates) reaches p, ties to the lower index, capped at
     k nodes (k = keep-all: no cap);
@@ -87,8 +89,9 @@ def zha_route_and_attend(q: np.ndarray, t: int, K, V, tree, geo: Geometry, top_p
         children = [n * b + c for n in expanded for c in range(b)]
         orphans = list(range(b * v_up, v[lev - 1]))
         cand = children + orphans
-        scores = [float(q @ np.asarray(tree.key(lev, n), np.float64)) * inv_sqrt_d
-                  for n in cand]
+        # a node with several reference keys [R, d] scores its best match
+        scores = [float(np.max(np.atleast_2d(np.asarray(tree.key(lev, n), np.float64)) @ q))
+                  * inv_sqrt_d for n in cand]
         if keep_override is not None:
             want = set(int(x) for x in keep_override[lev])
             idx = [i for i, n in enumerate(cand) if n in want]

@@ -564,3 +564,97 @@ def test_group_selection_is_head_order_free_and_the_best_subset():
             assert len(kept) == n and res["heads"][0]["kept"][lev] == kept
             best = max(sum(sc[i] for i in s) for s in itertools.combinations(range(len(sc)), n))
             assert abs(sum(sc[ids.index(x)] for x in kept) - best) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Several reference queries (R > 1, ZHA routing)
+# ---------------------------------------------------------------------------
+
+def test_multiref_copies_of_one_reference_are_the_single_tree():
+    rng = np.random.default_rng(31)
+    B, b, d, T, W, k = 4, 3, 8, 200, 6, 3
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    single = oracle.build_tree(K, V, r, B, b)
+    multi = oracle.build_tree_multi(K, V, np.stack([r, r, r]), B, b)
+    for (k1, v1), (k3, v3) in zip(single, multi):
+        assert k3.shape == (k1.shape[0], 3, d)
+        for j in range(3):
+            np.testing.assert_array_equal(k3[:, j], k1)
+        np.testing.assert_array_equal(v3, v1)
+    geo = Geometry(d, 1, 1, B, b, k, W, rope=True, rope_base=1e3)
+    for t in [40, 199]:
+        q = rng.standard_normal(d) * 2
+        a = oracle.zha_route_and_attend(q, t, K, V, oracle.FullTree(single), geo, 0.7)
+        c = oracle.zha_route_and_attend(q, t, K, V, oracle.MultiTree(multi), geo, 0.7)
+        assert a["kept"] == c["kept"]
+        np.testing.assert_allclose(a["out"], c["out"], atol=1e-15)
+
+
+def test_multiref_reference_j_is_its_own_recursive_tree():
+    """Reference j's parent keys pool reference j's child keys (not another
+    reference's): checked node by node against a direct recursive pooling."""
+    rng = np.random.default_rng(32)
+    B, b, d, T = 2, 3, 4, 60
+    K, V = _rand_kv(rng, T, d)
+    Rq = rng.standard_normal((2, d)) * 2
+    multi = oracle.build_tree_multi(K, V, Rq, B, b)
+    for j in range(2):
+        for lev in range(1, len(multi) + 1):
+            for n in range(multi[lev - 1][0].shape[0]):
+                key, val = oracle.node_summary(K, V, Rq[j], B, b, lev, n)
+                np.testing.assert_allclose(multi[lev - 1][0][n, j], key, atol=1e-13)
+                np.testing.assert_allclose(multi[lev - 1][1][n], val, atol=1e-13)
+    # the two references give different keys (the test above is not vacuous)
+    assert np.abs(multi[0][0][:, 0] - multi[0][0][:, 1]).max() > 1e-3
+
+
+def test_multiref_node_score_is_the_best_reference():
+    """Hand-built level of two nodes with two reference keys each (B = 1,
+    b = 4, W = 1, t = 2: both visible leaves are top-level orphans), k = 1,
+    p = 0.5, no RoPE, d = 2, q = (sqrt 2, 0).  Node 0's keys score (3, -3) and
+    node 1's (2, 2): the best-reference rule expands node 0 (3 > 2), while a
+    sum or a mean of the scores would expand node 1."""
+    s2 = math.sqrt(2.0)
+    keys = np.array([[[3.0, 0.0], [-3.0, 0.0]], [[2.0, 0.0], [2.0, 0.0]]])
+    vals = np.array([[1.0, 0.0], [0.0, 1.0]])
+
+    class Two:
+        def key(self, lev, n):
+            return keys[n]
+
+        def val(self, lev, n):
+            return vals[n]
+
+    K = np.array([[1.0, 0.0], [0.0, 1.0], [0.5, 0.5]])
+    V = np.array([[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]])
+    geo = Geometry(2, 1, 1, 1, 4, 1, 1, rope=False)
+    q = np.array([s2, 0.0])
+    res = oracle.zha_route_and_attend(q, 2, K, V, Two(), geo, 0.5)
+    assert res["top"] == 1 and res["cand"] == {1: 2}
+    np.testing.assert_allclose(res["scores"][1], [3.0, 2.0], atol=1e-15)
+    assert res["kept"] == {1: [0]}
+    # attention over leaf 0 (token 0) and the window [2, 2]
+    lg = np.array([q @ K[0], q @ K[2]]) / s2
+    w = np.exp(lg - lg.max())
+    np.testing.assert_allclose(res["out"], (w[:, None] * V[[0, 2]]).sum(0) / w.sum(),
+                               atol=1e-15)
+
+
+@pytest.mark.parametrize("rope", [False, True])
+def test_multiref_full_mass_is_dense(rope):
+    rng = np.random.default_rng(33)
+    B, b, d, T, W = 4, 3, 8, 120, 5
+    K, V = _rand_kv(rng, T, d)
+    Rq = rng.standard_normal((4, d))
+    tree = oracle.MultiTree(oracle.build_tree_multi(K, V, Rq, B, b))
+    geo = Geometry(d, 1, 1, B, b, oracle.recsa.KEEP_ALL, W, rope=rope, rope_base=1e3)
+    for t in [0, 37, 119]:
+        q = rng.standard_normal(d) * 2
+        res = oracle.zha_route_and_attend(q, t, K, V, tree, geo, top_p=1.0)
+        if rope:
+            qr = _rope_complex(q, t, 1e3)
+            Kr = np.stack([_rope_complex(K[j], j, 1e3) for j in range(t + 1)])
+        else:
+            qr, Kr = q, K[: t + 1]
+        np.testing.assert_allclose(res["out"], _sdpa(qr, Kr, V[: t + 1]), atol=1e-12)
