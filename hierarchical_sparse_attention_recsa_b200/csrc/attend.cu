@@ -203,7 +203,10 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     for (int pr = warp; pr < G * cmx; pr += kWarps) {
       const int h = pr / cmx, ii = pr % cmx;
       if (ii >= p.b * zkup[h] + norph) continue;  // warp-uniform
-      const float s = dot_row(h, keys + int64_t(cand[h * cmax + ii]) * d, zha ? -1 : ii);
+      // a node with several reference keys (ZHA) scores its best match
+      const float* kr = keys + int64_t(cand[h * cmax + ii]) * p.nref * d;
+      float s = dot_row(h, kr, zha ? -1 : ii);
+      for (int ref = 1; ref < p.nref; ++ref) s = fmaxf(s, dot_row(h, kr + ref * d, -1));
       if (lane == 0) score[h * cmax + ii] = s;
     }
     __syncthreads();

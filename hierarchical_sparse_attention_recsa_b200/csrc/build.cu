@@ -8,7 +8,10 @@
 // Hierarchical Tree-Structured Indexer", Figure 3: higher levels pool the
 // summaries of lower levels).  One warp pools one node with an online
 // softmax, so K and V are streamed exactly once; each lane owns d/32
-// contiguous channels and issues one 4..16-byte load per row.
+// contiguous channels and issues one 4..16-byte load per row.  With several
+// reference queries (ZHA, Figure 3 caption: the key nodes of each are stored
+// in parallel) the warp pools the node once per reference, reference j's
+// parent key from reference j's child keys; the value is the same for all.
 #include "recsa_internal.cuh"
 #include "pool.cuh"
 
@@ -24,15 +27,15 @@ __global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T
   const int64_t j = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int g = blockIdx.y;
   if (j >= n_leaf) return;
-  float rl[N];
-  load_r<N>(r + g * r_stride, lane, rl);
   const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
-  float key[N], val[N];
-  pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-  float* kd = level_keys(p, tree, 1, seq, g) + j * p.d;
-  float* vd = level_vals(p, tree, 1, seq, g) + j * p.d;
-  RowIO<float, N>::store(kd, lane, key);
-  RowIO<float, N>::store(vd, lane, val);
+  for (int ref = 0; ref < p.nref; ++ref) {
+    float rl[N];
+    load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
+    float key[N], val[N];
+    pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
+    RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + (j * p.nref + ref) * p.d, lane, key);
+    if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
+  }
 }
 
 // Level lev >= 2: one warp per node, pooling b child summaries.
@@ -44,14 +47,19 @@ __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, i
   const int64_t j = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int g = blockIdx.y;
   if (j >= n_nodes) return;
-  float rl[N];
-  load_r<N>(r + g * r_stride, lane, rl);
-  const float* ck = level_keys(p, tree, lev - 1, seq, g) + j * p.b * p.d;
   const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
-  float key[N], val[N];
-  pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
-  RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + j * p.d, lane, key);
-  RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + j * p.d, lane, val);
+  for (int ref = 0; ref < p.nref; ++ref) {
+    float rl[N];
+    load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
+    // reference ref's keys of the b children: row stride nref * d
+    const float* ck = level_keys(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.d;
+    float key[N], val[N];
+    pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val,
+                        int64_t(p.nref) * p.d);
+    RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d, lane,
+                           key);
+    if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + j * p.d, lane, val);
+  }
 }
 
 // Append one token per sequence; pool the leaf and ancestors it completes.
@@ -81,22 +89,30 @@ __global__ void __launch_bounds__(256) append_kernel(Params p, T* K, T* V, const
     const int nw = blockDim.x >> 5;
     const int64_t j = newlen / p.B - 1;
     for (int g = threadIdx.x >> 5; g < p.hkv; g += nw) {
-      float rl[N];
-      load_r<N>(r + g * r_stride, lane, rl);
-      const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
-      float key[N], val[N];
-      pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-      RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + j * p.d, lane, key);
-      RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
-      int64_t idx = j;
-      for (int lev = 2; lev <= p.lay.levels && (idx + 1) % p.b == 0; ++lev) {
-        idx = (idx + 1) / p.b - 1;
+      for (int ref = 0; ref < p.nref; ++ref) {
+        float rl[N];
+        load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
+        const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
+        float key[N], val[N];
+        pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
+        RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + (j * p.nref + ref) * p.d, lane,
+                               key);
+        if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
+        int64_t idx = j;
+        for (int lev = 2; lev <= p.lay.levels && (idx + 1) % p.b == 0; ++lev) {
+          idx = (idx + 1) / p.b - 1;
+          __syncwarp();
+          const float* ck =
+              level_keys(p, tree, lev - 1, seq, g) + (idx * p.b * p.nref + ref) * p.d;
+          const float* cv = level_vals(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
+          pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val,
+                              int64_t(p.nref) * p.d);
+          RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (idx * p.nref + ref) * p.d,
+                                 lane, key);
+          if (ref == 0)
+            RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + idx * p.d, lane, val);
+        }
         __syncwarp();
-        const float* ck = level_keys(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
-        const float* cv = level_vals(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
-        pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
-        RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + idx * p.d, lane, key);
-        RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + idx * p.d, lane, val);
       }
     }
   }

@@ -49,12 +49,14 @@ struct RowIO<__nv_bfloat16, 2> {
   }
 };
 
-// One warp pools `n` rows (keys at kbase, values at vbase, row stride d) into
-// this lane's N channels of key and value.  Rows are processed in groups of 8
-// so that eight loads per operand are in flight per lane.
+// One warp pools `n` rows (keys at kbase with row stride ks, values at vbase
+// with row stride d) into this lane's N channels of key and value.  Rows are
+// processed in groups of 8 so that eight loads per operand are in flight per
+// lane.
 template <typename T, int N>
 __device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const float* rl,
-                          float inv_sqrt_d, int lane, float* key, float* val) {
+                          float inv_sqrt_d, int lane, float* key, float* val, int64_t ks = 0) {
+  if (ks == 0) ks = d;
   float m = -INFINITY, l = 0.f;
   float ak[N], av[N];
 #pragma unroll
@@ -65,7 +67,7 @@ __device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const fl
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (i0 + u < n) {
-        RowIO<T, N>::load(kbase + int64_t(i0 + u) * d, lane, kx[u]);
+        RowIO<T, N>::load(kbase + int64_t(i0 + u) * ks, lane, kx[u]);
         RowIO<T, N>::load(vbase + int64_t(i0 + u) * d, lane, vx[u]);
       }
     }

@@ -27,7 +27,9 @@ recsa_status check_geometry(const recsa_geometry* g) {
   if (g->window < 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->rope_enabled != 0 && g->rope_enabled != 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->rope_enabled && !(g->rope_base > 1.0f)) return RECSA_ERR_INVALID_GEOMETRY;
-  if (g->batch < 1 || g->capacity < 1 || g->reserved != 0) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->batch < 1 || g->capacity < 1) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->n_ref < 0 || g->n_ref > 64) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->n_ref > 1 && g->mode != RECSA_MODE_ZHA) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA && g->mode != RECSA_MODE_GROUP)
     return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode == RECSA_MODE_ZHA && !(g->top_p > 0.f && g->top_p <= 1.f))
@@ -68,9 +70,9 @@ recsa_status make_layout(const recsa_geometry* g, TreeLayout* lay) {
   lay->rope_off = off;
   off = align_up(off + rows * (g->head_dim / 2) * 8, 256);
   for (int l = 0; l < D; ++l) {
-    int64_t bytes = int64_t(g->batch) * g->n_kv_heads * lay->nodes[l] * g->head_dim * 4;
+    const int64_t bytes = int64_t(g->batch) * g->n_kv_heads * lay->nodes[l] * g->head_dim * 4;
     lay->key_off[l] = off;
-    off = align_up(off + bytes, 256);
+    off = align_up(off + bytes * std::max(g->n_ref, 1), 256);
     lay->val_off[l] = off;
     off = align_up(off + bytes, 256);
   }
@@ -96,6 +98,7 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->rope = g->rope_enabled;
   p->mode = g->mode;
   p->top_p = g->top_p;
+  p->nref = std::max(g->n_ref, 1);
   p->batch = g->batch;
   p->cap = g->capacity;
   p->Bsh = p->bsh = -1;

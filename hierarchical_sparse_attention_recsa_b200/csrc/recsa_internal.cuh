@@ -22,8 +22,8 @@ struct TreeLayout {
   int32_t levels;                 // summary levels at capacity (D)
   int32_t rope_rows;              // rows of the RoPE table
   int64_t nodes[kMaxLevels];      // nodes per (sequence, KV head) at level l+1
-  int64_t key_off[kMaxLevels];    // fp32 keys  [batch][Hkv][nodes][d]
-  int64_t val_off[kMaxLevels];    // fp32 values, same shape
+  int64_t key_off[kMaxLevels];    // fp32 keys  [batch][Hkv][nodes][nref][d]
+  int64_t val_off[kMaxLevels];    // fp32 values [batch][Hkv][nodes][d]
   int64_t rope_off;               // float2 (cos, sin) [rope_rows][d/2]
   int64_t total;
 };
@@ -34,6 +34,7 @@ struct Params {
   int32_t Bsh, bsh;   // log2 of B and b when powers of two, else -1
   int32_t mode;       // RECSA_MODE_RECSA or RECSA_MODE_ZHA
   float top_p;        // ZHA routing mass
+  int32_t nref;       // reference queries per pooler (keys per node), >= 1
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;
@@ -53,7 +54,7 @@ __device__ __forceinline__ unsigned int* tree_error_word(void* tree) {
 __device__ __forceinline__ float* level_keys(const Params& p, void* tree, int lev /*1-based*/,
                                              int64_t seq, int g) {
   char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
-  return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.d;
+  return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.d;
 }
 __device__ __forceinline__ float* level_vals(const Params& p, void* tree, int lev, int64_t seq,
                                              int g) {

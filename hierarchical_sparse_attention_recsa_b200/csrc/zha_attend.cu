@@ -27,6 +27,8 @@
 //     for fp32) into registers, still packed, before it uses any of them.
 //   * Each warp keeps an online softmax (max, sum, its lanes' channels of the
 //     accumulator); the 16 states are merged through shared memory.
+#include <algorithm>
+
 #include "recsa_internal.cuh"
 
 namespace recsa {
@@ -36,6 +38,7 @@ constexpr int kZThreads = 512;
 constexpr int kZWarps = kZThreads / 32;
 constexpr int kZChain = 8;          // chain warps; the others attend the window first
 constexpr int kZMaxCand = kZChain * 32;   // one chain thread per candidate
+constexpr int kZMaxRows = 256;            // level key rows staged at once
 constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
 constexpr int kZBarChain = 1;       // named barrier of the chain warps
 
@@ -126,7 +129,8 @@ __global__ void __launch_bounds__(kZThreads, 1)
 zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                   const T* __restrict__ V, const void* __restrict__ tree,
                   const int64_t* __restrict__ len_dev, int64_t q_start, int n_q, int decode,
-                  T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax) {
+                  T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
+                  int krows) {
   constexpr int D = 64 * NP, HALF = 32 * NP;
   constexpr int RS = D + 2;                      // warp state row: acc[D], m, l
   const int qi = blockIdx.x;
@@ -136,8 +140,9 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   extern __shared__ __align__(16) unsigned char smem[];
-  float* kbuf = reinterpret_cast<float*>(smem);               // [cmax][D] level keys
-  float* score = kbuf + size_t(cmax) * D;                     // [cmax]
+  float* kbuf = reinterpret_cast<float*>(smem);               // [krows][D] level key rows
+  float* rowsc = kbuf + size_t(krows) * D;                    // [krows] row scores (R > 1)
+  float* score = rowsc + krows;                               // [cmax]
   float* wsort = score + cmax;                                // [cmax] weights by rank
   float* zsum = wsort + cmax;                                 // [kZChain] sums, [kZChain] max
   float* wst = zsum + kZChain + 1;                            // [kZWarps][RS] warp states
@@ -276,38 +281,59 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         return i < nch ? kprev[div_b(p, i)] * p.b + mod_b(p, i) : int(p.b * vup) + (i - nch);
       };
       const float* keys = level_keys(p, const_cast<void*>(tree), lev, seq, g);
+      // A node holds R = nref keys (one per reference query) and scores its
+      // best match.  The level's rows (candidate, reference) go through kbuf
+      // in chunks of krows / R candidates; with R = 1 that is one chunk.
+      const int R = p.nref;
+      const int cc = krows / R;
       constexpr int C16 = D / 4;                 // 16-byte pieces per fp32 row
-      for (int x = ct; x < c * C16; x += kZChain * 32) {
-        const int i = x / C16, pc = x % C16;
-        cp_async16(kbuf + size_t(i) * D + pc * 4, keys + int64_t(node(i)) * D + pc * 4);
-      }
-      cp_async_wait_all();
-      chain_sync();
-      // scores: rows warp, warp + 8, ...; four rows per warp at a time
-      for (int i0 = warp; i0 < c; i0 += 4 * kZChain) {
-        float sc4[4];
+      for (int i0c = 0; i0c < c; i0c += cc) {
+        const int i1c = min(c, i0c + cc);
+        const int nrow = (i1c - i0c) * R;
+        for (int x = ct; x < nrow * C16; x += kZChain * 32) {
+          const int q = x / C16, pc = x % C16;
+          const int i = i0c + q / R, ref = q % R;
+          cp_async16(kbuf + size_t(q) * D + pc * 4,
+                     keys + (int64_t(node(i)) * R + ref) * D + pc * 4);
+        }
+        cp_async_wait_all();
+        chain_sync();
+        float* rsc = R == 1 ? score + i0c : rowsc;   // row scores
+        // rows warp, warp + 8, ...; four rows per warp at a time
+        for (int q0 = warp; q0 < nrow; q0 += 4 * kZChain) {
+          float sc4[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int i = min(i0 + r * kZChain, c - 1);   // rows past c repeat the last
-          float x1[NP], x2[NP];
-          load_pairs<NP>(kbuf + size_t(i) * D, lane, x1, x2);
-          sc4[r] = 0.f;
+          for (int r = 0; r < 4; ++r) {
+            const int q = min(q0 + r * kZChain, nrow - 1);   // rows past nrow repeat the last
+            float x1[NP], x2[NP];
+            load_pairs<NP>(kbuf + size_t(q) * D, lane, x1, x2);
+            sc4[r] = 0.f;
 #pragma unroll
-          for (int u = 0; u < NP; ++u) {
-            sc4[r] = fmaf(q1[u], x1[u], sc4[r]);
-            sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
+            for (int u = 0; u < NP; ++u) {
+              sc4[r] = fmaf(q1[u], x1[u], sc4[r]);
+              sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) sc4[r] += __shfl_xor_sync(0xffffffffu, sc4[r], o);
+          if (lane < 4) {
+            float v = sc4[0];
+#pragma unroll
+            for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
+            const int q = q0 + lane * kZChain;
+            if (q < nrow) rsc[q] = v * p.inv_sqrt_d;
           }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) sc4[r] += __shfl_xor_sync(0xffffffffu, sc4[r], o);
-        if (lane < 4) {
-          float v = sc4[0];
-#pragma unroll
-          for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
-          const int i = i0 + lane * kZChain;
-          if (i < c) score[i] = v * p.inv_sqrt_d;
+        chain_sync();
+        if (R > 1) {   // a candidate's score: the best of its R rows
+          for (int i = i0c + ct; i < i1c; i += kZChain * 32) {
+            float m = rsc[(i - i0c) * R];
+            for (int ref = 1; ref < R; ++ref) m = fmaxf(m, rsc[(i - i0c) * R + ref]);
+            score[i] = m;
+          }
+          chain_sync();
         }
       }
       chain_sync();
@@ -457,7 +483,11 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   const int cmax = int(cm < 1 ? 1 : cm);
   if (cmax > kZMaxCand) return cudaErrorNotSupported;   // the generic kernel serves it
   const int kmax = int(kk < cmax ? kk : cmax);
-  const size_t bytes = (size_t(cmax) * D + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
+  // level key rows staged per chunk: the whole level at one reference
+  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, kZMaxRows));
+  if (krows < p.nref) return cudaErrorNotSupported;
+  const size_t bytes = (size_t(krows) * (D + 1) + 2 * size_t(cmax) + kZChain + 1 +
+                        kZWarps * (D + 2)) * 4 +
                        (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + kZChain) * 4;
   if (bytes > 227 * 1024) return cudaErrorNotSupported;
   if (p.batch > 65535) return cudaErrorNotSupported;
@@ -469,7 +499,8 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   kern<<<grid, kZThreads, bytes, s>>>(p, reinterpret_cast<const T*>(Q),
                                       reinterpret_cast<const T*>(K),
                                       reinterpret_cast<const T*>(V), tree, len_dev, q_start, n_q,
-                                      decode, reinterpret_cast<T*>(O), trace, cmax, kmax);
+                                      decode, reinterpret_cast<T*>(O), trace, cmax, kmax,
+                                      krows);
   return cudaGetLastError();
 }
 

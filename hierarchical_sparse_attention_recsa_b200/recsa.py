@@ -68,7 +68,7 @@ class CGeometry(ctypes.Structure):
         ("mode", ctypes.c_int32),
         ("capacity", ctypes.c_int64),
         ("top_p", ctypes.c_float),
-        ("reserved", ctypes.c_int32),
+        ("n_ref", ctypes.c_int32),
     ]
 
 
@@ -90,12 +90,13 @@ class Geometry:
     rope_base: float = 1e6
     mode: int = 0          # MODE_RECSA, MODE_ZHA or MODE_GROUP
     top_p: float = 0.0     # ZHA routing mass
+    n_ref: int = 1         # reference queries per pooler (ZHA mode for n_ref > 1)
 
     def c(self) -> CGeometry:
         return CGeometry(self.dtype, self.head_dim, self.n_q_heads, self.n_kv_heads,
                          self.leaf_block, self.branching, self.k, self.window,
                          self.rope_enabled, self.rope_base, self.batch, self.mode,
-                         self.capacity, self.top_p, 0)
+                         self.capacity, self.top_p, self.n_ref)
 
     @property
     def torch_dtype(self) -> torch.dtype:

@@ -19,8 +19,9 @@
  *       K, V          [batch][n_kv_heads][capacity][head_dim]   (dtype)
  *       Q, O          [batch][n_q][n_q_heads][head_dim]         (dtype)
  *       k_new, v_new  [batch][n_kv_heads][head_dim]             (dtype)
- *       pooler_r      [n_kv_heads][head_dim] fp32 with a head stride in
- *                     elements (0 = one vector shared by every KV head)
+ *       pooler_r      [n_kv_heads][n_ref][head_dim] fp32 with a head stride
+ *                     in elements (0 = one set shared by every KV head);
+ *                     n_ref = 1 unless the geometry sets n_ref > 1
  *       len           int64 [batch]: tokens currently in each sequence
  *     Query head h reads KV head h / (n_q_heads / n_kv_heads).
  *   - Work is enqueued on `stream` (a cudaStream_t, 0 = legacy default) and
@@ -99,6 +100,9 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   probability among the level's candidates, the top min(k, c) group scores
  *   are kept (ties -> lower index) for all G heads, and each head then
  *   attends as in RecSA.
+ *   n_ref: with R = n_ref > 1 (ZHA mode only) every node holds R keys, one per
+ *   reference query of the pooler, and a node's routing score is the largest
+ *   of its R scores q . key_j / sqrt(d).
  */
 typedef struct recsa_geometry {
   int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
@@ -115,7 +119,7 @@ typedef struct recsa_geometry {
   int32_t mode;         /* RECSA_MODE_RECSA (0), RECSA_MODE_ZHA (1), RECSA_MODE_GROUP (2) */
   int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
   float top_p;          /* ZHA: routing mass in (0, 1]; ignored in RECSA mode */
-  int32_t reserved;     /* must be 0 */
+  int32_t n_ref;        /* reference queries per pooler: 0 or 1 = one; 2..64 (ZHA mode only) */
 } recsa_geometry;
 
 /* Human-readable name of a status code (static string). */
@@ -130,8 +134,9 @@ recsa_status recsa_num_levels(const recsa_geometry* geom, int64_t length, int32_
 /*
  * Bytes of the tree buffer for `geom` at its capacity: a 256-byte header
  * (device error flags), the RoPE cos/sin table of the indices a traversal can
- * reach, and per level l: keys and values [batch][n_kv_heads][n_l][head_dim]
- * in fp32, n_l the level's node count at capacity.
+ * reach, and per level l: keys [batch][n_kv_heads][n_l][n_ref][head_dim] and
+ * values [batch][n_kv_heads][n_l][head_dim] in fp32, n_l the level's node
+ * count at capacity.
  */
 recsa_status recsa_tree_bytes(const recsa_geometry* geom, size_t* bytes);
 
@@ -142,7 +147,10 @@ recsa_status recsa_tree_bytes(const recsa_geometry* geom, size_t* bytes);
  * consecutive level-(l-1) summary keys ("Subquadratic Attention with a
  * Hierarchical Tree-Structured Indexer", Figure 3).  Pooling: weights =
  * softmax_i(r . k_i / sqrt(d)), key = sum_i weight_i k_i; value = mean of the
- * children's values.  Also clears the error flags and writes the RoPE table.
+ * children's values.  With n_ref > 1 reference queries r_1..r_R the keys of
+ * each are built in parallel (ZHA, Figure 3 caption): reference j's parent
+ * key pools reference j's child keys.  Also clears the error flags and writes
+ * the RoPE table.
  *   len_host: HOST int64 [batch], each in [0, capacity].
  */
 recsa_status recsa_build(const recsa_geometry* geom, const void* K, const void* V,

@@ -51,7 +51,8 @@ def alloc_tree(g: R.Geometry) -> torch.Tensor:
 
 
 def read_tree_level(g: R.Geometry, tree: torch.Tensor, lev: int):
-    """(keys, vals) [batch, Hkv, n_l, d] fp32 views of one level of the tree buffer."""
+    """(keys, vals) fp32 views of one level of the tree buffer: keys [batch, Hkv,
+    n_l, d] ([batch, Hkv, n_l, n_ref, d] with n_ref > 1), vals [batch, Hkv, n_l, d]."""
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
     kk = min(g.k, g.capacity)
     rows = min(max(g.branching * kk + g.branching, g.leaf_block * kk + g.window + g.leaf_block),
@@ -60,15 +61,18 @@ def read_tree_level(g: R.Geometry, tree: torch.Tensor, lev: int):
         rows = max(rows, g.capacity + 1)
     off = up(256 + rows * (g.head_dim // 2) * 8)
     span = g.leaf_block
+    nr = max(g.n_ref, 1)
     for l in range(1, lev + 1):
         n = g.capacity // span
         nbytes = g.batch * g.n_kv_heads * n * g.head_dim * 4
+        kbytes = nbytes * nr
         if l == lev:
             shape = (g.batch, g.n_kv_heads, n, g.head_dim)
-            keys = tree[off:off + nbytes].view(torch.float32).view(shape)
-            vals = tree[up(off + nbytes):up(off + nbytes) + nbytes].view(torch.float32).view(shape)
+            kshape = shape if nr == 1 else (g.batch, g.n_kv_heads, n, nr, g.head_dim)
+            keys = tree[off:off + kbytes].view(torch.float32).view(kshape)
+            vals = tree[up(off + kbytes):up(off + kbytes) + nbytes].view(torch.float32).view(shape)
             return keys, vals
-        off = up(up(off + nbytes) + nbytes)
+        off = up(up(off + kbytes) + nbytes)
         span *= g.branching
     raise ValueError(lev)
 

@@ -20,7 +20,7 @@ from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
 from hierarchical_sparse_attention_recsa_b200 import recsa as R
 
 from recsa_testlib import (Stats, alloc_tree, check_query_zha, geometry, oracle_geometry,
-                           parse_trace, to_np)
+                           parse_trace, read_tree_level, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -268,3 +268,205 @@ def test_zha_decode_step_equals_append_then_decode(zha_impl):
     st.check(torch.bfloat16, f"zha {zha_impl} decode step")
     assert torch.equal(Ka, Kb) and torch.equal(Va, Vb)
     assert torch.equal(tree_a[256:], tree_b[256:])
+
+
+# ---------------------------------------------------------------------------
+# Several reference queries per pooler (n_ref > 1)
+# ---------------------------------------------------------------------------
+
+def _refs(r, n_ref, seed):
+    """n_ref reference queries: the workload's r, then n_ref - 1 more from the
+    same distribution (N(0, 1/d)), seeded."""
+    gen = torch.Generator().manual_seed(seed)
+    d = r.shape[-1]
+    extra = torch.randn((n_ref - 1, d), generator=gen, dtype=torch.float64) / d ** 0.5
+    return torch.cat([r.double().reshape(1, d), extra]).float().contiguous()
+
+
+def _setup_multi(w, lens, capacity, top_p, n_ref, seed, k=None, rope=1):
+    batch = len(lens)
+    g = geometry(w, capacity, batch, k=k, rope=rope, top_p=top_p)
+    g.n_ref = n_ref
+    K, V, r = synth.make_kv(w, capacity, seed=seed, device="cpu", batch=batch)
+    Rq = _refs(r, n_ref, seed + 1000)
+    Kd, Vd, Rd = K.cuda(), V.cuda(), Rq.cuda()
+    tree = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, lens, Rd, 0, tree)
+    torch.cuda.synchronize()
+    return g, K, V, Rq, Kd, Vd, Rd, tree
+
+
+def _multi_trees(g, K, V, Rq, lens):
+    out = {}
+    for s, L in enumerate(lens):
+        for h in range(g.n_kv_heads):
+            Kh, Vh = to_np(K[s, h, :L]), to_np(V[s, h, :L])
+            out[(s, h)] = (Kh, Vh, oracle.MultiTree(oracle.build_tree_multi(
+                Kh, Vh, Rq.double().numpy(), g.leaf_block, g.branching)))
+    return out
+
+
+def test_zha_multiref_tree_matches_oracle():
+    L, Rn = TINY.length, 4
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(TINY, [L], L, 0.7, Rn, seed=50)
+    trees = _multi_trees(g, K, V, Rq, [L])
+    _, _, src = trees[(0, 0)]
+    st = Stats()
+    for lev, (kk, vv) in enumerate(src.levels, start=1):
+        gk, gv = read_tree_level(g, tree, lev)
+        n = kk.shape[0]
+        assert gk.shape[3] == Rn
+        st.add(to_np(gk[0, 0, :n]), kk)
+        st.add(to_np(gv[0, 0, :n]), vv)
+    st.check(torch.float32, "zha multiref tree")
+
+
+@pytest.mark.parametrize("Rn,top_p", [(4, 0.7), (16, 0.9)])
+def test_zha_multiref_decode_tiny(Rn, top_p, zha_impl):
+    L, nq = TINY.length, 64
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(TINY, [L], L, top_p, Rn, seed=52, k=ZK)
+    trees = _multi_trees(g, K, V, Rq, [L])
+    pos = torch.full((1, nq), L - 1, dtype=torch.int64)
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=53, n_needles=8)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for i in range(nq):
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh, Vh, src,
+                            og, top_p, g.k)
+    st.check(torch.float32, f"zha {zha_impl} multiref R={Rn} decode tiny")
+    assert st.clear > 0.6 * nq * g.n_q_heads
+
+
+def test_zha_multiref_prefill_tiny(zha_impl):
+    L, top_p, Rn = TINY.length, 0.8, 3
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(TINY, [L], L, top_p, Rn, seed=54, k=ZK)
+    trees = _multi_trees(g, K, V, Rq, [L])
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=55)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, L, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    rng = np.random.default_rng(7)
+    sample = sorted(set([0, 15, 16, 64, 65, 200, L - 1] + list(rng.integers(0, L, 25))))
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for t in sample:
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, t, h], tr[0, t, h], to_np(Q[0, t, h]), t, Kh, Vh, src, og,
+                            top_p, g.k)
+    st.check(torch.float32, f"zha {zha_impl} multiref prefill tiny")
+
+
+def test_zha_multiref_decode_model_small(zha_impl):
+    lens, top_p, Rn = [20000, 13001], 0.9, 3
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(MODEL, lens, 20480, top_p, Rn, seed=56)
+    trees = _multi_trees(g, K, V, Rq, lens)
+    nq = 2
+    pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(MODEL, K, pos, seed=57, n_needles=2)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for i in range(nq):
+            for h in range(g.n_q_heads):
+                Kh, Vh, src = trees[(s, h // G)]
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} multiref decode model small")
+
+
+def test_zha_multiref_append_matches_build(zha_impl):
+    """Appending tokens one by one (leaf and level-2 completions) gives the
+    tree a fresh build gives, for every reference query, and the decode after
+    the last append matches the oracle."""
+    w, top_p, Rn = MODEL, 0.9, 2
+    lens0 = [4000, 4031]
+    steps = 100
+    cap = 4096 + 256
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(w, lens0, cap, top_p, Rn, seed=58)
+    Kw, Vw = Kd.clone(), Vd.clone()
+    Kw[0, :, 4000:] = 0
+    Vw[0, :, 4000:] = 0
+    Kw[1, :, 4031:] = 0
+    Vw[1, :, 4031:] = 0
+    lens_d = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        R.recsa_append(g, Kw, Vw, kn, vn, lens_d, Rd, 0, tree)
+    new_lens = [L + steps for L in lens0]
+    fresh = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, new_lens, Rd, 0, fresh)
+    torch.cuda.synchronize()
+    for lev in range(1, R.recsa_num_levels(g, max(new_lens)) + 1):
+        a_k, a_v = read_tree_level(g, tree, lev)
+        b_k, b_v = read_tree_level(g, fresh, lev)
+        for s in range(2):
+            n = new_lens[s] // (g.leaf_block * g.branching ** (lev - 1))
+            torch.testing.assert_close(a_k[s, :, :n], b_k[s, :, :n], rtol=0, atol=1e-6)
+            torch.testing.assert_close(a_v[s, :, :n], b_v[s, :, :n], rtol=0, atol=1e-6)
+    pos = torch.tensor([[L - 1] for L in new_lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(w, K, pos, seed=59)
+    O = torch.empty_like(Q).cuda()
+    trace = torch.zeros((2, 1, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    R.recsa_decode(g, Q.cuda(), Kw, Vw, tree, lens_d, 1, O, trace)
+    torch.cuda.synchronize()
+    trees = _multi_trees(g, K, V, Rq, new_lens)
+    og = oracle_geometry(g)
+    G = g.n_q_heads // g.n_kv_heads
+    tr = trace.cpu().numpy()
+    st = Stats()
+    for s in range(2):
+        for h in range(0, g.n_q_heads, 5):
+            Kh, Vh, src = trees[(s, h // G)]
+            check_query_zha(st, to_np(O[s, 0, h]), tr[s, 0, h], to_np(Q[s, 0, h]),
+                            new_lens[s] - 1, Kh, Vh, src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} multiref after append")
+
+
+@pytest.mark.parametrize("rope", [1, 0])
+def test_zha_multiref_full_mass_is_dense(rope, zha_impl):
+    w = TINY
+    L = 1500
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(w, [L], L, 1.0, 3, seed=60, k=R.KEEP_ALL,
+                                                 rope=rope)
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(w, K, pos, seed=61)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O)
+    torch.cuda.synchronize()
+    O_ = to_np(O)
+    st = Stats()
+    for t in [0, 63, 64, 700, L - 1]:
+        for h in range(g.n_q_heads):
+            ref = oracle.dense_causal_attention(to_np(Q[0, t, h]), t, to_np(K[0, 0]),
+                                                to_np(V[0, 0]), rope=bool(rope),
+                                                rope_base=w.rope_base)
+            st.add(O_[0, t, h], ref)
+    st.check(torch.float32, f"zha {zha_impl} multiref full mass")
