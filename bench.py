@@ -353,6 +353,9 @@ def run_recsa(args, rank, world, dev):
     if not args.no_zha:
         out["zha"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
                                  peak_kind, R.MODE_ZHA, cpu_leg)
+        out["zha_multiref"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
+                                          hbm_gbs, peak_kind, R.MODE_ZHA, cpu_leg,
+                                          n_ref=ZHA_N_REF)
     if not args.no_group:
         out["group"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
                                    peak_kind, R.MODE_GROUP, cpu_leg)
@@ -360,14 +363,26 @@ def run_recsa(args, rank, world, dev):
 
 
 ZHA_TOP_P = 0.9
+ZHA_N_REF = 16     # reference queries per pooler in the pages' trained routers
 
 
-def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, mode, cpu):
+def reference_queries(r, n_ref, seed=7):
+    """n_ref reference queries: r, then n_ref - 1 more from its distribution
+    (N(0, 1/d)), seeded; [n_ref, d] fp32 on r's device."""
+    gen = torch.Generator().manual_seed(seed)
+    d = r.shape[-1]
+    extra = torch.randn((n_ref - 1, d), generator=gen) / d ** 0.5
+    return torch.cat([r.reshape(1, d).float().cpu(), extra]).contiguous().to(r.device)
+
+
+def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, mode, cpu,
+                n_ref=1):
     """A selection variant on the same cache: its own tree (same pooling),
     then the batch's decode queries at t = L - 1, timed per launch like the
     main decode.  MODE_ZHA: top-p expansion, exact tokens of the reached
     leaves and the window at true positions (the RoPE table covers every
-    position).  MODE_GROUP: RecSA with one selection per KV group."""
+    position), with n_ref reference queries per pooler.  MODE_GROUP: RecSA
+    with one selection per KV group."""
     batch = Kc.shape[0]
     zha = mode == R.MODE_ZHA
     g = R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
@@ -375,9 +390,10 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
                    batch=batch, capacity=cap,
                    dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
                    rope_enabled=1, rope_base=w.rope_base, mode=mode,
-                   top_p=ZHA_TOP_P if zha else 0.0)
+                   top_p=ZHA_TOP_P if zha else 0.0, n_ref=n_ref)
     tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
-    R.recsa_build(g, Kc, Vc, [L] * batch, r, 0, tree)
+    refs = reference_queries(r, n_ref) if n_ref > 1 else r
+    R.recsa_build(g, Kc, Vc, [L] * batch, refs, 0, tree)
     lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
     O = torch.empty_like(Qs[0])
     n = min(args.steps, Qs.shape[0])
@@ -399,7 +415,8 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     G = w.n_q_heads // w.n_kv_heads
     nb = [counts.decode_bytes_from_trace(tr[i], np.full(batch, L), w.leaf_block, w.branching,
                                          w.window, G, w.head_dim, elem_bytes(w), w.k,
-                                         summary_values=not zha)["bytes"] for i in range(n)]
+                                         summary_values=not zha,
+                                         keys_per_node=n_ref)["bytes"] for i in range(n)]
     kept = tr[..., 4 + 16:4 + 16 + R.recsa_num_levels(g, L)].astype(np.float64)
     nbytes = float(np.mean(nb))
     achieved = nbytes / (dec_ms / 1e3) / 1e9
@@ -413,11 +430,13 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
                         "bytes_per_launch": nbytes, "traffic": None}}
     if zha:
         res["top_p"] = ZHA_TOP_P
+        res["n_ref"] = n_ref
     del tree, traces
     torch.cuda.empty_cache()
     if cpu:
+        variant = ("zha" if n_ref == 1 else "zha_multiref") if zha else "group"
         res["cpu_baseline"] = cpu_baseline(args.workload, seconds=min(args.cpu_seconds, 10.0),
-                                           variant="zha" if zha else "group")
+                                           variant=variant)
     return res
 
 
@@ -561,6 +580,9 @@ class OracleDecode:
                                    rope=True, rope_base=w.rope_base)
         self.tree = oracle.LazyTree(self.K, self.V, r.double().numpy(), w.leaf_block,
                                     w.branching)
+        self.multi = oracle.LazyMultiTree(self.K, self.V,
+                                          reference_queries(r, ZHA_N_REF).double().numpy(),
+                                          w.leaf_block, w.branching)
         self.i = 0
         self.heads_per_query = w.n_q_heads
         # untimed: pool the nodes the first query visits (the oracle's tree build)
@@ -584,7 +606,8 @@ class OracleDecode:
                 self.oracle.traverse_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
                                                 self.geo)
             else:
-                self.oracle.zha_route_and_attend(self.Q[i, h], t, self.K, self.V, self.tree,
+                src = self.multi if variant == "zha_multiref" else self.tree
+                self.oracle.zha_route_and_attend(self.Q[i, h], t, self.K, self.V, src,
                                                  self.geo, ZHA_TOP_P)
             done += 1
             if h == self.G - 1:
@@ -612,6 +635,7 @@ def cpu_baseline(workload=WORKLOAD, seconds=15.0, variant=None):
     dt = time.perf_counter() - t0
     del lim
     what = {None: "decode", "zha": f"ZHA decode (top-p {ZHA_TOP_P})",
+            "zha_multiref": f"ZHA decode (top-p {ZHA_TOP_P}, {ZHA_N_REF} reference queries)",
             "group": "group-selection decode"}[variant]
     return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
             "kind": "oracle",

@@ -45,4 +45,4 @@ from .recsa import (  # noqa: F401
 from .dense import dense_causal_attention  # noqa: F401
 from .zha import top_p_prefix, zha_route_and_attend  # noqa: F401
 from .group import group_select, group_traverse_and_attend  # noqa: F401
-from .multiref import MultiTree, build_tree_multi  # noqa: F401
+from .multiref import LazyMultiTree, MultiTree, build_tree_multi  # noqa: F401

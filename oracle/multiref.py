@@ -31,7 +31,7 @@ from typing import List, Tuple
 
 import numpy as np
 
-from .recsa import build_tree
+from .recsa import LazyTree, build_tree
 
 
 def build_tree_multi(K: np.ndarray, V: np.ndarray, Rq: np.ndarray, B: int, b: int
@@ -57,3 +57,18 @@ class MultiTree:
 
     def val(self, level: int, j: int) -> np.ndarray:
         return self.levels[level - 1][1][j]
+
+
+class LazyMultiTree:
+    """On-demand counterpart of MultiTree for long caches: one LazyTree per
+    reference query (the R key trees are independent), values from the first."""
+
+    def __init__(self, K, V, Rq, B: int, b: int):
+        Rq = np.atleast_2d(np.asarray(Rq, dtype=np.float64))
+        self.trees = [LazyTree(K, V, Rq[j], B, b) for j in range(Rq.shape[0])]
+
+    def key(self, level: int, j: int) -> np.ndarray:
+        return np.stack([t.key(level, j) for t in self.trees])
+
+    def val(self, level: int, j: int) -> np.ndarray:
+        return self.trees[0].val(level, j)

@@ -658,3 +658,16 @@ def test_multiref_full_mass_is_dense(rope):
         else:
             qr, Kr = q, K[: t + 1]
         np.testing.assert_allclose(res["out"], _sdpa(qr, Kr, V[: t + 1]), atol=1e-12)
+
+
+def test_lazy_multiref_tree_equals_full_build():
+    rng = np.random.default_rng(34)
+    B, b, d, T = 4, 3, 8, 150
+    K, V = _rand_kv(rng, T, d)
+    Rq = rng.standard_normal((3, d))
+    full = oracle.MultiTree(oracle.build_tree_multi(K, V, Rq, B, b))
+    lazy = oracle.LazyMultiTree(K, V, Rq, B, b)
+    for lev in range(1, len(full.levels) + 1):
+        for n in range(full.levels[lev - 1][0].shape[0]):
+            np.testing.assert_allclose(lazy.key(lev, n), full.key(lev, n), atol=1e-13)
+            np.testing.assert_allclose(lazy.val(lev, n), full.val(lev, n), atol=1e-13)
