@@ -19,7 +19,8 @@ Sources (web pages, cited by title and section):
     Its routing variant (top-p expansion, attention over the reached leaves)
     is in ``zha.py``; its Table IX convention of a selection per KV group is
     applied to RecSA in ``group.py``; several reference queries per pooler
-    (Figure 3 caption) are in ``multiref.py``.
+    (Figure 3 caption) are in ``multiref.py``; low-precision router keys
+    (Figure 16 caption) in ``lowprec.py``.
   * "Efficient Sequence Modeling, Issue 13", highlights and editor's note on
     RecSA (normalisation shared with exact tokens; one pooler for selection and
     summary keys).
@@ -46,3 +47,5 @@ from .dense import dense_causal_attention  # noqa: F401
 from .zha import top_p_prefix, zha_route_and_attend  # noqa: F401
 from .group import group_select, group_traverse_and_attend  # noqa: F401
 from .multiref import LazyMultiTree, MultiTree, build_tree_multi  # noqa: F401
+from .lowprec import (build_tree_fp8, build_tree_fp8_multi, dequantize_row,  # noqa: F401
+                      e4m3_decode, e4m3_round, near_rounding_boundary, quantize_row)

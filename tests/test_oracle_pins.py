@@ -671,3 +671,72 @@ def test_lazy_multiref_tree_equals_full_build():
         for n in range(full.levels[lev - 1][0].shape[0]):
             np.testing.assert_allclose(lazy.key(lev, n), full.key(lev, n), atol=1e-13)
             np.testing.assert_allclose(lazy.val(lev, n), full.val(lev, n), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Low-precision router keys (FP8 E4M3, one scale per row)
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_the_format_table():
+    """All 256 codes: sign, exponent field 0 (subnormal: m/8 * 2^-6) or 1..15
+    (normal: (1 + m/8) * 2^(e-7)), NaN only at S.1111.111; spot values."""
+    vals = [oracle.e4m3_decode(c) for c in range(256)]
+    nan = [c for c in range(256) if math.isnan(vals[c])]
+    assert nan == [0x7F, 0xFF]
+    finite = sorted(set(v for v in vals if not math.isnan(v)))
+    assert len(finite) == 253                        # +-0 coincide
+    assert max(finite) == 448.0 and min(finite) == -448.0
+    assert oracle.e4m3_decode(0x01) == 2.0 ** -9     # smallest subnormal
+    assert oracle.e4m3_decode(0x08) == 2.0 ** -6     # smallest normal
+    assert oracle.e4m3_decode(0x38) == 1.0
+    assert oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_decode(0xC0) == -2.0
+
+
+def test_e4m3_round_fixed_points_ties_and_saturation():
+    vals = np.array([v for v in (oracle.e4m3_decode(c) for c in range(256))
+                     if not math.isnan(v)])
+    np.testing.assert_array_equal(oracle.e4m3_round(vals), vals)
+    pos = np.array(sorted(set(vals[vals >= 0])))
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = oracle.e4m3_round(mids)
+    for m, lo, hi, g in zip(mids, pos[:-1], pos[1:], got):
+        # ties to the neighbour whose mantissa is even
+        even = lo if (int(np.round(lo / _quantum(lo))) % 2 == 0) else hi
+        assert g == even, (m, lo, hi, g)
+    assert oracle.e4m3_round(np.array([463.9, 464.0, 1e6, -1e6])).tolist() == [448, 448, 448, -448]
+
+
+def _quantum(v):
+    _, e = np.frexp(v)
+    return 2.0 ** (max(e - 1, -6) - 3)
+
+
+def test_e4m3_round_agrees_with_torch_inside_the_range():
+    rng = np.random.default_rng(40)
+    x = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1, 30, 200)])
+    x = x[np.abs(x) < 440]
+    ref = torch.tensor(x, dtype=torch.float64).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_round(x), ref)
+
+
+def test_fp8_tree_keys_are_quantized_pools_of_quantized_children():
+    rng = np.random.default_rng(41)
+    B, b, d, T = 4, 3, 8, 120
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    levels = oracle.build_tree_fp8(K, V, r, B, b)
+    for lev, (keys, vals) in enumerate(levels, start=1):
+        fan = B if lev == 1 else b
+        src = K if lev == 1 else levels[lev - 2][0]
+        for j in range(keys.shape[0]):
+            pooled = oracle.pool_keys(src[j * fan:(j + 1) * fan], r)
+            amax = np.abs(pooled).max()
+            # each stored element is within half a quantum of the float value
+            q = 2.0 ** (np.maximum(np.frexp(np.abs(pooled) / (amax / 448))[1] - 1, -6) - 3)
+            assert np.all(np.abs(keys[j] - pooled) <= 0.5 * q * (amax / 448) * (1 + 1e-12))
+            # and is an E4M3 value times the row scale
+            unit = keys[j] / (amax / 448)
+            np.testing.assert_allclose(oracle.e4m3_round(unit), unit, rtol=1e-14)
+            np.testing.assert_allclose(vals[j], (V if lev == 1 else levels[lev - 2][1])
+                                       [j * fan:(j + 1) * fan].mean(0), atol=1e-14)
