@@ -31,6 +31,10 @@ template <>
 __device__ __forceinline__ float ld<__nv_bfloat16>(const __nv_bfloat16* p, int64_t i) {
   return __bfloat162float(p[i]);
 }
+template <>   // FP8 E4M3 key codes
+__device__ __forceinline__ float ld<unsigned char>(const unsigned char* p, int64_t i) {
+  return fp8_to_float(p[i]);
+}
 
 template <typename T, int P>  // head_dim = 64 * P
 __global__ void __launch_bounds__(kThreads)
@@ -204,9 +208,19 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       const int h = pr / cmx, ii = pr % cmx;
       if (ii >= p.b * zkup[h] + norph) continue;  // warp-uniform
       // a node with several reference keys (ZHA) scores its best match
-      const float* kr = keys + int64_t(cand[h * cmax + ii]) * p.nref * d;
-      float s = dot_row(h, kr, zha ? -1 : ii);
-      for (int ref = 1; ref < p.nref; ++ref) s = fmaxf(s, dot_row(h, kr + ref * d, -1));
+      const int64_t node = cand[h * cmax + ii];
+      float s;
+      if (p.kfmt == RECSA_KEYS_FP8) {   // codes times the row's scale
+        const unsigned char* kc = level_kcodes(p, const_cast<void*>(tree), lev, seq, g) +
+                                  node * p.nref * d;
+        const float* ks = level_kscales(p, const_cast<void*>(tree), lev, seq, g) + node * p.nref;
+        s = dot_row(h, kc, -1) * ks[0];
+        for (int ref = 1; ref < p.nref; ++ref) s = fmaxf(s, dot_row(h, kc + ref * d, -1) * ks[ref]);
+      } else {
+        const float* kr = keys + node * p.nref * d;
+        s = dot_row(h, kr, zha ? -1 : ii);
+        for (int ref = 1; ref < p.nref; ++ref) s = fmaxf(s, dot_row(h, kr + ref * d, -1));
+      }
       if (lane == 0) score[h * cmax + ii] = s;
     }
     __syncthreads();

@@ -18,6 +18,41 @@
 namespace recsa {
 namespace {
 
+// Store the pooled key of node j (level lev, reference ref): fp32 row, or
+// FP8 E4M3 codes with one fp32 scale (low-precision router keys).
+template <int N>
+__device__ void store_node_key(const Params& p, void* tree, int lev, int64_t seq, int g,
+                               int64_t j, int ref, int lane, const float* key) {
+  if (p.kfmt == RECSA_KEYS_FP8)
+    store_key_fp8<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d,
+                     level_kscales(p, tree, lev, seq, g) + j * p.nref + ref, lane, key);
+  else
+    RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d, lane,
+                           key);
+}
+
+// Pool node j of level lev >= 2 for reference ref from its b children's
+// stored keys (decoded when FP8) and values.
+template <int N>
+__device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, int g, int64_t j,
+                            int ref, const float* rl, int lane, float* key, float* val) {
+  const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
+  if (p.kfmt == RECSA_KEYS_FP8) {
+    const unsigned char* cc =
+        level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.d;
+    const float* cs = level_kscales(p, tree, lev - 1, seq, g) + j * p.b * p.nref + ref;
+    pool_children<float, N>(
+        [&](int i, float* x) {
+          load_key_fp8<N>(cc + int64_t(i) * p.nref * p.d, cs[int64_t(i) * p.nref], lane, x);
+        },
+        cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
+  } else {
+    const float* ck = level_keys(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.d;
+    pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val,
+                        int64_t(p.nref) * p.d);
+  }
+}
+
 // Level 1: one warp per leaf block of one (sequence, KV head).
 template <typename T, int N>
 __global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T* V,
@@ -33,7 +68,7 @@ __global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T
     load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
     float key[N], val[N];
     pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-    RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + (j * p.nref + ref) * p.d, lane, key);
+    store_node_key<N>(p, tree, 1, seq, g, j, ref, lane, key);
     if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
   }
 }
@@ -47,17 +82,12 @@ __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, i
   const int64_t j = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int g = blockIdx.y;
   if (j >= n_nodes) return;
-  const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
   for (int ref = 0; ref < p.nref; ++ref) {
     float rl[N];
     load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
-    // reference ref's keys of the b children: row stride nref * d
-    const float* ck = level_keys(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.d;
     float key[N], val[N];
-    pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val,
-                        int64_t(p.nref) * p.d);
-    RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d, lane,
-                           key);
+    pool_parent<N>(p, tree, lev, seq, g, j, ref, rl, lane, key, val);
+    store_node_key<N>(p, tree, lev, seq, g, j, ref, lane, key);
     if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + j * p.d, lane, val);
   }
 }
@@ -95,20 +125,14 @@ __global__ void __launch_bounds__(256) append_kernel(Params p, T* K, T* V, const
         const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
         float key[N], val[N];
         pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-        RowIO<float, N>::store(level_keys(p, tree, 1, seq, g) + (j * p.nref + ref) * p.d, lane,
-                               key);
+        store_node_key<N>(p, tree, 1, seq, g, j, ref, lane, key);
         if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
         int64_t idx = j;
         for (int lev = 2; lev <= p.lay.levels && (idx + 1) % p.b == 0; ++lev) {
           idx = (idx + 1) / p.b - 1;
           __syncwarp();
-          const float* ck =
-              level_keys(p, tree, lev - 1, seq, g) + (idx * p.b * p.nref + ref) * p.d;
-          const float* cv = level_vals(p, tree, lev - 1, seq, g) + idx * p.b * p.d;
-          pool_rows<float, N>(ck, cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val,
-                              int64_t(p.nref) * p.d);
-          RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (idx * p.nref + ref) * p.d,
-                                 lane, key);
+          pool_parent<N>(p, tree, lev, seq, g, idx, ref, rl, lane, key, val);
+          store_node_key<N>(p, tree, lev, seq, g, idx, ref, lane, key);
           if (ref == 0)
             RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + idx * p.d, lane, val);
         }

@@ -49,14 +49,13 @@ struct RowIO<__nv_bfloat16, 2> {
   }
 };
 
-// One warp pools `n` rows (keys at kbase with row stride ks, values at vbase
-// with row stride d) into this lane's N channels of key and value.  Rows are
-// processed in groups of 8 so that eight loads per operand are in flight per
-// lane.
-template <typename T, int N>
-__device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const float* rl,
-                          float inv_sqrt_d, int lane, float* key, float* val, int64_t ks = 0) {
-  if (ks == 0) ks = d;
+// One warp pools `n` children into this lane's N channels of key and value:
+// keyload(i, x) gives child i's key channels, vbase + i * d its value row.
+// Rows are processed in groups of 8 so that eight loads per operand are in
+// flight per lane.
+template <typename T, int N, typename KeyLoad>
+__device__ void pool_children(KeyLoad keyload, const T* vbase, int n, int d, const float* rl,
+                              float inv_sqrt_d, int lane, float* key, float* val) {
   float m = -INFINITY, l = 0.f;
   float ak[N], av[N];
 #pragma unroll
@@ -67,7 +66,7 @@ __device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const fl
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (i0 + u < n) {
-        RowIO<T, N>::load(kbase + int64_t(i0 + u) * ks, lane, kx[u]);
+        keyload(i0 + u, kx[u]);
         RowIO<T, N>::load(vbase + int64_t(i0 + u) * d, lane, vx[u]);
       }
     }
@@ -104,6 +103,46 @@ __device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const fl
     key[c] = ak[c] * il;
     val[c] = av[c] * in;
   }
+}
+
+// pool_children over rows (keys at kbase with row stride ks, default d).
+template <typename T, int N>
+__device__ void pool_rows(const T* kbase, const T* vbase, int n, int d, const float* rl,
+                          float inv_sqrt_d, int lane, float* key, float* val, int64_t ks = 0) {
+  if (ks == 0) ks = d;
+  pool_children<T, N>(
+      [&](int i, float* x) { RowIO<T, N>::load(kbase + int64_t(i) * ks, lane, x); }, vbase, n, d,
+      rl, inv_sqrt_d, lane, key, val);
+}
+
+// Row format of FP8 key storage: a lane's N contiguous channels as N bytes,
+// one fp32 scale = max|key| / 448 per row.
+template <int N>
+__device__ void store_key_fp8(unsigned char* codes, float* scale, int lane, const float* key) {
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < N; ++c) amax = fmaxf(amax, fabsf(key[c]));
+  amax = warp_max(amax);
+  const float sc = amax / 448.f;
+  unsigned int packed = 0;
+#pragma unroll
+  for (int c = 0; c < N; ++c)
+    packed |= unsigned(sc > 0.f ? float_to_fp8(key[c] / sc) : 0) << (8 * c);
+  if constexpr (N == 4)
+    reinterpret_cast<unsigned int*>(codes)[lane] = packed;
+  else
+    reinterpret_cast<unsigned short*>(codes)[lane] = static_cast<unsigned short>(packed);
+  if (lane == 0) *scale = sc;
+}
+template <int N>
+__device__ void load_key_fp8(const unsigned char* codes, float scale, int lane, float* x) {
+  unsigned int packed;
+  if constexpr (N == 4)
+    packed = reinterpret_cast<const unsigned int*>(codes)[lane];
+  else
+    packed = reinterpret_cast<const unsigned short*>(codes)[lane];
+#pragma unroll
+  for (int c = 0; c < N; ++c) x[c] = fp8_to_float((packed >> (8 * c)) & 0xFFu) * scale;
 }
 
 template <int N>

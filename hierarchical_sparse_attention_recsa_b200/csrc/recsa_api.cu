@@ -30,6 +30,11 @@ recsa_status check_geometry(const recsa_geometry* g) {
   if (g->batch < 1 || g->capacity < 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->n_ref < 0 || g->n_ref > 64) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->n_ref > 1 && g->mode != RECSA_MODE_ZHA) return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->key_format != RECSA_KEYS_F32 && g->key_format != RECSA_KEYS_FP8)
+    return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->key_format == RECSA_KEYS_FP8 && g->mode != RECSA_MODE_ZHA)
+    return RECSA_ERR_INVALID_GEOMETRY;
+  if (g->reserved != 0) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA && g->mode != RECSA_MODE_GROUP)
     return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode == RECSA_MODE_ZHA && !(g->top_p > 0.f && g->top_p <= 1.f))
@@ -70,9 +75,17 @@ recsa_status make_layout(const recsa_geometry* g, TreeLayout* lay) {
   lay->rope_off = off;
   off = align_up(off + rows * (g->head_dim / 2) * 8, 256);
   for (int l = 0; l < D; ++l) {
-    const int64_t bytes = int64_t(g->batch) * g->n_kv_heads * lay->nodes[l] * g->head_dim * 4;
+    const int64_t rows = int64_t(g->batch) * g->n_kv_heads * lay->nodes[l];
+    const int64_t bytes = rows * g->head_dim * 4;
+    const int64_t nref = std::max(g->n_ref, 1);
     lay->key_off[l] = off;
-    off = align_up(off + bytes * std::max(g->n_ref, 1), 256);
+    if (g->key_format == RECSA_KEYS_FP8) {   // codes, then one fp32 scale per key row
+      off = align_up(off + rows * nref * g->head_dim, 256);
+      lay->kscale_off[l] = off;
+      off = align_up(off + rows * nref * 4, 256);
+    } else {
+      off = align_up(off + bytes * nref, 256);
+    }
     lay->val_off[l] = off;
     off = align_up(off + bytes, 256);
   }
@@ -99,6 +112,7 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->mode = g->mode;
   p->top_p = g->top_p;
   p->nref = std::max(g->n_ref, 1);
+  p->kfmt = g->key_format;
   p->batch = g->batch;
   p->cap = g->capacity;
   p->Bsh = p->bsh = -1;

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -24,6 +25,7 @@ struct TreeLayout {
   int64_t nodes[kMaxLevels];      // nodes per (sequence, KV head) at level l+1
   int64_t key_off[kMaxLevels];    // fp32 keys  [batch][Hkv][nodes][nref][d]
   int64_t val_off[kMaxLevels];    // fp32 values [batch][Hkv][nodes][d]
+  int64_t kscale_off[kMaxLevels]; // FP8 keys: fp32 scales [batch][Hkv][nodes][nref]
   int64_t rope_off;               // float2 (cos, sin) [rope_rows][d/2]
   int64_t total;
 };
@@ -35,6 +37,7 @@ struct Params {
   int32_t mode;       // RECSA_MODE_RECSA or RECSA_MODE_ZHA
   float top_p;        // ZHA routing mass
   int32_t nref;       // reference queries per pooler (keys per node), >= 1
+  int32_t kfmt;       // RECSA_KEYS_F32 or RECSA_KEYS_FP8
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;
@@ -56,6 +59,18 @@ __device__ __forceinline__ float* level_keys(const Params& p, void* tree, int le
   char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
   return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.d;
 }
+// FP8 key storage: codes [nodes][nref][d] bytes and scales [nodes][nref].
+__device__ __forceinline__ unsigned char* level_kcodes(const Params& p, void* tree, int lev,
+                                                       int64_t seq, int g) {
+  char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
+  return reinterpret_cast<unsigned char*>(base) +
+         ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.d;
+}
+__device__ __forceinline__ float* level_kscales(const Params& p, void* tree, int lev, int64_t seq,
+                                                int g) {
+  char* base = reinterpret_cast<char*>(tree) + p.lay.kscale_off[lev - 1];
+  return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref;
+}
 __device__ __forceinline__ float* level_vals(const Params& p, void* tree, int lev, int64_t seq,
                                              int g) {
   char* base = reinterpret_cast<char*>(tree) + p.lay.val_off[lev - 1];
@@ -63,6 +78,17 @@ __device__ __forceinline__ float* level_vals(const Params& p, void* tree, int le
 }
 __device__ __forceinline__ const float2* rope_table(const Params& p, const void* tree) {
   return reinterpret_cast<const float2*>(reinterpret_cast<const char*>(tree) + p.lay.rope_off);
+}
+
+// FP8 E4M3 code <-> float with CUDA's conversions (nearest, ties to even,
+// saturated at +-448).
+__device__ __forceinline__ float fp8_to_float(unsigned char c) {
+  __nv_fp8_e4m3 v;
+  v.__x = c;
+  return float(v);
+}
+__device__ __forceinline__ unsigned char float_to_fp8(float x) {
+  return __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -90,6 +90,22 @@ template <> struct Raw<__nv_bfloat16, 1> { __nv_bfloat16 a, b; };
 template <> struct Raw<float, 2> { float2 a, b; };
 template <> struct Raw<float, 1> { float a, b; };
 
+// The lane's channels of an FP8 code row (decoded, before the row's scale).
+template <int NP>
+__device__ __forceinline__ void load_codes(const unsigned char* row, int lane, float (&x1)[NP],
+                                           float (&x2)[NP]) {
+  constexpr int HALF = 32 * NP;
+  if constexpr (NP == 2) {
+    const unsigned short a = *reinterpret_cast<const unsigned short*>(row + 2 * lane);
+    const unsigned short b = *reinterpret_cast<const unsigned short*>(row + HALF + 2 * lane);
+    x1[0] = fp8_to_float(a & 0xFF); x1[1] = fp8_to_float(a >> 8);
+    x2[0] = fp8_to_float(b & 0xFF); x2[1] = fp8_to_float(b >> 8);
+  } else {
+    x1[0] = fp8_to_float(row[lane]);
+    x2[0] = fp8_to_float(row[HALF + lane]);
+  }
+}
+
 template <typename T, int NP>
 __device__ __forceinline__ Raw<T, NP> load_raw(const T* row, int lane) {
   constexpr int HALF = 32 * NP;
@@ -140,9 +156,12 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   extern __shared__ __align__(16) unsigned char smem[];
+  const bool fp8 = p.kfmt == RECSA_KEYS_FP8;                  // FP8 key codes + row scales
   float* kbuf = reinterpret_cast<float*>(smem);               // [krows][D] level key rows
-  float* rowsc = kbuf + size_t(krows) * D;                    // [krows] row scores (R > 1)
-  float* score = rowsc + krows;                               // [cmax]
+  const unsigned char* kbyte = smem;                          // (FP8: [krows][D] codes)
+  float* rowsc = reinterpret_cast<float*>(smem + size_t(krows) * D * (fp8 ? 1 : 4));
+  float* ksc = rowsc + krows;                                 // [krows] FP8 row scales
+  float* score = ksc + krows;                                 // [cmax]
   float* wsort = score + cmax;                                // [cmax] weights by rank
   float* zsum = wsort + cmax;                                 // [kZChain] sums, [kZChain] max
   float* wst = zsum + kZChain + 1;                            // [kZWarps][RS] warp states
@@ -286,16 +305,25 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       // in chunks of krows / R candidates; with R = 1 that is one chunk.
       const int R = p.nref;
       const int cc = krows / R;
-      constexpr int C16 = D / 4;                 // 16-byte pieces per fp32 row
+      const unsigned char* kcodes = level_kcodes(p, const_cast<void*>(tree), lev, seq, g);
+      const float* kscales = level_kscales(p, const_cast<void*>(tree), lev, seq, g);
+      const int C16 = fp8 ? D / 16 : D / 4;      // 16-byte pieces per row
       for (int i0c = 0; i0c < c; i0c += cc) {
         const int i1c = min(c, i0c + cc);
         const int nrow = (i1c - i0c) * R;
         for (int x = ct; x < nrow * C16; x += kZChain * 32) {
           const int q = x / C16, pc = x % C16;
           const int i = i0c + q / R, ref = q % R;
-          cp_async16(kbuf + size_t(q) * D + pc * 4,
-                     keys + (int64_t(node(i)) * R + ref) * D + pc * 4);
+          const int64_t row = int64_t(node(i)) * R + ref;
+          if (fp8)
+            cp_async16(const_cast<unsigned char*>(kbyte) + size_t(q) * D + pc * 16,
+                       kcodes + row * D + pc * 16);
+          else
+            cp_async16(kbuf + size_t(q) * D + pc * 4, keys + row * D + pc * 4);
         }
+        if (fp8)
+          for (int q = ct; q < nrow; q += kZChain * 32)
+            ksc[q] = kscales[int64_t(node(i0c + q / R)) * R + q % R];
         cp_async_wait_all();
         chain_sync();
         float* rsc = R == 1 ? score + i0c : rowsc;   // row scores
@@ -306,7 +334,10 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           for (int r = 0; r < 4; ++r) {
             const int q = min(q0 + r * kZChain, nrow - 1);   // rows past nrow repeat the last
             float x1[NP], x2[NP];
-            load_pairs<NP>(kbuf + size_t(q) * D, lane, x1, x2);
+            if (fp8)
+              load_codes<NP>(kbyte + size_t(q) * D, lane, x1, x2);
+            else
+              load_pairs<NP>(kbuf + size_t(q) * D, lane, x1, x2);
             sc4[r] = 0.f;
 #pragma unroll
             for (int u = 0; u < NP; ++u) {
@@ -323,7 +354,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 #pragma unroll
             for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
             const int q = q0 + lane * kZChain;
-            if (q < nrow) rsc[q] = v * p.inv_sqrt_d;
+            if (q < nrow) rsc[q] = v * p.inv_sqrt_d * (fp8 ? ksc[q] : 1.f);
           }
         }
         chain_sync();
@@ -483,11 +514,12 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   const int cmax = int(cm < 1 ? 1 : cm);
   if (cmax > kZMaxCand) return cudaErrorNotSupported;   // the generic kernel serves it
   const int kmax = int(kk < cmax ? kk : cmax);
-  // level key rows staged per chunk: the whole level at one reference
-  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, kZMaxRows));
+  // level key rows staged per chunk (FP8 rows are a quarter of the bytes)
+  const bool fp8 = p.kfmt == RECSA_KEYS_FP8;
+  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, fp8 ? 4 * kZMaxRows : kZMaxRows));
   if (krows < p.nref) return cudaErrorNotSupported;
-  const size_t bytes = (size_t(krows) * (D + 1) + 2 * size_t(cmax) + kZChain + 1 +
-                        kZWarps * (D + 2)) * 4 +
+  const size_t bytes = size_t(krows) * D * (fp8 ? 1 : 4) +
+                       (2 * size_t(krows) + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
                        (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + kZChain) * 4;
   if (bytes > 227 * 1024) return cudaErrorNotSupported;
   if (p.batch > 65535) return cudaErrorNotSupported;

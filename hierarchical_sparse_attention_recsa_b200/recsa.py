@@ -24,6 +24,8 @@ DTYPE_BF16 = 1
 MODE_RECSA = 0
 MODE_ZHA = 1
 MODE_GROUP = 2
+KEYS_F32 = 0
+KEYS_FP8 = 1
 KEEP_ALL = 2**31 - 1
 MAX_LEVELS = 16
 TRACE_MAX_K = 64
@@ -69,6 +71,8 @@ class CGeometry(ctypes.Structure):
         ("capacity", ctypes.c_int64),
         ("top_p", ctypes.c_float),
         ("n_ref", ctypes.c_int32),
+        ("key_format", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -91,12 +95,13 @@ class Geometry:
     mode: int = 0          # MODE_RECSA, MODE_ZHA or MODE_GROUP
     top_p: float = 0.0     # ZHA routing mass
     n_ref: int = 1         # reference queries per pooler (ZHA mode for n_ref > 1)
+    key_format: int = 0    # KEYS_F32 or KEYS_FP8 (ZHA mode)
 
     def c(self) -> CGeometry:
         return CGeometry(self.dtype, self.head_dim, self.n_q_heads, self.n_kv_heads,
                          self.leaf_block, self.branching, self.k, self.window,
                          self.rope_enabled, self.rope_base, self.batch, self.mode,
-                         self.capacity, self.top_p, self.n_ref)
+                         self.capacity, self.top_p, self.n_ref, self.key_format, 0)
 
     @property
     def torch_dtype(self) -> torch.dtype:

@@ -67,6 +67,10 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
 #define RECSA_MODE_ZHA 1
 #define RECSA_MODE_GROUP 2
 
+/* recsa_geometry.key_format: storage of the summary keys */
+#define RECSA_KEYS_F32 0 /* fp32 rows */
+#define RECSA_KEYS_FP8 1 /* FP8 E4M3 codes with one fp32 scale per row (ZHA mode only) */
+
 /* Device error flags in the tree header (recsa_tree_error). */
 #define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
 #define RECSA_DEVERR_WAIT_TIMEOUT 0x2u /* a bounded wait of the decode kernel on its own
@@ -103,6 +107,13 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   n_ref: with R = n_ref > 1 (ZHA mode only) every node holds R keys, one per
  *   reference query of the pooler, and a node's routing score is the largest
  *   of its R scores q . key_j / sqrt(d).
+ *   key_format: RECSA_KEYS_FP8 (ZHA mode only) stores every summary key row
+ *   as FP8 E4M3 codes (OCP format, ties to even, saturated at +-448) of
+ *   key / scale with scale = max|key| / 448 in fp32: a low-precision router
+ *   key cache ("Subquadratic Attention with a Hierarchical Tree-Structured
+ *   Indexer", Figure 16 caption).  A parent key pools its children's stored
+ *   (decoded) keys; values stay fp32; the routing score is
+ *   scale * (q . codes) / sqrt(d).
  */
 typedef struct recsa_geometry {
   int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
@@ -120,6 +131,8 @@ typedef struct recsa_geometry {
   int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
   float top_p;          /* ZHA: routing mass in (0, 1]; ignored in RECSA mode */
   int32_t n_ref;        /* reference queries per pooler: 0 or 1 = one; 2..64 (ZHA mode only) */
+  int32_t key_format;   /* RECSA_KEYS_F32 or RECSA_KEYS_FP8 (ZHA mode only) */
+  int32_t reserved;     /* must be 0 */
 } recsa_geometry;
 
 /* Human-readable name of a status code (static string). */
@@ -136,7 +149,8 @@ recsa_status recsa_num_levels(const recsa_geometry* geom, int64_t length, int32_
  * (device error flags), the RoPE cos/sin table of the indices a traversal can
  * reach, and per level l: keys [batch][n_kv_heads][n_l][n_ref][head_dim] and
  * values [batch][n_kv_heads][n_l][head_dim] in fp32, n_l the level's node
- * count at capacity.
+ * count at capacity.  With RECSA_KEYS_FP8 the keys are one byte per element,
+ * followed by their fp32 scales [batch][n_kv_heads][n_l][n_ref].
  */
 recsa_status recsa_tree_bytes(const recsa_geometry* geom, size_t* bytes);
 

@@ -109,15 +109,16 @@ def build_tree_fp8_multi(K, V, Rq, B: int, b: int):
             for lev in range(len(per[0]))]
 
 
-def near_rounding_boundary(x: np.ndarray, rel: float) -> np.ndarray:
-    """Elements of x (already divided by the row scale) within rel * quantum
-    of a midpoint between two E4M3 values, where a float32 computation of x
-    may round to the other neighbour."""
+def near_rounding_boundary(x: np.ndarray, tol: float) -> np.ndarray:
+    """Elements of x (already divided by the row scale, so the row's largest
+    magnitude is 448) within tol of a midpoint between two E4M3 values, where
+    a float32 computation of x -- whose error scales with the row's largest
+    element, not with the element itself -- may round to the other neighbour."""
     a = np.abs(np.asarray(x, dtype=np.float64))
     _, e = np.frexp(a)
     quantum = np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
     frac = a / quantum - np.floor(a / quantum)
-    return np.abs(frac - 0.5) < rel * np.maximum(a / quantum, 1.0)
+    return np.abs(frac - 0.5) * quantum < tol
 
 
 __all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_round", "quantize_row", "dequantize_row",

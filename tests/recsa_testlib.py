@@ -276,3 +276,36 @@ def check_group(stats: Stats, gpu_out, trace_recs, Qg, t, K, V, tree_src, og, k_
     for h in range(len(gpu_out)):
         stats.add(gpu_out[h], res["out"][h])
     return res
+
+
+def read_tree_level_fp8(g: R.Geometry, tree: torch.Tensor, lev: int):
+    """(codes uint8 [batch, Hkv, n_l, n_ref, d], scales fp32 [batch, Hkv, n_l,
+    n_ref], vals fp32 [batch, Hkv, n_l, d]) of one level of an FP8-key tree."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    kk = min(g.k, g.capacity)
+    rows = min(max(g.branching * kk + g.branching, g.leaf_block * kk + g.window + g.leaf_block),
+               g.capacity + g.branching + 1)
+    if g.mode == R.MODE_ZHA:
+        rows = max(rows, g.capacity + 1)
+    off = up(256 + rows * (g.head_dim // 2) * 8)
+    span = g.leaf_block
+    nr = max(g.n_ref, 1)
+    for l in range(1, lev + 1):
+        n = g.capacity // span
+        nrows = g.batch * g.n_kv_heads * n
+        code_off, scale_off = off, up(off + nrows * nr * g.head_dim)
+        val_off = up(scale_off + nrows * nr * 4)
+        if l == lev:
+            codes = tree[code_off:code_off + nrows * nr * g.head_dim].view(
+                g.batch, g.n_kv_heads, n, nr, g.head_dim)
+            scales = tree[scale_off:scale_off + nrows * nr * 4].view(torch.float32).view(
+                g.batch, g.n_kv_heads, n, nr)
+            vals = tree[val_off:val_off + nrows * g.head_dim * 4].view(torch.float32).view(
+                g.batch, g.n_kv_heads, n, g.head_dim)
+            return codes, scales, vals
+        off = up(val_off + nrows * g.head_dim * 4)
+        span *= g.branching
+    raise ValueError(lev)
+
+
+E4M3_TABLE = np.array([oracle.e4m3_decode(c) for c in range(256)])

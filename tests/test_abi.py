@@ -41,11 +41,13 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_struct_layout_matches_header(lib):
-    # 12 int32/float fields, one int64, then top_p and n_ref: 64 bytes.
-    assert ctypes.sizeof(R.CGeometry) == 64
+    # 12 int32/float fields, one int64, then top_p, n_ref, key_format, reserved: 72 bytes.
+    assert ctypes.sizeof(R.CGeometry) == 72
     assert R.CGeometry.capacity.offset == 48
     assert R.CGeometry.top_p.offset == 56
     assert R.CGeometry.n_ref.offset == 60
+    assert R.CGeometry.key_format.offset == 64
+    assert R.CGeometry.reserved.offset == 68
 
 
 def test_status_strings(lib):
@@ -64,6 +66,8 @@ def test_status_strings(lib):
     dict(mode=R.MODE_ZHA, top_p=1.0, k=R.KEEP_ALL, capacity=8192),
     dict(mode=R.MODE_GROUP),
     dict(mode=R.MODE_ZHA, top_p=0.9, n_ref=16), dict(n_ref=0), dict(n_ref=1),
+    dict(mode=R.MODE_ZHA, top_p=0.9, key_format=R.KEYS_FP8),
+    dict(mode=R.MODE_ZHA, top_p=0.9, n_ref=16, key_format=R.KEYS_FP8),
 ])
 def test_valid_geometries(lib, kw):
     R.recsa_validate(geo(**kw))
@@ -74,7 +78,9 @@ def test_valid_geometries(lib, kw):
     dict(branching=1), dict(window=0), dict(k=0), dict(leaf_block=0), dict(batch=0),
     dict(capacity=0), dict(dtype=7), dict(rope_base=1.0), dict(n_kv_heads=0),
     dict(mode=3), dict(mode=-1), dict(n_ref=2), dict(mode=R.MODE_GROUP, n_ref=4),
-    dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=65), dict(n_ref=-1), dict(mode=R.MODE_ZHA, top_p=0.0), dict(mode=R.MODE_ZHA, top_p=1.5),
+    dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=65), dict(n_ref=-1), dict(mode=R.MODE_ZHA, top_p=0.0),
+    dict(key_format=R.KEYS_FP8), dict(mode=R.MODE_GROUP, key_format=R.KEYS_FP8),
+    dict(mode=R.MODE_ZHA, top_p=0.5, key_format=2), dict(mode=R.MODE_ZHA, top_p=1.5),
     dict(mode=R.MODE_ZHA, top_p=float("nan")),
 ])
 def test_invalid_geometries(lib, kw):
@@ -104,15 +110,23 @@ def expected_tree_bytes(g: R.Geometry) -> int:
     span = g.leaf_block
     while g.capacity // span >= 1:
         n = g.capacity // span
-        row_bytes = g.batch * g.n_kv_heads * n * g.head_dim * 4
-        total += up(row_bytes * max(g.n_ref, 1)) + up(row_bytes)
+        rows = g.batch * g.n_kv_heads * n
+        row_bytes = rows * g.head_dim * 4
+        nr = max(g.n_ref, 1)
+        if g.key_format == R.KEYS_FP8:   # one byte per key element, then fp32 row scales
+            total += up(rows * nr * g.head_dim) + up(rows * nr * 4) + up(row_bytes)
+        else:
+            total += up(row_bytes * nr) + up(row_bytes)
         span *= g.branching
     return total
 
 
 @pytest.mark.parametrize("kw", [dict(), dict(batch=1, capacity=4096 + 17), dict(k=R.KEEP_ALL),
                                 dict(mode=R.MODE_ZHA, top_p=0.5),
-                                dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=16)])
+                                dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=16),
+                                dict(mode=R.MODE_ZHA, top_p=0.5, key_format=R.KEYS_FP8),
+                                dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=4,
+                                     key_format=R.KEYS_FP8)])
 def test_tree_bytes(lib, kw):
     g = geo(**kw)
     assert R.recsa_tree_bytes(g) == expected_tree_bytes(g)

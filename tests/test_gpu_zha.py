@@ -19,8 +19,9 @@ import oracle
 from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
 from hierarchical_sparse_attention_recsa_b200 import recsa as R
 
-from recsa_testlib import (Stats, alloc_tree, check_query_zha, geometry, oracle_geometry,
-                           parse_trace, read_tree_level, to_np)
+from recsa_testlib import (E4M3_TABLE, Stats, alloc_tree, check_query_zha, geometry,
+                           oracle_geometry, parse_trace, read_tree_level, read_tree_level_fp8,
+                           to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -470,3 +471,201 @@ def test_zha_multiref_full_mass_is_dense(rope, zha_impl):
                                                 rope_base=w.rope_base)
             st.add(O_[0, t, h], ref)
     st.check(torch.float32, f"zha {zha_impl} multiref full mass")
+
+
+# ---------------------------------------------------------------------------
+# Low-precision router keys (FP8 E4M3 with one scale per key row)
+# ---------------------------------------------------------------------------
+
+def _setup_fp8(w, lens, capacity, top_p, n_ref, seed, k=None, rope=1):
+    batch = len(lens)
+    g = geometry(w, capacity, batch, k=k, rope=rope, top_p=top_p)
+    g.n_ref = n_ref
+    g.key_format = R.KEYS_FP8
+    K, V, r = synth.make_kv(w, capacity, seed=seed, device="cpu", batch=batch)
+    Rq = _refs(r, n_ref, seed + 1000) if n_ref > 1 else r.reshape(1, -1).contiguous()
+    Kd, Vd, Rd = K.cuda(), V.cuda(), Rq.cuda()
+    tree = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, lens, Rd, 0, tree)
+    torch.cuda.synchronize()
+    return g, K, V, Rq, Kd, Vd, Rd, tree
+
+
+def _fp8_trees(g, K, V, Rq, lens):
+    out = {}
+    for s, L in enumerate(lens):
+        for h in range(g.n_kv_heads):
+            Kh, Vh = to_np(K[s, h, :L]), to_np(V[s, h, :L])
+            levels = oracle.build_tree_fp8_multi(Kh, Vh, Rq.double().numpy(), g.leaf_block,
+                                                 g.branching)
+            if Rq.shape[0] == 1:
+                levels = [(kk[:, 0], vv) for kk, vv in levels]
+                out[(s, h)] = (Kh, Vh, oracle.FullTree(levels))
+            else:
+                out[(s, h)] = (Kh, Vh, oracle.MultiTree(levels))
+    return out
+
+
+@pytest.mark.parametrize("n_ref", [1, 2])
+def test_zha_fp8_tree_codes(n_ref):
+    """Every stored code is the oracle's E4M3 rounding of key / scale.  Level 1
+    differs only where the float64 and float32 quotients straddle a rounding
+    midpoint (then by one step); higher levels pool children that may carry
+    such a one-step difference, so a few adjacent codes may differ there."""
+    L = TINY.length
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(TINY, [L], L, 0.7, n_ref, seed=70)
+    Kh, Vh = to_np(K[0, 0]), to_np(V[0, 0])
+    Rn = Rq.double().numpy()
+    levels = oracle.build_tree_fp8_multi(Kh, Vh, Rn, g.leaf_block, g.branching)
+    for lev in range(1, len(levels) + 1):
+        codes, scales, vals = read_tree_level_fp8(g, tree, lev)
+        n = levels[lev - 1][0].shape[0]
+        got = E4M3_TABLE[codes[0, 0, :n].cpu().numpy().astype(np.int64)]
+        sc = scales[0, 0, :n].cpu().numpy().astype(np.float64)
+        fan = g.leaf_block if lev == 1 else g.branching
+        mism = 0
+        for j in range(n):
+            for ref in range(n_ref):
+                src = Kh if lev == 1 else levels[lev - 2][0][:, ref]
+                x = oracle.pool_keys(src[j * fan:(j + 1) * fan], Rn[ref])
+                want, scale = oracle.quantize_row(x)
+                np.testing.assert_allclose(sc[j, ref], scale, rtol=2e-5 if lev == 1 else 1e-3)
+                bad = got[j, ref] != want
+                if bad.any():
+                    mism += int(bad.sum())
+                    # one E4M3 step apart, and (level 1) at a rounding midpoint
+                    step = np.abs(got[j, ref][bad] - want[bad])
+                    assert np.all(step <= np.maximum(np.abs(want[bad]), 2.0 ** -6) / 8 + 1e-12)
+                    if lev == 1:   # float32 pooling errs by ~1e-6 of the row's max (448 here)
+                        assert np.all(oracle.near_rounding_boundary((x / scale)[bad], 448 * 2e-5))
+        assert mism <= max(2, 0.01 * n * n_ref * g.head_dim), (lev, mism)
+        np.testing.assert_allclose(vals[0, 0, :n].cpu().numpy(), levels[lev - 1][1],
+                                   atol=1e-5 if lev > 1 else 1e-6)
+
+
+@pytest.mark.parametrize("n_ref,top_p", [(1, 0.7), (4, 0.9)])
+def test_zha_fp8_decode_tiny(n_ref, top_p, zha_impl):
+    L, nq = TINY.length, 64
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(TINY, [L], L, top_p, n_ref, seed=72, k=ZK)
+    trees = _fp8_trees(g, K, V, Rq, [L])
+    pos = torch.full((1, nq), L - 1, dtype=torch.int64)
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=73, n_needles=8)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for i in range(nq):
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh, Vh, src,
+                            og, top_p, g.k)
+    st.check(torch.float32, f"zha {zha_impl} fp8 R={n_ref} decode tiny")
+    assert st.clear > 0.6 * nq * g.n_q_heads
+
+
+def test_zha_fp8_prefill_tiny(zha_impl):
+    L, top_p = TINY.length, 0.8
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(TINY, [L], L, top_p, 1, seed=74, k=ZK)
+    trees = _fp8_trees(g, K, V, Rq, [L])
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=75)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, L, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    rng = np.random.default_rng(8)
+    sample = sorted(set([0, 15, 16, 64, 65, 300, L - 1] + list(rng.integers(0, L, 25))))
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for t in sample:
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, t, h], tr[0, t, h], to_np(Q[0, t, h]), t, Kh, Vh, src, og,
+                            top_p, g.k)
+    st.check(torch.float32, f"zha {zha_impl} fp8 prefill tiny")
+
+
+def test_zha_fp8_decode_model_small(zha_impl):
+    lens, top_p = [20000, 13001], 0.9
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(MODEL, lens, 20480, top_p, 1, seed=76)
+    trees = _fp8_trees(g, K, V, Rq, lens)
+    nq = 2
+    pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(MODEL, K, pos, seed=77, n_needles=2)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for i in range(nq):
+            for h in range(g.n_q_heads):
+                Kh, Vh, src = trees[(s, h // G)]
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} fp8 decode model small")
+
+
+def test_zha_fp8_append_matches_build():
+    w, top_p = MODEL, 0.9
+    lens0 = [4000, 4031]
+    steps = 100
+    cap = 4096 + 256
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(w, lens0, cap, top_p, 2, seed=78)
+    Kw, Vw = Kd.clone(), Vd.clone()
+    Kw[0, :, 4000:] = 0
+    Vw[0, :, 4000:] = 0
+    Kw[1, :, 4031:] = 0
+    Vw[1, :, 4031:] = 0
+    lens_d = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        R.recsa_append(g, Kw, Vw, kn, vn, lens_d, Rd, 0, tree)
+    new_lens = [L + steps for L in lens0]
+    fresh = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, new_lens, Rd, 0, fresh)
+    torch.cuda.synchronize()
+    for lev in range(1, R.recsa_num_levels(g, max(new_lens)) + 1):
+        a_c, a_s, a_v = read_tree_level_fp8(g, tree, lev)
+        b_c, b_s, b_v = read_tree_level_fp8(g, fresh, lev)
+        for s in range(2):
+            n = new_lens[s] // (g.leaf_block * g.branching ** (lev - 1))
+            assert torch.equal(a_c[s, :, :n], b_c[s, :, :n]), lev
+            torch.testing.assert_close(a_s[s, :, :n], b_s[s, :, :n], rtol=0, atol=0)
+            torch.testing.assert_close(a_v[s, :, :n], b_v[s, :, :n], rtol=0, atol=1e-6)
+
+
+def test_zha_fp8_full_mass_is_dense(zha_impl):
+    w = TINY
+    L = 1500
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(w, [L], L, 1.0, 1, seed=79, k=R.KEEP_ALL)
+    pos = torch.arange(L, dtype=torch.int64)[None]
+    Q, _, _ = synth.make_queries(w, K, pos, seed=80)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, 0, L, O)
+    torch.cuda.synchronize()
+    O_ = to_np(O)
+    st = Stats()
+    for t in [0, 63, 64, 700, L - 1]:
+        for h in range(g.n_q_heads):
+            ref = oracle.dense_causal_attention(to_np(Q[0, t, h]), t, to_np(K[0, 0]),
+                                                to_np(V[0, 0]), rope=True, rope_base=w.rope_base)
+            st.add(O_[0, t, h], ref)
+    st.check(torch.float32, f"zha {zha_impl} fp8 full mass")
