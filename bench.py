@@ -356,6 +356,9 @@ def run_recsa(args, rank, world, dev):
         out["zha_multiref"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
                                           hbm_gbs, peak_kind, R.MODE_ZHA, cpu_leg,
                                           n_ref=ZHA_N_REF)
+        out["zha_multiref_fp8"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
+                                              hbm_gbs, peak_kind, R.MODE_ZHA, False,
+                                              n_ref=ZHA_N_REF, key_format=R.KEYS_FP8)
     if not args.no_group:
         out["group"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
                                    peak_kind, R.MODE_GROUP, cpu_leg)
@@ -376,13 +379,14 @@ def reference_queries(r, n_ref, seed=7):
 
 
 def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, mode, cpu,
-                n_ref=1):
+                n_ref=1, key_format=0):
     """A selection variant on the same cache: its own tree (same pooling),
     then the batch's decode queries at t = L - 1, timed per launch like the
     main decode.  MODE_ZHA: top-p expansion, exact tokens of the reached
     leaves and the window at true positions (the RoPE table covers every
-    position), with n_ref reference queries per pooler.  MODE_GROUP: RecSA
-    with one selection per KV group."""
+    position), with n_ref reference queries per pooler and fp32 or FP8
+    (key_format) summary keys.  MODE_GROUP: RecSA with one selection per KV
+    group."""
     batch = Kc.shape[0]
     zha = mode == R.MODE_ZHA
     g = R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
@@ -390,7 +394,7 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
                    batch=batch, capacity=cap,
                    dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
                    rope_enabled=1, rope_base=w.rope_base, mode=mode,
-                   top_p=ZHA_TOP_P if zha else 0.0, n_ref=n_ref)
+                   top_p=ZHA_TOP_P if zha else 0.0, n_ref=n_ref, key_format=key_format)
     tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
     refs = reference_queries(r, n_ref) if n_ref > 1 else r
     R.recsa_build(g, Kc, Vc, [L] * batch, refs, 0, tree)
@@ -415,8 +419,9 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     G = w.n_q_heads // w.n_kv_heads
     nb = [counts.decode_bytes_from_trace(tr[i], np.full(batch, L), w.leaf_block, w.branching,
                                          w.window, G, w.head_dim, elem_bytes(w), w.k,
-                                         summary_values=not zha,
-                                         keys_per_node=n_ref)["bytes"] for i in range(n)]
+                                         summary_values=not zha, keys_per_node=n_ref,
+                                         key_row_bytes=w.head_dim + 4 if key_format else 0
+                                         )["bytes"] for i in range(n)]
     kept = tr[..., 4 + 16:4 + 16 + R.recsa_num_levels(g, L)].astype(np.float64)
     nbytes = float(np.mean(nb))
     achieved = nbytes / (dec_ms / 1e3) / 1e9
@@ -431,6 +436,7 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     if zha:
         res["top_p"] = ZHA_TOP_P
         res["n_ref"] = n_ref
+        res["keys"] = "fp8_e4m3 + fp32 row scale" if key_format else "fp32"
     del tree, traces
     torch.cuda.empty_cache()
     if cpu:

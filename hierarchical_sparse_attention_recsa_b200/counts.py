@@ -41,7 +41,8 @@ def per_query_counts(t: np.ndarray, B: int, b: int, k: int, W: int, levels: int)
 
 def decode_bytes_from_trace(trace: np.ndarray, lens: np.ndarray, B: int, b: int, W: int,
                             G: int, d: int, elem: int, k: int,
-                            summary_values: bool = True, keys_per_node: int = 1) -> dict:
+                            summary_values: bool = True, keys_per_node: int = 1,
+                            key_row_bytes: int = 0) -> dict:
     """Distinct bytes one decode launch must touch, from its selection trace.
 
     trace [batch, n_q, H_q, ints] (n_q = 1); lens [batch] after the append.
@@ -50,7 +51,8 @@ def decode_bytes_from_trace(trace: np.ndarray, lens: np.ndarray, B: int, b: int,
     candidates (fp32 rows; none when ``summary_values`` is False, as in the
     ZHA routing variant, whose softmax holds exact tokens only), K and V rows
     of the union of exact tokens (dtype); plus Q read and O written.  A node
-    scored reads ``keys_per_node`` key rows (one per reference query).
+    scored reads ``keys_per_node`` key rows (one per reference query) of
+    ``key_row_bytes`` each (default fp32 rows: 4 d; FP8 rows: d + 4).
     """
     batch, n_q, hq, _ = trace.shape
     hkv = hq // G
@@ -94,7 +96,8 @@ def decode_bytes_from_trace(trace: np.ndarray, lens: np.ndarray, B: int, b: int,
                 val_rows += unsel_total if summary_values else 0
                 tok_rows += len(leaves) * B + (t + 1 - a * B)
     qo = 2 * batch * n_q * hq * d * elem
-    tree_bytes = (key_rows * keys_per_node + val_rows) * d * 4
+    krb = key_row_bytes or d * 4
+    tree_bytes = key_rows * keys_per_node * krb + val_rows * d * 4
     kv_bytes = tok_rows * d * elem * 2
     return dict(bytes=qo + tree_bytes + kv_bytes, qo=qo, tree=tree_bytes, kv=kv_bytes,
                 key_rows=key_rows, val_rows=val_rows, tok_rows=tok_rows)
