@@ -13,12 +13,12 @@
 //     exact window [a*B, t], at their true positions with standard RoPE.
 //
 // Layout for B200:
-//   * Warps 0-7 (the chain) walk the levels: a level's candidate key rows are
+//   * Warps 0-11 (the chain) walk the levels: a level's candidate key rows are
 //     copied into shared memory with 16-byte cp.async (the whole level in
 //     flight at once) and scored four rows per warp at a time; the top-p cut
 //     comes from every candidate's rank (one chain thread per candidate) and
 //     a warp scan of the weights laid out by rank.
-//   * Warps 8-15 attend the window, which does not depend on the routing,
+//   * Warps 12-15 attend the window, which does not depend on the routing,
 //     while the chain runs; then all 16 warps attend the reached leaves.
 //   * Exact tokens are taken in units of up to 16 consecutive positions: the
 //     query is rotated once per unit by R(t - first position) from the RoPE
@@ -36,7 +36,7 @@ namespace {
 
 constexpr int kZThreads = 512;
 constexpr int kZWarps = kZThreads / 32;
-constexpr int kZChain = 8;          // chain warps; the others attend the window first
+constexpr int kZChain = 12;         // chain warps; the others attend the window first
 constexpr int kZMaxCand = kZChain * 32;   // one chain thread per candidate
 constexpr int kZMaxRows = 256;            // level key rows staged at once
 constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
@@ -368,7 +368,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         }
       }
       chain_sync();
-      // Top-p by ranks: chain thread ct holds candidate ct (c <= 256).  Its rank
+      // Top-p by ranks: chain thread ct holds candidate ct (c <= 384).  Its rank
       // counts the better candidates (higher score, or equal at a lower
       // index); the weights exp(s - max) are laid out by rank, and warp 0
       // scans them for the shortest prefix whose mass reaches top_p of the
