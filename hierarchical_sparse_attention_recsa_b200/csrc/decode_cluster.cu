@@ -1264,8 +1264,8 @@ cudaError_t cluster_g(const Params& p, const void* Q, const void* K, const void*
 }
 
 // Heads per CTA (HPC) and candidate shares per head group (S) of a launch.
-// RECSA_DECODE_SPLIT="hpc,s" forces both (tests); otherwise the fewest heads
-// per CTA and the most shares that keep the grid within the 148 SMs.
+// RECSA_DECODE_SPLIT="hpc,s" forces both (tests); otherwise the rule below.
+// (The launch doubles S further when a share's rows do not fit shared memory.)
 void decode_split(const Params& p, int32_t n_q, int& hpc, int& S) {
   const int G = p.group;
   const char* env = getenv("RECSA_DECODE_SPLIT");
@@ -1279,11 +1279,20 @@ void decode_split(const Params& p, int32_t n_q, int& hpc, int& S) {
     }
   }
   const int64_t pairs = int64_t(p.batch) * p.hkv * n_q;
+  if (p.mode == RECSA_MODE_GROUP) {
+    // every head of the group in one CTA; shares fill the 148 SMs
+    hpc = G;
+    S = 1;
+    while (S * 2 <= kMaxCluster && pairs * S * 2 <= 148) S *= 2;
+    return;
+  }
+  // One query head per CTA, and a second candidate share when the grid still
+  // fits the 148 SMs.  Measured at 131K and 2M (batch 1), 1M (batch 8) and
+  // 524K (batch 4): more heads per CTA or more shares cost more in per-CTA
+  // work and cross-CTA level barriers than the extra SMs give back, even when
+  // the grid then needs several waves.
   hpc = 1;
-  while (hpc < G && (pairs * (G / hpc) > 148 || p.mode == RECSA_MODE_GROUP)) hpc *= 2;
-  const int ng = G / hpc;
-  S = 1;
-  while (ng * S * 2 <= kMaxCluster && pairs * ng * S * 2 <= 148) S *= 2;
+  S = pairs * G * 2 <= 148 ? 2 : 1;
 }
 
 cudaError_t cluster_dispatch(const Params& p, const void* Q, const void* K, const void* V,
