@@ -48,4 +48,5 @@ from .zha import top_p_prefix, zha_route_and_attend  # noqa: F401
 from .group import group_select, group_traverse_and_attend  # noqa: F401
 from .multiref import LazyMultiTree, MultiTree, build_tree_multi  # noqa: F401
 from .lowprec import (build_tree_fp8, build_tree_fp8_multi, dequantize_row,  # noqa: F401
-                      e4m3_decode, e4m3_round, near_rounding_boundary, quantize_row)
+                      e4m3_decode, e4m3_round, near_rounding_boundary, quantize_row,
+                      e2m1_decode, e2m1_round, quantize_row_nvfp4, build_tree_nvfp4_multi)

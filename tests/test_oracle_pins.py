@@ -740,3 +740,36 @@ def test_fp8_tree_keys_are_quantized_pools_of_quantized_children():
             np.testing.assert_allclose(oracle.e4m3_round(unit), unit, rtol=1e-14)
             np.testing.assert_allclose(vals[j], (V if lev == 1 else levels[lev - 2][1])
                                        [j * fan:(j + 1) * fan].mean(0), atol=1e-14)
+
+
+def test_e2m1_codes_rounding_and_saturation():
+    vals = [oracle.e2m1_decode(c) for c in range(16)]
+    assert vals[:8] == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert vals[8:] == [-v for v in vals[:8]]
+    pos = np.array(vals[:8])
+    np.testing.assert_array_equal(oracle.e2m1_round(pos), pos)
+    np.testing.assert_array_equal(oracle.e2m1_round(-pos), -pos)
+    # midpoints go to the neighbour with mantissa bit 0 (codes 0, 2, 4, 6 -> even)
+    mids = (pos[:-1] + pos[1:]) / 2                     # 0.25 .75 1.25 1.75 2.5 3.5 5
+    assert oracle.e2m1_round(mids).tolist() == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    assert oracle.e2m1_round(np.array([6.9, 7.0, 100.0, -50.0])).tolist() == [6, 6, 6, -6]
+
+
+def test_nvfp4_row_is_block_scaled_e2m1():
+    rng = np.random.default_rng(42)
+    for trial in range(50):
+        x = rng.standard_normal(64) * 10.0 ** rng.uniform(-3, 2)
+        y = oracle.quantize_row_nvfp4(x)
+        g = np.abs(x).max() / (6 * 448)
+        for b0 in range(0, 64, 16):
+            blk, qb = x[b0:b0 + 16], y[b0:b0 + 16]
+            sb = float(oracle.e4m3_round(np.abs(blk).max() / (6 * g)))
+            assert oracle.e4m3_round(np.array([sb]))[0] == sb and sb > 0
+            unit = qb / (sb * g)
+            np.testing.assert_allclose(oracle.e2m1_round(unit), unit, atol=1e-12)
+            # within half an E2M1 step of the scaled input (steps 0.5, 1, 2), or saturated
+            a = np.abs(blk / (sb * g))
+            step = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+            ok = (np.abs(unit - blk / (sb * g)) <= step / 2 + 1e-12) | (np.abs(unit) == 6.0)
+            assert ok.all()
+    assert not oracle.quantize_row_nvfp4(np.zeros(32)).any()
