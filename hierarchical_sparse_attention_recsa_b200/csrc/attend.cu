@@ -216,6 +216,29 @@ attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         const float* ks = level_kscales(p, const_cast<void*>(tree), lev, seq, g) + node * p.nref;
         s = dot_row(h, kc, -1) * ks[0];
         for (int ref = 1; ref < p.nref; ++ref) s = fmaxf(s, dot_row(h, kc + ref * d, -1) * ks[ref]);
+      } else if (p.kfmt == RECSA_KEYS_NVFP4) {   // E2M1 codes x block scale, x row scale
+        const unsigned char* kc = level_kcodes(p, const_cast<void*>(tree), lev, seq, g) +
+                                  node * p.nref * p.kcb;
+        const unsigned char* kb = level_kbscales(p, const_cast<void*>(tree), lev, seq, g) +
+                                  node * p.nref * (d / 16);
+        const float* ks = level_kscales(p, const_cast<void*>(tree), lev, seq, g) + node * p.nref;
+        s = -INFINITY;
+        for (int ref = 0; ref < p.nref; ++ref) {
+          const unsigned char* c0 = kc + ref * p.kcb;
+          const unsigned char* b0 = kb + ref * (d / 16);
+          float acc_ = 0.f;
+#pragma unroll
+          for (int u = 0; u < P; ++u) {
+            const int j = lane + 32 * u;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int e = j + hf * half;
+              const float v = fp4_to_float(c0[e >> 1] >> (4 * (e & 1))) * fp8_to_float(b0[e >> 4]);
+              acc_ = fmaf(qr[h * d + e], v, acc_);
+            }
+          }
+          s = fmaxf(s, warp_sum(acc_) * p.inv_sqrt_d * ks[ref]);
+        }
       } else {
         const float* kr = keys + node * p.nref * d;
         s = dot_row(h, kr, zha ? -1 : ii);

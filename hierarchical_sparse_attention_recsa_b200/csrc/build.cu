@@ -24,8 +24,12 @@ template <int N>
 __device__ void store_node_key(const Params& p, void* tree, int lev, int64_t seq, int g,
                                int64_t j, int ref, int lane, const float* key) {
   if (p.kfmt == RECSA_KEYS_FP8)
-    store_key_fp8<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d,
+    store_key_fp8<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.kcb,
                      level_kscales(p, tree, lev, seq, g) + j * p.nref + ref, lane, key);
+  else if (p.kfmt == RECSA_KEYS_NVFP4)
+    store_key_nvfp4<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.kcb,
+                       level_kbscales(p, tree, lev, seq, g) + (j * p.nref + ref) * (p.d / 16),
+                       level_kscales(p, tree, lev, seq, g) + j * p.nref + ref, lane, key);
   else
     RowIO<float, N>::store(level_keys(p, tree, lev, seq, g) + (j * p.nref + ref) * p.d, lane,
                            key);
@@ -39,11 +43,24 @@ __device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, i
   const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
   if (p.kfmt == RECSA_KEYS_FP8) {
     const unsigned char* cc =
-        level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.d;
+        level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.kcb;
     const float* cs = level_kscales(p, tree, lev - 1, seq, g) + j * p.b * p.nref + ref;
     pool_children<float, N>(
         [&](int i, float* x) {
-          load_key_fp8<N>(cc + int64_t(i) * p.nref * p.d, cs[int64_t(i) * p.nref], lane, x);
+          load_key_fp8<N>(cc + int64_t(i) * p.nref * p.kcb, cs[int64_t(i) * p.nref], lane, x);
+        },
+        cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
+  } else if (p.kfmt == RECSA_KEYS_NVFP4) {
+    const int nb = p.d / 16;
+    const unsigned char* cc =
+        level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.kcb;
+    const unsigned char* cb =
+        level_kbscales(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * nb;
+    const float* cs = level_kscales(p, tree, lev - 1, seq, g) + j * p.b * p.nref + ref;
+    pool_children<float, N>(
+        [&](int i, float* x) {
+          load_key_nvfp4<N>(cc + int64_t(i) * p.nref * p.kcb, cb + int64_t(i) * p.nref * nb,
+                            cs[int64_t(i) * p.nref], lane, x);
         },
         cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
   } else {

@@ -145,6 +145,50 @@ __device__ void load_key_fp8(const unsigned char* codes, float scale, int lane, 
   for (int c = 0; c < N; ++c) x[c] = fp8_to_float((packed >> (8 * c)) & 0xFFu) * scale;
 }
 
+// NVFP4 row format: E2M1 codes, two per byte (lower element in the low
+// nibble), one E4M3 scale per 16 elements, one fp32 scale per row.  A lane's
+// N contiguous channels are N / 2 bytes; a block of 16 spans 16 / N lanes.
+// row scale g = max|key| / (6 * 448); block scale sb = E4M3(block max / (6 g));
+// code = E2M1(key / (sb * g)).
+template <int N>
+__device__ void store_key_nvfp4(unsigned char* codes, unsigned char* bscales, float* rscale,
+                                int lane, const float* key) {
+  constexpr int LPB = 16 / N;   // lanes per block
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < N; ++c) amax = fmaxf(amax, fabsf(key[c]));
+  float bmax = amax;
+#pragma unroll
+  for (int o = 1; o < LPB; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+  amax = warp_max(amax);
+  const float g = amax / (6.f * 448.f);
+  const unsigned char sbc = g > 0.f ? float_to_fp8(bmax / (6.f * g)) : 0;
+  const float den = fp8_to_float(sbc) * g;
+  unsigned int packed = 0;
+#pragma unroll
+  for (int c = 0; c < N; ++c)
+    packed |= (den > 0.f ? float_to_fp4(key[c] / den) : 0u) << (4 * c);
+  if constexpr (N == 4)
+    reinterpret_cast<unsigned short*>(codes)[lane] = static_cast<unsigned short>(packed);
+  else
+    codes[lane] = static_cast<unsigned char>(packed);
+  if (lane % LPB == 0) bscales[lane / LPB] = sbc;
+  if (lane == 0) *rscale = g;
+}
+template <int N>
+__device__ void load_key_nvfp4(const unsigned char* codes, const unsigned char* bscales, float g,
+                               int lane, float* x) {
+  constexpr int LPB = 16 / N;
+  unsigned int packed;
+  if constexpr (N == 4)
+    packed = reinterpret_cast<const unsigned short*>(codes)[lane];
+  else
+    packed = codes[lane];
+  const float den = fp8_to_float(bscales[lane / LPB]) * g;
+#pragma unroll
+  for (int c = 0; c < N; ++c) x[c] = fp4_to_float(packed >> (4 * c)) * den;
+}
+
 template <int N>
 __device__ void load_r(const float* r, int lane, float* rl) {
 #pragma unroll

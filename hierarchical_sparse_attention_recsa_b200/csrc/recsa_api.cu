@@ -30,9 +30,10 @@ recsa_status check_geometry(const recsa_geometry* g) {
   if (g->batch < 1 || g->capacity < 1) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->n_ref < 0 || g->n_ref > 64) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->n_ref > 1 && g->mode != RECSA_MODE_ZHA) return RECSA_ERR_INVALID_GEOMETRY;
-  if (g->key_format != RECSA_KEYS_F32 && g->key_format != RECSA_KEYS_FP8)
+  if (g->key_format != RECSA_KEYS_F32 && g->key_format != RECSA_KEYS_FP8 &&
+      g->key_format != RECSA_KEYS_NVFP4)
     return RECSA_ERR_INVALID_GEOMETRY;
-  if (g->key_format == RECSA_KEYS_FP8 && g->mode != RECSA_MODE_ZHA)
+  if (g->key_format != RECSA_KEYS_F32 && g->mode != RECSA_MODE_ZHA)
     return RECSA_ERR_INVALID_GEOMETRY;
   if (g->reserved != 0) return RECSA_ERR_INVALID_GEOMETRY;
   if (g->mode != RECSA_MODE_RECSA && g->mode != RECSA_MODE_ZHA && g->mode != RECSA_MODE_GROUP)
@@ -83,6 +84,12 @@ recsa_status make_layout(const recsa_geometry* g, TreeLayout* lay) {
       off = align_up(off + rows * nref * g->head_dim, 256);
       lay->kscale_off[l] = off;
       off = align_up(off + rows * nref * 4, 256);
+    } else if (g->key_format == RECSA_KEYS_NVFP4) {   // codes, block scales, row scales
+      off = align_up(off + rows * nref * (g->head_dim / 2), 256);
+      lay->kbscale_off[l] = off;
+      off = align_up(off + rows * nref * (g->head_dim / 16), 256);
+      lay->kscale_off[l] = off;
+      off = align_up(off + rows * nref * 4, 256);
     } else {
       off = align_up(off + bytes * nref, 256);
     }
@@ -113,6 +120,7 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->top_p = g->top_p;
   p->nref = std::max(g->n_ref, 1);
   p->kfmt = g->key_format;
+  p->kcb = g->key_format == RECSA_KEYS_NVFP4 ? g->head_dim / 2 : g->head_dim;
   p->batch = g->batch;
   p->cap = g->capacity;
   p->Bsh = p->bsh = -1;

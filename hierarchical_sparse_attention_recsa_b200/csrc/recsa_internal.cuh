@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -25,7 +26,8 @@ struct TreeLayout {
   int64_t nodes[kMaxLevels];      // nodes per (sequence, KV head) at level l+1
   int64_t key_off[kMaxLevels];    // fp32 keys  [batch][Hkv][nodes][nref][d]
   int64_t val_off[kMaxLevels];    // fp32 values [batch][Hkv][nodes][d]
-  int64_t kscale_off[kMaxLevels]; // FP8 keys: fp32 scales [batch][Hkv][nodes][nref]
+  int64_t kscale_off[kMaxLevels]; // FP8 / NVFP4 keys: fp32 row scales [batch][Hkv][nodes][nref]
+  int64_t kbscale_off[kMaxLevels];// NVFP4 keys: E4M3 block scales [..][nref][d / 16]
   int64_t rope_off;               // float2 (cos, sin) [rope_rows][d/2]
   int64_t total;
 };
@@ -37,7 +39,8 @@ struct Params {
   int32_t mode;       // RECSA_MODE_RECSA or RECSA_MODE_ZHA
   float top_p;        // ZHA routing mass
   int32_t nref;       // reference queries per pooler (keys per node), >= 1
-  int32_t kfmt;       // RECSA_KEYS_F32 or RECSA_KEYS_FP8
+  int32_t kfmt;       // RECSA_KEYS_F32, RECSA_KEYS_FP8 or RECSA_KEYS_NVFP4
+  int32_t kcb;        // code bytes per key row (FP8: d, NVFP4: d / 2)
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;
@@ -59,12 +62,19 @@ __device__ __forceinline__ float* level_keys(const Params& p, void* tree, int le
   char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
   return reinterpret_cast<float*>(base) + ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.d;
 }
-// FP8 key storage: codes [nodes][nref][d] bytes and scales [nodes][nref].
+// Low-precision key storage: codes [nodes][nref][kcb] bytes, (NVFP4) block
+// scales [nodes][nref][d / 16] bytes, row scales [nodes][nref] fp32.
 __device__ __forceinline__ unsigned char* level_kcodes(const Params& p, void* tree, int lev,
                                                        int64_t seq, int g) {
   char* base = reinterpret_cast<char*>(tree) + p.lay.key_off[lev - 1];
   return reinterpret_cast<unsigned char*>(base) +
-         ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.d;
+         ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * p.kcb;
+}
+__device__ __forceinline__ unsigned char* level_kbscales(const Params& p, void* tree, int lev,
+                                                         int64_t seq, int g) {
+  char* base = reinterpret_cast<char*>(tree) + p.lay.kbscale_off[lev - 1];
+  return reinterpret_cast<unsigned char*>(base) +
+         ((seq * p.hkv + g) * p.lay.nodes[lev - 1]) * p.nref * (p.d / 16);
 }
 __device__ __forceinline__ float* level_kscales(const Params& p, void* tree, int lev, int64_t seq,
                                                 int g) {
@@ -89,6 +99,14 @@ __device__ __forceinline__ float fp8_to_float(unsigned char c) {
 }
 __device__ __forceinline__ unsigned char float_to_fp8(float x) {
   return __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+// FP4 E2M1 code (low nibble) <-> float, CUDA's conversions (nearest, ties to
+// even, saturated at +-6).
+__device__ __forceinline__ float fp4_to_float(unsigned int c) {
+  return __half2float(__half(__nv_cvt_fp4_to_halfraw(__nv_fp4_storage_t(c & 0xFu), __NV_E2M1)));
+}
+__device__ __forceinline__ unsigned int float_to_fp4(float x) {
+  return unsigned(__nv_cvt_float_to_fp4(x, __NV_E2M1, cudaRoundNearest)) & 0xFu;
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -106,6 +106,26 @@ __device__ __forceinline__ void load_codes(const unsigned char* row, int lane, f
   }
 }
 
+// The lane's channels of an NVFP4 code row: E2M1 values times their block's
+// E4M3 scale (before the row's scale).  Element e is nibble e & 1 of byte e / 2
+// and belongs to block e / 16.
+template <int NP>
+__device__ __forceinline__ void load_codes_nvfp4(const unsigned char* row,
+                                                 const unsigned char* bsc, int lane,
+                                                 float (&x1)[NP], float (&x2)[NP]) {
+  constexpr int HALF = 32 * NP;
+  if constexpr (NP == 2) {   // elements 2l, 2l + 1 and HALF + 2l, HALF + 2l + 1
+    const unsigned a = row[lane], b = row[HALF / 2 + lane];
+    const float sa = fp8_to_float(bsc[lane >> 3]), sb = fp8_to_float(bsc[(HALF >> 4) + (lane >> 3)]);
+    x1[0] = fp4_to_float(a) * sa; x1[1] = fp4_to_float(a >> 4) * sa;
+    x2[0] = fp4_to_float(b) * sb; x2[1] = fp4_to_float(b >> 4) * sb;
+  } else {                   // elements l and HALF + l
+    const int sh = 4 * (lane & 1);
+    x1[0] = fp4_to_float(row[lane >> 1] >> sh) * fp8_to_float(bsc[lane >> 4]);
+    x2[0] = fp4_to_float(row[(HALF + lane) >> 1] >> sh) * fp8_to_float(bsc[(HALF + lane) >> 4]);
+  }
+}
+
 template <typename T, int NP>
 __device__ __forceinline__ Raw<T, NP> load_raw(const T* row, int lane) {
   constexpr int HALF = 32 * NP;
@@ -157,9 +177,14 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 
   extern __shared__ __align__(16) unsigned char smem[];
   const bool fp8 = p.kfmt == RECSA_KEYS_FP8;                  // FP8 key codes + row scales
+  const bool nv4 = p.kfmt == RECSA_KEYS_NVFP4;                // E2M1 codes + block, row scales
+  const bool lowp = fp8 || nv4;
+  const int rowb = fp8 ? D : (nv4 ? D / 2 + D / 16 : 4 * D);  // staged bytes per key row
   float* kbuf = reinterpret_cast<float*>(smem);               // [krows][D] level key rows
-  const unsigned char* kbyte = smem;                          // (FP8: [krows][D] codes)
-  float* rowsc = reinterpret_cast<float*>(smem + size_t(krows) * D * (fp8 ? 1 : 4));
+  const unsigned char* kbyte = smem;                          // (FP8: [krows][D] codes;
+  unsigned char* kbs = smem + size_t(krows) * (D / 2);        //  NVFP4: [krows][D/2] codes,
+                                                              //  then [krows][D/16] scales)
+  float* rowsc = reinterpret_cast<float*>(smem + size_t(krows) * rowb);
   float* ksc = rowsc + krows;                                 // [krows] FP8 row scales
   float* score = ksc + krows;                                 // [cmax]
   float* wsort = score + cmax;                                // [cmax] weights by rank
@@ -307,7 +332,8 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       const int cc = krows / R;
       const unsigned char* kcodes = level_kcodes(p, const_cast<void*>(tree), lev, seq, g);
       const float* kscales = level_kscales(p, const_cast<void*>(tree), lev, seq, g);
-      const int C16 = fp8 ? D / 16 : D / 4;      // 16-byte pieces per row
+      const unsigned char* kbsc = level_kbscales(p, const_cast<void*>(tree), lev, seq, g);
+      const int C16 = fp8 ? D / 16 : (nv4 ? D / 32 : D / 4);   // 16-byte pieces per row
       for (int i0c = 0; i0c < c; i0c += cc) {
         const int i1c = min(c, i0c + cc);
         const int nrow = (i1c - i0c) * R;
@@ -318,12 +344,25 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           if (fp8)
             cp_async16(const_cast<unsigned char*>(kbyte) + size_t(q) * D + pc * 16,
                        kcodes + row * D + pc * 16);
+          else if (nv4)
+            cp_async16(const_cast<unsigned char*>(kbyte) + size_t(q) * (D / 2) + pc * 16,
+                       kcodes + row * (D / 2) + pc * 16);
           else
             cp_async16(kbuf + size_t(q) * D + pc * 4, keys + row * D + pc * 4);
         }
-        if (fp8)
-          for (int q = ct; q < nrow; q += kZChain * 32)
-            ksc[q] = kscales[int64_t(node(i0c + q / R)) * R + q % R];
+        if (lowp)
+          for (int q = ct; q < nrow; q += kZChain * 32) {
+            const int64_t row = int64_t(node(i0c + q / R)) * R + q % R;
+            ksc[q] = kscales[row];
+            if (nv4) {   // D / 16 block-scale bytes (8 at D = 128, 4 at D = 64)
+              if constexpr (D == 128)
+                *reinterpret_cast<uint2*>(kbs + size_t(q) * 8) =
+                    *reinterpret_cast<const uint2*>(kbsc + row * 8);
+              else
+                *reinterpret_cast<unsigned*>(kbs + size_t(q) * 4) =
+                    *reinterpret_cast<const unsigned*>(kbsc + row * 4);
+            }
+          }
         cp_async_wait_all();
         chain_sync();
         float* rsc = R == 1 ? score + i0c : rowsc;   // row scores
@@ -336,6 +375,9 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
             float x1[NP], x2[NP];
             if (fp8)
               load_codes<NP>(kbyte + size_t(q) * D, lane, x1, x2);
+            else if (nv4)
+              load_codes_nvfp4<NP>(kbyte + size_t(q) * (D / 2), kbs + size_t(q) * (D / 16), lane,
+                                   x1, x2);
             else
               load_pairs<NP>(kbuf + size_t(q) * D, lane, x1, x2);
             sc4[r] = 0.f;
@@ -354,7 +396,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 #pragma unroll
             for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
             const int q = q0 + lane * kZChain;
-            if (q < nrow) rsc[q] = v * p.inv_sqrt_d * (fp8 ? ksc[q] : 1.f);
+            if (q < nrow) rsc[q] = v * p.inv_sqrt_d * (lowp ? ksc[q] : 1.f);
           }
         }
         chain_sync();
@@ -515,10 +557,11 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   if (cmax > kZMaxCand) return cudaErrorNotSupported;   // the generic kernel serves it
   const int kmax = int(kk < cmax ? kk : cmax);
   // level key rows staged per chunk (FP8 rows are a quarter of the bytes)
-  const bool fp8 = p.kfmt == RECSA_KEYS_FP8;
-  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, fp8 ? 4 * kZMaxRows : kZMaxRows));
+  const bool lowp = p.kfmt != RECSA_KEYS_F32;
+  const int rowb = p.kfmt == RECSA_KEYS_FP8 ? D : (lowp ? D / 2 + D / 16 : 4 * D);
+  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, lowp ? 4 * kZMaxRows : kZMaxRows));
   if (krows < p.nref) return cudaErrorNotSupported;
-  const size_t bytes = size_t(krows) * D * (fp8 ? 1 : 4) +
+  const size_t bytes = size_t(krows) * rowb +
                        (2 * size_t(krows) + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
                        (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + kZChain) * 4;
   if (bytes > 227 * 1024) return cudaErrorNotSupported;

@@ -26,6 +26,7 @@ MODE_ZHA = 1
 MODE_GROUP = 2
 KEYS_F32 = 0
 KEYS_FP8 = 1
+KEYS_NVFP4 = 2
 KEEP_ALL = 2**31 - 1
 MAX_LEVELS = 16
 TRACE_MAX_K = 64
@@ -95,7 +96,7 @@ class Geometry:
     mode: int = 0          # MODE_RECSA, MODE_ZHA or MODE_GROUP
     top_p: float = 0.0     # ZHA routing mass
     n_ref: int = 1         # reference queries per pooler (ZHA mode for n_ref > 1)
-    key_format: int = 0    # KEYS_F32 or KEYS_FP8 (ZHA mode)
+    key_format: int = 0    # KEYS_F32, KEYS_FP8 or KEYS_NVFP4 (ZHA mode)
 
     def c(self) -> CGeometry:
         return CGeometry(self.dtype, self.head_dim, self.n_q_heads, self.n_kv_heads,

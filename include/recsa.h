@@ -70,6 +70,7 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
 /* recsa_geometry.key_format: storage of the summary keys */
 #define RECSA_KEYS_F32 0 /* fp32 rows */
 #define RECSA_KEYS_FP8 1 /* FP8 E4M3 codes with one fp32 scale per row (ZHA mode only) */
+#define RECSA_KEYS_NVFP4 2 /* E2M1 codes, E4M3 scale per 16, fp32 scale per row (ZHA only) */
 
 /* Device error flags in the tree header (recsa_tree_error). */
 #define RECSA_DEVERR_APPEND_FULL 0x1u /* recsa_append on a full sequence */
@@ -113,7 +114,11 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   key cache ("Subquadratic Attention with a Hierarchical Tree-Structured
  *   Indexer", Figure 16 caption).  A parent key pools its children's stored
  *   (decoded) keys; values stay fp32; the routing score is
- *   scale * (q . codes) / sqrt(d).
+ *   scale * (q . codes) / sqrt(d).  RECSA_KEYS_NVFP4 stores E2M1 codes (two
+ *   per byte, the lower element in the low nibble) with one E4M3 scale per 16
+ *   elements and one fp32 scale per row: row scale = max|key| / (6 * 448),
+ *   block scale = E4M3(block max / (6 * row scale)), code = E2M1(key /
+ *   (block scale * row scale)), nearest, ties to even, saturated.
  */
 typedef struct recsa_geometry {
   int32_t dtype;        /* RECSA_DTYPE_F32 or RECSA_DTYPE_BF16: K, V, Q, O, k_new, v_new */
@@ -131,7 +136,7 @@ typedef struct recsa_geometry {
   int64_t capacity;     /* tokens each sequence's K/V cache (and tree) can hold, < 2^31 */
   float top_p;          /* ZHA: routing mass in (0, 1]; ignored in RECSA mode */
   int32_t n_ref;        /* reference queries per pooler: 0 or 1 = one; 2..64 (ZHA mode only) */
-  int32_t key_format;   /* RECSA_KEYS_F32 or RECSA_KEYS_FP8 (ZHA mode only) */
+  int32_t key_format;   /* RECSA_KEYS_F32, _FP8 or _NVFP4 (the last two: ZHA mode only) */
   int32_t reserved;     /* must be 0 */
 } recsa_geometry;
 
@@ -150,7 +155,9 @@ recsa_status recsa_num_levels(const recsa_geometry* geom, int64_t length, int32_
  * reach, and per level l: keys [batch][n_kv_heads][n_l][n_ref][head_dim] and
  * values [batch][n_kv_heads][n_l][head_dim] in fp32, n_l the level's node
  * count at capacity.  With RECSA_KEYS_FP8 the keys are one byte per element,
- * followed by their fp32 scales [batch][n_kv_heads][n_l][n_ref].
+ * followed by their fp32 scales [batch][n_kv_heads][n_l][n_ref]; with
+ * RECSA_KEYS_NVFP4 half a byte per element, then the E4M3 block scales
+ * [batch][n_kv_heads][n_l][n_ref][head_dim / 16], then the fp32 row scales.
  */
 recsa_status recsa_tree_bytes(const recsa_geometry* geom, size_t* bytes);
 

@@ -4,6 +4,8 @@ compare with the oracle on the same seeded inputs.
 Tolerances:
   * bf16 inputs: max-abs 2e-2 and mean-abs 2e-3 on outputs and tree summaries
     against the float64 oracle fed the same bf16 values (the target bound);
+    the outputs are written in bf16, so the max-abs bound applies beyond that
+    final rounding (half a bf16 ulp of the value, 1/64 at magnitude 8);
   * fp32 inputs: max-abs 2e-4, mean-abs 2e-5 (fp32 dot products of length
     <= 128 and sums over <= ~2000 softmax entries: a few 1e-6 relative, with
     two orders of margin);
@@ -99,17 +101,33 @@ def gaps_clear(res: dict, k: int, gap: float = GAP) -> bool:
     return True
 
 
+def half_ulp_bf16(x) -> np.ndarray:
+    """Half a bf16 unit in the last place at |x| (8 significant bits): the
+    rounding error of writing x as bf16."""
+    a = np.abs(np.asarray(x, np.float64))
+    _, e = np.frexp(np.maximum(a, 2.0 ** -126))
+    return np.ldexp(1.0, e - 1 - 8)
+
+
 class Stats:
+    """Error statistics of GPU values against oracle values.  For bf16 runs the
+    GPU writes its outputs as bf16, so the max-abs bound applies to the error
+    beyond that final rounding (half a bf16 ulp of the oracle value): outputs
+    of magnitude 8 or more cannot be written closer than 1/64 in bf16."""
+
     def __init__(self):
         self.max_abs = 0.0
+        self.max_excess = 0.0
         self.sum_abs = 0.0
         self.n = 0
         self.clear = 0
         self.near_tie = 0
 
     def add(self, a, b):
-        e = np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))
+        b = np.asarray(b, np.float64)
+        e = np.abs(np.asarray(a, np.float64) - b)
         self.max_abs = max(self.max_abs, float(e.max()))
+        self.max_excess = max(self.max_excess, float(np.max(e - half_ulp_bf16(b))))
         self.sum_abs += float(e.sum())
         self.n += e.size
 
@@ -119,9 +137,11 @@ class Stats:
 
     def check(self, dtype, what=""):
         mx, mn = TOL[dtype]
-        print(f"{what}: max-abs {self.max_abs:.3e} mean-abs {self.mean_abs:.3e} "
+        worst = self.max_excess if dtype == torch.bfloat16 else self.max_abs
+        print(f"{what}: max-abs {self.max_abs:.3e} (beyond bf16 output rounding "
+              f"{self.max_excess:.3e}) mean-abs {self.mean_abs:.3e} "
               f"clear {self.clear} near-tie {self.near_tie}")
-        assert self.max_abs <= mx, f"{what}: max-abs {self.max_abs:.3e} > {mx}"
+        assert worst <= mx, f"{what}: max-abs {worst:.3e} > {mx}"
         assert self.mean_abs <= mn, f"{what}: mean-abs {self.mean_abs:.3e} > {mn}"
 
 
@@ -309,3 +329,49 @@ def read_tree_level_fp8(g: R.Geometry, tree: torch.Tensor, lev: int):
 
 
 E4M3_TABLE = np.array([oracle.e4m3_decode(c) for c in range(256)])
+
+
+def read_tree_level_nvfp4(g: R.Geometry, tree: torch.Tensor, lev: int):
+    """(codes uint8 [batch, Hkv, n_l, n_ref, d/2], block scales uint8 [..., d/16],
+    row scales fp32 [batch, Hkv, n_l, n_ref], vals fp32 [batch, Hkv, n_l, d])
+    of one level of an NVFP4-key tree."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    kk = min(g.k, g.capacity)
+    rows = min(max(g.branching * kk + g.branching, g.leaf_block * kk + g.window + g.leaf_block),
+               g.capacity + g.branching + 1)
+    if g.mode == R.MODE_ZHA:
+        rows = max(rows, g.capacity + 1)
+    off = up(256 + rows * (g.head_dim // 2) * 8)
+    span = g.leaf_block
+    nr = max(g.n_ref, 1)
+    d = g.head_dim
+    for l in range(1, lev + 1):
+        n = g.capacity // span
+        nrows = g.batch * g.n_kv_heads * n
+        c_off = off
+        b_off = up(c_off + nrows * nr * d // 2)
+        s_off = up(b_off + nrows * nr * d // 16)
+        v_off = up(s_off + nrows * nr * 4)
+        if l == lev:
+            shp = (g.batch, g.n_kv_heads, n, nr)
+            codes = tree[c_off:c_off + nrows * nr * d // 2].view(*shp, d // 2)
+            bsc = tree[b_off:b_off + nrows * nr * d // 16].view(*shp, d // 16)
+            rsc = tree[s_off:s_off + nrows * nr * 4].view(torch.float32).view(*shp)
+            vals = tree[v_off:v_off + nrows * d * 4].view(torch.float32).view(
+                g.batch, g.n_kv_heads, n, d)
+            return codes, bsc, rsc, vals
+        off = up(v_off + nrows * d * 4)
+        span *= g.branching
+    raise ValueError(lev)
+
+
+E2M1_TABLE = np.array([oracle.e2m1_decode(c) for c in range(16)])
+
+
+def decode_nvfp4(codes: np.ndarray, bsc: np.ndarray, rsc: np.ndarray) -> np.ndarray:
+    """Stored key values [..., d] from NVFP4 codes [..., d/2], block scales
+    [..., d/16] and row scales [...] (numpy)."""
+    c = codes.astype(np.int64)
+    el = np.stack([E2M1_TABLE[c & 0xF], E2M1_TABLE[c >> 4]], axis=-1).reshape(*c.shape[:-1], -1)
+    bs = np.repeat(E4M3_TABLE[bsc.astype(np.int64)], 16, axis=-1)
+    return el * bs * rsc[..., None]

@@ -68,6 +68,7 @@ def test_status_strings(lib):
     dict(mode=R.MODE_ZHA, top_p=0.9, n_ref=16), dict(n_ref=0), dict(n_ref=1),
     dict(mode=R.MODE_ZHA, top_p=0.9, key_format=R.KEYS_FP8),
     dict(mode=R.MODE_ZHA, top_p=0.9, n_ref=16, key_format=R.KEYS_FP8),
+    dict(mode=R.MODE_ZHA, top_p=0.9, n_ref=4, key_format=R.KEYS_NVFP4),
 ])
 def test_valid_geometries(lib, kw):
     R.recsa_validate(geo(**kw))
@@ -80,7 +81,7 @@ def test_valid_geometries(lib, kw):
     dict(mode=3), dict(mode=-1), dict(n_ref=2), dict(mode=R.MODE_GROUP, n_ref=4),
     dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=65), dict(n_ref=-1), dict(mode=R.MODE_ZHA, top_p=0.0),
     dict(key_format=R.KEYS_FP8), dict(mode=R.MODE_GROUP, key_format=R.KEYS_FP8),
-    dict(mode=R.MODE_ZHA, top_p=0.5, key_format=2), dict(mode=R.MODE_ZHA, top_p=1.5),
+    dict(mode=R.MODE_ZHA, top_p=0.5, key_format=3), dict(key_format=R.KEYS_NVFP4), dict(mode=R.MODE_ZHA, top_p=1.5),
     dict(mode=R.MODE_ZHA, top_p=float("nan")),
 ])
 def test_invalid_geometries(lib, kw):
@@ -115,6 +116,9 @@ def expected_tree_bytes(g: R.Geometry) -> int:
         nr = max(g.n_ref, 1)
         if g.key_format == R.KEYS_FP8:   # one byte per key element, then fp32 row scales
             total += up(rows * nr * g.head_dim) + up(rows * nr * 4) + up(row_bytes)
+        elif g.key_format == R.KEYS_NVFP4:   # half a byte, E4M3 per 16, fp32 per row
+            total += (up(rows * nr * g.head_dim // 2) + up(rows * nr * g.head_dim // 16) +
+                      up(rows * nr * 4) + up(row_bytes))
         else:
             total += up(row_bytes * nr) + up(row_bytes)
         span *= g.branching
@@ -126,7 +130,9 @@ def expected_tree_bytes(g: R.Geometry) -> int:
                                 dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=16),
                                 dict(mode=R.MODE_ZHA, top_p=0.5, key_format=R.KEYS_FP8),
                                 dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=4,
-                                     key_format=R.KEYS_FP8)])
+                                     key_format=R.KEYS_FP8),
+                                dict(mode=R.MODE_ZHA, top_p=0.5, n_ref=3,
+                                     key_format=R.KEYS_NVFP4)])
 def test_tree_bytes(lib, kw):
     g = geo(**kw)
     assert R.recsa_tree_bytes(g) == expected_tree_bytes(g)

@@ -19,9 +19,9 @@ import oracle
 from hierarchical_sparse_attention_recsa_b200 import build_lib, synth
 from hierarchical_sparse_attention_recsa_b200 import recsa as R
 
-from recsa_testlib import (E4M3_TABLE, Stats, alloc_tree, check_query_zha, geometry,
-                           oracle_geometry, parse_trace, read_tree_level, read_tree_level_fp8,
-                           to_np)
+from recsa_testlib import (E4M3_TABLE, Stats, alloc_tree, check_query_zha, decode_nvfp4,
+                           geometry, oracle_geometry, parse_trace, read_tree_level,
+                           read_tree_level_fp8, read_tree_level_nvfp4, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -477,11 +477,11 @@ def test_zha_multiref_full_mass_is_dense(rope, zha_impl):
 # Low-precision router keys (FP8 E4M3 with one scale per key row)
 # ---------------------------------------------------------------------------
 
-def _setup_fp8(w, lens, capacity, top_p, n_ref, seed, k=None, rope=1):
+def _setup_fp8(w, lens, capacity, top_p, n_ref, seed, k=None, rope=1, key_format=R.KEYS_FP8):
     batch = len(lens)
     g = geometry(w, capacity, batch, k=k, rope=rope, top_p=top_p)
     g.n_ref = n_ref
-    g.key_format = R.KEYS_FP8
+    g.key_format = key_format
     K, V, r = synth.make_kv(w, capacity, seed=seed, device="cpu", batch=batch)
     Rq = _refs(r, n_ref, seed + 1000) if n_ref > 1 else r.reshape(1, -1).contiguous()
     Kd, Vd, Rd = K.cuda(), V.cuda(), Rq.cuda()
@@ -492,12 +492,13 @@ def _setup_fp8(w, lens, capacity, top_p, n_ref, seed, k=None, rope=1):
 
 
 def _fp8_trees(g, K, V, Rq, lens):
+    build = (oracle.build_tree_nvfp4_multi if g.key_format == R.KEYS_NVFP4
+             else oracle.build_tree_fp8_multi)
     out = {}
     for s, L in enumerate(lens):
         for h in range(g.n_kv_heads):
             Kh, Vh = to_np(K[s, h, :L]), to_np(V[s, h, :L])
-            levels = oracle.build_tree_fp8_multi(Kh, Vh, Rq.double().numpy(), g.leaf_block,
-                                                 g.branching)
+            levels = build(Kh, Vh, Rq.double().numpy(), g.leaf_block, g.branching)
             if Rq.shape[0] == 1:
                 levels = [(kk[:, 0], vv) for kk, vv in levels]
                 out[(s, h)] = (Kh, Vh, oracle.FullTree(levels))
@@ -669,3 +670,120 @@ def test_zha_fp8_full_mass_is_dense(zha_impl):
                                                 to_np(V[0, 0]), rope=True, rope_base=w.rope_base)
             st.add(O_[0, t, h], ref)
     st.check(torch.float32, f"zha {zha_impl} fp8 full mass")
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 router keys (E2M1 codes, E4M3 scale per 16, fp32 scale per row)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n_ref", [1, 3])
+def test_zha_nvfp4_tree(n_ref):
+    """Level-1 keys decode to the oracle's NVFP4 rows except where float32 and
+    float64 pooling straddle a rounding midpoint (of an element, or of a block
+    scale, which moves its 16 elements together); row scales agree to float32
+    rounding; every stored element is an E2M1 value times its block scale."""
+    L = TINY.length
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(TINY, [L], L, 0.7, n_ref, seed=90,
+                                               key_format=R.KEYS_NVFP4)
+    Kh, Vh = to_np(K[0, 0]), to_np(V[0, 0])
+    Rn = Rq.double().numpy()
+    levels = oracle.build_tree_nvfp4_multi(Kh, Vh, Rn, g.leaf_block, g.branching)
+    for lev in range(1, len(levels) + 1):
+        codes, bsc, rsc, vals = read_tree_level_nvfp4(g, tree, lev)
+        n = levels[lev - 1][0].shape[0]
+        got = decode_nvfp4(codes[0, 0, :n].cpu().numpy(), bsc[0, 0, :n].cpu().numpy(),
+                           rsc[0, 0, :n].cpu().numpy().astype(np.float64))
+        want = levels[lev - 1][0]
+        if lev == 1:
+            amax = np.abs(want).max(axis=-1)
+            np.testing.assert_allclose(rsc[0, 0, :n].cpu().numpy(), amax / (6 * 448), rtol=1e-5)
+        frac = float(np.mean(np.abs(got - want) > 1e-6 * np.abs(want).max(axis=-1,
+                                                                          keepdims=True)))
+        assert frac <= (0.03 if lev == 1 else 0.08), (lev, frac)
+        np.testing.assert_allclose(vals[0, 0, :n].cpu().numpy(), levels[lev - 1][1],
+                                   atol=1e-5 if lev > 1 else 1e-6)
+
+
+@pytest.mark.parametrize("n_ref,top_p", [(1, 0.7), (4, 0.9)])
+def test_zha_nvfp4_decode_tiny(n_ref, top_p, zha_impl):
+    L, nq = TINY.length, 64
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(TINY, [L], L, top_p, n_ref, seed=92, k=ZK,
+                                               key_format=R.KEYS_NVFP4)
+    trees = _fp8_trees(g, K, V, Rq, [L])
+    pos = torch.full((1, nq), L - 1, dtype=torch.int64)
+    Q, _, _ = synth.make_queries(TINY, K, pos, seed=93, n_needles=8)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((1, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens = torch.tensor([L], dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    Kh, Vh, src = trees[(0, 0)]
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    for i in range(nq):
+        for h in range(g.n_q_heads):
+            check_query_zha(st, O_[0, i, h], tr[0, i, h], to_np(Q[0, i, h]), L - 1, Kh, Vh, src,
+                            og, top_p, g.k)
+    st.check(torch.float32, f"zha {zha_impl} nvfp4 R={n_ref} decode tiny")
+    assert st.clear > 0.5 * nq * g.n_q_heads
+
+
+def test_zha_nvfp4_decode_model_small(zha_impl):
+    lens, top_p = [20000, 13001], 0.9
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(MODEL, lens, 20480, top_p, 1, seed=94,
+                                               key_format=R.KEYS_NVFP4)
+    trees = _fp8_trees(g, K, V, Rq, lens)
+    nq = 2
+    pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(MODEL, K, pos, seed=95, n_needles=2)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for i in range(nq):
+            for h in range(g.n_q_heads):
+                Kh, Vh, src = trees[(s, h // G)]
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} nvfp4 decode model small")
+
+
+def test_zha_nvfp4_append_matches_build():
+    w, top_p = MODEL, 0.9
+    lens0 = [4000, 4031]
+    steps = 100
+    cap = 4096 + 256
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(w, lens0, cap, top_p, 2, seed=96,
+                                               key_format=R.KEYS_NVFP4)
+    Kw, Vw = Kd.clone(), Vd.clone()
+    Kw[0, :, 4000:] = 0
+    Vw[0, :, 4000:] = 0
+    Kw[1, :, 4031:] = 0
+    Vw[1, :, 4031:] = 0
+    lens_d = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        R.recsa_append(g, Kw, Vw, kn, vn, lens_d, Rd, 0, tree)
+    new_lens = [L + steps for L in lens0]
+    fresh = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, new_lens, Rd, 0, fresh)
+    torch.cuda.synchronize()
+    for lev in range(1, R.recsa_num_levels(g, max(new_lens)) + 1):
+        a = read_tree_level_nvfp4(g, tree, lev)
+        b = read_tree_level_nvfp4(g, fresh, lev)
+        for s in range(2):
+            n = new_lens[s] // (g.leaf_block * g.branching ** (lev - 1))
+            for x, y in zip(a, b):
+                assert torch.equal(x[s, :, :n], y[s, :, :n]), lev
