@@ -359,6 +359,9 @@ def run_recsa(args, rank, world, dev):
         out["zha_multiref_fp8"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
                                               hbm_gbs, peak_kind, R.MODE_ZHA, False,
                                               n_ref=ZHA_N_REF, key_format=R.KEYS_FP8)
+        out["zha_multiref_nvfp4"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
+                                                hbm_gbs, peak_kind, R.MODE_ZHA, False,
+                                                n_ref=ZHA_N_REF, key_format=R.KEYS_NVFP4)
     if not args.no_group:
         out["group"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
                                    peak_kind, R.MODE_GROUP, cpu_leg)
@@ -417,11 +420,12 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     dec_ms = sum(elapsed(a, b) for a, b in ev) / n
     tr = traces.cpu().numpy()
     G = w.n_q_heads // w.n_kv_heads
+    d = w.head_dim   # stored bytes of one key row
+    key_bytes = {R.KEYS_F32: 4 * d, R.KEYS_FP8: d + 4, R.KEYS_NVFP4: d // 2 + d // 16 + 4}[key_format]
     nb = [counts.decode_bytes_from_trace(tr[i], np.full(batch, L), w.leaf_block, w.branching,
                                          w.window, G, w.head_dim, elem_bytes(w), w.k,
                                          summary_values=not zha, keys_per_node=n_ref,
-                                         key_row_bytes=w.head_dim + 4 if key_format else 0
-                                         )["bytes"] for i in range(n)]
+                                         key_row_bytes=key_bytes)["bytes"] for i in range(n)]
     kept = tr[..., 4 + 16:4 + 16 + R.recsa_num_levels(g, L)].astype(np.float64)
     nbytes = float(np.mean(nb))
     achieved = nbytes / (dec_ms / 1e3) / 1e9
@@ -436,7 +440,8 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     if zha:
         res["top_p"] = ZHA_TOP_P
         res["n_ref"] = n_ref
-        res["keys"] = "fp8_e4m3 + fp32 row scale" if key_format else "fp32"
+        res["keys"] = {R.KEYS_F32: "fp32", R.KEYS_FP8: "fp8_e4m3 + fp32 row scale",
+                       R.KEYS_NVFP4: "nvfp4 (e2m1, e4m3 per 16, fp32 per row)"}[key_format]
     del tree, traces
     torch.cuda.empty_cache()
     if cpu:
