@@ -38,13 +38,22 @@ constexpr int kZThreads = 512;
 constexpr int kZWarps = kZThreads / 32;
 constexpr int kZChain = 12;         // chain warps; the others attend the window first
 constexpr int kZMaxCand = kZChain * 32;   // one chain thread per candidate
-constexpr int kZMaxRows = 256;            // level key rows staged at once
+constexpr size_t kZStageBytes = 180 * 1024;   // shared memory for a level's staged key rows
 constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
 constexpr int kZBarChain = 1;       // named barrier of the chain warps
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
+// 4- and 8-byte copies (row scales, NVFP4 block scales), also asynchronous.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;\n" ::: "memory");
@@ -350,17 +359,15 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           else
             cp_async16(kbuf + size_t(q) * D + pc * 4, keys + row * D + pc * 4);
         }
-        if (lowp)
+        if (lowp)   // row scales (and NVFP4 block scales) ride with the code rows
           for (int q = ct; q < nrow; q += kZChain * 32) {
             const int64_t row = int64_t(node(i0c + q / R)) * R + q % R;
-            ksc[q] = kscales[row];
+            cp_async4(ksc + q, kscales + row);
             if (nv4) {   // D / 16 block-scale bytes (8 at D = 128, 4 at D = 64)
               if constexpr (D == 128)
-                *reinterpret_cast<uint2*>(kbs + size_t(q) * 8) =
-                    *reinterpret_cast<const uint2*>(kbsc + row * 8);
+                cp_async8(kbs + size_t(q) * 8, kbsc + row * 8);
               else
-                *reinterpret_cast<unsigned*>(kbs + size_t(q) * 4) =
-                    *reinterpret_cast<const unsigned*>(kbsc + row * 4);
+                cp_async4(kbs + size_t(q) * 4, kbsc + row * 4);
             }
           }
         cp_async_wait_all();
@@ -559,7 +566,9 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   // level key rows staged per chunk (FP8 rows are a quarter of the bytes)
   const bool lowp = p.kfmt != RECSA_KEYS_F32;
   const int rowb = p.kfmt == RECSA_KEYS_FP8 ? D : (lowp ? D / 2 + D / 16 : 4 * D);
-  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, lowp ? 4 * kZMaxRows : kZMaxRows));
+  // as many (candidate, reference) rows per chunk as the staging budget holds
+  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref,
+                                          int64_t(kZStageBytes / size_t(rowb + 8))));
   if (krows < p.nref) return cudaErrorNotSupported;
   const size_t bytes = size_t(krows) * rowb +
                        (2 * size_t(krows) + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
