@@ -14,6 +14,16 @@
 // Scores are one warp per (head, entry) dot product over fp32 rows with the
 // rotation folded in; the online-softmax state (max, sum, acc[d]) of each head
 // lives in registers of the threads that own its channels.
+//
+// The same kernel serves the selection variants of the geometry's mode:
+//   * RECSA_MODE_GROUP: the G heads' scores give one group score per candidate
+//     (the sum of the heads' softmax probabilities over the level's
+//     candidates), ranked once and shared by the heads;
+//   * RECSA_MODE_ZHA ("Subquadratic Attention with a Hierarchical
+//     Tree-Structured Indexer", Figure 3 caption): un-rotated routing scores
+//     (the best of a node's reference keys, decoded from FP8 or NVFP4 when the
+//     keys are stored so), a per-head top-p set capped at k, no summaries in
+//     the softmax, and the reached leaves plus the window at true positions.
 #include "recsa_internal.cuh"
 
 namespace recsa {
