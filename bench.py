@@ -183,6 +183,24 @@ def elapsed(a, b):
     return a.elapsed_time(b)
 
 
+def max_over_ranks(ms: float, world: int) -> float:
+    """The largest of the ranks' device times (every rank calls it, in the same
+    order); one rank: unchanged.  The tensor lives where the process group's
+    backend communicates (CUDA for NCCL, host memory for gloo)."""
+    if world == 1:
+        return ms
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed (weak scaling: the
+    same number per rank) over the slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 def make_prefill_queries(w, K, q0, L, chunk=65536):
     Q = torch.empty((1, L - q0, w.n_q_heads, w.head_dim), dtype=w.dtype, device="cuda")
     for c0 in range(q0, L, chunk):
@@ -265,11 +283,8 @@ def run_recsa(args, rank, world, dev):
     torch.cuda.synchronize()
     app_ms = sum(elapsed(e[0], e[1]) for e in ev3) / K_steps
     two_dec_ms = sum(elapsed(e[1], e[2]) for e in ev3) / K_steps
-    if world > 1:
-        t = torch.tensor([step_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(t.item())
-    value = batch * K_steps * world / (step_ms / 1e3)
+    step_ms = max_over_ranks(step_ms, world)
+    value = job_rate(batch * K_steps, world, step_ms)
 
     # algorithmic bytes of the decode launches, from the traces
     tr = traces.cpu().numpy()
@@ -302,11 +317,8 @@ def run_recsa(args, rank, world, dev):
             ev2[i][1].record(stream)
         torch.cuda.synchronize()
         e2e_ms = sum(elapsed(a, b) for a, b in ev2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        return {"value": batch * K_steps * world / (e2e_ms / 1e3), "unit": "queries/s",
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        return {"value": job_rate(batch * K_steps, world, e2e_ms), "unit": "queries/s",
                 "h2d_bytes_per_step": int(Qd.numel() * 2 + knd.numel() * 2 + vnd.numel() * 2),
                 "d2h_bytes_per_step": int(O.numel() * 2)}
 
