@@ -179,6 +179,36 @@ def measured_traffic(workload, L, batch):
     return float(fields["traffic_bytes_per_launch"])
 
 
+VARIANT_SOURCES = ["zha_attend.cu", "decode_cluster.cu", "rows.cuh", "pool.cuh",
+                   "recsa_internal.cuh"]
+VARIANT_PROFILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                               "selection_variants_qwen3-4b-524k_traffic.md")
+
+
+def measured_variant_traffic(leg, workload, L, batch):
+    """DRAM bytes per launch of a selection-variant leg from the committed ncu
+    capture of the same workload, or None (other workload, or the kernel
+    sources changed since the capture)."""
+    if workload != WORKLOAD or L != synth.WORKLOADS[WORKLOAD].length or \
+            batch != synth.WORKLOADS[WORKLOAD].batch or not os.path.exists(VARIANT_PROFILE):
+        return None
+    fields = {}
+    for line in open(VARIANT_PROFILE):
+        if ":" in line and (line.startswith("traffic_bytes_per_launch[") or
+                            line.startswith("source_sha256")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(R.__file__)), "csrc")
+    for f in VARIANT_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    key = f"traffic_bytes_per_launch[{leg}]"
+    if fields.get("source_sha256") != h.hexdigest() or key not in fields:
+        return None
+    return float(fields[key])
+
+
 def elapsed(a, b):
     return a.elapsed_time(b)
 
@@ -364,19 +394,21 @@ def run_recsa(args, rank, world, dev):
     cpu_leg = rank == 0 and world == 1 and not args.no_cpu
     if not args.no_zha:
         out["zha"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
-                                 peak_kind, R.MODE_ZHA, cpu_leg)
+                                 peak_kind, R.MODE_ZHA, cpu_leg, leg="zha")
         out["zha_multiref"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
                                           hbm_gbs, peak_kind, R.MODE_ZHA, cpu_leg,
-                                          n_ref=ZHA_N_REF)
+                                          n_ref=ZHA_N_REF, leg="zha_multiref")
         out["zha_multiref_fp8"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
                                               hbm_gbs, peak_kind, R.MODE_ZHA, False,
-                                              n_ref=ZHA_N_REF, key_format=R.KEYS_FP8)
+                                              n_ref=ZHA_N_REF, key_format=R.KEYS_FP8,
+                                              leg="zha_multiref_fp8")
         out["zha_multiref_nvfp4"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
                                                 hbm_gbs, peak_kind, R.MODE_ZHA, False,
-                                                n_ref=ZHA_N_REF, key_format=R.KEYS_NVFP4)
+                                                n_ref=ZHA_N_REF, key_format=R.KEYS_NVFP4,
+                                                leg="zha_multiref_nvfp4")
     if not args.no_group:
         out["group"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
-                                   peak_kind, R.MODE_GROUP, cpu_leg)
+                                   peak_kind, R.MODE_GROUP, cpu_leg, leg="group")
     return out
 
 
@@ -394,7 +426,7 @@ def reference_queries(r, n_ref, seed=7):
 
 
 def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kind, mode, cpu,
-                n_ref=1, key_format=0):
+                n_ref=1, key_format=0, leg=""):
     """A selection variant on the same cache: its own tree (same pooling),
     then the batch's decode queries at t = L - 1, timed per launch like the
     main decode.  MODE_ZHA: top-p expansion, exact tokens of the reached
@@ -448,7 +480,8 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
            "exact_tokens_mean": float(tr[..., 3].mean()),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                         "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
-                        "bytes_per_launch": nbytes, "traffic": None}}
+                        "bytes_per_launch": nbytes,
+                        "traffic": measured_variant_traffic(leg, args.workload, L, batch)}}
     if zha:
         res["top_p"] = ZHA_TOP_P
         res["n_ref"] = n_ref
