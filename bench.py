@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -62,7 +63,8 @@ class Clocks:
 
     def __init__(self, device: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device}.csv")
+        self.path = os.path.join(tempfile.gettempdir(),
+                                 f"recsa_clocks_rank{device}_{os.getpid()}.csv")
         self.sel = []
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid).lower()
