@@ -275,6 +275,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   uint64_t* mb_win = mb_lev + 6;                                   // [kWinRing]
   uint64_t* mb_tok = mb_win + kWinRing;                            // [HPC][NRH] leaf arrived
   uint64_t* mb_empty = mb_tok + HPC * NRH;                         // [HPC][NRH] slot consumed
+  uint64_t* mb_never = mb_lev + 63;   // no thread ever arrives (expiry test, last mbarrier slot)
   float* qf = reinterpret_cast<float*>(smem + pl.qf);       // [G][D] raw query
   float* qtok = reinterpret_cast<float*>(smem + pl.qtok);   // [G][D] rotated to n0 - 1
   float* qlev = reinterpret_cast<float*>(smem + pl.qlev);   // [levels][HPC][D] rotated to c_l
@@ -362,6 +363,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     mbar_init(mb_val, 1);
     mbar_init(mb_kept, HPC);
     mbar_init(mb_folded, 1);
+    mbar_init(mb_never, 1);
     mbar_init(mb_ready, unsigned(S));
     mbar_init(mb_ready + 1, unsigned(S));
     for (int i = 0; i < kWinRing; ++i) mbar_init(mb_win + i, 1);
@@ -980,6 +982,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (tid == 0) mbar_arrive(mb_folded);
     }
     if (top > 0) token_pass();
+    // Expiry test: with the work done, one more bounded wait on a barrier that
+    // no thread arrives at; it runs out and the launch reports the timeout.
+    if (p.test_expire) mbar_wait(mb_never, 0u, timed_out);
   };
 
   // The producer warp issues the chain's copies as soon as their addresses

@@ -129,6 +129,9 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
     if ((1 << sh) == p->b) p->bsh = sh;
   }
   p->inv_sqrt_d = 1.0f / sqrtf(float(g->head_dim));
+  // tests of the bounded waits: the decode kernel's chain threads end with a
+  // wait that nothing completes, which must expire into RECSA_DEVERR_WAIT_TIMEOUT
+  p->test_expire = getenv("RECSA_TEST_EXPIRE_WAIT") != nullptr;
   return RECSA_OK;
 }
 

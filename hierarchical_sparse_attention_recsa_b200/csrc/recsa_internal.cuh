@@ -41,6 +41,7 @@ struct Params {
   int32_t nref;       // reference queries per pooler (keys per node), >= 1
   int32_t kfmt;       // RECSA_KEYS_F32, RECSA_KEYS_FP8 or RECSA_KEYS_NVFP4
   int32_t kcb;        // code bytes per key row (FP8: d, NVFP4: d / 2)
+  int32_t test_expire;   // decode: one extra wait nothing completes (bounded-wait tests)
   int64_t cap;
   float inv_sqrt_d;
   TreeLayout lay;

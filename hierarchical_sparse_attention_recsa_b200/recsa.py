@@ -31,6 +31,7 @@ KEEP_ALL = 2**31 - 1
 MAX_LEVELS = 16
 TRACE_MAX_K = 64
 DEVERR_APPEND_FULL = 0x1
+DEVERR_WAIT_TIMEOUT = 0x2
 
 STATUS = {
     0: "RECSA_OK",

@@ -439,3 +439,42 @@ def test_decode_empty_sequence_gives_zeros():
     torch.cuda.synchronize()
     assert torch.all(O[0] == 0)
     assert torch.all(O[1] != 7.0)
+
+
+def test_bounded_wait_expiry_reports_status_and_context_stays_usable():
+    """Failure detection without a fault: RECSA_TEST_EXPIRE_WAIT makes the
+    decode kernel's chain threads end with a wait on a barrier that nothing
+    completes.  The wait runs out (50 ms), the launch finishes, the tree header
+    carries RECSA_DEVERR_WAIT_TIMEOUT, and the next launch runs normally."""
+    w = MODEL
+    lens = [3000, 2500]
+    g, K, V, r, Kd, Vd, rd, tree = _setup(w, lens, 4096, seed=14)
+    pos = torch.tensor([[L - 1] for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(w, K, pos, seed=15)
+    Qd = Q.cuda()
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    O1, O2 = torch.empty_like(Qd), torch.empty_like(Qd)
+    assert R.recsa_tree_error(g, tree) == 0
+    os.environ["RECSA_TEST_EXPIRE_WAIT"] = "1"
+    try:
+        R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, 1, O1)
+        torch.cuda.synchronize()
+    finally:
+        os.environ.pop("RECSA_TEST_EXPIRE_WAIT", None)
+    assert R.recsa_tree_error(g, tree, clear=True) & R.DEVERR_WAIT_TIMEOUT
+    assert R.recsa_tree_error(g, tree) == 0
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, 1, O2)
+    torch.cuda.synchronize()
+    assert R.recsa_tree_error(g, tree) == 0
+    # the expiring wait came after the work: both launches wrote the same output
+    assert torch.equal(O1, O2)
+    og = oracle_geometry(g)
+    trees = _oracle_trees(g, K, V, r, lens)
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for h in range(0, g.n_q_heads, 7):
+            Kh, Vh, levels = trees[(s, h // G)]
+            check_query(st, to_np(O2[s, 0, h]), None, to_np(Q[s, 0, h]), L - 1, Kh, Vh,
+                        oracle.FullTree(levels), og, g.k)
+    st.check(torch.bfloat16, "decode after an expired wait")
