@@ -400,6 +400,8 @@ def run_recsa(args, rank, world, dev):
     torch.cuda.empty_cache()
     if not args.no_prefill and args.workload != "decode-1m":
         out["prefill"] = run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs)
+        if not args.no_zha:
+            out["zha_prefill"] = run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream)
     if not args.no_dense:
         out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -569,6 +571,56 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
             "build_roofline": {"bound": "hbm", "achieved": kv_bytes / (build_ms / 1e3) / 1e9,
                                "peak": hbm_gbs, "unit": "GB/s",
                                "frac": kv_bytes / (build_ms / 1e3) / 1e9 / hbm_gbs}}
+
+
+ZHA_PREFILL_QUERIES = 65536
+
+
+def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
+    """ZHA routing (p = ZHA_TOP_P, fp32 keys) prefill of the last
+    ZHA_PREFILL_QUERIES positions of one sequence on zha_attend_kernel (a
+    bounded sample of the workload's full prefill).  ALU roofline with flops =
+    2 d (summary keys scored + exact tokens) per query head, the counts taken
+    from a traced prefill of 256 of the queries."""
+    L = w.length
+    nq = min(ZHA_PREFILL_QUERIES, L)
+    q0 = L - nq
+    g = R.Geometry(head_dim=w.head_dim, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                   leaf_block=w.leaf_block, branching=w.branching, k=w.k, window=w.window,
+                   batch=1, capacity=cap,
+                   dtype=R.DTYPE_BF16 if w.dtype == torch.bfloat16 else R.DTYPE_F32,
+                   rope_enabled=1, rope_base=w.rope_base, mode=R.MODE_ZHA, top_p=ZHA_TOP_P)
+    K0, V0 = Kc[:1], Vc[:1]
+    tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
+    R.recsa_build(g, K0, V0, [L], r, 0, tree)
+    Q = make_prefill_queries(w, Kc, q0, L)
+    O = torch.empty_like(Q)
+    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O)      # warm-up
+    torch.cuda.synchronize()
+    flush()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = elapsed(e0, e1)
+    ns = min(256, nq)
+    trace = torch.zeros((1, ns, w.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    R.recsa_prefill(g, Q[:, nq - ns:].contiguous(), K0, V0, tree, L - ns, ns,
+                    O[:, nq - ns:].contiguous(), trace)
+    tr = trace.cpu().numpy()
+    per_head = float((tr[..., 2].astype(np.float64) + tr[..., 3]).mean())   # keys + exact
+    flops = 2.0 * w.head_dim * per_head * nq * w.n_q_heads
+    del Q, O, tree, trace
+    torch.cuda.empty_cache()
+    return {"value": nq / (ms / 1e3), "unit": "tokens/s", "ms": ms, "queries": nq,
+            "q_start": q0, "top_p": ZHA_TOP_P, "kernel": "zha_attend_kernel",
+            "sample": f"the last {nq} of {L} positions of one sequence",
+            "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
+                         "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": flops / (ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS, "flops": flops,
+                         "traffic": None}}
 
 
 def run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, prefill):
