@@ -97,7 +97,9 @@ enum { RECSA_DTYPE_F32 = 0, RECSA_DTYPE_BF16 = 1 };
  *   the smallest set of highest-scoring candidates whose softmax mass reaches
  *   top_p (at most k of them), scores are q . key / sqrt(d) without rotation,
  *   and the attention covers only the tokens of the reached leaves and the
- *   window, at their true positions with standard RoPE (no summaries); or
+ *   window, at their true positions with standard RoPE (no summaries; the
+ *   tree's RoPE table then covers every position, so capacity < 2^24, else
+ *   RECSA_ERR_UNSUPPORTED); or
  *   RECSA_MODE_GROUP, RecSA with one selection per KV group (the "per KV
  *   group" convention of the same page's Table IX): the G query heads of a
  *   KV head score the shared candidates with their own RecSA logits, a
