@@ -180,3 +180,14 @@ def test_argument_errors_return_before_device(lib):
     assert lib.recsa_decode(ctypes.byref(g2), ok, ok, ok, ok, ok, 1, ok, ok, None) == 5
     # zero queries: nothing to do
     assert lib.recsa_prefill(ctypes.byref(cg), ok, ok, ok, ok, 0, 0, ok, None, None, 0, None) == 0
+
+
+def test_zha_capacity_limit(lib):
+    """A ZHA tree's RoPE table has a row per position: capacity below 2^24."""
+    ok = geo(mode=R.MODE_ZHA, top_p=0.5, batch=1, capacity=(1 << 24) - 2)
+    assert R.recsa_tree_bytes(ok) > 0
+    with pytest.raises(R.RecsaError) as e:
+        R.recsa_tree_bytes(geo(mode=R.MODE_ZHA, top_p=0.5, batch=1, capacity=(1 << 24) + 10))
+    assert e.value.status == 5
+    # RecSA's table covers only candidate-local indices: no such limit
+    assert R.recsa_tree_bytes(geo(batch=1, capacity=(1 << 24) + 10)) > 0
