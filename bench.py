@@ -578,8 +578,10 @@ ZHA_PREFILL_QUERIES = 65536
 
 def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
     """ZHA routing (p = ZHA_TOP_P, fp32 keys) prefill of the last
-    ZHA_PREFILL_QUERIES positions of one sequence on zha_attend_kernel (a
-    bounded sample of the workload's full prefill).  ALU roofline with flops =
+    ZHA_PREFILL_QUERIES positions of one sequence: the window on
+    window_mma_kernel, the routing and the leaves on zha_attend_kernel, which
+    merges the window's partials (a bounded sample of the workload's full
+    prefill).  ALU roofline with flops =
     2 d (summary keys scored + exact tokens) per query head, the counts taken
     from a traced prefill of 256 of the queries."""
     L = w.length
@@ -595,12 +597,13 @@ def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
     R.recsa_build(g, K0, V0, [L], r, 0, tree)
     Q = make_prefill_queries(w, Kc, q0, L)
     O = torch.empty_like(Q)
-    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O)      # warm-up
+    ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8, device="cuda")
+    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O, workspace=ws)      # warm-up
     torch.cuda.synchronize()
     flush()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O)
+    R.recsa_prefill(g, Q, K0, V0, tree, q0, nq, O, workspace=ws)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = elapsed(e0, e1)
@@ -612,10 +615,10 @@ def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
     tr = trace.cpu().numpy()
     per_head = float((tr[..., 2].astype(np.float64) + tr[..., 3]).mean())   # keys + exact
     flops = 2.0 * w.head_dim * per_head * nq * w.n_q_heads
-    del Q, O, tree, trace
+    del Q, O, tree, trace, ws
     torch.cuda.empty_cache()
     return {"value": nq / (ms / 1e3), "unit": "tokens/s", "ms": ms, "queries": nq,
-            "q_start": q0, "top_p": ZHA_TOP_P, "kernel": "zha_attend_kernel",
+            "q_start": q0, "top_p": ZHA_TOP_P, "kernel": "window_mma_kernel + zha_attend_kernel",
             "sample": f"the last {nq} of {L} positions of one sequence",
             "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
                          "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",

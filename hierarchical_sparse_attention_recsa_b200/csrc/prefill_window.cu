@@ -263,7 +263,9 @@ window_mma_kernel(Params p, const __nv_bfloat16* __restrict__ Q,
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, int64_t q_start, int32_t n_q, void* part,
                                   cudaStream_t s) {
-  if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
+  // the window is attended at true distances t - pos: the same for RecSA and
+  // ZHA (group selection attends it in the generic kernel)
+  if (p.mode != RECSA_MODE_RECSA && p.mode != RECSA_MODE_ZHA) return cudaErrorNotSupported;
   if (p.dtype != RECSA_DTYPE_BF16) return cudaErrorNotSupported;
   if (p.group < 1 || kRows % p.group) return cudaErrorNotSupported;
   const int QB = kRows / p.group;

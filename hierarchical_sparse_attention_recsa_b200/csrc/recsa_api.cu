@@ -258,8 +258,17 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (p.mode == RECSA_MODE_ZHA) {
-    if (!getenv("RECSA_ZHA_GENERIC"))
-      e = launch_zha(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, s);
+    if (!getenv("RECSA_ZHA_GENERIC")) {
+      // prefill: the window (true-position RoPE there too) on tensor cores first
+      const void* wpart = nullptr;
+      if (!decode && workspace) {
+        e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, workspace, s);
+        if (e == cudaSuccess) wpart = workspace;
+        else if (e != cudaErrorNotSupported) return cuda_status(e);
+        else cudaGetLastError();
+      }
+      e = launch_zha(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, wpart, s);
+    }
   } else if (decode && !getenv("RECSA_DECODE_GENERIC")) {
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
   } else if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
@@ -351,7 +360,7 @@ recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, con
   cudaError_t e = cudaErrorNotSupported;
   if (p.mode == RECSA_MODE_ZHA) {
     if (!getenv("RECSA_ZHA_GENERIC"))
-      e = launch_zha(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, s);
+      e = launch_zha(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, nullptr, s);
   } else {
     e = launch_prefill_static(p, Q, K, V, tree, q_start, n_q, O, trace, s);
   }

@@ -146,10 +146,12 @@ cudaError_t launch_attend(const Params& p, const void* Q, const void* K, const v
                           int decode, void* O, int32_t* trace, cudaStream_t s);
 // Cluster decode kernel; cudaErrorNotSupported when the geometry is outside its limits.
 // ZHA routing variant (mode RECSA_MODE_ZHA): one CTA per (query, sequence,
-// query head).  cudaErrorNotSupported outside its limits (c <= 256).
+// query head); a prefill given the window kernel's partials (wpart) merges
+// them instead of attending the window.  cudaErrorNotSupported outside its
+// limits.
 cudaError_t launch_zha(const Params& p, const void* Q, const void* K, const void* V,
                        const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
-                       int decode, void* O, int32_t* trace, cudaStream_t s);
+                       int decode, void* O, int32_t* trace, const void* wpart, cudaStream_t s);
 cudaError_t launch_decode_cluster(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, const int64_t* len_dev, int32_t n_q, void* O,
                                   int32_t* trace, cudaStream_t s);

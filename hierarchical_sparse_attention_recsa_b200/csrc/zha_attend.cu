@@ -34,10 +34,13 @@
 namespace recsa {
 namespace {
 
-constexpr int kZThreads = 512;
-constexpr int kZWarps = kZThreads / 32;
-constexpr int kZChain = 12;         // chain warps; the others attend the window first
-constexpr int kZMaxCand = kZChain * 32;   // one chain thread per candidate
+// Launch shapes: decode (and prefill without window partials) runs 12 routing
+// warps and 4 window warps per query head; prefill with the tensor-core
+// window kernel's partials runs 4 routing warps and no window warps, in a
+// CTA small enough for four to share an SM.
+constexpr int kZDecChain = 12, kZDecWin = 4;
+constexpr int kZPreChain = 4;
+constexpr int kZMaxCand = 1024;     // candidates per level (smem per CTA)
 constexpr size_t kZStageBytes = 180 * 1024;   // shared memory for a level's staged key rows
 constexpr int kZUnit = 16;          // consecutive exact tokens per work unit
 constexpr int kZBarChain = 1;       // named barrier of the chain warps
@@ -58,8 +61,9 @@ __device__ __forceinline__ void cp_async8(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;\n" ::: "memory");
 }
+template <int NTH>
 __device__ __forceinline__ void chain_sync() {
-  asm volatile("bar.sync %0, %1;\n" ::"n"(kZBarChain), "n"(kZChain * 32) : "memory");
+  asm volatile("bar.sync %0, %1;\n" ::"n"(kZBarChain), "n"(NTH) : "memory");
 }
 
 // Lane l holds channel pairs (NP * l + u, NP * l + u + D/2), u < NP, of a row.
@@ -169,14 +173,18 @@ __device__ __forceinline__ void unpack(const Raw<T, NP>& r, float (&x1)[NP], flo
   }
 }
 
-template <typename T, int NP>
-__global__ void __launch_bounds__(kZThreads, 1)
+// NCH routing-chain warps, NWIN window warps; NWIN = 0 takes the window's
+// softmax state from wpart (the window kernel's partials, per query head:
+// normalised output [D], max, sum).
+template <typename T, int NP, int NCH, int NWIN>
+__global__ void __launch_bounds__((NCH + NWIN) * 32, NWIN == 0 ? 4 : 1)
 zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                   const T* __restrict__ V, const void* __restrict__ tree,
                   const int64_t* __restrict__ len_dev, int64_t q_start, int n_q, int decode,
                   T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
-                  int krows) {
+                  int krows, const float* __restrict__ wpart) {
   constexpr int D = 64 * NP, HALF = 32 * NP;
+  constexpr int NW = NCH + NWIN, NT = NW * 32, CT = NCH * 32;
   constexpr int RS = D + 2;                      // warp state row: acc[D], m, l
   const int qi = blockIdx.x;
   const int64_t seq = blockIdx.y;
@@ -197,17 +205,18 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   float* ksc = rowsc + krows;                                 // [krows] FP8 row scales
   float* score = ksc + krows;                                 // [cmax]
   float* wsort = score + cmax;                                // [cmax] weights by rank
-  float* zsum = wsort + cmax;                                 // [kZChain] sums, [kZChain] max
-  float* wst = zsum + kZChain + 1;                            // [kZWarps][RS] warp states
-  int* kept = reinterpret_cast<int*>(wst + kZWarps * RS);     // [2][kmax] by level parity
+  float* zsum = wsort + cmax;                                 // [NCH] sums, [NCH] max
+  float* wst = zsum + NCH + 1;                                // [NW][RS] warp states
+  int* kept = reinterpret_cast<int*>(wst + NW * RS);          // [2][kmax] by level parity
   int* zc = kept + 2 * kmax;                                  // [kMaxLevels + 1] candidates
   int* zk = zc + kMaxLevels + 1;                              // [kMaxLevels + 1] expanded
-  int* zcnt = zk + kMaxLevels + 1;                            // [kZChain] expanded per warp
+  int* rankv = zk + kMaxLevels + 1;                           // [cmax] candidate ranks
+  int* zcnt = rankv + cmax;                                   // [rounds][NCH] expanded
 
   const int64_t t = decode ? len_dev[seq] - 1 : q_start + qi;
   const int64_t orow = ((seq * n_q + qi) * p.hq + h) * D;
   if (t < 0 || t >= p.cap) {   // empty sequence, or a length beyond capacity: zeros
-    for (int x = tid; x < D; x += kZThreads) O[orow + x] = T(0.f);
+    for (int x = tid; x < D; x += NT) O[orow + x] = T(0.f);
     return;
   }
   const float2* rope = rope_table(p, tree);
@@ -321,7 +330,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
   };
 
-  if (warp < kZChain) {
+  if (warp < NCH) {
     // ---- routing chain ----------------------------------------------------
     const int ct = tid;                          // 0 .. 255
     int kup = 0;
@@ -346,7 +355,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       for (int i0c = 0; i0c < c; i0c += cc) {
         const int i1c = min(c, i0c + cc);
         const int nrow = (i1c - i0c) * R;
-        for (int x = ct; x < nrow * C16; x += kZChain * 32) {
+        for (int x = ct; x < nrow * C16; x += CT) {
           const int q = x / C16, pc = x % C16;
           const int i = i0c + q / R, ref = q % R;
           const int64_t row = int64_t(node(i)) * R + ref;
@@ -360,7 +369,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
             cp_async16(kbuf + size_t(q) * D + pc * 4, keys + row * D + pc * 4);
         }
         if (lowp)   // row scales (and NVFP4 block scales) ride with the code rows
-          for (int q = ct; q < nrow; q += kZChain * 32) {
+          for (int q = ct; q < nrow; q += CT) {
             const int64_t row = int64_t(node(i0c + q / R)) * R + q % R;
             cp_async4(ksc + q, kscales + row);
             if (nv4) {   // D / 16 block-scale bytes (8 at D = 128, 4 at D = 64)
@@ -371,14 +380,14 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
             }
           }
         cp_async_wait_all();
-        chain_sync();
+        chain_sync<CT>();
         float* rsc = R == 1 ? score + i0c : rowsc;   // row scores
         // rows warp, warp + 8, ...; four rows per warp at a time
-        for (int q0 = warp; q0 < nrow; q0 += 4 * kZChain) {
+        for (int q0 = warp; q0 < nrow; q0 += 4 * NCH) {
           float sc4[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const int q = min(q0 + r * kZChain, nrow - 1);   // rows past nrow repeat the last
+            const int q = min(q0 + r * NCH, nrow - 1);   // rows past nrow repeat the last
             float x1[NP], x2[NP];
             if (fp8)
               load_codes<NP>(kbyte + size_t(q) * D, lane, x1, x2);
@@ -402,44 +411,48 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
             float v = sc4[0];
 #pragma unroll
             for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
-            const int q = q0 + lane * kZChain;
+            const int q = q0 + lane * NCH;
             if (q < nrow) rsc[q] = v * p.inv_sqrt_d * (lowp ? ksc[q] : 1.f);
           }
         }
-        chain_sync();
+        chain_sync<CT>();
         if (R > 1) {   // a candidate's score: the best of its R rows
-          for (int i = i0c + ct; i < i1c; i += kZChain * 32) {
+          for (int i = i0c + ct; i < i1c; i += CT) {
             float m = rsc[(i - i0c) * R];
             for (int ref = 1; ref < R; ++ref) m = fmaxf(m, rsc[(i - i0c) * R + ref]);
             score[i] = m;
           }
-          chain_sync();
+          chain_sync<CT>();
         }
       }
-      chain_sync();
-      // Top-p by ranks: chain thread ct holds candidate ct (c <= 384).  Its rank
-      // counts the better candidates (higher score, or equal at a lower
+      chain_sync<CT>();
+      // Top-p by ranks: chain thread ct holds candidates ct, ct + CT, ...  A
+      // rank counts the better candidates (higher score, or equal at a lower
       // index); the weights exp(s - max) are laid out by rank, and warp 0
       // scans them for the shortest prefix whose mass reaches top_p of the
       // total, capped at min(k, c).
-      const bool mine = ct < c;
-      const float si = mine ? score[ct] : 0.f;
-      int ri = 0;
-      if (mine) {
+      for (int i = ct; i < c; i += CT) {
+        const float si = score[i];
+        int ri = 0;
         for (int j = 0; j < c; ++j) {
           const float sj = score[j];
-          ri += (sj > si) || (sj == si && j < ct);
+          ri += (sj > si) || (sj == si && j < i);
         }
-        if (ri == 0) zsum[kZChain] = si;   // the level's maximum
+        rankv[i] = ri;
+        if (ri == 0) zsum[NCH] = si;   // the level's maximum
       }
-      chain_sync();
-      const float ei = mine ? expf(si - zsum[kZChain]) : 0.f;
-      if (mine) wsort[ri] = ei;
-      const float ws = warp_sum(ei);
+      chain_sync<CT>();
+      float ws = 0.f;
+      for (int i = ct; i < c; i += CT) {
+        const float ei = expf(score[i] - zsum[NCH]);
+        wsort[rankv[i]] = ei;
+        ws += ei;
+      }
+      ws = warp_sum(ws);
       if (lane == 0) zsum[warp] = ws;
-      chain_sync();
+      chain_sync<CT>();
       if (warp == 0) {
-        const float tot = warp_sum(lane < kZChain ? zsum[lane] : 0.f);
+        const float tot = warp_sum(lane < NCH ? zsum[lane] : 0.f);
         const float thr = p.top_p * tot;
         const int cap = c < p.k ? c : p.k;
         int cnt = cap;
@@ -466,26 +479,37 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
           zk[lev] = cnt;
         }
       }
-      chain_sync();
-      // expanded nodes in candidate order
-      const bool on = mine && ri < zk[lev];
-      const unsigned bal = __ballot_sync(0xffffffffu, on);
-      if (lane == 0) zcnt[warp] = __popc(bal);
-      chain_sync();
-      if (on) {
-        int pos = __popc(bal & ((1u << lane) - 1u));
-        for (int w = 0; w < warp; ++w) pos += zcnt[w];
-        const int id = node(ct);
-        kept[(lev & 1) * kmax + pos] = id;
-        if (rec) rec[kTraceHead + (lev - 1) * p.k + pos] = id;
+      chain_sync<CT>();
+      // expanded nodes in candidate order: rounds of CT candidates, a ballot
+      // per warp and round, positions from the counts of earlier rounds/warps
+      const int nrounds = (c + CT - 1) / CT;
+      for (int r = 0; r < nrounds; ++r) {
+        const int i = r * CT + ct;
+        const unsigned bal = __ballot_sync(0xffffffffu, i < c && rankv[i] < zk[lev]);
+        if (lane == 0) zcnt[r * NCH + warp] = __popc(bal);
       }
-      chain_sync();
+      chain_sync<CT>();
+      int before = 0;
+      for (int r = 0; r < nrounds; ++r) {
+        const int i = r * CT + ct;
+        const bool on = i < c && rankv[i] < zk[lev];
+        const unsigned bal = __ballot_sync(0xffffffffu, on);
+        if (on) {
+          int pos = before + __popc(bal & ((1u << lane) - 1u));
+          for (int w = 0; w < warp; ++w) pos += zcnt[r * NCH + w];
+          const int id = node(i);
+          kept[(lev & 1) * kmax + pos] = id;
+          if (rec) rec[kTraceHead + (lev - 1) * p.k + pos] = id;
+        }
+        for (int w = 0; w < NCH; ++w) before += zcnt[r * NCH + w];
+      }
+      chain_sync<CT>();
       kup = zk[lev];
     }
-  } else {
+  } else if constexpr (NWIN > 0) {
     // ---- window warps: [a*B, t], units of kZUnit positions ------------------
     const int nu = int((n_win + kZUnit - 1) / kZUnit);
-    for (int u = warp - kZChain; u < nu; u += kZWarps - kZChain) {
+    for (int u = warp - NCH; u < nu; u += NWIN) {
       const int64_t p0 = a * p.B + int64_t(u) * kZUnit;
       const int n = int(n_win - int64_t(u) * kZUnit < kZUnit ? n_win - int64_t(u) * kZUnit
                                                                : kZUnit);
@@ -499,7 +523,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   const int upl = (p.B + kZUnit - 1) / kZUnit;   // units per leaf
   const int* leaves = kept + 1 * kmax;           // level 1 (odd parity)
   // the window warps take the first units: the chain warps start later
-  for (int u = (warp + kZWarps - kZChain) % kZWarps; u < nleaf * upl; u += kZWarps) {
+  for (int u = (warp + NW - NCH) % NW; u < nleaf * upl; u += NW) {
     const int r = u / upl, m = u % upl;
     const int n = p.B - m * kZUnit < kZUnit ? p.B - m * kZUnit : kZUnit;
     attend_unit(int64_t(leaves[r]) * p.B + m * kZUnit, n);
@@ -518,10 +542,17 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
   }
   __syncthreads();
   if (tid < D) {
-    float M = -INFINITY;
-    for (int w = 0; w < kZWarps; ++w) M = fmaxf(M, wst[w * RS + D]);
+    // the window's state: from the window warps, or the window kernel's partial
+    const float* wrow = NWIN == 0 ? wpart + ((seq * n_q + qi) * p.hq + h) * (D + 2) : nullptr;
+    float M = NWIN == 0 ? wrow[D] : -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wst[w * RS + D]);
     float L = 0.f, A = 0.f;
-    for (int w = 0; w < kZWarps; ++w) {
+    if (NWIN == 0 && wrow[D] != -INFINITY) {
+      const float e = expf(wrow[D] - M) * wrow[D + 1];   // normalised output x sum
+      L = e;
+      A = wrow[tid] * e;
+    }
+    for (int w = 0; w < NW; ++w) {
       const float mw = wst[w * RS + D];
       if (mw == -INFINITY) continue;
       const float e = expf(mw - M);
@@ -553,7 +584,7 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 template <typename T, int NP>
 cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void* V,
                       const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
-                      int decode, void* O, int32_t* trace, cudaStream_t s) {
+                      int decode, void* O, int32_t* trace, const float* wpart, cudaStream_t s) {
   constexpr int D = 64 * NP;
   const int64_t kk = p.k < p.cap ? p.k : p.cap;
   int64_t maxn = 1;
@@ -563,28 +594,33 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   const int cmax = int(cm < 1 ? 1 : cm);
   if (cmax > kZMaxCand) return cudaErrorNotSupported;   // the generic kernel serves it
   const int kmax = int(kk < cmax ? kk : cmax);
-  // level key rows staged per chunk (FP8 rows are a quarter of the bytes)
+  const bool part = wpart != nullptr;   // prefill with window partials: small CTAs
+  const int nch = part ? kZPreChain : kZDecChain, nw = part ? kZPreChain : kZDecChain + kZDecWin;
+  // level key rows staged per chunk (FP8 rows are a quarter of the bytes, NVFP4
+  // rows less); small CTAs keep their staging to 40 KB so that four share an SM
   const bool lowp = p.kfmt != RECSA_KEYS_F32;
   const int rowb = p.kfmt == RECSA_KEYS_FP8 ? D : (lowp ? D / 2 + D / 16 : 4 * D);
-  // as many (candidate, reference) rows per chunk as the staging budget holds
-  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref,
-                                          int64_t(kZStageBytes / size_t(rowb + 8))));
+  const size_t stage = part ? 40 * 1024 : kZStageBytes;
+  const int krows = int(std::min<int64_t>(int64_t(cmax) * p.nref, int64_t(stage / size_t(rowb + 8))));
   if (krows < p.nref) return cudaErrorNotSupported;
+  const int rounds = (cmax + nch * 32 - 1) / (nch * 32);
   const size_t bytes = size_t(krows) * rowb +
-                       (2 * size_t(krows) + 2 * size_t(cmax) + kZChain + 1 + kZWarps * (D + 2)) * 4 +
-                       (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + kZChain) * 4;
+                       (2 * size_t(krows) + 2 * size_t(cmax) + nch + 1 + size_t(nw) * (D + 2)) * 4 +
+                       (2 * size_t(kmax) + 2 * (kMaxLevels + 1) + size_t(cmax) +
+                        size_t(rounds) * nch) * 4;
   if (bytes > 227 * 1024) return cudaErrorNotSupported;
   if (p.batch > 65535) return cudaErrorNotSupported;
-  auto kern = zha_attend_kernel<T, NP>;
+  auto kern = part ? zha_attend_kernel<T, NP, kZPreChain, 0>
+                   : zha_attend_kernel<T, NP, kZDecChain, kZDecWin>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(bytes));
   if (e != cudaSuccess) return e;
   dim3 grid(n_q, p.batch, p.hq);
-  kern<<<grid, kZThreads, bytes, s>>>(p, reinterpret_cast<const T*>(Q),
-                                      reinterpret_cast<const T*>(K),
-                                      reinterpret_cast<const T*>(V), tree, len_dev, q_start, n_q,
-                                      decode, reinterpret_cast<T*>(O), trace, cmax, kmax,
-                                      krows);
+  kern<<<grid, nw * 32, bytes, s>>>(p, reinterpret_cast<const T*>(Q),
+                                    reinterpret_cast<const T*>(K),
+                                    reinterpret_cast<const T*>(V), tree, len_dev, q_start, n_q,
+                                    decode, reinterpret_cast<T*>(O), trace, cmax, kmax, krows,
+                                    wpart);
   return cudaGetLastError();
 }
 
@@ -592,17 +628,18 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
 
 cudaError_t launch_zha(const Params& p, const void* Q, const void* K, const void* V,
                        const void* tree, const int64_t* len_dev, int64_t q_start, int32_t n_q,
-                       int decode, void* O, int32_t* trace, cudaStream_t s) {
+                       int decode, void* O, int32_t* trace, const void* wpart, cudaStream_t s) {
   if (p.mode != RECSA_MODE_ZHA) return cudaErrorNotSupported;
+  const float* wp = decode ? nullptr : reinterpret_cast<const float*>(wpart);
   if (p.dtype == RECSA_DTYPE_BF16)
     return p.d == 128 ? zha_typed<__nv_bfloat16, 2>(p, Q, K, V, tree, len_dev, q_start, n_q,
-                                                    decode, O, trace, s)
+                                                    decode, O, trace, wp, s)
                       : zha_typed<__nv_bfloat16, 1>(p, Q, K, V, tree, len_dev, q_start, n_q,
-                                                    decode, O, trace, s);
+                                                    decode, O, trace, wp, s);
   return p.d == 128 ? zha_typed<float, 2>(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O,
-                                          trace, s)
+                                          trace, wp, s)
                     : zha_typed<float, 1>(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O,
-                                          trace, s);
+                                          trace, wp, s);
 }
 
 }  // namespace recsa

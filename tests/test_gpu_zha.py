@@ -787,3 +787,36 @@ def test_zha_nvfp4_append_matches_build():
             n = new_lens[s] // (g.leaf_block * g.branching ** (lev - 1))
             for x, y in zip(a, b):
                 assert torch.equal(x[s, :, :n], y[s, :, :n]), lev
+
+
+@pytest.mark.parametrize("workspace", [True, False])
+def test_zha_prefill_model_small(workspace, zha_impl):
+    """bf16 prefill: with a workspace the window comes from the tensor-core
+    window kernel's partials and the ZHA kernel runs its small-CTA prefill
+    shape; without, the ZHA kernel attends the window itself."""
+    lens, top_p = [20000, 13001], 0.8
+    g, K, V, r, Kd, Vd, rd, tree = _setup(MODEL, lens, 20480, top_p, seed=130)
+    trees = _trees(g, K, V, r, lens)
+    q0, nq = 12000, 1001
+    pos = (q0 + torch.arange(nq, dtype=torch.int64))[None].expand(2, nq)
+    Q, _, _ = synth.make_queries(MODEL, K, pos.contiguous(), seed=131)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    ws = (torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8, device="cuda")
+          if workspace else None)
+    R.recsa_prefill(g, Qd, Kd, Vd, tree, q0, nq, O, trace, workspace=ws)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    rng = np.random.default_rng(9)
+    for s in range(2):
+        for i in [0, 1, 63, 64, 500, nq - 1] + list(rng.integers(0, nq, 4)):
+            for h in range(0, g.n_q_heads, 3):
+                Kh, Vh, src = trees[(s, h // G)]
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), q0 + i, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} prefill model small workspace={workspace}")
