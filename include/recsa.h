@@ -235,7 +235,8 @@ recsa_status recsa_decode_step(const recsa_geometry* geom, const void* Q, void* 
  *   head_dim + 2: the window's normalised output, max and sum) is kept there
  *   until the tree kernel merges it and writes O once; without one, the window
  *   is attended by the tree kernel itself.  Both give the same result within
- *   rounding.
+ *   rounding.  This holds in RECSA_MODE_RECSA and RECSA_MODE_ZHA (both attend
+ *   the window at true distances); RECSA_MODE_GROUP ignores the workspace.
  *   The workspace is only read and written by this call; calls that share one
  *   must not overlap on the device.
  */
