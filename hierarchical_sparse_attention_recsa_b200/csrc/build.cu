@@ -19,14 +19,17 @@ namespace recsa {
 namespace {
 
 // Store the pooled key of node j (level lev, reference ref): fp32 row, or
-// FP8 E4M3 codes with one fp32 scale (low-precision router keys).
-template <int N>
+// FP8 E4M3 codes with one fp32 scale (low-precision router keys).  KF is the
+// key format when known at compile time (the build kernels, which then carry
+// no code, and no registers, for the other formats), or -1 for p.kfmt.
+template <int N, int KF = -1>
 __device__ void store_node_key(const Params& p, void* tree, int lev, int64_t seq, int g,
                                int64_t j, int ref, int lane, const float* key) {
-  if (p.kfmt == RECSA_KEYS_FP8)
+  const int kf = KF >= 0 ? KF : p.kfmt;
+  if (kf == RECSA_KEYS_FP8)
     store_key_fp8<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.kcb,
                      level_kscales(p, tree, lev, seq, g) + j * p.nref + ref, lane, key);
-  else if (p.kfmt == RECSA_KEYS_NVFP4)
+  else if (kf == RECSA_KEYS_NVFP4)
     store_key_nvfp4<N>(level_kcodes(p, tree, lev, seq, g) + (j * p.nref + ref) * p.kcb,
                        level_kbscales(p, tree, lev, seq, g) + (j * p.nref + ref) * (p.d / 16),
                        level_kscales(p, tree, lev, seq, g) + j * p.nref + ref, lane, key);
@@ -36,12 +39,13 @@ __device__ void store_node_key(const Params& p, void* tree, int lev, int64_t seq
 }
 
 // Pool node j of level lev >= 2 for reference ref from its b children's
-// stored keys (decoded when FP8) and values.
-template <int N>
+// stored keys (decoded when FP8) and values; KF as for store_node_key.
+template <int N, int KF = -1>
 __device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, int g, int64_t j,
                             int ref, const float* rl, int lane, float* key, float* val) {
   const float* cv = level_vals(p, tree, lev - 1, seq, g) + j * p.b * p.d;
-  if (p.kfmt == RECSA_KEYS_FP8) {
+  const int kf = KF >= 0 ? KF : p.kfmt;
+  if (kf == RECSA_KEYS_FP8) {
     const unsigned char* cc =
         level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.kcb;
     const float* cs = level_kscales(p, tree, lev - 1, seq, g) + j * p.b * p.nref + ref;
@@ -50,7 +54,7 @@ __device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, i
           load_key_fp8<N>(cc + int64_t(i) * p.nref * p.kcb, cs[int64_t(i) * p.nref], lane, x);
         },
         cv, p.b, p.d, rl, p.inv_sqrt_d, lane, key, val);
-  } else if (p.kfmt == RECSA_KEYS_NVFP4) {
+  } else if (kf == RECSA_KEYS_NVFP4) {
     const int nb = p.d / 16;
     const unsigned char* cc =
         level_kcodes(p, tree, lev - 1, seq, g) + (j * p.b * p.nref + ref) * p.kcb;
@@ -70,9 +74,106 @@ __device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, i
   }
 }
 
-// Level 1: one warp per leaf block of one (sequence, KV head).
-template <typename T, int N>
-__global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T* V,
+// pool_rows for bf16 leaf rows, with the same arithmetic in the same order
+// (so the same bits), arranged for the HBM stream: a lane holds its channels
+// of a row as packed bf16 words (half the registers of floats), the row
+// stride is a compile-time constant (immediate load offsets), and the loads
+// of the next 4 rows are in flight while the current 4 are pooled.
+template <int N>
+__device__ __forceinline__ void load_bf16_words(const __nv_bfloat16* row, int lane,
+                                                unsigned* w) {
+  if constexpr (N == 4) {
+    const uint2 u = reinterpret_cast<const uint2*>(row)[lane];
+    w[0] = u.x;
+    w[1] = u.y;
+  } else {
+    w[0] = reinterpret_cast<const unsigned*>(row)[lane];
+  }
+}
+__device__ __forceinline__ float2 bf16_word_to_float2(unsigned w) {
+  __nv_bfloat162 h;
+  memcpy(&h, &w, sizeof(h));
+  return __bfloat1622float2(h);
+}
+
+template <int N>
+__device__ void pool_leaf_bf16(const __nv_bfloat16* kbase, const __nv_bfloat16* vbase, int n,
+                               const float* rl, float inv_sqrt_d, int lane, float* key,
+                               float* val) {
+  constexpr int U = 4, NW = N / 2, DD = 32 * N;   // a lane owns N of the d = 32 N channels
+  unsigned ka[U][NW], va[U][NW], kb[U][NW], vb[U][NW];
+  float m = -INFINITY, l = 0.f;
+  float ak[N], av[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) ak[c] = av[c] = 0.f;
+  auto issue = [&](unsigned (&kw)[U][NW], unsigned (&vw)[U][NW], int i0) {
+    const __nv_bfloat16* kr = kbase + int64_t(i0) * DD;
+    const __nv_bfloat16* vr = vbase + int64_t(i0) * DD;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (i0 + u < n) {
+        load_bf16_words<N>(kr + u * DD, lane, kw[u]);
+        load_bf16_words<N>(vr + u * DD, lane, vw[u]);
+      }
+  };
+  auto consume = [&](const unsigned (&kw)[U][NW], const unsigned (&vw)[U][NW], int i0) {
+    float s[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float acc = 0.f;
+      if (i0 + u < n) {
+#pragma unroll
+        for (int h = 0; h < NW; ++h) {
+          const float2 f = bf16_word_to_float2(kw[u][h]);
+          acc = fmaf(rl[2 * h], f.x, acc);
+          acc = fmaf(rl[2 * h + 1], f.y, acc);
+        }
+      }
+      s[u] = acc;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) s[u] = warp_sum(s[u]) * inv_sqrt_d;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (i0 + u < n) {
+        const float mn = fmaxf(m, s[u]);
+        const float sc = expf(m - mn);
+        const float w = expf(s[u] - mn);
+        l = l * sc + w;
+#pragma unroll
+        for (int h = 0; h < NW; ++h) {
+          const float2 k = bf16_word_to_float2(kw[u][h]);
+          const float2 v = bf16_word_to_float2(vw[u][h]);
+          ak[2 * h] = fmaf(w, k.x, ak[2 * h] * sc);
+          ak[2 * h + 1] = fmaf(w, k.y, ak[2 * h + 1] * sc);
+          av[2 * h] += v.x;
+          av[2 * h + 1] += v.y;
+        }
+        m = mn;
+      }
+    }
+  };
+  issue(ka, va, 0);
+  for (int i0 = 0; i0 < n; i0 += 2 * U) {
+    issue(kb, vb, i0 + U);
+    consume(ka, va, i0);
+    issue(ka, va, i0 + 2 * U);
+    consume(kb, vb, i0 + U);
+  }
+  const float il = 1.f / l, in = 1.f / float(n);
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    key[c] = ak[c] * il;
+    val[c] = av[c] * in;
+  }
+}
+
+// Level 1: one warp per leaf block of one (sequence, KV head).  With bf16
+// rows, two CTAs per SM (at most 128 registers a thread) keep 16 warps' row
+// loads in flight, which the HBM stream needs (one CTA per SM, at the
+// unbounded register count, reached a quarter of the bandwidth).
+template <typename T, int N, int KF>
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) leaf_kernel(Params p, const T* K, const T* V,
                                                    const float* r, int64_t r_stride, void* tree,
                                                    int64_t seq, int64_t n_leaf) {
   const int lane = threadIdx.x & 31;
@@ -84,14 +185,17 @@ __global__ void __launch_bounds__(256) leaf_kernel(Params p, const T* K, const T
     float rl[N];
     load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
     float key[N], val[N];
-    pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-    store_node_key<N>(p, tree, 1, seq, g, j, ref, lane, key);
+    if constexpr (sizeof(T) == 2 && N == 4)
+      pool_leaf_bf16<N>(K + row0, V + row0, p.B, rl, p.inv_sqrt_d, lane, key, val);
+    else
+      pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
+    store_node_key<N, KF>(p, tree, 1, seq, g, j, ref, lane, key);
     if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
   }
 }
 
 // Level lev >= 2: one warp per node, pooling b child summaries.
-template <int N>
+template <int N, int KF>
 __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, int64_t r_stride,
                                                      void* tree, int64_t seq, int lev,
                                                      int64_t n_nodes) {
@@ -103,8 +207,8 @@ __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, i
     float rl[N];
     load_r<N>(r + g * r_stride + ref * p.d, lane, rl);
     float key[N], val[N];
-    pool_parent<N>(p, tree, lev, seq, g, j, ref, rl, lane, key, val);
-    store_node_key<N>(p, tree, lev, seq, g, j, ref, lane, key);
+    pool_parent<N, KF>(p, tree, lev, seq, g, j, ref, rl, lane, key, val);
+    store_node_key<N, KF>(p, tree, lev, seq, g, j, ref, lane, key);
     if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + j * p.d, lane, val);
   }
 }
@@ -174,25 +278,35 @@ __global__ void rope_table_kernel(float2* table, int rows, int half, int d, doub
   table[idx] = make_float2(float(c), float(s));
 }
 
-template <typename T, int N>
-cudaError_t build_typed(const Params& p, const void* K, const void* V, const int64_t* len_host,
-                        const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
+template <typename T, int N, int KF>
+cudaError_t build_format(const Params& p, const void* K, const void* V, const int64_t* len_host,
+                         const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
   const int warps = 8;
   for (int64_t seq = 0; seq < p.batch; ++seq) {
     int64_t n = len_host[seq] / p.B;
     if (n == 0) continue;
     dim3 grid(unsigned((n + warps - 1) / warps), p.hkv);
-    leaf_kernel<T, N><<<grid, warps * 32, 0, s>>>(p, reinterpret_cast<const T*>(K),
+    leaf_kernel<T, N, KF><<<grid, warps * 32, 0, s>>>(p, reinterpret_cast<const T*>(K),
                                                   reinterpret_cast<const T*>(V), r, r_stride,
                                                   tree, seq, n);
     for (int lev = 2; lev <= p.lay.levels; ++lev) {
       n /= p.b;
       if (n == 0) break;
       dim3 g2(unsigned((n + warps - 1) / warps), p.hkv);
-      parent_kernel<N><<<g2, warps * 32, 0, s>>>(p, r, r_stride, tree, seq, lev, n);
+      parent_kernel<N, KF><<<g2, warps * 32, 0, s>>>(p, r, r_stride, tree, seq, lev, n);
     }
   }
   return cudaGetLastError();
+}
+
+template <typename T, int N>
+cudaError_t build_typed(const Params& p, const void* K, const void* V, const int64_t* len_host,
+                        const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
+  if (p.kfmt == RECSA_KEYS_FP8)
+    return build_format<T, N, RECSA_KEYS_FP8>(p, K, V, len_host, r, r_stride, tree, s);
+  if (p.kfmt == RECSA_KEYS_NVFP4)
+    return build_format<T, N, RECSA_KEYS_NVFP4>(p, K, V, len_host, r, r_stride, tree, s);
+  return build_format<T, N, RECSA_KEYS_F32>(p, K, V, len_host, r, r_stride, tree, s);
 }
 
 }  // namespace
