@@ -78,7 +78,8 @@ __device__ void pool_parent(const Params& p, void* tree, int lev, int64_t seq, i
 // (so the same bits), arranged for the HBM stream: a lane holds its channels
 // of a row as packed bf16 words (half the registers of floats), the row
 // stride is a compile-time constant (immediate load offsets), and the loads
-// of the next 4 rows are in flight while the current 4 are pooled.
+// of the next 2 rows are in flight while the current 2 are pooled: few
+// registers, so that many warps stream at once.
 template <int N>
 __device__ __forceinline__ void load_bf16_words(const __nv_bfloat16* row, int lane,
                                                 unsigned* w) {
@@ -100,7 +101,7 @@ template <int N>
 __device__ void pool_leaf_bf16(const __nv_bfloat16* kbase, const __nv_bfloat16* vbase, int n,
                                const float* rl, float inv_sqrt_d, int lane, float* key,
                                float* val) {
-  constexpr int U = 4, NW = N / 2, DD = 32 * N;   // a lane owns N of the d = 32 N channels
+  constexpr int U = 2, NW = N / 2, DD = 32 * N;   // a lane owns N of the d = 32 N channels
   unsigned ka[U][NW], va[U][NW], kb[U][NW], vb[U][NW];
   float m = -INFINITY, l = 0.f;
   float ak[N], av[N];
@@ -169,11 +170,12 @@ __device__ void pool_leaf_bf16(const __nv_bfloat16* kbase, const __nv_bfloat16* 
 }
 
 // Level 1: one warp per leaf block of one (sequence, KV head).  With bf16
-// rows, two CTAs per SM (at most 128 registers a thread) keep 16 warps' row
-// loads in flight, which the HBM stream needs (one CTA per SM, at the
-// unbounded register count, reached a quarter of the bandwidth).
+// rows at d = 128, three CTAs per SM (at most 80 registers a thread) keep 24
+// warps' row loads in flight, which the HBM stream needs (one CTA per SM, at
+// the unbounded register count, reached a quarter of the bandwidth); other
+// bf16 rows run two CTAs per SM.
 template <typename T, int N, int KF>
-__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 2 : 1) leaf_kernel(Params p, const T* K, const T* V,
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? (N == 4 ? 3 : 2) : 1) leaf_kernel(Params p, const T* K, const T* V,
                                                    const float* r, int64_t r_stride, void* tree,
                                                    int64_t seq, int64_t n_leaf) {
   const int lane = threadIdx.x & 31;
