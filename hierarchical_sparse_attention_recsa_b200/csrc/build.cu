@@ -216,8 +216,9 @@ __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, i
 }
 
 // Append one token per sequence; pool the leaf and ancestors it completes.
-// One CTA per sequence; warp w handles KV heads w, w + 8, ...
-template <typename T, int N>
+// One CTA per sequence; warp w handles KV heads w, w + 8, ...  Compiled per
+// key format, as the build kernels are.
+template <typename T, int N, int KF>
 __global__ void __launch_bounds__(256) append_kernel(Params p, T* K, T* V, const T* k_new,
                                                      const T* v_new, int64_t* len_dev,
                                                      const float* r, int64_t r_stride,
@@ -248,14 +249,14 @@ __global__ void __launch_bounds__(256) append_kernel(Params p, T* K, T* V, const
         const int64_t row0 = ((seq * p.hkv + g) * p.cap + j * p.B) * p.d;
         float key[N], val[N];
         pool_rows<T, N>(K + row0, V + row0, p.B, p.d, rl, p.inv_sqrt_d, lane, key, val);
-        store_node_key<N>(p, tree, 1, seq, g, j, ref, lane, key);
+        store_node_key<N, KF>(p, tree, 1, seq, g, j, ref, lane, key);
         if (ref == 0) RowIO<float, N>::store(level_vals(p, tree, 1, seq, g) + j * p.d, lane, val);
         int64_t idx = j;
         for (int lev = 2; lev <= p.lay.levels && (idx + 1) % p.b == 0; ++lev) {
           idx = (idx + 1) / p.b - 1;
           __syncwarp();
-          pool_parent<N>(p, tree, lev, seq, g, idx, ref, rl, lane, key, val);
-          store_node_key<N>(p, tree, lev, seq, g, idx, ref, lane, key);
+          pool_parent<N, KF>(p, tree, lev, seq, g, idx, ref, rl, lane, key, val);
+          store_node_key<N, KF>(p, tree, lev, seq, g, idx, ref, lane, key);
           if (ref == 0)
             RowIO<float, N>::store(level_vals(p, tree, lev, seq, g) + idx * p.d, lane, val);
         }
@@ -311,6 +312,27 @@ cudaError_t build_typed(const Params& p, const void* K, const void* V, const int
   return build_format<T, N, RECSA_KEYS_F32>(p, K, V, len_host, r, r_stride, tree, s);
 }
 
+template <typename T, int N>
+cudaError_t append_typed(const Params& p, void* K, void* V, const void* k_new, const void* v_new,
+                         int64_t* len_dev, const float* r, int64_t r_stride, void* tree,
+                         cudaStream_t s) {
+  const dim3 grid(p.batch);
+  T* Kt = static_cast<T*>(K);
+  T* Vt = static_cast<T*>(V);
+  const T* kn = static_cast<const T*>(k_new);
+  const T* vn = static_cast<const T*>(v_new);
+  if (p.kfmt == RECSA_KEYS_FP8)
+    append_kernel<T, N, RECSA_KEYS_FP8><<<grid, 256, 0, s>>>(p, Kt, Vt, kn, vn, len_dev, r,
+                                                             r_stride, tree);
+  else if (p.kfmt == RECSA_KEYS_NVFP4)
+    append_kernel<T, N, RECSA_KEYS_NVFP4><<<grid, 256, 0, s>>>(p, Kt, Vt, kn, vn, len_dev, r,
+                                                               r_stride, tree);
+  else
+    append_kernel<T, N, RECSA_KEYS_F32><<<grid, 256, 0, s>>>(p, Kt, Vt, kn, vn, len_dev, r,
+                                                             r_stride, tree);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_rope_table(const Params& p, void* tree, double rope_base, cudaStream_t s) {
@@ -335,25 +357,13 @@ cudaError_t launch_build(const Params& p, const void* K, const void* V, const in
 cudaError_t launch_append(const Params& p, void* K, void* V, const void* k_new, const void* v_new,
                           int64_t* len_dev, const float* r, int64_t r_stride, void* tree,
                           cudaStream_t s) {
-  dim3 grid(p.batch);
-  if (p.dtype == RECSA_DTYPE_BF16) {
-    using T = __nv_bfloat16;
-    if (p.d == 128)
-      append_kernel<T, 4><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
-                                               len_dev, r, r_stride, tree);
-    else
-      append_kernel<T, 2><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
-                                               len_dev, r, r_stride, tree);
-  } else {
-    using T = float;
-    if (p.d == 128)
-      append_kernel<T, 4><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
-                                               len_dev, r, r_stride, tree);
-    else
-      append_kernel<T, 2><<<grid, 256, 0, s>>>(p, (T*)K, (T*)V, (const T*)k_new, (const T*)v_new,
-                                               len_dev, r, r_stride, tree);
-  }
-  return cudaGetLastError();
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? append_typed<__nv_bfloat16, 4>(p, K, V, k_new, v_new, len_dev, r, r_stride,
+                                                      tree, s)
+                      : append_typed<__nv_bfloat16, 2>(p, K, V, k_new, v_new, len_dev, r, r_stride,
+                                                      tree, s);
+  return p.d == 128 ? append_typed<float, 4>(p, K, V, k_new, v_new, len_dev, r, r_stride, tree, s)
+                    : append_typed<float, 2>(p, K, V, k_new, v_new, len_dev, r, r_stride, tree, s);
 }
 
 }  // namespace recsa
