@@ -138,8 +138,13 @@ def test_tree_bytes(lib, kw):
     assert R.recsa_tree_bytes(g) == expected_tree_bytes(g)
 
 
-def test_prefill_workspace_bytes(lib):
-    g = geo(batch=2, capacity=4096)
+@pytest.mark.parametrize("mode", ["recsa", "zha", "group"])
+def test_prefill_workspace_bytes(lib, mode):
+    # one fp32 window partial (normalised output, max, sum) per query head, in
+    # every mode: ZHA prefill uses the same window partials as RecSA
+    extra = {"recsa": {}, "zha": dict(mode=R.MODE_ZHA, top_p=0.9),
+             "group": dict(mode=R.MODE_GROUP)}[mode]
+    g = geo(batch=2, capacity=4096, **extra)
     assert R.recsa_prefill_workspace_bytes(g, 100) == 2 * 100 * 32 * (128 + 2) * 4
 
 
