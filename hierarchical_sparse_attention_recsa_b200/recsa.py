@@ -196,6 +196,10 @@ def recsa_trace_ints(geom: Geometry) -> int:
 def recsa_build(geom: Geometry, K: torch.Tensor, V: torch.Tensor, len_host: Sequence[int],
                 pooler_r: torch.Tensor, pooler_head_stride: int, tree: torch.Tensor,
                 stream=None) -> None:
+    """Pool the tree over the first len_host[s] tokens of each sequence (K, V
+    [batch][n_kv_heads][capacity][head_dim]); pooler_r holds the pooler's
+    reference vector(s), pooler_head_stride elements apart per KV head (0: one
+    vector shared by every head)."""
     g = geom.c()
     lens = (ctypes.c_int64 * geom.batch)(*[int(x) for x in len_host])
     _check(lib().recsa_build(ctypes.byref(g), _ptr(K), _ptr(V), lens, _ptr(pooler_r),
@@ -205,6 +209,8 @@ def recsa_build(geom: Geometry, K: torch.Tensor, V: torch.Tensor, len_host: Sequ
 def recsa_append(geom: Geometry, K: torch.Tensor, V: torch.Tensor, k_new: torch.Tensor,
                  v_new: torch.Tensor, len_dev: torch.Tensor, pooler_r: torch.Tensor,
                  pooler_head_stride: int, tree: torch.Tensor, stream=None) -> None:
+    """Write one token per sequence (k_new, v_new [batch][n_kv_heads][head_dim])
+    at position len_dev[s], pool the nodes it completes and advance len_dev."""
     g = geom.c()
     _check(lib().recsa_append(ctypes.byref(g), _ptr(K), _ptr(V), _ptr(k_new), _ptr(v_new),
                               _ptr(len_dev), _ptr(pooler_r), pooler_head_stride, _ptr(tree),
@@ -214,6 +220,7 @@ def recsa_append(geom: Geometry, K: torch.Tensor, V: torch.Tensor, k_new: torch.
 def recsa_decode(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                  tree: torch.Tensor, len_dev: torch.Tensor, n_q: int, O: torch.Tensor,
                  trace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Attend n_q queries per sequence, all at position len_dev[s] - 1."""
     g = geom.c()
     _check(lib().recsa_decode(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree),
                               _ptr(len_dev), n_q, _ptr(O), _ptr(trace), _stream(stream)),
@@ -225,6 +232,7 @@ def recsa_decode_step(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch
                       pooler_r: torch.Tensor, pooler_head_stride: int, tree: torch.Tensor,
                       n_q: int, O: torch.Tensor, trace: Optional[torch.Tensor] = None,
                       stream=None) -> None:
+    """recsa_append followed by recsa_decode, in one launch."""
     g = geom.c()
     _check(lib().recsa_decode_step(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(k_new),
                                    _ptr(v_new), _ptr(len_dev), _ptr(pooler_r),
@@ -236,6 +244,11 @@ def recsa_prefill(geom: Geometry, Q: torch.Tensor, K: torch.Tensor, V: torch.Ten
                   tree: torch.Tensor, q_start: int, n_q: int, O: torch.Tensor,
                   trace: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                   stream=None) -> None:
+    """Causal prefill of queries q_start .. q_start + n_q - 1 (Q and O are
+    [batch][n_q][n_q_heads][head_dim]).  ``workspace``: optional device bytes,
+    at least recsa_prefill_workspace_bytes(geom, n_q); with one and bf16 data
+    the exact window runs on the tensor-core window kernel (RecSA and ZHA
+    modes), without one the tree kernel attends it."""
     g = geom.c()
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().recsa_prefill(ctypes.byref(g), _ptr(Q), _ptr(K), _ptr(V), _ptr(tree), q_start,
