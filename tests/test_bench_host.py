@@ -1,9 +1,13 @@
 """Host logic of bench.py that needs no GPU: the DRAM-traffic figures are read
 from a committed ncu summary only while the kernel sources hash to the value
-the summary records, and only for the workload it was captured on."""
+the summary records, and only for the workload it was captured on; the
+algorithmic bytes of a decode launch (the roofline numerator) agree with a
+hand-worked trace."""
 
 import hashlib
 import os
+
+import numpy as np
 
 import bench
 from hierarchical_sparse_attention_recsa_b200 import recsa as R
@@ -60,3 +64,34 @@ def test_committed_summaries_parse():
     for path in (bench.TRAFFIC_PROFILE, bench.VARIANT_PROFILE):
         text = open(path).read()
         assert "source_sha256: " in text and "traffic_bytes_per_launch" in text
+
+
+def test_decode_bytes_from_a_hand_worked_trace():
+    """B = 4, b = 2, W = 4, k = 1, two query heads on one KV head, d = 4,
+    bf16; one sequence of 20 tokens, so t = 19, a = 4 and levels 3/2/1 hold
+    1/2/4 visible nodes.  Head 0 keeps nodes 0, 0, 1 and head 1 nodes 0, 1, 3
+    (levels 3, 2, 1).  Distinct rows by hand:
+      keys scored   level 3 {0}, level 2 {0, 1}, level 1 {0, 1} | {2, 3}  -> 7
+      unselected    level 3 {}, level 2 {1} | {0}, level 1 {0} | {2}      -> 4
+      exact tokens  leaves {1, 3} (8 tokens) + window [16, 19] (4)        -> 12
+    """
+    from hierarchical_sparse_attention_recsa_b200 import counts
+    B, b, W, k, G, d, elem = 4, 2, 4, 1, 2, 4, 2
+    ints = 4 + 32 + 16 * k
+    tr = np.zeros((1, 1, G, ints), dtype=np.int32)
+    kept = {0: {3: 0, 2: 0, 1: 1}, 1: {3: 0, 2: 1, 1: 3}}
+    for h in range(G):
+        tr[0, 0, h, 0] = 3
+        for lev in (1, 2, 3):
+            tr[0, 0, h, 4 + 16 + lev - 1] = 1
+            tr[0, 0, h, counts.TRACE_HEAD + (lev - 1) * k] = kept[h][lev]
+    lens = np.array([20])
+    r = counts.decode_bytes_from_trace(tr, lens, B, b, W, G, d, elem, k)
+    assert (r["key_rows"], r["val_rows"], r["tok_rows"]) == (7, 4, 12)
+    qo = 2 * 1 * 1 * G * d * elem
+    assert r["bytes"] == qo + 7 * d * 4 + 4 * d * 4 + 12 * d * elem * 2 == 400
+    # ZHA routing: no summary values in the softmax; R key rows per node of
+    # FP8 codes plus a scale
+    z = counts.decode_bytes_from_trace(tr, lens, B, b, W, G, d, elem, k, summary_values=False,
+                                       keys_per_node=3, key_row_bytes=d + 4)
+    assert z["bytes"] == qo + 7 * 3 * (d + 4) + 12 * d * elem * 2
