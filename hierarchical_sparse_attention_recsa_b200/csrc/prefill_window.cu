@@ -17,9 +17,12 @@
 // the A operand of P V), then O = P V.  The result is this window's partial
 // softmax: per (query, head) a row of the caller workspace receives the
 // normalised output, the max and the sum in fp32; the tree kernel folds the
-// summaries and kept leaves into it and writes O once.  Work per CTA is ~20 MFLOP against ~0.3 MB of
-// K/V reads, so the kernel is far from both rooflines; the tree part of the
-// prefill dominates.
+// summaries and kept leaves into it and writes O once.  ZHA routing attends
+// the same window at true positions ("Subquadratic Attention with a
+// Hierarchical Tree-Structured Indexer", Figure 3 caption), so its prefill
+// takes the same partials and its routing kernel merges the reached leaves
+// into them.  Work per CTA is ~20 MFLOP against ~0.3 MB of K/V reads, so the
+// kernel is far from both rooflines; the tree part of the prefill dominates.
 #include <cuda_fp16.h>
 
 #include "recsa_internal.cuh"
