@@ -452,6 +452,35 @@ def test_zha_tiny_p_is_greedy_descent():
                                    atol=1e-12)
 
 
+def test_zha_partial_routing_attends_at_true_positions():
+    """With 0 < p < 1 and RoPE on, the attention is textbook RoPE attention
+    over the reached leaves' tokens and the window, each rotated by its true
+    position (not by its index in the exact list, which equals the position
+    only when every token is reached): checked with complex-number RoPE and a
+    plain softmax, given the oracle's routing (pinned separately above)."""
+    rng = np.random.default_rng(13)
+    B, b, d, T, W = 4, 3, 8, 240, 6
+    K, V = _rand_kv(rng, T, d)
+    r = rng.standard_normal(d)
+    tree = oracle.FullTree(oracle.build_tree(K, V, r, B, b))
+    geo = Geometry(d, 1, 1, B, b, 3, W, rope=True, rope_base=1e3)
+    gaps = 0
+    for t in [50, 117, 239]:
+        for trial in range(4):
+            q = rng.standard_normal(d) * 2
+            res = oracle.zha_route_and_attend(q, t, K, V, tree, geo, top_p=0.6)
+            a = max(0, t + 1 - W) // B
+            leaves = res["kept"].get(1, [])
+            exact = sorted({j for n in leaves for j in range(n * B, n * B + B)} |
+                           set(range(a * B, t + 1)))
+            gaps += int(exact != list(range(exact[0], exact[-1] + 1)))
+            assert res["n_exact"] == len(exact)
+            qr = _rope_complex(q, t, 1e3)
+            Kr = np.stack([_rope_complex(K[j], j, 1e3) for j in exact])
+            np.testing.assert_allclose(res["out"], _sdpa(qr, Kr, V[exact]), atol=1e-12)
+    assert gaps > 0     # some cases skip tokens, where index and position differ
+
+
 # ---------------------------------------------------------------------------
 # Per-KV-group shared selection
 # ---------------------------------------------------------------------------
