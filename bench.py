@@ -247,7 +247,7 @@ def make_prefill_queries(w, K, q0, L, chunk=65536):
 # RecSA arm
 # ---------------------------------------------------------------------------
 
-def run_recsa(args, rank, world, dev):
+def run_recsa(args, rank, world, dev, cpu=None):
     w = synth.WORKLOADS[args.workload]
     if args.length:
         w = synth.Workload(**{**w.__dict__, "length": args.length})
@@ -404,9 +404,9 @@ def run_recsa(args, rank, world, dev):
             out["zha_prefill"] = run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream)
     if not args.no_dense:
         out["dense"] = run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, out.get("prefill"))
-    if rank == 0 and world == 1 and not args.no_cpu:
-        out["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
-    cpu_leg = rank == 0 and world == 1 and not args.no_cpu
+    if cpu is not None:
+        out["cpu_baseline"] = cpu_baseline(cpu, seconds=args.cpu_seconds)
+    cpu_leg = cpu
     if not args.no_zha:
         out["zha"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs,
                                  peak_kind, R.MODE_ZHA, cpu_leg, leg="zha")
@@ -414,11 +414,11 @@ def run_recsa(args, rank, world, dev):
                                           hbm_gbs, peak_kind, R.MODE_ZHA, cpu_leg,
                                           n_ref=ZHA_N_REF, leg="zha_multiref")
         out["zha_multiref_fp8"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
-                                              hbm_gbs, peak_kind, R.MODE_ZHA, False,
+                                              hbm_gbs, peak_kind, R.MODE_ZHA, None,
                                               n_ref=ZHA_N_REF, key_format=R.KEYS_FP8,
                                               leg="zha_multiref_fp8")
         out["zha_multiref_nvfp4"] = run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream,
-                                                hbm_gbs, peak_kind, R.MODE_ZHA, False,
+                                                hbm_gbs, peak_kind, R.MODE_ZHA, None,
                                                 n_ref=ZHA_N_REF, key_format=R.KEYS_NVFP4,
                                                 leg="zha_multiref_nvfp4")
     if not args.no_group:
@@ -504,9 +504,9 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
                        R.KEYS_NVFP4: "nvfp4 (e2m1, e4m3 per 16, fp32 per row)"}[key_format]
     del tree, traces
     torch.cuda.empty_cache()
-    if cpu:
+    if cpu is not None:
         variant = ("zha" if n_ref == 1 else "zha_multiref") if zha else "group"
-        res["cpu_baseline"] = cpu_baseline(args.workload, seconds=min(args.cpu_seconds, 10.0),
+        res["cpu_baseline"] = cpu_baseline(cpu, seconds=min(args.cpu_seconds, 10.0),
                                            variant=variant)
     return res
 
@@ -557,20 +557,45 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
     attend_ms = ms - min(build_t)
     kv_bytes = 2 * L * w.n_kv_heads * w.head_dim * elem_bytes(w)
     build_ms = min(build_t)
+    # bytes the prefill touches (the workload definition's HBM roofline): the
+    # sequence's K and V (every token is in some query's window or kept leaf),
+    # every tree node (fp32 key and value), Q read and O written once
+    nodes = sum(L // (w.leaf_block * w.branching ** l) for l in range(R.recsa_num_levels(gp, L)))
+    tree_bytes = nodes * w.n_kv_heads * w.head_dim * 4 * 2
+    qo_bytes = 2 * (L - q0) * w.n_q_heads * w.head_dim * elem_bytes(w)
+    touched = kv_bytes + tree_bytes + qo_bytes
     del Q, O, tree
     torch.cuda.empty_cache()
+    hbm_ach = touched / (attend_ms / 1e3) / 1e9
     return {"value": (L - q0) / (ms / 1e3), "unit": "tokens/s", "ms": ms,
             "reps": args.prefill_reps, "build_ms": build_ms, "attend_ms": attend_ms,
             "queries": L - q0, "q_start": q0, "tokens_built": L,
-            "roofline": {"bound": "alu",
-                         "kernel": "window_mma_kernel + prefill_warp_kernel",
-                         "achieved": flops / (attend_ms / 1e3) / 1e12,
-                         "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
-                         "frac": flops / (attend_ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS,
-                         "flops": flops, "traffic": None},
-            "build_roofline": {"bound": "hbm", "achieved": kv_bytes / (build_ms / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "kernel": PREFILL_KERNELS,
+                         "achieved": hbm_ach, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": hbm_ach / hbm_gbs, "frac_of_8tbs": hbm_ach / NOMINAL_HBM_GBS,
+                         "bytes": touched, "bytes_kv": kv_bytes, "bytes_tree": tree_bytes,
+                         "bytes_qo": qo_bytes, "traffic": None,
+                         "note": "touched K/V, tree and Q/O over the prefill time (after the "
+                                 "build); the path is compute-bound, see compute_roofline"},
+            "compute_roofline": {"bound": "alu", "kernel": PREFILL_KERNELS,
+                                 "achieved": flops / (attend_ms / 1e3) / 1e12,
+                                 "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
+                                 "frac": flops / (attend_ms / 1e3) / 1e12 / ALU_PEAK_TFLOPS,
+                                 "flops": flops,
+                                 "flops_rule": "2 d (keys read + softmax entries) per query "
+                                               "head, closed-form counts"},
+            "build_roofline": {"bound": "hbm", "kernel": "leaf_kernel + parent_kernel",
+                               "achieved": kv_bytes / (build_ms / 1e3) / 1e9,
                                "peak": hbm_gbs, "unit": "GB/s",
-                               "frac": kv_bytes / (build_ms / 1e3) / 1e9 / hbm_gbs}}
+                               "frac": kv_bytes / (build_ms / 1e3) / 1e9 / hbm_gbs,
+                               "tensor_pipe_frac": 0.0,
+                               "tensor_note": "one reference query: the pooler scores each "
+                                              "row with one dot product (a [B x d] by [d x 1] "
+                                              "product) on CUDA cores; the tensor pipe is "
+                                              "unused"}}
+
+
+PREFILL_KERNELS = "window_mma_kernel + prefill_warp_kernel"
 
 
 ZHA_PREFILL_QUERIES = 65536
@@ -651,6 +676,12 @@ def run_dense(args, w, Kc, Vc, Qs, cap, flush, stream, prefill):
         ms = statistics.median(ts)
         res["decode_ms"] = ms
         res["decode_queries_per_s"] = w.batch / (ms / 1e3)
+        kv = 2 * Kd.numel() * Kd.element_size()
+        hbm_gbs, _, peak_kind = peaks()
+        res["decode_achieved_gbs"] = kv / (ms / 1e3) / 1e9
+        res["decode_hbm_frac"] = res["decode_achieved_gbs"] / hbm_gbs
+        res["decode_note"] = (f"reads all of K and V ({kv / 1e9:.2f} GB) once per step; "
+                              f"fraction of {peak_kind} HBM bandwidth")
     except Exception as e:  # library kernel unavailable for this shape
         res["decode_error"] = str(e).splitlines()[0][:200]
     if prefill is not None and not args.no_dense_prefill and prefill.get("q_start", 0) == 0:
@@ -747,51 +778,116 @@ def _single_thread():
         return None
 
 
-def cpu_baseline(workload=WORKLOAD, seconds=15.0, variant=None):
-    lim = _single_thread()
-    o = OracleDecode(workload)
-    if variant is not None:
-        o.query_heads(o.G, variant)    # untimed: pool the nodes this selection visits first
+# The oracle runs on every host core: one worker process per core, each a
+# single-threaded numpy process over its own queries.  The pool is forked
+# from the parent before CUDA is initialised (a process forked after CUDA
+# initialisation cannot use it safely; the workers use only numpy), and the
+# workers share the parent's oracle inputs copy-on-write.
+_ORACLE = None
+_LIMIT = None
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _worker_init():
+    global _LIMIT
+    _LIMIT = _single_thread()
+
+
+def _worker_time(arg):
+    """One worker: `seconds` of (query, head) pairs of `variant`, starting at
+    its own query; returns (query-heads, seconds)."""
+    variant, seconds, idx = arg
+    o = _ORACLE
+    o.i = idx
+    o.query_heads(o.G, variant)     # untimed: pool the nodes this worker visits first
     t0 = time.perf_counter()
     heads = 0
     while time.perf_counter() - t0 < seconds:
         heads += o.query_heads(o.G, variant)
-    dt = time.perf_counter() - t0
-    del lim
+    return heads, time.perf_counter() - t0
+
+
+def _worker_steps(arg):
+    """One worker's share of `n` reference-arm steps (G query heads each)."""
+    n, idx = arg
+    o = _ORACLE
+    o.i = idx
+    heads = 0
+    for _ in range(n):
+        heads += o.query_heads(o.G)
+    return heads
+
+
+class CpuPool:
+    """The oracle's inputs and a fork pool of one worker per host core."""
+
+    def __init__(self, workload):
+        import multiprocessing
+        global _ORACLE
+        _ORACLE = OracleDecode(workload)
+        self.oracle = _ORACLE
+        self.cores = host_cores()
+        self.pool = multiprocessing.get_context("fork").Pool(self.cores, initializer=_worker_init)
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline(cpu: CpuPool, seconds=15.0, variant=None):
+    o = cpu.oracle
+    t0 = time.perf_counter()
+    res = cpu.pool.map_async(_worker_time, [(variant, seconds, 5 * i)
+                                            for i in range(cpu.cores)],
+                             chunksize=1).get(timeout=seconds + 300)
+    wall = time.perf_counter() - t0
+    heads = sum(h for h, _ in res)
+    dt = max(d for _, d in res)
     what = {None: "decode", "zha": f"ZHA decode (top-p {ZHA_TOP_P})",
             "zha_multiref": f"ZHA decode (top-p {ZHA_TOP_P}, {ZHA_N_REF} reference queries)",
             "group": "group-selection decode"}[variant]
-    return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": 1,
+    return {"value": heads / o.heads_per_query / dt, "unit": "queries/s", "cores": cpu.cores,
             "kind": "oracle",
-            "sample": f"{heads} query-heads ({what} at t=L, one KV head's tree, G={o.G}) in "
-                      f"{dt:.1f} s; queries/s = query-heads/{o.heads_per_query}/s; tree pooling "
-                      "untimed"}
+            "sample": f"{heads} query-heads ({what} at t=L, one KV head's tree, G={o.G}) on "
+                      f"{cpu.cores} worker processes (one per host core, single-threaded "
+                      f"numpy) for {dt:.1f} s each ({wall:.1f} s wall); queries/s = "
+                      f"query-heads/{o.heads_per_query}/s; each worker's first query (its "
+                      "tree pooling) untimed"}
 
 
-def run_reference(args, rank, world):
+def run_reference(args, rank, world, cpu):
     if rank != 0:
         return None
-    lim = _single_thread()
-    o = OracleDecode(args.workload)
-    for _ in range(args.warmup):
-        o.query_heads(o.G)
+    o = cpu.oracle
+    n = cpu.cores
+    cpu.pool.map_async(_worker_steps, [(max(args.warmup, 1), 5 * i) for i in range(n)],
+                       chunksize=1).get(timeout=600)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        o.query_heads(o.G)
+    heads = 0
+    for step in range(args.steps):
+        heads += sum(cpu.pool.map_async(_worker_steps, [(1, 5 * i + args.warmup + step)
+                                                        for i in range(n)],
+                                        chunksize=1).get(timeout=300))
     dt = time.perf_counter() - t0
-    del lim
-    value = args.steps * o.G / o.heads_per_query / dt
+    value = heads / o.heads_per_query / dt
     return {"impl": "reference", "metric": metric_for(args.workload, o.L), "value": value,
             "unit": "queries/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic, seeded",
             "config": {"workload": args.workload, "L": o.L,
-                       "step": f"{o.G} query heads of one decode query (one KV head's tree)",
+                       "step": f"{n} x {o.G} query heads of decode queries (one KV head's "
+                               f"tree), one worker process per host core",
                        "parallelism": "rank 0 only"},
-            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{args.steps} steps x {o.G} query heads; queries/s = "
-                                       f"query-heads/{o.heads_per_query}/s"},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": n, "kind": "oracle",
+                             "sample": f"{args.steps} steps x {n} workers x {o.G} query heads; "
+                                       f"queries/s = query-heads/{o.heads_per_query}/s"},
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -828,17 +924,32 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
-        out = run_reference(args, rank, world)
+        cpu = CpuPool(args.workload) if rank == 0 else None
+        try:
+            out = run_reference(args, rank, world, cpu)
+        finally:
+            if cpu is not None:
+                cpu.close()
         if out is not None:
             print(json.dumps(out), flush=True)
         return
+    # the oracle's worker pool is forked before CUDA is initialised
+    cpu = CpuPool(args.workload) if rank == 0 and world == 1 and not args.no_cpu else None
+    try:
+        _run_gpu(args, rank, world, local, cpu)
+    finally:
+        if cpu is not None:
+            cpu.close()
+
+
+def _run_gpu(args, rank, world, local, cpu):
     torch.cuda.set_device(local)
     if world > 1:
         from datetime import timedelta
         torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
                                              device_id=torch.device("cuda", local))
     R.lib()
-    out = run_recsa(args, rank, world, local)
+    out = run_recsa(args, rank, world, local, cpu)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -10,10 +10,12 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librecsa.so")
+OBJ_DIR = os.path.join(HERE, "_build")
 SOURCES = ["recsa_api.cu", "build.cu", "attend.cu", "decode_cluster.cu",
            "prefill_warp.cu", "prefill_window.cu",
            "prefill_static.cu", "zha_attend.cu"]
@@ -29,26 +31,52 @@ def sources():
     return [os.path.join(CSRC, s) for s in SOURCES]
 
 
+def headers():
+    hs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
+    hs.append(os.path.join(HERE, "..", "include", "recsa.h"))
+    return [h for h in hs if os.path.exists(h)]
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
-    deps.append(os.path.join(HERE, "..", "include", "recsa.h"))
-    return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
+    return any(os.path.getmtime(p) > t for p in sources() + headers())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-cudart", "shared",
-           "-Xcompiler", "-fPIC",
-           "-shared", "-o", tmp, *sources()]
+def _compile(src: str, obj: str, verbose: bool) -> None:
+    cmd = [nvcc_path(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+           "-c", "-o", obj + ".tmp", src]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
+    os.replace(obj + ".tmp", obj)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every translation unit (in parallel, only those older than their
+    source or a header) and link librecsa.so."""
+    if not force and not needs_build():
+        return LIB
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    newest_header = max(os.path.getmtime(h) for h in headers())
+    jobs = []
+    objs = []
+    for src in sources():
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
+        objs.append(obj)
+        if force or not os.path.exists(obj) or \
+                os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header):
+            jobs.append((src, obj))
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    if jobs:
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            for f in [ex.submit(_compile, s_, o_, verbose) for s_, o_ in jobs]:
+                f.result()
+    tmp = LIB + ".tmp"
+    subprocess.run([nvcc_path(), *ARCH, "-shared", "-cudart", "shared", "-o", tmp, *objs],
+                   check=True)
     os.replace(tmp, LIB)
     return LIB
 

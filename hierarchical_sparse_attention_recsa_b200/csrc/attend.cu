@@ -460,8 +460,7 @@ cudaError_t attend_typed(const Params& p, const void* Q, const void* K, const vo
                  size_t(8 + 16 * (kMaxLevels + 1) + 16) * 4;
   if (bytes > 200 * 1024) return cudaErrorInvalidConfiguration;
   auto kern = attend_kernel<T, P>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(bytes));
+  cudaError_t e = ensure_smem(kern, int(bytes));
   if (e != cudaSuccess) return e;
   if (p.batch > 65535 || p.hkv > 65535) return cudaErrorInvalidConfiguration;
   dim3 grid(n_q, p.batch, p.hkv);

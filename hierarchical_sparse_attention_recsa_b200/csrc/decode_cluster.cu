@@ -1225,11 +1225,10 @@ cudaError_t cluster_typed(const Params& p, const void* Q, const void* K, const v
     cs *= 2;
   }
   auto kern = decode_cluster_kernel<T, D, G, HPC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(pl.total));
+  cudaError_t e = ensure_smem(kern, int(pl.total));
   if (e != cudaSuccess) return e;
   if (cs > 8) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = ensure_nonportable_cluster(kern);
     if (e != cudaSuccess) return e;
   }
   if (int64_t(p.batch) * p.hkv > 65535 || n_q > 65535) return cudaErrorNotSupported;
@@ -1273,11 +1272,11 @@ cudaError_t cluster_g(const Params& p, const void* Q, const void* K, const void*
 // (The launch doubles S further when a share's rows do not fit shared memory.)
 void decode_split(const Params& p, int32_t n_q, int& hpc, int& S) {
   const int G = p.group;
-  const char* env = getenv("RECSA_DECODE_SPLIT");
-  if (env) {
-    int h = 0, s = 0;
-    if (sscanf(env, "%d,%d", &h, &s) == 2 && h >= 1 && h <= G && G % h == 0 &&
-        (h & (h - 1)) == 0 && s >= 1 && (s & (s - 1)) == 0 && (G / h) * s <= kMaxCluster) {
+  const Switches& sw = switches();
+  if (sw.split_hpc) {
+    const int h = sw.split_hpc, s = sw.split_s;
+    if (h <= G && G % h == 0 && (h & (h - 1)) == 0 && (s & (s - 1)) == 0 &&
+        (G / h) * s <= kMaxCluster) {
       hpc = h;
       S = s;
       return;

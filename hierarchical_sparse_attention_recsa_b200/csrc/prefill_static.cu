@@ -24,19 +24,28 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side symbol is only a stand-in for it).
-cudaError_t scratch_address(void** out) {
+// Device address of the scratch array on the current device.  The host-side
+// symbol is only a stand-in for it.  Outside stream capture the address is
+// looked up on every call (a host-side table lookup), so a call after a
+// device reset, which reloads the module, gets the array's new address.
+// During capture the address recorded by the last call outside capture is
+// used, and a device never set up that way is refused.
+cudaError_t scratch_address(cudaStream_t s, void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_prefill_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
+  } else if (!g_scratch_ptr[dev]) {
+    return cudaErrorStreamCaptureUnsupported;
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -51,7 +60,7 @@ cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K,
                                   int32_t* trace, cudaStream_t s) {
   if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
   void* ml = nullptr;
-  cudaError_t e = scratch_address(&ml);
+  cudaError_t e = scratch_address(s, &ml);
   if (e != cudaSuccess) return e;
   // The window kernel writes every partial row of the range before the tree
   // kernel reads it, so the array needs no clearing between calls.

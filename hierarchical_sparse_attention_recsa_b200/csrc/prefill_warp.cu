@@ -436,8 +436,7 @@ cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const v
   const size_t bytes = size_t(warp_bytes) * kPWarps;
   if (bytes > 200 * 1024) return cudaErrorNotSupported;
   auto kern = prefill_warp_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(bytes));
+  cudaError_t e = ensure_smem(kern, int(bytes));
   if (e != cudaSuccess) return e;
   const int64_t items = int64_t(n_q) * p.group;
   const int64_t blocks = (items + kPWarps - 1) / kPWarps;

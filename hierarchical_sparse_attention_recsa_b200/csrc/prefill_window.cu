@@ -281,14 +281,14 @@ cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K,
   cudaError_t e;
   if (D == 128) {
     auto kern = window_mma_kernel<128>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    e = ensure_smem(kern, int(bytes));
     if (e != cudaSuccess) return e;
     kern<<<grid, kWThreads, bytes, s>>>(p, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                         (const __nv_bfloat16*)V, tree, q_start, n_q,
                                         (float*)part);
   } else {
     auto kern = window_mma_kernel<64>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+    e = ensure_smem(kern, int(bytes));
     if (e != cudaSuccess) return e;
     kern<<<grid, kWThreads, bytes, s>>>(p, (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
                                         (const __nv_bfloat16*)V, tree, q_start, n_q,

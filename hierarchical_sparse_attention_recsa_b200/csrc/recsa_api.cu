@@ -4,10 +4,97 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include "recsa_internal.cuh"
 
 using namespace recsa;
+
+namespace recsa {
+namespace {
+
+std::mutex g_switch_mutex;
+std::atomic<bool> g_switch_loaded{false};
+Switches g_switches = {};
+
+void read_switches_locked() {
+  Switches sw = {};
+  sw.zha_generic = getenv("RECSA_ZHA_GENERIC") != nullptr;
+  sw.decode_generic = getenv("RECSA_DECODE_GENERIC") != nullptr;
+  sw.prefill_generic = getenv("RECSA_PREFILL_GENERIC") != nullptr;
+  sw.test_expire = getenv("RECSA_TEST_EXPIRE_WAIT") != nullptr;
+  if (const char* e = getenv("RECSA_DECODE_SPLIT")) {
+    int h = 0, sh = 0;
+    if (sscanf(e, "%d,%d", &h, &sh) == 2 && h >= 1 && sh >= 1) {
+      sw.split_hpc = h;
+      sw.split_s = sh;
+    }
+  }
+  if (const char* e = getenv("RECSA_PREFILL_PATH")) sw.prefill_path = atoi(e);
+  g_switches = sw;
+  g_switch_loaded.store(true, std::memory_order_release);
+}
+
+// Dynamic shared memory limits already set, per (kernel, device).
+struct AttrEntry {
+  const void* func;
+  int dev;
+  int smem;
+  int nonportable;
+};
+std::mutex g_attr_mutex;
+AttrEntry g_attr[512];
+int g_attr_n = 0;
+
+AttrEntry* attr_entry_locked(const void* func, int dev) {
+  for (int i = 0; i < g_attr_n; ++i)
+    if (g_attr[i].func == func && g_attr[i].dev == dev) return &g_attr[i];
+  if (g_attr_n == int(sizeof(g_attr) / sizeof(g_attr[0]))) return nullptr;
+  g_attr[g_attr_n] = AttrEntry{func, dev, -1, 0};
+  return &g_attr[g_attr_n++];
+}
+
+}  // namespace
+
+const Switches& switches() {
+  if (!g_switch_loaded.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_switch_mutex);
+    if (!g_switch_loaded.load(std::memory_order_relaxed)) read_switches_locked();
+  }
+  return g_switches;
+}
+
+void reload_switches() {
+  std::lock_guard<std::mutex> lock(g_switch_mutex);
+  read_switches_locked();
+}
+
+cudaError_t ensure_smem(const void* func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  AttrEntry* a = attr_entry_locked(func, dev);
+  if (a && a->smem >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && a) a->smem = bytes;
+  return e;
+}
+
+cudaError_t ensure_nonportable_cluster(const void* func) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  AttrEntry* a = attr_entry_locked(func, dev);
+  if (a && a->nonportable) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess && a) a->nonportable = 1;
+  return e;
+}
+
+}  // namespace recsa
 
 namespace {
 
@@ -131,7 +218,7 @@ recsa_status make_params(const recsa_geometry* g, Params* p) {
   p->inv_sqrt_d = 1.0f / sqrtf(float(g->head_dim));
   // tests of the bounded waits: the decode kernel's chain threads end with a
   // wait that nothing completes, which must expire into RECSA_DEVERR_WAIT_TIMEOUT
-  p->test_expire = getenv("RECSA_TEST_EXPIRE_WAIT") != nullptr;
+  p->test_expire = switches().test_expire;
   return RECSA_OK;
 }
 
@@ -258,7 +345,7 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (p.mode == RECSA_MODE_ZHA) {
-    if (!getenv("RECSA_ZHA_GENERIC")) {
+    if (!switches().zha_generic) {
       // prefill: the window (true-position RoPE there too) on tensor cores first
       const void* wpart = nullptr;
       if (!decode && workspace) {
@@ -269,9 +356,9 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
       }
       e = launch_zha(p, Q, K, V, tree, len_dev, q_start, n_q, decode, O, trace, wpart, s);
     }
-  } else if (decode && !getenv("RECSA_DECODE_GENERIC")) {
+  } else if (decode && !switches().decode_generic) {
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
-  } else if (!decode && !getenv("RECSA_PREFILL_GENERIC")) {
+  } else if (!decode && !switches().prefill_generic) {
     const void* wpart = nullptr;
     if (workspace) {
       e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, workspace, s);
@@ -316,7 +403,7 @@ recsa_status recsa_decode_step(const recsa_geometry* geom, const void* Q, void* 
   if (trace && geom->k > RECSA_TRACE_MAX_K) return RECSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
-  if (!getenv("RECSA_DECODE_GENERIC"))
+  if (!switches().decode_generic)
     e = launch_decode_step(p, Q, K, V, k_new, v_new, len_dev, pooler_r, pooler_head_stride,
                            tree, n_q, O, trace, s);
   if (e == cudaErrorNotSupported) {
@@ -359,7 +446,7 @@ recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (p.mode == RECSA_MODE_ZHA) {
-    if (!getenv("RECSA_ZHA_GENERIC"))
+    if (!switches().zha_generic)
       e = launch_zha(p, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, nullptr, s);
   } else {
     e = launch_prefill_static(p, Q, K, V, tree, q_start, n_q, O, trace, s);
@@ -393,6 +480,8 @@ recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void
   return attend_common(geom, Q, K, V, tree, nullptr, q_start, n_q, 0, O, trace, workspace,
                        workspace_bytes, stream);
 }
+
+void recsa_reload_switches(void) { reload_switches(); }
 
 recsa_status recsa_tree_error(const recsa_geometry* geom, void* tree, int32_t clear,
                               uint32_t* flags, void* stream) {

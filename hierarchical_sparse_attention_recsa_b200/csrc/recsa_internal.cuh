@@ -134,6 +134,34 @@ __device__ __forceinline__ void store_elem(void* base, int64_t idx, float v, int
     reinterpret_cast<float*>(base)[idx] = v;
 }
 
+// Kernel-variant switches taken from the environment (RECSA_ZHA_GENERIC,
+// RECSA_DECODE_GENERIC, RECSA_PREFILL_GENERIC, RECSA_DECODE_SPLIT="hpc,s",
+// RECSA_PREFILL_PATH, RECSA_TEST_EXPIRE_WAIT).  They are read once, on the
+// first call into the library, and again only by recsa_reload_switches(), so
+// no launch pays for getenv().
+struct Switches {
+  int zha_generic, decode_generic, prefill_generic, test_expire;
+  int split_hpc, split_s;   // forced decode launch shape; 0 = automatic
+  int prefill_path;         // forced prefill path (0 = automatic); see recsa_api.cu
+};
+const Switches& switches();
+void reload_switches();
+
+// Raise `func`'s dynamic shared memory limit on the current device to at
+// least `bytes`, calling cudaFuncSetAttribute only when the limit recorded for
+// this (kernel, device) is lower: launches then cost no attribute call.
+cudaError_t ensure_smem(const void* func, int bytes);
+template <typename F>
+cudaError_t ensure_smem(F* func, int bytes) {
+  return ensure_smem(reinterpret_cast<const void*>(func), bytes);
+}
+// cudaFuncAttributeNonPortableClusterSizeAllowed = 1, once per (kernel, device).
+cudaError_t ensure_nonportable_cluster(const void* func);
+template <typename F>
+cudaError_t ensure_nonportable_cluster(F* func) {
+  return ensure_nonportable_cluster(reinterpret_cast<const void*>(func));
+}
+
 // Host-side launchers (defined in the .cu files).
 cudaError_t launch_rope_table(const Params& p, void* tree, double rope_base, cudaStream_t s);
 cudaError_t launch_build(const Params& p, const void* K, const void* V, const int64_t* len_host,

@@ -612,8 +612,7 @@ cudaError_t zha_typed(const Params& p, const void* Q, const void* K, const void*
   if (p.batch > 65535) return cudaErrorNotSupported;
   auto kern = part ? zha_attend_kernel<T, NP, kZPreChain, 0>
                    : zha_attend_kernel<T, NP, kZDecChain, kZDecWin>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(bytes));
+  cudaError_t e = ensure_smem(kern, int(bytes));
   if (e != cudaSuccess) return e;
   dim3 grid(n_q, p.batch, p.hq);
   kern<<<grid, nw * 32, bytes, s>>>(p, reinterpret_cast<const T*>(Q),

@@ -47,7 +47,7 @@ STATUS = {
 EXPORTS = ["recsa_status_string", "recsa_validate", "recsa_num_levels", "recsa_tree_bytes",
            "recsa_build", "recsa_append", "recsa_decode", "recsa_decode_step", "recsa_prefill",
            "recsa_prefill_workspace_bytes", "recsa_prefill_static", "recsa_trace_ints",
-           "recsa_tree_error"]
+           "recsa_tree_error", "recsa_reload_switches"]
 
 
 class RecsaError(RuntimeError):
@@ -139,8 +139,10 @@ def lib() -> ctypes.CDLL:
         L.recsa_prefill_static.argtypes = [G, vp, vp, vp, vp, i64, i32, vp, vp, vp]
         L.recsa_trace_ints.argtypes = [G, ctypes.POINTER(i32)]
         L.recsa_tree_error.argtypes = [G, vp, i32, ctypes.POINTER(ctypes.c_uint32), vp]
+        L.recsa_reload_switches.argtypes = []
+        L.recsa_reload_switches.restype = None
         for name in EXPORTS:
-            if name != "recsa_status_string":
+            if name not in ("recsa_status_string", "recsa_reload_switches"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -282,6 +284,12 @@ def recsa_tree_error(geom: Geometry, tree: torch.Tensor, clear: bool = False,
     _check(lib().recsa_tree_error(ctypes.byref(g), _ptr(tree), int(clear), ctypes.byref(out),
                                   _stream(stream)), "recsa_tree_error")
     return out.value
+
+
+def recsa_reload_switches() -> None:
+    """Make changes of the RECSA_* kernel-variant environment switches take
+    effect (the library reads them once, at its first call)."""
+    lib().recsa_reload_switches()
 
 
 def recsa_status_string(status: int) -> str:

@@ -259,9 +259,13 @@ recsa_status recsa_prefill(const recsa_geometry* geom, const void* Q, const void
  *   query range.  RECSA_MODE_ZHA uses no window partials and no scratch.
  *   The array needs no clearing (each call writes what it reads), but every
  *   call shares it: calls that overlap on the device race.
- *   Set-up: the first call on each device, with that device current, looks up
- *   the array's device address; make that first call before any stream
- *   capture.  Nothing is allocated by this call.
+ *   Set-up: every call made outside stream capture looks up the array's
+ *   device address on the current device (so a call after a device reset,
+ *   which reloads the library's module, finds the array again); a call during
+ *   capture uses the address found by the last call outside capture on that
+ *   device, so make the first call on each device before any stream capture
+ *   (a device never called outside capture is refused with RECSA_ERR_CUDA).
+ *   Nothing is allocated by this call.
  */
 recsa_status recsa_prefill_static(const recsa_geometry* geom, const void* Q, const void* K,
                                   const void* V, const void* tree, int64_t q_start, int32_t n_q,
@@ -279,6 +283,22 @@ recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n
  *   [4 + 32 + (l - 1) * k + j]       j-th kept node id at level l, in position order
  */
 recsa_status recsa_trace_ints(const recsa_geometry* geom, int32_t* ints);
+
+/*
+ * Re-read the environment switches that force a kernel variant (the tests use
+ * them to run every kernel of a call on the same inputs):
+ *   RECSA_DECODE_GENERIC, RECSA_PREFILL_GENERIC, RECSA_ZHA_GENERIC   (set: use
+ *     the generic one-CTA-per-query kernel), RECSA_DECODE_SPLIT="hpc,s" (decode
+ *     launch shape: query heads per CTA, candidate shares per head group),
+ *     RECSA_PREFILL_PATH (unset or 0: automatic; a positive value forces one
+ *     prefill path),
+ *     RECSA_TEST_EXPIRE_WAIT (set: the decode kernel ends with a bounded wait
+ *     that nothing completes, to test the timeout status).
+ * The library reads them once, at its first call; this entry point makes a
+ * change of the environment take effect.  It must not run concurrently with
+ * other calls into the library.  Not part of the method (no passage defines it).
+ */
+void recsa_reload_switches(void);
 
 /* Read (and optionally clear) the device error flags of a tree; synchronises `stream`. */
 recsa_status recsa_tree_error(const recsa_geometry* geom, void* tree, int32_t clear,

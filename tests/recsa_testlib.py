@@ -5,7 +5,7 @@ Tolerances:
   * bf16 inputs: max-abs 2e-2 and mean-abs 2e-3 on outputs and tree summaries
     against the float64 oracle fed the same bf16 values (the target bound);
     the outputs are written in bf16, so the max-abs bound applies beyond that
-    final rounding (half a bf16 ulp of the value, 1/64 at magnitude 8);
+    final rounding (half a bf16 ulp of the value, 1/32 at magnitude 8);
   * fp32 inputs: max-abs 2e-4, mean-abs 2e-5 (fp32 dot products of length
     <= 128 and sums over <= ~2000 softmax entries: a few 1e-6 relative, with
     two orders of margin);
@@ -113,7 +113,7 @@ class Stats:
     """Error statistics of GPU values against oracle values.  For bf16 runs the
     GPU writes its outputs as bf16, so the max-abs bound applies to the error
     beyond that final rounding (half a bf16 ulp of the oracle value): outputs
-    of magnitude 8 or more cannot be written closer than 1/64 in bf16."""
+    of magnitude 8 or more cannot be written closer than 1/32 in bf16."""
 
     def __init__(self):
         self.max_abs = 0.0
@@ -375,3 +375,93 @@ def decode_nvfp4(codes: np.ndarray, bsc: np.ndarray, rsc: np.ndarray) -> np.ndar
     el = np.stack([E2M1_TABLE[c & 0xF], E2M1_TABLE[c >> 4]], axis=-1).reshape(*c.shape[:-1], -1)
     bs = np.repeat(E4M3_TABLE[bsc.astype(np.int64)], 16, axis=-1)
     return el * bs * rsc[..., None]
+
+
+# ---------------------------------------------------------------------------
+# Low-precision key rows: code-level comparison with the oracle's rounding
+# ---------------------------------------------------------------------------
+
+POOL_TOL = 2e-5   # float32 pooling error of a key row, relative to the row's largest element
+
+
+def _e4m3_quantum(v):
+    v = np.abs(np.asarray(v, np.float64))
+    _, e = np.frexp(np.maximum(v, 2.0 ** -9))
+    return np.ldexp(1.0, np.maximum(e - 1, -6) - 3)
+
+
+def _e2m1_step(v):
+    a = np.abs(np.asarray(v, np.float64))
+    return np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+
+
+def nvfp4_row_flips(x, got_el, got_sb, got_g, tol=POOL_TOL):
+    """Compare one NVFP4 key row of the GPU with the oracle's rounding of the
+    float64 pooled row x [d] (ZHA, Figure 16 caption; readings F1b):
+    got_el [d] are the GPU's E2M1 element values, got_sb [d/16] its block
+    scales (E4M3 values), got_g its row scale.  The row scale must equal
+    max|x| / (6 * 448) to float32 pooling error.  A block scale may differ from
+    E4M3(block max / (6 * row scale)) only by one E4M3 step, and only where
+    that quotient lies within pooling error of the midpoint between the two;
+    an element, given the GPU's block and row scales, may differ from the
+    E2M1 rounding of x / (block scale * row scale) only by one E2M1 step, and
+    only where the float32 value of x can fall on the other side of that
+    midpoint.  Returns (element flips, block-scale flips)."""
+    x = np.asarray(x, np.float64)
+    amax = float(np.abs(x).max())
+    if amax == 0.0:
+        assert not np.any(got_el) and got_g == 0.0
+        return 0, 0
+    g_or = amax / (6 * 448)
+    assert abs(got_g - g_or) <= 2 * tol * g_or, (got_g, g_or)
+    fe = fb = 0
+    for bi in range(x.shape[0] // 16):
+        xb = x[bi * 16:(bi + 1) * 16]
+        el = np.asarray(got_el[bi * 16:(bi + 1) * 16], np.float64)
+        ratio = float(np.abs(xb).max()) / (6 * g_or)
+        sb_or = float(oracle.e4m3_round(np.array([ratio]))[0])
+        sb = float(got_sb[bi])
+        if sb != sb_or:
+            fb += 1
+            lo = min(sb, sb_or)
+            assert abs(sb - sb_or) == _e4m3_quantum(lo), (bi, sb, sb_or)
+            # ratio = 448 * blockmax / amax: both from the float32 pooled row
+            assert abs(ratio - (sb + sb_or) / 2) <= 448 * 2 * tol, (bi, ratio, sb, sb_or)
+        if sb == 0.0:
+            assert not np.any(el)
+            continue
+        unit = sb * float(got_g)
+        u = xb / unit
+        want = oracle.e2m1_round(u)
+        bad = el != want
+        if bad.any():
+            fe += int(bad.sum())
+            lo = np.minimum(np.abs(el[bad]), np.abs(want[bad]))
+            assert np.all(np.abs(el[bad] - want[bad]) == _e2m1_step(lo)), (bi, el[bad], want[bad])
+            mid = (el[bad] + want[bad]) / 2
+            assert np.all(np.abs(u[bad] - mid) * unit <= tol * amax), (bi, u[bad], mid)
+    return fe, fb
+
+
+def fp8_row_flips(x, got_codes_val, got_scale, tol=POOL_TOL):
+    """Compare one FP8 key row of the GPU (E4M3 values of the codes, row scale)
+    with the oracle's rounding of the float64 pooled row x (readings F2): the
+    scale equals max|x| / 448 to float32 pooling error; a code may differ from
+    E4M3(x / scale) only by one E4M3 step, only where x / scale lies within
+    pooling error (relative to the row's largest element, 448 in scaled units)
+    of the midpoint.  Returns the number of differing codes."""
+    x = np.asarray(x, np.float64)
+    amax = float(np.abs(x).max())
+    if amax == 0.0:
+        assert not np.any(got_codes_val) and got_scale == 0.0
+        return 0
+    assert abs(got_scale - amax / 448) <= 2 * tol * amax / 448, (got_scale, amax / 448)
+    u = x / float(got_scale)
+    want = oracle.e4m3_round(u)
+    got = np.asarray(got_codes_val, np.float64)
+    bad = got != want
+    if bad.any():
+        lo = np.minimum(np.abs(got[bad]), np.abs(want[bad]))
+        assert np.all(np.abs(got[bad] - want[bad]) == _e4m3_quantum(lo)), (got[bad], want[bad])
+        assert np.all(np.abs(u[bad] - (got[bad] + want[bad]) / 2) <= 448 * tol), u[bad]
+    return int(bad.sum())

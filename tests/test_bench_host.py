@@ -95,3 +95,19 @@ def test_decode_bytes_from_a_hand_worked_trace():
     z = counts.decode_bytes_from_trace(tr, lens, B, b, W, G, d, elem, k, summary_values=False,
                                        keys_per_node=3, key_row_bytes=d + 4)
     assert z["bytes"] == qo + 7 * 3 * (d + 4) + 12 * d * elem * 2
+
+
+def test_oracle_runs_on_every_host_core():
+    """cpu_baseline and the reference arm time the oracle with one worker
+    process per host core and report that count."""
+    cpu = bench.CpuPool("tiny-4k")
+    try:
+        res = bench.cpu_baseline(cpu, seconds=0.3)
+        assert res["cores"] == bench.host_cores() >= 1
+        assert res["value"] > 0 and res["kind"] == "oracle"
+        args = type("A", (), dict(workload="tiny-4k", warmup=1, steps=2))()
+        ref = bench.run_reference(args, 0, 1, cpu)
+        assert ref["impl"] == "reference" and ref["cpu_baseline"]["cores"] == cpu.cores
+        assert ref["value"] > 0 and ref["e2e"]["value"] == ref["value"]
+    finally:
+        cpu.close()

@@ -45,12 +45,14 @@ def decode_impl(request):
         os.environ["RECSA_DECODE_GENERIC"] = "1"
     elif request.param == "cluster-4,1":
         os.environ["RECSA_DECODE_SPLIT"] = "4,1"
+    R.recsa_reload_switches()
     yield request.param
     for k, v in old.items():
         if v is None:
             os.environ.pop(k, None)
         else:
             os.environ[k] = v
+    R.recsa_reload_switches()
 
 
 def _setup(w, lens, capacity, seed=0, k=None, rope=1):

@@ -37,6 +37,7 @@ def _env(generic):
     if generic:
         os.environ["RECSA_ZHA_GENERIC"] = "1"
         os.environ["RECSA_DECODE_GENERIC"] = "1"
+    R.recsa_reload_switches()
 
 
 def _run(w, g, lens, seed):

@@ -40,12 +40,14 @@ def decode_impl(request):
         os.environ["RECSA_DECODE_GENERIC"] = "1"
     elif request.param != "cluster-auto":
         os.environ["RECSA_DECODE_SPLIT"] = request.param.split("-")[1]
+    R.recsa_reload_switches()
     yield request.param
     for k, v in old.items():
         if v is None:
             os.environ.pop(k, None)
         else:
             os.environ[k] = v
+    R.recsa_reload_switches()
 
 
 @pytest.fixture(params=["warp", "window", "generic"])
@@ -56,10 +58,12 @@ def prefill_impl(request):
     old = os.environ.pop("RECSA_PREFILL_GENERIC", None)
     if request.param == "generic":
         os.environ["RECSA_PREFILL_GENERIC"] = "1"
+    R.recsa_reload_switches()
     yield request.param
     os.environ.pop("RECSA_PREFILL_GENERIC", None)
     if old is not None:
         os.environ["RECSA_PREFILL_GENERIC"] = old
+    R.recsa_reload_switches()
 
 
 def _prefill(g, impl, Q, K, V, tree, q0, nq, O, trace=None):
@@ -456,11 +460,13 @@ def test_bounded_wait_expiry_reports_status_and_context_stays_usable():
     O1, O2 = torch.empty_like(Qd), torch.empty_like(Qd)
     assert R.recsa_tree_error(g, tree) == 0
     os.environ["RECSA_TEST_EXPIRE_WAIT"] = "1"
+    R.recsa_reload_switches()
     try:
         R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, 1, O1)
         torch.cuda.synchronize()
     finally:
         os.environ.pop("RECSA_TEST_EXPIRE_WAIT", None)
+        R.recsa_reload_switches()
     assert R.recsa_tree_error(g, tree, clear=True) & R.DEVERR_WAIT_TIMEOUT
     assert R.recsa_tree_error(g, tree) == 0
     R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, 1, O2)

@@ -33,7 +33,8 @@ def _rank_main(rank: int, world: int, port: int, out):
         slowest = bench.max_over_ranks(ms, world)
         rate = bench.job_rate(100, world, slowest)
         ref = bench.run_reference(type("A", (), dict(workload=bench.WORKLOAD, warmup=0,
-                                                     steps=0))(), rank, world) if rank else None
+                                                     steps=0))(), rank, world,
+                                  None) if rank else None
         dist.barrier()
         out.put((rank, slowest, rate, ref))
     finally:
@@ -57,7 +58,6 @@ def test_two_gloo_ranks_take_the_slowest_time_and_the_whole_job_rate():
         assert rate == pytest.approx(200 / 2.25e-3)   # 100 units per rank, 2 ranks
         if rank:
             assert ref is None                     # the reference arm runs on rank 0 only
-
 
 
 def test_one_rank_is_unchanged():

@@ -802,3 +802,91 @@ def test_nvfp4_row_is_block_scaled_e2m1():
             ok = (np.abs(unit - blk / (sb * g)) <= step / 2 + 1e-12) | (np.abs(unit) == 6.0)
             assert ok.all()
     assert not oracle.quantize_row_nvfp4(np.zeros(32)).any()
+
+
+def test_nvfp4_golden_row(golden_dir):
+    """The NVFP4 scale reading pinned by a hand-worked row (tests/golden/nvfp4_row.txt):
+    row scale, block scales (with an E4M3 tie and a rounded scale), element codes
+    (ties to even, saturation after a rounded-down block scale) and a zero block."""
+    xs, codes = [], []
+    with open(os.path.join(golden_dir, "nvfp4_row.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, *vals = line.split()
+            if key == "x":
+                xs += [float(v) for v in vals]
+            elif key == "code":
+                codes += [float(v) for v in vals]
+            elif key == "row_scale":
+                g = float(vals[0])
+            elif key == "block_scale":
+                sb = [float(v) for v in vals]
+    x = np.array(xs)
+    assert x.shape == (64,) and len(codes) == 64 and len(sb) == 4
+    assert g == np.abs(x).max() / (6 * 448)
+    want = np.array(codes) * np.repeat(sb, 16) * g
+    np.testing.assert_array_equal(oracle.quantize_row_nvfp4(x), want)
+
+
+def _f32_nvfp4(x64, rng):
+    """A float32 computation of one NVFP4 row, as a GPU would do it: the
+    pooled row carries float32 error, then every quotient is taken in float32."""
+    amax = np.abs(x64).max()
+    x32 = (x64 + rng.standard_normal(x64.shape) * 1e-7 * amax).astype(np.float32)
+    g32 = np.float32(np.abs(x32).max()) / np.float32(6 * 448)
+    el = np.zeros_like(x64)
+    sbs = np.zeros(x64.shape[0] // 16)
+    for b in range(x64.shape[0] // 16):
+        blk = x32[b * 16:(b + 1) * 16]
+        sb = float(oracle.e4m3_round(np.float32(np.abs(blk).max()) / (np.float32(6) * g32)))
+        sbs[b] = sb
+        if sb > 0:
+            el[b * 16:(b + 1) * 16] = oracle.e2m1_round(blk / (np.float32(sb) * g32))
+    return el, sbs, float(g32)
+
+
+def test_lowprec_row_checkers_accept_float32_rounding_and_reject_planted_errors():
+    """The code-level checkers of the GPU's FP8 / NVFP4 key rows
+    (recsa_testlib.nvfp4_row_flips, fp8_row_flips) accept a float32 computation
+    of the oracle's rounding -- including rows built to sit on rounding
+    midpoints -- and reject a wrong element, a wrong block scale and a wrong
+    row scale."""
+    from recsa_testlib import fp8_row_flips, nvfp4_row_flips
+    rng = np.random.default_rng(50)
+    flips = 0
+    for trial in range(300):
+        x = rng.standard_normal(64) * 10.0 ** rng.uniform(-2, 2)
+        if trial % 3 == 0:      # put some elements exactly on E2M1 midpoints of their block
+            g = np.abs(x).max() / 2688
+            for b in range(4):
+                sb = float(oracle.e4m3_round(np.abs(x[b * 16:(b + 1) * 16]).max() / (6 * g)))
+                x[b * 16 + 3] = 1.25 * sb * g
+                x[b * 16 + 5] = -2.5 * sb * g
+        el, sb, g32 = _f32_nvfp4(x, rng)
+        fe, fb = nvfp4_row_flips(x, el, sb, g32)
+        flips += fe + fb
+        q, s = oracle.quantize_row(x)
+        x32 = (x + rng.standard_normal(64) * 1e-7 * np.abs(x).max()).astype(np.float32)
+        s32 = float(np.float32(np.abs(x32).max()) / np.float32(448))
+        fp8_row_flips(x, oracle.e4m3_round(x32 / np.float32(s32)), s32)
+    assert flips > 0        # the midpoint rows did exercise the one-step allowance
+    x = rng.standard_normal(64)
+    el, sb, g32 = _f32_nvfp4(x, rng)
+    nvfp4_row_flips(x, el, sb, g32)
+    bad = el.copy()
+    i = int(np.argmin(np.abs(np.abs(bad) - 1.0)))      # an element far from any midpoint
+    bad[i] = bad[i] + (2.0 if bad[i] < 4 else -2.0)
+    with pytest.raises(AssertionError):
+        nvfp4_row_flips(x, bad, sb, g32)
+    wrong_sb = sb.copy()
+    wrong_sb[1] = float(oracle.e4m3_round(np.array([sb[1] * 1.3]))[0])
+    with pytest.raises(AssertionError):
+        nvfp4_row_flips(x, el, wrong_sb, g32)
+    with pytest.raises(AssertionError):
+        nvfp4_row_flips(x, el, sb, g32 * 1.01)
+    q, s = oracle.quantize_row(x)
+    q_bad = q.copy()
+    q_bad[7] = q_bad[7] * 1.5 if q_bad[7] != 0 else 1.0
+    with pytest.raises(AssertionError):
+        fp8_row_flips(x, q_bad, s)
