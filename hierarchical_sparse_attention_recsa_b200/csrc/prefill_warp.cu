@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(kPThreads, 3)
 prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                     const T* __restrict__ V, const void* __restrict__ tree, int64_t q_start,
                     int n_q, T* __restrict__ O, int32_t* __restrict__ trace, int cmax, int kmax,
-                    int warp_bytes, const float* __restrict__ wpart) {
+                    int warp_bytes, const float* wpart, LeafOut lo) {
   constexpr int HALF = D / 2, LPR = HALF / 4, SPW = 32 / LPR;
   const int G = p.group;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -357,7 +357,18 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
       run_pass(false, lev, lev + 1, false);
       topk(lev);
     }
-    run_pass(false, 0, 1, true);
+    if (lo.counts) {
+      // kept leaves are attended by the tensor-core leaf path: list them and
+      // take each pair's position in its leaf's pair list
+      const int64_t qh_row = (seq * n_q + qi) * p.hq + h;
+      const int* kept1 = kept + 1 * kmax;
+      for (int s = lane; s < nleaf; s += 32) {
+        const int64_t bucket = (seq * p.hkv + g) * int64_t(lo.nleaf) + kept1[s];
+        const int pos = atomicAdd(lo.counts + bucket, 1);
+        lo.kept[qh_row * lo.kmax + s] = make_int2(int(bucket), pos);
+      }
+    }
+    run_pass(false, 0, 1, lo.counts == nullptr);
   } else if (own_window) {
     run_pass(true, 0, 0, false);
   }
@@ -378,7 +389,42 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
     m = mn;
   }
-  if (lane < LPR) {
+  if (lo.counts) {
+    // partial softmax of the window and the summaries (normalised output, max, sum)
+    const int64_t qh_row = (seq * n_q + qi) * p.hq + h;
+    float mm = m, ra_ = 1.f, rb_ = 0.f;
+    float o1[4], o2[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o1[c] = o2[c] = 0.f;
+    if (!own_window) {
+      const float* wrow = wpart + qh_row * (D + 2);
+      const float2 w = *reinterpret_cast<const float2*>(wrow + D);
+      mm = fmaxf(m, w.x);
+      ra_ = (m == -INFINITY) ? 0.f : __expf(m - mm);
+      rb_ = (w.x == -INFINITY) ? 0.f : __expf(w.x - mm) * w.y;
+      if (lane < LPR) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          o1[c] = wrow[j0 + c];
+          o2[c] = wrow[HALF + j0 + c];
+        }
+      }
+    }
+    const float lsum = l * ra_ + rb_;
+    const float il = 1.f / lsum;
+    // every lane has read its window values before any lane overwrites the row
+    __syncwarp();
+    if (lane < LPR) {
+      float* prow = lo.part + qh_row * (D + 2);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        prow[j0 + c] = (acc[c] * ra_ + o1[c] * rb_) * il;
+        prow[HALF + j0 + c] = (acc[4 + c] * ra_ + o2[c] * rb_) * il;
+      }
+      if (lane == 0) *reinterpret_cast<float2*>(prow + D) = make_float2(mm, lsum);
+    }
+    if (lane == 0) lo.nkept[qh_row] = nleaf;
+  } else if (lane < LPR) {
     if (own_window) {
       const float il = 1.f / l;
 #pragma unroll
@@ -423,7 +469,7 @@ prefill_warp_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 template <typename T, int D>
 cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const void* V,
                           const void* tree, int64_t q_start, int32_t n_q, void* O, int32_t* trace,
-                          const void* wpart, cudaStream_t s) {
+                          const void* wpart, const LeafOut& lo, cudaStream_t s) {
   const int64_t kk = p.k < p.cap ? p.k : p.cap;
   int64_t maxn = 1;
   for (int l = 0; l < p.lay.levels; ++l) maxn = p.lay.nodes[l] > maxn ? p.lay.nodes[l] : maxn;
@@ -446,7 +492,7 @@ cudaError_t prefill_typed(const Params& p, const void* Q, const void* K, const v
                                       reinterpret_cast<const T*>(K),
                                       reinterpret_cast<const T*>(V), tree, q_start, n_q,
                                       reinterpret_cast<T*>(O), trace, cmax, kmax, warp_bytes,
-                                      reinterpret_cast<const float*>(wpart));
+                                      reinterpret_cast<const float*>(wpart), lo);
   return cudaGetLastError();
 }
 
@@ -456,11 +502,24 @@ cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, c
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
                                 int32_t* trace, const void* wpart, cudaStream_t s) {
   if (p.mode != RECSA_MODE_RECSA) return cudaErrorNotSupported;   // other modes: own kernels
+  const LeafOut none = {};
   if (p.dtype == RECSA_DTYPE_BF16)
-    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s)
-                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);
-  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s)
-                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, s);
+    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, none, s)
+                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, none, s);
+  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, none, s)
+                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, O, trace, wpart, none, s);
+}
+
+cudaError_t launch_prefill_warp_leafout(const Params& p, const void* Q, const void* K,
+                                        const void* V, const void* tree, int64_t q_start,
+                                        int32_t n_q, int32_t* trace, const void* wpart,
+                                        const LeafOut& lo, cudaStream_t s) {
+  if (p.mode != RECSA_MODE_RECSA || !lo.counts) return cudaErrorNotSupported;
+  if (p.dtype == RECSA_DTYPE_BF16)
+    return p.d == 128 ? prefill_typed<__nv_bfloat16, 128>(p, Q, K, V, tree, q_start, n_q, nullptr, trace, wpart, lo, s)
+                      : prefill_typed<__nv_bfloat16, 64>(p, Q, K, V, tree, q_start, n_q, nullptr, trace, wpart, lo, s);
+  return p.d == 128 ? prefill_typed<float, 128>(p, Q, K, V, tree, q_start, n_q, nullptr, trace, wpart, lo, s)
+                    : prefill_typed<float, 64>(p, Q, K, V, tree, q_start, n_q, nullptr, trace, wpart, lo, s);
 }
 
 }  // namespace recsa

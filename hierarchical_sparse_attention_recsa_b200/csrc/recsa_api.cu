@@ -360,6 +360,15 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
     e = launch_decode_cluster(p, Q, K, V, tree, len_dev, n_q, O, trace, s);
   } else if (!decode && !switches().prefill_generic) {
     const void* wpart = nullptr;
+    // RECSA_PREFILL_PATH: 0 automatic, 1 window + traversal kernels only (the
+    // kept leaves attended by the traversal), 2 the tensor-core leaf path
+    const int path = switches().prefill_path;
+    if (workspace && path != 1 && prefill_tc_supported(p) &&
+        workspace_bytes >= prefill_tc_workspace_need(p, n_q)) {
+      e = launch_prefill_tc(p, Q, K, V, tree, q_start, n_q, O, trace, workspace, s);
+      if (e != cudaErrorNotSupported) return cuda_status(e);
+      cudaGetLastError();
+    }
     if (workspace) {
       e = launch_prefill_window(p, Q, K, V, tree, q_start, n_q, workspace, s);
       if (e == cudaSuccess) wpart = workspace;
@@ -470,6 +479,9 @@ recsa_status recsa_prefill_workspace_bytes(const recsa_geometry* geom, int32_t n
   if (st != RECSA_OK) return st;
   if (n_q < 0) return RECSA_ERR_CAPACITY;
   *bytes = prefill_workspace_need(p, n_q);
+  // the tensor-core kept-leaf path keeps more intermediates: report its size
+  // where the geometry allows it (a smaller workspace selects the window path)
+  if (prefill_tc_supported(p)) *bytes = std::max(*bytes, prefill_tc_workspace_need(p, n_q));
   return RECSA_OK;
 }
 

@@ -197,6 +197,29 @@ cudaError_t launch_decode_step(const Params& p, const void* Q, void* K, void* V,
 cudaError_t launch_prefill_warp(const Params& p, const void* Q, const void* K, const void* V,
                                 const void* tree, int64_t q_start, int32_t n_q, void* O,
                                 int32_t* trace, const void* wpart, cudaStream_t s);
+// Output of the prefill traversal when the kept leaves are attended by the
+// tensor-core leaf path (prefill_leaf.cu) instead of by the traversal itself.
+struct LeafOut {
+  float* part;    // [rows][d + 2]: partial softmax (normalised output, max, sum) of
+                  // the window and the unselected summaries; may alias the window partials
+  int2* kept;     // [rows][kmax]: {leaf bucket, position in that bucket's pair list}
+  int* nkept;     // [rows]: kept leaves of the query head
+  int* counts;    // [batch * n_kv_heads * nleaf]: pairs per leaf bucket (zeroed first)
+  int nleaf;      // level-1 nodes per (sequence, KV head) at capacity
+  int kmax;       // kept-leaf slots per query head
+};
+// The traversal of launch_prefill_warp writing a LeafOut instead of O.
+cudaError_t launch_prefill_warp_leafout(const Params& p, const void* Q, const void* K,
+                                        const void* V, const void* tree, int64_t q_start,
+                                        int32_t n_q, int32_t* trace, const void* wpart,
+                                        const LeafOut& lo, cudaStream_t s);
+// Prefill with the kept leaves on the tensor cores (prefill_leaf.cu): the
+// workspace holds every intermediate (prefill_tc_workspace_need bytes).
+bool prefill_tc_supported(const Params& p);
+size_t prefill_tc_workspace_need(const Params& p, int32_t n_q);
+cudaError_t launch_prefill_tc(const Params& p, const void* Q, const void* K, const void* V,
+                              const void* tree, int64_t q_start, int32_t n_q, void* O,
+                              int32_t* trace, void* ws, cudaStream_t s);
 // Prefill with the window partials kept in a fixed device array (no caller
 // workspace) of prefill_static_bytes() bytes.
 cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K, const void* V,

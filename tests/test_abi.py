@@ -140,12 +140,25 @@ def test_tree_bytes(lib, kw):
 
 @pytest.mark.parametrize("mode", ["recsa", "zha", "group"])
 def test_prefill_workspace_bytes(lib, mode):
-    # one fp32 window partial (normalised output, max, sum) per query head, in
-    # every mode: ZHA prefill uses the same window partials as RecSA
+    # ZHA and group selection: one fp32 window partial (normalised output, max,
+    # sum) per query head.  RecSA: the tensor-core kept-leaf path's
+    # intermediates, each section 256-byte aligned: the window + summary
+    # partial per query head, one partial per (query head, kept-leaf slot), the
+    # kept-leaf records (int2) and counts, the per-leaf counts and offsets
+    # (int32 per (sequence, KV head, leaf)) and the pairs (int2 per slot).
     extra = {"recsa": {}, "zha": dict(mode=R.MODE_ZHA, top_p=0.9),
              "group": dict(mode=R.MODE_GROUP)}[mode]
     g = geo(batch=2, capacity=4096, **extra)
-    assert R.recsa_prefill_workspace_bytes(g, 100) == 2 * 100 * 32 * (128 + 2) * 4
+    rows = 2 * 100 * 32
+    part = rows * (128 + 2) * 4
+    if mode != "recsa":
+        assert R.recsa_prefill_workspace_bytes(g, 100) == part
+        return
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    kmax, buckets = 8, 2 * 8 * (4096 // 64)
+    want = (up(part) + up(rows * kmax * (128 + 2) * 4) + up(rows * kmax * 8) + up(rows * 4) +
+            2 * up(buckets * 4) + up(rows * kmax * 8))
+    assert R.recsa_prefill_workspace_bytes(g, 100) == want
 
 
 def test_trace_ints(lib):

@@ -50,25 +50,35 @@ def decode_impl(request):
     R.recsa_reload_switches()
 
 
-@pytest.fixture(params=["warp", "window", "generic"])
+@pytest.fixture(params=["warp", "window", "leaf-tc", "generic"])
 def prefill_impl(request):
-    """Select the prefill path: the warp-per-(query, head) kernel alone, the
-    tensor-core window kernel plus the warp kernel (needs a workspace; bf16
-    only, fp32 falls back to the warp kernel), or the generic kernel."""
-    old = os.environ.pop("RECSA_PREFILL_GENERIC", None)
+    """Select the prefill path: the warp-per-(query, head) kernel alone (no
+    workspace), the window kernel plus the warp kernel attending the kept
+    leaves (a workspace of the window partials' size; bf16 only, fp32 falls
+    back to the warp kernel), the tensor-core kept-leaf path (a workspace of
+    recsa_prefill_workspace_bytes), or the generic kernel."""
+    keys = ("RECSA_PREFILL_GENERIC", "RECSA_PREFILL_PATH")
+    old = {k: os.environ.pop(k, None) for k in keys}
     if request.param == "generic":
         os.environ["RECSA_PREFILL_GENERIC"] = "1"
+    elif request.param == "leaf-tc":
+        os.environ["RECSA_PREFILL_PATH"] = "2"
     R.recsa_reload_switches()
     yield request.param
-    os.environ.pop("RECSA_PREFILL_GENERIC", None)
-    if old is not None:
-        os.environ["RECSA_PREFILL_GENERIC"] = old
+    for k, v in old.items():
+        os.environ.pop(k, None)
+        if v is not None:
+            os.environ[k] = v
     R.recsa_reload_switches()
 
 
 def _prefill(g, impl, Q, K, V, tree, q0, nq, O, trace=None):
     ws = None
     if impl == "window":
+        # exactly the window partials: the window + traversal path
+        n = g.batch * nq * g.n_q_heads * (g.head_dim + 2) * 4
+        ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    elif impl == "leaf-tc":
         ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8,
                          device="cuda")
     R.recsa_prefill(g, Q, K, V, tree, q0, nq, O, trace, workspace=ws)
