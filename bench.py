@@ -460,6 +460,8 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
     tree = torch.zeros(R.recsa_tree_bytes(g), dtype=torch.uint8, device="cuda")
     refs = reference_queries(r, n_ref) if n_ref > 1 else r
     R.recsa_build(g, Kc, Vc, [L] * batch, refs, 0, tree)
+    build = time_build(g, Kc, Vc, L, batch, refs, tree, flush, stream, w, n_ref) \
+        if n_ref > 1 else None
     lens = torch.full((batch,), L, dtype=torch.int64, device="cuda")
     O = torch.empty_like(Qs[0])
     n = min(args.steps, Qs.shape[0])
@@ -497,6 +499,8 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
                         "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                         "bytes_per_launch": nbytes,
                         "traffic": measured_variant_traffic(leg, args.workload, L, batch)}}
+    if build is not None:
+        res["build"] = build
     if zha:
         res["top_p"] = ZHA_TOP_P
         res["n_ref"] = n_ref
@@ -509,6 +513,39 @@ def run_variant(args, w, Kc, Vc, r, L, cap, Qs, flush, stream, hbm_gbs, peak_kin
         res["cpu_baseline"] = cpu_baseline(cpu, seconds=min(args.cpu_seconds, 10.0),
                                            variant=variant)
     return res
+
+
+def time_build(g, Kc, Vc, L, batch, refs, tree, flush, stream, w, n_ref, reps=3):
+    """recsa_build of the batch's trees with n_ref reference queries (level 1
+    on the tensor-core pooler: one read of K and V, the scores and the pooling
+    as TF32 products with split fp32 operands).  HBM roofline over the K and V
+    read; tensor fraction = TF32 flops (scores and pooling, each 2 x tokens x d
+    x R x 2 operand parts, R padded to a multiple of 16) over the TF32 peak,
+    taken as the measured bf16 peak x 1/2 (the nominal TF32 : BF16 ratio)."""
+    ts = []
+    for _ in range(reps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        R.recsa_build(g, Kc, Vc, [L] * batch, refs, 0, tree)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(elapsed(e0, e1))
+    ms = min(ts)
+    hbm_gbs, bf16_tflops, peak_kind = peaks()
+    kv = 2 * batch * w.n_kv_heads * L * w.head_dim * elem_bytes(w)
+    nr = (n_ref + 15) // 16 * 16
+    flops = 2 * 2 * 2 * float(batch * w.n_kv_heads * (L // w.leaf_block) * w.leaf_block) * \
+        w.head_dim * nr
+    tf32_peak = bf16_tflops / 2
+    return {"ms": ms, "kernel": "leaf_multiref_tc_kernel + parent_kernel",
+            "roofline": {"bound": "hbm", "achieved": kv / (ms / 1e3) / 1e9, "peak": hbm_gbs,
+                         "unit": "GB/s", "frac": kv / (ms / 1e3) / 1e9 / hbm_gbs,
+                         "peak_kind": peak_kind, "bytes": kv},
+            "tensor": {"achieved": flops / (ms / 1e3) / 1e12, "peak": tf32_peak,
+                       "unit": "TFLOP/s", "frac": flops / (ms / 1e3) / 1e12 / tf32_peak,
+                       "peak_note": "tf32 = measured bf16 x 1/2 (nominal ratio)",
+                       "flops": flops}}
 
 
 def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
@@ -595,7 +632,8 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
                                               "unused"}}
 
 
-PREFILL_KERNELS = "window_mma_kernel + prefill_warp_kernel"
+PREFILL_KERNELS = ("window_mma_kernel + select_kernel + score_tc_kernel + leaf_tc_kernel + "
+                   "merge_kernel (tree levels and kept leaves on tcgen05)")
 
 
 ZHA_PREFILL_QUERIES = 65536

@@ -18,7 +18,8 @@ LIB = os.path.join(HERE, "librecsa.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 SOURCES = ["recsa_api.cu", "build.cu", "attend.cu", "decode_cluster.cu",
            "prefill_warp.cu", "prefill_window.cu",
-           "prefill_static.cu", "zha_attend.cu", "prefill_leaf.cu"]
+           "prefill_static.cu", "zha_attend.cu", "prefill_leaf.cu",
+           "prefill_tree.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -14,6 +14,7 @@
 // parent key from reference j's child keys; the value is the same for all.
 #include "recsa_internal.cuh"
 #include "pool.cuh"
+#include "tc05.cuh"
 
 namespace recsa {
 namespace {
@@ -215,6 +216,266 @@ __global__ void __launch_bounds__(256) parent_kernel(Params p, const float* r, i
   }
 }
 
+// Level 1 with R >= 4 reference queries (bf16 rows, d = 128), on the tensor
+// cores in one pass over K and V: a CTA takes 128 consecutive tokens (128 / B
+// leaves) of one (sequence, KV head) and computes
+//   S = K r^T             [128 tokens x R]   (the pooler scores of every reference),
+//   W = softmax over each leaf's B tokens of S / sqrt(d)   (registers, fp32),
+//   key_l^T = K_l^T W_l   [d x R] per leaf l (the pooled keys of every reference),
+// as tcgen05 TF32 MMAs into TMEM.  K (bf16) is exact in TF32; r and W are fp32
+// and enter as the sum of their high and low TF32 parts (two MMAs each), so
+// both products keep fp32 accuracy ("ZHA", Figure 3 caption: the key nodes of
+// every reference query are stored in parallel; the scores and the pooling
+// are a [B x d] x [d x R] and an [R x B] x [B x d] product per leaf).  The
+// value (the mean of the leaf's values, the same for every reference) is
+// summed on CUDA cores in the same token order as the one-reference kernel.
+constexpr int kMrThreads = 256;
+constexpr unsigned long long kMrWaitNs = 200000000ull;
+
+template <int BL, int NR>
+struct MrSmem {
+  static constexpr int LPT = 128 / BL;                     // leaves per tile
+  static constexpr int kA = 0;                             // K [128 tok][128 d]
+  static constexpr int kA2 = kA + 128 * 128 * 4;           // K^T per leaf [128 d][BL tok]
+  static constexpr int kB1 = kA2 + 128 * 128 * 4;          // r hi, lo [NR][128 d]
+  static constexpr int kB1n = NR * 128 * 4;
+  static constexpr int kB2 = kB1 + 2 * kB1n;               // W hi, lo per leaf [NR][BL tok]
+  static constexpr int kB2n = NR * BL * 4;
+  static_assert(2 * LPT * kB2n >= 16 * 128 * 4, "value partials use the W operand's bytes");
+  static constexpr int kS = kB2 + 2 * LPT * kB2n;          // S [NR][128 tok] fp32
+  static constexpr int kBar = kS + 128 * NR * 4;
+  static constexpr int kTotal = kBar + 32;
+  static constexpr int kPk = kA;       // pooled keys [LPT][NR][128] over the operands (after MMA 2)
+  static constexpr int kCols = NR * (1 + LPT) <= 32 ? 32 : NR * (1 + LPT) <= 64 ? 64
+                               : NR * (1 + LPT) <= 128 ? 128 : NR * (1 + LPT) <= 256 ? 256 : 512;
+  static_assert(kTotal <= 227 * 1024, "multi-reference tile does not fit");
+  static_assert(LPT * NR * 128 * 4 <= kBar, "pooled keys must fit over the operands");
+};
+
+__device__ __forceinline__ int kmj(int R, int r, int k) { return (k >> 2) * 16 * R + r * 16 + (k & 3) * 4; }
+
+__device__ __forceinline__ void st_split4(unsigned char* dst, int lo_off, float a, float b,
+                                          float c, float d) {
+  const float ha = tc05::to_tf32(a), hb = tc05::to_tf32(b), hc = tc05::to_tf32(c),
+              hd = tc05::to_tf32(d);
+  *reinterpret_cast<float4*>(dst) = make_float4(ha, hb, hc, hd);
+  *reinterpret_cast<float4*>(dst + lo_off) =
+      make_float4(tc05::to_tf32(a - ha), tc05::to_tf32(b - hb), tc05::to_tf32(c - hc),
+                  tc05::to_tf32(d - hd));
+}
+
+template <int BL, int NR, int KF>
+__global__ void __launch_bounds__(kMrThreads, 1)
+leaf_multiref_tc_kernel(Params p, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                        const float* r, int64_t r_stride, void* tree, int64_t seq,
+                        int64_t n_leaf) {
+  using L = MrSmem<BL, NR>;
+  constexpr int LPT = L::LPT, D = 128;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::kBar + 16);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.y;
+  const int64_t j0 = int64_t(blockIdx.x) * LPT;             // first leaf of the tile
+  const int nl = int(n_leaf - j0 < LPT ? n_leaf - j0 : LPT);  // leaves present
+  const int ntok = nl * BL;
+  const int R = p.nref;
+  if (warp == 0) {
+    tc05::tmem_alloc(tslot, L::kCols);
+    tc05::tmem_relinquish();
+  }
+  if (tid == 0) {
+    tc05::mbar_init(&bar[0], 1);
+    tc05::mbar_init(&bar[1], 1);
+    tc05::mbar_fence_init();
+  }
+  const __nv_bfloat16* kb = K + ((seq * p.hkv + g) * p.cap + j0 * BL) * D;
+  const __nv_bfloat16* vb = V + ((seq * p.hkv + g) * p.cap + j0 * BL) * D;
+  // K tile ([token][d] for the scores) and, from the same registers, every
+  // leaf's K^T ([d][token] for the pooling); tokens past the leaves are zero
+  for (int task = tid; task < 128 * (D / 8); task += kMrThreads) {
+    const int t = task % 128, c = task / 128;
+    float x[8];
+    if (t < ntok) {
+      const uint4 u = *reinterpret_cast<const uint4*>(kb + int64_t(t) * D + 8 * c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[2 * e] = __uint_as_float(w[e] << 16);
+        x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    }
+    *reinterpret_cast<float4*>(sm + L::kA + kmj(128, t, 8 * c)) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(sm + L::kA + kmj(128, t, 8 * c + 4)) = make_float4(x[4], x[5], x[6], x[7]);
+    unsigned char* kt = sm + L::kA2 + (t / BL) * (D * BL * 4);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) *reinterpret_cast<float*>(kt + kmj(D, 8 * c + e, t % BL)) = x[e];
+  }
+  // values: every thread sums 8 consecutive tokens of 8 channels (16-byte
+  // loads, all issued at once); the groups are added in token order below
+  float* vpart = reinterpret_cast<float*>(sm + L::kB2);    // [128 / 8 groups][128 d]
+  for (int task = tid; task < (128 / 8) * (D / 8); task += kMrThreads) {
+    const int tg = task % 16, c = task / 16;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    uint4 u[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int t = 8 * tg + q;
+      u[q] = t < ntok ? *reinterpret_cast<const uint4*>(vb + int64_t(t) * D + 8 * c)
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t w[4] = {u[q].x, u[q].y, u[q].z, u[q].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += __uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += __uint_as_float(w[e] & 0xffff0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) vpart[tg * D + 8 * c + e] = acc[e];
+  }
+  __syncthreads();
+  for (int task = tid; task < nl * D; task += kMrThreads) {
+    const int leaf = task / D, n = task % D;
+    float acc = 0.f;
+    for (int q = 0; q < BL / 8; ++q) acc += vpart[(leaf * (BL / 8) + q) * D + n];
+    level_vals(p, tree, 1, seq, g)[(j0 + leaf) * D + n] = acc * (1.f / float(BL));
+  }
+  __syncthreads();   // vpart's bytes are the W operand below
+  // r of every reference query (rows >= R are zero), split into TF32 high and low parts
+  for (int task = tid; task < NR * (D / 4); task += kMrThreads) {
+    const int ref = task % NR, c = task / NR;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (ref < R) x = *reinterpret_cast<const float4*>(r + g * r_stride + int64_t(ref) * D + 4 * c);
+    st_split4(sm + L::kB1 + kmj(NR, ref, 4 * c), L::kB1n, x.x, x.y, x.z, x.w);
+  }
+  tc05::fence_smem_to_async();
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  const uint32_t tmem = *tslot;
+  const uint32_t aA = tc05::smem_u32(sm + L::kA), aA2 = tc05::smem_u32(sm + L::kA2);
+  const uint32_t aB1 = tc05::smem_u32(sm + L::kB1), aB2 = tc05::smem_u32(sm + L::kB2);
+  constexpr uint32_t id1 = tc05::idesc(tc05::kFmtTF32, 128, NR);
+  if (tid == 0) {
+#pragma unroll
+    for (int kk = 0; kk < D / 8; ++kk) {
+      const uint32_t a = aA + kk * 32 * 128, b = aB1 + kk * 32 * NR;
+      tc05::mma_tf32(tmem, tc05::desc_kmajor(a, 16 * 128, 128),
+                     tc05::desc_kmajor(b, 16 * NR, 128), id1, kk > 0);
+      tc05::mma_tf32(tmem, tc05::desc_kmajor(a, 16 * 128, 128),
+                     tc05::desc_kmajor(b + L::kB1n, 16 * NR, 128), id1, 1);
+    }
+    tc05::mma_commit(&bar[0]);
+  }
+  bool ok = __syncthreads_and(tid != 0 || tc05::mbar_wait_bounded(&bar[0], 0, kMrWaitNs));
+  tc05::fence_after_sync();
+  float* Ssm = reinterpret_cast<float*>(sm + L::kS);   // [NR][128 tokens]
+  if (warp < 4 && ok) {
+    float sv[NR];
+#pragma unroll
+    for (int c = 0; c < NR / 16; ++c)
+      tc05::tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + 16 * c, sv + 16 * c);
+    tc05::tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < NR; ++c) Ssm[c * 128 + tid] = sv[c] * p.inv_sqrt_d;
+  }
+  __syncthreads();
+  // softmax over each leaf's tokens: one warp per (leaf, reference) column,
+  // lanes over the tokens
+  for (int col = warp; col < LPT * NR; col += kMrThreads / 32) {
+    const int leaf = col / NR, ref = col % NR;
+    const float* s = Ssm + ref * 128 + leaf * BL;
+    constexpr int PER = BL >= 32 ? BL / 32 : 1;
+    float x[PER];
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const int t = lane + 32 * e;
+      x[e] = t < BL ? s[t] : -INFINITY;
+      m = fmaxf(m, x[e]);
+    }
+    m = warp_max(m);
+    float l = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      x[e] = lane + 32 * e < BL ? expf(x[e] - m) : 0.f;
+      l += x[e];
+    }
+    const float il = 1.f / warp_sum(l);
+    unsigned char* wb = sm + L::kB2 + leaf * 2 * L::kB2n;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const int t = lane + 32 * e;
+      if (t < BL) {
+        const float w = x[e] * il, hi = tc05::to_tf32(w);
+        *reinterpret_cast<float*>(wb + kmj(NR, ref, t)) = hi;
+        *reinterpret_cast<float*>(wb + L::kB2n + kmj(NR, ref, t)) = tc05::to_tf32(w - hi);
+      }
+    }
+  }
+  tc05::fence_smem_to_async();
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  if (tid == 0 && ok) {
+    for (int leaf = 0; leaf < LPT; ++leaf) {
+      const uint32_t dcol = tmem + NR * (1 + leaf);
+#pragma unroll
+      for (int kk = 0; kk < BL / 8; ++kk) {
+        const uint32_t a = aA2 + leaf * (D * BL * 4) + kk * 32 * D;
+        const uint32_t b = aB2 + leaf * 2 * L::kB2n + kk * 32 * NR;
+        tc05::mma_tf32(dcol, tc05::desc_kmajor(a, 16 * D, 128),
+                       tc05::desc_kmajor(b, 16 * NR, 128), id1, kk > 0);
+        tc05::mma_tf32(dcol, tc05::desc_kmajor(a, 16 * D, 128),
+                       tc05::desc_kmajor(b + L::kB2n, 16 * NR, 128), id1, 1);
+      }
+    }
+    tc05::mma_commit(&bar[1]);
+  }
+  ok = __syncthreads_and(tid != 0 || !ok || tc05::mbar_wait_bounded(&bar[1], 0, kMrWaitNs)) && ok;
+  tc05::fence_after_sync();
+  // pooled keys: thread t of warps 0-3 holds dimension t of every (leaf, reference)
+  float* Pk = reinterpret_cast<float*>(sm + L::kPk);
+  if (warp < 4 && ok) {
+    for (int leaf = 0; leaf < LPT; ++leaf) {
+#pragma unroll
+      for (int c = 0; c < NR / 16; ++c) {
+        float kv[16];
+        tc05::tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + NR * (1 + leaf) + 16 * c, kv);
+        tc05::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) Pk[(leaf * NR + 16 * c + e) * D + tid] = kv[e];
+      }
+    }
+  }
+  tc05::fence_before_sync();
+  __syncthreads();
+  tc05::fence_after_sync();
+  if (ok) {
+    // key rows (fp32, FP8 or NVFP4 storage, as the one-reference kernel stores them)
+    for (int row = warp; row < nl * R; row += kMrThreads / 32) {
+      const int leaf = row / R, ref = row % R;
+      float key[4];
+      RowIO<float, 4>::load(Pk + (leaf * NR + ref) * D, lane, key);
+      store_node_key<4, KF>(p, tree, 1, seq, g, j0 + leaf, ref, lane, key);
+    }
+  } else if (tid == 0) {
+    atomicOr(tree_error_word(tree), RECSA_DEVERR_WAIT_TIMEOUT);
+    tc05::mbar_wait_bounded(&bar[0], 0, kMrWaitNs);
+    tc05::mbar_wait_bounded(&bar[1], 0, kMrWaitNs);
+  }
+  __syncthreads();
+  if (warp == 0) tc05::tmem_dealloc(tmem, L::kCols);
+}
+
 // Append one token per sequence; pool the leaf and ancestors it completes.
 // One CTA per sequence; warp w handles KV heads w, w + 8, ...  Compiled per
 // key format, as the build kernels are.
@@ -281,6 +542,42 @@ __global__ void rope_table_kernel(float2* table, int rows, int half, int d, doub
   table[idx] = make_float2(float(c), float(s));
 }
 
+template <int BL, int NR, int KF>
+cudaError_t launch_multiref_tc(const Params& p, const void* K, const void* V, const float* r,
+                               int64_t r_stride, void* tree, int64_t seq, int64_t n,
+                               cudaStream_t s) {
+  using L = MrSmem<BL, NR>;
+  auto kern = leaf_multiref_tc_kernel<BL, NR, KF>;
+  cudaError_t e = ensure_smem(kern, L::kTotal);
+  if (e != cudaSuccess) return e;
+  dim3 grid(unsigned((n + L::LPT - 1) / L::LPT), p.hkv);
+  kern<<<grid, kMrThreads, L::kTotal, s>>>(p, reinterpret_cast<const __nv_bfloat16*>(K),
+                                           reinterpret_cast<const __nv_bfloat16*>(V), r,
+                                           r_stride, tree, seq, n);
+  return cudaGetLastError();
+}
+
+// The tensor-core level-1 kernel for R >= 4 reference queries (up to 32),
+// bf16 rows of d = 128 and B in {16, 32, 64}; cudaErrorNotSupported otherwise.
+template <int KF>
+cudaError_t leaf_multiref_dispatch(const Params& p, const void* K, const void* V, const float* r,
+                                   int64_t r_stride, void* tree, int64_t seq, int64_t n,
+                                   cudaStream_t s) {
+  if (p.dtype != RECSA_DTYPE_BF16 || p.d != 128 || p.nref < 4 || p.nref > 32 ||
+      switches().prefill_path == 1)
+    return cudaErrorNotSupported;
+  const bool wide = p.nref > 16;
+#define RECSA_MR_CASE(BLV)                                                                  \
+  if (p.B == BLV)                                                                           \
+    return wide ? launch_multiref_tc<BLV, 32, KF>(p, K, V, r, r_stride, tree, seq, n, s)     \
+                : launch_multiref_tc<BLV, 16, KF>(p, K, V, r, r_stride, tree, seq, n, s);
+  RECSA_MR_CASE(16)
+  RECSA_MR_CASE(32)
+  RECSA_MR_CASE(64)
+#undef RECSA_MR_CASE
+  return cudaErrorNotSupported;
+}
+
 template <typename T, int N, int KF>
 cudaError_t build_format(const Params& p, const void* K, const void* V, const int64_t* len_host,
                          const float* r, int64_t r_stride, void* tree, cudaStream_t s) {
@@ -288,10 +585,16 @@ cudaError_t build_format(const Params& p, const void* K, const void* V, const in
   for (int64_t seq = 0; seq < p.batch; ++seq) {
     int64_t n = len_host[seq] / p.B;
     if (n == 0) continue;
-    dim3 grid(unsigned((n + warps - 1) / warps), p.hkv);
-    leaf_kernel<T, N, KF><<<grid, warps * 32, 0, s>>>(p, reinterpret_cast<const T*>(K),
-                                                  reinterpret_cast<const T*>(V), r, r_stride,
-                                                  tree, seq, n);
+    cudaError_t e = leaf_multiref_dispatch<KF>(p, K, V, r, r_stride, tree, seq, n, s);
+    if (e == cudaErrorNotSupported) {
+      cudaGetLastError();
+      dim3 grid(unsigned((n + warps - 1) / warps), p.hkv);
+      leaf_kernel<T, N, KF><<<grid, warps * 32, 0, s>>>(p, reinterpret_cast<const T*>(K),
+                                                    reinterpret_cast<const T*>(V), r, r_stride,
+                                                    tree, seq, n);
+    } else if (e != cudaSuccess) {
+      return e;
+    }
     for (int lev = 2; lev <= p.lay.levels; ++lev) {
       n /= p.b;
       if (n == 0) break;

@@ -44,12 +44,14 @@ constexpr unsigned long long kLeafWaitNs = 200000000ull;   // 200 ms per MMA wai
 
 struct LeafPaths {
   float* part;       // [rows][d + 2]: window + summaries partial per query head
-  float* lpart;      // [rows * kmax][d + 2]: partial per (query head, slot)
+  float* lpart;      // [rows * kmax][d]: normalised output per (query head, slot)
+  float2* lml;       // [rows * kmax]: its (max, sum)
   int2* kept;        // [rows * kmax]: {leaf bucket, position in the bucket}
   int* nkept;        // [rows]
   int* counts;       // [buckets]
   int* offsets;      // [buckets]
   int2* pairs;       // [rows * kmax]: {query-head row, slot << 24 | query rotation}
+  void* tree_ws;     // the tree levels' workspace (prefill_tree.cu), or null
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -68,26 +70,30 @@ LeafPaths carve(const Params& p, int32_t n_q, void* ws, size_t* total) {
   const size_t rows = size_t(p.batch) * n_q * p.hq;
   const int kmax = kmax_of(p);
   const size_t nb = size_t(buckets_of(p));
-  size_t off[8];
+  size_t off[10];
   off[0] = 0;                                                  // part
   off[1] = align256(off[0] + rows * (p.d + 2) * 4);            // lpart
-  off[2] = align256(off[1] + rows * kmax * (p.d + 2) * 4);     // kept
-  off[3] = align256(off[2] + rows * kmax * 8);                 // nkept
-  off[4] = align256(off[3] + rows * 4);                        // counts
-  off[5] = align256(off[4] + nb * 4);                          // offsets
-  off[6] = align256(off[5] + nb * 4);                          // pairs
-  off[7] = align256(off[6] + rows * kmax * 8);
-  if (total) *total = off[7];
+  off[2] = align256(off[1] + rows * kmax * p.d * 4);           // lml
+  off[3] = align256(off[2] + rows * kmax * 8);                 // kept
+  off[4] = align256(off[3] + rows * kmax * 8);                 // nkept
+  off[5] = align256(off[4] + rows * 4);                        // counts
+  off[6] = align256(off[5] + nb * 4);                          // offsets
+  off[7] = align256(off[6] + nb * 4);                          // pairs
+  off[8] = align256(off[7] + rows * kmax * 8);                 // tree levels
+  off[9] = align256(off[8] + (prefill_tree_supported(p) ? prefill_tree_workspace_need(p, n_q) : 0));
+  if (total) *total = off[9];
   LeafPaths lp = {};
   if (ws) {
     char* base = reinterpret_cast<char*>(ws);
     lp.part = reinterpret_cast<float*>(base + off[0]);
     lp.lpart = reinterpret_cast<float*>(base + off[1]);
-    lp.kept = reinterpret_cast<int2*>(base + off[2]);
-    lp.nkept = reinterpret_cast<int*>(base + off[3]);
-    lp.counts = reinterpret_cast<int*>(base + off[4]);
-    lp.offsets = reinterpret_cast<int*>(base + off[5]);
-    lp.pairs = reinterpret_cast<int2*>(base + off[6]);
+    lp.lml = reinterpret_cast<float2*>(base + off[2]);
+    lp.kept = reinterpret_cast<int2*>(base + off[3]);
+    lp.nkept = reinterpret_cast<int*>(base + off[4]);
+    lp.counts = reinterpret_cast<int*>(base + off[5]);
+    lp.offsets = reinterpret_cast<int*>(base + off[6]);
+    lp.pairs = reinterpret_cast<int2*>(base + off[7]);
+    lp.tree_ws = prefill_tree_supported(p) ? base + off[8] : nullptr;
   }
   return lp;
 }
@@ -314,8 +320,11 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 
   for (int t0 = 0; t0 < cnt && ok; t0 += kTile) {
     const int nt = cnt - t0 < kTile ? cnt - t0 : kTile;
-    // gather and rotate the tile's queries (rows past nt are zero)
-    for (int task = tid; task < kTile * (HALF / 8); task += kLThreads) {
+    // gather and rotate the tile's queries (rows past nt are zero); the
+    // loads of all of a thread's tasks are issued together
+#pragma unroll
+    for (int it = 0; it < kTile * (HALF / 8) / kLThreads; ++it) {
+      const int task = tid + it * kLThreads;
       const int r = task % kTile, c = task / kTile;
       float x1[8], x2[8];
       int rot = 0;
@@ -396,28 +405,43 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
     ok = __syncthreads_and(tid != 0 || !ok || tc05::mbar_wait_bounded(&bar[1], phase, kLeafWaitNs)) && ok;
     tc05::fence_after_sync();
+    // O rows: thread i of warps 0-3 reads row i from TMEM (warp-collective
+    // loads: every lane loads) into a staging copy in the query tile's bytes
+    // (free since the first product completed), 16-byte chunks rotated by the
+    // row so that the writes spread over the banks; then every warp stores
+    // whole rows, coalesced
+    constexpr int CPR = D / 4;                     // 16-byte chunks per row
+    unsigned char* stg = sm + L::kA1;
     if (warp < 4 && ok) {
-      // tcgen05.ld is warp-collective (.sync.aligned): every lane of the warp
-      // loads, and only the lanes of real pairs store
-      const bool real = tid < nt;
-      float* dst = nullptr;
-      if (real) {
-        const int2 pr = lp.pairs[off + t0 + tid];
-        dst = lp.lpart + (int64_t(pr.x) * kmax + (pr.y >> 24)) * (D + 2);
-      }
       const float il = 1.f / l;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        float o[16];
-        tc05::tmem_ld16(tO + (uint32_t(warp * 32) << 16) + 16 * c, o);
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tc05::tmem_ld16(tO + (uint32_t(warp * 32) << 16) + 32 * c, o);
+        tc05::tmem_ld16(tO + (uint32_t(warp * 32) << 16) + 32 * c + 16, o + 16);
         tc05::tmem_wait_ld();
-        if (real) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 2)
-            *reinterpret_cast<float2*>(dst + 16 * c + e) = make_float2(o[e] * il, o[e + 1] * il);
+        for (int e = 0; e < 8; ++e) {
+          const int ch = 8 * c + e;
+          *reinterpret_cast<float4*>(stg + tid * (D * 4) + ((ch + tid) % CPR) * 16) =
+              make_float4(o[4 * e] * il, o[4 * e + 1] * il, o[4 * e + 2] * il, o[4 * e + 3] * il);
         }
       }
-      if (real) *reinterpret_cast<float2*>(dst + D) = make_float2(m, l);
+      if (tid < nt) {
+        const int2 pr = lp.pairs[off + t0 + tid];
+        lp.lml[int64_t(pr.x) * kmax + (pr.y >> 24)] = make_float2(m, l);
+      }
+    }
+    __syncthreads();
+    if (ok) {
+      constexpr int RPW = 32 / CPR;                  // rows per warp instruction
+      const int sub = (threadIdx.x & 31) / CPR, ch = (threadIdx.x & 31) % CPR;
+      for (int r = warp * RPW + sub; r < nt; r += (kLThreads / 32) * RPW) {
+        const int2 pr = lp.pairs[off + t0 + r];
+        float* dst = lp.lpart + (int64_t(pr.x) * kmax + (pr.y >> 24)) * D;
+        *reinterpret_cast<float4*>(dst + 4 * ch) =
+            *reinterpret_cast<const float4*>(stg + r * (D * 4) + ((ch + r) % CPR) * 16);
+      }
     }
     tc05::fence_before_sync();
     __syncthreads();
@@ -450,8 +474,8 @@ __global__ void merge_kernel(Params p, LeafPaths lp, int64_t rows, int kmax, T* 
   for (int c = 0; c < PER; ++c) acc[c] = pr[lane * PER + c] * ml.y;
   const int nk = lp.nkept[row];
   for (int s = 0; s < nk; ++s) {
-    const float* q = lp.lpart + (row * kmax + s) * (D + 2);
-    const float2 ms = *reinterpret_cast<const float2*>(q + D);
+    const float* q = lp.lpart + (row * kmax + s) * D;
+    const float2 ms = lp.lml[row * kmax + s];
     const float mn = fmaxf(M, ms.x);
     const float ra = M == -INFINITY ? 0.f : __expf(M - mn);
     const float rb = __expf(ms.x - mn) * ms.y;
@@ -554,7 +578,9 @@ cudaError_t launch_prefill_tc(const Params& p, const void* Q, const void* K, con
   } else {
     return e;
   }
-  // 2. traversal: summaries + window into lp.part, kept leaves, per-leaf counts
+  // 2. traversal: summaries + window into lp.part, kept leaves, per-leaf counts;
+  // by parent-node tiles on the tensor cores (needs the window partials), else
+  // by the warp-per-query-head kernel
   LeafOut lo;
   lo.part = lp.part;
   lo.kept = lp.kept;
@@ -562,7 +588,13 @@ cudaError_t launch_prefill_tc(const Params& p, const void* Q, const void* K, con
   lo.counts = lp.counts;
   lo.nleaf = int(p.lay.nodes[0]);
   lo.kmax = kmax;
-  e = launch_prefill_warp_leafout(p, Q, K, V, tree, q_start, n_q, trace, wpart, lo, s);
+  e = cudaErrorNotSupported;
+  if (wpart && lp.tree_ws && switches().prefill_path != 2)
+    e = launch_prefill_tree(p, Q, tree, q_start, n_q, trace, lo, lp.tree_ws, s);
+  if (e == cudaErrorNotSupported) {
+    cudaGetLastError();
+    e = launch_prefill_warp_leafout(p, Q, K, V, tree, q_start, n_q, trace, wpart, lo, s);
+  }
   if (e != cudaSuccess) return e;
   // 3. offsets, 4. pairs grouped by leaf
   scan_kernel<<<1, 1024, 0, s>>>(lp.counts, lp.offsets, nb);

@@ -361,7 +361,9 @@ static recsa_status attend_common(const recsa_geometry* geom, const void* Q, con
   } else if (!decode && !switches().prefill_generic) {
     const void* wpart = nullptr;
     // RECSA_PREFILL_PATH: 0 automatic, 1 window + traversal kernels only (the
-    // kept leaves attended by the traversal), 2 the tensor-core leaf path
+    // kept leaves attended by the traversal), 2 the tensor-core leaf path with
+    // the warp-per-query-head traversal, 3 the tensor-core leaf path with the
+    // tree levels as parent-node tiles (the automatic choice when possible)
     const int path = switches().prefill_path;
     if (workspace && path != 1 && prefill_tc_supported(p) &&
         workspace_bytes >= prefill_tc_workspace_need(p, n_q)) {

@@ -213,6 +213,14 @@ cudaError_t launch_prefill_warp_leafout(const Params& p, const void* Q, const vo
                                         const void* V, const void* tree, int64_t q_start,
                                         int32_t n_q, int32_t* trace, const void* wpart,
                                         const LeafOut& lo, cudaStream_t s);
+// The tree levels of a prefill as tensor-core tiles grouped by parent node
+// (prefill_tree.cu): lo.part holds the window partial on entry and the window
+// + summaries partial on return; the kept leaves go to lo.kept/nkept/counts.
+bool prefill_tree_supported(const Params& p);
+size_t prefill_tree_workspace_need(const Params& p, int32_t n_q);
+cudaError_t launch_prefill_tree(const Params& p, const void* Q, const void* tree,
+                                int64_t q_start, int32_t n_q, int32_t* trace, const LeafOut& lo,
+                                void* ws, cudaStream_t s);
 // Prefill with the kept leaves on the tensor cores (prefill_leaf.cu): the
 // workspace holds every intermediate (prefill_tc_workspace_need bytes).
 bool prefill_tc_supported(const Params& p);

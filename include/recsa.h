@@ -290,8 +290,12 @@ recsa_status recsa_trace_ints(const recsa_geometry* geom, int32_t* ints);
  *   RECSA_DECODE_GENERIC, RECSA_PREFILL_GENERIC, RECSA_ZHA_GENERIC   (set: use
  *     the generic one-CTA-per-query kernel), RECSA_DECODE_SPLIT="hpc,s" (decode
  *     launch shape: query heads per CTA, candidate shares per head group),
- *     RECSA_PREFILL_PATH (unset or 0: automatic; a positive value forces one
- *     prefill path),
+ *     RECSA_PREFILL_PATH (unset or 0: automatic; 1: the CUDA-core paths only --
+ *     the prefill's kept leaves attended by its traversal kernel, several
+ *     reference queries pooled by warps; 2: the tensor-core kept-leaf path
+ *     with the warp-per-query-head traversal; 3: the tensor-core kept-leaf
+ *     path with the tree levels as tensor-core tiles, the automatic choice
+ *     when the geometry and the workspace allow it),
  *     RECSA_TEST_EXPIRE_WAIT (set: the decode kernel ends with a bounded wait
  *     that nothing completes, to test the timeout status).
  * The library reads them once, at its first call; this entry point makes a

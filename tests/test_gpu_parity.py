@@ -50,19 +50,24 @@ def decode_impl(request):
     R.recsa_reload_switches()
 
 
-@pytest.fixture(params=["warp", "window", "leaf-tc", "generic"])
+@pytest.fixture(params=["warp", "window", "leaf-tc", "tree-tc", "generic"])
 def prefill_impl(request):
     """Select the prefill path: the warp-per-(query, head) kernel alone (no
     workspace), the window kernel plus the warp kernel attending the kept
     leaves (a workspace of the window partials' size; bf16 only, fp32 falls
-    back to the warp kernel), the tensor-core kept-leaf path (a workspace of
-    recsa_prefill_workspace_bytes), or the generic kernel."""
+    back to the warp kernel), the tensor-core kept-leaf path with the warp
+    traversal ("leaf-tc") or with the tree levels as tensor-core tiles
+    ("tree-tc"; bf16, where the window kernel runs; fp32 falls back to the
+    warp traversal) -- both with a workspace of recsa_prefill_workspace_bytes
+    -- or the generic kernel."""
     keys = ("RECSA_PREFILL_GENERIC", "RECSA_PREFILL_PATH")
     old = {k: os.environ.pop(k, None) for k in keys}
     if request.param == "generic":
         os.environ["RECSA_PREFILL_GENERIC"] = "1"
     elif request.param == "leaf-tc":
         os.environ["RECSA_PREFILL_PATH"] = "2"
+    elif request.param == "tree-tc":
+        os.environ["RECSA_PREFILL_PATH"] = "3"
     R.recsa_reload_switches()
     yield request.param
     for k, v in old.items():
@@ -78,7 +83,7 @@ def _prefill(g, impl, Q, K, V, tree, q0, nq, O, trace=None):
         # exactly the window partials: the window + traversal path
         n = g.batch * nq * g.n_q_heads * (g.head_dim + 2) * 4
         ws = torch.empty(n, dtype=torch.uint8, device="cuda")
-    elif impl == "leaf-tc":
+    elif impl in ("leaf-tc", "tree-tc"):
         ws = torch.empty(R.recsa_prefill_workspace_bytes(g, nq), dtype=torch.uint8,
                          device="cuda")
     R.recsa_prefill(g, Q, K, V, tree, q0, nq, O, trace, workspace=ws)

@@ -829,3 +829,131 @@ def test_zha_prefill_model_small(workspace, zha_impl):
                 check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), q0 + i, Kh, Vh,
                                 src, og, top_p, g.k)
     st.check(torch.bfloat16, f"zha {zha_impl} prefill model small workspace={workspace}")
+
+
+# ---------------------------------------------------------------------------
+# Several reference queries pooled on the tensor cores (R >= 4, bf16, d = 128):
+# one pass over each leaf's K and V (the scores [B x d] x [d x R] and the
+# pooling [R x B] x [B x d] as tcgen05 products with split fp32 operands)
+# ---------------------------------------------------------------------------
+
+def _model_variant(B, b):
+    return synth.Workload(**{**MODEL.__dict__, "leaf_block": B, "branching": b})
+
+
+@pytest.mark.parametrize("Rn,B", [(16, 64), (20, 64), (16, 32), (16, 16)])
+def test_zha_multiref_tc_tree_matches_oracle(Rn, B):
+    """Every node of a model-shaped multi-reference tree (level 1 on the
+    tensor-core pooler, higher levels pooling its keys) against the float64
+    oracle, at the fp32 tolerance: two sequences of ragged lengths, so the
+    last tile of a sequence holds fewer than 128 / B leaves."""
+    w = _model_variant(B, 16 if B == 64 else 8)
+    lens = [20000, 13001]
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(w, lens, 20480, 0.9, Rn, seed=200 + Rn + B)
+    st = Stats()
+    for s, L in enumerate(lens):
+        for h in (0, 5):
+            Kh, Vh = to_np(K[s, h, :L]), to_np(V[s, h, :L])
+            levels = oracle.build_tree_multi(Kh, Vh, Rq.double().numpy(), g.leaf_block,
+                                             g.branching)
+            for lev, (kk, vv) in enumerate(levels, start=1):
+                gk, gv = read_tree_level(g, tree, lev)
+                n = kk.shape[0]
+                st.add(to_np(gk[s, h, :n]), kk)
+                st.add(to_np(gv[s, h, :n]), vv)
+    st.check(torch.float32, f"multiref tc tree R={Rn} B={B}")
+
+
+@pytest.mark.parametrize("key_format", [R.KEYS_FP8, R.KEYS_NVFP4])
+def test_zha_multiref_tc_lowprec_tree_codes(key_format):
+    """Level-1 FP8 / NVFP4 key rows written from the tensor-core pooler are the
+    oracle's rounding of the float64 pooled keys, up to one step at a rounding
+    midpoint (recsa_testlib.fp8_row_flips / nvfp4_row_flips)."""
+    L, Rn = 6000, 16
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_fp8(MODEL, [L], 6144, 0.9, Rn, seed=210,
+                                               key_format=key_format)
+    Rn_np = Rq.double().numpy()
+    d = g.head_dim
+    for h in (0, 3):
+        Kh = to_np(K[0, h, :L])
+        n = L // g.leaf_block
+        flips = 0
+        if key_format == R.KEYS_FP8:
+            codes, scales, _ = read_tree_level_fp8(g, tree, 1)
+            got = E4M3_TABLE[codes[0, h, :n].cpu().numpy().astype(np.int64)]
+            sc = scales[0, h, :n].cpu().numpy().astype(np.float64)
+        else:
+            codes, bsc, rsc, _ = read_tree_level_nvfp4(g, tree, 1)
+            c = codes[0, h, :n].cpu().numpy().astype(np.int64)
+            el = np.stack([E2M1_TABLE[c & 0xF], E2M1_TABLE[c >> 4]], axis=-1).reshape(n, Rn, d)
+            sb = E4M3_TABLE[bsc[0, h, :n].cpu().numpy().astype(np.int64)]
+            rs = rsc[0, h, :n].cpu().numpy().astype(np.float64)
+        for j in range(n):
+            for ref in range(Rn):
+                x = oracle.pool_keys(Kh[j * g.leaf_block:(j + 1) * g.leaf_block], Rn_np[ref])
+                if key_format == R.KEYS_FP8:
+                    flips += fp8_row_flips(x, got[j, ref], sc[j, ref])
+                else:
+                    fe, fb = nvfp4_row_flips(x, el[j, ref], sb[j, ref], rs[j, ref])
+                    flips += fe + fb
+        assert flips <= max(2, 0.01 * n * Rn * d), flips
+
+
+def test_zha_multiref_tc_append_matches_build():
+    """Appending tokens (level 1 pooled on CUDA cores) gives, to fp32 rounding,
+    the nodes a fresh build pooled on the tensor cores (R = 16)."""
+    w, top_p, Rn = MODEL, 0.9, 16
+    lens0 = [4000, 4031]
+    steps = 70
+    cap = 4096 + 256
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(w, lens0, cap, top_p, Rn, seed=220)
+    Kw, Vw = Kd.clone(), Vd.clone()
+    Kw[0, :, 4000:] = 0
+    Vw[0, :, 4000:] = 0
+    Kw[1, :, 4031:] = 0
+    Vw[1, :, 4031:] = 0
+    lens_d = torch.tensor(lens0, dtype=torch.int64, device="cuda")
+    for step in range(steps):
+        kn = torch.stack([Kd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        vn = torch.stack([Vd[s, :, lens0[s] + step] for s in range(2)]).contiguous()
+        R.recsa_append(g, Kw, Vw, kn, vn, lens_d, Rd, 0, tree)
+    new_lens = [L + steps for L in lens0]
+    fresh = alloc_tree(g)
+    R.recsa_build(g, Kd, Vd, new_lens, Rd, 0, fresh)
+    torch.cuda.synchronize()
+    for lev in range(1, R.recsa_num_levels(g, max(new_lens)) + 1):
+        a_k, a_v = read_tree_level(g, tree, lev)
+        b_k, b_v = read_tree_level(g, fresh, lev)
+        for s in range(2):
+            n = new_lens[s] // (g.leaf_block * g.branching ** (lev - 1))
+            torch.testing.assert_close(a_k[s, :, :n], b_k[s, :, :n], rtol=0, atol=2e-6)
+            torch.testing.assert_close(a_v[s, :, :n], b_v[s, :, :n], rtol=0, atol=1e-6)
+
+
+def test_zha_multiref_tc_decode_model(zha_impl):
+    """Routing over a tensor-core-pooled tree (R = 16) on both ZHA kernels,
+    checked against the oracle with the routing rule of check_query_zha."""
+    lens, top_p, Rn = [20000, 13001], 0.9, 16
+    g, K, V, Rq, Kd, Vd, Rd, tree = _setup_multi(MODEL, lens, 20480, top_p, Rn, seed=230)
+    nq = 2
+    pos = torch.tensor([[L - 1] * nq for L in lens], dtype=torch.int64)
+    Q, _, _ = synth.make_queries(MODEL, K, pos, seed=231, n_needles=2)
+    Qd = Q.cuda()
+    O = torch.empty_like(Qd)
+    trace = torch.zeros((2, nq, g.n_q_heads, R.recsa_trace_ints(g)), dtype=torch.int32,
+                        device="cuda")
+    lens_d = torch.tensor(lens, dtype=torch.int64, device="cuda")
+    R.recsa_decode(g, Qd, Kd, Vd, tree, lens_d, nq, O, trace)
+    torch.cuda.synchronize()
+    og = oracle_geometry(g)
+    O_, tr = to_np(O), trace.cpu().numpy()
+    st = Stats()
+    G = g.n_q_heads // g.n_kv_heads
+    for s, L in enumerate(lens):
+        for h in (0, 7, 21, 30):
+            Kh, Vh = to_np(K[s, h // G, :L]), to_np(V[s, h // G, :L])
+            src = oracle.LazyMultiTree(Kh, Vh, Rq.double().numpy(), g.leaf_block, g.branching)
+            for i in range(nq):
+                check_query_zha(st, O_[s, i, h], tr[s, i, h], to_np(Q[s, i, h]), L - 1, Kh, Vh,
+                                src, og, top_p, g.k)
+    st.check(torch.bfloat16, f"zha {zha_impl} multiref tc decode model")
