@@ -19,7 +19,7 @@ OBJ_DIR = os.path.join(HERE, "_build")
 SOURCES = ["recsa_api.cu", "build.cu", "attend.cu", "decode_cluster.cu",
            "prefill_warp.cu", "prefill_window.cu",
            "prefill_static.cu", "zha_attend.cu", "prefill_leaf.cu",
-           "prefill_tree.cu"]
+           "prefill_tree.cu", "window_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -38,8 +38,8 @@
 namespace recsa {
 namespace {
 
-constexpr int kLThreads = 256;
-constexpr int kTile = 128;                   // pairs per tile (MMA rows)
+constexpr int kLThreads = 128;
+constexpr int kTile = 64;                    // pairs per tile (MMA rows, M = 64)
 constexpr unsigned long long kLeafWaitNs = 200000000ull;   // 200 ms per MMA wait
 
 struct LeafPaths {
@@ -170,15 +170,10 @@ struct LeafSmem {
   static constexpr int kB1 = kA1 + NS * kA1n;         // keys      [BL][D]
   static constexpr int kA2 = kB1 + NS * kB1n;         // probs     [128][BL]
   static constexpr int kB2 = kA2 + NS * kA2n;         // values^T  [D][BL]
-  static constexpr int kBar = kB2 + NS * kB2n;        // 2 mbarriers + TMEM address
+  static constexpr int kDst = kB2 + NS * kB2n;        // per tile row: partial offset
+  static constexpr int kBar = kDst + kTile * 8;       // 2 mbarriers + TMEM address
   static constexpr int kTotal = kBar + 32;
-  // Allocated: every operand read the descriptors can describe (either
-  // reading of their two strides) stays inside the CTA's shared memory.
-  static constexpr int kAlloc = 210 * 1024;
-  static constexpr bool kFits =
-      kTotal <= kAlloc &&
-      kB2 + (NS - 1) * kB2n + 32 * (BL / 8 - 1) * D + 16 * D + 16 * (D - 8) + 16 * BL + 128 <=
-          kAlloc;
+  static constexpr bool kFits = kTotal <= 227 * 1024;
 };
 
 // Element (r, k) of a K-major no-swizzle fp32 operand with R rows: byte offset.
@@ -258,7 +253,7 @@ __device__ __forceinline__ void rotate_store(const Params& p, const float2* rope
 // in registers (thread i owns pair i), O = P V on tcgen05, and the pair's
 // partial (normalised output, max, sum) is written out.
 template <typename T, int D, int BL, int NS>
-__global__ void __launch_bounds__(kLThreads, 1)
+__global__ void __launch_bounds__(kLThreads, 2)
 leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
                const T* __restrict__ V, void* tree, LeafPaths lp, int kmax, int nleaf) {
   using L = LeafSmem<D, BL, NS>;
@@ -320,25 +315,36 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
 
   for (int t0 = 0; t0 < cnt && ok; t0 += kTile) {
     const int nt = cnt - t0 < kTile ? cnt - t0 : kTile;
-    // gather and rotate the tile's queries (rows past nt are zero); the
-    // loads of all of a thread's tasks are issued together
+    // gather and rotate the tile's queries (rows past nt are zero); every load
+    // of this thread's tasks is issued before any store
+    constexpr int NT = kTile * (HALF / 8) / kLThreads;
+    int2 prs[NT];
 #pragma unroll
-    for (int it = 0; it < kTile * (HALF / 8) / kLThreads; ++it) {
+    for (int it = 0; it < NT; ++it) {
+      const int r = (tid + it * kLThreads) % kTile;
+      prs[it] = r < nt ? lp.pairs[off + t0 + r] : make_int2(0, 0);
+    }
+    float xa[NT][8], xb[NT][8];
+#pragma unroll
+    for (int it = 0; it < NT; ++it) {
       const int task = tid + it * kLThreads;
       const int r = task % kTile, c = task / kTile;
-      float x1[8], x2[8];
-      int rot = 0;
       if (r < nt) {
-        const int2 pr = lp.pairs[off + t0 + r];
-        rot = pr.y & 0xffffff;
-        const T* q = Q + int64_t(pr.x) * D;
-        load8<T>(q + 8 * c, x1);
-        load8<T>(q + HALF + 8 * c, x2);
+        const T* q = Q + int64_t(prs[it].x) * D;
+        load8<T>(q + 8 * c, xa[it]);
+        load8<T>(q + HALF + 8 * c, xb[it]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x1[e] = x2[e] = 0.f;
+        for (int e = 0; e < 8; ++e) xa[it][e] = xb[it][e] = 0.f;
       }
-      rotate_store(p, rope, rot, 8 * c, x1, x2, sm + L::kA1, NS > 1 ? L::kA1n : 0, kTile, r);
+    }
+#pragma unroll
+    for (int it = 0; it < NT; ++it) {
+      const int task = tid + it * kLThreads;
+      const int r = task % kTile, c = task / kTile;
+      const int rot = r < nt ? (prs[it].y & 0xffffff) : 0;
+      rotate_store(p, rope, rot, 8 * c, xa[it], xb[it], sm + L::kA1, NS > 1 ? L::kA1n : 0,
+                   kTile, r);
     }
     tc05::fence_smem_to_async();
     tc05::fence_before_sync();
@@ -361,9 +367,14 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
     ok = __syncthreads_and(tid != 0 || tc05::mbar_wait_bounded(&bar[0], phase, kLeafWaitNs));
     tc05::fence_after_sync();
+    // M = 64 accumulators: row 16 w + i sits in TMEM lane 32 w + i (i < 16);
+    // lane i < 16 of warp w owns that row, the other lanes take part in the
+    // warp-collective loads only
+    const int lane = tid & 31;
+    const int myrow = 16 * warp + lane;
+    const bool rowthr = lane < 16;
     float m = -INFINITY, l = 0.f;
-    if (warp < 4 && ok) {
-      // thread i owns pair i: its BL logits from TMEM lanes 32 w + lane
+    if (ok) {
       float s[BL];
 #pragma unroll
       for (int c = 0; c < BL / 16; ++c)
@@ -379,10 +390,12 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         s[c] = __expf(s[c] - m);
         l += s[c];
       }
+      if (rowthr) {
 #pragma unroll
-      for (int c = 0; c < BL; c += 4)
-        store4(sm + L::kA2 + kmaj(kTile, tid, c), NS > 1 ? L::kA2n : 0, s[c], s[c + 1],
-               s[c + 2], s[c + 3]);
+        for (int c = 0; c < BL; c += 4)
+          store4(sm + L::kA2 + kmaj(kTile, myrow, c), NS > 1 ? L::kA2n : 0, s[c], s[c + 1],
+                 s[c + 2], s[c + 3]);
+      }
     }
     tc05::fence_smem_to_async();
     tc05::fence_before_sync();
@@ -405,14 +418,15 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
     }
     ok = __syncthreads_and(tid != 0 || !ok || tc05::mbar_wait_bounded(&bar[1], phase, kLeafWaitNs)) && ok;
     tc05::fence_after_sync();
-    // O rows: thread i of warps 0-3 reads row i from TMEM (warp-collective
-    // loads: every lane loads) into a staging copy in the query tile's bytes
-    // (free since the first product completed), 16-byte chunks rotated by the
-    // row so that the writes spread over the banks; then every warp stores
-    // whole rows, coalesced
+    // O rows: the row's owner reads it from TMEM (warp-collective loads:
+    // every lane loads) into a staging copy in the query tile's bytes (free
+    // since the first product completed), 16-byte chunks rotated by the row so
+    // that the writes spread over the banks; then every warp stores whole
+    // rows, coalesced
     constexpr int CPR = D / 4;                     // 16-byte chunks per row
     unsigned char* stg = sm + L::kA1;
-    if (warp < 4 && ok) {
+    static_assert(kTile * D * 4 <= L::kA1n, "staging fits the query tile");
+    if (ok) {
       const float il = 1.f / l;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -420,25 +434,31 @@ leaf_tc_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
         tc05::tmem_ld16(tO + (uint32_t(warp * 32) << 16) + 32 * c, o);
         tc05::tmem_ld16(tO + (uint32_t(warp * 32) << 16) + 32 * c + 16, o + 16);
         tc05::tmem_wait_ld();
+        if (rowthr) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = 8 * c + e;
-          *reinterpret_cast<float4*>(stg + tid * (D * 4) + ((ch + tid) % CPR) * 16) =
-              make_float4(o[4 * e] * il, o[4 * e + 1] * il, o[4 * e + 2] * il, o[4 * e + 3] * il);
+          for (int e = 0; e < 8; ++e) {
+            const int ch = 8 * c + e;
+            *reinterpret_cast<float4*>(stg + myrow * (D * 4) + ((ch + myrow) % CPR) * 16) =
+                make_float4(o[4 * e] * il, o[4 * e + 1] * il, o[4 * e + 2] * il,
+                            o[4 * e + 3] * il);
+          }
         }
       }
-      if (tid < nt) {
-        const int2 pr = lp.pairs[off + t0 + tid];
-        lp.lml[int64_t(pr.x) * kmax + (pr.y >> 24)] = make_float2(m, l);
+      if (rowthr && myrow < nt) {
+        const int2 pr = lp.pairs[off + t0 + myrow];
+        const int64_t slot = int64_t(pr.x) * kmax + (pr.y >> 24);
+        lp.lml[slot] = make_float2(m, l);
+        reinterpret_cast<int64_t*>(sm + L::kDst)[myrow] = slot * D;
       }
     }
     __syncthreads();
     if (ok) {
+      // destination rows from shared memory: no global load between the stores
       constexpr int RPW = 32 / CPR;                  // rows per warp instruction
       const int sub = (threadIdx.x & 31) / CPR, ch = (threadIdx.x & 31) % CPR;
+      const int64_t* dsts = reinterpret_cast<const int64_t*>(sm + L::kDst);
       for (int r = warp * RPW + sub; r < nt; r += (kLThreads / 32) * RPW) {
-        const int2 pr = lp.pairs[off + t0 + r];
-        float* dst = lp.lpart + (int64_t(pr.x) * kmax + (pr.y >> 24)) * D;
+        float* dst = lp.lpart + dsts[r];
         *reinterpret_cast<float4*>(dst + 4 * ch) =
             *reinterpret_cast<const float4*>(stg + r * (D * 4) + ((ch + r) % CPR) * 16);
       }
@@ -501,10 +521,10 @@ cudaError_t leaf_typed(const Params& p, const void* Q, const void* K, const void
     return cudaErrorNotSupported;
   } else {
     auto kern = leaf_tc_kernel<T, D, BL, NS>;
-    cudaError_t e = ensure_smem(kern, L::kAlloc);
+    cudaError_t e = ensure_smem(kern, L::kTotal);
     if (e != cudaSuccess) return e;
     const int nleaf = int(p.lay.nodes[0]);
-    kern<<<unsigned(buckets_of(p)), kLThreads, L::kAlloc, s>>>(
+    kern<<<unsigned(buckets_of(p)), kLThreads, L::kTotal, s>>>(
         p, reinterpret_cast<const T*>(Q), reinterpret_cast<const T*>(K),
         reinterpret_cast<const T*>(V), tree, lp, kmax, nleaf);
     return cudaGetLastError();

@@ -40,10 +40,12 @@ constexpr unsigned long long kTreeWaitNs = 200000000ull;
 struct TreeBufs {
   float* scores;     // [rows][cmax]: the current level's logits
   int* kept;         // [2][rows][kmax]: kept nodes of the last two levels (by parity)
-  int4* stage;       // [rows][kmax + 1]: the next level's runs {row, i0 | n << 16, rot, 0}
+  int4* stage;       // [rows][kmax + 1]: the next level's runs {row, i0 | n << 16, rot, run}
   int2* spos;        // [rows][kmax + 1]: {bucket, position in the bucket}
   int* nruns;        // [rows]
   int4* pairs;       // [rows * (kmax + 1)]: runs grouped by parent
+  float* runpart;    // [rows][kmax + 1][d]: per run, sum_j exp(s_j - m_run) value_j
+  float2* runml;     // [rows][kmax + 1]: per run, (m_run, sum_j exp(s_j - m_run))
   int* counts;       // per level l: [batch][hkv][np_l] at cbase[l]
   int* offsets;
   int64_t cbase[kMaxLevels + 2];
@@ -80,7 +82,7 @@ TreeBufs tree_carve(const Params& p, int32_t n_q, void* ws, size_t* total) {
     nb += size_t(p.batch) * p.hkv * t.np[l];
   }
   const size_t runs = rows * (t.kmax + 1);
-  size_t off[9];
+  size_t off[11];
   off[0] = 0;                                           // scores
   off[1] = al256(off[0] + rows * t.cmax * 4);           // kept
   off[2] = al256(off[1] + 2 * rows * t.kmax * 4);       // stage
@@ -89,8 +91,10 @@ TreeBufs tree_carve(const Params& p, int32_t n_q, void* ws, size_t* total) {
   off[5] = al256(off[4] + rows * 4);                    // pairs
   off[6] = al256(off[5] + runs * 16);                   // counts
   off[7] = al256(off[6] + nb * 4);                      // offsets
-  off[8] = al256(off[7] + nb * 4);
-  if (total) *total = off[8];
+  off[8] = al256(off[7] + nb * 4);                      // runpart
+  off[9] = al256(off[8] + runs * p.d * 4);              // runml
+  off[10] = al256(off[9] + runs * 8);
+  if (total) *total = off[10];
   if (ws) {
     char* b = reinterpret_cast<char*>(ws);
     t.scores = reinterpret_cast<float*>(b + off[0]);
@@ -101,6 +105,8 @@ TreeBufs tree_carve(const Params& p, int32_t n_q, void* ws, size_t* total) {
     t.pairs = reinterpret_cast<int4*>(b + off[5]);
     t.counts = reinterpret_cast<int*>(b + off[6]);
     t.offsets = reinterpret_cast<int*>(b + off[7]);
+    t.runpart = reinterpret_cast<float*>(b + off[8]);
+    t.runml = reinterpret_cast<float2*>(b + off[9]);
   }
   return t;
 }
@@ -184,6 +190,7 @@ select_kernel(Params p, TreeBufs tb, LeafOut lo, const void* __restrict__ tree, 
     const int kup = L < top ? kL1 : 0;
     const int vup = vL1;
     const float* sc = tb.scores + int64_t(row) * tb.cmax;
+    const float* vals = level_vals(p, const_cast<void*>(tree), L, seq, g);
     // candidate i -> node: children of the kept parents, then the orphans
     auto node_of = [&](int i) -> int {
       if (i < p.b * kup) return keptUp[div_b(p, i)] * p.b + mod_b(p, i);
@@ -191,13 +198,11 @@ select_kernel(Params p, TreeBufs tb, LeafOut lo, const void* __restrict__ tree, 
     };
     float sv[kSelRegSlots];
     unsigned key[kSelRegSlots];
-    float mloc = -INFINITY;
 #pragma unroll
     for (int s = 0; s < kSelRegSlots; ++s) {
       const int i = s * 32 + lane;
       sv[s] = i < c ? sc[i] : -INFINITY;
       key[s] = i < c ? order_key_f(sv[s]) : 0u;
-      mloc = fmaxf(mloc, sv[s]);
     }
     // top-k: kap rounds of a warp arg-max (ties -> lower index)
     unsigned taken = 0;
@@ -245,67 +250,100 @@ select_kernel(Params p, TreeBufs tb, LeafOut lo, const void* __restrict__ tree, 
       }
       cnt += __popc(bal);
     }
-    // fold the unselected candidates' summaries into the partial softmax
-    float mw = mloc;
+    // fold the unselected candidates' summaries into the partial softmax: the
+    // score tiles left, per run r, U_r = sum_j exp(s_j - m_r) value_j over all
+    // of its children and L_r = sum_j exp(s_j - m_r); the unselected part is
+    // sum_r exp(m_r - M) (U_r, L_r) minus exp(s_i - M) (value_i, 1) for each
+    // kept candidate i
+    if (kap < c) {
+      const int nrun = kup + ((vL - p.b * vL1) > 0 ? 1 : 0);
+      const int64_t rb = int64_t(row) * (kmax + 1);
+      float2 mr = lane < nrun ? tb.runml[rb + lane] : make_float2(-INFINITY, 0.f);
+      float mx = mr.x;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
-    float* prow = lo.part + int64_t(row) * (D + 2);
-    const float2 ml = *reinterpret_cast<const float2*>(prow + D);
-    const float Mn = fmaxf(ml.x, mw);
-    const float scale = ml.x == -INFINITY ? 0.f : __expf(ml.x - Mn);
-    float acc[PER];
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float* prow = lo.part + int64_t(row) * (D + 2);
+      const float2 ml = *reinterpret_cast<const float2*>(prow + D);
+      const float Mn = fmaxf(ml.x, mx);
+      float ua[PER], ka[PER];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = prow[lane * PER + e] * ml.y * scale;
-    float lsum = ml.y * scale;
-    const float* vals = level_vals(p, const_cast<void*>(tree), L, seq, g);
-#pragma unroll
-    for (int s = 0; s < kSelRegSlots; ++s) {
-      if (s * 32 >= c) break;
-      const int i = s * 32 + lane;
-      const bool un = i < c && !((taken >> s) & 1u);
-      const float w = un ? __expf(sv[s] - Mn) : 0.f;
-      const int node = un ? node_of(i) : 0;
-      unsigned m = __ballot_sync(0xffffffffu, un);
-      while (m) {
-        // eight rows at a time, their loads issued together
-        constexpr int U = 8;
-        float ws[U];
-        int nd[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int src = m ? __ffs(m) - 1 : 0;
-          const bool real = m != 0;
-          m &= m - 1;
-          ws[u] = real ? __shfl_sync(0xffffffffu, w, src) : 0.f;
-          nd[u] = __shfl_sync(0xffffffffu, node, src);
-          if (!real) nd[u] = -1;
+      for (int e = 0; e < PER; ++e) ua[e] = ka[e] = 0.f;
+      float ul = 0.f, kl = 0.f;
+      // all runs
+      for (int r = 0; r < nrun; ++r) {
+        const float mrr = __shfl_sync(0xffffffffu, mr.x, r);
+        const float lrr = __shfl_sync(0xffffffffu, mr.y, r);
+        const float w = __expf(mrr - Mn);
+        const float* ur = tb.runpart + (rb + r) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(ur);
+          ua[0] = fmaf(w, x.x, ua[0]);
+          ua[1] = fmaf(w, x.y, ua[1]);
+          ua[2] = fmaf(w, x.z, ua[2]);
+          ua[3] = fmaf(w, x.w, ua[3]);
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(ur);
+          ua[0] = fmaf(w, x.x, ua[0]);
+          ua[1] = fmaf(w, x.y, ua[1]);
         }
-        float v[U][PER];
+        ul = fmaf(w, lrr, ul);
+      }
+      // the kept candidates (at most k, their rows loaded together)
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const float* vr = vals + int64_t(nd[u] < 0 ? 0 : nd[u]) * D + lane * PER;
-          if constexpr (PER == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(vr);
-            v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
-          } else {
-            const float2 x = *reinterpret_cast<const float2*>(vr);
-            v[u][0] = x.x; v[u][1] = x.y;
+      for (int s = 0; s < kSelRegSlots; ++s) {
+        if (s * 32 >= c) break;
+        const int i = s * 32 + lane;
+        const bool sel = i < c && ((taken >> s) & 1u);
+        const float w = sel ? __expf(sv[s] - Mn) : 0.f;
+        const int node = sel ? node_of(i) : 0;
+        unsigned m = __ballot_sync(0xffffffffu, sel);
+        while (m) {
+          constexpr int U = 8;
+          float ws[U];
+          int nd[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int src = m ? __ffs(m) - 1 : 0;
+            const bool real = m != 0;
+            m &= m - 1;
+            ws[u] = real ? __shfl_sync(0xffffffffu, w, src) : 0.f;
+            nd[u] = __shfl_sync(0xffffffffu, node, src);
+            if (!real) nd[u] = 0;
+          }
+          float v[U][PER];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const float* vr = vals + int64_t(nd[u]) * D + lane * PER;
+            if constexpr (PER == 4) {
+              const float4 x = *reinterpret_cast<const float4*>(vr);
+              v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+            } else {
+              const float2 x = *reinterpret_cast<const float2*>(vr);
+              v[u][0] = x.x; v[u][1] = x.y;
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int e = 0; e < PER; ++e) ka[e] = fmaf(ws[u], v[u][e], ka[e]);
+            kl += ws[u];
           }
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-          for (int e = 0; e < PER; ++e) acc[e] = fmaf(ws[u], v[u][e], acc[e]);
-          lsum += ws[u];
-        }
       }
-    }
-    const float il = 1.f / lsum;
+      // the unselected mass; below fp32 resolution of the runs' mass it is dropped
+      float dl = ul - kl;
+      const bool keep = dl > 1e-6f * ul;
+      const float scale = ml.x == -INFINITY ? 0.f : __expf(ml.x - Mn);
+      const float lsum = ml.y * scale + (keep ? dl : 0.f);
+      const float il = 1.f / lsum;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) prow[lane * PER + e] = acc[e] * il;
-    __syncwarp();
-    if (lane == 0) *reinterpret_cast<float2*>(prow + D) = make_float2(Mn, lsum);
-    __syncwarp();
+      for (int e = 0; e < PER; ++e)
+        prow[lane * PER + e] =
+            (prow[lane * PER + e] * ml.y * scale + (keep ? ua[e] - ka[e] : 0.f)) * il;
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<float2*>(prow + D) = make_float2(Mn, lsum);
+      __syncwarp();
+    }
   }
 
   // emit the runs of level L - 1
@@ -322,7 +360,7 @@ select_kernel(Params p, TreeBufs tb, LeafOut lo, const void* __restrict__ tree, 
       const int n = r < kprev ? p.b : orph;
       const int64_t bucket = hb + P;
       const int pos = atomicAdd(tb.counts + tb.cbase[Ln] + bucket, 1);
-      tb.stage[int64_t(row) * (kmax + 1) + r] = make_int4(row, i0 | (n << 16), cn - i0, 0);
+      tb.stage[int64_t(row) * (kmax + 1) + r] = make_int4(row, i0 | (n << 16), cn - i0, r);
       tb.spos[int64_t(row) * (kmax + 1) + r] = make_int2(int(bucket), pos);
     }
     if (lane == 0) tb.nruns[row] = nrun;
@@ -467,16 +505,25 @@ template <int D, int NB>
 struct ScoreSmem {
   static constexpr int kAn = kTTile * D * 4;          // one TF32 part of the queries
   static constexpr int kBn = NB * D * 4;              // one part of the child keys
+  static constexpr int kA2n = kTTile * NB * 4;        // one part of the probabilities
+  static constexpr int kB2n = D * NB * 4;             // one part of the child values^T
   static constexpr int kA = 0;
   static constexpr int kB = kA + 2 * kAn;
-  static constexpr int kBar = kB + 2 * kBn;
+  static constexpr int kA2 = kB + 2 * kBn;
+  static constexpr int kB2 = kA2 + 2 * kA2n;
+  static constexpr int kDst = kB2 + 2 * kB2n;           // per tile row: run partial offset
+  static constexpr int kBar = kDst + kTTile * 8;
   static constexpr int kTotal = kBar + 32;
-  static_assert(kTotal <= 227 * 1024, "score tile does not fit");
+  static constexpr bool kFits = kTotal <= 227 * 1024;
 };
 
-// One CTA per parent P (sequence, KV head, level-(l+1) node): its children's
-// keys at level l, rotated by their offset j, against tiles of 128 pairs'
-// queries rotated by c_l - i0; scores written to tb.scores[row][i0 + j].
+// One CTA per parent P (sequence, KV head, level-(l+1) node) and tile split:
+// its children's keys at level l, rotated by their offset j, against tiles of
+// 128 pairs' queries rotated by c_l - i0.  The scores go to
+// tb.scores[row][i0 + j]; then, per pair, P_j = exp(s_j - m) over its n
+// children (m their maximum) meets the children's values in a second product,
+// and U = P V and (m, sum P) are written as the run's partial, which the
+// select pass folds after removing the kept children.
 template <typename T, int D, int NB>
 __global__ void __launch_bounds__(kTThreads, 1)
 score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int lev) {
@@ -496,18 +543,21 @@ score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int 
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S::kBar);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + S::kBar + 16);
   const int tid = threadIdx.x, warp = tid >> 5;
-  constexpr uint32_t kCols = NB < 32 ? 32 : NB;
+  constexpr uint32_t kCols = 256;                // scores in [0, NB), U in [32, 32 + D)
   if (warp == 0) {
     tc05::tmem_alloc(tslot, kCols);
     tc05::tmem_relinquish();
   }
   if (tid == 0) {
     tc05::mbar_init(&bar[0], 1);
+    tc05::mbar_init(&bar[1], 1);
     tc05::mbar_fence_init();
   }
   const float2* rope = rope_table(p, tree);
-  // the parent's children (rows past the level's nodes are zero), rotated by j
+  // the parent's children (rows past the level's nodes are zero): keys rotated
+  // by j, values transposed ([d][child])
   const float* keys = level_keys(p, tree, lev, seq, g);
+  const float* vals = level_vals(p, tree, lev, seq, g);
   const int64_t nlev = p.lay.nodes[lev - 1];
   for (int task = tid; task < NB * (HALF / 8); task += kTThreads) {
     const int j = task % NB, c = task / NB;
@@ -529,31 +579,62 @@ score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int 
     }
     rot_split_store(p, rope, j < p.b ? j : 0, 8 * c, x1, x2, sm + S::kB, S::kBn, NB, j);
   }
+  for (int task = tid; task < D * (NB / 4); task += kTThreads) {
+    const int n = task % D, jq = task / D;
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * jq + e;
+      const int64_t node = int64_t(P) * p.b + j;
+      v[e] = (j < p.b && node < nlev) ? vals[node * D + n] : 0.f;
+    }
+    split_store4(sm + S::kB2 + kmaj4(D, n, 4 * jq), S::kB2n, v[0], v[1], v[2], v[3]);
+  }
+  tc05::fence_smem_to_async();
   tc05::fence_before_sync();
   __syncthreads();
   tc05::fence_after_sync();
-  const uint32_t tmem = *tslot;
+  const uint32_t tmem = *tslot, tU = tmem + 32;
   const uint32_t aA = tc05::smem_u32(sm + S::kA), aB = tc05::smem_u32(sm + S::kB);
-  constexpr uint32_t id = tc05::idesc(tc05::kFmtTF32, kTTile, NB);
+  const uint32_t aA2 = tc05::smem_u32(sm + S::kA2), aB2 = tc05::smem_u32(sm + S::kB2);
+  constexpr uint32_t id1 = tc05::idesc(tc05::kFmtTF32, kTTile, NB);
+  constexpr uint32_t id2 = tc05::idesc(tc05::kFmtTF32, kTTile, D);
   const float inv_sqrt_d = p.inv_sqrt_d;
   bool ok = true;
   unsigned phase = 0;
   for (int t0 = split * kTTile; t0 < cnt && ok; t0 += nsplit * kTTile) {
     const int nt = cnt - t0 < kTTile ? cnt - t0 : kTTile;
+    // gather: every load of this thread's tasks is issued before any store
+    constexpr int NT = kTTile * (HALF / 8) / kTThreads;
+    int4 prs[NT];
 #pragma unroll
-    for (int it = 0; it < kTTile * (HALF / 8) / kTThreads; ++it) {
+    for (int it = 0; it < NT; ++it) {
+      const int r = (tid + it * kTThreads) % kTTile;
+      prs[it] = r < nt ? tb.pairs[off + t0 + r] : make_int4(0, 0, 0, 0);
+    }
+    uint4 qa[NT][2];
+#pragma unroll
+    for (int it = 0; it < NT; ++it) {
+      const int task = tid + it * kTThreads;
+      const int r = task % kTTile, c = task / kTTile;
+      if (sizeof(T) == 2 && r < nt) {
+        const T* q = Q + int64_t(prs[it].x) * D;
+        qa[it][0] = *reinterpret_cast<const uint4*>(q + 8 * c);
+        qa[it][1] = *reinterpret_cast<const uint4*>(q + HALF + 8 * c);
+      } else {
+        qa[it][0] = qa[it][1] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int it = 0; it < NT; ++it) {
       const int task = tid + it * kTThreads;
       const int r = task % kTTile, c = task / kTTile;
       float x1[8], x2[8];
-      int rot = 0;
+      const int rot = r < nt ? prs[it].z : 0;
       if (r < nt) {
-        const int4 pr = tb.pairs[off + t0 + r];
-        rot = pr.z;
-        const T* q = Q + int64_t(pr.x) * D;
         if constexpr (sizeof(T) == 2) {
-          const uint4 u1 = *reinterpret_cast<const uint4*>(q + 8 * c);
-          const uint4 u2 = *reinterpret_cast<const uint4*>(q + HALF + 8 * c);
-          const uint32_t w1[4] = {u1.x, u1.y, u1.z, u1.w}, w2[4] = {u2.x, u2.y, u2.z, u2.w};
+          const uint32_t w1[4] = {qa[it][0].x, qa[it][0].y, qa[it][0].z, qa[it][0].w};
+          const uint32_t w2[4] = {qa[it][1].x, qa[it][1].y, qa[it][1].z, qa[it][1].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             x1[2 * e] = __uint_as_float(w1[e] << 16);
@@ -562,6 +643,7 @@ score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int 
             x2[2 * e + 1] = __uint_as_float(w2[e] & 0xffff0000u);
           }
         } else {
+          const T* q = Q + int64_t(prs[it].x) * D;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             x1[e] = reinterpret_cast<const float*>(q)[8 * c + e];
@@ -586,43 +668,124 @@ score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int 
         const uint64_t alo = tc05::desc_kmajor(a + S::kAn, 16 * kTTile, 128);
         const uint64_t bhi = tc05::desc_kmajor(bb, 16 * NB, 128);
         const uint64_t blo = tc05::desc_kmajor(bb + S::kBn, 16 * NB, 128);
-        tc05::mma_tf32(tmem, ahi, bhi, id, kk > 0);
-        tc05::mma_tf32(tmem, ahi, blo, id, 1);
-        tc05::mma_tf32(tmem, alo, bhi, id, 1);
+        tc05::mma_tf32(tmem, ahi, bhi, id1, kk > 0);
+        tc05::mma_tf32(tmem, ahi, blo, id1, 1);
+        tc05::mma_tf32(tmem, alo, bhi, id1, 1);
       }
       tc05::mma_commit(&bar[0]);
     }
     ok = __syncthreads_and(tid != 0 || tc05::mbar_wait_bounded(&bar[0], phase, kTreeWaitNs));
     tc05::fence_after_sync();
-    if (warp < 4 && ok) {
-      // tcgen05.ld is warp-collective: every lane loads, real pairs store
+    // thread i of warps 0-3 owns row i (TMEM lane i); the loads are
+    // warp-collective
+    const int myrow = tid;
+    const bool rowthr = warp < 4;
+    float m = -INFINITY, l = 0.f;
+    int4 pr = make_int4(0, 0, 0, 0);
+    if (ok && warp < 4) {
       float s[NB];
 #pragma unroll
       for (int c = 0; c < NB / 16; ++c)
         tc05::tmem_ld16(tmem + (uint32_t(warp * 32) << 16) + 16 * c, s + 16 * c);
       tc05::tmem_wait_ld();
-      if (tid < nt) {
-        const int4 pr = tb.pairs[off + t0 + tid];
-        const int i0 = pr.y & 0xffff, n = pr.y >> 16;
+      int n = 0;
+      if (rowthr && myrow < nt) {
+        pr = tb.pairs[off + t0 + myrow];
+        const int i0 = pr.y & 0xffff;
+        n = pr.y >> 16;
         float* dst = tb.scores + int64_t(pr.x) * tb.cmax + i0;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) s[j] *= inv_sqrt_d;
         if ((i0 & 3) == 0) {
 #pragma unroll
           for (int j = 0; j < NB; j += 4) {
             if (j + 4 <= n) {
-              *reinterpret_cast<float4*>(dst + j) =
-                  make_float4(s[j] * inv_sqrt_d, s[j + 1] * inv_sqrt_d, s[j + 2] * inv_sqrt_d,
-                              s[j + 3] * inv_sqrt_d);
+              *reinterpret_cast<float4*>(dst + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
             } else {
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                if (j + e < n) dst[j + e] = s[j + e] * inv_sqrt_d;
+                if (j + e < n) dst[j + e] = s[j + e];
             }
           }
         } else {
 #pragma unroll
           for (int j = 0; j < NB; ++j)
-            if (j < n) dst[j] = s[j] * inv_sqrt_d;
+            if (j < n) dst[j] = s[j];
         }
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+          if (j < n) m = fmaxf(m, s[j]);
+      }
+      // P over the run's n children (zero elsewhere and for rows past the tile)
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        s[j] = j < n ? __expf(s[j] - m) : 0.f;
+        l += s[j];
+      }
+      if (rowthr) {
+#pragma unroll
+        for (int j = 0; j < NB; j += 4)
+          split_store4(sm + S::kA2 + kmaj4(kTTile, myrow, j), S::kA2n, s[j], s[j + 1], s[j + 2],
+                       s[j + 3]);
+      }
+    }
+    tc05::fence_smem_to_async();
+    tc05::fence_before_sync();
+    __syncthreads();
+    tc05::fence_after_sync();
+    if (tid == 0 && ok) {
+#pragma unroll
+      for (int kk = 0; kk < NB / 8; ++kk) {
+        const uint32_t a = aA2 + kk * 32 * kTTile, bb = aB2 + kk * 32 * D;
+        const uint64_t ahi = tc05::desc_kmajor(a, 16 * kTTile, 128);
+        const uint64_t alo = tc05::desc_kmajor(a + S::kA2n, 16 * kTTile, 128);
+        const uint64_t bhi = tc05::desc_kmajor(bb, 16 * D, 128);
+        const uint64_t blo = tc05::desc_kmajor(bb + S::kB2n, 16 * D, 128);
+        tc05::mma_tf32(tU, ahi, bhi, id2, kk > 0);
+        tc05::mma_tf32(tU, ahi, blo, id2, 1);
+        tc05::mma_tf32(tU, alo, bhi, id2, 1);
+      }
+      tc05::mma_commit(&bar[1]);
+    }
+    ok = __syncthreads_and(tid != 0 || !ok || tc05::mbar_wait_bounded(&bar[1], phase, kTreeWaitNs)) && ok;
+    tc05::fence_after_sync();
+    // U rows: staged (16-byte chunks rotated by the row) in the query tile's
+    // bytes, then stored whole, coalesced
+    constexpr int CPR = D / 4;
+    unsigned char* stg = sm + S::kA;
+    static_assert(kTTile * D * 4 <= S::kAn, "staging fits the query tile");
+    if (ok && warp < 4) {
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        tc05::tmem_ld16(tU + (uint32_t(warp * 32) << 16) + 32 * c, o);
+        tc05::tmem_ld16(tU + (uint32_t(warp * 32) << 16) + 32 * c + 16, o + 16);
+        tc05::tmem_wait_ld();
+        if (rowthr) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int ch = 8 * c + e;
+            *reinterpret_cast<float4*>(stg + myrow * (D * 4) + ((ch + myrow) % CPR) * 16) =
+                make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          }
+        }
+      }
+      if (rowthr && myrow < nt) {
+        const int64_t slot = int64_t(pr.x) * (tb.kmax + 1) + pr.w;
+        tb.runml[slot] = make_float2(m, l);
+        reinterpret_cast<int64_t*>(sm + S::kDst)[myrow] = slot * D;
+      }
+    }
+    __syncthreads();
+    if (ok) {
+      // destination rows from shared memory: no global load between the stores
+      constexpr int RPW = 32 / CPR;
+      const int sub = (threadIdx.x & 31) / CPR, ch = (threadIdx.x & 31) % CPR;
+      const int64_t* dsts = reinterpret_cast<const int64_t*>(sm + S::kDst);
+      for (int r = warp * RPW + sub; r < nt; r += (kTThreads / 32) * RPW) {
+        float* dst = tb.runpart + dsts[r];
+        *reinterpret_cast<float4*>(dst + 4 * ch) =
+            *reinterpret_cast<const float4*>(stg + r * (D * 4) + ((ch + r) % CPR) * 16);
       }
     }
     tc05::fence_before_sync();
@@ -633,6 +796,7 @@ score_tc_kernel(Params p, const T* __restrict__ Q, void* tree, TreeBufs tb, int 
   if (!ok && tid == 0) {
     atomicOr(tree_error_word(tree), RECSA_DEVERR_WAIT_TIMEOUT);
     tc05::mbar_wait_bounded(&bar[0], phase, kTreeWaitNs);
+    tc05::mbar_wait_bounded(&bar[1], phase, kTreeWaitNs);
   }
   __syncthreads();
   if (warp == 0) tc05::tmem_dealloc(tmem, kCols);
@@ -642,6 +806,7 @@ template <typename T, int D, int NB>
 cudaError_t score_launch(const Params& p, const void* Q, void* tree, const TreeBufs& tb, int lev,
                          cudaStream_t s) {
   using S = ScoreSmem<D, NB>;
+  static_assert(S::kFits, "score tile does not fit");
   auto kern = score_tc_kernel<T, D, NB>;
   cudaError_t e = ensure_smem(kern, S::kTotal);
   if (e != cudaSuccess) return e;
@@ -660,7 +825,7 @@ cudaError_t score_dispatch(const Params& p, const void* Q, void* tree, const Tre
                            int lev, cudaStream_t s) {
   if (p.b <= 16) return score_launch<T, D, 16>(p, Q, tree, tb, lev, s);
   if (p.b <= 32) return score_launch<T, D, 32>(p, Q, tree, tb, lev, s);
-  return score_launch<T, D, 64>(p, Q, tree, tb, lev, s);
+  return cudaErrorNotSupported;
 }
 
 }  // namespace
@@ -670,7 +835,7 @@ bool prefill_tree_supported(const Params& p) {
   if (p.d != 64 && p.d != 128) return false;
   if (p.lay.levels < 1) return false;
   if (tree_cmax(p) > 32 * kSelRegSlots) return false;
-  if (p.b > 64 || p.b * int64_t(tree_kmax(p)) >= 65536) return false;
+  if (p.b > 32 || p.b * int64_t(tree_kmax(p)) >= 65536) return false;
   return true;
 }
 

@@ -266,6 +266,12 @@ window_mma_kernel(Params p, const __nv_bfloat16* __restrict__ Q,
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,
                                   const void* tree, int64_t q_start, int32_t n_q, void* part,
                                   cudaStream_t s) {
+  // the tcgen05 kernel first (RECSA_PREFILL_PATH = 1 keeps this mma.sync one)
+  if (switches().prefill_path != 1) {
+    const cudaError_t e = launch_prefill_window_tc(p, Q, K, V, tree, q_start, n_q, part, s);
+    if (e != cudaErrorNotSupported) return e;
+    cudaGetLastError();
+  }
   // the window is attended at true distances t - pos: the same for RecSA and
   // ZHA (group selection attends it in the generic kernel)
   if (p.mode != RECSA_MODE_RECSA && p.mode != RECSA_MODE_ZHA) return cudaErrorNotSupported;

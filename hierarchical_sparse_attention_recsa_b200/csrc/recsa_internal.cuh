@@ -236,6 +236,10 @@ cudaError_t launch_prefill_static(const Params& p, const void* Q, const void* K,
 size_t prefill_static_bytes();
 // Bytes of window partials for n_q queries per sequence (fp32 rows of d + 2).
 size_t prefill_workspace_need(const Params& p, int32_t n_q);
+// The same window partials from the tcgen05 window kernel (window_tc.cu).
+cudaError_t launch_prefill_window_tc(const Params& p, const void* Q, const void* K,
+                                     const void* V, const void* tree, int64_t q_start,
+                                     int32_t n_q, void* part, cudaStream_t s);
 // Tensor-core window partials for a prefill range (bf16) into part (fp32
 // rows of d + 2); cudaErrorNotSupported outside its limits.
 cudaError_t launch_prefill_window(const Params& p, const void* Q, const void* K, const void* V,

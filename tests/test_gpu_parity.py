@@ -50,12 +50,13 @@ def decode_impl(request):
     R.recsa_reload_switches()
 
 
-@pytest.fixture(params=["warp", "window", "leaf-tc", "tree-tc", "generic"])
+@pytest.fixture(params=["warp", "window", "window-mma", "leaf-tc", "tree-tc", "generic"])
 def prefill_impl(request):
     """Select the prefill path: the warp-per-(query, head) kernel alone (no
-    workspace), the window kernel plus the warp kernel attending the kept
-    leaves (a workspace of the window partials' size; bf16 only, fp32 falls
-    back to the warp kernel), the tensor-core kept-leaf path with the warp
+    workspace), the window kernel (tcgen05; "window-mma": the mma.sync one)
+    plus the warp kernel attending the kept leaves (a workspace of the window
+    partials' size; bf16 only, fp32 falls back to the warp kernel), the
+    tensor-core kept-leaf path with the warp
     traversal ("leaf-tc") or with the tree levels as tensor-core tiles
     ("tree-tc"; bf16, where the window kernel runs; fp32 falls back to the
     warp traversal) -- both with a workspace of recsa_prefill_workspace_bytes
@@ -64,6 +65,8 @@ def prefill_impl(request):
     old = {k: os.environ.pop(k, None) for k in keys}
     if request.param == "generic":
         os.environ["RECSA_PREFILL_GENERIC"] = "1"
+    elif request.param == "window-mma":
+        os.environ["RECSA_PREFILL_PATH"] = "1"
     elif request.param == "leaf-tc":
         os.environ["RECSA_PREFILL_PATH"] = "2"
     elif request.param == "tree-tc":
@@ -79,7 +82,7 @@ def prefill_impl(request):
 
 def _prefill(g, impl, Q, K, V, tree, q0, nq, O, trace=None):
     ws = None
-    if impl == "window":
+    if impl in ("window", "window-mma"):
         # exactly the window partials: the window + traversal path
         n = g.batch * nq * g.n_q_heads * (g.head_dim + 2) * 4
         ws = torch.empty(n, dtype=torch.uint8, device="cuda")
