@@ -161,10 +161,12 @@ def test_prefill_workspace_bytes(lib, mode):
     # the next level (int4 + int2 per run, k + 1 runs a query head) and the
     # count per query head, the runs grouped by parent (int4), and per-parent
     # counts and offsets: 64 and 4 nodes at levels 1 and 2 -> 64 / 16 + 1 and
-    # 4 / 16 + 1 parents per (sequence, KV head)
+    # 4 / 16 + 1 parents per (sequence, KV head); and per run its partial
+    # (d fp32) and its (max, sum)
     cmax, runs, parents = 64, rows * (kmax + 1), 2 * 8 * ((64 // 16 + 1) + (4 // 16 + 1))
     tree = (up(rows * cmax * 4) + up(2 * rows * kmax * 4) + up(runs * 16) + up(runs * 8) +
-            up(rows * 4) + up(runs * 16) + 2 * up(parents * 4))
+            up(rows * 4) + up(runs * 16) + 2 * up(parents * 4) + up(runs * 128 * 4) +
+            up(runs * 8))
     want = (up(part) + up(rows * kmax * 128 * 4) + up(rows * kmax * 8) + up(rows * kmax * 8) +
             up(rows * 4) + 2 * up(buckets * 4) + up(rows * kmax * 8) + up(tree))
     assert R.recsa_prefill_workspace_bytes(g, 100) == want
