@@ -43,6 +43,10 @@ NOMINAL_HBM_GBS = 8000.0     # roofline denominator named by the workload defini
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 x max SM clock
 
 
+def bf16_peak():
+    return peaks()[1]
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -614,6 +618,14 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
                          "bytes_qo": qo_bytes, "traffic": None,
                          "note": "touched K/V, tree and Q/O over the prefill time (after the "
                                  "build); the path is compute-bound, see compute_roofline"},
+            "tensor_roofline": {"bound": "tensor", "kernel": PREFILL_KERNELS,
+                                "achieved": flops / (attend_ms / 1e3) / 1e12,
+                                "peak": bf16_peak() / 2, "unit": "TFLOP/s",
+                                "frac": flops / (attend_ms / 1e3) / 1e12 / (bf16_peak() / 2),
+                                "peak_note": "TF32 = measured bf16 peak x 1/2 (nominal ratio): "
+                                             "the window, tree-level and kept-leaf products run "
+                                             "as TF32 tcgen05 MMAs; algorithmic flops as below",
+                                "flops": flops},
             "compute_roofline": {"bound": "alu", "kernel": PREFILL_KERNELS,
                                  "achieved": flops / (attend_ms / 1e3) / 1e12,
                                  "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
