@@ -58,6 +58,7 @@ constexpr int kWinRing = 4;       // window ring slots
 constexpr int kWinChunk = 24;     // window rows per ring slot
 constexpr int kMaxCluster = 16;
 constexpr int kMaxTokSlots = 4;   // kept-leaf ring slots per head
+constexpr int kMergeW = kChainWarps + kWinWarps + 2;   // per head: warp weights, max, sum
 constexpr unsigned long long kWaitNs = 50000000ull;   // a wait gives up after 50 ms
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -198,8 +199,8 @@ __device__ __forceinline__ void merge_xor(float& m, float& l, float* acc, int o)
 
 // Shared-memory plan of one CTA (byte offsets), the same on host and device.
 struct Plan {
-  unsigned mb, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, mrg, kept, kfl, rmask, wbuf, kbuf, vbuf,
-      total;
+  unsigned mb, geo, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, mwt, mrg, kept, tk, rmask, wbuf,
+      kbuf, vbuf, total;
   int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
   unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
 };
@@ -210,6 +211,7 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   Plan q;
   unsigned o = 0;
   q.mb = o;   o += 512;                                   // mbarriers
+  q.geo = o;  o += (kMaxLevels + 2) * 16 + 16;            // per-level counts, top level
   q.qf = o;   o += G * D * 4;
   q.qtok = o; o += G * D * 4;
   q.qlev = o; o += unsigned(levels) * HPC * D * 4;        // query rotated per level
@@ -218,9 +220,11 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   q.agg = o;  o += unsigned(cmax) * 4;                    // group scores (RECSA_MODE_GROUP)
   q.wsc = o;  o += kChainWarps * RS * 4;
   q.wwin = o; o += kWinWarps * G * RS * 4;
+  q.mwt = o;  o += G * kMergeW * 4;                       // merge weights per head
   q.mrg = o;  o += unsigned(CS) * HPC * RS * 4;
   q.kept = o; o += 2 * HPC * unsigned(kmax) * 4;
-  q.kfl = o;  o += 2 * HPC * unsigned(cmax);
+  o = (o + 7u) & ~7u;
+  q.tk = o;   o += HPC * 32 * 8;                          // selection scratch (key, index)
   o = (o + 15u) & ~15u;
   q.rmask = o; o += HPC * 32 * 4;
   o = (o + 127u) & ~127u;
@@ -287,15 +291,34 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* agg = reinterpret_cast<float*>(smem + pl.agg);     // [cmax] group scores
   float* wsc = reinterpret_cast<float*>(smem + pl.wsc);     // [kChainWarps][RS]
   float* wwin = reinterpret_cast<float*>(smem + pl.wwin);   // [kWinWarps][G][RS]
+  float* mwt = reinterpret_cast<float*>(smem + pl.mwt);     // [G][kMergeW]
   float* mrg = reinterpret_cast<float*>(smem + pl.mrg);     // [CS][HPC][RS] received
   int* kept = reinterpret_cast<int*>(smem + pl.kept);       // [2][HPC][kmax]
-  unsigned char* kfl = smem + pl.kfl;                       // [2][HPC][cmax]
+  uint2* tkl = reinterpret_cast<uint2*>(smem + pl.tk);     // [HPC][32] selection scratch
   unsigned* rmask = reinterpret_cast<unsigned*>(smem + pl.rmask);   // [HPC][32] kept bits
   T* wbuf = reinterpret_cast<T*>(smem + pl.wbuf);           // [kWinRing][2][kWinChunk][D]
   float* kbuf = reinterpret_cast<float*>(smem + pl.kbuf);   // [HB][rows][D] level keys
   float* vbuf = reinterpret_cast<float*>(smem + pl.vbuf);   // [HB][rows][D] level values
   T* tbuf = reinterpret_cast<T*>(smem + pl.kbuf);           // [HB][NRH][2][B][D] kept leaves
 
+  // The query and the chain slots' RoPE steps do not depend on the sequence
+  // length: their loads are issued first, beside the length's.
+  static_assert(G * D <= kThreads, "one query element per thread");
+  const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
+  const float qpre = tid < G * D ? load_elem(Q, qrow + tid, p.dtype) : 0.f;
+  const float2* rope = rope_table(p, tree);
+  const int rmax = p.lay.rope_rows - 1;
+  // Chain warps [h * WPH, (h + 1) * WPH) serve local query head h (global
+  // head hg * HPC + h); hs is the lane slot's index within the head's warps.
+  const int hw = warp / WPH;
+  const int hb = grp ? 0 : hw;   // its buffer head
+  const int hs = (warp % WPH) * SPW + lane / LPR;
+  // RoPE of the slot's first row and of its row step, for the recurrences
+  float cs_hs[8], cs_st[8];
+  if (p.rope && warp < kChainWarps) {
+    load_cs(rope, min(hs, rmax), HALF, j0, cs_hs);
+    load_cs(rope, min(HSLOT, rmax), HALF, j0, cs_st);
+  }
   // Fused step: the new token is appended at len (this kernel writes it and
   // pools what it completes), and the query sits on it.  A full sequence is
   // flagged and decoded without the append, as recsa_append would leave it.
@@ -304,37 +327,37 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   const int64_t t = do_append ? len0 : len0 - 1;
   const T* knew = reinterpret_cast<const T*>(st.k_new) + (seq * p.hkv + g) * D;
   const T* vnew = reinterpret_cast<const T*>(st.v_new) + (seq * p.hkv + g) * D;
-  const int64_t qrow = ((seq * n_q + qi) * p.hq + int64_t(g) * G) * D;
   const bool empty = t < 0 || t >= p.cap;   // uniform over the cluster
-  const float2* rope = rope_table(p, tree);
-  const int rmax = p.lay.rope_rows - 1;
   const int64_t s0 = t + 1 - p.W > 0 ? t + 1 - p.W : 0;
-  const int64_t a = empty ? 0 : s0 / p.B;
-  int64_t vis[kMaxLevels + 2];
-  int top = 0;
-  {
-    int64_t per = 1;
+  const int64_t a = empty ? 0 : (s0 <= 0x7fffffff ? int64_t(div_B(p, int(s0))) : s0 / p.B);
+  // Per-level counts, the same for every head, computed once into shared
+  // memory (indexed by level at run time, so registers cannot hold them):
+  // vis[l] = complete nodes of level l visible to the query (before the
+  // window), cnt_c[l] / cnt_k[l] = candidates / kept at level l, and the top
+  // level with a visible node.
+  int64_t* vis = reinterpret_cast<int64_t*>(smem + pl.geo);
+  int* cnt_c = reinterpret_cast<int*>(vis + kMaxLevels + 2);
+  int* cnt_k = cnt_c + kMaxLevels + 2;
+  int* top_s = cnt_k + kMaxLevels + 2;
+  if (tid == 0) {
+    int tp = 0;
+    int64_t v = a;
     for (int lev = 1; lev <= p.lay.levels; ++lev) {
-      vis[lev] = a / per;
-      if (vis[lev] == 0) break;
-      top = lev;
-      per *= p.b;
+      vis[lev] = v;
+      if (v == 0) break;
+      tp = lev;
+      v = v <= 0x7fffffff ? int64_t(div_b(p, int(v))) : v / p.b;
     }
-  }
-  // Candidate and kept counts per level: the same for every head.
-  int cnt_c[kMaxLevels + 2], cnt_k[kMaxLevels + 2];
-  {
     int kup = 0;
-    for (int lev = top; lev >= 1; --lev) {
-      const int64_t vup = lev < top ? vis[lev + 1] : 0;
+    for (int lev = tp; lev >= 1; --lev) {
+      const int64_t vup = lev < tp ? vis[lev + 1] : 0;
       cnt_c[lev] = p.b * kup + int(vis[lev] - p.b * vup);
       cnt_k[lev] = cnt_c[lev] < p.k ? cnt_c[lev] : p.k;
       kup = cnt_k[lev];
     }
+    *top_s = tp;
   }
-  const int nleaf = top > 0 ? cnt_k[1] : 0;
   const int64_t n_win = empty ? 0 : t + 1 - a * p.B;
-  const int64_t n0 = int64_t(nleaf) * p.B + n_win;
   const int64_t kvbase = (seq * p.hkv + g) * p.cap;
   const float inv_sqrt_d = p.inv_sqrt_d;
   const int tstride = kTraceHead + kMaxLevels * p.k;
@@ -355,11 +378,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   }
   const int nwr = w_hi - w_lo;
   const int nwch = (nwr + kWinChunk - 1) / kWinChunk;
-  // kept leaves of this share (leaf ranks sh, sh + S, ...)
-  const int ntok = nleaf > sh ? (nleaf - sh + S - 1) / S : 0;
 
   if (tid == 0) {
-    mbar_init(mb_lev, 1);
+    mbar_init(mb_lev, unsigned(HB));   // one arrival per buffer head (its selection warp)
     mbar_init(mb_val, 1);
     mbar_init(mb_kept, HPC);
     mbar_init(mb_folded, 1);
@@ -375,6 +396,11 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   }
   __syncthreads();
   if (CS > 1) cluster_arrive_relaxed();   // waited on before the first remote access
+  const int top = *top_s;
+  const int nleaf = top > 0 ? cnt_k[1] : 0;
+  const int64_t n0 = int64_t(nleaf) * p.B + n_win;
+  // kept leaves of this share (leaf ranks sh, sh + S, ...)
+  const int ntok = nleaf > sh ? (nleaf - sh + S - 1) / S : 0;
 
   // ---- producers (bulk copies) ----------------------------------------------
   // Node id of candidate i of local head h at level lev (kept list of lev + 1).
@@ -389,32 +415,21 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   // list of each local head) into kbuf (vbuf) in candidate order, completing
   // on mb_lev (mb_val).  Run by the whole producer warp: lane 0 arms the
   // barrier, the lanes copy one run each (the children of a kept node of
-  // level lev + 1, or the orphans; the top level is one run).
-  // Index (in candidate order) of the r-th kept candidate of local head h at
-  // the level just selected, straight from the top-k's row masks (the
-  // compacted kept list may not exist yet).
-  auto kept_idx = [&](int h, int r) -> int {
-    const unsigned* msk = rmask + h * 32;
-    int acc = 0;
-    for (int s = 0; s < 32; ++s) {
-      unsigned mk = msk[s];
-      const int n = __popc(mk);
-      if (r < acc + n) {
-        for (int t = acc; t < r; ++t) mk &= mk - 1;
-        return s * 32 + __ffs(mk) - 1;
-      }
-      acc += n;
-    }
-    return 0;
-  };
-  auto issue_level = [&](int lev, bool values, bool from_mask) {
+  // level lev + 1, or the orphans; the top level is one run).  Below the top
+  // level the keys are issued by the selection warps instead (one arrival
+  // per buffer head on mb_lev), so the top level's keys arrive HB times too.
+  auto issue_level = [&](int lev, bool values) {
     const int c = cnt_c[lev];
     int lo, hi;
     share(c, lo, hi);
     const unsigned rb = D * 4;
     uint64_t* mb = values ? mb_val : mb_lev;
     float* dst = values ? vbuf : kbuf;
-    if (lane == 0) mbar_expect_tx(mb, unsigned(HB) * unsigned(hi - lo) * rb);
+    if (lane == 0) {
+      mbar_expect_tx(mb, unsigned(HB) * unsigned(hi - lo) * rb);
+      if (!values)
+        for (int n = 1; n < HB; ++n) mbar_arrive(mb);
+    }
     __syncwarp();
     if (hi <= lo) return;
     const float* src = values ? level_vals(p, const_cast<void*>(tree), lev, seq, g)
@@ -430,7 +445,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (r < kup) {
         c0 = r * p.b;
         c1 = c0 + p.b;
-        node0 = (from_mask ? cand_node(lev + 1, h, kept_idx(h, r)) : keptu[h * kmax + r]) * p.b;
+        node0 = keptu[h * kmax + r] * p.b;
       } else {
         c0 = nch;
         c1 = c;
@@ -465,12 +480,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       bulk_g2s(dV + size_t(nk) * D, vnew, eb, mb);
     }
   };
-  // Kept leaf j of local head h's share (leaf rank sh + j * S) into its ring
-  // slot: B rows of K, then B rows of V.
-  auto issue_tok = [&](int h, int j, bool from_mask) {
+  // Kept leaf j of buffer head h's share (leaf rank sh + j * S, leaf `node`)
+  // into its ring slot: B rows of K, then B rows of V.
+  auto issue_tok_node = [&](int h, int j, int node) {
     const int slot = j % NRH;
-    const int node = from_mask ? cand_node(1, h, kept_idx(h, sh + j * S))
-                               : kept[1 * HPC * kmax + h * kmax + sh + j * S];   // level 1
     const unsigned lb = unsigned(p.B) * D * unsigned(sizeof(T));
     uint64_t* mb = mb_tok + h * NRH + slot;
     mbar_expect_tx(mb, 2u * lb);
@@ -478,29 +491,20 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     bulk_g2s(dK, K + (kvbase + int64_t(node) * p.B) * D, lb, mb);
     bulk_g2s(dK + size_t(p.B) * D, V + (kvbase + int64_t(node) * p.B) * D, lb, mb);
   };
+  auto issue_tok = [&](int h, int j) {
+    issue_tok_node(h, j, kept[1 * HPC * kmax + h * kmax + sh + j * S]);   // level 1's list
+  };
 
-  // Chain warps [h * WPH, (h + 1) * WPH) serve local query head h (global
-  // head hg * HPC + h); hs is the lane slot's index within the head's warps.
-  const int hw = warp / WPH;
-  const int hb = grp ? 0 : hw;   // its buffer head
-  const int hs = (warp % WPH) * SPW + lane / LPR;
-  // RoPE of the slot's first row and of its row step, for the recurrences
-  float cs_hs[8], cs_st[8];
-  if (p.rope && warp < kChainWarps) {
-    load_cs(rope, min(hs, rmax), HALF, j0, cs_hs);
-    load_cs(rope, min(HSLOT, rmax), HALF, j0, cs_st);
-  }
 
   // First copies: the top level's keys and values (the producer warp), before
   // the query is loaded.
   if (warp == kProducerWarp && top > 0) {
-    issue_level(top, false, false);
-    issue_level(top, true, false);
+    issue_level(top, false);
+    issue_level(top, true);
   }
   // The query and the RoPE table rows the kernel needs (loaded together: one
   // memory round trip), then the query rotated to every level's index.
-  for (int x = tid; x < G * D; x += kThreads)
-    qf[x] = empty ? 0.f : load_elem(Q, qrow + x, p.dtype);
+  if (tid < G * D) qf[tid] = empty ? 0.f : qpre;
   if (p.rope) {
     const int lv = p.lay.levels;
     for (int x = tid; x < (2 * lv + 3) * HALF; x += kThreads) {
@@ -572,6 +576,9 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     // a slot's rows are gsl, gsl + WSL, ... across all chunks: its RoPE
     // index grows by WSL per row, so its (cos, sin) advance by a fixed step
     const int widx0 = nleaf * p.B + w_lo;
+    float qr[G][8];   // the query of every head, rotated to n0 - 1
+#pragma unroll
+    for (int h = 0; h < G; ++h) lds_pairs(qtok + h * D, j0, HALF, qr[h]);
     float csc[8], cstep[8];
     const bool recur = WSL <= rmax;
     if (p.rope && recur && nwch > 0) {
@@ -597,14 +604,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float* qv = qtok + h * D;
-          float s = 0.f;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            s = fmaf(qv[j0 + c], xk[c], s);
-            s = fmaf(qv[HALF + j0 + c], xk[4 + c], s);
-          }
-          s = slot_sum<LPR>(s) * inv_sqrt_d;
+          const float s = slot_sum<LPR>(dot8(qr[h], xk)) * inv_sqrt_d;
           if (on) fold8(mW[h], lW[h], accW[h], s, xv);
         }
       }
@@ -718,10 +718,11 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int nr = hi - lo;
     const float* vb = vbuf + size_t(hb) * pl.rows * D;
     const float* scV = sc + (lev & 1) * HPC * cmax + hw * cmax + lo;
-    const unsigned char* flV = kfl + (lev & 1) * HPC * cmax + hw * cmax + lo;
+    const unsigned* msk = rmask + hw * 32;
+    auto kept_bit = [&](int i) { return (msk[i >> 5] >> (i & 31)) & 1u; };
     for (int e = hs; e < nr; e += 2 * HSLOT) {
       const int e1 = e + HSLOT;
-      const bool on0 = !flV[e], on1 = e1 < nr && !flV[e1];
+      const bool on0 = !kept_bit(lo + e), on1 = e1 < nr && !kept_bit(lo + e1);
       float x0[8], x1[8];
       SharedPairs<float, HALF>::load(vb + size_t(e) * D, j0, x0);
       SharedPairs<float, HALF>::load(vb + size_t(on1 ? e1 : e) * D, j0, x1);
@@ -730,21 +731,35 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   };
 
 
-  // Top-k of local head h = warp (warps 0 .. HPC - 1) at level lev over the
-  // head's full score table (with S > 1 every CTA of the head group runs the
-  // same selection on the same scores).  kap rounds of a warp arg-max: lane l
-  // holds the order-preserving keys of candidates l, l + 32, ... in registers
-  // (0 = none or taken; every finite score maps above 0); redux.sync gives
-  // the round's maximum, a ballot the lanes holding it, and on a tie of keys
-  // across lanes the lowest index wins (within a lane the lowest slot).  Bit
-  // s of `taken` marks candidate 32 s + l as kept.  Candidates beyond
-  // 32 * kRegSlots are read from shared memory in the same rounds.  The kept
-  // list is compacted in index order with one ballot per slot row.
+  // Slot s of local head h lies inside kbuf (free once the level-1 keys are
+  // scored) rather than reaching into vbuf (free once the level-1 values are
+  // folded).
+  auto early_slot = [&](int h, int s) {
+    const size_t sb = size_t(2) * p.B * D * sizeof(T);
+    return (size_t(h) * NRH + s + 1) * sb <= pl.kbytes;
+  };
+  // Selection of level lev for local head h = 3 - warp (warps 4 - HPC .. 3,
+  // one per head) over the head's full score table; with S > 1 every CTA of
+  // the head group runs the same selection on the same scores.
   // RECSA_MODE_GROUP (all G heads in the CTA): head 0's warp selects once for
   // the group on the group scores -- the sum over the heads of each
   // candidate's softmax probability among the level's candidates -- and
-  // hands the same masks to every head.
-  auto topk = [&](int lev) {
+  // hands the same selection to every head.
+  //   Candidates are ranked by order-preserving keys (0 = none), ties to the
+  // lower index.  Lane l holds the keys of candidates l, l + 32, ... (the
+  // first 32 * kRegSlots in registers, the rest read from shared memory).
+  //   1. thr = the kap-th largest of the 32 lane maxima: at least kap
+  //      candidates have a key >= thr, so the top kap are among them.
+  //   2. The candidates with key >= thr (usually a few more than kap) are listed
+  //      in the warp's scratch and ranked against each other by shuffles.
+  //   (With more than 32 of them -- ties at the threshold -- or kap > 32, kap
+  //   rounds of a warp arg-max pick the top kap instead.)
+  // The kept bits land in rmask (bit l of word s = candidate 32 s + l); from
+  // them the warp writes the kept list in index order (and the trace), and
+  // then issues the copies that depend on it straight away: the next level's
+  // key runs of this buffer head (one run per kept node, plus the orphans),
+  // or, at level 1, the kept leaves whose ring slots lie in kbuf.
+  auto select_level = [&](int lev) {
     const int c = cnt_c[lev], kap = cnt_k[lev];
     const int par = lev & 1;
     const int h = 3 - warp;
@@ -774,93 +789,172 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       row = agg;
     }
     const int ns = (c + 31) >> 5;
-    unsigned taken = 0;
+    const unsigned full = 0xffffffffu, lt = (1u << lane) - 1u;
+    unsigned word = 0;   // lane s < ns: the kept bits of candidates 32 s .. 32 s + 31
     if (kap >= c) {
-      for (int s = 0; s < ns; ++s)
-        if (s * 32 + lane < c) taken |= 1u << s;
+      if (lane < ns) word = (lane == ns - 1 && (c & 31)) ? (1u << (c & 31)) - 1u : full;
     } else {
       unsigned key[kRegSlots];
+      unsigned lm = 0;
 #pragma unroll
       for (int s = 0; s < kRegSlots; ++s) {
         const int i = s * 32 + lane;
         key[s] = i < c ? order_key(row[i]) : 0u;
+        lm = max(lm, key[s]);
       }
-      for (int r = 0; r < kap; ++r) {
-        unsigned bk = key[0];
-        int bs = 0;
+      for (int s = kRegSlots; s < ns; ++s) {
+        const int i = s * 32 + lane;
+        if (i < c) lm = max(lm, order_key(row[i]));
+      }
+      bool fast = kap <= 32;
+      unsigned thr = 1;
+      if (fast) {
+        int rk = 0;
 #pragma unroll
-        for (int s = 1; s < kRegSlots; ++s)
-          if (key[s] > bk) {
-            bk = key[s];
-            bs = s;
-          }
+        for (int j = 0; j < 32; ++j) {
+          const unsigned o = __shfl_sync(full, lm, j);
+          rk += (o > lm) | ((o == lm) & (j < lane));
+        }
+        const unsigned who = __ballot_sync(full, rk == kap - 1);
+        thr = max(1u, __shfl_sync(full, lm, __ffs(who) - 1));
+      }
+      int cnt = 0;
+#pragma unroll
+      for (int s = 0; s < kRegSlots; ++s) cnt += key[s] >= thr;
+      for (int s = kRegSlots; s < ns; ++s) {
+        const int i = s * 32 + lane;
+        if (i < c && order_key(row[i]) >= thr) ++cnt;
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(full, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int nc = __shfl_sync(full, incl, 31);
+      fast = fast && nc <= 32;
+      if (fast) {
+        uint2* tk = tkl + h * 32;
+        int pos = incl - cnt;
+#pragma unroll
+        for (int s = 0; s < kRegSlots; ++s)
+          if (key[s] >= thr) tk[pos++] = make_uint2(key[s], unsigned(s * 32 + lane));
         for (int s = kRegSlots; s < ns; ++s) {
           const int i = s * 32 + lane;
-          if (i < c && !((taken >> s) & 1u)) {
+          if (i < c) {
             const unsigned kk = order_key(row[i]);
-            if (kk > bk) {
-              bk = kk;
-              bs = s;
-            }
+            if (kk >= thr) tk[pos++] = make_uint2(kk, unsigned(i));
           }
         }
-        const unsigned M = __reduce_max_sync(0xffffffffu, bk);
-        unsigned who = __ballot_sync(0xffffffffu, bk == M);
-        if (__popc(who) > 1) {
-          const unsigned I =
-              __reduce_min_sync(0xffffffffu, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
-          who = 1u << (I & 31u);
+        __syncwarp();
+        const uint2 me = lane < nc ? tk[lane] : make_uint2(0u, 0u);
+        int r = 0;
+        for (int j = 0; j < nc; ++j) {
+          const unsigned ok = __shfl_sync(full, me.x, j), oi = __shfl_sync(full, me.y, j);
+          r += (ok > me.x) | ((ok == me.x) & (oi < me.y));
         }
-        if ((who >> lane) & 1u) {
-          taken |= 1u << bs;
+        const bool kp = lane < nc && r < kap;
+        for (int s = 0; s < ns; ++s) {
+          const unsigned R =
+              __reduce_or_sync(full, (kp && int(me.y >> 5) == s) ? 1u << (me.y & 31u) : 0u);
+          if (lane == s) word = R;
+        }
+        __syncwarp();
+      } else {
+        unsigned taken = 0;
+        for (int r = 0; r < kap; ++r) {
+          unsigned bk = key[0];
+          int bs = 0;
 #pragma unroll
-          for (int s = 0; s < kRegSlots; ++s)
-            if (s == bs) key[s] = 0u;
+          for (int s = 1; s < kRegSlots; ++s)
+            if (key[s] > bk) {
+              bk = key[s];
+              bs = s;
+            }
+          for (int s = kRegSlots; s < ns; ++s) {
+            const int i = s * 32 + lane;
+            if (i < c && !((taken >> s) & 1u)) {
+              const unsigned kk = order_key(row[i]);
+              if (kk > bk) {
+                bk = kk;
+                bs = s;
+              }
+            }
+          }
+          const unsigned M = __reduce_max_sync(full, bk);
+          unsigned who = __ballot_sync(full, bk == M);
+          if (__popc(who) > 1) {
+            const unsigned I =
+                __reduce_min_sync(full, bk == M ? unsigned(bs * 32 + lane) : 0xffffffffu);
+            who = 1u << (I & 31u);
+          }
+          if ((who >> lane) & 1u) {
+            taken |= 1u << bs;
+#pragma unroll
+            for (int s = 0; s < kRegSlots; ++s)
+              if (s == bs) key[s] = 0u;
+          }
+        }
+        for (int s = 0; s < ns; ++s) {
+          const unsigned R = __ballot_sync(full, (taken >> s) & 1u);
+          if (lane == s) word = R;
         }
       }
-    }
-    // kept bits by candidate row (bit l of rmask[h][s] = candidate 32 s + l)
-    unsigned mine = 0;
-    for (int s = 0; s < ns; ++s) {
-      const unsigned R = __ballot_sync(0xffffffffu, (taken >> s) & 1u);
-      if (lane == s) mine = R;
     }
     if (lane < ns) {
       if (grp) {
 #pragma unroll
-        for (int hh = 0; hh < HPC; ++hh) rmask[hh * 32 + lane] = mine;
+        for (int hh = 0; hh < HPC; ++hh) rmask[hh * 32 + lane] = word;
       } else {
-        rmask[h * 32 + lane] = mine;
+        rmask[h * 32 + lane] = word;
       }
     }
+    // The kept list in index order, the trace, and the copies it unlocks.
+    const int nxt = lev - 1;
+    int lo2 = 0, hi2 = 0;
+    if (nxt >= 1) share(cnt_c[nxt], lo2, hi2);
+    const unsigned rb = D * 4;
+    float* kdst = kbuf + size_t(h) * pl.rows * D;   // buffer head h (0 in group mode)
+    const float* ksrc = nxt >= 1 ? level_keys(p, const_cast<void*>(tree), nxt, seq, g) : nullptr;
+    fence_proxy_async();   // kbuf was read by the scoring threads (before the level barrier)
+    if (nxt >= 1 && lane == 0) mbar_expect_tx(mb_lev, unsigned(hi2 - lo2) * rb);
     __syncwarp();
-    if (lane == 0)   // the producer reads the masks (one arrival per head)
-      for (int n = 0; n < (grp ? HPC : 1); ++n) mbar_arrive(mb_kept);
-  };
-
-  // Kept flags and the kept list (in index order) of level lev from the row
-  // masks, by every chain thread (one candidate each).
-  auto compact = [&](int lev) {
-    const int c = cnt_c[lev];
-    const int par = lev & 1;
-    for (int x = tid; x < HPC * c; x += kChainThreads) {
-      const int h = x / c, i = x % c;
-      const int s = i >> 5, l = i & 31;
-      const unsigned R = rmask[h * 32 + s];
-      const bool f = (R >> l) & 1u;
-      kfl[par * HPC * cmax + h * cmax + i] = f;
-      if (f) {
-        int pos = __popc(R & ((1u << l) - 1u));
-        for (int t = 0; t < s; ++t) pos += __popc(rmask[h * 32 + t]);
-        const int node = cand_node(lev, h, i);
-        kept[par * HPC * kmax + h * kmax + pos] = node;
-        if (trace && sh == 0) {
-          const int64_t rec =
-              ((seq * n_q + qi) * p.hq + int64_t(g) * G + hg * HPC + h) * tstride;
-          trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
+    int base = 0;
+    for (int s = 0; s < ns; ++s) {
+      const unsigned wv = __shfl_sync(full, word, s);
+      if ((wv >> lane) & 1u) {
+        const int pos = base + __popc(wv & lt);
+        const int node = cand_node(lev, h, s * 32 + lane);
+        for (int hh = grp ? 0 : h; hh < (grp ? HPC : h + 1); ++hh) {
+          kept[par * HPC * kmax + hh * kmax + pos] = node;
+          if (trace && sh == 0) {
+            const int64_t rec =
+                ((seq * n_q + qi) * p.hq + int64_t(g) * G + hg * HPC + hh) * tstride;
+            trace[rec + kTraceHead + (lev - 1) * p.k + pos] = node;
+          }
+        }
+        if (nxt >= 1) {
+          const int c0 = pos * p.b, a0 = max(c0, lo2), a1 = min(c0 + p.b, hi2);
+          if (a1 > a0)
+            bulk_g2s(kdst + size_t(a0 - lo2) * D, ksrc + (int64_t(node) * p.b + (a0 - c0)) * D,
+                     unsigned(a1 - a0) * rb, mb_lev);
+        } else if (pos >= sh && (pos - sh) % S == 0) {
+          const int j = (pos - sh) / S;
+          if (j < NRH && early_slot(h, j)) issue_tok_node(h, j, node);
         }
       }
+      base += __popc(wv);
     }
+    if (nxt >= 1 && lane == 0) {   // the orphans of the next level
+      const int nch = p.b * kap, a0 = max(nch, lo2), a1 = min(cnt_c[nxt], hi2);
+      if (a1 > a0)
+        bulk_g2s(kdst + size_t(a0 - lo2) * D,
+                 ksrc + (int64_t(p.b) * vis[lev] + (a0 - nch)) * D, unsigned(a1 - a0) * rb,
+                 mb_lev);
+    }
+    __syncwarp();
+    if (lane == 0)   // the producer reads the kept list (one arrival per head)
+      for (int n = 0; n < (grp ? HPC : 1); ++n) mbar_arrive(mb_kept);
   };
 
   // Level barrier: the head group's scores of this level are complete and
@@ -959,22 +1053,13 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     }
   };
 
-  // Slot s of local head h lies inside kbuf (free once the level-1 keys are
-  // scored) rather than reaching into vbuf (free once the level-1 values are
-  // folded).
-  auto early_slot = [&](int h, int s) {
-    const size_t sb = size_t(2) * p.B * D * sizeof(T);
-    return (size_t(h) * NRH + s + 1) * sb <= pl.kbytes;
-  };
   auto chain_warps = [&]() {
     for (int lev = top; lev >= 1; --lev) {
       mbar_wait(mb_lev, unsigned(use) & 1u, timed_out);
       score_level(lev);
       level_sync();
       const int u = use++;
-      if (warp >= 4 - HPC && warp < 4) topk(lev);
-      named_sync(kBarChain, kChainThreads);
-      compact(lev);
+      if (warp >= 4 - HPC && warp < 4) select_level(lev);
       named_sync(kBarChain, kChainThreads);
       mbar_wait(mb_val, unsigned(u) & 1u, timed_out);
       fold_values(lev);
@@ -987,23 +1072,16 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     if (p.test_expire) mbar_wait(mb_never, 0u, timed_out);
   };
 
-  // The producer warp issues the chain's copies as soon as their addresses
-  // are known: a level's keys once the kept list above it is compacted, its
-  // values once the level above is folded (vbuf is free), the kept leaves of
-  // level 1 (slots inside kbuf first, the rest once vbuf is free), and each
-  // ring slot again when its head's warps have consumed it.
+  // The producer warp issues the chain's other copies: a level's values once
+  // the level above is folded (vbuf is free) and the level's keys have landed,
+  // the kept leaves of level 1 whose ring slots reach into vbuf (once it is
+  // free), and each ring slot again when its head's warps have consumed it.
+  // (The top level's copies are issued before the query is loaded; the keys
+  // of the levels below and the kept leaves in kbuf by the selection warps.)
   auto producer_warp = [&]() {
     for (int u = 0; u < top; ++u) {
       const int lev = top - u;
       mbar_wait(mb_kept, unsigned(u) & 1u, timed_out);
-      if (lane == 0) fence_proxy_async();
-      __syncwarp();
-      if (lev > 1) {
-        issue_level(lev - 1, false, true);
-      } else if (lane < HB) {
-        for (int j = 0; j < NRH && j < ntok; ++j)
-          if (early_slot(lane, j)) issue_tok(lane, j, true);
-      }
       mbar_wait(mb_folded, unsigned(u) & 1u, timed_out);
       // the next level's values are not needed before its top-k: let its keys
       // land first, so that they get the memory bandwidth to themselves
@@ -1011,10 +1089,10 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       if (lane == 0) fence_proxy_async();
       __syncwarp();
       if (lev > 1) {
-        issue_level(lev - 1, true, false);
+        issue_level(lev - 1, true);
       } else if (lane < HB) {
         for (int j = 0; j < NRH && j < ntok; ++j)
-          if (!early_slot(lane, j)) issue_tok(lane, j, false);
+          if (!early_slot(lane, j)) issue_tok(lane, j);
       }
     }
     if (top > 0 && lane < HB) {
@@ -1022,7 +1100,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       for (int j = NRH; j < ntok; ++j) {
         mbar_wait(mb_empty + h * NRH + j % NRH, unsigned(j / NRH - 1) & 1u, timed_out);
         fence_proxy_async();
-        issue_tok(h, j, false);
+        issue_tok(h, j);
       }
     }
   };
@@ -1063,29 +1141,42 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     while (global_ns() - t0 < 1000000ull) __nanosleep(10000);
   }
   __syncthreads();
+  // Per head of the group: the weight of every contributing warp's partial
+  // (the head's chain warps when this CTA owns it, and the window warps)
+  // relative to their common maximum, then the weighted sum per element.
+  if (tid < G) {
+    const int h = tid, lh = h % HPC;
+    const bool mine = h / HPC == hg;
+    float* wt = mwt + h * kMergeW;
+    float mm = -INFINITY;
+    if (mine)
+      for (int w = 0; w < WPH; ++w) mm = fmaxf(mm, wsc[(lh * WPH + w) * RS + D]);
+    for (int w = 0; w < kWinWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * RS + D]);
+    float ll = 0.f;
+    for (int w = 0; w < WPH + kWinWarps; ++w) {
+      float r = 0.f;
+      if (w < WPH ? mine : true) {
+        const float* ws = w < WPH ? wsc + (lh * WPH + w) * RS : wwin + ((w - WPH) * G + h) * RS;
+        r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+        ll = fmaf(ws[D + 1], r, ll);
+      }
+      wt[w] = r;
+    }
+    wt[kMergeW - 2] = mm;
+    wt[kMergeW - 1] = ll;
+  }
+  __syncthreads();
   for (int x = tid; x < G * D; x += kThreads) {
     const int h = x / D, c = x % D;
     const int lh = h % HPC;
-    const bool mine = h / HPC == hg;
-    float mm = -INFINITY;
-    if (mine)
-      for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * RS + D]);
-    for (int w = 0; w < kWinWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * RS + D]);
-    float aa = 0.f, ll = 0.f;
+    const float* wt = mwt + h * kMergeW;
+    const float mm = wt[kMergeW - 2], ll = wt[kMergeW - 1];
+    float aa = 0.f;
     if (mm != -INFINITY) {
-      if (mine)
-        for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) {
-          const float* ws = wsc + w * RS;
-          const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
-          aa = fmaf(ws[c], r, aa);
-          ll = fmaf(ws[D + 1], r, ll);
-        }
-      for (int w = 0; w < kWinWarps; ++w) {
-        const float* ws = wwin + (w * G + h) * RS;
-        const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
-        aa = fmaf(ws[c], r, aa);
-        ll = fmaf(ws[D + 1], r, ll);
-      }
+      if (h / HPC == hg)
+        for (int w = 0; w < WPH; ++w) aa = fmaf(wsc[(lh * WPH + w) * RS + c], wt[w], aa);
+      for (int w = 0; w < kWinWarps; ++w)
+        aa = fmaf(wwin[(w * G + h) * RS + c], wt[WPH + w], aa);
     }
     float* dst = (CS == 1 ? mrg : cluster.map_shared_rank(mrg, (h / HPC) * S)) +
                  (rank * HPC + lh) * RS;
