@@ -58,7 +58,6 @@ constexpr int kWinRing = 4;       // window ring slots
 constexpr int kWinChunk = 24;     // window rows per ring slot
 constexpr int kMaxCluster = 16;
 constexpr int kMaxTokSlots = 4;   // kept-leaf ring slots per head
-constexpr int kMergeW = kChainWarps + kWinWarps + 2;   // per head: warp weights, max, sum
 constexpr unsigned long long kWaitNs = 50000000ull;   // a wait gives up after 50 ms
 constexpr size_t kSmemLimit = 227 * 1024;
 
@@ -199,7 +198,7 @@ __device__ __forceinline__ void merge_xor(float& m, float& l, float* acc, int o)
 
 // Shared-memory plan of one CTA (byte offsets), the same on host and device.
 struct Plan {
-  unsigned mb, geo, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, mwt, mrg, kept, tk, rmask, wbuf,
+  unsigned mb, geo, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, gsc, mrg, kept, tk, rmask, wbuf,
       kbuf, vbuf, total;
   int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
   unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
@@ -220,7 +219,7 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   q.agg = o;  o += unsigned(cmax) * 4;                    // group scores (RECSA_MODE_GROUP)
   q.wsc = o;  o += kChainWarps * RS * 4;
   q.wwin = o; o += kWinWarps * G * RS * 4;
-  q.mwt = o;  o += G * kMergeW * 4;                       // merge weights per head
+  q.gsc = o;  o += 2 * kChainWarps * 4;                   // group scores: per-warp (max, sum)
   q.mrg = o;  o += unsigned(CS) * HPC * RS * 4;
   q.kept = o; o += 2 * HPC * unsigned(kmax) * 4;
   o = (o + 7u) & ~7u;
@@ -240,9 +239,35 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   return q;
 }
 
+// Pooling after the fused step's append (one warp): the leaf the new token
+// completes, then every ancestor it completes in turn.  Out of line: it runs
+// in one CTA per (sequence, KV head) at the end of the step.
+template <typename T, int D>
+__device__ __noinline__ void pool_appended(const Params& p, const T* K, const T* V, const void* tree,
+                                           const float* r, int64_t kvbase, int64_t t, int64_t seq,
+                                           int g, int lane) {
+  constexpr int N = D / 32;
+  float rl[N], key[N], val[N];
+  load_r<N>(r, lane, rl);
+  int64_t j = (t + 1) / p.B - 1;
+  const int64_t row0 = (kvbase + j * p.B) * D;
+  pool_rows<T, N>(K + row0, V + row0, p.B, D, rl, p.inv_sqrt_d, lane, key, val);
+  RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane, key);
+  RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane, val);
+  for (int lev = 2; lev <= p.lay.levels && (j + 1) % p.b == 0; ++lev) {
+    j = (j + 1) / p.b - 1;
+    __syncwarp();
+    const float* ck = level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
+    const float* cv = level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
+    pool_rows<float, N>(ck, cv, p.b, D, rl, p.inv_sqrt_d, lane, key, val);
+    RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), lev, seq, g) + j * D, lane, key);
+    RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), lev, seq, g) + j * D, lane, val);
+  }
+}
+
 template <typename T, int D, int G, int HPC>
 __global__ void __launch_bounds__(kThreads, 1)
-decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
+decode_cluster_kernel(const __grid_constant__ Params p, const T* __restrict__ Q, const T* __restrict__ K,
                       const T* __restrict__ V, const void* __restrict__ tree,
                       const int64_t* __restrict__ len_dev, int n_q, T* __restrict__ O,
                       int32_t* __restrict__ trace, int cmax, int kmax, int S, int NRH,
@@ -291,7 +316,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
   float* agg = reinterpret_cast<float*>(smem + pl.agg);     // [cmax] group scores
   float* wsc = reinterpret_cast<float*>(smem + pl.wsc);     // [kChainWarps][RS]
   float* wwin = reinterpret_cast<float*>(smem + pl.wwin);   // [kWinWarps][G][RS]
-  float* mwt = reinterpret_cast<float*>(smem + pl.mwt);     // [G][kMergeW]
+  float* gsc = reinterpret_cast<float*>(smem + pl.gsc);     // [kChainWarps][2]
   float* mrg = reinterpret_cast<float*>(smem + pl.mrg);     // [CS][HPC][RS] received
   int* kept = reinterpret_cast<int*>(smem + pl.kept);       // [2][HPC][kmax]
   uint2* tkl = reinterpret_cast<uint2*>(smem + pl.tk);     // [HPC][32] selection scratch
@@ -738,6 +763,69 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const size_t sb = size_t(2) * p.B * D * sizeof(T);
     return (size_t(h) * NRH + s + 1) * sb <= pl.kbytes;
   };
+  // RECSA_MODE_GROUP (every head of the group in the CTA, HPC == G): the
+  // group score of candidate i is the sum over the heads of its softmax
+  // probability among the level's candidates, computed by all chain threads.
+  // Chain warp w takes head w % G and a strided part of the candidates: an
+  // online (max, sum of exp) pass, reduced over the warp into gsc; then each
+  // thread combines the parts of every head for its candidates.  Ends with a
+  // chain barrier (agg complete).
+  auto group_scores = [&](int lev) {
+    constexpr int NP = kChainWarps / G;   // parts per head
+    static_assert(kChainWarps % G == 0, "chain warps split evenly over the heads");
+    const int c = cnt_c[lev], par = lev & 1;
+    const float* scl = sc + par * HPC * cmax;
+    {
+      const int h = warp % G, part = warp / G;
+      const float* rw = scl + h * cmax;
+      float mx = -INFINITY, sm = 0.f;
+      for (int i = part * 32 + lane; i < c; i += NP * 32) {
+        const float v = rw[i];
+        if (v > mx) {
+          sm = (mx == -INFINITY ? 0.f : sm * expf(mx - v)) + 1.f;
+          mx = v;
+        } else {
+          sm += expf(v - mx);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, mx, o);
+        const float so = __shfl_xor_sync(0xffffffffu, sm, o);
+        const float mn = fmaxf(mx, mo);
+        sm = (mx == -INFINITY ? 0.f : sm * expf(mx - mn)) + (mo == -INFINITY ? 0.f : so * expf(mo - mn));
+        mx = mn;
+      }
+      if (lane == 0) {
+        gsc[2 * warp] = mx;
+        gsc[2 * warp + 1] = sm;
+      }
+    }
+    named_sync(kBarChain, kChainThreads);
+    float mh[G], zh[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) mx = fmaxf(mx, gsc[2 * (q * G + h)]);
+      float z = 0.f;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const float mq = gsc[2 * (q * G + h)];
+        if (mq != -INFINITY) z += gsc[2 * (q * G + h) + 1] * expf(mq - mx);
+      }
+      mh[h] = mx;
+      zh[h] = z;
+    }
+    for (int i = tid; i < c; i += kChainThreads) {
+      float a_ = 0.f;
+#pragma unroll
+      for (int h = 0; h < G; ++h) a_ += expf(scl[h * cmax + i] - mh[h]) / zh[h];
+      agg[i] = a_;
+    }
+    named_sync(kBarChain, kChainThreads);
+  };
+
   // Selection of level lev for local head h = 3 - warp (warps 4 - HPC .. 3,
   // one per head) over the head's full score table; with S > 1 every CTA of
   // the head group runs the same selection on the same scores.
@@ -765,29 +853,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     const int h = 3 - warp;
     if (grp && h != 0) return;
     const float* row = sc + par * HPC * cmax + h * cmax;
-    if (grp) {
-      float mxh[HPC], smh[HPC];
-#pragma unroll
-      for (int hh = 0; hh < HPC; ++hh) {
-        const float* rw = sc + par * HPC * cmax + hh * cmax;
-        float mx = -INFINITY;
-        for (int i = lane; i < c; i += 32) mx = fmaxf(mx, rw[i]);
-        mx = warp_max(mx);
-        float sm = 0.f;
-        for (int i = lane; i < c; i += 32) sm += expf(rw[i] - mx);
-        mxh[hh] = mx;
-        smh[hh] = warp_sum(sm);
-      }
-      for (int i = lane; i < c; i += 32) {
-        float a_ = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < HPC; ++hh)
-          a_ += expf(sc[par * HPC * cmax + hh * cmax + i] - mxh[hh]) / smh[hh];
-        agg[i] = a_;
-      }
-      __syncwarp();
-      row = agg;
-    }
+    if (grp) row = agg;   // the group scores (group_scores, all chain warps)
     const int ns = (c + 31) >> 5;
     const unsigned full = 0xffffffffu, lt = (1u << lane) - 1u;
     unsigned word = 0;   // lane s < ns: the kept bits of candidates 32 s .. 32 s + 31
@@ -1059,6 +1125,7 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
       score_level(lev);
       level_sync();
       const int u = use++;
+      if (grp && cnt_k[lev] < cnt_c[lev]) group_scores(lev);
       if (warp >= 4 - HPC && warp < 4) select_level(lev);
       named_sync(kBarChain, kChainThreads);
       mbar_wait(mb_val, unsigned(u) & 1u, timed_out);
@@ -1141,42 +1208,29 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
     while (global_ns() - t0 < 1000000ull) __nanosleep(10000);
   }
   __syncthreads();
-  // Per head of the group: the weight of every contributing warp's partial
-  // (the head's chain warps when this CTA owns it, and the window warps)
-  // relative to their common maximum, then the weighted sum per element.
-  if (tid < G) {
-    const int h = tid, lh = h % HPC;
-    const bool mine = h / HPC == hg;
-    float* wt = mwt + h * kMergeW;
-    float mm = -INFINITY;
-    if (mine)
-      for (int w = 0; w < WPH; ++w) mm = fmaxf(mm, wsc[(lh * WPH + w) * RS + D]);
-    for (int w = 0; w < kWinWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * RS + D]);
-    float ll = 0.f;
-    for (int w = 0; w < WPH + kWinWarps; ++w) {
-      float r = 0.f;
-      if (w < WPH ? mine : true) {
-        const float* ws = w < WPH ? wsc + (lh * WPH + w) * RS : wwin + ((w - WPH) * G + h) * RS;
-        r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
-        ll = fmaf(ws[D + 1], r, ll);
-      }
-      wt[w] = r;
-    }
-    wt[kMergeW - 2] = mm;
-    wt[kMergeW - 1] = ll;
-  }
-  __syncthreads();
   for (int x = tid; x < G * D; x += kThreads) {
     const int h = x / D, c = x % D;
     const int lh = h % HPC;
-    const float* wt = mwt + h * kMergeW;
-    const float mm = wt[kMergeW - 2], ll = wt[kMergeW - 1];
-    float aa = 0.f;
+    const bool mine = h / HPC == hg;
+    float mm = -INFINITY;
+    if (mine)
+      for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) mm = fmaxf(mm, wsc[w * RS + D]);
+    for (int w = 0; w < kWinWarps; ++w) mm = fmaxf(mm, wwin[(w * G + h) * RS + D]);
+    float aa = 0.f, ll = 0.f;
     if (mm != -INFINITY) {
-      if (h / HPC == hg)
-        for (int w = 0; w < WPH; ++w) aa = fmaf(wsc[(lh * WPH + w) * RS + c], wt[w], aa);
-      for (int w = 0; w < kWinWarps; ++w)
-        aa = fmaf(wwin[(w * G + h) * RS + c], wt[WPH + w], aa);
+      if (mine)
+        for (int w = lh * WPH; w < (lh + 1) * WPH; ++w) {
+          const float* ws = wsc + w * RS;
+          const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+          aa = fmaf(ws[c], r, aa);
+          ll = fmaf(ws[D + 1], r, ll);
+        }
+      for (int w = 0; w < kWinWarps; ++w) {
+        const float* ws = wwin + (w * G + h) * RS;
+        const float r = (ws[D] == -INFINITY) ? 0.f : __expf(ws[D] - mm);
+        aa = fmaf(ws[c], r, aa);
+        ll = fmaf(ws[D + 1], r, ll);
+      }
     }
     float* dst = (CS == 1 ? mrg : cluster.map_shared_rank(mrg, (h / HPC) * S)) +
                  (rank * HPC + lh) * RS;
@@ -1241,29 +1295,8 @@ decode_cluster_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K
         Vw[x] = vnew[x];
       }
       __syncthreads();
-      if ((t + 1) % p.B == 0 && warp == 0) {
-        constexpr int N = D / 32;
-        float rl[N], key[N], val[N];
-        load_r<N>(st.r + g * st.r_stride, lane, rl);
-        int64_t j = (t + 1) / p.B - 1;
-        const int64_t row0 = (kvbase + j * p.B) * D;
-        pool_rows<T, N>(K + row0, V + row0, p.B, D, rl, inv_sqrt_d, lane, key, val);
-        RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane,
-                               key);
-        RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), 1, seq, g) + j * D, lane,
-                               val);
-        for (int lev = 2; lev <= p.lay.levels && (j + 1) % p.b == 0; ++lev) {
-          j = (j + 1) / p.b - 1;
-          __syncwarp();
-          const float* ck = level_keys(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
-          const float* cv = level_vals(p, const_cast<void*>(tree), lev - 1, seq, g) + j * p.b * D;
-          pool_rows<float, N>(ck, cv, p.b, D, rl, inv_sqrt_d, lane, key, val);
-          RowIO<float, N>::store(level_keys(p, const_cast<void*>(tree), lev, seq, g) + j * D,
-                                 lane, key);
-          RowIO<float, N>::store(level_vals(p, const_cast<void*>(tree), lev, seq, g) + j * D,
-                                 lane, val);
-        }
-      }
+      if ((t + 1) % p.B == 0 && warp == 0)
+        pool_appended<T, D>(p, K, V, tree, st.r + g * st.r_stride, kvbase, t, seq, g, lane);
     }
     // Length: every cluster of the sequence read len at its start; the last
     // one to finish (per-sequence counter) publishes len + 1 and resets it.
