@@ -201,7 +201,8 @@ struct Plan {
   unsigned mb, geo, qf, qtok, qlev, rrow, sc, agg, wsc, wwin, gsc, mrg, kept, tk, rmask, wbuf,
       kbuf, vbuf, total;
   int rows;         // summary rows per local head in kbuf and vbuf (one share of a level)
-  unsigned kbytes;  // bytes of kbuf (the kept-leaf ring starts there and may run into vbuf)
+  unsigned kbytes;  // bytes of a level's keys in kbuf
+  unsigned kreg;    // bytes before vbuf (the kept-leaf ring starts at kbuf and may run into vbuf)
 };
 template <typename T, int D, int G, int HPC>
 __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, int CS, int NRH,
@@ -232,9 +233,15 @@ __host__ __device__ __forceinline__ Plan make_plan(int cmax, int kmax, int S, in
   q.kbuf = o;
   q.rows = (cmax + S - 1) / S;
   q.kbytes = unsigned(HB) * unsigned(q.rows) * D * 4;   // HB heads' level rows
-  q.vbuf = o + q.kbytes;
-  const unsigned toks = unsigned(HB) * unsigned(NRH) * 2 * unsigned(B) * D * unsigned(sizeof(T));
-  o += 2 * q.kbytes > toks ? 2 * q.kbytes : toks;
+  // with one buffer head, at least two kept-leaf slots before vbuf, so that
+  // the first leaves can be copied as soon as level 1 is selected (the rest
+  // once its values are folded)
+  const unsigned slot = 2 * unsigned(B) * D * unsigned(sizeof(T));
+  const unsigned early = HB == 1 ? unsigned(NRH < 2 ? NRH : 2) * slot : 0u;
+  q.kreg = q.kbytes > early ? q.kbytes : early;
+  q.vbuf = o + q.kreg;
+  const unsigned toks = unsigned(HB) * unsigned(NRH) * slot;
+  o += q.kreg + q.kbytes > toks ? q.kreg + q.kbytes : toks;
   q.total = o;
   return q;
 }
@@ -761,7 +768,7 @@ decode_cluster_kernel(const __grid_constant__ Params p, const T* __restrict__ Q,
   // folded).
   auto early_slot = [&](int h, int s) {
     const size_t sb = size_t(2) * p.B * D * sizeof(T);
-    return (size_t(h) * NRH + s + 1) * sb <= pl.kbytes;
+    return (size_t(h) * NRH + s + 1) * sb <= pl.kreg;
   };
   // RECSA_MODE_GROUP (every head of the group in the CTA, HPC == G): the
   // group score of candidate i is the sum over the heads of its softmax
