@@ -644,8 +644,8 @@ def run_prefill(args, w, Kc, Vc, r, cap, flush, stream, hbm_gbs):
                                               "unused"}}
 
 
-PREFILL_KERNELS = ("window_mma_kernel + select_kernel + score_tc_kernel + leaf_tc_kernel + "
-                   "merge_kernel (tree levels and kept leaves on tcgen05)")
+PREFILL_KERNELS = ("window_tc_kernel + score_tc_kernel + select_kernel + leaf_tc_kernel + "
+                   "merge_kernel (window, tree levels and kept leaves on tcgen05)")
 
 
 ZHA_PREFILL_QUERIES = 65536
@@ -654,7 +654,7 @@ ZHA_PREFILL_QUERIES = 65536
 def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
     """ZHA routing (p = ZHA_TOP_P, fp32 keys) prefill of the last
     ZHA_PREFILL_QUERIES positions of one sequence: the window on
-    window_mma_kernel, the routing and the leaves on zha_attend_kernel, which
+    window_tc_kernel, the routing and the leaves on zha_attend_kernel, which
     merges the window's partials (a bounded sample of the workload's full
     prefill).  ALU roofline with flops =
     2 d (summary keys scored + exact tokens) per query head, the counts taken
@@ -693,7 +693,7 @@ def run_zha_prefill(args, w, Kc, Vc, r, cap, flush, stream):
     del Q, O, tree, trace, ws
     torch.cuda.empty_cache()
     return {"value": nq / (ms / 1e3), "unit": "tokens/s", "ms": ms, "queries": nq,
-            "q_start": q0, "top_p": ZHA_TOP_P, "kernel": "window_mma_kernel + zha_attend_kernel",
+            "q_start": q0, "top_p": ZHA_TOP_P, "kernel": "window_tc_kernel + zha_attend_kernel",
             "sample": f"the last {nq} of {L} positions of one sequence",
             "roofline": {"bound": "alu", "achieved": flops / (ms / 1e3) / 1e12,
                          "peak": ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
