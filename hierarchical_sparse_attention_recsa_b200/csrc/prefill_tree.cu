@@ -119,7 +119,7 @@ __device__ __forceinline__ unsigned order_key_f(float f) {
 // One warp per query head (row).  L: the level selected here (L > top: no
 // selection); emits the runs of level L - 1 (or the kept leaves at L = 1).
 template <int D>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(256, 4)
 select_kernel(Params p, TreeBufs tb, LeafOut lo, const void* __restrict__ tree, int L,
               int64_t q_start, int n_q, int32_t* __restrict__ trace) {
   constexpr int PER = D / 32;
