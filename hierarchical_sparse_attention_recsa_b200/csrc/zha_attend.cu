@@ -403,15 +403,20 @@ zha_attend_kernel(Params p, const T* __restrict__ Q, const T* __restrict__ K,
               sc4[r] = fmaf(q2[u], x2[u], sc4[r]);
             }
           }
+          // the four rows' sums by a transposed reduction (6 shuffles, not 20):
+          // across lanes 16 apart each lane keeps two of the rows, across
+          // lanes 8 apart one, then the remaining lanes fold; lane 8 r (r < 4)
+          // ends with row r's sum
+          const bool u4 = (lane >> 4) & 1, u3 = (lane >> 3) & 1;
+          float a0 = u4 ? sc4[2] : sc4[0], a1 = u4 ? sc4[3] : sc4[1];
+          a0 += __shfl_xor_sync(0xffffffffu, u4 ? sc4[0] : sc4[2], 16);
+          a1 += __shfl_xor_sync(0xffffffffu, u4 ? sc4[1] : sc4[3], 16);
+          float v = u3 ? a1 : a0;
+          v += __shfl_xor_sync(0xffffffffu, u3 ? a0 : a1, 8);
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) sc4[r] += __shfl_xor_sync(0xffffffffu, sc4[r], o);
-          if (lane < 4) {
-            float v = sc4[0];
-#pragma unroll
-            for (int r = 1; r < 4; ++r) v = lane == r ? sc4[r] : v;
-            const int q = q0 + lane * NCH;
+          for (int o = 4; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          if ((lane & 7) == 0) {
+            const int q = q0 + (lane >> 3) * NCH;
             if (q < nrow) rsc[q] = v * p.inv_sqrt_d * (lowp ? ksc[q] : 1.f);
           }
         }
