@@ -20,12 +20,14 @@
 //     mbarrier.  HPC and S are chosen per launch so that the grid fills the
 //     148 SMs.
 //   * Warps are specialised.  Twelve chain warps walk the levels (score,
-//     top-k, issue the next level's copies, fold the unselected summary
-//     values while those copies fly) and then stream the kept leaves through a
-//     ring of bulk-copy slots.  Four window warps attend the exact window,
-//     which does not depend on the selection, through their own ring of
-//     bulk-copy slots, concurrently with the chain; each CTA sends its window
-//     partial of every head to that head's owner at the end.
+//     then one warp per head selects, writes the kept list and issues the
+//     next level's key copies, then all fold the unselected summary values
+//     while those copies fly) and then stream the kept leaves through a ring
+//     of bulk-copy slots.  Three window warps attend the exact window, which
+//     does not depend on the selection, through their own ring of bulk-copy
+//     slots, concurrently with the chain; each CTA sends its window partial of
+//     every head to that head's owner at the end.  One producer warp issues
+//     the level values' and the later kept leaves' copies.
 //   * Rows are read from shared memory with 16-byte (fp32) or 8-byte (bf16)
 //     loads: a row is spread over d/8 lanes, each lane holding four
 //     rotate-half pairs (j, j + d/2), so the RoPE rotation is local to the
